@@ -1,0 +1,376 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized MoE layer on B200: MoE-layer tokens/s and the roofline fraction.
+
+One step = one full MoE layer forward (router + top-k, expert FFN, combine; plus permute for
+prefill) over one batch of synthetic tokens, through the library's C ABI. Workloads (synthetic,
+seeded; shapes from the pages' model: 512 experts, top-10, 48 layers, 8,192-token prefill
+chunks, 1-4 token decode / MTP-verify passes):
+  decode1   T=1,    H=2048, E=512, k=10, I=512, shared expert, Q2, Zipf(1.1) router bias   (default)
+  decode4   T=4,    same
+  prefill8k T=8192, uniform router, shared expert, Q2
+  prefill2k_q3  T=2048, Q3, Zipf(1.2), no shared expert
+Decode steps rotate over 48 distinct layer weight sets (24 GB, larger than L2) so the weights
+come from HBM as in a real 48-layer decode; prefill steps rotate over 4 layers (503 MB each).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+Under torchrun each rank runs an independent replica (the layer shards by tokens with no
+exchange); rank 0 prints one JSON line with the whole-job throughput (max time over ranks).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOADS = {
+    "decode1": dict(shape="decode1", layers=48),
+    "decode4": dict(shape="decode4", layers=48),
+    "prefill8k": dict(shape="prefill8k", layers=4),
+    "prefill2k_q3": dict(shape="prefill2k_q3", layers=4),
+}
+METRIC = "MoE-layer tokens/s at T=1/4/8192; % of HBM or bf16 tensor-core roofline"
+DEFAULT_STEPS = {"decode1": 4800, "decode4": 4800, "prefill8k": 40, "prefill2k_q3": 60}
+DEFAULT_WARMUP = {"decode1": 480, "decode4": 480, "prefill8k": 5, "prefill2k_q3": 5}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], tc=d["bf16_tflops"], tc_sus=d["bf16_tflops_sustained"], src="measured")
+    return dict(hbm=6650.0, tc=1590.0, tc_sus=1400.0, src="fallback")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in self.rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- workload on device
+def build_layers(shape: synth.LayerShape, n_layers: int, device="cuda"):
+    """Per-layer device tensors: (Wr, bias, routed, shared); codes/scales drawn on the GPU."""
+    layers = []
+    for l in range(n_layers):
+        Wr = synth.make_router(shape.seed, l, shape.E, shape.H).to(device)
+        b = synth.zipf_bias(shape.seed, l, shape.E, shape.zipf_s).to(device) if shape.zipf_s else None
+        rs = synth.make_expert_set(shape.seed, l, synth.SET_ROUTED, shape.qtype, shape.E, shape.H, shape.I, device)
+        ss = (synth.make_expert_set(shape.seed, l, synth.SET_SHARED, shape.qtype, 1, shape.H, shape.I, device)
+              if shape.shared else None)
+        layers.append((Wr, b, rs, ss))
+    return layers
+
+
+def expert_bytes(shape: synth.LayerShape):
+    """Packed bytes of one expert: (gate+up, down)."""
+    per_w = 0.25 + (0.125 if shape.qtype == synth.Q3 else 0.0) + 2.0 / 32
+    gu = 2 * shape.I * shape.H * per_w
+    dn = shape.H * shape.I * per_w
+    return gu, dn
+
+
+def run_ours(args, world, rank, local):
+    import quantized_expert_ffn_gemm_b200 as moe
+    wl = WORKLOADS[args.workload]
+    shape = synth.WORKLOADS[wl["shape"]]
+    T, H, E, k, I = shape.T, shape.H, shape.E, shape.k, shape.I
+    n_layers = wl["layers"]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    layers = build_layers(shape, n_layers)
+    n_x = 64 if T <= 8 else 2
+    xs = [synth.make_x(shape.seed, T, H, stream=1000 * rank + i).to(dev) for i in range(n_x)]
+    ws = moe.Workspace.for_layer(H, E, k, I, shape.shared, T)
+    y = torch.empty(T, H, dtype=torch.float32, device=dev)
+
+    def step(i, x=None, yy=None):
+        Wr, b, rs, ss = layers[i % n_layers]
+        moe.layer_forward(xs[i % n_x] if x is None else x, Wr, b, rs, ss, k, ws, y=y if yy is None else yy)
+
+    K, W = args.steps, args.warmup
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize()
+    assert moe.read_device_error(ws) == 0
+
+    # ---------------- timed region (device time, CUDA events on the launching stream)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(K):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    clk = clocks.stop()
+    ms_max = max_over_ranks(ms, world)
+    value = T * K * world / (ms_max / 1e3)
+    assert moe.read_device_error(ws) == 0
+
+    # ---------------- per-kernel device time (separate pass, events around each kernel)
+    Kt = min(K, 960 if T <= 8 else 20)
+    units_total = 0
+    moe.timing_enable(True)
+    for i in range(Kt):
+        Wr, b, rs, ss = layers[i % n_layers]
+        _, idx, _ = moe.layer_forward(xs[i % n_x], Wr, b, rs, ss, k, ws, y=y, want_routing=True)
+        if T <= 8:
+            units_total += len(np.unique(idx.cpu().numpy())) + (1 if shape.shared else 0)
+    torch.cuda.synchronize()
+    moe.timing_enable(False)
+    kt = moe.timing_read()
+    launches_per_step = sum(n for (_, n) in kt.values()) / Kt
+    pk = peaks()
+
+    if T <= 8:
+        # decode: HBM bound; dominant kernel = the gate/up dequant-GEMV
+        gu_b, dn_b = expert_bytes(shape)
+        units_avg = units_total / Kt
+        dom = "dec_gate_up"
+        d_ms, d_n = kt[dom]
+        algo = units_avg * gu_b + T * H * 2 + units_avg * 8 * I * 2
+        achieved = algo / (d_ms / d_n / 1e3) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"], "unit": "GB/s",
+                "frac": round(achieved / pk["hbm"], 4), "traffic": None, "peak_source": pk["src"],
+                "algorithmic_bytes_per_launch": int(algo), "avg_launch_us": round(d_ms / d_n * 1e3, 3)}
+        layer_bytes = units_avg * (gu_b + dn_b) + E * H * 4 + T * H * 2 + T * H * 4
+        layer_gbs = layer_bytes / (ms_max / K / 1e3) / 1e9
+        roof_layer = {"bound": "hbm", "bytes_per_step": int(layer_bytes), "achieved": round(layer_gbs, 1),
+                      "frac": round(layer_gbs / pk["hbm"], 4), "distinct_experts_avg": round(units_avg, 2)}
+    else:
+        rows = T * k + (T if shape.shared else 0)
+        dom = "gemm_gate_up"
+        d_ms, d_n = kt[dom]
+        flops = 2.0 * 2 * rows * H * I
+        achieved = flops / (d_ms / d_n / 1e3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": pk["tc_sus"],
+                "unit": "TFLOP/s", "frac": round(achieved / pk["tc_sus"], 4), "traffic": None,
+                "peak_source": pk["src"] + " (sustained bf16; fp16 MMA runs at the same rate)",
+                "algorithmic_flops_per_launch": flops, "avg_launch_us": round(d_ms / d_n * 1e3, 1)}
+        layer_flops = 2.0 * 3 * rows * H * I + 2.0 * T * E * H
+        tf = layer_flops / (ms_max / K / 1e3) / 1e12
+        roof_layer = {"bound": "tensor", "flops_per_step": layer_flops, "achieved": round(tf, 1),
+                      "frac": round(tf / pk["tc_sus"], 4)}
+
+    # ---------------- end to end through host buffers (pinned), copies inside the timed region
+    Ke = min(K, 2000 if T <= 8 else 20)
+    xh = [x.cpu().pin_memory() for x in xs[:8]]
+    yh = torch.empty(T, H, dtype=torch.float32).pin_memory()
+    xd = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize()
+    barrier(world)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for i in range(Ke):
+        xd.copy_(xh[i % len(xh)], non_blocking=True)
+        step(i, x=xd)
+        yh.copy_(y, non_blocking=True)
+    f1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
+    e2e = {"value": round(T * Ke * world / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
+           "d2h_bytes_per_step": T * H * 4, "steps": Ke}
+
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(ms_max / K, 6), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp16 MMA operands, fp32 accumulate / router / y (weights Q2/Q3)", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: MoE layer T={T}, H={H}, E={E}, top-{k}, I={I}, "
+                               f"{'Q3' if shape.qtype == 3 else 'Q2'}, shared={int(shape.shared)}, "
+                               f"router bias={'Zipf(%s)' % shape.zipf_s if shape.zipf_s else 'none'}",
+                   "T": T, "layers_rotated": n_layers,
+                   "l2": "inputs larger than L2: steps rotate over %d layer weight sets (%.1f GB)" % (
+                       n_layers, n_layers * (layers[0][2].nbytes + (layers[0][3].nbytes if layers[0][3] else 0)
+                                             + E * H * 4) / 1e9),
+                   "parallelism": f"replicas x{world} (token-parallel, no collective)"},
+        "roofline": roof, "roofline_layer": roof_layer,
+        "kernels_ms_per_step": {n: round(ms_ / Kt, 5) for n, (ms_, _) in sorted(kt.items())},
+        "e2e": e2e, "gpu_launches": int(round(launches_per_step * K)), "clocks": clk,
+    }
+    return out, shape, layers
+
+
+def cpu_baseline(shape: synth.LayerShape, budget_s: float = 12.0):
+    """The oracle, as it stands, on a bounded sample of the same workload on the host cores."""
+    import oracle
+    L = synth.make_layer(shape)
+    nthr = oracle.max_threads()
+    ntok = 1
+    t0 = time.time()
+    oracle.layer_forward(L.x[:1], L.Wr, L.bias, shape.k, L.routed, L.shared, nthreads=nthr)
+    one = max(time.time() - t0, 1e-3)
+    ntok = int(max(1, min(shape.T, (budget_s / one) * min(nthr, shape.T))))
+    ntok = min(ntok, 4 * nthr) if shape.T > 8 else min(ntok, shape.T if shape.T > 1 else 16)
+    xs = synth.make_x(shape.seed, ntok, shape.H, stream=777) if shape.T <= 8 else L.x[:ntok]
+    t0 = time.time()
+    oracle.layer_forward(xs, L.Wr, L.bias, shape.k, L.routed, L.shared, nthreads=nthr)
+    dt = time.time() - t0
+    return {"value": round(ntok / dt, 3), "unit": "tokens/s", "cores": min(nthr, ntok), "kind": "oracle",
+            "sample": f"{ntok} tokens of the {shape.name} layer (layer 0 weights), fp64 C oracle, {dt:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle on this arm's workload, timed on the host cores."""
+    if rank != 0:
+        return None
+    import oracle
+    wl = WORKLOADS[args.workload]
+    shape = synth.WORKLOADS[wl["shape"]]
+    L = synth.make_layer(shape)
+    nthr = oracle.max_threads()
+    T = shape.T
+    # one step = the oracle on a bounded sample of the step's tokens (all of them when T <= 8)
+    sample_T = T if T <= 8 else min(T, 2 * nthr)
+    xs = [synth.make_x(shape.seed, T, shape.H, stream=i)[:sample_T] for i in range(4)]
+    for i in range(max(0, min(args.warmup, 1))):
+        oracle.layer_forward(xs[i % 4], L.Wr, L.bias, shape.k, L.routed, L.shared, nthreads=nthr)
+    budget = 150.0
+    t0 = time.time()
+    done = 0
+    for i in range(args.steps):
+        oracle.layer_forward(xs[i % 4], L.Wr, L.bias, shape.k, L.routed, L.shared, nthreads=nthr)
+        done += 1
+        if time.time() - t0 > budget:
+            break
+    dt = time.time() - t0
+    value = sample_T * done / dt
+    return {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": done,
+            "warmup": min(args.warmup, 1), "ms_per_step": round(dt / done * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.workload, "T": T, "sample_tokens_per_step": sample_T},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": min(nthr, sample_T),
+                             "kind": "oracle",
+                             "sample": f"{done} steps x {sample_T} tokens of {shape.name}, fp64 C oracle"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--workload", default="decode1", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--breakdown", action="store_true", help="also time T=4 and T=8192 on rank 0 (extra keys)")
+    args = ap.parse_args()
+    if args.steps is None:
+        args.steps = DEFAULT_STEPS[args.workload]
+    if args.warmup is None:
+        args.warmup = DEFAULT_WARMUP[args.workload]
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    world, rank, local = dist_setup()
+    try:
+        out, shape, _ = run_ours(args, world, rank, local)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(shape)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

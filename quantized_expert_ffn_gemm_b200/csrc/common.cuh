@@ -1,0 +1,149 @@
+// Internal declarations shared by the kernels and the C-ABI layer of libmoe_ffn.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe_ffn.h"
+
+namespace moe {
+
+constexpr int kMaxK = 32;          // routing slots per token
+constexpr int kMaxE = 4096;        // experts per layer
+constexpr int kDecodeMaxT = 8;     // tokens the decode (GEMV) path takes at once (MMA N = 8)
+constexpr int kPermChunk = 256;    // (token, slot) pairs per permute CTA
+
+// ---------------------------------------------------------------- control area (workspace head)
+// Everything here is left at zero by the kernels that use it (tickets are reset by the last CTA).
+struct Ctrl {
+  int err;                  // MOE_OK / MOE_ERR_DEVICE_CHECK / MOE_ERR_TIMEOUT (first error wins)
+  int err_info;             // diagnostic: the offending value
+  unsigned router_ticket;   // last-CTA election in the decode router
+  unsigned pad0;
+  unsigned gemm_ticket[4];  // tile counters of the persistent grouped GEMM
+  int n_units;              // decode: number of (expert, token-set) units built by the router
+  int n_tiles;              // prefill: number of (group, row-tile) entries in the tile list
+  int pad1[22];
+};
+static_assert(sizeof(Ctrl) == 128, "control area is 128 bytes");
+
+// A decode "unit": one expert applied to up to 8 activation rows (MMA columns).
+//   rows xrow0 .. xrow0+7 of the activation source, column c present iff bit c of mask;
+//   w[c]: routing weight of column c (combine mode); h is stored at h[(u*8 + c)*I ..].
+struct DecUnit {
+  int expert;
+  int set;       // 0 routed, 1 shared
+  int mask;
+  int xrow0;
+  float w[8];
+};
+
+// ---------------------------------------------------------------- workspace layout
+struct WsLayout {
+  size_t ctrl, logits, idx, w, hist, units, hdec, counts, offsets, row_of, src, xperm, hperm, operm, u16, tiles, total;
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline WsLayout ws_layout(int H, int E, int k, int I, int has_shared, int T) {
+  WsLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+  size_t Tk = (size_t)T * k;
+  size_t rows = Tk + (has_shared ? (size_t)T : 0);
+  size_t nchunks = (Tk + kPermChunk - 1) / kPermChunk;
+  // decode units (distinct experts of <= 8 tokens) or row-chunk units of the GEMV rows path
+  size_t units = (size_t)kDecodeMaxT * k + 1;
+  size_t row_units = (rows + 7) / 8 + (size_t)E + 2;
+  if (row_units > units) units = row_units;
+  L.ctrl = take(sizeof(Ctrl));
+  L.logits = take((size_t)T * E * 4);
+  L.idx = take(Tk * 4);
+  L.w = take(Tk * 4);
+  L.hist = take((nchunks + 1) * (size_t)E * 4);
+  L.units = take(units * sizeof(DecUnit));
+  L.hdec = take(units * 8 * (size_t)I * 2);
+  L.counts = take((size_t)(E + 2) * 4);
+  L.offsets = take((size_t)(E + 2) * 4);
+  L.row_of = take(Tk * 4);
+  L.src = take(rows * 4);
+  L.xperm = take(rows * (size_t)H * 2);
+  L.hperm = take(rows * (size_t)I * 2);
+  L.operm = take(rows * (size_t)H * 2);
+  L.u16 = take((size_t)T * H * 2);
+  L.tiles = take((rows / 16 + (size_t)E + 4) * 8);
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------- device helpers
+__device__ __forceinline__ void set_device_error(Ctrl *c, int code, int info) {
+  if (atomicCAS(&c->err, 0, code) == 0) c->err_info = info;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(((uint32_t)b) << 16);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ---------------------------------------------------------------- kernel launchers (one per .cu)
+// All return cudaSuccess or the launch error; none synchronises.
+cudaError_t launch_router_decode(const uint16_t *x, int T, int H, const float *Wr, const float *bias, int E, int k,
+                                 int32_t *idx, float *w, float *logits, int build_units, int has_shared,
+                                 DecUnit *units, Ctrl *ctrl, cudaStream_t s);
+cudaError_t launch_router_prefill(const uint16_t *x, int T, int H, const float *Wr, const float *bias, int E, int k,
+                                  int32_t *idx, float *w, float *logits, cudaStream_t s);
+cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const uint16_t *x, int H, int with_shared,
+                           int32_t *counts, int32_t *offsets, int32_t *row_of, int32_t *src, uint16_t *x_perm,
+                           int32_t *hist, Ctrl *ctrl, cudaStream_t s);
+cudaError_t launch_combine(const uint16_t *out_perm, const int32_t *row_of, const float *w, int T, int k, int H,
+                           const uint16_t *shared_out, const float *residual, float *y, cudaStream_t s);
+cudaError_t launch_rmsnorm(const float *r, int T, int H, float eps, uint16_t *u, cudaStream_t s);
+cudaError_t launch_dequant_rows(const moe_qmat &m, int expert, int row0, int nrows, float *out_f32, uint16_t *out_f16,
+                                cudaStream_t s);
+
+// decode path: units are read from `units` (count in ctrl->n_units, at most max_units)
+cudaError_t launch_decode_units_from_offsets(const int32_t *offsets, int n_groups, int has_shared_group, int n_rows,
+                                             DecUnit *units, Ctrl *ctrl, cudaStream_t s);
+cudaError_t launch_decode_gate_up(const void *x, int x_is_bf16, int H, int I, const moe_expert_set &routed,
+                                  const moe_expert_set *shared, const DecUnit *units, int max_units, Ctrl *ctrl,
+                                  uint16_t *hdec, cudaStream_t s);
+// combine mode (y != NULL): y[t] = sum_u w_u[t] * down_u h_u[t] (+ residual); rows mode: out rows fp16
+cudaError_t launch_decode_down(int H, int I, const moe_expert_set &routed, const moe_expert_set *shared,
+                               const DecUnit *units, int max_units, Ctrl *ctrl, const uint16_t *hdec, float *y,
+                               const float *residual, int T, uint16_t *out_rows, cudaStream_t s);
+
+// prefill path (tcgen05 grouped GEMM)
+int gemm_shape_supported(int H, int I);
+cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, int n_rows, int E, int H, int I,
+                               const moe_expert_set &routed, const moe_expert_set *shared, uint16_t *h_perm,
+                               uint16_t *out_perm, int2 *tiles, Ctrl *ctrl, cudaStream_t s);
+
+int num_sms();
+
+// ---------------------------------------------------------------- per-kernel timing (optional)
+enum KernelId {
+  KID_ROUTER_DECODE = 0, KID_ROUTER_GEMM, KID_TOPK, KID_PERM_HIST, KID_PERM_SCAN, KID_PERM_SCATTER, KID_PERM_FILL,
+  KID_PERM_GATHER, KID_COMBINE, KID_RMSNORM, KID_DEQUANT_ROWS, KID_DEC_UNITS, KID_DEC_GATE_UP, KID_DEC_DOWN,
+  KID_TILE_LIST, KID_GEMM_GATE_UP, KID_GEMM_DOWN, KID_COUNT
+};
+void timer_begin(int kid, cudaStream_t s);
+void timer_end(int kid, cudaStream_t s);
+
+// brackets one kernel launch with timing events when timing is enabled
+struct KTimer {
+  int kid;
+  cudaStream_t s;
+  KTimer(int k, cudaStream_t st) : kid(k), s(st) { timer_begin(kid, s); }
+  ~KTimer() { timer_end(kid, s); }
+};
+
+}  // namespace moe

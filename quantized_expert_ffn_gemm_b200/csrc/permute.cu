@@ -1,0 +1,316 @@
+// Token permutation, weighted combine, RMSNorm and the dequantization test hook.
+//
+// Permutation: the routed (token, slot) pairs are grouped into expert-contiguous rows so each
+// expert's rows form one GEMM operand (the more tokens an expert collects in a prefill chunk,
+// the more its weights are reused: "Two-Day Port, 8x Faster Prefill: Strata Engine
+// Benchmarked", "Where Strata Is Fast: Not Magic, but Logistics", MoE paragraph). It is a
+// stable counting sort: per-chunk histograms, one exclusive scan over (expert, chunk), then a
+// stable scatter in which one warp walks its chunk in order and ranks equal experts with
+// __match_any_sync, so the rows of an expert come out in token order, deterministically.
+#include "common.cuh"
+#include "dequant.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------- histogram per chunk
+__global__ void __launch_bounds__(256)
+perm_hist_kernel(const int32_t *__restrict__ idx, int P, int E, int32_t *__restrict__ hist, Ctrl *ctrl) {
+  extern __shared__ int32_t sh[];
+  const int c = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) sh[e] = 0;
+  __syncthreads();
+  const int p0 = c * kPermChunk;
+  for (int p = p0 + threadIdx.x; p < min(P, p0 + kPermChunk); p += blockDim.x) {
+    int e = idx[p];
+    if (e >= 0 && e < E) atomicAdd(&sh[e], 1);
+    else set_device_error(ctrl, MOE_ERR_DEVICE_CHECK, e);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(size_t)c * E + e] = sh[e];
+}
+
+// ---------------------------------------------------------------- scan (one CTA)
+// counts[e] = sum_c hist[c][e]; offsets = exclusive scan; hist[c][e] <- first row of chunk c in e
+__global__ void __launch_bounds__(1024)
+perm_scan_kernel(int32_t *__restrict__ hist, int nchunks, int E, int P, int T, int with_shared,
+                 int32_t *__restrict__ counts, int32_t *__restrict__ offsets) {
+  __shared__ int32_t s_warp[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (E + 1023) / 1024;  // experts per thread (contiguous)
+  int local[4];
+  int mysum = 0;
+  for (int i = 0; i < per; ++i) {
+    int e = tid * per + i, s = 0;
+    if (e < E)
+      for (int c = 0; c < nchunks; ++c) s += hist[(size_t)c * E + e];
+    local[i] = s;
+    mysum += s;
+  }
+  // block exclusive scan of mysum
+  int v = mysum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) s_warp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int wv = s_warp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int n = __shfl_up_sync(0xffffffffu, wv, o);
+      if (lane >= o) wv += n;
+    }
+    s_warp[lane] = wv;
+  }
+  __syncthreads();
+  int base = v - mysum + (warp > 0 ? s_warp[warp - 1] : 0);
+  for (int i = 0; i < per; ++i) {
+    int e = tid * per + i;
+    if (e < E) {
+      counts[e] = local[i];
+      offsets[e] = base;
+      int run = base;
+      for (int c = 0; c < nchunks; ++c) {
+        int h = hist[(size_t)c * E + e];
+        hist[(size_t)c * E + e] = run;
+        run += h;
+      }
+    }
+    base += local[i];
+  }
+  if (tid == 0) {
+    offsets[E] = P;
+    if (with_shared) {
+      offsets[E + 1] = P + T;
+      counts[E] = T;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- stable scatter (one warp per chunk)
+__global__ void __launch_bounds__(32)
+perm_scatter_kernel(const int32_t *__restrict__ idx, int P, int k, int E, const int32_t *__restrict__ hist,
+                    int32_t *__restrict__ row_of, int32_t *__restrict__ src) {
+  extern __shared__ int32_t cursor[];
+  const int c = blockIdx.x, lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) cursor[e] = hist[(size_t)c * E + e];
+  __syncwarp();
+  const int p0 = c * kPermChunk, p1 = min(P, p0 + kPermChunk);
+  for (int pb = p0; pb < p1; pb += 32) {
+    int p = pb + lane;
+    int e = (p < p1) ? idx[p] : -1;
+    bool ok = (p < p1) && e >= 0 && e < E;
+    int key = ok ? e : -1 - lane;  // invalid lanes form singleton groups
+    unsigned grp = __match_any_sync(0xffffffffu, key);
+    int rank = __popc(grp & ((1u << lane) - 1u));
+    int base = ok ? cursor[e] : 0;
+    __syncwarp();
+    if (ok) {
+      int row = base + rank;
+      row_of[p] = row;
+      src[row] = p / k;
+      if (rank == 0) cursor[e] = base + __popc(grp);
+    } else if (p < p1) {
+      row_of[p] = -1;  // flagged by the histogram kernel
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------- gather rows (bf16 -> fp16)
+__global__ void __launch_bounds__(256)
+perm_gather_kernel(const uint16_t *__restrict__ x, int H, const int32_t *__restrict__ src, int P, int rows,
+                   uint16_t *__restrict__ x_perm) {
+  const int H8 = H >> 3;
+  const size_t total = (size_t)rows * H8;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    int r = (int)(i / H8), c = (int)(i % H8);
+    int t = (r < P) ? src[r] : r - P;
+    uint4 v = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * H) + c);
+    uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      __half2 h = __floats2half2_rn(__uint_as_float(in[j] << 16), __uint_as_float(in[j] & 0xffff0000u));
+      out[j] = *reinterpret_cast<uint32_t *>(&h);
+    }
+    reinterpret_cast<uint4 *>(x_perm + (size_t)r * H)[c] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+__global__ void fill_iota_kernel(int32_t *p, int n) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = i;
+}
+
+cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const uint16_t *x, int H, int with_shared,
+                           int32_t *counts, int32_t *offsets, int32_t *row_of, int32_t *src, uint16_t *x_perm,
+                           int32_t *hist, Ctrl *ctrl, cudaStream_t s) {
+  const int P = T * k;
+  const int nchunks = (P + kPermChunk - 1) / kPermChunk;
+  const size_t esm = (size_t)E * 4;
+  {
+    KTimer kt_(KID_PERM_HIST, s);
+    perm_hist_kernel<<<nchunks, 256, esm, s>>>(idx, P, E, hist, ctrl);
+  }
+  {
+    KTimer kt_(KID_PERM_SCAN, s);
+    perm_scan_kernel<<<1, 1024, 0, s>>>(hist, nchunks, E, P, T, with_shared, counts, offsets);
+  }
+  {
+    KTimer kt_(KID_PERM_SCATTER, s);
+    perm_scatter_kernel<<<nchunks, 32, esm, s>>>(idx, P, k, E, hist, row_of, src);
+  }
+  if (with_shared) {  // src[P + t] = t
+    {
+      KTimer kt_(KID_PERM_FILL, s);
+      fill_iota_kernel<<<(T + 255) / 256, 256, 0, s>>>(src + P, T);
+    }
+  }
+  const int rows = P + (with_shared ? T : 0);
+  size_t want = ((size_t)rows * (H / 8) + 255) / 256, cap = (size_t)num_sms() * 16;
+  int grid = (int)(want < cap ? want : cap);
+  {
+    KTimer kt_(KID_PERM_GATHER, s);
+    perm_gather_kernel<<<grid, 256, 0, s>>>(x, H, src, P, rows, x_perm);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- combine
+// y[t,h] = sum_j w[t,j] out[row_of[t,j], h] (fixed j order) + shared[t,h] + residual[t,h]
+__global__ void __launch_bounds__(256)
+combine_kernel(const uint16_t *__restrict__ out, const int32_t *__restrict__ row_of, const float *__restrict__ w,
+               int T, int k, int H, const uint16_t *__restrict__ shared, const float *residual, float *y) {
+  const int H8 = H >> 3;
+  const size_t total = (size_t)T * H8;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    int t = (int)(i / H8), c = (int)(i % H8);
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+    if (residual) {
+      float4 r0 = reinterpret_cast<const float4 *>(residual + (size_t)t * H)[2 * c];
+      float4 r1 = reinterpret_cast<const float4 *>(residual + (size_t)t * H)[2 * c + 1];
+      acc[0] = r0.x; acc[1] = r0.y; acc[2] = r0.z; acc[3] = r0.w;
+      acc[4] = r1.x; acc[5] = r1.y; acc[6] = r1.z; acc[7] = r1.w;
+    }
+    for (int j = 0; j < k; ++j) {
+      int row = row_of[(size_t)t * k + j];
+      if (row < 0) continue;
+      float wj = w[(size_t)t * k + j];
+      uint4 v = __ldg(reinterpret_cast<const uint4 *>(out + (size_t)row * H) + c);
+      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&vv[q]));
+        acc[2 * q] = fmaf(wj, f.x, acc[2 * q]);
+        acc[2 * q + 1] = fmaf(wj, f.y, acc[2 * q + 1]);
+      }
+    }
+    if (shared) {
+      uint4 v = __ldg(reinterpret_cast<const uint4 *>(shared + (size_t)t * H) + c);
+      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&vv[q]));
+        acc[2 * q] += f.x;
+        acc[2 * q + 1] += f.y;
+      }
+    }
+    float4 *yo = reinterpret_cast<float4 *>(y + (size_t)t * H);
+    yo[2 * c] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    yo[2 * c + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+}
+
+cudaError_t launch_combine(const uint16_t *out_perm, const int32_t *row_of, const float *w, int T, int k, int H,
+                           const uint16_t *shared_out, const float *residual, float *y, cudaStream_t s) {
+  size_t want = ((size_t)T * (H / 8) + 255) / 256, cap = (size_t)num_sms() * 16;
+  int grid = (int)(want < cap ? want : cap);
+  {
+    KTimer kt_(KID_COMBINE, s);
+    combine_kernel<<<grid, 256, 0, s>>>(out_perm, row_of, w, T, k, H, shared_out, residual, y);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- RMSNorm
+__global__ void __launch_bounds__(256)
+rmsnorm_kernel(const float *__restrict__ r, int H, float eps, uint16_t *__restrict__ u) {
+  __shared__ float s_part[8];
+  const int t = blockIdx.x;
+  const float *row = r + (size_t)t * H;
+  float ss = 0.0f;
+  for (int h = threadIdx.x; h < H; h += blockDim.x) ss = fmaf(row[h], row[h], ss);
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) tot += s_part[i];
+  const float inv = 1.0f / sqrtf(tot / (float)H + eps);
+  for (int h = threadIdx.x; h < H; h += blockDim.x) {
+    __nv_bfloat16 b = __float2bfloat16_rn(row[h] * inv);
+    u[(size_t)t * H + h] = *reinterpret_cast<uint16_t *>(&b);
+  }
+}
+
+cudaError_t launch_rmsnorm(const float *r, int T, int H, float eps, uint16_t *u, cudaStream_t s) {
+  {
+    KTimer kt_(KID_RMSNORM, s);
+    rmsnorm_kernel<<<T, 256, 0, s>>>(r, H, eps, u);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- dequant test hook
+// thread per (row, 16-weight word); fp16 output through the same pair decoder the GEMM uses
+__global__ void dequant_rows_kernel(moe_qmat m, int expert, int row0, int nrows, float *out_f32, uint16_t *out_f16) {
+  const int words = m.K / 16;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= nrows * words) return;
+  const int r = i / words, wq = i % words;
+  const size_t row = (size_t)expert * m.rows + row0 + r;
+  const int blk = wq >> 1, q = wq & 1;
+  const uint32_t w = reinterpret_cast<const uint32_t *>(m.codes + row * (m.K / 4))[wq];
+  const uint16_t dbits = m.scales[row * (m.K / 32) + blk];
+  const __half d = __ushort_as_half(dbits);
+  uint32_t pairs[8];
+  if (m.qtype == MOE_Q2) {
+    dq2_word(w, __half2half2(d), pairs);
+  } else {
+    const uint32_t hw = reinterpret_cast<const uint32_t *>(m.hibits + row * (m.K / 8))[blk];
+    dq3_word(w, hw, q, __half2half2(d), pairs);
+  }
+  const float df = __half2float(d);
+  const int q0 = (m.qtype == MOE_Q2) ? 2 : 4;
+  for (int j = 0; j < 16; ++j) {
+    const int kk = wq * 16 + j;
+    const uint16_t hb = (uint16_t)((pairs[j >> 1] >> (16 * (j & 1))) & 0xffffu);
+    if (out_f16) out_f16[(size_t)r * m.K + kk] = hb;
+    if (out_f32) {
+      // integer code recovered from the packed planes (independent of the fp16 path)
+      const int jj = j, ii = jj >> 1, h = jj & 1;
+      int c = (int)((w >> (16 * h + 2 * ii)) & 3u);
+      if (m.qtype == MOE_Q3) {
+        const uint32_t hw = reinterpret_cast<const uint32_t *>(m.hibits + row * (m.K / 8))[blk];
+        c |= (int)((hw >> (16 * h + 8 * q + ii)) & 1u) << 2;
+      }
+      out_f32[(size_t)r * m.K + kk] = df * (float)(c - q0);
+    }
+  }
+}
+
+cudaError_t launch_dequant_rows(const moe_qmat &m, int expert, int row0, int nrows, float *out_f32, uint16_t *out_f16,
+                                cudaStream_t s) {
+  const int n = nrows * (m.K / 16);
+  {
+    KTimer kt_(KID_DEQUANT_ROWS, s);
+    dequant_rows_kernel<<<(n + 255) / 256, 256, 0, s>>>(m, expert, row0, nrows, out_f32, out_f16);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

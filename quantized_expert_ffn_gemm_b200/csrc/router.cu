@@ -1,0 +1,380 @@
+// Router + top-k.
+//
+// Each token is scored against every routed expert and sent to the k best ("Strata vs Llama.cpp
+// vs vLLM", chapter "How Strata is designed to work": 10 of 512 experts per layer). Logits are
+// fp32 (x is exact in fp32), the top-k is taken on the fp32 logits with the lower expert index
+// winning ties, slots are stored in descending logit order, and the weights are the softmax
+// restricted to the selected set (the full softmax renormalised over the set).
+//
+// Decode (T <= 8): one kernel. Every warp produces whole logits (one expert, all T tokens,
+// Wr read once with 128-bit loads); the last CTA to finish (atomic ticket) runs the top-k and,
+// for the decode expert path, groups the selected (token, slot) pairs by distinct expert.
+// Prefill: a tiled fp32 GEMM for the logits, then one warp per token for the top-k.
+#include "common.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------- top-k within one warp
+
+// order-preserving 32-bit key of an fp32 logit (NaN sorts lowest, -0 == +0)
+__device__ __forceinline__ uint32_t logit_key(float f) {
+  if (f != f) return 0u;
+  if (f == 0.0f) f = 0.0f;
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Top-k of E logits (l[0..E) in shared or global memory) by one warp. Writes idx[0..k) and
+// w[0..k). Rounds of: per-lane best among untaken candidates (ascending index scan, strict >,
+// so the lower index wins a tie inside a lane), warp max of the key, then warp min of the index
+// among lanes holding that key.
+template <int PER_LANE>
+__device__ void warp_topk(const float *l, const float *bias, int E, int k, int32_t *idx, float *w) {
+  const int lane = threadIdx.x & 31;
+  uint32_t key[PER_LANE];
+  float val[PER_LANE];
+#pragma unroll
+  for (int i = 0; i < PER_LANE; ++i) {
+    int e = lane + 32 * i;
+    float v = -INFINITY;
+    if (e < E) v = l[e] + (bias ? bias[e] : 0.0f);
+    val[i] = v;
+    key[i] = (e < E) ? logit_key(v) : 0u;
+  }
+  uint32_t taken = 0;
+  float sel_val[kMaxK];
+  int sel_idx[kMaxK];
+  for (int j = 0; j < k; ++j) {
+    uint32_t bk = 0;
+    int bi = 0x7fffffff;
+    float bv = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i) {
+      int e = lane + 32 * i;
+      bool ok = (e < E) && !((taken >> i) & 1u);
+      if (ok && (key[i] > bk || bi == 0x7fffffff)) { bk = key[i]; bi = e; bv = val[i]; }
+    }
+    uint32_t m = __reduce_max_sync(0xffffffffu, bi == 0x7fffffff ? 0u : bk);
+    uint32_t cand = (bi != 0x7fffffff && bk == m) ? (uint32_t)bi : 0xffffffffu;
+    uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+    if ((uint32_t)bi == win) taken |= 1u << ((bi - lane) / 32);
+    float wv = __shfl_sync(0xffffffffu, bv, (int)(win & 31u));
+    sel_val[j] = wv;
+    sel_idx[j] = (int)win;
+  }
+  if (lane == 0) {
+    float l0 = sel_val[0], z = 0.0f;
+    for (int j = 0; j < k; ++j) z += expf(sel_val[j] - l0);
+    float inv = 1.0f / z;
+    for (int j = 0; j < k; ++j) {
+      idx[j] = sel_idx[j];
+      w[j] = expf(sel_val[j] - l0) * inv;
+    }
+  }
+}
+
+// generic E (up to kMaxE) from shared memory: lanes rescan their strided candidates each round
+__device__ void warp_topk_generic(const float *l, const float *bias, int E, int k, int32_t *idx, float *w,
+                                  uint32_t *taken_words /* smem, E/32 words, zeroed */) {
+  const int lane = threadIdx.x & 31;
+  float sel_val[kMaxK];
+  int sel_idx[kMaxK];
+  for (int j = 0; j < k; ++j) {
+    uint32_t bk = 0;
+    int bi = 0x7fffffff;
+    float bv = -INFINITY;
+    for (int e = lane; e < E; e += 32) {
+      if ((taken_words[e >> 5] >> (e & 31)) & 1u) continue;
+      float v = l[e] + (bias ? bias[e] : 0.0f);
+      uint32_t kk = logit_key(v);
+      if (kk > bk || bi == 0x7fffffff) { bk = kk; bi = e; bv = v; }
+    }
+    uint32_t m = __reduce_max_sync(0xffffffffu, bi == 0x7fffffff ? 0u : bk);
+    uint32_t cand = (bi != 0x7fffffff && bk == m) ? (uint32_t)bi : 0xffffffffu;
+    uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+    if ((uint32_t)bi == win) taken_words[bi >> 5] |= 1u << (bi & 31);
+    __syncwarp();
+    sel_val[j] = __shfl_sync(0xffffffffu, bv, (int)(win & 31u));
+    sel_idx[j] = (int)win;
+  }
+  if (lane == 0) {
+    float l0 = sel_val[0], z = 0.0f;
+    for (int j = 0; j < k; ++j) z += expf(sel_val[j] - l0);
+    float inv = 1.0f / z;
+    for (int j = 0; j < k; ++j) {
+      idx[j] = sel_idx[j];
+      w[j] = expf(sel_val[j] - l0) * inv;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- decode units
+// Group the T*k selected (token, slot) pairs by distinct expert, in order of first appearance
+// (token-major), plus the always-on shared expert as the last unit. One warp.
+__device__ void build_units(const int32_t *sidx, const float *sw, int T, int k, int has_shared, DecUnit *units,
+                            Ctrl *ctrl, int *s_first, int *s_unit) {
+  const int lane = threadIdx.x & 31;
+  const int P = T * k;
+  for (int p = lane; p < P; p += 32) {
+    int e = sidx[p], f = p;
+    for (int q = 0; q < p; ++q)
+      if (sidx[q] == e) { f = q; break; }
+    s_first[p] = f;
+  }
+  __syncwarp();
+  if (lane == 0) {  // unit numbering of the leaders in pair order (P <= 256)
+    int nu = 0;
+    for (int p = 0; p < P; ++p) s_unit[p] = (s_first[p] == p) ? nu++ : -1;
+    ctrl->n_units = nu + (has_shared ? 1 : 0);
+    for (int u = 0; u < nu + (has_shared ? 1 : 0); ++u) {
+      units[u].mask = 0;
+      units[u].xrow0 = 0;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) units[u].w[c] = 0.0f;
+    }
+    for (int p = 0; p < P; ++p) {
+      int u = s_unit[s_first[p]];
+      int t = p / k;
+      units[u].expert = sidx[p];
+      units[u].set = 0;
+      units[u].mask |= 1 << t;
+      units[u].w[t] = sw[p];
+    }
+    if (has_shared) {
+      units[nu].expert = 0;
+      units[nu].set = 1;
+      units[nu].mask = (1 << T) - 1;
+      for (int t = 0; t < T; ++t) units[nu].w[t] = 1.0f;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- decode router kernel
+constexpr int kRouterDecWarps = 4;
+
+__global__ void __launch_bounds__(kRouterDecWarps * 32)
+router_decode_kernel(const uint16_t *__restrict__ x, int T, int H, const float *__restrict__ Wr,
+                     const float *__restrict__ bias, int E, int k, int32_t *__restrict__ idx, float *__restrict__ w,
+                     float *__restrict__ logits, int build, int has_shared, DecUnit *__restrict__ units,
+                     Ctrl *__restrict__ ctrl) {
+  extern __shared__ float4 smem4[];
+  float *xs = reinterpret_cast<float *>(smem4);  // [T][H] fp32, later reused for [T][E] logits
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < T * H; i += blockDim.x) xs[i] = bf16_bits_to_float(x[i]);
+  __syncthreads();
+
+  const int H4 = H >> 2;
+  for (int e = blockIdx.x * kRouterDecWarps + warp; e < E; e += gridDim.x * kRouterDecWarps) {
+    const float4 *wr = reinterpret_cast<const float4 *>(Wr + (size_t)e * H);
+    float acc[kDecodeMaxT];
+#pragma unroll
+    for (int t = 0; t < kDecodeMaxT; ++t) acc[t] = 0.0f;
+    for (int h0 = 0; h0 < H4; h0 += 32 * 8) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        int h4 = h0 + lane + 32 * u;
+        v[u] = (h4 < H4) ? __ldcs(wr + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        int h4 = h0 + lane + 32 * u;
+        if (h4 < H4) {
+#pragma unroll
+          for (int t = 0; t < kDecodeMaxT; ++t) {
+            if (t < T) {
+              float4 xv = reinterpret_cast<const float4 *>(xs + (size_t)t * H)[h4];
+              acc[t] = fmaf(v[u].x, xv.x, acc[t]);
+              acc[t] = fmaf(v[u].y, xv.y, acc[t]);
+              acc[t] = fmaf(v[u].z, xv.z, acc[t]);
+              acc[t] = fmaf(v[u].w, xv.w, acc[t]);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kDecodeMaxT; ++t) {
+      if (t < T) {
+        float s = warp_sum(acc[t]);
+        if (lane == 0) logits[(size_t)t * E + e] = s;
+      }
+    }
+  }
+
+  // last CTA to arrive does the top-k
+  __shared__ unsigned s_last;
+  __threadfence();
+  __syncthreads();
+  // atomicInc wraps the ticket back to 0 when the last CTA takes it
+  if (tid == 0) s_last = (atomicInc(&ctrl->router_ticket, gridDim.x - 1) == gridDim.x - 1) ? 1u : 0u;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  float *ls = xs;  // [T][E]
+  for (int i = tid; i < T * E; i += blockDim.x) ls[i] = __ldcg(logits + i);
+  __shared__ int32_t s_idx[kDecodeMaxT * kMaxK];
+  __shared__ float s_w[kDecodeMaxT * kMaxK];
+  __shared__ uint32_t s_taken[kRouterDecWarps][kMaxE / 32];
+  __syncthreads();
+  for (int t = warp; t < T; t += kRouterDecWarps) {
+    if (E <= 512) {
+      warp_topk<16>(ls + (size_t)t * E, bias, E, k, s_idx + t * k, s_w + t * k);
+    } else {
+      for (int i = lane; i < kMaxE / 32; i += 32) s_taken[warp][i] = 0;
+      __syncwarp();
+      warp_topk_generic(ls + (size_t)t * E, bias, E, k, s_idx + t * k, s_w + t * k, s_taken[warp]);
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < T * k; i += blockDim.x) {
+    idx[i] = s_idx[i];
+    w[i] = s_w[i];
+  }
+  if (bias) {  // logits output includes the bias
+    for (int i = tid; i < T * E; i += blockDim.x) logits[i] = ls[i] + bias[i % E];
+  }
+  if (build && warp == 0) {
+    __shared__ int s_first[kDecodeMaxT * kMaxK], s_unit[kDecodeMaxT * kMaxK];
+    build_units(s_idx, s_w, T, k, has_shared, units, ctrl, s_first, s_unit);
+  }
+}
+
+cudaError_t launch_router_decode(const uint16_t *x, int T, int H, const float *Wr, const float *bias, int E, int k,
+                                 int32_t *idx, float *w, float *logits, int build_units_flag, int has_shared,
+                                 DecUnit *units, Ctrl *ctrl, cudaStream_t s) {
+  size_t smem = (size_t)T * (H > E ? H : E) * sizeof(float);
+  int grid = (E + kRouterDecWarps - 1) / kRouterDecWarps;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(router_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  {
+    KTimer kt_(KID_ROUTER_DECODE, s);
+    router_decode_kernel<<<grid, kRouterDecWarps * 32, smem, s>>>(x, T, H, Wr, bias, E, k, idx, w, logits,
+                                                                 build_units_flag, has_shared, units, ctrl);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- prefill: fp32 logits GEMM
+// C[T][E] = X[T][H] Wr[E][H]^T, 128x128 tile per CTA, 256 threads, 8x8 outputs per thread,
+// K-steps of 16 staged k-major in shared memory (double buffered).
+constexpr int RBM = 128, RBN = 128, RBK = 16;
+
+__global__ void __launch_bounds__(256)
+router_gemm_kernel(const uint16_t *__restrict__ x, int T, int H, const float *__restrict__ Wr, int E,
+                   float *__restrict__ C) {
+  __shared__ __align__(16) float As[2][RBK][RBM + 4];
+  __shared__ __align__(16) float Bs[2][RBK][RBN + 4];
+  const int tid = threadIdx.x;
+  const int m0 = blockIdx.y * RBM, n0 = blockIdx.x * RBN;
+  const int ty = tid / 16, tx = tid % 16;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+
+  // loaders: A: 128 rows x 16 bf16 = 256 threads x 8 values (16 bytes); B: 128 rows x 16 fp32 = 256 x 8
+  const int lrow = tid >> 1, lk = (tid & 1) * 8;
+  auto load_regs = [&](int k0, uint4 &ra, float4 &rb0, float4 &rb1) {
+    int gm = m0 + lrow, gn = n0 + lrow;
+    ra = (gm < T) ? *reinterpret_cast<const uint4 *>(x + (size_t)gm * H + k0 + lk) : make_uint4(0, 0, 0, 0);
+    if (gn < E) {
+      const float4 *p = reinterpret_cast<const float4 *>(Wr + (size_t)gn * H + k0 + lk);
+      rb0 = __ldg(p);
+      rb1 = __ldg(p + 1);
+    } else {
+      rb0 = rb1 = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto store_smem = [&](int buf, const uint4 &ra, const float4 &rb0, const float4 &rb1) {
+    const uint32_t av[4] = {ra.x, ra.y, ra.z, ra.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      As[buf][lk + 2 * i][lrow] = __uint_as_float(av[i] << 16);
+      As[buf][lk + 2 * i + 1][lrow] = __uint_as_float(av[i] & 0xffff0000u);
+    }
+    Bs[buf][lk + 0][lrow] = rb0.x; Bs[buf][lk + 1][lrow] = rb0.y;
+    Bs[buf][lk + 2][lrow] = rb0.z; Bs[buf][lk + 3][lrow] = rb0.w;
+    Bs[buf][lk + 4][lrow] = rb1.x; Bs[buf][lk + 5][lrow] = rb1.y;
+    Bs[buf][lk + 6][lrow] = rb1.z; Bs[buf][lk + 7][lrow] = rb1.w;
+  };
+  uint4 ra;
+  float4 rb0, rb1;
+  load_regs(0, ra, rb0, rb1);
+  store_smem(0, ra, rb0, rb1);
+  __syncthreads();
+  const int nk = H / RBK;
+  for (int kt = 0; kt < nk; ++kt) {
+    const int buf = kt & 1;
+    if (kt + 1 < nk) load_regs((kt + 1) * RBK, ra, rb0, rb1);
+#pragma unroll
+    for (int kk = 0; kk < RBK; ++kk) {
+      float a[8], b[8];
+      float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 4]);
+      float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][kk][64 + ty * 4]);
+      float4 b0 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 4]);
+      float4 b1 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][64 + tx * 4]);
+      a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w; a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
+      b[0] = b0.x; b[1] = b0.y; b[2] = b0.z; b[3] = b0.w; b[4] = b1.x; b[5] = b1.y; b[6] = b1.z; b[7] = b1.w;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    if (kt + 1 < nk) store_smem(buf ^ 1, ra, rb0, rb1);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int gm = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
+    if (gm >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      int gn = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
+      if (gn < E) C[(size_t)gm * E + gn] = acc[i][j];
+    }
+  }
+}
+
+// one warp per token; adds the bias into the stored logits
+constexpr int kTopkWarps = 8;
+__global__ void __launch_bounds__(kTopkWarps * 32)
+topk_kernel(float *__restrict__ logits, const float *__restrict__ bias, int T, int E, int k, int32_t *__restrict__ idx,
+            float *__restrict__ w) {
+  __shared__ uint32_t s_taken[kTopkWarps][kMaxE / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kTopkWarps + warp;
+  if (t >= T) return;
+  float *l = logits + (size_t)t * E;
+  if (E <= 512) {
+    warp_topk<16>(l, bias, E, k, idx + (size_t)t * k, w + (size_t)t * k);
+  } else {
+    for (int i = lane; i < kMaxE / 32; i += 32) s_taken[warp][i] = 0;
+    __syncwarp();
+    warp_topk_generic(l, bias, E, k, idx + (size_t)t * k, w + (size_t)t * k, s_taken[warp]);
+  }
+  __syncwarp();
+  if (bias)
+    for (int e = lane; e < E; e += 32) l[e] += bias[e];
+}
+
+cudaError_t launch_router_prefill(const uint16_t *x, int T, int H, const float *Wr, const float *bias, int E, int k,
+                                  int32_t *idx, float *w, float *logits, cudaStream_t s) {
+  dim3 grid((E + RBN - 1) / RBN, (T + RBM - 1) / RBM);
+  {
+    KTimer kt_(KID_ROUTER_GEMM, s);
+    router_gemm_kernel<<<grid, 256, 0, s>>>(x, T, H, Wr, E, logits);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  {
+    KTimer kt_(KID_TOPK, s);
+    topk_kernel<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(logits, bias, T, E, k, idx, w);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

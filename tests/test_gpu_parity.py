@@ -1,0 +1,238 @@
+"""GPU parity: every C-ABI entry point against the CPU oracle on the same seeded inputs.
+
+Integers (top-k indices, counts, offsets, permutation, dequantized values) must match bit for bit
+(an index may differ only at an oracle near-tie, gap < 1e-5, and the oracle then recomputes y
+with the GPU's selection); floating outputs must satisfy max|y - y_ref| / rms(y_ref) <= 1e-2 and
+routing weights <= 1e-5 absolute. Full-size configs are checked on sampled tokens (tokens are
+independent, so each sampled row is exact, not an approximation).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_expert_ffn_gemm_b200 as moe
+import synth
+from tests.gpu_util import W_TOL, Y_TOL, check_layer, compare_routing, rel_err, to_dev
+
+pytestmark = pytest.mark.gpu
+
+MID = synth.LayerShape("mid", 300, 512, 32, 4, 256, synth.Q2, True, 1.1, seed=3)
+MID_Q3 = synth.LayerShape("mid_q3", 200, 512, 32, 4, 256, synth.Q3, False, 1.2, seed=4)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    moe.lib()
+    torch.cuda.init()
+
+
+_cache = {}
+
+
+def layer_of(name):
+    if name not in _cache:
+        shape = {"mid": MID, "mid_q3": MID_Q3}.get(name) or synth.WORKLOADS[name]
+        L = synth.make_layer(shape)
+        _cache[name] = (L, to_dev(L))
+    return _cache[name]
+
+
+def ws_for(L, T=None):
+    s = L.shape
+    return moe.Workspace.for_layer(s.H, s.E, s.k, s.I, s.shared, T or s.T)
+
+
+# ----------------------------------------------------------------------------- generator on device
+def test_generator_device_bits_match_cpu():
+    a = synth.make_qmat(0, 1, 0, 2, synth.Q3, 3, 64, 256, device="cpu")
+    b = synth.make_qmat(0, 1, 0, 2, synth.Q3, 3, 64, 256, device="cuda")
+    assert torch.equal(a.codes, b.codes.cpu()) and torch.equal(a.hibits, b.hibits.cpu())
+    assert torch.equal(a.scales.view(torch.int16), b.scales.cpu().view(torch.int16))
+
+
+# ----------------------------------------------------------------------------- dequant
+@pytest.mark.parametrize("qtype", [synth.Q2, synth.Q3])
+def test_dequant_rows_bit_exact(qtype):
+    qm = synth.make_qmat(7, 0, 0, 0, qtype, 4, 96, 512)
+    dm = qm.to("cuda")
+    for e, r0, n in ((0, 0, 96), (3, 17, 5)):
+        f32, f16 = moe.dequant_rows(dm, e, r0, n)
+        ref, ref16 = oracle.dequant_rows(qm, e, r0, n)
+        assert np.array_equal(f32.cpu().double().numpy(), ref)
+        assert np.array_equal(f16.cpu().view(torch.int16).numpy().view(np.uint16), ref16)
+
+
+# ----------------------------------------------------------------------------- router
+@pytest.mark.parametrize("name", ["tiny", "decode1", "decode4", "mid", "prefill2k_q3"])
+def test_router_topk(name):
+    L, (x, Wr, b, _, _) = layer_of(name)
+    ws = ws_for(L)
+    idx, w, logits = moe.router_topk(x, Wr, b, L.shape.k, ws, want_logits=True)
+    idx_ref, w_ref, lg_ref, gap = oracle.router_topk(L.x, L.Wr, L.bias, L.shape.k)
+    lg = logits.cpu().double().numpy()
+    assert np.abs(lg - lg_ref).max() < 1e-5 * max(1.0, np.abs(lg_ref).max())
+    compare_routing(idx.cpu().numpy(), w.cpu().numpy(), idx_ref, w_ref, gap, lg_ref)
+    assert moe.read_device_error(ws) == 0
+
+
+def test_router_prefill_8k_all_tokens():
+    L, (x, Wr, b, _, _) = layer_of("prefill8k")
+    ws = ws_for(L)
+    idx, w = moe.router_topk(x, Wr, b, 10, ws)
+    idx_ref, w_ref, lg_ref, gap = oracle.router_topk(L.x, L.Wr, L.bias, 10)
+    flips = compare_routing(idx.cpu().numpy(), w.cpu().numpy(), idx_ref, w_ref, gap, lg_ref)
+    assert len(flips) < 64
+    # uniform router: every expert gets a share near T*k/E = 160 rows
+    counts = np.bincount(idx.cpu().numpy().reshape(-1), minlength=512)
+    assert counts.min() > 60 and counts.max() < 320
+
+
+# ----------------------------------------------------------------------------- permute / combine
+@pytest.mark.parametrize("T,k,E,shared", [(8192, 10, 512, True), (37, 3, 16, False), (1, 10, 512, True),
+                                          (5, 1, 4, False)])
+def test_permute_bit_exact(T, k, E, shared):
+    rng = np.random.default_rng(T + k)
+    idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    x = synth.make_x(1, T, 256)
+    ws = moe.Workspace.for_layer(256, E, k, 64, shared, T)
+    out = moe.permute(torch.from_numpy(idx).cuda(), E, x.cuda(), shared, ws)
+    counts, offsets, row_of, src = oracle.permute(idx, E)
+    assert np.array_equal(out["counts"][:E].cpu().numpy(), counts)
+    assert np.array_equal(out["offsets"][:E + 1].cpu().numpy(), offsets)
+    assert np.array_equal(out["row_of"].cpu().numpy(), row_of)
+    P = T * k
+    assert np.array_equal(out["src"][:P].cpu().numpy(), src)
+    xp = out["x_perm"].cpu()
+    ref = x.float().half()
+    assert torch.equal(xp[:P].view(torch.int16), ref[torch.from_numpy(src).long()].view(torch.int16))
+    if shared:
+        assert out["offsets"][E + 1].item() == P + T
+        assert np.array_equal(out["src"][P:].cpu().numpy(), np.arange(T))
+        assert torch.equal(xp[P:].view(torch.int16), ref.view(torch.int16))
+    assert moe.read_device_error(ws) == 0
+
+
+def test_permute_flags_bad_expert_index():
+    idx = torch.tensor([[0, 1], [2, 7], [3, 0]], dtype=torch.int32, device="cuda")  # 7 >= E = 4
+    ws = moe.Workspace.for_layer(256, 4, 2, 64, False, 3)
+    out = moe.permute(idx, 4, synth.make_x(0, 3, 256).cuda(), False, ws)
+    assert moe.read_device_error(ws) == moe.MOE_ERR_DEVICE_CHECK
+    assert out["row_of"][1, 1].item() == -1
+    assert moe.read_device_error(ws) == 0   # reading clears the word
+
+
+def test_combine_matches_definition():
+    rng = np.random.default_rng(0)
+    T, k, H = 33, 4, 512
+    rows = T * k + T
+    outp = torch.from_numpy(rng.normal(size=(rows, H)).astype(np.float16))
+    perm = rng.permutation(T * k).astype(np.int32).reshape(T, k)
+    w = torch.from_numpy(rng.uniform(size=(T, k)).astype(np.float32))
+    res = torch.from_numpy(rng.normal(size=(T, H)).astype(np.float32))
+    y = moe.combine(outp.cuda(), torch.from_numpy(perm).cuda(), w.cuda(), outp[T * k:].cuda(), res.cuda()).cpu()
+    o = outp.double().numpy()
+    ref = res.double().numpy() + o[T * k:] + np.einsum("tk,tkh->th", w.double().numpy(), o[perm])
+    assert np.abs(y.double().numpy() - ref).max() < 1e-4
+
+
+# ----------------------------------------------------------------------------- expert FFN (both paths)
+@pytest.mark.parametrize("name", ["tiny", "mid", "mid_q3"])
+@pytest.mark.parametrize("path", [moe.PATH_GEMV, moe.PATH_GEMM])
+def test_expert_ffn_rows(name, path):
+    L, (x, Wr, b, routed, shared) = layer_of(name)
+    s = L.shape
+    idx_ref, _, _, _ = oracle.router_topk(L.x, L.Wr, L.bias, s.k)
+    ws = ws_for(L)
+    pm = moe.permute(torch.from_numpy(idx_ref).cuda(), s.E, x, s.shared, ws)
+    n_rows = s.T * s.k + (s.T if s.shared else 0)
+    ws2 = moe.Workspace.for_layer(s.H, s.E, 1, s.I, False, n_rows)
+    out = moe.expert_ffn(pm["x_perm"], pm["offsets"], s.E, routed, shared, ws2, path=path)
+    assert moe.read_device_error(ws2) == 0
+    # oracle: each sampled row through its group's expert
+    offs = pm["offsets"].cpu().numpy()
+    xp = pm["x_perm"].cpu().double().numpy()
+    rng = np.random.default_rng(1)
+    sample = np.sort(rng.choice(n_rows, size=min(n_rows, 96), replace=False))
+    ref = np.zeros((len(sample), s.H))
+    for i, r in enumerate(sample):
+        g = int(np.searchsorted(offs[:s.E + (1 if s.shared else 0) + 1], r, side="right") - 1)
+        es, e = (L.shared, 0) if g == s.E else (L.routed, g)
+        ref[i] = oracle.expert_ffn_rows(es, e, xp[r:r + 1])[0]
+    got = out.cpu().double().numpy()[sample]
+    assert rel_err(got, ref) <= Y_TOL
+
+
+# ----------------------------------------------------------------------------- layer forward
+@pytest.mark.parametrize("name,ntok", [("tiny", 64), ("decode1", 1), ("decode4", 4), ("mid", 300),
+                                       ("mid_q3", 200), ("prefill8k", 24), ("prefill2k_q3", 24)])
+def test_layer_forward(name, ntok):
+    L, (x, Wr, b, routed, shared) = layer_of(name)
+    s = L.shape
+    ws = ws_for(L)
+    y, idx, w = moe.layer_forward(x, Wr, b, routed, shared, s.k, ws, want_routing=True)
+    assert moe.read_device_error(ws) == 0
+    tokens = np.arange(s.T) if ntok >= s.T else np.sort(np.random.default_rng(5).choice(s.T, ntok, replace=False))
+    err, flips = check_layer(y.cpu().numpy(), idx.cpu().numpy(), L, tokens)
+    print(f"{name}: max|dy|/rms = {err:.3e}, near-tie flips {len(flips)}")
+
+
+def test_layer_forward_with_residual_in_place():
+    L, (x, Wr, b, routed, shared) = layer_of("mid")
+    s = L.shape
+    r = synth.make_residual(9, s.T, s.H).cuda()
+    ws = ws_for(L)
+    y, idx, _ = moe.layer_forward(x, Wr, b, routed, shared, s.k, ws, residual=r.clone(), want_routing=True)
+    y2 = r.clone()
+    moe.layer_forward(x, Wr, b, routed, shared, s.k, ws, residual=y2, y=y2)  # aliasing residual and y
+    assert torch.equal(y, y2)
+    check_layer(y.cpu().numpy(), idx.cpu().numpy(), L, range(0, s.T, 7), residual=r.cpu().numpy())
+
+
+@pytest.mark.parametrize("name,T", [("mid", 64), ("mid", 4), ("mid_q3", 4), ("tiny", 4)])
+def test_cross_path_gemv_vs_gemm(name, T):
+    L, (x, Wr, b, routed, shared) = layer_of(name)
+    s = L.shape
+    ws = moe.Workspace.for_layer(s.H, s.E, s.k, s.I, s.shared, T)
+    ya = moe.layer_forward(x[:T], Wr, b, routed, shared, s.k, ws, path=moe.PATH_GEMV)
+    yb = moe.layer_forward(x[:T], Wr, b, routed, shared, s.k, ws, path=moe.PATH_GEMM)
+    assert rel_err(ya.cpu().numpy(), yb.cpu().numpy()) <= Y_TOL
+
+
+def test_mtp_verify_T4_equals_four_T1():
+    L, (x, Wr, b, routed, shared) = layer_of("decode4")
+    ws = ws_for(L)
+    y4 = moe.layer_forward(x, Wr, b, routed, shared, 10, ws).cpu().numpy()
+    for t in range(4):
+        y1 = moe.layer_forward(x[t:t + 1], Wr, b, routed, shared, 10, ws).cpu().numpy()
+        assert rel_err(y1, y4[t:t + 1]) < 1e-5  # same arithmetic up to fp32 summation order
+
+
+def test_zero_tokens_is_noop():
+    L, (x, Wr, b, routed, shared) = layer_of("tiny")
+    ws = ws_for(L)
+    y = moe.layer_forward(x[:0], Wr, b, routed, shared, 2, ws)
+    assert y.shape == (0, 256)
+
+
+# ----------------------------------------------------------------------------- RMSNorm and stacks
+def test_rmsnorm_matches_oracle():
+    r = synth.make_residual(2, 64, 2048) * 3.0
+    u = moe.rmsnorm_bf16(r.cuda()).cpu().view(torch.int16).numpy().view(np.uint16)
+    ref = oracle.rmsnorm_bf16(r)
+    diff = np.abs(u.astype(np.int32) - ref.astype(np.int32))
+    assert diff.max() <= 1                  # at most one bf16 ulp (fp32 vs fp64 rounding boundary)
+    assert (diff > 0).mean() < 0.01
+
+
+def test_stack_small_full_compare():
+    H, E, k, I, Lyr, T = 256, 16, 2, 128, 4, 12
+    Wrs = [synth.make_router(0, l, E, H) for l in range(Lyr)]
+    rs = [synth.make_expert_set(0, l, 0, 2, E, H, I) for l in range(Lyr)]
+    ss = [synth.make_expert_set(0, l, 1, 2, 1, H, I) for l in range(Lyr)]
+    r0 = synth.make_residual(0, T, H)
+    st = moe.Stack([w.cuda() for w in Wrs], None, [r.to("cuda") for r in rs], [s.to("cuda") for s in ss], k)
+    ws = moe.Workspace.for_layer(H, E, k, I, True, T)
+    r_out = moe.stack_forward(r0.cuda(), st, ws).cpu().numpy()
+    ref, _ = oracle.stack_forward(r0, list(zip(Wrs, [None] * Lyr, rs, ss)), k)
+    assert rel_err(r_out, ref) <= Y_TOL
