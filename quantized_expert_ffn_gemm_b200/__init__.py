@@ -279,3 +279,39 @@ def timing_read() -> dict:
         if cnt.value:
             out[n] = (ms.value, cnt.value)
     return out
+
+
+# ----------------------------------------------------------------------------- low-overhead layer handle
+class LayerHandle:
+    """A layer's weights bound once: descriptor and weight-plane structs are built at construction, so
+    each forward() is a single C call with plain integer arguments (suitable for CUDA-graph capture
+    and for tight decode loops)."""
+
+    _fast = None
+
+    def __init__(self, Wr: torch.Tensor, bias: Optional[torch.Tensor], routed, shared, k: int, ws: Workspace):
+        L = lib()
+        if LayerHandle._fast is None:
+            vp, i32 = ctypes.c_void_p, ctypes.c_int32
+            proto = ctypes.CFUNCTYPE(i32, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, ctypes.c_size_t, vp)
+            LayerHandle._fast = proto(("moe_layer_forward", L))
+        self.refs = (Wr, bias, routed, shared, ws)  # keep the tensors alive
+        self.H, self.E, self.k, self.I = Wr.shape[1], Wr.shape[0], k, routed.gate.rows
+        self.desc = layer_desc(self.H, self.E, k, self.I, shared is not None)
+        self.rs = expert_set(routed)
+        self.ss = expert_set(shared) if shared is not None else None
+        self._a = (Wr.data_ptr(), None if bias is None else bias.data_ptr(), ctypes.addressof(self.desc),
+                   ctypes.addressof(self.rs), None if self.ss is None else ctypes.addressof(self.ss))
+        self._ws = (ws.buf.data_ptr(), ws.nbytes)
+        self._fn = LayerHandle._fast
+
+    def forward(self, x: torch.Tensor, y: torch.Tensor, residual: Optional[torch.Tensor] = None,
+                idx_out: Optional[torch.Tensor] = None, w_out: Optional[torch.Tensor] = None, path: int = PATH_AUTO):
+        wr, b, d, rs, ss = self._a
+        code = self._fn(x.data_ptr(), x.shape[0], wr, b, d, rs, ss,
+                        None if residual is None else residual.data_ptr(), y.data_ptr(),
+                        None if idx_out is None else idx_out.data_ptr(), None if w_out is None else w_out.data_ptr(),
+                        path, self._ws[0], self._ws[1], torch.cuda.current_stream().cuda_stream)
+        if code != MOE_OK:
+            raise MoeError("moe_layer_forward", code)
+        return y

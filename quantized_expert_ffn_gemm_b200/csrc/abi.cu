@@ -64,6 +64,19 @@ int num_sms() {
   return cached[dev];
 }
 
+cudaError_t smem_limit_once_impl(const void *func, size_t bytes) {
+  // per-kernel record of the limit already set (keyed by the kernel's host stub address)
+  static std::mutex mu;
+  static std::vector<std::pair<const void *, size_t>> done;
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  std::lock_guard<std::mutex> lk(mu);
+  for (auto &d : done)
+    if (d.first == func && d.second >= bytes) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done.push_back({func, bytes});
+  return e;
+}
+
 }  // namespace moe
 
 using namespace moe;

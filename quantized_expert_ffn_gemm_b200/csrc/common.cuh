@@ -129,6 +129,14 @@ cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, i
 
 int num_sms();
 
+// Raise a kernel's dynamic shared memory limit once per process (kept out of later launches so
+// that launches can be captured into CUDA graphs).
+cudaError_t smem_limit_once_impl(const void *func, size_t bytes);
+template <class F>
+cudaError_t smem_limit_once(F *func, size_t bytes) {
+  return smem_limit_once_impl(reinterpret_cast<const void *>(func), bytes);
+}
+
 // ---------------------------------------------------------------- per-kernel timing (optional)
 enum KernelId {
   KID_ROUTER_DECODE = 0, KID_ROUTER_GEMM, KID_TOPK, KID_PERM_HIST, KID_PERM_SCAN, KID_PERM_SCATTER, KID_PERM_FILL,

@@ -55,9 +55,10 @@ __device__ __forceinline__ MatView mat_of(const moe_qmat &m, int expert) {
   return v;
 }
 
-// acc[4] += W[rows r0..r0+15] * X^T over the full K, X in shared memory (ncols columns, row
-// stride `xstride` halves, rotated layout). Columns >= ncols read as zero.
-__device__ __forceinline__ void warp_rows16(const MatView &m, int r0, const __half *xs, int xstride, int ncols,
+// acc[4] += W[rows r0..r0+15] * X^T over the full K, X in shared memory (column c present iff
+// bit c of `mask`, row stride `xstride` halves, rotated layout). Absent columns read as zero (their
+// shared memory was never staged and may hold anything).
+__device__ __forceinline__ void warp_rows16(const MatView &m, int r0, const __half *xs, int xstride, int mask,
                                             float acc[4]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int K = m.K;
@@ -66,7 +67,7 @@ __device__ __forceinline__ void warp_rows16(const MatView &m, int r0, const __ha
   const uint16_t *s0 = m.scales + (size_t)(r0 + g) * ss, *s1 = m.scales + (size_t)(r0 + g + 8) * ss;
   const uint8_t *h0 = m.q3 ? m.hibits + (size_t)(r0 + g) * hs : nullptr;
   const uint8_t *h1 = m.q3 ? m.hibits + (size_t)(r0 + g + 8) * hs : nullptr;
-  const bool colok = g < ncols;
+  const bool colok = (mask >> g) & 1;
   const __half *xcol = xs + (size_t)g * xstride;
   const int nsteps = (K + kStepK - 1) / kStepK;
   for (int sb = 0; sb < nsteps; sb += kMaxSteps) {
@@ -168,11 +169,8 @@ dec_gate_up_kernel(const void *__restrict__ x, int H, int I, moe_expert_set rout
   const moe_expert_set &es = un.set ? shared : routed;
   const MatView mv = mat_of(warp == 0 ? es.gate : es.up, un.expert);
   const int r0 = blockIdx.y * 16;
-  int ncols = 0;
-  for (int c = 0; c < 8; ++c)
-    if ((un.mask >> c) & 1) ncols = c + 1;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  warp_rows16(mv, r0, xs, xstride, ncols, acc);
+  warp_rows16(mv, r0, xs, xstride, un.mask, acc);
   if (warp == 1) {
     exch[g][2 * t] = acc[0];
     exch[g][2 * t + 1] = acc[1];
@@ -199,15 +197,15 @@ cudaError_t launch_decode_gate_up(const void *x, int x_is_bf16, int H, int I, co
   dim3 grid(max_units, I / 16);
   size_t smem = (size_t)8 * (H + 4) * 2;
   if (x_is_bf16) {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(dec_gate_up_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = smem_limit_once(dec_gate_up_kernel<true>, smem);
+    if (e != cudaSuccess) return e;
     {
       KTimer kt_(KID_DEC_GATE_UP, s);
       dec_gate_up_kernel<true><<<grid, 64, smem, s>>>(x, H, I, routed, sh, units, ctrl, hdec);
     }
   } else {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(dec_gate_up_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = smem_limit_once(dec_gate_up_kernel<false>, smem);
+    if (e != cudaSuccess) return e;
     {
       KTimer kt_(KID_DEC_GATE_UP, s);
       dec_gate_up_kernel<false><<<grid, 64, smem, s>>>(x, H, I, routed, sh, units, ctrl, hdec);
@@ -249,13 +247,10 @@ dec_down_kernel(int H, int I, moe_expert_set routed, moe_expert_set shared, cons
         *reinterpret_cast<uint32_t *>(myh + (size_t)c * xstride + xs_pos(2 * i)) = __ldcg(src + i);
     }
     __syncwarp();
-    int ncols = 0;
-    for (int c = 0; c < 8; ++c)
-      if ((un.mask >> c) & 1) ncols = c + 1;
     const moe_expert_set &es = un.set ? shared : routed;
     const MatView mv = mat_of(es.down, un.expert);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    warp_rows16(mv, r0, myh, xstride, ncols, acc);
+    warp_rows16(mv, r0, myh, xstride, un.mask, acc);
     __syncwarp();
     if (out_rows) {
 #pragma unroll
@@ -293,8 +288,8 @@ cudaError_t launch_decode_down(int H, int I, const moe_expert_set &routed, const
   (void)max_units;
   moe_expert_set sh = shared ? *shared : routed;
   size_t smem = (size_t)kDownWarps * 8 * (I + 4) * 2;
-  if (smem > 48 * 1024)
-    cudaFuncSetAttribute(dec_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = smem_limit_once(dec_down_kernel, smem);
+  if (e != cudaSuccess) return e;
   {
     KTimer kt_(KID_DEC_DOWN, s);
     dec_down_kernel<<<H / 16, kDownWarps * 32, smem, s>>>(H, I, routed, sh, units, ctrl, hdec, y, residual, T, out_rows);

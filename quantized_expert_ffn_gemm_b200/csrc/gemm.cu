@@ -434,7 +434,7 @@ template <int NMAT, int STAGES>
 cudaError_t launch_one(const CUtensorMap &tb, const CUtensorMap &c0r, const CUtensorMap &c1r, const CUtensorMap &c0s,
                        const CUtensorMap &c1s, const GemmArgs &a, int grid_x, int grid_y, cudaStream_t s) {
   const int smem = Smem<NMAT, STAGES>::kBytes + 1024;
-  cudaError_t e = cudaFuncSetAttribute(grouped_ffn_kernel<NMAT, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = smem_limit_once(grouped_ffn_kernel<NMAT, STAGES>, smem);
   if (e != cudaSuccess) return e;
   {
     KTimer kt_(NMAT == 2 ? KID_GEMM_GATE_UP : KID_GEMM_DOWN, s);

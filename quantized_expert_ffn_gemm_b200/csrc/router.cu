@@ -245,10 +245,8 @@ cudaError_t launch_router_decode(const uint16_t *x, int T, int H, const float *W
                                  DecUnit *units, Ctrl *ctrl, cudaStream_t s) {
   size_t smem = (size_t)T * (H > E ? H : E) * sizeof(float);
   int grid = (E + kRouterDecWarps - 1) / kRouterDecWarps;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(router_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
+  cudaError_t e = smem_limit_once(router_decode_kernel, smem);
+  if (e != cudaSuccess) return e;
   {
     KTimer kt_(KID_ROUTER_DECODE, s);
     router_decode_kernel<<<grid, kRouterDecWarps * 32, smem, s>>>(x, T, H, Wr, bias, E, k, idx, w, logits,
