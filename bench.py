@@ -160,7 +160,7 @@ def run_ours(args, world, rank, local):
     wl = WORKLOADS[args.workload]
     shape = synth.WORKLOADS[wl["shape"]]
     T, H, E, k, I = shape.T, shape.H, shape.E, shape.k, shape.I
-    n_layers = wl["layers"]
+    n_layers = args.layers or wl["layers"]
     dev = torch.device("cuda", torch.cuda.current_device())
     layers = build_layers(shape, n_layers)
     n_x = 64 if T <= 8 else 2
@@ -369,6 +369,8 @@ def main():
     ap.add_argument("--workload", default="decode1", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="distinct layer weight sets to rotate over (default 48 for decode, 4 for prefill)")
     ap.add_argument("--breakdown", action="store_true", help="also time T=4 and T=8192 on rank 0 (extra keys)")
     args = ap.parse_args()
     if args.steps is None:

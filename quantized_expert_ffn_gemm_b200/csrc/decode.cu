@@ -19,7 +19,6 @@
 namespace moe {
 
 constexpr int kStepK = 256;       // K covered by one warp step (4 lanes x 64 weights)
-constexpr int kMaxSteps = 8;      // steps whose loads are issued together (K <= 2048 in one batch)
 
 __device__ __forceinline__ void mma16816(float c[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -41,8 +40,28 @@ struct MatView {
   const uint8_t *hibits;
   const uint16_t *scales;
   int K;
-  int q3;
 };
+
+// matrix `which` (0 gate, 1 up, 2 down) of expert `expert` in set `set` (0 routed, 1 shared); scalar
+// selects only, so the kernel-parameter structs are never copied to local memory
+__device__ __forceinline__ MatView mat_sel(const moe_expert_set &r, const moe_expert_set &sh, int set, int which,
+                                           int expert) {
+#define MOE_SEL(field)                                                                                  \
+  (which == 0 ? (set ? sh.gate.field : r.gate.field)                                                    \
+              : which == 1 ? (set ? sh.up.field : r.up.field) : (set ? sh.down.field : r.down.field))
+  const uint8_t *codes = MOE_SEL(codes);
+  const uint8_t *hib = MOE_SEL(hibits);
+  const uint16_t *sc = MOE_SEL(scales);
+  const int rows = MOE_SEL(rows), K = MOE_SEL(K);
+#undef MOE_SEL
+  MatView v;
+  const size_t row0 = (size_t)expert * rows;
+  v.codes = codes + row0 * (K / 4);
+  v.hibits = hib ? hib + row0 * (K / 8) : nullptr;
+  v.scales = sc + row0 * (K / 32);
+  v.K = K;
+  return v;
+}
 
 __device__ __forceinline__ MatView mat_of(const moe_qmat &m, int expert) {
   MatView v;
@@ -51,104 +70,138 @@ __device__ __forceinline__ MatView mat_of(const moe_qmat &m, int expert) {
   v.hibits = m.hibits ? m.hibits + row0 * (m.K / 8) : nullptr;
   v.scales = m.scales + row0 * (m.K / 32);
   v.K = m.K;
-  v.q3 = (m.qtype == MOE_Q3);
   return v;
 }
 
-// acc[4] += W[rows r0..r0+15] * X^T over the full K, X in shared memory (column c present iff
-// bit c of `mask`, row stride `xstride` halves, rotated layout). Absent columns read as zero (their
-// shared memory was never staged and may hold anything).
-__device__ __forceinline__ void warp_rows16(const MatView &m, int r0, const __half *xs, int xstride, int mask,
-                                            float acc[4]) {
+// one lane's share of a 16-row x 256-wide K step: 16 code bytes of rows g and g+8, their two
+// block scales, and (Q3) the two blocks' hi-bit words
+struct StepFrag {
+  uint4 w0, w1;
+  uint32_t d0, d1;
+  uint2 h0, h1;
+};
+
+template <bool Q3>
+__device__ __forceinline__ void load_step(StepFrag &f, const MatView &m, int r0, int step, bool valid) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int K = m.K;
-  const size_t rs = (size_t)K / 4, ss = (size_t)K / 32, hs = (size_t)K / 8;
-  const uint8_t *c0 = m.codes + (size_t)(r0 + g) * rs, *c1 = m.codes + (size_t)(r0 + g + 8) * rs;
-  const uint16_t *s0 = m.scales + (size_t)(r0 + g) * ss, *s1 = m.scales + (size_t)(r0 + g + 8) * ss;
-  const uint8_t *h0 = m.q3 ? m.hibits + (size_t)(r0 + g) * hs : nullptr;
-  const uint8_t *h1 = m.q3 ? m.hibits + (size_t)(r0 + g + 8) * hs : nullptr;
-  const bool colok = (mask >> g) & 1;
-  const __half *xcol = xs + (size_t)g * xstride;
-  const int nsteps = (K + kStepK - 1) / kStepK;
-  for (int sb = 0; sb < nsteps; sb += kMaxSteps) {
-    uint4 w0[kMaxSteps], w1[kMaxSteps];
-    uint32_t d0[kMaxSteps], d1[kMaxSteps];
-    uint2 hb0[kMaxSteps], hb1[kMaxSteps];
+  const int k0 = step * kStepK + 64 * t;
+  const bool ok = valid && k0 < m.K;
+  const size_t rs = (size_t)m.K / 4, ss = (size_t)m.K / 32, hs = (size_t)m.K / 8;
+  const size_t ra = (size_t)(r0 + g), rb = (size_t)(r0 + g + 8);
+  f.w0 = ok ? __ldcs(reinterpret_cast<const uint4 *>(m.codes + ra * rs + k0 / 4)) : make_uint4(0, 0, 0, 0);
+  f.w1 = ok ? __ldcs(reinterpret_cast<const uint4 *>(m.codes + rb * rs + k0 / 4)) : make_uint4(0, 0, 0, 0);
+  f.d0 = ok ? __ldcs(reinterpret_cast<const uint32_t *>(m.scales + ra * ss + k0 / 32)) : 0u;
+  f.d1 = ok ? __ldcs(reinterpret_cast<const uint32_t *>(m.scales + rb * ss + k0 / 32)) : 0u;
+  if (Q3) {
+    f.h0 = ok ? __ldcs(reinterpret_cast<const uint2 *>(m.hibits + ra * hs + k0 / 8)) : make_uint2(0, 0);
+    f.h1 = ok ? __ldcs(reinterpret_cast<const uint2 *>(m.hibits + rb * hs + k0 / 8)) : make_uint2(0, 0);
+  }
+}
+
+// dequantize the fragment (zero codes with zero scales give zero weights) and run the step's 16
+// MMAs; B fragments come from the lane's column in shared memory when `bok`, else zero
+template <bool Q3>
+__device__ __forceinline__ void mma_step(float acc[4], const StepFrag &f, const __half *xcol, int kbase, bool bok) {
+  const uint32_t wr0[4] = {f.w0.x, f.w0.y, f.w0.z, f.w0.w};
+  const uint32_t wr1[4] = {f.w1.x, f.w1.y, f.w1.z, f.w1.w};
 #pragma unroll
-    for (int s = 0; s < kMaxSteps; ++s) {
-      const int k0 = (sb + s) * kStepK + 64 * t;
-      const bool ok = (sb + s < nsteps) && (k0 < K);
-      w0[s] = ok ? __ldcs(reinterpret_cast<const uint4 *>(c0 + k0 / 4)) : make_uint4(0, 0, 0, 0);
-      w1[s] = ok ? __ldcs(reinterpret_cast<const uint4 *>(c1 + k0 / 4)) : make_uint4(0, 0, 0, 0);
-      d0[s] = ok ? __ldcs(reinterpret_cast<const uint32_t *>(s0 + k0 / 32)) : 0u;
-      d1[s] = ok ? __ldcs(reinterpret_cast<const uint32_t *>(s1 + k0 / 32)) : 0u;
-      if (m.q3) {
-        hb0[s] = ok ? __ldcs(reinterpret_cast<const uint2 *>(h0 + k0 / 8)) : make_uint2(0, 0);
-        hb1[s] = ok ? __ldcs(reinterpret_cast<const uint2 *>(h1 + k0 / 8)) : make_uint2(0, 0);
-      } else {
-        hb0[s] = hb1[s] = make_uint2(0, 0);
-      }
+  for (int wq = 0; wq < 4; ++wq) {  // word wq: block wq/2, half q = wq%2
+    const int blk = wq >> 1, q = wq & 1;
+    const __half2 dd0 = __half2half2(__ushort_as_half((uint16_t)(f.d0 >> (16 * blk))));
+    const __half2 dd1 = __half2half2(__ushort_as_half((uint16_t)(f.d1 >> (16 * blk))));
+    uint32_t p0[8], p1[8];
+    if (Q3) {
+      dq3_word(wr0[wq], blk ? f.h0.y : f.h0.x, q, dd0, p0);
+      dq3_word(wr1[wq], blk ? f.h1.y : f.h1.x, q, dd1, p1);
+    } else {
+      dq2_word(wr0[wq], dd0, p0);
+      dq2_word(wr1[wq], dd1, p1);
     }
 #pragma unroll
-    for (int s = 0; s < kMaxSteps; ++s) {
-      if (sb + s >= nsteps) break;
-      const int kbase = (sb + s) * kStepK + 64 * t;
-      // lanes past the K tail hold zero codes and zero scales (A = 0) and read no activations;
-      // every lane still issues the warp-wide MMA
-      const bool kin = kbase < K;
-      const uint32_t wr0[4] = {w0[s].x, w0[s].y, w0[s].z, w0[s].w};
-      const uint32_t wr1[4] = {w1[s].x, w1[s].y, w1[s].z, w1[s].w};
-      const uint32_t hr0[2] = {hb0[s].x, hb0[s].y}, hr1[2] = {hb1[s].x, hb1[s].y};
-#pragma unroll
-      for (int wq = 0; wq < 4; ++wq) {  // word wq: block wq/2, half q = wq%2
-        const int blk = wq >> 1, q = wq & 1;
-        const __half2 dd0 = __half2half2(__ushort_as_half((uint16_t)(d0[s] >> (16 * blk))));
-        const __half2 dd1 = __half2half2(__ushort_as_half((uint16_t)(d1[s] >> (16 * blk))));
-        uint32_t p0[8], p1[8];
-        if (m.q3) {
-          dq3_word(wr0[wq], hr0[blk], q, dd0, p0);
-          dq3_word(wr1[wq], hr1[blk], q, dd1, p1);
-        } else {
-          dq2_word(wr0[wq], dd0, p0);
-          dq2_word(wr1[wq], dd1, p1);
-        }
-#pragma unroll
-        for (int mm = 0; mm < 4; ++mm) {  // MMA m = 4*wq + mm uses pairs 2mm, 2mm+1 of this word
-          const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
-          uint32_t b0 = 0, b1 = 0;
-          if (colok && kin) {
-            const int kk = kbase + 16 * wq + 4 * mm;
-            const uint2 bv = *reinterpret_cast<const uint2 *>(xcol + xs_pos(kk));
-            b0 = bv.x;
-            b1 = bv.y;
-          }
-          mma16816(acc, a, b0, b1);
-        }
+    for (int mm = 0; mm < 4; ++mm) {  // MMA 4*wq + mm uses pairs 2mm, 2mm+1 of this word
+      const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
+      uint32_t b0 = 0, b1 = 0;
+      if (bok) {
+        const uint2 bv = *reinterpret_cast<const uint2 *>(xcol + xs_pos(kbase + 16 * wq + 4 * mm));
+        b0 = bv.x;
+        b1 = bv.y;
       }
+      mma16816(acc, a, b0, b1);
     }
   }
 }
 
-// stage columns of the activation source into shared memory (fp16, rotated layout)
+// acc += W[r0..r0+15, steps s0..s0+NS-1] * X^T; all of the batch's loads are issued first
+template <bool Q3, int NS>
+__device__ __forceinline__ void rows16_batch(const MatView &m, int r0, int s0, int nsteps, const __half *xcol,
+                                             bool colok, float acc[4]) {
+  const int t = threadIdx.x & 3;
+  StepFrag f[NS];
+#pragma unroll
+  for (int s = 0; s < NS; ++s) load_step<Q3>(f[s], m, r0, s0 + s, s0 + s < nsteps);
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    const int kbase = (s0 + s) * kStepK + 64 * t;
+    mma_step<Q3>(acc, f[s], xcol, kbase, colok && (s0 + s < nsteps) && kbase < m.K);
+  }
+}
+
+// full K of 16 rows: batches of 8 steps, then a tail batch of 4, 2 or 1
+template <bool Q3>
+__device__ __forceinline__ void rows16(const MatView &m, int r0, const __half *xcol, bool colok, float acc[4]) {
+  const int nsteps = (m.K + kStepK - 1) / kStepK;
+  int s = 0;
+  for (; s + 8 <= nsteps; s += 8) rows16_batch<Q3, 8>(m, r0, s, nsteps, xcol, colok, acc);
+  const int rem = nsteps - s;
+  if (rem > 4) rows16_batch<Q3, 8>(m, r0, s, nsteps, xcol, colok, acc);
+  else if (rem > 2) rows16_batch<Q3, 4>(m, r0, s, nsteps, xcol, colok, acc);
+  else if (rem == 2) rows16_batch<Q3, 2>(m, r0, s, nsteps, xcol, colok, acc);
+  else if (rem == 1) rows16_batch<Q3, 1>(m, r0, s, nsteps, xcol, colok, acc);
+}
+
+// stage columns of the activation source into shared memory (fp16, rotated layout). 16-byte
+// loads, several issued before the first store, so the staging costs one memory round trip.
 template <bool SRC_BF16>
 __device__ __forceinline__ void stage_x(const void *src, int row0, int mask, int H, __half *xs, int xstride) {
-  const int H2 = H / 2;
+  const int H8 = H / 8;
+  const uint16_t *base = static_cast<const uint16_t *>(src);
   for (int c = 0; c < 8; ++c) {
     if (!((mask >> c) & 1)) continue;
-    const uint32_t *s = reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(src) + (size_t)(row0 + c) * H);
-    for (int i = threadIdx.x; i < H2; i += blockDim.x) {
-      uint32_t v = s[i];
-      __half2 h;
-      if (SRC_BF16) h = __floats2half2_rn(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
-      else h = *reinterpret_cast<__half2 *>(&v);
-      *reinterpret_cast<__half2 *>(xs + (size_t)c * xstride + xs_pos(2 * i)) = h;
+    const uint4 *sp = reinterpret_cast<const uint4 *>(base + (size_t)(row0 + c) * H);
+    for (int i0 = threadIdx.x; i0 < H8; i0 += 4 * blockDim.x) {
+      uint4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = i0 + j * blockDim.x;
+        v[j] = (i < H8) ? __ldg(sp + i) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = i0 + j * blockDim.x;
+        if (i >= H8) break;
+        uint4 o = v[j];
+        if (SRC_BF16) {
+          const uint32_t in[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+          uint32_t out[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            __half2 h = __floats2half2_rn(__uint_as_float(in[q] << 16), __uint_as_float(in[q] & 0xffff0000u));
+            out[q] = *reinterpret_cast<uint32_t *>(&h);
+          }
+          o = make_uint4(out[0], out[1], out[2], out[3]);
+        }
+        // rows are 8-byte aligned (stride H+4 halves): two 8-byte stores
+        uint2 *d = reinterpret_cast<uint2 *>(xs + (size_t)c * xstride + xs_pos(8 * i));
+        d[0] = make_uint2(o.x, o.y);
+        d[1] = make_uint2(o.z, o.w);
+      }
     }
   }
 }
 
 // ---------------------------------------------------------------- gate/up + SwiGLU
 // grid (max_units, I/16); block = 2 warps: warp 0 gate rows, warp 1 up rows (same 16 rows)
-template <bool SRC_BF16>
+template <bool SRC_BF16, bool Q3>
 __global__ void __launch_bounds__(64)
 dec_gate_up_kernel(const void *__restrict__ x, int H, int I, moe_expert_set routed, moe_expert_set shared,
                    const DecUnit *__restrict__ units, Ctrl *__restrict__ ctrl, uint16_t *__restrict__ hdec) {
@@ -163,14 +216,26 @@ dec_gate_up_kernel(const void *__restrict__ x, int H, int I, moe_expert_set rout
   const int xstride = H + 4;
   __half *xs = reinterpret_cast<__half *>(smem_raw);
   __shared__ float exch[16][8];
-  stage_x<SRC_BF16>(x, un.xrow0, un.mask, H, xs, xstride);
-  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const moe_expert_set &es = un.set ? shared : routed;
-  const MatView mv = mat_of(warp == 0 ? es.gate : es.up, un.expert);
+  const MatView mv = mat_sel(routed, shared, un.set, warp, un.expert);
   const int r0 = blockIdx.y * 16;
+  const bool colok = (un.mask >> g) & 1;
+  // the first batch's weight loads go out before the activations are staged
+  const int nsteps = (H + kStepK - 1) / kStepK;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  warp_rows16(mv, r0, xs, xstride, un.mask, acc);
+  if (nsteps == 8) {
+    StepFrag f[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) load_step<Q3>(f[s], mv, r0, s, true);
+    stage_x<SRC_BF16>(x, un.xrow0, un.mask, H, xs, xstride);
+    __syncthreads();
+#pragma unroll
+    for (int s = 0; s < 8; ++s) mma_step<Q3>(acc, f[s], xs + (size_t)g * xstride, s * kStepK + 64 * t, colok);
+  } else {
+    stage_x<SRC_BF16>(x, un.xrow0, un.mask, H, xs, xstride);
+    __syncthreads();
+    rows16<Q3>(mv, r0, xs + (size_t)g * xstride, colok, acc);
+  }
   if (warp == 1) {
     exch[g][2 * t] = acc[0];
     exch[g][2 * t + 1] = acc[1];
@@ -190,36 +255,45 @@ dec_gate_up_kernel(const void *__restrict__ x, int H, int I, moe_expert_set rout
   }
 }
 
-cudaError_t launch_decode_gate_up(const void *x, int x_is_bf16, int H, int I, const moe_expert_set &routed,
-                                  const moe_expert_set *shared, const DecUnit *units, int max_units, Ctrl *ctrl,
-                                  uint16_t *hdec, cudaStream_t s) {
-  moe_expert_set sh = shared ? *shared : routed;
-  dim3 grid(max_units, I / 16);
-  size_t smem = (size_t)8 * (H + 4) * 2;
-  if (x_is_bf16) {
-    cudaError_t e = smem_limit_once(dec_gate_up_kernel<true>, smem);
-    if (e != cudaSuccess) return e;
-    {
-      KTimer kt_(KID_DEC_GATE_UP, s);
-      dec_gate_up_kernel<true><<<grid, 64, smem, s>>>(x, H, I, routed, sh, units, ctrl, hdec);
-    }
-  } else {
-    cudaError_t e = smem_limit_once(dec_gate_up_kernel<false>, smem);
-    if (e != cudaSuccess) return e;
-    {
-      KTimer kt_(KID_DEC_GATE_UP, s);
-      dec_gate_up_kernel<false><<<grid, 64, smem, s>>>(x, H, I, routed, sh, units, ctrl, hdec);
-    }
+template <bool B, bool Q>
+static cudaError_t launch_gu(dim3 grid, size_t smem, cudaStream_t s, const void *x, int H, int I,
+                             const moe_expert_set &routed, const moe_expert_set &sh, const DecUnit *units, Ctrl *ctrl,
+                             uint16_t *hdec) {
+  cudaError_t e = smem_limit_once(dec_gate_up_kernel<B, Q>, smem);
+  if (e != cudaSuccess) return e;
+  {
+    KTimer kt_(KID_DEC_GATE_UP, s);
+    dec_gate_up_kernel<B, Q><<<grid, 64, smem, s>>>(x, H, I, routed, sh, units, ctrl, hdec);
   }
   return cudaGetLastError();
 }
 
-// ---------------------------------------------------------------- down (+ weighted combine)
-// grid H/16 (one 16-row output group per CTA); kDownWarps warps split the units. Combine mode:
-// acc_total += w_u[col] * (W_down[u] h_u) over units, reduced across warps in fixed order, then
-// y = acc (+ residual). Rows mode: each unit's 16 x ncols result is written to its output rows.
-constexpr int kDownWarps = 8;
+cudaError_t launch_decode_gate_up(const void *x, int x_is_bf16, int H, int I, const moe_expert_set &routed,
+                                  const moe_expert_set *shared, const DecUnit *units, int max_units, Ctrl *ctrl,
+                                  uint16_t *hdec, cudaStream_t s) {
+  const moe_expert_set sh = shared ? *shared : routed;
+  const dim3 grid(max_units, I / 16);
+  const size_t smem = (size_t)8 * (H + 4) * 2;
+  const bool q3 = routed.gate.qtype == MOE_Q3;
+  if (x_is_bf16)
+    return q3 ? launch_gu<true, true>(grid, smem, s, x, H, I, routed, sh, units, ctrl, hdec)
+              : launch_gu<true, false>(grid, smem, s, x, H, I, routed, sh, units, ctrl, hdec);
+  return q3 ? launch_gu<false, true>(grid, smem, s, x, H, I, routed, sh, units, ctrl, hdec)
+            : launch_gu<false, false>(grid, smem, s, x, H, I, routed, sh, units, ctrl, hdec);
+}
 
+// ---------------------------------------------------------------- down (+ weighted combine)
+// grid H/16 (one 16-row output group per CTA); kDownWarps warps split the units (a whole unit per
+// warp). Units are taken in chunks whose present h columns fit the shared budget; each warp
+// issues its unit's weight loads, then the chunk's h columns are staged, then the MMAs run.
+// Combine mode (y != NULL): acc_total += w_u[col] * (W_down[u] h_u) over units, reduced across
+// warps in fixed order, then y = acc (+ residual). Rows mode: each unit's 16 x 8 result goes to
+// its output rows.
+constexpr int kDownWarps = 8;
+constexpr int kDownSlots = 64;     // h columns staged at once
+constexpr int kDownMaxUnits = 128; // unit records cached in shared memory at a time
+
+template <bool Q3>
 __global__ void __launch_bounds__(kDownWarps * 32)
 dec_down_kernel(int H, int I, moe_expert_set routed, moe_expert_set shared, const DecUnit *__restrict__ units,
                 Ctrl *__restrict__ ctrl, const uint16_t *__restrict__ hdec, float *__restrict__ y,
@@ -229,42 +303,118 @@ dec_down_kernel(int H, int I, moe_expert_set routed, moe_expert_set shared, cons
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int r0 = blockIdx.x * 16;
   const int xstride = I + 4;
-  __half *hs = reinterpret_cast<__half *>(smem_raw);  // per warp: 8 columns x (I+4)
-  __half *myh = hs + (size_t)warp * 8 * xstride;
+  __half *hs = reinterpret_cast<__half *>(smem_raw);  // kDownSlots columns x (I + 4)
   __shared__ float red[kDownWarps][16][8];
+  __shared__ __align__(16) DecUnit s_units[kDownMaxUnits];
+  __shared__ int s_slot[kDownMaxUnits + 1];           // first staged slot of each unit of the chunk
+  __shared__ int s_src[kDownSlots];                   // h row (unit*8 + column) of each staged slot
+  __shared__ int s_u1;
   float tot[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int u = warp; u < nu; u += kDownWarps) {
-    const DecUnit un = units[u];
-    if (un.expert < 0 || un.expert >= (un.set ? shared.down.n_experts : routed.down.n_experts)) {
-      if (lane == 0 && blockIdx.x == 0) set_device_error(ctrl, MOE_ERR_DEVICE_CHECK, un.expert);
-      continue;
+  const int nsteps = (I + kStepK - 1) / kStepK;
+  for (int ub = 0; ub < nu; ub += kDownMaxUnits) {
+    const int ue = min(nu, ub + kDownMaxUnits);
+    // cache this batch of unit records (one coalesced read)
+    {
+      const int nwords = (ue - ub) * (int)(sizeof(DecUnit) / 16);
+      const uint4 *src = reinterpret_cast<const uint4 *>(units + ub);
+      uint4 *dst = reinterpret_cast<uint4 *>(s_units);
+      for (int i = threadIdx.x; i < nwords; i += blockDim.x) dst[i] = __ldg(src + i);
     }
-    // stage this unit's h columns (warp-local)
-    for (int c = 0; c < 8; ++c) {
-      if (!((un.mask >> c) & 1)) continue;
-      const uint32_t *src = reinterpret_cast<const uint32_t *>(hdec + ((size_t)u * 8 + c) * I);
-      for (int i = lane; i < I / 2; i += 32)
-        *reinterpret_cast<uint32_t *>(myh + (size_t)c * xstride + xs_pos(2 * i)) = __ldcg(src + i);
-    }
-    __syncwarp();
-    const moe_expert_set &es = un.set ? shared : routed;
-    const MatView mv = mat_of(es.down, un.expert);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    warp_rows16(mv, r0, myh, xstride, un.mask, acc);
-    __syncwarp();
-    if (out_rows) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int row = g + (e >> 1) * 8, col = 2 * t + (e & 1);
-        if ((un.mask >> col) & 1)
-          out_rows[(size_t)(un.xrow0 + col) * H + r0 + row] = __half_as_ushort(__float2half_rn(acc[e]));
+    __syncthreads();
+    int u0 = ub;
+    while (u0 < ue) {
+      if (threadIdx.x == 0) {  // chunk [u0, u1): whole units whose columns fit kDownSlots slots
+        int u1 = u0, used = 0;
+        while (u1 < ue) {
+          const int m = s_units[u1 - ub].mask & 0xff;
+          const int c = __popc(m);
+          if (used + c > kDownSlots) break;
+          s_slot[u1 - u0] = used;
+          for (int cc = 0; cc < 8; ++cc)
+            if ((m >> cc) & 1) s_src[used++] = u1 * 8 + cc;
+          ++u1;
+        }
+        s_slot[u1 - u0] = used;
+        s_u1 = u1;
       }
-    } else {
-      const float wa = un.w[2 * t], wb = un.w[2 * t + 1];
-      tot[0] = fmaf(wa, acc[0], tot[0]);
-      tot[1] = fmaf(wb, acc[1], tot[1]);
-      tot[2] = fmaf(wa, acc[2], tot[2]);
-      tot[3] = fmaf(wb, acc[3], tot[3]);
+      __syncthreads();
+      const int u1 = s_u1, nslots = s_slot[u1 - u0];
+      // each warp owns units u0 + warp, u0 + warp + kDownWarps, ...; its first unit's weights are
+      // requested before the chunk's h columns are staged
+      const int my_u = u0 + warp;
+      StepFrag f[2];
+      MatView mv{};
+      if (my_u < u1 && nsteps <= 2) {
+        const DecUnit &un = s_units[my_u - ub];
+        if (un.expert >= 0 && un.expert < (un.set ? shared.down.n_experts : routed.down.n_experts)) {
+          mv = mat_sel(routed, shared, un.set, 2, un.expert);
+          load_step<Q3>(f[0], mv, r0, 0, true);
+          load_step<Q3>(f[1], mv, r0, 1, nsteps > 1);
+        }
+      }
+      {  // stage the chunk's h columns: 16-byte loads, all of a thread's loads before its stores
+        const int I8 = I / 8, total = nslots * I8;
+        for (int v0 = threadIdx.x; v0 < total; v0 += 4 * blockDim.x) {
+          uint4 v[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int vi = v0 + j * blockDim.x;
+            v[j] = (vi < total) ? __ldcg(reinterpret_cast<const uint4 *>(hdec + (size_t)s_src[vi / I8] * I) + vi % I8)
+                                : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int vi = v0 + j * blockDim.x;
+            if (vi < total) {  // rows are 8-byte aligned (stride I+4 halves): two 8-byte stores
+              uint2 *d = reinterpret_cast<uint2 *>(hs + (size_t)(vi / I8) * xstride + xs_pos(8 * (vi % I8)));
+              d[0] = make_uint2(v[j].x, v[j].y);
+              d[1] = make_uint2(v[j].z, v[j].w);
+            }
+          }
+        }
+      }
+      __syncthreads();
+      for (int uu = my_u; uu < u1; uu += kDownWarps) {
+        const DecUnit &un = s_units[uu - ub];
+        if (un.expert < 0 || un.expert >= (un.set ? shared.down.n_experts : routed.down.n_experts)) {
+          if (lane == 0 && blockIdx.x == 0) set_device_error(ctrl, MOE_ERR_DEVICE_CHECK, un.expert);
+          continue;
+        }
+        if (uu != my_u || nsteps > 2) {
+          mv = mat_sel(routed, shared, un.set, 2, un.expert);
+          if (nsteps <= 2) {
+            load_step<Q3>(f[0], mv, r0, 0, true);
+            load_step<Q3>(f[1], mv, r0, 1, nsteps > 1);
+          }
+        }
+        // this lane's column slot (absent columns feed zeros)
+        const bool colok = (un.mask >> g) & 1;
+        const int slot = s_slot[uu - u0] + __popc(un.mask & ((1u << g) - 1u));
+        const __half *xcol = hs + (size_t)(colok ? slot : 0) * xstride;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        if (nsteps <= 2) {
+          mma_step<Q3>(acc, f[0], xcol, 64 * t, colok && 64 * t < I);
+          if (nsteps > 1) mma_step<Q3>(acc, f[1], xcol, kStepK + 64 * t, colok && kStepK + 64 * t < I);
+        } else {
+          rows16<Q3>(mv, r0, xcol, colok, acc);
+        }
+        if (out_rows) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int row = g + (e >> 1) * 8, col = 2 * t + (e & 1);
+            if ((un.mask >> col) & 1)
+              out_rows[(size_t)(un.xrow0 + col) * H + r0 + row] = __half_as_ushort(__float2half_rn(acc[e]));
+          }
+        } else {
+          const float wa = un.w[2 * t], wb = un.w[2 * t + 1];
+          tot[0] = fmaf(wa, acc[0], tot[0]);
+          tot[1] = fmaf(wb, acc[1], tot[1]);
+          tot[2] = fmaf(wa, acc[2], tot[2]);
+          tot[3] = fmaf(wb, acc[3], tot[3]);
+        }
+      }
+      __syncthreads();  // before the next chunk overwrites the staged columns and slot tables
+      u0 = u1;
     }
   }
   if (out_rows) return;
@@ -275,10 +425,10 @@ dec_down_kernel(int H, int I, moe_expert_set routed, moe_expert_set shared, cons
   __syncthreads();
   for (int i = threadIdx.x; i < 16 * T; i += blockDim.x) {
     const int row = i % 16, col = i / 16;  // consecutive threads -> consecutive output features
-    float s = residual ? residual[(size_t)col * H + r0 + row] : 0.0f;
+    float sum = residual ? residual[(size_t)col * H + r0 + row] : 0.0f;
 #pragma unroll
-    for (int wi = 0; wi < kDownWarps; ++wi) s += red[wi][row][col];
-    y[(size_t)col * H + r0 + row] = s;
+    for (int wi = 0; wi < kDownWarps; ++wi) sum += red[wi][row][col];
+    y[(size_t)col * H + r0 + row] = sum;
   }
 }
 
@@ -286,13 +436,19 @@ cudaError_t launch_decode_down(int H, int I, const moe_expert_set &routed, const
                                const DecUnit *units, int max_units, Ctrl *ctrl, const uint16_t *hdec, float *y,
                                const float *residual, int T, uint16_t *out_rows, cudaStream_t s) {
   (void)max_units;
-  moe_expert_set sh = shared ? *shared : routed;
-  size_t smem = (size_t)kDownWarps * 8 * (I + 4) * 2;
-  cudaError_t e = smem_limit_once(dec_down_kernel, smem);
+  const moe_expert_set sh = shared ? *shared : routed;
+  const size_t smem = (size_t)kDownSlots * (I + 4) * 2;
+  const bool q3 = routed.gate.qtype == MOE_Q3;
+  cudaError_t e = q3 ? smem_limit_once(dec_down_kernel<true>, smem) : smem_limit_once(dec_down_kernel<false>, smem);
   if (e != cudaSuccess) return e;
   {
     KTimer kt_(KID_DEC_DOWN, s);
-    dec_down_kernel<<<H / 16, kDownWarps * 32, smem, s>>>(H, I, routed, sh, units, ctrl, hdec, y, residual, T, out_rows);
+    if (q3)
+      dec_down_kernel<true><<<H / 16, kDownWarps * 32, smem, s>>>(H, I, routed, sh, units, ctrl, hdec, y, residual, T,
+                                                                  out_rows);
+    else
+      dec_down_kernel<false><<<H / 16, kDownWarps * 32, smem, s>>>(H, I, routed, sh, units, ctrl, hdec, y, residual,
+                                                                   T, out_rows);
   }
   return cudaGetLastError();
 }

@@ -240,9 +240,11 @@ grouped_ffn_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_consta
     const uint16_t *scp[NMAT];
     const uint8_t *hbp[NMAT];
 #pragma unroll
-    for (int m = 0; m < NMAT; ++m) {
-      scp[m] = args.scales[set][m] + grow * (K / 32);
-      hbp[m] = args.q3 ? args.hibits[set][m] + grow * (K / 8) : nullptr;
+    for (int m = 0; m < NMAT; ++m) {  // scalar selects keep the parameter block out of local memory
+      const uint16_t *sc = set ? args.scales[1][m] : args.scales[0][m];
+      const uint8_t *hb = set ? args.hibits[1][m] : args.hibits[0][m];
+      scp[m] = sc + grow * (K / 32);
+      hbp[m] = args.q3 ? hb + grow * (K / 8) : nullptr;
     }
     // scales (and Q3 hi words) for groups of 4 stages, prefetched one group ahead
     uint32_t sc_cur[NMAT][4], sc_nxt[NMAT][4], hb_cur[NMAT][4], hb_nxt[NMAT][4];

@@ -27,7 +27,19 @@ __device__ __forceinline__ uint32_t logit_key(float f) {
 // Top-k of E logits (l[0..E) in shared or global memory) by one warp. Writes idx[0..k) and
 // w[0..k). Rounds of: per-lane best among untaken candidates (ascending index scan, strict >,
 // so the lower index wins a tie inside a lane), warp max of the key, then warp min of the index
-// among lanes holding that key.
+// among lanes holding that key. Lane j keeps the winner of round j, so the k selections end up
+// spread over lanes 0..k-1 and the softmax over the set is one warp reduction.
+__device__ __forceinline__ void topk_finish(float my_val, int my_idx, int k, int32_t *idx, float *w) {
+  const int lane = threadIdx.x & 31;
+  const float l0 = __shfl_sync(0xffffffffu, my_val, 0);
+  const float ev = (lane < k) ? expf(my_val - l0) : 0.0f;
+  const float z = warp_sum(ev);
+  if (lane < k) {
+    idx[lane] = my_idx;
+    w[lane] = ev / z;
+  }
+}
+
 template <int PER_LANE>
 __device__ void warp_topk(const float *l, const float *bias, int E, int k, int32_t *idx, float *w) {
   const int lane = threadIdx.x & 31;
@@ -35,118 +47,124 @@ __device__ void warp_topk(const float *l, const float *bias, int E, int k, int32
   float val[PER_LANE];
 #pragma unroll
   for (int i = 0; i < PER_LANE; ++i) {
-    int e = lane + 32 * i;
-    float v = -INFINITY;
-    if (e < E) v = l[e] + (bias ? bias[e] : 0.0f);
+    const int e = lane + 32 * i;
+    const float v = (e < E) ? l[e] + (bias ? bias[e] : 0.0f) : -INFINITY;
     val[i] = v;
     key[i] = (e < E) ? logit_key(v) : 0u;
   }
   uint32_t taken = 0;
-  float sel_val[kMaxK];
-  int sel_idx[kMaxK];
+  float my_val = -INFINITY;
+  int my_idx = 0;
   for (int j = 0; j < k; ++j) {
     uint32_t bk = 0;
     int bi = 0x7fffffff;
     float bv = -INFINITY;
 #pragma unroll
     for (int i = 0; i < PER_LANE; ++i) {
-      int e = lane + 32 * i;
-      bool ok = (e < E) && !((taken >> i) & 1u);
+      const int e = lane + 32 * i;
+      const bool ok = (e < E) && !((taken >> i) & 1u);
       if (ok && (key[i] > bk || bi == 0x7fffffff)) { bk = key[i]; bi = e; bv = val[i]; }
     }
-    uint32_t m = __reduce_max_sync(0xffffffffu, bi == 0x7fffffff ? 0u : bk);
-    uint32_t cand = (bi != 0x7fffffff && bk == m) ? (uint32_t)bi : 0xffffffffu;
-    uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bi == 0x7fffffff ? 0u : bk);
+    const uint32_t cand = (bi != 0x7fffffff && bk == m) ? (uint32_t)bi : 0xffffffffu;
+    const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
     if ((uint32_t)bi == win) taken |= 1u << ((bi - lane) / 32);
-    float wv = __shfl_sync(0xffffffffu, bv, (int)(win & 31u));
-    sel_val[j] = wv;
-    sel_idx[j] = (int)win;
+    const float wv = __shfl_sync(0xffffffffu, bv, (int)(win & 31u));
+    if (lane == j) { my_val = wv; my_idx = (int)win; }
   }
-  if (lane == 0) {
-    float l0 = sel_val[0], z = 0.0f;
-    for (int j = 0; j < k; ++j) z += expf(sel_val[j] - l0);
-    float inv = 1.0f / z;
-    for (int j = 0; j < k; ++j) {
-      idx[j] = sel_idx[j];
-      w[j] = expf(sel_val[j] - l0) * inv;
-    }
-  }
+  topk_finish(my_val, my_idx, k, idx, w);
 }
 
 // generic E (up to kMaxE) from shared memory: lanes rescan their strided candidates each round
 __device__ void warp_topk_generic(const float *l, const float *bias, int E, int k, int32_t *idx, float *w,
                                   uint32_t *taken_words /* smem, E/32 words, zeroed */) {
   const int lane = threadIdx.x & 31;
-  float sel_val[kMaxK];
-  int sel_idx[kMaxK];
+  float my_val = -INFINITY;
+  int my_idx = 0;
   for (int j = 0; j < k; ++j) {
     uint32_t bk = 0;
     int bi = 0x7fffffff;
     float bv = -INFINITY;
     for (int e = lane; e < E; e += 32) {
       if ((taken_words[e >> 5] >> (e & 31)) & 1u) continue;
-      float v = l[e] + (bias ? bias[e] : 0.0f);
-      uint32_t kk = logit_key(v);
+      const float v = l[e] + (bias ? bias[e] : 0.0f);
+      const uint32_t kk = logit_key(v);
       if (kk > bk || bi == 0x7fffffff) { bk = kk; bi = e; bv = v; }
     }
-    uint32_t m = __reduce_max_sync(0xffffffffu, bi == 0x7fffffff ? 0u : bk);
-    uint32_t cand = (bi != 0x7fffffff && bk == m) ? (uint32_t)bi : 0xffffffffu;
-    uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bi == 0x7fffffff ? 0u : bk);
+    const uint32_t cand = (bi != 0x7fffffff && bk == m) ? (uint32_t)bi : 0xffffffffu;
+    const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
     if ((uint32_t)bi == win) taken_words[bi >> 5] |= 1u << (bi & 31);
     __syncwarp();
-    sel_val[j] = __shfl_sync(0xffffffffu, bv, (int)(win & 31u));
-    sel_idx[j] = (int)win;
+    const float wv = __shfl_sync(0xffffffffu, bv, (int)(win & 31u));
+    if (lane == j) { my_val = wv; my_idx = (int)win; }
   }
-  if (lane == 0) {
-    float l0 = sel_val[0], z = 0.0f;
-    for (int j = 0; j < k; ++j) z += expf(sel_val[j] - l0);
-    float inv = 1.0f / z;
-    for (int j = 0; j < k; ++j) {
-      idx[j] = sel_idx[j];
-      w[j] = expf(sel_val[j] - l0) * inv;
-    }
-  }
+  topk_finish(my_val, my_idx, k, idx, w);
 }
 
 // ---------------------------------------------------------------- decode units
 // Group the T*k selected (token, slot) pairs by distinct expert, in order of first appearance
-// (token-major), plus the always-on shared expert as the last unit. One warp.
+// (token-major), plus the always-on shared expert as the last unit. One warp, built in shared
+// memory and written out with coalesced stores.
+struct UnitScratch {
+  int first[kDecodeMaxT * kMaxK];
+  int unit[kDecodeMaxT * kMaxK];
+  int expert[kDecodeMaxT * kMaxK + 1];
+  int mask[kDecodeMaxT * kMaxK + 1];
+  float w[kDecodeMaxT * kMaxK + 1][8];
+};
+
 __device__ void build_units(const int32_t *sidx, const float *sw, int T, int k, int has_shared, DecUnit *units,
-                            Ctrl *ctrl, int *s_first, int *s_unit) {
+                            Ctrl *ctrl, UnitScratch &us) {
   const int lane = threadIdx.x & 31;
   const int P = T * k;
   for (int p = lane; p < P; p += 32) {
-    int e = sidx[p], f = p;
+    const int e = sidx[p];
+    int f = p;
     for (int q = 0; q < p; ++q)
       if (sidx[q] == e) { f = q; break; }
-    s_first[p] = f;
+    us.first[p] = f;
   }
   __syncwarp();
-  if (lane == 0) {  // unit numbering of the leaders in pair order (P <= 256)
-    int nu = 0;
-    for (int p = 0; p < P; ++p) s_unit[p] = (s_first[p] == p) ? nu++ : -1;
-    ctrl->n_units = nu + (has_shared ? 1 : 0);
-    for (int u = 0; u < nu + (has_shared ? 1 : 0); ++u) {
-      units[u].mask = 0;
-      units[u].xrow0 = 0;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) units[u].w[c] = 0.0f;
-    }
-    for (int p = 0; p < P; ++p) {
-      int u = s_unit[s_first[p]];
-      int t = p / k;
-      units[u].expert = sidx[p];
-      units[u].set = 0;
-      units[u].mask |= 1 << t;
-      units[u].w[t] = sw[p];
-    }
-    if (has_shared) {
-      units[nu].expert = 0;
-      units[nu].set = 1;
-      units[nu].mask = (1 << T) - 1;
-      for (int t = 0; t < T; ++t) units[nu].w[t] = 1.0f;
-    }
+  int nu = 0;  // leaders numbered in pair order
+  for (int base = 0; base < P; base += 32) {
+    const int p = base + lane;
+    const bool lead = (p < P) && us.first[p] == p;
+    const unsigned bal = __ballot_sync(0xffffffffu, lead);
+    if (lead) us.unit[p] = nu + __popc(bal & ((1u << lane) - 1u));
+    nu += __popc(bal);
   }
+  const int total = nu + (has_shared ? 1 : 0);
+  for (int u = lane; u < total; u += 32) {
+    us.mask[u] = 0;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) us.w[u][c] = 0.0f;
+  }
+  __syncwarp();
+  for (int p = lane; p < P; p += 32) {  // each (unit, token) is hit once: an expert appears once per token
+    const int u = us.unit[us.first[p]], t = p / k;
+    us.expert[u] = sidx[p];
+    atomicOr(&us.mask[u], 1 << t);
+    us.w[u][t] = sw[p];
+  }
+  __syncwarp();
+  if (has_shared && lane == 0) {
+    us.expert[nu] = 0;
+    us.mask[nu] = (1 << T) - 1;
+    for (int t = 0; t < T; ++t) us.w[nu][t] = 1.0f;
+  }
+  __syncwarp();
+  for (int u = lane; u < total; u += 32) {
+    DecUnit d;
+    d.expert = us.expert[u];
+    d.set = (u == nu) ? 1 : 0;
+    d.mask = us.mask[u];
+    d.xrow0 = 0;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) d.w[c] = us.w[u][c];
+    units[u] = d;
+  }
+  if (lane == 0) ctrl->n_units = total;
 }
 
 // ---------------------------------------------------------------- decode router kernel
@@ -160,7 +178,28 @@ router_decode_kernel(const uint16_t *__restrict__ x, int T, int H, const float *
   extern __shared__ float4 smem4[];
   float *xs = reinterpret_cast<float *>(smem4);  // [T][H] fp32, later reused for [T][E] logits
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int i = tid; i < T * H; i += blockDim.x) xs[i] = bf16_bits_to_float(x[i]);
+  {  // 16-byte loads of x, all of a thread's loads issued before its stores
+    const int n8 = T * H / 8;
+    for (int i0 = tid; i0 < n8; i0 += 4 * blockDim.x) {
+      uint4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = i0 + j * blockDim.x;
+        v[j] = (i < n8) ? __ldg(reinterpret_cast<const uint4 *>(x) + i) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = i0 + j * blockDim.x;
+        if (i < n8) {
+          float4 *d = reinterpret_cast<float4 *>(xs + 8 * i);
+          d[0] = make_float4(__uint_as_float(v[j].x << 16), __uint_as_float(v[j].x & 0xffff0000u),
+                             __uint_as_float(v[j].y << 16), __uint_as_float(v[j].y & 0xffff0000u));
+          d[1] = make_float4(__uint_as_float(v[j].z << 16), __uint_as_float(v[j].z & 0xffff0000u),
+                             __uint_as_float(v[j].w << 16), __uint_as_float(v[j].w & 0xffff0000u));
+        }
+      }
+    }
+  }
   __syncthreads();
 
   const int H4 = H >> 2;
@@ -212,7 +251,12 @@ router_decode_kernel(const uint16_t *__restrict__ x, int T, int H, const float *
   if (!s_last) return;
   __threadfence();
   float *ls = xs;  // [T][E]
-  for (int i = tid; i < T * E; i += blockDim.x) ls[i] = __ldcg(logits + i);
+  if ((E & 3) == 0) {
+    for (int i = tid; i < T * E / 4; i += blockDim.x)
+      reinterpret_cast<float4 *>(ls)[i] = __ldcg(reinterpret_cast<const float4 *>(logits) + i);
+  } else {
+    for (int i = tid; i < T * E; i += blockDim.x) ls[i] = __ldcg(logits + i);
+  }
   __shared__ int32_t s_idx[kDecodeMaxT * kMaxK];
   __shared__ float s_w[kDecodeMaxT * kMaxK];
   __shared__ uint32_t s_taken[kRouterDecWarps][kMaxE / 32];
@@ -235,8 +279,8 @@ router_decode_kernel(const uint16_t *__restrict__ x, int T, int H, const float *
     for (int i = tid; i < T * E; i += blockDim.x) logits[i] = ls[i] + bias[i % E];
   }
   if (build && warp == 0) {
-    __shared__ int s_first[kDecodeMaxT * kMaxK], s_unit[kDecodeMaxT * kMaxK];
-    build_units(s_idx, s_w, T, k, has_shared, units, ctrl, s_first, s_unit);
+    __shared__ UnitScratch s_us;
+    build_units(s_idx, s_w, T, k, has_shared, units, ctrl, s_us);
   }
 }
 
