@@ -101,7 +101,8 @@ __device__ __forceinline__ void load_step(StepFrag &f, const MatView &m, int r0,
 // dequantize the fragment (zero codes with zero scales give zero weights) and run the step's 16
 // MMAs; B fragments come from the lane's column in shared memory when `bok`, else zero
 template <bool Q3>
-__device__ __forceinline__ void mma_step(float acc[4], const StepFrag &f, const __half *xcol, int kbase, bool bok) {
+__device__ __forceinline__ void mma_step(float acc[4], float acc2[4], const StepFrag &f, const __half *xcol, int kbase,
+                                         bool bok) {
   const uint32_t wr0[4] = {f.w0.x, f.w0.y, f.w0.z, f.w0.w};
   const uint32_t wr1[4] = {f.w1.x, f.w1.y, f.w1.z, f.w1.w};
 #pragma unroll
@@ -126,7 +127,7 @@ __device__ __forceinline__ void mma_step(float acc[4], const StepFrag &f, const 
         b0 = bv.x;
         b1 = bv.y;
       }
-      mma16816(acc, a, b0, b1);
+      mma16816((mm & 1) ? acc2 : acc, a, b0, b1);
     }
   }
 }
@@ -139,11 +140,14 @@ __device__ __forceinline__ void rows16_batch(const MatView &m, int r0, int s0, i
   StepFrag f[NS];
 #pragma unroll
   for (int s = 0; s < NS; ++s) load_step<Q3>(f[s], m, r0, s0 + s, s0 + s < nsteps);
+  float acc2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int s = 0; s < NS; ++s) {
     const int kbase = (s0 + s) * kStepK + 64 * t;
-    mma_step<Q3>(acc, f[s], xcol, kbase, colok && (s0 + s < nsteps) && kbase < m.K);
+    mma_step<Q3>(acc, acc2, f[s], xcol, kbase, colok && (s0 + s < nsteps) && kbase < m.K);
   }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) acc[e] += acc2[e];
 }
 
 // full K of 16 rows: batches of 8 steps, then a tail batch of 4, 2 or 1
@@ -200,9 +204,13 @@ __device__ __forceinline__ void stage_x(const void *src, int row0, int mask, int
 }
 
 // ---------------------------------------------------------------- gate/up + SwiGLU
-// grid (max_units, I/16); block = 2 warps: warp 0 gate rows, warp 1 up rows (same 16 rows)
+// grid (max_units, I/16); block = 8 warps: warps 0-3 gate, 4-7 up, for the same 16 rows; warp
+// slice q takes K steps q, q+4, ... so every warp has a short MMA chain and the SM has many
+// warps in flight. Partials are summed in shared memory in fixed order.
+constexpr int kGuWarps = 8;
+
 template <bool SRC_BF16, bool Q3>
-__global__ void __launch_bounds__(64)
+__global__ void __launch_bounds__(kGuWarps * 32)
 dec_gate_up_kernel(const void *__restrict__ x, int H, int I, moe_expert_set routed, moe_expert_set shared,
                    const DecUnit *__restrict__ units, Ctrl *__restrict__ ctrl, uint16_t *__restrict__ hdec) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -215,40 +223,45 @@ dec_gate_up_kernel(const void *__restrict__ x, int H, int I, moe_expert_set rout
   }
   const int xstride = H + 4;
   __half *xs = reinterpret_cast<__half *>(smem_raw);
-  __shared__ float exch[16][8];
+  __shared__ float part[kGuWarps][16][8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const MatView mv = mat_sel(routed, shared, un.set, warp, un.expert);
+  const int mat = warp >> 2, slice = warp & 3;
+  const MatView mv = mat_sel(routed, shared, un.set, mat, un.expert);
   const int r0 = blockIdx.y * 16;
   const bool colok = (un.mask >> g) & 1;
-  // the first batch's weight loads go out before the activations are staged
   const int nsteps = (H + kStepK - 1) / kStepK;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  if (nsteps == 8) {
-    StepFrag f[8];
-#pragma unroll
-    for (int s = 0; s < 8; ++s) load_step<Q3>(f[s], mv, r0, s, true);
+  const __half *xcol = xs + (size_t)g * xstride;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
+  if (nsteps <= 8) {
+    // at most two steps per slice: request them before staging the activations
+    StepFrag f[2];
+    load_step<Q3>(f[0], mv, r0, slice, slice < nsteps);
+    load_step<Q3>(f[1], mv, r0, slice + 4, slice + 4 < nsteps);
     stage_x<SRC_BF16>(x, un.xrow0, un.mask, H, xs, xstride);
     __syncthreads();
-#pragma unroll
-    for (int s = 0; s < 8; ++s) mma_step<Q3>(acc, f[s], xs + (size_t)g * xstride, s * kStepK + 64 * t, colok);
+    if (slice < nsteps) mma_step<Q3>(acc, acc2, f[0], xcol, slice * kStepK + 64 * t,
+                                     colok && slice * kStepK + 64 * t < H);
+    if (slice + 4 < nsteps) mma_step<Q3>(acc, acc2, f[1], xcol, (slice + 4) * kStepK + 64 * t,
+                                         colok && (slice + 4) * kStepK + 64 * t < H);
   } else {
     stage_x<SRC_BF16>(x, un.xrow0, un.mask, H, xs, xstride);
     __syncthreads();
-    rows16<Q3>(mv, r0, xs + (size_t)g * xstride, colok, acc);
+    for (int st = slice; st < nsteps; st += 4) {
+      StepFrag f;
+      load_step<Q3>(f, mv, r0, st, true);
+      mma_step<Q3>(acc, acc2, f, xcol, st * kStepK + 64 * t, colok && st * kStepK + 64 * t < H);
+    }
   }
-  if (warp == 1) {
-    exch[g][2 * t] = acc[0];
-    exch[g][2 * t + 1] = acc[1];
-    exch[g + 8][2 * t] = acc[2];
-    exch[g + 8][2 * t + 1] = acc[3];
-  }
+  part[warp][g][2 * t] = acc[0] + acc2[0];
+  part[warp][g][2 * t + 1] = acc[1] + acc2[1];
+  part[warp][g + 8][2 * t] = acc[2] + acc2[2];
+  part[warp][g + 8][2 * t + 1] = acc[3] + acc2[3];
   __syncthreads();
-  if (warp == 0) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int row = g + (e >> 1) * 8, col = 2 * t + (e & 1);
-      if (!((un.mask >> col) & 1)) continue;
-      const float gv = acc[e], uv = exch[row][col];
+  if (threadIdx.x < 128) {  // one (row, column) per thread
+    const int row = threadIdx.x & 15, col = threadIdx.x >> 4;
+    if ((un.mask >> col) & 1) {
+      const float gv = (part[0][row][col] + part[1][row][col]) + (part[2][row][col] + part[3][row][col]);
+      const float uv = (part[4][row][col] + part[5][row][col]) + (part[6][row][col] + part[7][row][col]);
       const float hv = gv / (1.0f + expf(-gv)) * uv;
       hdec[((size_t)u * 8 + col) * I + r0 + row] = __half_as_ushort(__float2half_rn(hv));
     }
@@ -263,7 +276,7 @@ static cudaError_t launch_gu(dim3 grid, size_t smem, cudaStream_t s, const void 
   if (e != cudaSuccess) return e;
   {
     KTimer kt_(KID_DEC_GATE_UP, s);
-    dec_gate_up_kernel<B, Q><<<grid, 64, smem, s>>>(x, H, I, routed, sh, units, ctrl, hdec);
+    dec_gate_up_kernel<B, Q><<<grid, kGuWarps * 32, smem, s>>>(x, H, I, routed, sh, units, ctrl, hdec);
   }
   return cudaGetLastError();
 }
@@ -289,7 +302,7 @@ cudaError_t launch_decode_gate_up(const void *x, int x_is_bf16, int H, int I, co
 // Combine mode (y != NULL): acc_total += w_u[col] * (W_down[u] h_u) over units, reduced across
 // warps in fixed order, then y = acc (+ residual). Rows mode: each unit's 16 x 8 result goes to
 // its output rows.
-constexpr int kDownWarps = 8;
+constexpr int kDownWarps = 16;
 constexpr int kDownSlots = 64;     // h columns staged at once
 constexpr int kDownMaxUnits = 128; // unit records cached in shared memory at a time
 
@@ -339,17 +352,22 @@ dec_down_kernel(int H, int I, moe_expert_set routed, moe_expert_set shared, cons
       }
       __syncthreads();
       const int u1 = s_u1, nslots = s_slot[u1 - u0];
-      // each warp owns units u0 + warp, u0 + warp + kDownWarps, ...; its first unit's weights are
-      // requested before the chunk's h columns are staged
-      const int my_u = u0 + warp;
+      // work items: combine mode (unit, K step) pairs, rows mode whole units; item i goes to warp
+      // i % kDownWarps. A warp's first two items' weights are requested before h is staged.
+      const int per_unit = out_rows ? 1 : nsteps;
+      const int n_items = (u1 - u0) * per_unit;
       StepFrag f[2];
-      MatView mv{};
-      if (my_u < u1 && nsteps <= 2) {
-        const DecUnit &un = s_units[my_u - ub];
-        if (un.expert >= 0 && un.expert < (un.set ? shared.down.n_experts : routed.down.n_experts)) {
-          mv = mat_sel(routed, shared, un.set, 2, un.expert);
-          load_step<Q3>(f[0], mv, r0, 0, true);
-          load_step<Q3>(f[1], mv, r0, 1, nsteps > 1);
+      bool okv[2] = {false, false};
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int it = warp + j * kDownWarps;
+        if (it < n_items && (per_unit > 1 || nsteps == 1)) {
+          const DecUnit &un = s_units[u0 + it / per_unit - ub];
+          if (un.expert >= 0 && un.expert < (un.set ? shared.down.n_experts : routed.down.n_experts)) {
+            load_step<Q3>(f[j], mat_sel(routed, shared, un.set, 2, un.expert), r0, per_unit > 1 ? it % per_unit : 0,
+                          true);
+            okv[j] = true;
+          }
         }
       }
       {  // stage the chunk's h columns: 16-byte loads, all of a thread's loads before its stores
@@ -374,29 +392,36 @@ dec_down_kernel(int H, int I, moe_expert_set routed, moe_expert_set shared, cons
         }
       }
       __syncthreads();
-      for (int uu = my_u; uu < u1; uu += kDownWarps) {
+      for (int it = warp, j = 0; it < n_items; it += kDownWarps, ++j) {
+        const int uu = u0 + it / per_unit;
         const DecUnit &un = s_units[uu - ub];
         if (un.expert < 0 || un.expert >= (un.set ? shared.down.n_experts : routed.down.n_experts)) {
           if (lane == 0 && blockIdx.x == 0) set_device_error(ctrl, MOE_ERR_DEVICE_CHECK, un.expert);
           continue;
         }
-        if (uu != my_u || nsteps > 2) {
-          mv = mat_sel(routed, shared, un.set, 2, un.expert);
-          if (nsteps <= 2) {
-            load_step<Q3>(f[0], mv, r0, 0, true);
-            load_step<Q3>(f[1], mv, r0, 1, nsteps > 1);
-          }
-        }
         // this lane's column slot (absent columns feed zeros)
         const bool colok = (un.mask >> g) & 1;
         const int slot = s_slot[uu - u0] + __popc(un.mask & ((1u << g) - 1u));
         const __half *xcol = hs + (size_t)(colok ? slot : 0) * xstride;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        if (nsteps <= 2) {
-          mma_step<Q3>(acc, f[0], xcol, 64 * t, colok && 64 * t < I);
-          if (nsteps > 1) mma_step<Q3>(acc, f[1], xcol, kStepK + 64 * t, colok && kStepK + 64 * t < I);
-        } else {
-          rows16<Q3>(mv, r0, xcol, colok, acc);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
+        if (per_unit > 1 || nsteps == 1) {  // one K step
+          const int st = per_unit > 1 ? it % per_unit : 0;
+          StepFrag fl;
+          if (j == 0 && okv[0]) fl = f[0];
+          else if (j == 1 && okv[1]) fl = f[1];
+          else load_step<Q3>(fl, mat_sel(routed, shared, un.set, 2, un.expert), r0, st, true);
+          mma_step<Q3>(acc, acc2, fl, xcol, st * kStepK + 64 * t, colok && st * kStepK + 64 * t < I);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[e] += acc2[e];
+        } else {  // rows mode with several K steps: one step at a time (keeps register use low)
+          const MatView mv = mat_sel(routed, shared, un.set, 2, un.expert);
+          for (int st = 0; st < nsteps; ++st) {
+            StepFrag fl;
+            load_step<Q3>(fl, mv, r0, st, true);
+            mma_step<Q3>(acc, acc2, fl, xcol, st * kStepK + 64 * t, colok && st * kStepK + 64 * t < I);
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[e] += acc2[e];
         }
         if (out_rows) {
 #pragma unroll

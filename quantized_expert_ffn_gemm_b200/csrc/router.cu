@@ -208,15 +208,15 @@ router_decode_kernel(const uint16_t *__restrict__ x, int T, int H, const float *
     float acc[kDecodeMaxT];
 #pragma unroll
     for (int t = 0; t < kDecodeMaxT; ++t) acc[t] = 0.0f;
-    for (int h0 = 0; h0 < H4; h0 += 32 * 8) {
-      float4 v[8];
+    for (int h0 = 0; h0 < H4; h0 += 32 * 16) {  // H = 2048: the whole row in one round of loads
+      float4 v[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 16; ++u) {
         int h4 = h0 + lane + 32 * u;
         v[u] = (h4 < H4) ? __ldcs(wr + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 16; ++u) {
         int h4 = h0 + lane + 32 * u;
         if (h4 < H4) {
 #pragma unroll
