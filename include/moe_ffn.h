@@ -206,6 +206,19 @@ moe_status moe_stack_forward(const float *r_in, int32_t T, int32_t L, const floa
 moe_status moe_dequant_rows(const moe_qmat *m, int32_t expert, int32_t row0, int32_t nrows, float *out_f32,
                             uint16_t *out_f16, void *stream);
 
+/* Router and top-k without a workspace, for callers that cannot allocate device memory (code
+ * running under CUDA-graph capture, plugins whose host application owns all device memory,
+ * runtimes with no device allocator). The pages have no counterpart: this is a variant of
+ * moe_router_topk (same arguments, same results) whose scratch -- a control word and the [T][E]
+ * fp32 logits -- is a fixed array inside the library (about 128 KB, held on every GPU that loads
+ * the library until the process exits). Limits: T <= 8, E <= 4096 (and T * max(H, E) * 4 <=
+ * 200 KB); larger requests return MOE_ERR_UNSUPPORTED. The first call on each device looks up
+ * the array's device address and should come before any stream capture. All calls share the
+ * array: calls that overlap on the GPU race and must be serialised by the caller. It allocates
+ * no memory. */
+moe_status moe_router_topk_static(const uint16_t *x, int32_t T, int32_t H, const float *Wr, const float *bias,
+                                  int32_t E, int32_t k, int32_t *idx, float *w, float *logits_opt, void *stream);
+
 /* Per-kernel device timing, off by default. While enabled, the library records a pair of CUDA
  * events on the launching stream around every kernel it launches (from the calling host thread;
  * not for use during CUDA-graph capture) and keeps them in a process-wide list. Enabling (on = 1)

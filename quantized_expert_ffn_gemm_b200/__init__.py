@@ -26,7 +26,7 @@ Q2, Q3 = 2, 3
 EXPORTED = ["moe_status_string", "moe_workspace_bytes", "moe_workspace_init", "moe_rmsnorm_bf16",
             "moe_router_topk", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
             "moe_stack_forward", "moe_dequant_rows", "moe_read_device_error", "moe_timing_enable",
-            "moe_timing_read", "moe_kernel_count", "moe_kernel_name"]
+            "moe_timing_read", "moe_kernel_count", "moe_kernel_name", "moe_router_topk_static"]
 
 
 class MoeError(RuntimeError):
@@ -153,6 +153,19 @@ def router_topk(x: torch.Tensor, Wr: torch.Tensor, bias: Optional[torch.Tensor],
     logits = torch.empty(T, E, dtype=torch.float32, device=x.device) if want_logits else None
     _check("moe_router_topk", lib().moe_router_topk(_p(x), T, H, _p(Wr), _p(bias), E, k, _p(idx), _p(w), _p(logits),
                                                     ws.ptr, ws.size, _stream()))
+    return (idx, w, logits) if want_logits else (idx, w)
+
+
+def router_topk_static(x: torch.Tensor, Wr: torch.Tensor, bias: Optional[torch.Tensor], k: int,
+                       want_logits: bool = False):
+    """moe_router_topk_static: the same routing without a workspace (fixed scratch inside the library)."""
+    T, H = x.shape
+    E = Wr.shape[0]
+    idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
+    w = torch.empty(T, k, dtype=torch.float32, device=x.device)
+    logits = torch.empty(T, E, dtype=torch.float32, device=x.device) if want_logits else None
+    _check("moe_router_topk_static", lib().moe_router_topk_static(_p(x), T, H, _p(Wr), _p(bias), E, k, _p(idx),
+                                                                  _p(w), _p(logits), _stream()))
     return (idx, w, logits) if want_logits else (idx, w)
 
 
