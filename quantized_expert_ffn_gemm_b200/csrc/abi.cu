@@ -34,7 +34,7 @@ cudaEvent_t take_event() {
 const char *const kKernelNames[KID_COUNT] = {
     "router_decode", "router_gemm", "topk", "perm_hist", "perm_scan", "perm_scatter", "perm_fill",
     "perm_gather", "combine", "rmsnorm", "dequant_rows", "dec_units", "dec_gate_up", "dec_down",
-    "tile_list", "gemm_gate_up", "gemm_down"};
+    "tile_list", "gemm_gate_up", "gemm_down", "router_split", "router_tc"};
 }  // namespace
 
 void timer_begin(int kid, cudaStream_t s) {
@@ -187,7 +187,8 @@ moe_status moe_router_topk(const uint16_t *x, int32_t T, int32_t H, const float 
   if (decode_router_fits(T, H, E))
     return cuda_status(launch_router_decode(x, T, H, Wr, bias, E, k, idx, w, logits, 0, 0, at<DecUnit>(ws, L.units),
                                             ctrl, s));
-  return cuda_status(launch_router_prefill(x, T, H, Wr, bias, E, k, idx, w, logits, s));
+  return cuda_status(
+      launch_router_prefill(x, T, H, Wr, bias, E, k, idx, w, logits, at<uint16_t>(ws, L.wsplit), ctrl, s));
 }
 
 moe_status moe_permute(const int32_t *idx, int32_t T, int32_t k, int32_t E, const uint16_t *x, int32_t H,
@@ -308,7 +309,7 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
     if (decode_router_fits(T, H, E))
       e = launch_router_decode(x, T, H, Wr, bias, E, k, idx, w, logits, 0, 0, at<DecUnit>(ws, L.units), ctrl, s);
     else
-      e = launch_router_prefill(x, T, H, Wr, bias, E, k, idx, w, logits, s);
+      e = launch_router_prefill(x, T, H, Wr, bias, E, k, idx, w, logits, at<uint16_t>(ws, L.wsplit), ctrl, s);
     if (e == cudaSuccess)
       e = launch_permute(idx, T, k, E, x, H, hs, counts, offsets, row_of, src, xperm, at<int32_t>(ws, L.hist), ctrl,
                          s);

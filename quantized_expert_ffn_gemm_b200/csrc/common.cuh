@@ -1,6 +1,7 @@
 // Internal declarations shared by the kernels and the C-ABI layer of libmoe_ffn.so.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -43,7 +44,8 @@ struct DecUnit {
 
 // ---------------------------------------------------------------- workspace layout
 struct WsLayout {
-  size_t ctrl, logits, idx, w, hist, units, hdec, counts, offsets, row_of, src, xperm, hperm, operm, u16, tiles, total;
+  size_t ctrl, logits, idx, w, hist, units, hdec, counts, offsets, row_of, src, xperm, hperm, operm, u16, tiles, wsplit,
+      total;
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -75,6 +77,7 @@ inline WsLayout ws_layout(int H, int E, int k, int I, int has_shared, int T) {
   L.operm = take(rows * (size_t)H * 2);
   L.u16 = take((size_t)T * H * 2);
   L.tiles = take((rows / 16 + (size_t)E + 4) * 8);
+  L.wsplit = take((size_t)E * 3 * H * 2);
   L.total = off;
   return L;
 }
@@ -100,7 +103,14 @@ cudaError_t launch_router_decode(const uint16_t *x, int T, int H, const float *W
                                  int32_t *idx, float *w, float *logits, int build_units, int has_shared,
                                  DecUnit *units, Ctrl *ctrl, cudaStream_t s);
 cudaError_t launch_router_prefill(const uint16_t *x, int T, int H, const float *Wr, const float *bias, int E, int k,
-                                  int32_t *idx, float *w, float *logits, cudaStream_t s);
+                                  int32_t *idx, float *w, float *logits, uint16_t *wsplit, Ctrl *ctrl, cudaStream_t s);
+// tensor-core router logits (fp32 weights split into three bf16 planes); logits include the bias
+bool router_tc_supported(int H, int E);
+cudaError_t launch_router_tc(const uint16_t *x, int T, int H, const float *Wr, const float *bias, int E,
+                             uint16_t *wsplit, float *logits, Ctrl *ctrl, cudaStream_t s);
+// 2-D TMA descriptor over a row-major [rows][inner] tensor
+bool encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dt, int esize, const void *ptr, uint64_t inner,
+                          uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw);
 cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const uint16_t *x, int H, int with_shared,
                            int32_t *counts, int32_t *offsets, int32_t *row_of, int32_t *src, uint16_t *x_perm,
                            int32_t *hist, Ctrl *ctrl, cudaStream_t s);
@@ -141,7 +151,7 @@ cudaError_t smem_limit_once(F *func, size_t bytes) {
 enum KernelId {
   KID_ROUTER_DECODE = 0, KID_ROUTER_GEMM, KID_TOPK, KID_PERM_HIST, KID_PERM_SCAN, KID_PERM_SCATTER, KID_PERM_FILL,
   KID_PERM_GATHER, KID_COMBINE, KID_RMSNORM, KID_DEQUANT_ROWS, KID_DEC_UNITS, KID_DEC_GATE_UP, KID_DEC_DOWN,
-  KID_TILE_LIST, KID_GEMM_GATE_UP, KID_GEMM_DOWN, KID_COUNT
+  KID_TILE_LIST, KID_GEMM_GATE_UP, KID_GEMM_DOWN, KID_ROUTER_SPLIT, KID_ROUTER_TC, KID_COUNT
 };
 void timer_begin(int kid, cudaStream_t s);
 void timer_end(int kid, cudaStream_t s);

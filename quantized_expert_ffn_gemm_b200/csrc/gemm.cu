@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "dequant.cuh"
+#include "tc.cuh"
 
 namespace moe {
 
@@ -34,7 +35,6 @@ constexpr int kBNMax = 256;        // token rows per tile (MMA N upper bound)
 constexpr int kBoxRows = 32;       // rows per TMA box of the activation tile
 constexpr int kThreads = 320;      // warp 0 TMA, warp 1 MMA/TMEM, warps 2..9 dequant + epilogue
 constexpr int kDqThreads = 256;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 struct GemmArgs {
   const int32_t *offsets;
@@ -49,82 +49,6 @@ struct GemmArgs {
   const uint16_t *scales[2][2];    // [set][mat]
   const uint8_t *hibits[2][2];     // [set][mat]
 };
-
-// ---------------------------------------------------------------- PTX wrappers
-__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t tx) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(tx) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-// wait for the completion of the phase with parity `parity`; false if it did not come in time
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
-  }
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-          "r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t r[8]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// UMMA shared-memory descriptor: K-major, 128B swizzle, 8-row atoms 1024 bytes apart
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)1u << 16;              // leading byte offset (unused for swizzled K-major)
-  d |= (uint64_t)(1024u >> 4) << 32;    // stride byte offset
-  d |= (uint64_t)1u << 46;              // descriptor version
-  d |= (uint64_t)2u << 61;              // SWIZZLE_128B
-  return d;
-}
-// instruction descriptor, kind::f16: A = B = fp16, D = fp32, both K-major, M = 128, N
-__device__ __forceinline__ uint32_t idesc_f16(int N) {
-  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
-}
 
 __device__ __forceinline__ void record_timeout(Ctrl *c, int where) { set_device_error(c, MOE_ERR_TIMEOUT, where); }
 
@@ -400,35 +324,12 @@ __global__ void __launch_bounds__(1024) tile_list_kernel(const int32_t *__restri
 
 // ---------------------------------------------------------------- host side
 namespace {
+}  // namespace
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// 2-D map over a row-major [rows][inner] tensor
-bool make_map(CUtensorMap *map, CUtensorMapDataType dt, int esize, const void *ptr, uint64_t inner, uint64_t rows,
-              uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
-  auto enc = get_encode();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner * (uint64_t)esize};
-  cuuint32_t box[2] = {box_inner, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
+namespace {
 
 bool make_code_map(CUtensorMap *map, const moe_qmat &m) {
-  return make_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, m.codes, (uint64_t)m.K / 4, (uint64_t)m.n_experts * m.rows,
+  return encode_tensor_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, m.codes, (uint64_t)m.K / 4, (uint64_t)m.n_experts * m.rows,
                   kBK / 4, kBM, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
@@ -447,6 +348,31 @@ cudaError_t launch_one(const CUtensorMap &tb, const CUtensorMap &c0r, const CUte
 
 }  // namespace
 
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+bool encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dt, int esize, const void *ptr, uint64_t inner,
+                          uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * (uint64_t)esize};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int gemm_shape_supported(int H, int I) { return (H % 128 == 0 && I % 128 == 0 && H >= 128 && I >= 128) ? 1 : 0; }
 
 cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, int n_rows, int E, int H, int I,
@@ -463,10 +389,10 @@ cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, i
   const int max_tiles = n_rows / kBNMax + G + 1;
 
   CUtensorMap tx, th, cg, cu, cd, sg, su, sd;
-  bool ok = make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x_perm, H, n_rows, kBK, kBoxRows,
-                     CU_TENSOR_MAP_SWIZZLE_128B) &&
-            make_map(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h_perm, I, n_rows, kBK, kBoxRows,
-                     CU_TENSOR_MAP_SWIZZLE_128B) &&
+  bool ok = encode_tensor_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x_perm, H, n_rows, kBK, kBoxRows,
+                                 CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_tensor_map_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h_perm, I, n_rows, kBK, kBoxRows,
+                                 CU_TENSOR_MAP_SWIZZLE_128B) &&
             make_code_map(&cg, routed.gate) && make_code_map(&cu, routed.up) && make_code_map(&cd, routed.down) &&
             make_code_map(&sg, sh.gate) && make_code_map(&su, sh.up) && make_code_map(&sd, sh.down);
   if (!ok) return cudaErrorInvalidValue;

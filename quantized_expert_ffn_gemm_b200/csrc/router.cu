@@ -403,18 +403,128 @@ topk_kernel(float *__restrict__ logits, const float *__restrict__ bias, int T, i
     for (int e = lane; e < E; e += 32) l[e] += bias[e];
 }
 
-cudaError_t launch_router_prefill(const uint16_t *x, int T, int H, const float *Wr, const float *bias, int E, int k,
-                                  int32_t *idx, float *w, float *logits, cudaStream_t s) {
-  dim3 grid((E + RBN - 1) / RBN, (T + RBM - 1) / RBM);
-  {
-    KTimer kt_(KID_ROUTER_GEMM, s);
-    router_gemm_kernel<<<grid, 256, 0, s>>>(x, T, H, Wr, E, logits);
+// ---------------------------------------------------------------- screen + exact refine
+// After the tensor-core logits (accurate to ~1e-5 only: the tensor core's fp32 accumulation over
+// 3H terms is not an fp32 FMA chain), every expert whose approximate logit is within kMargin of
+// the approximate k-th logit is a candidate; the exact top-k is always among them because the
+// margin is far above twice the approximation error. Candidates get their logit recomputed with
+// an fp32 dot product (x is exact in fp32) plus bias, the top-k (lower index wins ties) and the
+// weights are taken from those exact values, and the exact values are written back.
+constexpr float kRefineMargin = 2e-3f;
+constexpr int kRefineWarps = 8;
+
+__global__ void __launch_bounds__(kRefineWarps * 32)
+topk_refine_kernel(float *__restrict__ logits, const uint16_t *__restrict__ x, const float *__restrict__ Wr,
+                   const float *__restrict__ bias, int T, int H, int E, int k, int32_t *__restrict__ idx,
+                   float *__restrict__ w) {
+  __shared__ float s_ex[kRefineWarps][512];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kRefineWarps + warp;
+  if (t >= T) return;
+  float *l = logits + (size_t)t * E;
+  // approximate logits (bias included) and the approximate k-th value
+  float val[16];
+  uint32_t key[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int e = lane + 32 * i;
+    val[i] = (e < E) ? l[e] : -INFINITY;
+    key[i] = (e < E) ? logit_key(val[i]) : 0u;
   }
-  cudaError_t e = cudaGetLastError();
+  uint32_t taken = 0;
+  float vk = 0.0f;
+  for (int j = 0; j < k; ++j) {
+    uint32_t bk = 0;
+    int bi = 0x7fffffff;
+    float bv = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int e = lane + 32 * i;
+      const bool ok = (e < E) && !((taken >> i) & 1u);
+      if (ok && (key[i] > bk || bi == 0x7fffffff)) { bk = key[i]; bi = e; bv = val[i]; }
+    }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bi == 0x7fffffff ? 0u : bk);
+    const uint32_t cand = (bi != 0x7fffffff && bk == m) ? (uint32_t)bi : 0xffffffffu;
+    const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+    if ((uint32_t)bi == win) taken |= 1u << ((bi - lane) / 32);
+    vk = __shfl_sync(0xffffffffu, bv, (int)(win & 31u));
+  }
+  const float thr = vk - kRefineMargin;
+  // x row in registers (fp32, exact), lane holds h = 4 * (lane + 32 j)
+  float4 xr[16];
+  const int H4 = H / 4;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int h4 = lane + 32 * j;
+    if (h4 < H4) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2 *>(x + (size_t)t * H) + h4);
+      xr[j] = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u), __uint_as_float(v.y << 16),
+                          __uint_as_float(v.y & 0xffff0000u));
+    } else {
+      xr[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  float *ex = s_ex[warp];
+  for (int e = lane; e < E; e += 32) ex[e] = -INFINITY;
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    unsigned bal = __ballot_sync(0xffffffffu, (lane + 32 * i < E) && val[i] >= thr);
+    while (bal) {
+      const int e = (__ffs(bal) - 1) + 32 * i;
+      bal &= bal - 1;
+      const float4 *wr = reinterpret_cast<const float4 *>(Wr + (size_t)e * H);
+      float acc = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int h4 = lane + 32 * j;
+        if (h4 < H4) {
+          const float4 wv = __ldg(wr + h4);
+          acc = fmaf(wv.x, xr[j].x, acc);
+          acc = fmaf(wv.y, xr[j].y, acc);
+          acc = fmaf(wv.z, xr[j].z, acc);
+          acc = fmaf(wv.w, xr[j].w, acc);
+        }
+      }
+      acc = warp_sum(acc);
+      if (lane == 0) ex[e] = acc + (bias ? bias[e] : 0.0f);
+    }
+  }
+  __syncwarp();
+  warp_topk<16>(ex, nullptr, E, k, idx + (size_t)t * k, w + (size_t)t * k);
+  __syncwarp();
+  for (int e = lane; e < E; e += 32)  // exact values where computed
+    if (ex[e] != -INFINITY) l[e] = ex[e];
+}
+
+bool router_refine_supported(int H, int E) { return H <= 2048 && E <= 512; }
+
+cudaError_t launch_router_prefill(const uint16_t *x, int T, int H, const float *Wr, const float *bias, int E, int k,
+                                  int32_t *idx, float *w, float *logits, uint16_t *wsplit, Ctrl *ctrl, cudaStream_t s) {
+  cudaError_t e;
+  if (router_tc_supported(H, E) && router_refine_supported(H, E)) {
+    e = launch_router_tc(x, T, H, Wr, bias, E, wsplit, logits, ctrl, s);  // logits include the bias
+    if (e != cudaSuccess) return e;
+    {
+      KTimer kt_(KID_TOPK, s);
+      topk_refine_kernel<<<(T + kRefineWarps - 1) / kRefineWarps, kRefineWarps * 32, 0, s>>>(logits, x, Wr, bias, T,
+                                                                                         H, E, k, idx, w);
+    }
+    return cudaGetLastError();
+  }
+  const float *topk_bias = bias;
+  {
+    dim3 grid((E + RBN - 1) / RBN, (T + RBM - 1) / RBM);
+    {
+      KTimer kt_(KID_ROUTER_GEMM, s);
+      router_gemm_kernel<<<grid, 256, 0, s>>>(x, T, H, Wr, E, logits);
+    }
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
   {
     KTimer kt_(KID_TOPK, s);
-    topk_kernel<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(logits, bias, T, E, k, idx, w);
+    topk_kernel<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(logits, topk_bias, T, E, k, idx, w);
   }
   return cudaGetLastError();
 }
