@@ -53,58 +53,110 @@ struct GemmArgs {
 __device__ __forceinline__ void record_timeout(Ctrl *c, int where) { set_device_error(c, MOE_ERR_TIMEOUT, where); }
 
 // ---------------------------------------------------------------- the grouped GEMM kernel
-template <int NMAT, int STAGES>
-struct Smem {
+// Persistent: gridDim.x CTAs walk the tile list round-robin (tile ti = blockIdx.x + i * gridDim.x,
+// entry = ti / n_mtiles, m-tile = ti % n_mtiles), so consecutive CTAs share a token block and the
+// roles never drain between tiles.
+//   warp 0      TMA producer: activation rows (swizzled) + the 128 weight rows' code plane
+//   warp 1      TMEM owner and single-thread MMA issuer
+//   warps 2-9   dequant: code plane + per-block scales (+ Q3 hi bits) -> fp16 A tile
+//   warps 10-13 epilogue: TMEM -> registers -> global, one lane quadrant each
+// Shared-memory ring of kStages stages (full_b: TMA landed, full_a: A written, empty: MMAs done),
+// TMEM ring of 2 accumulators of 256 columns (acc_full: tile's MMAs done, acc_empty: drained).
+// MODE_GU: A rows 0-63 are gate rows f0..f0+63 and rows 64-127 the up rows of the same features
+// (one accumulator holds both); the epilogue pairs quadrant 0 with 2 and 1 with 3 through shared
+// memory and writes h = silu(gate) * up. MODE_DN: A rows are 128 rows of W_down.
+enum { MODE_GU = 0, MODE_DN = 1 };
+
+constexpr int kStages = 4;
+constexpr int kThreadsV2 = 448;
+constexpr int kEpiWarp0 = 10;
+
+struct SmemV2 {
   static constexpr int kB = kBNMax * kBK * 2;   // 32 KB activation tile
   static constexpr int kA = kBM * kBK * 2;      // 16 KB dequantized weight tile
   static constexpr int kRaw = kBM * kBK / 4;    // 2 KB packed codes
-  static constexpr int kStage = kB + NMAT * kA + NMAT * kRaw;
-  static constexpr int kBar = STAGES * kStage;  // barriers after the stages
-  static constexpr int kBytes = kBar + (3 * STAGES + 1) * 8 + 16;
+  static constexpr int kStage = kB + kA + kRaw;
+  static constexpr int kXch = 2 * 16 * 32 * 4;  // gate/up exchange: 2 pairs x 16 columns x 32 lanes
+  static constexpr int kXchOff = kStages * kStage;
+  static constexpr int kBar = kXchOff + kXch;
+  static constexpr int kNumBars = 3 * kStages + 4 + 4;  // + gate/up exchange: full and free per pair
+  static constexpr int kBytes = kBar + kNumBars * 8 + 16;
 };
 
-template <int NMAT, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
-grouped_ffn_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c0r,
-                   const __grid_constant__ CUtensorMap tm_c1r, const __grid_constant__ CUtensorMap tm_c0s,
-                   const __grid_constant__ CUtensorMap tm_c1s, const GemmArgs args) {
-  using SL = Smem<NMAT, STAGES>;
+struct TileInfo {
+  int expert, set, row_base, n_valid, N, mt;
+};
+
+__device__ __forceinline__ TileInfo get_tile(const GemmArgs &a, int ti, int n_mtiles) {
+  TileInfo t;
+  const int entry = ti / n_mtiles;
+  t.mt = ti - entry * n_mtiles;
+  const int2 e = a.tiles[entry];
+  t.set = (e.x == a.shared_group) ? 1 : 0;
+  t.expert = t.set ? 0 : e.x;
+  t.row_base = a.offsets[e.x] + e.y;
+  t.n_valid = min(kBNMax, a.offsets[e.x + 1] - t.row_base);
+  t.N = (t.n_valid + 15) & ~15;
+  return t;
+}
+
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t r[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreadsV2, 1)
+grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c0r,
+                  const __grid_constant__ CUtensorMap tm_c1r, const __grid_constant__ CUtensorMap tm_c0s,
+                  const __grid_constant__ CUtensorMap tm_c1s, const GemmArgs args) {
+  using SL = SmemV2;
   extern __shared__ uint8_t smem_raw[];
   Ctrl *ctrl = args.ctrl;
-  if ((int)blockIdx.x >= ctrl->n_tiles) return;
-  const int2 tl = args.tiles[blockIdx.x];
-  const int grp = tl.x, n0 = tl.y;
-  const int set = (grp == args.shared_group) ? 1 : 0;
-  const int expert = set ? 0 : grp;
-  const int row_base = args.offsets[grp] + n0;
-  const int n_valid = min(kBNMax, args.offsets[grp + 1] - row_base);
-  if (n_valid <= 0) return;
-  const int N = (n_valid + 15) & ~15;
-  const int nbox = (N + kBoxRows - 1) / kBoxRows;
-  const int m0 = blockIdx.y * kBM;
+  const int n_mtiles = (MODE == MODE_GU) ? args.M / 64 : args.M / kBM;
+  const int total = ctrl->n_tiles * n_mtiles;
+  const int G = gridDim.x;
+  const int n_my = (total > (int)blockIdx.x) ? (total - (int)blockIdx.x + G - 1) / G : 0;
+  if (n_my == 0) return;
   const int K = args.K, nk = K / kBK;
 
-  // 1024-byte aligned base (the 128B swizzle pattern is taken from address bits 4..9)
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t *gbase = smem_raw + (base - smem_u32(smem_raw));
   auto sB = [&](int s) { return base + s * SL::kStage; };
-  auto sA = [&](int s, int m) { return base + s * SL::kStage + SL::kB + m * SL::kA; };
-  auto sR = [&](int s, int m) { return base + s * SL::kStage + SL::kB + NMAT * SL::kA + m * SL::kRaw; };
+  auto sA = [&](int s) { return base + s * SL::kStage + SL::kB; };
+  auto sR = [&](int s) { return base + s * SL::kStage + SL::kB + SL::kA; };
   const uint32_t bar0 = base + SL::kBar;
   auto full_b = [&](int s) { return bar0 + 8u * s; };
-  auto full_a = [&](int s) { return bar0 + 8u * (STAGES + s); };
-  auto empty = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
-  const uint32_t accum_full = bar0 + 8u * (3 * STAGES);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + SL::kBar + (3 * STAGES + 1) * 8);
+  auto full_a = [&](int s) { return bar0 + 8u * (kStages + s); };
+  auto empty = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
+  auto acc_full = [&](int b) { return bar0 + 8u * (3 * kStages + b); };
+  auto acc_empty = [&](int b) { return bar0 + 8u * (3 * kStages + 2 + b); };
+  auto x_full = [&](int pr) { return bar0 + 8u * (3 * kStages + 4 + pr); };
+  auto x_free = [&](int pr) { return bar0 + 8u * (3 * kStages + 6 + pr); };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + SL::kBar + SL::kNumBars * 8);
+  float *xch = reinterpret_cast<float *>(gbase + SL::kXchOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(full_b(s), 1);
       mbar_init(full_a(s), kDqThreads);
       mbar_init(empty(s), 1);
     }
-    mbar_init(accum_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full(b), 1);
+      mbar_init(acc_empty(b), 4);
+      mbar_init(x_full(b), 1);
+      mbar_init(x_free(b), 1);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -120,142 +172,211 @@ grouped_ffn_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_consta
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
-      const CUtensorMap *mc0 = set ? &tm_c0s : &tm_c0r;
-      const CUtensorMap *mc1 = set ? &tm_c1s : &tm_c1r;
-      const uint32_t tx = (uint32_t)nbox * kBoxRows * kBK * 2 + NMAT * SL::kRaw;
-      const int wrow = expert * args.M + m0;
-      for (int ks = 0; ks < nk; ++ks) {
-        const int s = ks % STAGES;
-        const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
-        if (!mbar_wait(empty(s), ph ^ 1u)) { record_timeout(ctrl, 1); break; }
-        mbar_arrive_expect_tx(full_b(s), tx);
-        for (int b = 0; b < nbox; ++b)
-          tma_load_2d(sB(s) + b * kBoxRows * kBK * 2, &tm_b, ks * kBK, row_base + b * kBoxRows, full_b(s));
-        tma_load_2d(sR(s, 0), mc0, ks * (kBK / 4), wrow, full_b(s));
-        if (NMAT == 2) tma_load_2d(sR(s, 1), mc1, ks * (kBK / 4), wrow, full_b(s));
+      TileInfo cur = get_tile(args, blockIdx.x, n_mtiles);
+      bool ok = true;
+      for (int tl = 0; tl < n_my && ok; ++tl) {
+        const TileInfo nxt = (tl + 1 < n_my) ? get_tile(args, blockIdx.x + (tl + 1) * G, n_mtiles) : cur;
+        const int nbox = (cur.N + kBoxRows - 1) / kBoxRows;
+        const uint32_t tx = (uint32_t)nbox * kBoxRows * kBK * 2 + SL::kRaw;
+        const CUtensorMap *mc0 = cur.set ? &tm_c0s : &tm_c0r;
+        const CUtensorMap *mc1 = cur.set ? &tm_c1s : &tm_c1r;
+        const int wrow = (MODE == MODE_GU) ? cur.expert * args.M + cur.mt * 64 : cur.expert * args.M + cur.mt * kBM;
+        for (int ks = 0; ks < nk; ++ks) {
+          const int g = tl * nk + ks;
+          const int s = g % kStages;
+          const uint32_t ph = (uint32_t)(g / kStages) & 1u;
+          if (!mbar_wait(empty(s), ph ^ 1u)) { record_timeout(ctrl, 21); ok = false; break; }
+          mbar_arrive_expect_tx(full_b(s), tx);
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d(sB(s) + b * kBoxRows * kBK * 2, &tm_b, ks * kBK, cur.row_base + b * kBoxRows, full_b(s));
+          if (MODE == MODE_GU) {  // gate rows -> A rows 0..63, up rows -> A rows 64..127
+            tma_load_2d(sR(s), mc0, ks * (kBK / 4), wrow, full_b(s));
+            tma_load_2d(sR(s) + 64 * (kBK / 4), mc1, ks * (kBK / 4), wrow, full_b(s));
+          } else {
+            tma_load_2d(sR(s), mc0, ks * (kBK / 4), wrow, full_b(s));
+          }
+        }
+        cur = nxt;
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_f16(N);
+      TileInfo cur = get_tile(args, blockIdx.x, n_mtiles);
       bool ok = true;
-      for (int ks = 0; ks < nk && ok; ++ks) {
-        const int s = ks % STAGES;
-        const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
-        if (!mbar_wait(full_b(s), ph) || !mbar_wait(full_a(s), ph)) { record_timeout(ctrl, 2); ok = false; break; }
+      for (int tl = 0; tl < n_my && ok; ++tl) {
+        const TileInfo nxt = (tl + 1 < n_my) ? get_tile(args, blockIdx.x + (tl + 1) * G, n_mtiles) : cur;
+        const int b = tl & 1;
+        if (!mbar_wait(acc_empty(b), (((uint32_t)tl >> 1) & 1u) ^ 1u)) { record_timeout(ctrl, 22); ok = false; break; }
         tc_fence_after();
+        const uint32_t idesc = idesc_f16(cur.N);
+        const uint32_t d = tmem + (uint32_t)(b * 256);
+        for (int ks = 0; ks < nk; ++ks) {
+          const int g = tl * nk + ks;
+          const int s = g % kStages;
+          const uint32_t ph = (uint32_t)(g / kStages) & 1u;
+          if (!mbar_wait(full_b(s), ph) || !mbar_wait(full_a(s), ph)) { record_timeout(ctrl, 23); ok = false; break; }
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          const uint64_t bd = sw128_desc(sB(s) + kk * 32);
-#pragma unroll
-          for (int m = 0; m < NMAT; ++m)
-            tc_mma(tmem + m * 256, sw128_desc(sA(s, m) + kk * 32), bd, idesc, (ks | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            tc_mma(d, sw128_desc(sA(s) + kk * 32), sw128_desc(sB(s) + kk * 32), idesc, (ks | kk) != 0 ? 1u : 0u);
+          tc_commit(empty(s));
         }
-        tc_commit(empty(s));
+        if (ok) tc_commit(acc_full(b));
+        cur = nxt;
       }
-      if (ok) tc_commit(accum_full);
     }
-  } else {
+  } else if (warp < kEpiWarp0) {
     // ------------------------------------------------ dequant warps
     const int td = threadIdx.x - 64;          // 0..255
-    const int r = td >> 1, blk = td & 1;      // weight row within the tile, 32-weight block of the stage
-    const size_t grow = (size_t)expert * args.M + m0 + r;
-    const uint16_t *scp[NMAT];
-    const uint8_t *hbp[NMAT];
-#pragma unroll
-    for (int m = 0; m < NMAT; ++m) {  // scalar selects keep the parameter block out of local memory
-      const uint16_t *sc = set ? args.scales[1][m] : args.scales[0][m];
-      const uint8_t *hb = set ? args.hibits[1][m] : args.hibits[0][m];
-      scp[m] = sc + grow * (K / 32);
-      hbp[m] = args.q3 ? hb + grow * (K / 8) : nullptr;
-    }
-    // scales (and Q3 hi words) for groups of 4 stages, prefetched one group ahead
-    uint32_t sc_cur[NMAT][4], sc_nxt[NMAT][4], hb_cur[NMAT][4], hb_nxt[NMAT][4];
-    auto load_group = [&](int gi, uint32_t (&sc)[NMAT][4], uint32_t (&hb)[NMAT][4]) {
-#pragma unroll
-      for (int m = 0; m < NMAT; ++m)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int ks = 4 * gi + j;
-          sc[m][j] = (ks < nk) ? (uint32_t)__ldg(scp[m] + 2 * ks + blk) : 0u;
-          hb[m][j] = (args.q3 && ks < nk) ? __ldg(reinterpret_cast<const uint32_t *>(hbp[m]) + 2 * ks + blk) : 0u;
-        }
+    const int r = td >> 1, blk = td & 1;      // A row, 32-weight block of the 64-wide stage
+    const int mat = (MODE == MODE_GU) ? (r >> 6) : 0;
+    const int total_g = n_my * nk;
+    // per-tile pointer to this thread's scales (and hi words); stage ks of the tile reads [2*ks]
+    auto row_ptrs = [&](int tl, const uint16_t *&sp, const uint32_t *&hp) {
+      const int ti = blockIdx.x + tl * G;
+      const int entry = ti / n_mtiles, mt = ti - entry * n_mtiles;
+      const int grp = args.tiles[entry].x;
+      const int set = (grp == args.shared_group) ? 1 : 0;
+      const int expert = set ? 0 : grp;
+      const int wrow = (MODE == MODE_GU) ? mt * 64 + (r & 63) : mt * kBM + r;
+      const size_t grow = (size_t)expert * args.M + wrow;
+      const uint16_t *sc = set ? (mat ? args.scales[1][1] : args.scales[1][0])
+                               : (mat ? args.scales[0][1] : args.scales[0][0]);
+      const uint8_t *hb = set ? (mat ? args.hibits[1][1] : args.hibits[1][0])
+                              : (mat ? args.hibits[0][1] : args.hibits[0][0]);
+      sp = sc + grow * (K / 32) + blk;
+      hp = args.q3 ? reinterpret_cast<const uint32_t *>(hb + grow * (K / 8)) + blk : nullptr;
     };
-    load_group(0, sc_cur, hb_cur);
+    // scales (and Q3 hi words) are fetched 4 stages ahead into a 4-entry register ring
+    int pf_tl = 0;
+    const uint16_t *pf_sp;
+    const uint32_t *pf_hp;
+    row_ptrs(0, pf_sp, pf_hp);
+    uint32_t sc[4], hb[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      sc[j] = 0u;
+      hb[j] = 0u;
+      if (j < total_g) {
+        const int tl = j / nk;
+        if (tl != pf_tl) { pf_tl = tl; row_ptrs(tl, pf_sp, pf_hp); }
+        sc[j] = __ldg(pf_sp + 2 * (j % nk));
+        if (args.q3) hb[j] = __ldg(pf_hp + 2 * (j % nk));
+      }
+    }
     bool ok = true;
-    for (int gi = 0; gi * 4 < nk && ok; ++gi) {
-      if ((gi + 1) * 4 < nk) load_group(gi + 1, sc_nxt, hb_nxt);
+    for (int g0 = 0; g0 < total_g && ok; g0 += 4) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int ks = 4 * gi + j;
-        if (ks >= nk) break;
-        const int s = ks % STAGES;
-        const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
-        if (!mbar_wait(full_b(s), ph)) { record_timeout(ctrl, 3); ok = false; break; }
+        const int g = g0 + j;
+        if (g >= total_g) break;
+        const int s = g % kStages;
+        const uint32_t ph = (uint32_t)(g / kStages) & 1u;
+        if (!mbar_wait(full_b(s), ph)) { record_timeout(ctrl, 24); ok = false; break; }
+        const uint2 cw = *reinterpret_cast<const uint2 *>(gbase + (sR(s) - base) + r * 16 + blk * 8);
+        const __half2 d2 = __half2half2(__ushort_as_half((uint16_t)sc[j]));
+        uint32_t p[16];
+        if (args.q3) {
+          dq3_word(cw.x, hb[j], 0, d2, p);
+          dq3_word(cw.y, hb[j], 1, d2, p + 8);
+        } else {
+          dq2_word(cw.x, d2, p);
+          dq2_word(cw.y, d2, p + 8);
+        }
+        uint8_t *arow = gbase + (sA(s) - base) + r * 128;
 #pragma unroll
-        for (int m = 0; m < NMAT; ++m) {
-          const uint2 cw = *reinterpret_cast<const uint2 *>(gbase + (sR(s, m) - base) + r * 16 + blk * 8);
-          const __half2 d2 = __half2half2(__ushort_as_half((uint16_t)sc_cur[m][j]));
-          uint32_t p[16];
-          if (args.q3) {
-            dq3_word(cw.x, hb_cur[m][j], 0, d2, p);
-            dq3_word(cw.y, hb_cur[m][j], 1, d2, p + 8);
-          } else {
-            dq2_word(cw.x, d2, p);
-            dq2_word(cw.y, d2, p + 8);
-          }
-          uint8_t *arow = gbase + (sA(s, m) - base) + r * 128;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int chunk = 4 * blk + c;
-            *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) =
-                make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
-          }
+        for (int c = 0; c < 4; ++c) {
+          const int chunk = 4 * blk + c;
+          *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) =
+              make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
         }
         fence_async_smem();
         mbar_arrive(full_a(s));
-      }
-      if ((gi + 1) * 4 < nk) {
-#pragma unroll
-        for (int m = 0; m < NMAT; ++m)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            sc_cur[m][j] = sc_nxt[m][j];
-            hb_cur[m][j] = hb_nxt[m][j];
-          }
-      }
-    }
-    // ------------------------------------------------ epilogue (same 8 warps)
-    // the decision is made warp-uniform: tcgen05.ld is a warp-wide instruction
-    bool go = __all_sync(0xffffffffu, ok);
-    if (go) go = __all_sync(0xffffffffu, mbar_wait(accum_full, 0));
-    if (go) {
-      tc_fence_after();
-      const int q = warp & 3, half = (warp - 2) >> 2;
-      const int row = 32 * q + lane;
-      const int f = m0 + row;
-      const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
-      const int c_begin = half * (N / 2), c_end = c_begin + N / 2;
-      for (int c0 = c_begin; c0 < c_end; c0 += 8) {
-        uint32_t a[8], b[8];
-        tmem_ld8(lane_addr + c0, a);
-        if (NMAT == 2) tmem_ld8(lane_addr + 256 + c0, b);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int n = c0 + j;
-          if (n >= n_valid) break;
-          float v = __uint_as_float(a[j]);
-          if (NMAT == 2) {
-            const float u = __uint_as_float(b[j]);
-            v = v / (1.0f + expf(-v)) * u;
-          }
-          args.out[(size_t)(row_base + n) * args.ldo + f] = __half_as_ushort(__float2half_rn(v));
+        // refill this ring slot with the scale of stage g + 4
+        const int gp = g + 4;
+        if (gp < total_g) {
+          const int tl = gp / nk;
+          if (tl != pf_tl) { pf_tl = tl; row_ptrs(tl, pf_sp, pf_hp); }
+          sc[j] = __ldg(pf_sp + 2 * (gp % nk));
+          if (args.q3) hb[j] = __ldg(pf_hp + 2 * (gp % nk));
         }
       }
-    } else if (ok && lane == 0) {
-      record_timeout(ctrl, 4);
+    }
+  } else {
+    // ------------------------------------------------ epilogue warps 10..13 (lane quadrants 2, 3, 0, 1)
+    const int q = warp & 3;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    uint32_t xphase = 0;  // gate/up exchange rounds of this warp's pair
+    bool ok = true;
+    TileInfo cur = get_tile(args, blockIdx.x, n_mtiles);
+    for (int tl = 0; tl < n_my && ok; ++tl) {
+      const TileInfo nxt = (tl + 1 < n_my) ? get_tile(args, blockIdx.x + (tl + 1) * G, n_mtiles) : cur;
+      const int b = tl & 1;
+      const bool go = __all_sync(0xffffffffu, mbar_wait(acc_full(b), ((uint32_t)tl >> 1) & 1u));
+      if (!go) {
+        if (lane == 0) record_timeout(ctrl, 25);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem + lane_base + (uint32_t)(b * 256);
+      if (MODE == MODE_DN) {
+        const int f = cur.mt * kBM + 32 * q + lane;
+        for (int c0 = 0; c0 < cur.N; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(taddr + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = c0 + j;
+            if (n < cur.n_valid)
+              args.out[(size_t)(cur.row_base + n) * args.ldo + f] = __half_as_ushort(__float2half_rn(__uint_as_float(v[j])));
+          }
+        }
+      } else {
+        // gate quadrants 0/1 hand their values to up quadrants 2/3 (pairs 0-2 and 1-3) through a
+        // 16-column shared buffer per pair, handed back and forth with two mbarriers (bounded waits)
+        const int pair = q & 1;
+        float *xb = xch + pair * 16 * 32;
+        const int f = cur.mt * 64 + 32 * pair + lane;
+        for (int c0 = 0; c0 < cur.N && ok; c0 += 16, ++xphase) {
+          uint32_t v[16];
+          tmem_ld16(taddr + c0, v);
+          tmem_ld_wait();
+          if (q < 2) {
+            ok = __all_sync(0xffffffffu, mbar_wait(x_free(pair), (xphase & 1u) ^ 1u));
+            if (!ok) break;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) xb[j * 32 + lane] = __uint_as_float(v[j]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(x_full(pair));
+          } else {
+            ok = __all_sync(0xffffffffu, mbar_wait(x_full(pair), xphase & 1u));
+            if (!ok) break;
+            float gv[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) gv[j] = xb[j * 32 + lane];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(x_free(pair));
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int n = c0 + j;
+              const float uv = __uint_as_float(v[j]);
+              const float hv = gv[j] / (1.0f + expf(-gv[j])) * uv;
+              if (n < cur.n_valid)
+                args.out[(size_t)(cur.row_base + n) * args.ldo + f] = __half_as_ushort(__float2half_rn(hv));
+            }
+          }
+        }
+        if (!ok) {
+          if (lane == 0) record_timeout(ctrl, 26);
+          break;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty(b));
+      cur = nxt;
     }
   }
   tc_fence_before();
@@ -328,20 +449,20 @@ namespace {
 
 namespace {
 
-bool make_code_map(CUtensorMap *map, const moe_qmat &m) {
-  return encode_tensor_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, m.codes, (uint64_t)m.K / 4, (uint64_t)m.n_experts * m.rows,
-                  kBK / 4, kBM, CU_TENSOR_MAP_SWIZZLE_NONE);
+bool make_code_map(CUtensorMap *map, const moe_qmat &m, int box_rows) {
+  return encode_tensor_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, m.codes, (uint64_t)m.K / 4,
+                              (uint64_t)m.n_experts * m.rows, kBK / 4, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-template <int NMAT, int STAGES>
-cudaError_t launch_one(const CUtensorMap &tb, const CUtensorMap &c0r, const CUtensorMap &c1r, const CUtensorMap &c0s,
-                       const CUtensorMap &c1s, const GemmArgs &a, int grid_x, int grid_y, cudaStream_t s) {
-  const int smem = Smem<NMAT, STAGES>::kBytes + 1024;
-  cudaError_t e = smem_limit_once(grouped_ffn_kernel<NMAT, STAGES>, smem);
+template <int MODE>
+cudaError_t launch_v2(const CUtensorMap &tb, const CUtensorMap &c0r, const CUtensorMap &c1r, const CUtensorMap &c0s,
+                      const CUtensorMap &c1s, const GemmArgs &a, cudaStream_t s) {
+  const int smem = SmemV2::kBytes + 1024;
+  cudaError_t e = smem_limit_once(grouped_v2_kernel<MODE>, smem);
   if (e != cudaSuccess) return e;
   {
-    KTimer kt_(NMAT == 2 ? KID_GEMM_GATE_UP : KID_GEMM_DOWN, s);
-    grouped_ffn_kernel<NMAT, STAGES><<<dim3(grid_x, grid_y), kThreads, smem, s>>>(tb, c0r, c1r, c0s, c1s, a);
+    KTimer kt_(MODE == MODE_GU ? KID_GEMM_GATE_UP : KID_GEMM_DOWN, s);
+    grouped_v2_kernel<MODE><<<num_sms(), kThreadsV2, smem, s>>>(tb, c0r, c1r, c0s, c1s, a);
   }
   return cudaGetLastError();
 }
@@ -386,15 +507,15 @@ cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, i
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int max_tiles = n_rows / kBNMax + G + 1;
 
   CUtensorMap tx, th, cg, cu, cd, sg, su, sd;
   bool ok = encode_tensor_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x_perm, H, n_rows, kBK, kBoxRows,
                                  CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_tensor_map_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h_perm, I, n_rows, kBK, kBoxRows,
                                  CU_TENSOR_MAP_SWIZZLE_128B) &&
-            make_code_map(&cg, routed.gate) && make_code_map(&cu, routed.up) && make_code_map(&cd, routed.down) &&
-            make_code_map(&sg, sh.gate) && make_code_map(&su, sh.up) && make_code_map(&sd, sh.down);
+            make_code_map(&cg, routed.gate, 64) && make_code_map(&cu, routed.up, 64) &&
+            make_code_map(&cd, routed.down, kBM) && make_code_map(&sg, sh.gate, 64) && make_code_map(&su, sh.up, 64) &&
+            make_code_map(&sd, sh.down, kBM);
   if (!ok) return cudaErrorInvalidValue;
 
   GemmArgs a{};
@@ -416,7 +537,7 @@ cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, i
   a.hibits[0][1] = routed.up.hibits;
   a.hibits[1][0] = sh.gate.hibits;
   a.hibits[1][1] = sh.up.hibits;
-  e = launch_one<2, 3>(tx, cg, cu, sg, su, a, max_tiles, I / kBM, s);
+  e = launch_v2<MODE_GU>(tx, cg, cu, sg, su, a, s);
   if (e != cudaSuccess) return e;
   // kernel 2: down -> out_perm
   a.out = out_perm;
@@ -431,7 +552,7 @@ cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, i
   a.hibits[0][1] = nullptr;
   a.hibits[1][0] = sh.down.hibits;
   a.hibits[1][1] = nullptr;
-  return launch_one<1, 4>(th, cd, cd, sd, sd, a, max_tiles, H / kBM, s);
+  return launch_v2<MODE_DN>(th, cd, cd, sd, sd, a, s);
 }
 
 }  // namespace moe
