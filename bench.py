@@ -236,12 +236,18 @@ def run_ours(args, world, rank, local):
     pk = peaks()
 
     if T <= 8:
-        # decode: HBM bound; dominant kernel = the gate/up dequant-GEMV
+        # decode: HBM bound. With the fused kernel the whole layer is one launch and its algorithmic
+        # bytes are the distinct active experts + the fp32 router + x + y; with the separate kernels
+        # the dominant one is the gate/up dequant-GEMV.
         gu_b, dn_b = expert_bytes(shape)
         units_avg = units_total / Kt
-        dom = "dec_gate_up"
+        if "decode_fused" in kt:
+            dom = "decode_fused"
+            algo = units_avg * (gu_b + dn_b) + E * H * 4 + T * H * 2 + T * H * 4
+        else:
+            dom = "dec_gate_up"
+            algo = units_avg * gu_b + T * H * 2 + units_avg * T * I * 2
         d_ms, d_n = kt[dom]
-        algo = units_avg * gu_b + T * H * 2 + units_avg * T * I * 2
         achieved = algo / (d_ms / d_n / 1e3) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"], "unit": "GB/s",
                 "frac": round(achieved / pk["hbm"], 4), "traffic": None, "peak_source": pk["src"],

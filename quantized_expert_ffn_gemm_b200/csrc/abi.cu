@@ -34,7 +34,7 @@ cudaEvent_t take_event() {
 const char *const kKernelNames[KID_COUNT] = {
     "router_decode", "router_gemm", "topk", "perm_hist", "perm_scan", "perm_scatter", "perm_fill",
     "perm_gather", "combine", "rmsnorm", "dequant_rows", "dec_units", "dec_gate_up", "dec_down",
-    "tile_list", "gemm_gate_up", "gemm_down", "router_split", "router_tc"};
+    "tile_list", "gemm_gate_up", "gemm_down", "router_split", "router_tc", "decode_fused"};
 }  // namespace
 
 void timer_begin(int kid, cudaStream_t s) {
@@ -297,10 +297,22 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
     DecUnit *units = at<DecUnit>(ws, L.units);
     uint16_t *hdec = at<uint16_t>(ws, L.hdec);
     const int max_units = T * k + hs;
-    e = launch_router_decode(x, T, H, Wr, bias, E, k, idx, w, logits, 1, hs, units, ctrl, s);
-    if (e == cudaSuccess) e = launch_decode_gate_up(x, 1, H, I, *routed, sh, units, max_units, ctrl, hdec, s);
-    if (e == cudaSuccess)
-      e = launch_decode_down(H, I, *routed, sh, units, max_units, ctrl, hdec, y, residual_opt, T, nullptr, s);
+    // auto: one cooperative kernel when the shape fits it; path GEMV (or a shape the fused kernel
+    // does not take): separate router / gate-up / down kernels
+    e = cudaErrorNotSupported;
+    if (path == MOE_PATH_AUTO) {
+      e = launch_decode_fused(x, T, H, Wr, bias, E, k, I, *routed, sh, residual_opt, y, logits, idx, w, hdec, ctrl, s);
+      if (e == cudaErrorCooperativeLaunchTooLarge) {
+        (void)cudaGetLastError();
+        e = cudaErrorNotSupported;
+      }
+    }
+    if (e == cudaErrorNotSupported) {
+      e = launch_router_decode(x, T, H, Wr, bias, E, k, idx, w, logits, 1, hs, units, ctrl, s);
+      if (e == cudaSuccess) e = launch_decode_gate_up(x, 1, H, I, *routed, sh, units, max_units, ctrl, hdec, s);
+      if (e == cudaSuccess)
+        e = launch_decode_down(H, I, *routed, sh, units, max_units, ctrl, hdec, y, residual_opt, T, nullptr, s);
+    }
   } else {
     const int P = T * k, rows = P + (hs ? T : 0);
     int32_t *counts = at<int32_t>(ws, L.counts), *offsets = at<int32_t>(ws, L.offsets);

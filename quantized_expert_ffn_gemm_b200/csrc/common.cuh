@@ -27,7 +27,8 @@ struct Ctrl {
   unsigned gemm_ticket[4];  // tile counters of the persistent grouped GEMM
   int n_units;              // decode: number of (expert, token-set) units built by the router
   int n_tiles;              // prefill: number of (group, row-tile) entries in the tile list
-  int pad1[22];
+  unsigned long long bar_arrivals;  // fused decode: grid barrier arrivals (every launch adds 2 x grid)
+  int pad1[20];
 };
 static_assert(sizeof(Ctrl) == 128, "control area is 128 bytes");
 
@@ -131,6 +132,13 @@ cudaError_t launch_decode_down(int H, int I, const moe_expert_set &routed, const
                                const DecUnit *units, int max_units, Ctrl *ctrl, const uint16_t *hdec, float *y,
                                const float *residual, int T, uint16_t *out_rows, cudaStream_t s);
 
+// fused decode layer (one cooperative kernel: router, top-k, gate/up, down + combine);
+// returns cudaErrorNotSupported when the shape or the device cannot take it (callers fall back)
+cudaError_t launch_decode_fused(const uint16_t *x, int T, int H, const float *Wr, const float *bias, int E, int k,
+                                int I, const moe_expert_set &routed, const moe_expert_set *shared,
+                                const float *residual, float *y, float *logits, int32_t *idx, float *w,
+                                uint16_t *hdec, Ctrl *ctrl, cudaStream_t s);
+
 // prefill path (tcgen05 grouped GEMM)
 int gemm_shape_supported(int H, int I);
 cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, int n_rows, int E, int H, int I,
@@ -151,7 +159,7 @@ cudaError_t smem_limit_once(F *func, size_t bytes) {
 enum KernelId {
   KID_ROUTER_DECODE = 0, KID_ROUTER_GEMM, KID_TOPK, KID_PERM_HIST, KID_PERM_SCAN, KID_PERM_SCATTER, KID_PERM_FILL,
   KID_PERM_GATHER, KID_COMBINE, KID_RMSNORM, KID_DEQUANT_ROWS, KID_DEC_UNITS, KID_DEC_GATE_UP, KID_DEC_DOWN,
-  KID_TILE_LIST, KID_GEMM_GATE_UP, KID_GEMM_DOWN, KID_ROUTER_SPLIT, KID_ROUTER_TC, KID_COUNT
+  KID_TILE_LIST, KID_GEMM_GATE_UP, KID_GEMM_DOWN, KID_ROUTER_SPLIT, KID_ROUTER_TC, KID_DECODE_FUSED, KID_COUNT
 };
 void timer_begin(int kid, cudaStream_t s);
 void timer_end(int kid, cudaStream_t s);

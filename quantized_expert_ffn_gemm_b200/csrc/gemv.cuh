@@ -1,0 +1,200 @@
+// Dequant-GEMV building blocks for 1-8 activation columns (decode / MTP verify): a warp owns 16
+// weight rows; lane (g, t) holds rows g and g+8 and a 64-weight slice of each 256-wide K step
+// (one 16-byte code load per row per step); each 16-weight word is dequantized to fp16 pairs and
+// fed to mma.sync m16n8k16 with the activation columns as the 8 MMA columns (fp32 accumulate).
+// Activations are staged in shared memory as fp16 with a per-64-chunk rotation so the fragment
+// loads of the four K slices hit distinct banks.
+#pragma once
+
+#include "common.cuh"
+#include "dequant.cuh"
+
+namespace moe {
+
+constexpr int kStepK = 256;       // K covered by one warp step (4 lanes x 64 weights)
+
+__device__ __forceinline__ void mma16816(float c[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// shared-memory position of activation element k of a column (row stride added by the caller):
+// 64-element chunk ch keeps its elements rotated by 16*(ch%4)
+__device__ __forceinline__ int xs_pos(int k) {
+  const int ch = k >> 6, q = k & 63;
+  return (ch << 6) + ((q + 16 * (ch & 3)) & 63);
+}
+
+struct MatView {
+  const uint8_t *codes;
+  const uint8_t *hibits;
+  const uint16_t *scales;
+  int K;
+};
+
+// matrix `which` (0 gate, 1 up, 2 down) of expert `expert` in set `set` (0 routed, 1 shared); scalar
+// selects only, so the kernel-parameter structs are never copied to local memory
+__device__ __forceinline__ MatView mat_sel(const moe_expert_set &r, const moe_expert_set &sh, int set, int which,
+                                           int expert) {
+#define MOE_SEL(field)                                                                                  \
+  (which == 0 ? (set ? sh.gate.field : r.gate.field)                                                    \
+              : which == 1 ? (set ? sh.up.field : r.up.field) : (set ? sh.down.field : r.down.field))
+  const uint8_t *codes = MOE_SEL(codes);
+  const uint8_t *hib = MOE_SEL(hibits);
+  const uint16_t *sc = MOE_SEL(scales);
+  const int rows = MOE_SEL(rows), K = MOE_SEL(K);
+#undef MOE_SEL
+  MatView v;
+  const size_t row0 = (size_t)expert * rows;
+  v.codes = codes + row0 * (K / 4);
+  v.hibits = hib ? hib + row0 * (K / 8) : nullptr;
+  v.scales = sc + row0 * (K / 32);
+  v.K = K;
+  return v;
+}
+
+__device__ __forceinline__ MatView mat_of(const moe_qmat &m, int expert) {
+  MatView v;
+  const size_t row0 = (size_t)expert * m.rows;
+  v.codes = m.codes + row0 * (m.K / 4);
+  v.hibits = m.hibits ? m.hibits + row0 * (m.K / 8) : nullptr;
+  v.scales = m.scales + row0 * (m.K / 32);
+  v.K = m.K;
+  return v;
+}
+
+// one lane's share of a 16-row x 256-wide K step: 16 code bytes of rows g and g+8, their two
+// block scales, and (Q3) the two blocks' hi-bit words
+struct StepFrag {
+  uint4 w0, w1;
+  uint32_t d0, d1;
+  uint2 h0, h1;
+};
+
+template <bool Q3>
+__device__ __forceinline__ void load_step(StepFrag &f, const MatView &m, int r0, int step, bool valid) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int k0 = step * kStepK + 64 * t;
+  const bool ok = valid && k0 < m.K;
+  const size_t rs = (size_t)m.K / 4, ss = (size_t)m.K / 32, hs = (size_t)m.K / 8;
+  const size_t ra = (size_t)(r0 + g), rb = (size_t)(r0 + g + 8);
+  f.w0 = ok ? __ldcs(reinterpret_cast<const uint4 *>(m.codes + ra * rs + k0 / 4)) : make_uint4(0, 0, 0, 0);
+  f.w1 = ok ? __ldcs(reinterpret_cast<const uint4 *>(m.codes + rb * rs + k0 / 4)) : make_uint4(0, 0, 0, 0);
+  f.d0 = ok ? __ldcs(reinterpret_cast<const uint32_t *>(m.scales + ra * ss + k0 / 32)) : 0u;
+  f.d1 = ok ? __ldcs(reinterpret_cast<const uint32_t *>(m.scales + rb * ss + k0 / 32)) : 0u;
+  if (Q3) {
+    f.h0 = ok ? __ldcs(reinterpret_cast<const uint2 *>(m.hibits + ra * hs + k0 / 8)) : make_uint2(0, 0);
+    f.h1 = ok ? __ldcs(reinterpret_cast<const uint2 *>(m.hibits + rb * hs + k0 / 8)) : make_uint2(0, 0);
+  }
+}
+
+// dequantize the fragment (zero codes with zero scales give zero weights) and run the step's 16
+// MMAs; B fragments come from the lane's column in shared memory when `bok`, else zero
+template <bool Q3>
+__device__ __forceinline__ void mma_step(float acc[4], float acc2[4], const StepFrag &f, const __half *xcol, int kbase,
+                                         bool bok) {
+  const uint32_t wr0[4] = {f.w0.x, f.w0.y, f.w0.z, f.w0.w};
+  const uint32_t wr1[4] = {f.w1.x, f.w1.y, f.w1.z, f.w1.w};
+#pragma unroll
+  for (int wq = 0; wq < 4; ++wq) {  // word wq: block wq/2, half q = wq%2
+    const int blk = wq >> 1, q = wq & 1;
+    const __half2 dd0 = __half2half2(__ushort_as_half((uint16_t)(f.d0 >> (16 * blk))));
+    const __half2 dd1 = __half2half2(__ushort_as_half((uint16_t)(f.d1 >> (16 * blk))));
+    uint32_t p0[8], p1[8];
+    if (Q3) {
+      dq3_word(wr0[wq], blk ? f.h0.y : f.h0.x, q, dd0, p0);
+      dq3_word(wr1[wq], blk ? f.h1.y : f.h1.x, q, dd1, p1);
+    } else {
+      dq2_word(wr0[wq], dd0, p0);
+      dq2_word(wr1[wq], dd1, p1);
+    }
+#pragma unroll
+    for (int mm = 0; mm < 4; ++mm) {  // MMA 4*wq + mm uses pairs 2mm, 2mm+1 of this word
+      const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
+      uint32_t b0 = 0, b1 = 0;
+      if (bok) {
+        const uint2 bv = *reinterpret_cast<const uint2 *>(xcol + xs_pos(kbase + 16 * wq + 4 * mm));
+        b0 = bv.x;
+        b1 = bv.y;
+      }
+      mma16816((mm & 1) ? acc2 : acc, a, b0, b1);
+    }
+  }
+}
+
+// acc += W[r0..r0+15, steps s0..s0+NS-1] * X^T; all of the batch's loads are issued first
+template <bool Q3, int NS>
+__device__ __forceinline__ void rows16_batch(const MatView &m, int r0, int s0, int nsteps, const __half *xcol,
+                                             bool colok, float acc[4]) {
+  const int t = threadIdx.x & 3;
+  StepFrag f[NS];
+#pragma unroll
+  for (int s = 0; s < NS; ++s) load_step<Q3>(f[s], m, r0, s0 + s, s0 + s < nsteps);
+  float acc2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    const int kbase = (s0 + s) * kStepK + 64 * t;
+    mma_step<Q3>(acc, acc2, f[s], xcol, kbase, colok && (s0 + s < nsteps) && kbase < m.K);
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) acc[e] += acc2[e];
+}
+
+// full K of 16 rows: batches of 8 steps, then a tail batch of 4, 2 or 1
+template <bool Q3>
+__device__ __forceinline__ void rows16(const MatView &m, int r0, const __half *xcol, bool colok, float acc[4]) {
+  const int nsteps = (m.K + kStepK - 1) / kStepK;
+  int s = 0;
+  for (; s + 8 <= nsteps; s += 8) rows16_batch<Q3, 8>(m, r0, s, nsteps, xcol, colok, acc);
+  const int rem = nsteps - s;
+  if (rem > 4) rows16_batch<Q3, 8>(m, r0, s, nsteps, xcol, colok, acc);
+  else if (rem > 2) rows16_batch<Q3, 4>(m, r0, s, nsteps, xcol, colok, acc);
+  else if (rem == 2) rows16_batch<Q3, 2>(m, r0, s, nsteps, xcol, colok, acc);
+  else if (rem == 1) rows16_batch<Q3, 1>(m, r0, s, nsteps, xcol, colok, acc);
+}
+
+// stage columns of the activation source into shared memory (fp16, rotated layout). 16-byte
+// loads, several issued before the first store, so the staging costs one memory round trip.
+template <bool SRC_BF16>
+__device__ __forceinline__ void stage_x(const void *src, int row0, int mask, int H, __half *xs, int xstride) {
+  const int H8 = H / 8;
+  const uint16_t *base = static_cast<const uint16_t *>(src);
+  for (int c = 0; c < 8; ++c) {
+    if (!((mask >> c) & 1)) continue;
+    const uint4 *sp = reinterpret_cast<const uint4 *>(base + (size_t)(row0 + c) * H);
+    for (int i0 = threadIdx.x; i0 < H8; i0 += 4 * blockDim.x) {
+      uint4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = i0 + j * blockDim.x;
+        v[j] = (i < H8) ? __ldg(sp + i) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = i0 + j * blockDim.x;
+        if (i >= H8) break;
+        uint4 o = v[j];
+        if (SRC_BF16) {
+          const uint32_t in[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+          uint32_t out[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            __half2 h = __floats2half2_rn(__uint_as_float(in[q] << 16), __uint_as_float(in[q] & 0xffff0000u));
+            out[q] = *reinterpret_cast<uint32_t *>(&h);
+          }
+          o = make_uint4(out[0], out[1], out[2], out[3]);
+        }
+        // rows are 8-byte aligned (stride H+4 halves): two 8-byte stores
+        uint2 *d = reinterpret_cast<uint2 *>(xs + (size_t)c * xstride + xs_pos(8 * i));
+        d[0] = make_uint2(o.x, o.y);
+        d[1] = make_uint2(o.z, o.w);
+      }
+    }
+  }
+}
+
+
+}  // namespace moe

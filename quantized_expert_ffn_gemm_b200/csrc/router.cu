@@ -11,161 +11,9 @@
 // for the decode expert path, groups the selected (token, slot) pairs by distinct expert.
 // Prefill: a tiled fp32 GEMM for the logits, then one warp per token for the top-k.
 #include "common.cuh"
+#include "topk.cuh"
 
 namespace moe {
-
-// ---------------------------------------------------------------- top-k within one warp
-
-// order-preserving 32-bit key of an fp32 logit (NaN sorts lowest, -0 == +0)
-__device__ __forceinline__ uint32_t logit_key(float f) {
-  if (f != f) return 0u;
-  if (f == 0.0f) f = 0.0f;
-  uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// Top-k of E logits (l[0..E) in shared or global memory) by one warp. Writes idx[0..k) and
-// w[0..k). Rounds of: per-lane best among untaken candidates (ascending index scan, strict >,
-// so the lower index wins a tie inside a lane), warp max of the key, then warp min of the index
-// among lanes holding that key. Lane j keeps the winner of round j, so the k selections end up
-// spread over lanes 0..k-1 and the softmax over the set is one warp reduction.
-__device__ __forceinline__ void topk_finish(float my_val, int my_idx, int k, int32_t *idx, float *w) {
-  const int lane = threadIdx.x & 31;
-  const float l0 = __shfl_sync(0xffffffffu, my_val, 0);
-  const float ev = (lane < k) ? expf(my_val - l0) : 0.0f;
-  const float z = warp_sum(ev);
-  if (lane < k) {
-    idx[lane] = my_idx;
-    w[lane] = ev / z;
-  }
-}
-
-template <int PER_LANE>
-__device__ void warp_topk(const float *l, const float *bias, int E, int k, int32_t *idx, float *w) {
-  const int lane = threadIdx.x & 31;
-  uint32_t key[PER_LANE];
-  float val[PER_LANE];
-#pragma unroll
-  for (int i = 0; i < PER_LANE; ++i) {
-    const int e = lane + 32 * i;
-    const float v = (e < E) ? l[e] + (bias ? bias[e] : 0.0f) : -INFINITY;
-    val[i] = v;
-    key[i] = (e < E) ? logit_key(v) : 0u;
-  }
-  uint32_t taken = 0;
-  float my_val = -INFINITY;
-  int my_idx = 0;
-  for (int j = 0; j < k; ++j) {
-    uint32_t bk = 0;
-    int bi = 0x7fffffff;
-    float bv = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < PER_LANE; ++i) {
-      const int e = lane + 32 * i;
-      const bool ok = (e < E) && !((taken >> i) & 1u);
-      if (ok && (key[i] > bk || bi == 0x7fffffff)) { bk = key[i]; bi = e; bv = val[i]; }
-    }
-    const uint32_t m = __reduce_max_sync(0xffffffffu, bi == 0x7fffffff ? 0u : bk);
-    const uint32_t cand = (bi != 0x7fffffff && bk == m) ? (uint32_t)bi : 0xffffffffu;
-    const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
-    if ((uint32_t)bi == win) taken |= 1u << ((bi - lane) / 32);
-    const float wv = __shfl_sync(0xffffffffu, bv, (int)(win & 31u));
-    if (lane == j) { my_val = wv; my_idx = (int)win; }
-  }
-  topk_finish(my_val, my_idx, k, idx, w);
-}
-
-// generic E (up to kMaxE) from shared memory: lanes rescan their strided candidates each round
-__device__ void warp_topk_generic(const float *l, const float *bias, int E, int k, int32_t *idx, float *w,
-                                  uint32_t *taken_words /* smem, E/32 words, zeroed */) {
-  const int lane = threadIdx.x & 31;
-  float my_val = -INFINITY;
-  int my_idx = 0;
-  for (int j = 0; j < k; ++j) {
-    uint32_t bk = 0;
-    int bi = 0x7fffffff;
-    float bv = -INFINITY;
-    for (int e = lane; e < E; e += 32) {
-      if ((taken_words[e >> 5] >> (e & 31)) & 1u) continue;
-      const float v = l[e] + (bias ? bias[e] : 0.0f);
-      const uint32_t kk = logit_key(v);
-      if (kk > bk || bi == 0x7fffffff) { bk = kk; bi = e; bv = v; }
-    }
-    const uint32_t m = __reduce_max_sync(0xffffffffu, bi == 0x7fffffff ? 0u : bk);
-    const uint32_t cand = (bi != 0x7fffffff && bk == m) ? (uint32_t)bi : 0xffffffffu;
-    const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
-    if ((uint32_t)bi == win) taken_words[bi >> 5] |= 1u << (bi & 31);
-    __syncwarp();
-    const float wv = __shfl_sync(0xffffffffu, bv, (int)(win & 31u));
-    if (lane == j) { my_val = wv; my_idx = (int)win; }
-  }
-  topk_finish(my_val, my_idx, k, idx, w);
-}
-
-// ---------------------------------------------------------------- decode units
-// Group the T*k selected (token, slot) pairs by distinct expert, in order of first appearance
-// (token-major), plus the always-on shared expert as the last unit. One warp, built in shared
-// memory and written out with coalesced stores.
-struct UnitScratch {
-  int first[kDecodeMaxT * kMaxK];
-  int unit[kDecodeMaxT * kMaxK];
-  int expert[kDecodeMaxT * kMaxK + 1];
-  int mask[kDecodeMaxT * kMaxK + 1];
-  float w[kDecodeMaxT * kMaxK + 1][8];
-};
-
-__device__ void build_units(const int32_t *sidx, const float *sw, int T, int k, int has_shared, DecUnit *units,
-                            Ctrl *ctrl, UnitScratch &us) {
-  const int lane = threadIdx.x & 31;
-  const int P = T * k;
-  for (int p = lane; p < P; p += 32) {
-    const int e = sidx[p];
-    int f = p;
-    for (int q = 0; q < p; ++q)
-      if (sidx[q] == e) { f = q; break; }
-    us.first[p] = f;
-  }
-  __syncwarp();
-  int nu = 0;  // leaders numbered in pair order
-  for (int base = 0; base < P; base += 32) {
-    const int p = base + lane;
-    const bool lead = (p < P) && us.first[p] == p;
-    const unsigned bal = __ballot_sync(0xffffffffu, lead);
-    if (lead) us.unit[p] = nu + __popc(bal & ((1u << lane) - 1u));
-    nu += __popc(bal);
-  }
-  const int total = nu + (has_shared ? 1 : 0);
-  for (int u = lane; u < total; u += 32) {
-    us.mask[u] = 0;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) us.w[u][c] = 0.0f;
-  }
-  __syncwarp();
-  for (int p = lane; p < P; p += 32) {  // each (unit, token) is hit once: an expert appears once per token
-    const int u = us.unit[us.first[p]], t = p / k;
-    us.expert[u] = sidx[p];
-    atomicOr(&us.mask[u], 1 << t);
-    us.w[u][t] = sw[p];
-  }
-  __syncwarp();
-  if (has_shared && lane == 0) {
-    us.expert[nu] = 0;
-    us.mask[nu] = (1 << T) - 1;
-    for (int t = 0; t < T; ++t) us.w[nu][t] = 1.0f;
-  }
-  __syncwarp();
-  for (int u = lane; u < total; u += 32) {
-    DecUnit d;
-    d.expert = us.expert[u];
-    d.set = (u == nu) ? 1 : 0;
-    d.mask = us.mask[u];
-    d.xrow0 = 0;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) d.w[c] = us.w[u][c];
-    units[u] = d;
-  }
-  if (lane == 0) ctrl->n_units = total;
-}
 
 // ---------------------------------------------------------------- decode router kernel
 constexpr int kRouterDecWarps = 4;
@@ -278,9 +126,9 @@ router_decode_kernel(const uint16_t *__restrict__ x, int T, int H, const float *
   if (bias) {  // logits output includes the bias
     for (int i = tid; i < T * E; i += blockDim.x) logits[i] = ls[i] + bias[i % E];
   }
-  if (build && warp == 0) {
+  if (build) {  // every thread of this (last) CTA takes part
     __shared__ UnitScratch s_us;
-    build_units(s_idx, s_w, T, k, has_shared, units, ctrl, s_us);
+    build_units(s_idx, s_w, T, k, E, has_shared, units, &ctrl->n_units, s_us);
   }
 }
 
