@@ -40,10 +40,24 @@ WORKLOADS = {
     "decode4": dict(shape="decode4", layers=48),
     "prefill8k": dict(shape="prefill8k", layers=4),
     "prefill2k_q3": dict(shape="prefill2k_q3", layers=4),
+    # the 48-layer stack (RMSNorm before each router, residual stream, prefill-shaped layers with
+    # a uniform router): one step = one token (decode, T=1) or one 8192-token chunk through all 48
+    "stack_decode": dict(shape="stack", T=1, layers=48, stack=True),
+    "stack_prefill": dict(shape="stack", T=8192, layers=48, stack=True),
 }
 METRIC = "MoE-layer tokens/s at T=1/4/8192; % of HBM or bf16 tensor-core roofline"
-DEFAULT_STEPS = {"decode1": 4800, "decode4": 4800, "prefill8k": 40, "prefill2k_q3": 60}
-DEFAULT_WARMUP = {"decode1": 480, "decode4": 480, "prefill8k": 5, "prefill2k_q3": 5}
+DEFAULT_STEPS = {"decode1": 4800, "decode4": 4800, "prefill8k": 40, "prefill2k_q3": 60, "stack_decode": 256,
+                 "stack_prefill": 4}
+DEFAULT_WARMUP = {"decode1": 480, "decode4": 480, "prefill8k": 5, "prefill2k_q3": 5, "stack_decode": 16,
+                  "stack_prefill": 3}
+
+
+def workload_shape(name: str) -> synth.LayerShape:
+    wl = WORKLOADS[name]
+    if wl.get("stack"):
+        st = synth.STACK
+        return synth.LayerShape("stack", wl["T"], st["H"], st["E"], st["k"], st["I"], st["qtype"], st["shared"], None)
+    return synth.WORKLOADS[wl["shape"]]
 
 
 def peaks():
@@ -104,17 +118,20 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- distributed
-def dist_setup():
+def dist_setup(backend: str | None = None):
+    """One process per GPU: rank/world from the torchrun environment. NCCL on GPUs; gloo only
+    where no GPU is present (the CPU tests of the multi-rank host logic)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend is None:
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if backend == "nccl":
+        torch.cuda.set_device(local if world > 1 else 0)
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    elif torch.cuda.is_available():
-        torch.cuda.set_device(0)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
     return world, rank, local
 
 
@@ -125,12 +142,24 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The slowest rank's time: every rank contributes its own device-timed duration."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_throughput(tokens_per_step: int, steps: int, world: int, ms_max: float) -> float:
+    """Tokens processed by all replicas / the slowest replica's time (weak scaling)."""
+    return tokens_per_step * steps * world / (ms_max / 1e3)
+
+
+def replica_x_stream(rank: int, i: int) -> int:
+    """Input stream id of rank `rank`'s i-th token batch: replicas see distinct tokens."""
+    return 1000 * rank + i
 
 
 # ----------------------------------------------------------------------------- workload on device
@@ -158,19 +187,30 @@ def expert_bytes(shape: synth.LayerShape):
 def run_ours(args, world, rank, local):
     import quantized_expert_ffn_gemm_b200 as moe
     wl = WORKLOADS[args.workload]
-    shape = synth.WORKLOADS[wl["shape"]]
+    shape = workload_shape(args.workload)
+    is_stack = bool(wl.get("stack"))
     T, H, E, k, I = shape.T, shape.H, shape.E, shape.k, shape.I
     n_layers = args.layers or wl["layers"]
     dev = torch.device("cuda", torch.cuda.current_device())
     layers = build_layers(shape, n_layers)
-    n_x = 64 if T <= 8 else 2
-    xs = [synth.make_x(shape.seed, T, H, stream=1000 * rank + i).to(dev) for i in range(n_x)]
     ws = moe.Workspace.for_layer(H, E, k, I, shape.shared, T)
-    handles = [moe.LayerHandle(Wr, b, rs, ss, k, ws) for (Wr, b, rs, ss) in layers]
     y = torch.empty(T, H, dtype=torch.float32, device=dev)
+    if is_stack:
+        # independent seeded residual-stream inputs, one per step (tokens do not feed each other)
+        n_x = min(args.steps, 256) if T <= 8 else 2
+        xs = [synth.make_residual(shape.seed, T, H, stream=replica_x_stream(rank, i)).to(dev) for i in range(n_x)]
+        stack = moe.Stack([l[0] for l in layers], None, [l[2] for l in layers],
+                          [l[3] for l in layers] if shape.shared else None, k)
 
-    def step(i, x=None, idx_out=None):
-        handles[i % n_layers].forward(xs[i % n_x] if x is None else x, y, idx_out=idx_out)
+        def step(i, x=None, idx_out=None):
+            moe.stack_forward(xs[i % n_x] if x is None else x, stack, ws, eps=synth.STACK["eps"], r_out=y)
+    else:
+        n_x = 64 if T <= 8 else 2
+        xs = [synth.make_x(shape.seed, T, H, stream=replica_x_stream(rank, i)).to(dev) for i in range(n_x)]
+        handles = [moe.LayerHandle(Wr, b, rs, ss, k, ws) for (Wr, b, rs, ss) in layers]
+
+        def step(i, x=None, idx_out=None):
+            handles[i % n_layers].forward(xs[i % n_x] if x is None else x, y, idx_out=idx_out)
 
     K, W = args.steps, args.warmup
     for i in range(W):
@@ -178,8 +218,12 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     assert moe.read_device_error(ws) == 0
 
-    # ---------------- CUDA graphs: G consecutive steps per graph (one pass over the rotated layers)
-    G = n_layers if T <= 8 else min(n_layers, K)
+    # ---------------- CUDA graphs: G consecutive steps per graph (one pass over the rotated layers;
+    # a stack step already walks all layers, so its graphs hold 16 decode steps or one prefill chunk)
+    if is_stack:
+        G = min(16, K) if T <= 8 else 1
+    else:
+        G = n_layers if T <= 8 else min(n_layers, K)
     graphs = {}
 
     def graph_for(n, first):
@@ -192,7 +236,10 @@ def run_ours(args, world, rank, local):
             graphs[key] = g
         return graphs[key]
 
-    plan = [(G, 0)] * (K // G) + ([(K % G, 0)] if K % G else [])
+    if is_stack and T <= 8:  # every step of the pass its own token
+        plan = [(G, j * G) for j in range(K // G)] + ([(K % G, (K // G) * G)] if K % G else [])
+    else:
+        plan = [(G, 0)] * (K // G) + ([(K % G, 0)] if K % G else [])
     for (n, f) in set(plan):
         graph_for(n, f).replay()
     torch.cuda.synchronize()
@@ -213,13 +260,15 @@ def run_ours(args, world, rank, local):
     ms = e0.elapsed_time(e1)
     clk = clocks.stop()
     ms_max = max_over_ranks(ms, world)
-    value = T * K * world / (ms_max / 1e3)
+    value = whole_job_throughput(T, K, world, ms_max)
     assert moe.read_device_error(ws) == 0
 
     # ---------------- per-kernel device time: blocks of G steps queued behind a sleep kernel so that
     # the event pair around each kernel brackets device execution, not host launch latency
     nblk = max(1, min(10 if T <= 8 else 3, K // G))
-    idx_bufs = [torch.empty(T, k, dtype=torch.int32, device=dev) for _ in range(G)] if T <= 8 else None
+    if is_stack:
+        nblk = 1
+    idx_bufs = [torch.empty(T, k, dtype=torch.int32, device=dev) for _ in range(G)] if (T <= 8 and not is_stack) else None
     units_total = 0
     moe.timing_enable(True)
     for bi in range(nblk):
@@ -229,10 +278,14 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         if idx_bufs is not None:
             units_total += sum(len(torch.unique(t)) + (1 if shape.shared else 0) for t in idx_bufs)
+        elif T == 1:  # one token: its k experts are distinct
+            units_total += G * (k + (1 if shape.shared else 0))
     moe.timing_enable(False)
     kt = moe.timing_read()
     Kt = nblk * G
     launches_per_step = sum(n for (_, n) in kt.values()) / Kt
+    lps = n_layers if is_stack else 1  # layer passes per step
+    Ktl = Kt * lps
     pk = peaks()
 
     if T <= 8:
@@ -253,7 +306,7 @@ def run_ours(args, world, rank, local):
                 "frac": round(achieved / pk["hbm"], 4), "traffic": None, "peak_source": pk["src"],
                 "algorithmic_bytes_per_launch": int(algo), "avg_launch_us": round(d_ms / d_n * 1e3, 3)}
         layer_bytes = units_avg * (gu_b + dn_b) + E * H * 4 + T * H * 2 + T * H * 4
-        layer_gbs = layer_bytes / (ms_max / K / 1e3) / 1e9
+        layer_gbs = layer_bytes / (ms_max / K / lps / 1e3) / 1e9
         roof_layer = {"bound": "hbm", "bytes_per_step": int(layer_bytes), "achieved": round(layer_gbs, 1),
                       "frac": round(layer_gbs / pk["hbm"], 4), "distinct_experts_avg": round(units_avg, 2),
                       "note": "all bytes of a layer step (active experts + fp32 router + x + y) / step time"}
@@ -268,16 +321,18 @@ def run_ours(args, world, rank, local):
                 "peak_source": pk["src"] + " sustained bf16 (fp16 MMA runs at the bf16 rate)",
                 "algorithmic_flops_per_launch": flops, "avg_launch_us": round(d_ms / d_n * 1e3, 1)}
         layer_flops = 2.0 * 3 * rows * H * I + 2.0 * T * E * H
-        tf = layer_flops / (ms_max / K / 1e3) / 1e12
+        tf = layer_flops / (ms_max / K / lps / 1e3) / 1e12
         roof_layer = {"bound": "tensor", "flops_per_step": layer_flops, "achieved": round(tf, 1),
                       "frac": round(tf / pk["tc_sus"], 4)}
 
     # ---------------- end to end through the public API with host buffers (pinned); the
     # host-to-device copy of each step's tokens and the read-back of y are inside the timed region
     Ke = min(K, 2000 if T <= 8 else 20)
+    if is_stack:
+        Ke = min(K, 64 if T <= 8 else 2)
     xh = [x.cpu().pin_memory() for x in xs[:8]]
     yh = torch.empty(T, H, dtype=torch.float32).pin_memory()
-    xd = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    xd = torch.empty(T, H, dtype=xs[0].dtype, device=dev)
     torch.cuda.synchronize()
     barrier(world)
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -290,16 +345,19 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
-    e2e = {"value": round(T * Ke * world / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
+    e2e = {"value": round(whole_job_throughput(T, Ke, world, e2e_ms), 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": T * H * xs[0].element_size(),
            "d2h_bytes_per_step": T * H * 4, "steps": Ke,
-           "note": "one C-ABI call per step from Python (LayerHandle.forward), no graph"}
+           "note": "one C-ABI call per step from Python (%s), no graph" % (
+               "moe_stack_forward" if is_stack else "LayerHandle.forward")}
     del graphs
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(ms_max / K, 6), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16 (MMA operands; fp32 accumulate, router, y; weights Q2/Q3)", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: MoE layer T={T}, H={H}, E={E}, top-{k}, I={I}, "
+        "config": {"workload": f"{args.workload}: {'48-layer stack of MoE layers' if is_stack else 'MoE layer'} "
+                               f"T={T}, H={H}, E={E}, top-{k}, I={I}, "
                                f"{'Q3' if shape.qtype == 3 else 'Q2'}, shared={int(shape.shared)}, "
                                f"router bias={'Zipf(%s)' % shape.zipf_s if shape.zipf_s else 'none'}",
                    "T": T, "layers_rotated": n_layers, "graph_steps": G,
@@ -309,13 +367,16 @@ def run_ours(args, world, rank, local):
                    "parallelism": f"replicas x{world} (token-parallel, no collective)"},
         "roofline": roof, "roofline_layer": roof_layer,
         "kernels_us_per_step": {n: round(ms_ / Kt * 1e3, 3) for n, (ms_, _) in sorted(kt.items())},
+        "ms_per_layer": round(ms_max / K / lps, 6),
         "e2e": e2e, "gpu_launches": int(round(launches_per_step * K)), "clocks": clk,
     }
     return out, shape, layers
 
 
-def cpu_baseline(shape: synth.LayerShape, budget_s: float = 15.0):
-    """The oracle, as it stands, on a bounded sample of the same workload on the host cores."""
+def cpu_baseline(shape: synth.LayerShape, n_layers: int = 1, budget_s: float = 15.0):
+    """The oracle, as it stands, on a bounded sample of the same workload on the host cores. For
+    the 48-layer stack the sample is one layer's worth of tokens and the rate is divided by the
+    layer count (extrapolated: every layer of the stack has the same shape and cost)."""
     import oracle
     L = synth.make_layer(shape)
     nthr = oracle.max_threads()
@@ -327,9 +388,13 @@ def cpu_baseline(shape: synth.LayerShape, budget_s: float = 15.0):
     t0 = time.time()
     oracle.layer_forward(xs, L.Wr, L.bias, shape.k, L.routed, L.shared, nthreads=nthr)
     dt = time.time() - t0
-    return {"value": round(ntok / dt, 3), "unit": "tokens/s", "cores": min(nthr, ntok), "kind": "oracle",
-            "sample": f"{ntok} independent tokens through the {shape.name} layer (layer 0 weights), "
-                      f"fp64 C oracle, one thread per token, {dt:.1f} s"}
+    value = ntok / dt / n_layers
+    sample = (f"{ntok} independent tokens through the {shape.name} layer (layer 0 weights), "
+              f"fp64 C oracle, one thread per token, {dt:.1f} s")
+    if n_layers > 1:
+        sample += f"; tokens/s divided by {n_layers} layers (extrapolated from one layer)"
+    return {"value": round(value, 3), "unit": "tokens/s", "cores": min(nthr, ntok), "kind": "oracle",
+            "sample": sample}
 
 
 def run_reference(args, world, rank):
@@ -338,13 +403,18 @@ def run_reference(args, world, rank):
         return None
     import oracle
     wl = WORKLOADS[args.workload]
-    shape = synth.WORKLOADS[wl["shape"]]
+    shape = workload_shape(args.workload)
+    lps = wl["layers"] if wl.get("stack") else 1
     L = synth.make_layer(shape)
     nthr = oracle.max_threads()
     T = shape.T
-    # one step = the oracle on a bounded sample of the step's tokens (all of them when T <= 8)
+    # one step = the oracle on a bounded sample of the step's tokens (all of them when T <= 8);
+    # for the stack, one layer of it, the rate divided by the layer count (extrapolated)
     sample_T = T if T <= 8 else min(T, 2 * nthr)
-    xs = [synth.make_x(shape.seed, T, shape.H, stream=i)[:sample_T] for i in range(4)]
+    mk = synth.make_residual if wl.get("stack") else synth.make_x
+    xs = [mk(shape.seed, T, shape.H, stream=i)[:sample_T] for i in range(4)]
+    if wl.get("stack"):
+        xs = [oracle.rmsnorm_bf16(r, synth.STACK["eps"]) for r in xs]  # bf16 bits of the first layer's input
     for i in range(max(0, min(args.warmup, 1))):
         oracle.layer_forward(xs[i % 4], L.Wr, L.bias, shape.k, L.routed, L.shared, nthreads=nthr)
     budget = 150.0
@@ -356,14 +426,16 @@ def run_reference(args, world, rank):
         if time.time() - t0 > budget:
             break
     dt = time.time() - t0
-    value = sample_T * done / dt
+    value = sample_T * done / dt / lps
+    note = f"{done} steps x {sample_T} tokens of {shape.name}, fp64 C oracle"
+    if lps > 1:
+        note += f", one layer per step, rate divided by {lps} layers (extrapolated)"
     return {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": done,
-            "warmup": min(args.warmup, 1), "ms_per_step": round(dt / done * 1e3, 3), "higher_is_better": True,
+            "warmup": min(args.warmup, 1), "ms_per_step": round(dt / done * 1e3 * lps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": args.workload, "T": T, "sample_tokens_per_step": sample_T},
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": min(nthr, sample_T),
-                             "kind": "oracle",
-                             "sample": f"{done} steps x {sample_T} tokens of {shape.name}, fp64 C oracle"},
+                             "kind": "oracle", "sample": note},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -397,7 +469,8 @@ def main():
     try:
         out, shape, _ = run_ours(args, world, rank, local)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            out["cpu_baseline"] = cpu_baseline(shape)
+            wl = WORKLOADS[args.workload]
+            out["cpu_baseline"] = cpu_baseline(shape, wl["layers"] if wl.get("stack") else 1)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

@@ -160,8 +160,8 @@ moe_status moe_permute(const int32_t *idx, int32_t T, int32_t k, int32_t E, cons
  * Groups 0..E-1 use `routed`; with shared_opt != NULL, group E (rows offsets[E]..offsets[E+1])
  * uses the shared expert. offsets (device) has E+1 (+1) monotone entries with
  * offsets[last] <= n_rows. path: MOE_PATH_GEMM = tcgen05 grouped GEMM (needs H % 128 == 0
- * and I % 128 == 0), MOE_PATH_GEMV = dequant-GEMV, MOE_PATH_AUTO picks GEMM for n_rows > 4*...
- * (GEMV when n_rows <= 4*k+1 or the GEMM shape rule fails).
+ * and I % 128 == 0), MOE_PATH_GEMV = dequant-GEMV, MOE_PATH_AUTO picks the GEMM when
+ * n_rows > 64 and the GEMM shape rule holds, the GEMV otherwise.
  * x_perm fp16 [n_rows,H]; out_perm fp16 [n_rows,H]. */
 moe_status moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, int32_t n_rows, int32_t E, int32_t H,
                           int32_t I, const moe_expert_set *routed, const moe_expert_set *shared_opt,
