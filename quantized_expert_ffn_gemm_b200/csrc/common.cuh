@@ -15,7 +15,7 @@ namespace moe {
 constexpr int kMaxK = 32;          // routing slots per token
 constexpr int kMaxE = 4096;        // experts per layer
 constexpr int kDecodeMaxT = 8;     // tokens the decode (GEMV) path takes at once (MMA N = 8)
-constexpr int kPermChunk = 256;    // (token, slot) pairs per permute CTA
+constexpr int kPermChunk = 1024;   // (token, slot) pairs per permute chunk (one CTA / one warp)
 
 // ---------------------------------------------------------------- control area (workspace head)
 // Everything here is left at zero by the kernels that use it (tickets are reset by the last CTA).
@@ -133,11 +133,13 @@ cudaError_t launch_decode_down(int H, int I, const moe_expert_set &routed, const
                                const float *residual, int T, uint16_t *out_rows, cudaStream_t s);
 
 // fused decode layer (one cooperative kernel: router, top-k, gate/up, down + combine);
-// returns cudaErrorNotSupported when the shape or the device cannot take it (callers fall back)
-cudaError_t launch_decode_fused(const uint16_t *x, int T, int H, const float *Wr, const float *bias, int E, int k,
-                                int I, const moe_expert_set &routed, const moe_expert_set *shared,
-                                const float *residual, float *y, float *logits, int32_t *idx, float *w,
-                                uint16_t *hdec, Ctrl *ctrl, cudaStream_t s);
+// returns cudaErrorNotSupported when the shape or the device cannot take it (callers fall back).
+// With r_norm != NULL the tokens are x = bf16(RMSNorm_eps(r_norm)) (x unused), bit-identical to
+// launch_rmsnorm followed by the layer.
+cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float eps, int T, int H, const float *Wr,
+                                const float *bias, int E, int k, int I, const moe_expert_set &routed,
+                                const moe_expert_set *shared, const float *residual, float *y, float *logits,
+                                int32_t *idx, float *w, uint16_t *hdec, Ctrl *ctrl, cudaStream_t s);
 
 // prefill path (tcgen05 grouped GEMM)
 int gemm_shape_supported(int H, int I);

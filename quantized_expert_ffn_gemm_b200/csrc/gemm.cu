@@ -9,10 +9,13 @@
 //   TMA      activation rows (fp16, 128B-swizzled K-major) and the packed 2-bit code plane of
 //            the 128 weight rows -> shared memory, one mbarrier per pipeline stage
 //   dequant  8 warps turn codes (+ per-block fp16 scales, + the Q3 hi-bit plane) into fp16
-//            weights written straight into the UMMA canonical 128B-swizzled K-major layout
+//            weights and store them straight into tensor memory (tcgen05.st), one weight row per
+//            TMEM lane: the A operand never touches shared memory, which leaves the shared-memory
+//            bandwidth to the activation tiles (TMA writes and MMA reads)
 //   MMA      one thread issues tcgen05.mma kind::f16 (fp16 x fp16 -> fp32) with the weights as
-//            A (M = 128) and the tokens as B (N = token rows of the tile, multiple of 16), so a
-//            group of ~160 rows is one N = 160 tile (swap-AB); accumulators live in TMEM
+//            A (M = 128, from TMEM) and the tokens as B (N = token rows of the tile, multiple of
+//            16, <= 192), so a group of ~160 rows is one N = 160 tile (swap-AB); accumulators
+//            live in TMEM too
 //   epilogue tcgen05.ld -> registers; gate/up: h = silu(g) * u (both accumulators in TMEM),
 //            down: the expert output row; stored as fp16
 //
@@ -31,7 +34,7 @@ namespace moe {
 
 constexpr int kBK = 64;            // K per pipeline stage (one 128-byte swizzle row of fp16)
 constexpr int kBM = 128;           // weight rows per tile (MMA M)
-constexpr int kBNMax = 256;        // token rows per tile (MMA N upper bound)
+constexpr int kBNMax = 192;        // token rows per tile (MMA N upper bound; TMEM: 2 x 192 + A ring)
 constexpr int kBoxRows = 32;       // rows per TMA box of the activation tile
 constexpr int kThreads = 320;      // warp 0 TMA, warp 1 MMA/TMEM, warps 2..9 dequant + epilogue
 constexpr int kDqThreads = 256;
@@ -60,28 +63,38 @@ __device__ __forceinline__ void record_timeout(Ctrl *c, int where) { set_device_
 //   warp 1      TMEM owner and single-thread MMA issuer
 //   warps 2-9   dequant: code plane + per-block scales (+ Q3 hi bits) -> fp16 A tile
 //   warps 10-13 epilogue: TMEM -> registers -> global, one lane quadrant each
-// Shared-memory ring of kStages stages (full_b: TMA landed, full_a: A written, empty: MMAs done),
-// TMEM ring of 2 accumulators of 256 columns (acc_full: tile's MMAs done, acc_empty: drained).
+// Two rings. Shared memory: kStagesB stages of activation tile + code plane (full_b: TMA landed,
+// empty_b: the stage's MMAs are done). TMEM: kStagesA stages of the dequantized A tile, 128
+// lanes x 32 columns (full_a: written by the dequant warps, empty_a: the stage's MMAs are done).
+// TMEM (512 columns): accumulators at columns 0 and 256 (up to 192 columns each; acc_full:
+// tile's MMAs done, acc_empty: drained), A stages at 192, 224, 448 and 480. The deeper
+// shared-memory ring lets the TMA run far enough ahead to cover HBM latency.
 // MODE_GU: A rows 0-63 are gate rows f0..f0+63 and rows 64-127 the up rows of the same features
 // (one accumulator holds both); the epilogue pairs quadrant 0 with 2 and 1 with 3 through shared
 // memory and writes h = silu(gate) * up. MODE_DN: A rows are 128 rows of W_down.
 enum { MODE_GU = 0, MODE_DN = 1 };
 
-constexpr int kStages = 4;
+constexpr int kStagesB = 8;
+constexpr int kStagesA = 4;
 constexpr int kThreadsV2 = 448;
 constexpr int kEpiWarp0 = 10;
 
 struct SmemV2 {
-  static constexpr int kB = kBNMax * kBK * 2;   // 32 KB activation tile
-  static constexpr int kA = kBM * kBK * 2;      // 16 KB dequantized weight tile
+  static constexpr int kB = kBNMax * kBK * 2;   // 24 KB activation tile
   static constexpr int kRaw = kBM * kBK / 4;    // 2 KB packed codes
-  static constexpr int kStage = kB + kA + kRaw;
+  static constexpr int kStage = kB + kRaw;      // multiple of 1024 (128B-swizzle atoms)
   static constexpr int kXch = 2 * 16 * 32 * 4;  // gate/up exchange: 2 pairs x 16 columns x 32 lanes
-  static constexpr int kXchOff = kStages * kStage;
+  static constexpr int kXchOff = kStagesB * kStage;
   static constexpr int kBar = kXchOff + kXch;
-  static constexpr int kNumBars = 3 * kStages + 4 + 4;  // + gate/up exchange: full and free per pair
+  static constexpr int kNumBars = 2 * kStagesB + 2 * kStagesA + 4 + 4;  // + gate/up exchange: full and free per pair
   static constexpr int kBytes = kBar + kNumBars * 8 + 16;
 };
+
+static_assert(SmemV2::kStage % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+static_assert(kStagesA == 4, "TMEM holds four A stages");
+
+// TMEM column of A stage s
+__device__ __forceinline__ uint32_t a_col(int s) { return 192u + 32u * (uint32_t)(s & 1) + 256u * (uint32_t)(s >> 1); }
 
 struct TileInfo {
   int expert, set, row_base, n_valid, N, mt;
@@ -131,25 +144,29 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t *gbase = smem_raw + (base - smem_u32(smem_raw));
   auto sB = [&](int s) { return base + s * SL::kStage; };
-  auto sA = [&](int s) { return base + s * SL::kStage + SL::kB; };
-  auto sR = [&](int s) { return base + s * SL::kStage + SL::kB + SL::kA; };
+  auto sR = [&](int s) { return base + s * SL::kStage + SL::kB; };
   const uint32_t bar0 = base + SL::kBar;
   auto full_b = [&](int s) { return bar0 + 8u * s; };
-  auto full_a = [&](int s) { return bar0 + 8u * (kStages + s); };
-  auto empty = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
-  auto acc_full = [&](int b) { return bar0 + 8u * (3 * kStages + b); };
-  auto acc_empty = [&](int b) { return bar0 + 8u * (3 * kStages + 2 + b); };
-  auto x_full = [&](int pr) { return bar0 + 8u * (3 * kStages + 4 + pr); };
-  auto x_free = [&](int pr) { return bar0 + 8u * (3 * kStages + 6 + pr); };
+  auto empty_b = [&](int s) { return bar0 + 8u * (kStagesB + s); };
+  auto full_a = [&](int s) { return bar0 + 8u * (2 * kStagesB + s); };
+  auto empty_a = [&](int s) { return bar0 + 8u * (2 * kStagesB + kStagesA + s); };
+  constexpr int kB0 = 2 * kStagesB + 2 * kStagesA;
+  auto acc_full = [&](int b) { return bar0 + 8u * (kB0 + b); };
+  auto acc_empty = [&](int b) { return bar0 + 8u * (kB0 + 2 + b); };
+  auto x_full = [&](int pr) { return bar0 + 8u * (kB0 + 4 + pr); };
+  auto x_free = [&](int pr) { return bar0 + 8u * (kB0 + 6 + pr); };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + SL::kBar + SL::kNumBars * 8);
   float *xch = reinterpret_cast<float *>(gbase + SL::kXchOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStagesB; ++s) {
       mbar_init(full_b(s), 1);
-      mbar_init(full_a(s), kDqThreads);
-      mbar_init(empty(s), 1);
+      mbar_init(empty_b(s), 1);
+    }
+    for (int s = 0; s < kStagesA; ++s) {
+      mbar_init(full_a(s), 128);  // the four dequant warps of the stage's parity
+      mbar_init(empty_a(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(acc_full(b), 1);
@@ -183,9 +200,9 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
         const int wrow = (MODE == MODE_GU) ? cur.expert * args.M + cur.mt * 64 : cur.expert * args.M + cur.mt * kBM;
         for (int ks = 0; ks < nk; ++ks) {
           const int g = tl * nk + ks;
-          const int s = g % kStages;
-          const uint32_t ph = (uint32_t)(g / kStages) & 1u;
-          if (!mbar_wait(empty(s), ph ^ 1u)) { record_timeout(ctrl, 21); ok = false; break; }
+          const int s = g % kStagesB;
+          const uint32_t ph = (uint32_t)(g / kStagesB) & 1u;
+          if (!mbar_wait(empty_b(s), ph ^ 1u)) { record_timeout(ctrl, 21); ok = false; break; }
           mbar_arrive_expect_tx(full_b(s), tx);
           for (int b = 0; b < nbox; ++b)
             tma_load_2d(sB(s) + b * kBoxRows * kBK * 2, &tm_b, ks * kBK, cur.row_base + b * kBoxRows, full_b(s));
@@ -213,14 +230,15 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
         const uint32_t d = tmem + (uint32_t)(b * 256);
         for (int ks = 0; ks < nk; ++ks) {
           const int g = tl * nk + ks;
-          const int s = g % kStages;
-          const uint32_t ph = (uint32_t)(g / kStages) & 1u;
-          if (!mbar_wait(full_b(s), ph) || !mbar_wait(full_a(s), ph)) { record_timeout(ctrl, 23); ok = false; break; }
+          const int s = g % kStagesB, sa = g % kStagesA;
+          const uint32_t ph = (uint32_t)(g / kStagesB) & 1u, pha = (uint32_t)(g / kStagesA) & 1u;
+          if (!mbar_wait(full_b(s), ph) || !mbar_wait(full_a(sa), pha)) { record_timeout(ctrl, 23); ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            tc_mma(d, sw128_desc(sA(s) + kk * 32), sw128_desc(sB(s) + kk * 32), idesc, (ks | kk) != 0 ? 1u : 0u);
-          tc_commit(empty(s));
+            tc_mma_ts(d, tmem + a_col(sa) + 8u * kk, sw128_desc(sB(s) + kk * 32), idesc, (ks | kk) != 0 ? 1u : 0u);
+          tc_commit(empty_b(s));
+          tc_commit(empty_a(sa));
         }
         if (ok) tc_commit(acc_full(b));
         cur = nxt;
@@ -228,12 +246,16 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
     }
   } else if (warp < kEpiWarp0) {
     // ------------------------------------------------ dequant warps
-    const int td = threadIdx.x - 64;          // 0..255
-    const int r = td >> 1, blk = td & 1;      // A row, 32-weight block of the 64-wide stage
+    // warp w writes TMEM lanes 32*(w%4)..+31 (the lanes a warp may access): A row r = that lane.
+    // Warps 2-5 dequantize the even stages and warps 6-9 the odd ones, a thread a whole 64-weight
+    // row slice (both 32-weight blocks) of its stage, so two stages are in flight at once.
+    const int qd = warp & 3;
+    const int r = 32 * qd + lane, par = (warp - 2) >> 2;
+    const uint32_t a_lane = (uint32_t)(32 * qd) << 16;
     const int mat = (MODE == MODE_GU) ? (r >> 6) : 0;
     const int total_g = n_my * nk;
-    // per-tile pointer to this thread's scales (and hi words); stage ks of the tile reads [2*ks]
-    auto row_ptrs = [&](int tl, const uint16_t *&sp, const uint32_t *&hp) {
+    // per-tile pointers to this row's scales (two per stage: one u32) and Q3 hi words (two per stage)
+    auto row_ptrs = [&](int tl, const uint32_t *&sp, const uint2 *&hp) {
       const int ti = blockIdx.x + tl * G;
       const int entry = ti / n_mtiles, mt = ti - entry * n_mtiles;
       const int grp = args.tiles[entry].x;
@@ -245,62 +267,63 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
                                : (mat ? args.scales[0][1] : args.scales[0][0]);
       const uint8_t *hb = set ? (mat ? args.hibits[1][1] : args.hibits[1][0])
                               : (mat ? args.hibits[0][1] : args.hibits[0][0]);
-      sp = sc + grow * (K / 32) + blk;
-      hp = args.q3 ? reinterpret_cast<const uint32_t *>(hb + grow * (K / 8)) + blk : nullptr;
+      sp = reinterpret_cast<const uint32_t *>(sc + grow * (K / 32));
+      hp = args.q3 ? reinterpret_cast<const uint2 *>(hb + grow * (K / 8)) : nullptr;
     };
-    // scales (and Q3 hi words) are fetched 4 stages ahead into a 4-entry register ring
+    // scales (and Q3 hi words) are fetched four of this warp's stages (eight stages) ahead into a
+    // 4-entry register ring
     int pf_tl = 0;
-    const uint16_t *pf_sp;
-    const uint32_t *pf_hp;
+    const uint32_t *pf_sp;
+    const uint2 *pf_hp;
     row_ptrs(0, pf_sp, pf_hp);
-    uint32_t sc[4], hb[4];
+    auto fetch = [&](int g, uint32_t &scv, uint2 &hv) {
+      const int tl = g / nk;
+      if (tl != pf_tl) { pf_tl = tl; row_ptrs(tl, pf_sp, pf_hp); }
+      scv = __ldg(pf_sp + g % nk);
+      if (args.q3) hv = __ldg(pf_hp + g % nk);
+    };
+    uint32_t sc[4];
+    uint2 hw[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       sc[j] = 0u;
-      hb[j] = 0u;
-      if (j < total_g) {
-        const int tl = j / nk;
-        if (tl != pf_tl) { pf_tl = tl; row_ptrs(tl, pf_sp, pf_hp); }
-        sc[j] = __ldg(pf_sp + 2 * (j % nk));
-        if (args.q3) hb[j] = __ldg(pf_hp + 2 * (j % nk));
-      }
+      hw[j] = make_uint2(0u, 0u);
+      const int g = par + 2 * j;
+      if (g < total_g) fetch(g, sc[j], hw[j]);
     }
     bool ok = true;
-    for (int g0 = 0; g0 < total_g && ok; g0 += 4) {
+    for (int i0 = 0; par + 2 * i0 < total_g && ok; i0 += 4) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int g = g0 + j;
+        const int g = par + 2 * (i0 + j);
         if (g >= total_g) break;
-        const int s = g % kStages;
-        const uint32_t ph = (uint32_t)(g / kStages) & 1u;
-        if (!mbar_wait(full_b(s), ph)) { record_timeout(ctrl, 24); ok = false; break; }
-        const uint2 cw = *reinterpret_cast<const uint2 *>(gbase + (sR(s) - base) + r * 16 + blk * 8);
-        const __half2 d2 = __half2half2(__ushort_as_half((uint16_t)sc[j]));
-        uint32_t p[16];
+        const int s = g % kStagesB, sa = g % kStagesA;
+        const uint32_t ph = (uint32_t)(g / kStagesB) & 1u, pha = (uint32_t)(g / kStagesA) & 1u;
+        // codes landed; the MMAs that read this A stage last time are complete
+        if (!mbar_wait(full_b(s), ph) || !mbar_wait(empty_a(sa), pha ^ 1u)) { record_timeout(ctrl, 24); ok = false; break; }
+        tc_fence_after();
+        const uint4 cw = *reinterpret_cast<const uint4 *>(gbase + (sR(s) - base) + r * 16);
+        const __half2 d0 = __half2half2(__ushort_as_half((uint16_t)(sc[j] & 0xffffu)));
+        const __half2 d1 = __half2half2(__ushort_as_half((uint16_t)(sc[j] >> 16)));
+        uint32_t p[32];
         if (args.q3) {
-          dq3_word(cw.x, hb[j], 0, d2, p);
-          dq3_word(cw.y, hb[j], 1, d2, p + 8);
+          dq3_word(cw.x, hw[j].x, 0, d0, p);
+          dq3_word(cw.y, hw[j].x, 1, d0, p + 8);
+          dq3_word(cw.z, hw[j].y, 0, d1, p + 16);
+          dq3_word(cw.w, hw[j].y, 1, d1, p + 24);
         } else {
-          dq2_word(cw.x, d2, p);
-          dq2_word(cw.y, d2, p + 8);
+          dq2_word(cw.x, d0, p);
+          dq2_word(cw.y, d0, p + 8);
+          dq2_word(cw.z, d1, p + 16);
+          dq2_word(cw.w, d1, p + 24);
         }
-        uint8_t *arow = gbase + (sA(s) - base) + r * 128;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int chunk = 4 * blk + c;
-          *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) =
-              make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
-        }
-        fence_async_smem();
-        mbar_arrive(full_a(s));
-        // refill this ring slot with the scale of stage g + 4
-        const int gp = g + 4;
-        if (gp < total_g) {
-          const int tl = gp / nk;
-          if (tl != pf_tl) { pf_tl = tl; row_ptrs(tl, pf_sp, pf_hp); }
-          sc[j] = __ldg(pf_sp + 2 * (gp % nk));
-          if (args.q3) hb[j] = __ldg(pf_hp + 2 * (gp % nk));
-        }
+        tmem_st16(tmem + a_lane + a_col(sa), p);
+        tmem_st16(tmem + a_lane + a_col(sa) + 16u, p + 16);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(full_a(sa));
+        const int gp = g + 8;  // refill this ring slot
+        if (gp < total_g) fetch(gp, sc[j], hw[j]);
       }
     }
   } else {

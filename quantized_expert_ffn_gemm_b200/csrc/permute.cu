@@ -4,9 +4,10 @@
 // expert's rows form one GEMM operand (the more tokens an expert collects in a prefill chunk,
 // the more its weights are reused: "Two-Day Port, 8x Faster Prefill: Strata Engine
 // Benchmarked", "Where Strata Is Fast: Not Magic, but Logistics", MoE paragraph). It is a
-// stable counting sort: per-chunk histograms, one exclusive scan over (expert, chunk), then a
-// stable scatter in which one warp walks its chunk in order and ranks equal experts with
-// __match_any_sync, so the rows of an expert come out in token order, deterministically.
+// stable counting sort: per-chunk histograms (stored expert-major, hist[e][chunk]), one
+// exclusive scan over (expert, chunk), then a stable scatter in which one warp walks its chunk
+// in order and ranks equal experts with __match_any_sync, so the rows of an expert come out in
+// token order, deterministically.
 #include "common.cuh"
 #include "dequant.cuh"
 
@@ -26,40 +27,50 @@ perm_hist_kernel(const int32_t *__restrict__ idx, int P, int E, int32_t *__restr
     else set_device_error(ctrl, MOE_ERR_DEVICE_CHECK, e);
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(size_t)c * E + e] = sh[e];
+  const int nchunks = gridDim.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(size_t)e * nchunks + c] = sh[e];
 }
 
 // ---------------------------------------------------------------- scan (one CTA)
-// counts[e] = sum_c hist[c][e]; offsets = exclusive scan; hist[c][e] <- first row of chunk c in e
+// counts[e] = sum_c hist[e][c]; offsets = exclusive scan over e; hist[e][c] <- first row of
+// chunk c in expert e. One warp per expert at a time: its lanes read the expert's chunk counts
+// (contiguous) and scan them with shuffles, so the loads of all warps are in flight together.
 __global__ void __launch_bounds__(1024)
 perm_scan_kernel(int32_t *__restrict__ hist, int nchunks, int E, int P, int T, int with_shared,
                  int32_t *__restrict__ counts, int32_t *__restrict__ offsets) {
+  extern __shared__ int32_t s_cnt[];  // [E] totals, then exclusive offsets
   __shared__ int32_t s_warp[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = (E + 1023) / 1024;  // experts per thread (contiguous)
-  int local[4];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  // pass 1: per-expert totals
+  for (int e = warp; e < E; e += nw) {
+    const int32_t *h = hist + (size_t)e * nchunks;
+    int s = 0;
+    for (int c = lane; c < nchunks; c += 32) s += h[c];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) s_cnt[e] = s;
+  }
+  __syncthreads();
+  // exclusive scan of the E totals (contiguous runs per thread, then a block scan of the runs)
+  const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;
   int mysum = 0;
   for (int i = 0; i < per; ++i) {
-    int e = tid * per + i, s = 0;
-    if (e < E)
-      for (int c = 0; c < nchunks; ++c) s += hist[(size_t)c * E + e];
-    local[i] = s;
-    mysum += s;
+    const int e = tid * per + i;
+    if (e < E) mysum += s_cnt[e];
   }
-  // block exclusive scan of mysum
   int v = mysum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    int n = __shfl_up_sync(0xffffffffu, v, o);
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
     if (lane >= o) v += n;
   }
   if (lane == 31) s_warp[warp] = v;
   __syncthreads();
   if (warp == 0) {
-    int wv = s_warp[lane];
+    int wv = (lane < nw) ? s_warp[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      int n = __shfl_up_sync(0xffffffffu, wv, o);
+      const int n = __shfl_up_sync(0xffffffffu, wv, o);
       if (lane >= o) wv += n;
     }
     s_warp[lane] = wv;
@@ -67,18 +78,32 @@ perm_scan_kernel(int32_t *__restrict__ hist, int nchunks, int E, int P, int T, i
   __syncthreads();
   int base = v - mysum + (warp > 0 ? s_warp[warp - 1] : 0);
   for (int i = 0; i < per; ++i) {
-    int e = tid * per + i;
+    const int e = tid * per + i;
     if (e < E) {
-      counts[e] = local[i];
+      const int c = s_cnt[e];
+      counts[e] = c;
       offsets[e] = base;
-      int run = base;
-      for (int c = 0; c < nchunks; ++c) {
-        int h = hist[(size_t)c * E + e];
-        hist[(size_t)c * E + e] = run;
-        run += h;
-      }
+      s_cnt[e] = base;  // this thread alone reads and rewrites entry e
+      base += c;
     }
-    base += local[i];
+  }
+  __syncthreads();
+  // pass 2: first row of every (expert, chunk): the expert's offset + the exclusive prefix over chunks
+  for (int e = warp; e < E; e += nw) {
+    int32_t *h = hist + (size_t)e * nchunks;
+    int run = s_cnt[e];
+    for (int c0 = 0; c0 < nchunks; c0 += 32) {
+      const int c = c0 + lane;
+      const int x = (c < nchunks) ? h[c] : 0;
+      int incl = x;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      if (c < nchunks) h[c] = run + incl - x;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
   }
   if (tid == 0) {
     offsets[E] = P;
@@ -94,8 +119,8 @@ __global__ void __launch_bounds__(32)
 perm_scatter_kernel(const int32_t *__restrict__ idx, int P, int k, int E, const int32_t *__restrict__ hist,
                     int32_t *__restrict__ row_of, int32_t *__restrict__ src) {
   extern __shared__ int32_t cursor[];
-  const int c = blockIdx.x, lane = threadIdx.x;
-  for (int e = lane; e < E; e += 32) cursor[e] = hist[(size_t)c * E + e];
+  const int c = blockIdx.x, lane = threadIdx.x, nchunks = gridDim.x;
+  for (int e = lane; e < E; e += 32) cursor[e] = hist[(size_t)e * nchunks + c];
   __syncwarp();
   const int p0 = c * kPermChunk, p1 = min(P, p0 + kPermChunk);
   for (int pb = p0; pb < p1; pb += 32) {
@@ -156,7 +181,7 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const uint16
   }
   {
     KTimer kt_(KID_PERM_SCAN, s);
-    perm_scan_kernel<<<1, 1024, 0, s>>>(hist, nchunks, E, P, T, with_shared, counts, offsets);
+    perm_scan_kernel<<<1, 1024, esm, s>>>(hist, nchunks, E, P, T, with_shared, counts, offsets);
   }
   {
     KTimer kt_(KID_PERM_SCATTER, s);
