@@ -301,7 +301,8 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
     // does not take): separate router / gate-up / down kernels
     e = cudaErrorNotSupported;
     if (path == MOE_PATH_AUTO) {
-      e = launch_decode_fused(x, T, H, Wr, bias, E, k, I, *routed, sh, residual_opt, y, logits, idx, w, hdec, ctrl, s);
+      e = launch_decode_fused(x, nullptr, 0.0f, T, H, Wr, bias, E, k, I, *routed, sh, residual_opt, y, logits, idx, w,
+                              hdec, ctrl, s);
       if (e == cudaErrorCooperativeLaunchTooLarge) {
         (void)cudaGetLastError();
         e = cudaErrorNotSupported;
@@ -376,8 +377,20 @@ moe_status moe_stack_forward(const float *r_in, int32_t T, int32_t L, const floa
   }
   uint16_t *u = at<uint16_t>(ws, LY.u16);
   cudaStream_t s = (cudaStream_t)stream;
+  // decode-sized batches: RMSNorm runs inside the fused layer kernel (one launch per layer)
+  const bool fused = path == MOE_PATH_AUTO && T <= 4 && decode_router_fits(T, H, E);
   for (int l = 0; l < L; ++l) {
     const float *r = (l == 0) ? r_in : r_out;
+    const float *b = bias ? bias[l] : nullptr;
+    if (!aligned16(Wr[l]) || (b && !aligned16(b))) return MOE_ERR_ALIGNMENT;
+    if (fused) {
+      cudaError_t e = launch_decode_fused(nullptr, r, eps, T, H, Wr[l], b, E, k, I, routed[l], hs ? &shared[l] : nullptr,
+                                          r, r_out, at<float>(ws, LY.logits), at<int32_t>(ws, LY.idx),
+                                          at<float>(ws, LY.w), at<uint16_t>(ws, LY.hdec), at<Ctrl>(ws, LY.ctrl), s);
+      if (e == cudaSuccess) continue;
+      if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge) return cuda_status(e);
+      (void)cudaGetLastError();
+    }
     if ((st = moe_rmsnorm_bf16(r, T, H, eps, u, stream)) != MOE_OK) return st;
     st = moe_layer_forward(u, T, Wr[l], bias ? bias[l] : nullptr, desc, &routed[l], hs ? &shared[l] : nullptr, r, r_out,
                            nullptr, nullptr, path, ws, ws_bytes, s);

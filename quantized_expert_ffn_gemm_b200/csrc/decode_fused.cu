@@ -1,25 +1,35 @@
 // Fused decode / MTP-verify layer (1-8 tokens): one cooperative kernel per MoE layer.
 //
 // A decode step is bound by reading weights ("Strata vs Llama.cpp vs vLLM", chapter "Why LLM
-// inference is a systems problem"), and at 1-4 tokens a layer moves only ~15 MB, so separate
-// router / gate-up / down kernels spend most of their time in launch gaps and dependent memory
-// round trips. Here one grid of one CTA per SM runs the three phases with two grid barriers:
-//   P1  router logits: four warps per expert split H (128-bit loads of the fp32 router rows);
-//       meanwhile the always-on shared expert's gate/up rows are prefetched into L2.
+// inference is a systems problem"), and at 1-4 tokens a layer moves only ~15 MB: spread over 148
+// SMs that is ~100 KB per SM, less than one SM's shared memory. So the kernel asks for all of it
+// at once: as soon as the routing is known, the warps of every CTA issue 16-byte async copies
+// (cp.async, each warp's completion counted on one mbarrier per slot) of the CTA's whole share of
+// gate/up rows and down rows into a ring of shared-memory slots, and then work from shared memory
+// as the slots fill; a slot that is read out is refilled at once by the warp that freed it. HBM
+// then sees the layer's expert bytes requested within a few hundred nanoseconds instead of as a
+// chain of dependent round trips.
+//
+// One grid of one CTA per SM (16 warps) runs three phases with two grid barriers:
+//   P1  router logits: four warps per expert split H (the fp32 router rows are requested before
+//       the tokens are staged); the shared expert's rows are prefetched into L2 meanwhile.
 //   --  grid barrier
-//   P1b every CTA computes the same top-k (partial top-k of 32-expert slices in all warps, then
-//       one merge warp per token) and distinct-expert unit list from the logits (deterministic),
-//       so no second exchange is needed; each CTA prefetches into L2 the down-projection rows it
-//       will need in P3.
-//   P2  gate/up + SwiGLU: one (unit, 16-row block) group per CTA at a time, 16 warps = gate/up x
-//       8 K steps on the tensor cores (mma.sync, fp16 operands, fp32 accumulate), the next
-//       group's weights requested before the current one is computed; h goes to the workspace.
+//   P1b every CTA computes the same top-k (each warp sorts a 32-expert slice, one warp per token
+//       merges the slices' heads) and the distinct-expert unit list (deterministic), so no second
+//       exchange is needed. The warps then issue this CTA's copies: gate/up items (unit, 8
+//       features: 8 gate rows + 8 up rows over all of H) dealt round-robin over CTAs, then the
+//       down rows of the CTA's 16 output features for every unit.
+//   P2  gate/up + SwiGLU: two groups of 8 warps take alternate items; in a group warp j runs
+//       K step j (256 wide) on the tensor cores (mma.sync m16n8k16 with A rows 0-7 = gate and
+//       8-15 = up rows of the same features, fp16 operands, fp32 accumulate); the partials are
+//       summed in fixed order and h goes to the workspace.
 //   --  grid barrier
 //   P3  down projection fused with the weighted combine: each CTA owns 16 output features, its
 //       warps split the (unit, K step) items, partials are reduced in fixed order (no atomics).
 // The grid barrier is one 64-bit arrival counter in the workspace (every launch adds 2 x grid;
-// a CTA waits for the launch's base + j x grid); its wait is bounded in time and reports
-// MOE_ERR_TIMEOUT instead of hanging. Cross-CTA data is read with L1-bypassing loads.
+// a CTA waits for the launch's base + j x grid). It and every mbarrier wait are bounded in time
+// and report MOE_ERR_TIMEOUT instead of hanging; before the CTA exits every thread waits for its
+// own outstanding copies (cp.async.wait_all), so no copy is still writing its shared memory.
 #include "common.cuh"
 #include "dequant.cuh"
 #include "gemv.cuh"
@@ -32,11 +42,19 @@ namespace {
 
 constexpr int kFWarps = 16;
 constexpr int kFThreads = kFWarps * 32;
-constexpr int kFMaxUnits = kDecodeMaxT * kMaxK + 1;
-constexpr int kFSlots = 64;  // h columns (token, expert) of a step staged for the down phase
+constexpr int kFSlots = 64;                 // h columns (token, expert) of a step staged for the down phase
+constexpr int kFMaxUnits = kFSlots + 1;
+constexpr int kFMaxRing = 16;               // shared-memory slots for weight copies
+constexpr int kFMaxE = 512;                 // experts the fused kernel takes
+constexpr int kFSmemMax = 226 * 1024;       // dynamic shared memory (a little is left for static)
+
+// named barriers (0 is __syncthreads): one per gate/up group
+constexpr int kBarGroup0 = 1;
 
 struct FusedArgs {
-  const uint16_t *x;
+  const uint16_t *x;       // bf16 tokens, or NULL when r_norm is given
+  const float *r_norm;     // fp32 residual stream: x = bf16(RMSNorm_eps(r)) is computed here
+  float eps;
   int T, H, E, k, I, has_shared;
   const float *Wr;
   const float *bias;
@@ -48,46 +66,58 @@ struct FusedArgs {
   float *w;
   uint16_t *hdec;
   Ctrl *ctrl;
+  int ring;        // slots in the ring
+  int slot_bytes;  // bytes per slot
+  int gu_bytes;    // bytes of one gate/up item
+  int dn_bytes;    // bytes of one unit's 16 down rows
+  int dpu;         // units per down slot
 };
 
 struct FusedLayout {
-  size_t xraw, x16, hs, part, red, units, scratch, sidx, sw, misc, slot, src, plist, total;
+  size_t xraw, x16, hs, part, red, units, sidx, sw, misc, slot, src, plist, firstof, pcnt, bars, ring, total;
 };
 
-__host__ __device__ inline size_t fl_align(size_t v) { return (v + 15) & ~(size_t)15; }
+__host__ __device__ inline size_t fl_align(size_t v, size_t a = 16) { return (v + a - 1) & ~(a - 1); }
 
-__host__ __device__ inline FusedLayout fused_layout(int T, int H, int I) {
+__host__ __device__ inline FusedLayout fused_layout(int T, int H, int E, int I, int hs_cols, int ring, int slot_bytes) {
   FusedLayout L{};
   size_t o = 0;
   auto take = [&](size_t b) { size_t r = o; o = fl_align(o + b); return r; };
   L.xraw = take((size_t)T * H * 2);
-  L.x16 = take((size_t)8 * (H + 4) * 2);
-  L.hs = take((size_t)kFSlots * (I + 4) * 2);
-  L.part = take((size_t)kFWarps * 16 * 8 * 4);
+  L.x16 = take((size_t)T * (H + 4) * 2);
+  L.hs = take((size_t)hs_cols * (I + 4) * 2);    // staged h columns (down phase)
+  L.part = take((size_t)2 * 2 * 8 * 16 * 8 * 4);  // [group][buffer][K step][16 rows][8 columns]
   L.red = take((size_t)kFWarps * 16 * 8 * 4);
   L.units = take((size_t)kFMaxUnits * sizeof(DecUnit));
-  L.scratch = take(sizeof(UnitScratch));
   L.sidx = take((size_t)kDecodeMaxT * kMaxK * 4);
   L.sw = take((size_t)kDecodeMaxT * kMaxK * 4);
   L.misc = take(16 * 4);
   L.slot = take((size_t)(kFMaxUnits + 1) * 4);
   L.src = take((size_t)kFSlots * 4);
-  L.plist = take((size_t)2 * kDecodeMaxT * 16 * 16 * 8);  // top-16 code lists (tokens x 32-expert chunks), x2
+  L.plist = take((size_t)T * 16 * 16 * 8);      // top-16 code lists (tokens x 32-expert chunks)
+  L.firstof = take((size_t)E * 4);                // expert -> first pair choosing it
+  L.pcnt = take((size_t)(kFMaxUnits + 1) * 4);
+  L.bars = take((size_t)kFMaxRing * 8);
+  o = fl_align(o, 128);
+  L.ring = o;
+  o += (size_t)ring * slot_bytes;
   L.total = o;
   return L;
 }
 
 // all CTAs are co-resident (cooperative launch). Barrier j of a launch completes when the arrival
-// counter reaches base + j * nblocks; false when the wait gave up.
-__device__ bool grid_barrier(Ctrl *c, unsigned long long target, int where) {
+// counter reaches base + j * nblocks. Every CTA arrives, even after an earlier failure, so the
+// count stays whole; it waits only when `wait` is set. Returns false when the wait gave up (or
+// was not made). Called by every thread of the CTA.
+__device__ bool grid_barrier(Ctrl *c, unsigned long long target, int where, bool wait) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
     asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(&c->bar_arrivals) : "memory");
-    int ok = 1;
+    int ok = wait ? 1 : 0;
     const uint64_t t0 = global_ns();
-    while (true) {
+    while (wait) {
       unsigned long long v;
       asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(&c->bar_arrivals) : "memory");
       if ((long long)(v - target) >= 0) break;
@@ -114,42 +144,196 @@ __device__ __forceinline__ void prefetch_range(const void *p, size_t bytes, int 
   for (size_t off = (size_t)first * 128; off < bytes; off += (size_t)nthr * 128) prefetch_l2(c + off);
 }
 
+// 16-byte global -> shared async copy (L2 only); both addresses 16-byte aligned
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// arrive on `bar` once every cp.async this thread issued so far has landed (counts against the
+// barrier's expected arrivals)
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// One contiguous piece of a slot fill, as (source, offset in the slot, bytes).
+//   gate/up slot: [gate codes 8 x H/4][up codes 8 x H/4][gate scales 8 x H/32][up scales]
+//                 [gate hi 8 x H/8][up hi]                     (5H bytes; Q3 7H)
+//   down slot:    dpu pieces of [codes 16 x I/4][scales 16 x I/32][hi 16 x I/8]   (5I; Q3 7I)
+struct CopyDesc {
+  const void *src;
+  uint32_t off, bytes;
+};
+
+template <bool Q3>
+__device__ __forceinline__ CopyDesc gu_copy(const FusedArgs &a, const DecUnit &un, int r0, int c) {
+  const int H = a.H;
+  const int which = c & 1;  // 0 gate, 1 up
+  const MatView m = mat_sel(a.routed, a.shared, un.set, which, un.expert);
+  CopyDesc d;
+  if (c < 2) {
+    d.src = m.codes + (size_t)r0 * (H / 4);
+    d.bytes = 2 * H;
+    d.off = which * 2 * H;
+  } else if (c < 4) {
+    d.src = m.scales + (size_t)r0 * (H / 32);
+    d.bytes = H / 2;
+    d.off = 4 * H + which * (H / 2);
+  } else {
+    d.src = m.hibits + (size_t)r0 * (H / 8);
+    d.bytes = H;
+    d.off = 5 * H + which * H;
+  }
+  return d;
+}
+
+template <bool Q3>
+__device__ __forceinline__ CopyDesc dn_copy(const FusedArgs &a, const DecUnit &un, int rb, int slot_unit, int c) {
+  const int I = a.I;
+  const MatView m = mat_sel(a.routed, a.shared, un.set, 2, un.expert);
+  const size_t row = (size_t)rb * 16;
+  const uint32_t base = (uint32_t)(slot_unit * a.dn_bytes);
+  CopyDesc d;
+  if (c == 0) {
+    d.src = m.codes + row * (I / 4);
+    d.bytes = 4 * I;
+    d.off = base;
+  } else if (c == 1) {
+    d.src = m.scales + row * (I / 32);
+    d.bytes = I;
+    d.off = base + 4 * I;
+  } else {
+    d.src = m.hibits + row * (I / 8);
+    d.bytes = 2 * I;
+    d.off = base + 5 * I;
+  }
+  return d;
+}
+
+// one lane's share of a 16-row x 256-wide K step read from a staged slot: the code rows of MMA
+// rows g and g+8 start at ca / cb, their scales at sa / sb (halves), their hi bits at ha / hb
+template <bool Q3>
+__device__ __forceinline__ void frag_from_smem(StepFrag &f, const uint8_t *ca, const uint8_t *cb, const uint16_t *sa,
+                                               const uint16_t *sb, const uint8_t *ha, const uint8_t *hb, int k0) {
+  f.w0 = *reinterpret_cast<const uint4 *>(ca + k0 / 4);
+  f.w1 = *reinterpret_cast<const uint4 *>(cb + k0 / 4);
+  f.d0 = *reinterpret_cast<const uint32_t *>(sa + k0 / 32);
+  f.d1 = *reinterpret_cast<const uint32_t *>(sb + k0 / 32);
+  if (Q3) {
+    f.h0 = *reinterpret_cast<const uint2 *>(ha + k0 / 8);
+    f.h1 = *reinterpret_cast<const uint2 *>(hb + k0 / 8);
+  }
+}
+
 }  // namespace
 
 template <bool Q3>
 __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedArgs a) {
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(128) unsigned char smem[];
   const int T = a.T, H = a.H, E = a.E, k = a.k, I = a.I;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
-  const FusedLayout L = fused_layout(T, H, I);
+  const int hs_cols = T * k + (a.has_shared ? T : 0);
+  const FusedLayout L = fused_layout(T, H, E, I, hs_cols, a.ring, a.slot_bytes);
   uint16_t *xraw = reinterpret_cast<uint16_t *>(smem + L.xraw);
   __half *x16 = reinterpret_cast<__half *>(smem + L.x16);
   __half *hs = reinterpret_cast<__half *>(smem + L.hs);
   float *part = reinterpret_cast<float *>(smem + L.part);
   float *red = reinterpret_cast<float *>(smem + L.red);
   DecUnit *su = reinterpret_cast<DecUnit *>(smem + L.units);
-  UnitScratch &us = *reinterpret_cast<UnitScratch *>(smem + L.scratch);
   int32_t *s_idx = reinterpret_cast<int32_t *>(smem + L.sidx);
   float *s_w = reinterpret_cast<float *>(smem + L.sw);
   int *misc = reinterpret_cast<int *>(smem + L.misc);
   int *s_slot = reinterpret_cast<int *>(smem + L.slot);
   int *s_src = reinterpret_cast<int *>(smem + L.src);
   unsigned long long *plist = reinterpret_cast<unsigned long long *>(smem + L.plist);
+  int *s_firstof = reinterpret_cast<int *>(smem + L.firstof);
+  int *s_pcnt = reinterpret_cast<int *>(smem + L.pcnt);
+  const uint32_t bar_full0 = smem_u32(smem + L.bars);
+  const uint32_t ring0 = smem_u32(smem + L.ring);
+  const uint8_t *ringp = smem + L.ring;
+  const int R = a.ring, S = a.slot_bytes;
+  auto full = [&](int s) { return bar_full0 + 8u * (uint32_t)s; };
   Ctrl *ctrl = a.ctrl;
   const int xs16 = H + 4;
+  const int G = gridDim.x;
   const unsigned nblk = gridDim.x;
   __shared__ unsigned long long s_base;
+  __shared__ volatile int s_abort;
   if (tid == 0) {  // arrivals of earlier launches: a whole number of 2 x grid (before this CTA arrives)
     unsigned long long v;
     asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(&ctrl->bar_arrivals) : "memory");
     s_base = v - v % nblk;
+    s_abort = 0;
+    for (int s = 0; s < R; ++s) mbar_init(full(s), 32);  // one arrival per lane of the filling warp
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  // a bounded wait that gives up at once after an earlier wait of this CTA gave up
+  auto wait_bar = [&](uint32_t bar, uint32_t parity, int where) -> bool {
+    if (s_abort) return false;
+    if (mbar_wait(bar, parity)) return true;
+    s_abort = 1;
+    set_device_error(ctrl, MOE_ERR_TIMEOUT, where);
+    return false;
+  };
 
-  // ---------------- P0: tokens into shared memory (raw bf16 for the router, fp16 rotated for the MMAs)
+  // ---------------- P0: this warp's router rows are requested first, then the tokens are staged
+  const int H4 = H / 4, HQ = H4 / 4;  // float4 per quarter of a router row (<= 128: H <= 2048)
+  const int es = warp >> 2, qh = warp & 3;
+  float4 rv[4];
+  auto load_router = [&](int e) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int h4 = lane + 32 * u;
+      rv[u] = (e < E && h4 < HQ) ? __ldcs(reinterpret_cast<const float4 *>(a.Wr + (size_t)e * H) + qh * HQ + h4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  load_router((int)blockIdx.x + es * G);
+  __shared__ float s_inv[kDecodeMaxT];
+  if (a.r_norm) {
+    // RMSNorm of the residual stream (no gain): the same summation order and rounding as the
+    // stand-alone RMSNorm kernel (256 threads: strided fmaf chains, warp butterflies, 8 warp
+    // partials in order), so u is bit-identical to it
+    __shared__ float s_part[kDecodeMaxT][8];
+    if (tid < 256) {
+      for (int t = 0; t < T; ++t) {
+        const float *row = a.r_norm + (size_t)t * H;
+        float ss = 0.0f;
+        for (int h = tid; h < H; h += 256) ss = fmaf(__ldg(row + h), __ldg(row + h), ss);
+        ss = warp_sum(ss);
+        if (lane == 0) s_part[t][warp] = ss;
+      }
+    }
+    __syncthreads();
+    if (tid < T) {
+      float tot = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) tot += s_part[tid][i];
+      s_inv[tid] = 1.0f / sqrtf(tot / (float)H + a.eps);
+    }
+    __syncthreads();
+  }
   {
     const int H8 = H / 8, n = T * H8;
     for (int i = tid; i < n; i += kFThreads) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(a.x) + i);
+      uint4 v;
+      if (a.r_norm) {
+        const int t = i / H8;
+        const float4 f0 = __ldg(reinterpret_cast<const float4 *>(a.r_norm) + 2 * i);
+        const float4 f1 = __ldg(reinterpret_cast<const float4 *>(a.r_norm) + 2 * i + 1);
+        const float iv = s_inv[t];
+        auto pk = [&](float lo, float hi) {
+          const __nv_bfloat16 bl = __float2bfloat16_rn(lo * iv), bh = __float2bfloat16_rn(hi * iv);
+          return (uint32_t)*reinterpret_cast<const uint16_t *>(&bl) |
+                 ((uint32_t)*reinterpret_cast<const uint16_t *>(&bh) << 16);
+        };
+        v = make_uint4(pk(f0.x, f0.y), pk(f0.z, f0.w), pk(f1.x, f1.y), pk(f1.z, f1.w));
+      } else {
+        v = __ldg(reinterpret_cast<const uint4 *>(a.x) + i);
+      }
       reinterpret_cast<uint4 *>(xraw)[i] = v;
       const int t = i / H8, c = i % H8;
       const uint32_t in[4] = {v.x, v.y, v.z, v.w};
@@ -164,17 +348,20 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       d[1] = make_uint2(o[2], o[3]);
     }
   }
-  {  // into L2 while the router runs: the shared expert's gate/up rows and the router bias
+  {  // into L2 while the router runs: the shared expert's rows and the router bias
     const int nthr = gridDim.x * kFThreads, first = blockIdx.x * kFThreads + tid;
     if (a.has_shared) {
       const size_t cb = (size_t)I * H / 4, sb = (size_t)I * H / 32 * 2;
       prefetch_range(a.shared.gate.codes, cb, first, nthr);
       prefetch_range(a.shared.up.codes, cb, first, nthr);
+      prefetch_range(a.shared.down.codes, cb, first, nthr);
       prefetch_range(a.shared.gate.scales, sb, first, nthr);
       prefetch_range(a.shared.up.scales, sb, first, nthr);
+      prefetch_range(a.shared.down.scales, sb, first, nthr);
       if (Q3) {
         prefetch_range(a.shared.gate.hibits, cb / 2, first, nthr);
         prefetch_range(a.shared.up.hibits, cb / 2, first, nthr);
+        prefetch_range(a.shared.down.hibits, cb / 2, first, nthr);
       }
     }
     if (a.bias) prefetch_range(a.bias, (size_t)E * 4, tid, kFThreads);
@@ -183,36 +370,26 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
 
   // ---------------- P1: router logits, four warps per expert (each a quarter of H), fp32
   {
-    const int H4 = H / 4, HQ = H4 / 4;  // float4 per quarter
-    const int es = warp >> 2, qh = warp & 3;
     float *rp = red;  // [4 experts][4 quarters][T]
-    for (int e0 = blockIdx.x; e0 < E; e0 += 4 * gridDim.x) {
-      const int e = e0 + es * gridDim.x;
+    for (int e0 = blockIdx.x, it = 0; e0 < E; e0 += 4 * G, ++it) {
+      const int e = e0 + es * G;
+      if (it > 0) load_router(e);
       float acc[kDecodeMaxT];
 #pragma unroll
       for (int t = 0; t < kDecodeMaxT; ++t) acc[t] = 0.0f;
       if (e < E) {
-        const float4 *wr = reinterpret_cast<const float4 *>(a.Wr + (size_t)e * H) + qh * HQ;
-        for (int h0 = 0; h0 < HQ; h0 += 32 * 4) {
-          float4 v[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int h4 = h0 + lane + 32 * u;
-            v[u] = (h4 < HQ) ? __ldcs(wr + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
+        for (int u = 0; u < 4; ++u) {
+          const int h4 = lane + 32 * u;
+          if (h4 >= HQ) continue;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int h4 = h0 + lane + 32 * u;
-            if (h4 >= HQ) continue;
-#pragma unroll
-            for (int t = 0; t < kDecodeMaxT; ++t) {
-              if (t < T) {
-                const uint2 xb = reinterpret_cast<const uint2 *>(xraw + (size_t)t * H)[qh * HQ + h4];
-                acc[t] = fmaf(v[u].x, __uint_as_float(xb.x << 16), acc[t]);
-                acc[t] = fmaf(v[u].y, __uint_as_float(xb.x & 0xffff0000u), acc[t]);
-                acc[t] = fmaf(v[u].z, __uint_as_float(xb.y << 16), acc[t]);
-                acc[t] = fmaf(v[u].w, __uint_as_float(xb.y & 0xffff0000u), acc[t]);
-              }
+          for (int t = 0; t < kDecodeMaxT; ++t) {
+            if (t < T) {
+              const uint2 xb = reinterpret_cast<const uint2 *>(xraw + (size_t)t * H)[qh * HQ + h4];
+              acc[t] = fmaf(rv[u].x, __uint_as_float(xb.x << 16), acc[t]);
+              acc[t] = fmaf(rv[u].y, __uint_as_float(xb.x & 0xffff0000u), acc[t]);
+              acc[t] = fmaf(rv[u].z, __uint_as_float(xb.y << 16), acc[t]);
+              acc[t] = fmaf(rv[u].w, __uint_as_float(xb.y & 0xffff0000u), acc[t]);
             }
           }
         }
@@ -226,173 +403,250 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       }
       __syncthreads();
       if (tid < 4 * T) {  // fixed-order sum of the four quarters
-        const int ee = tid / T, t = tid % T, eg = e0 + ee * gridDim.x;
+        const int ee = tid / T, t = tid % T, eg = e0 + ee * G;
         if (eg < E) {
-          const float* q4 = rp + ee * 4 * kDecodeMaxT;
-          a.logits[(size_t)t * E + eg] = (q4[t] + q4[kDecodeMaxT + t]) + (q4[2 * kDecodeMaxT + t] + q4[3 * kDecodeMaxT + t]);
+          const float *q4 = rp + ee * 4 * kDecodeMaxT;
+          a.logits[(size_t)t * E + eg] =
+              (q4[t] + q4[kDecodeMaxT + t]) + (q4[2 * kDecodeMaxT + t] + q4[3 * kDecodeMaxT + t]);
         }
       }
       __syncthreads();
     }
   }
   __threadfence();
-  if (!grid_barrier(ctrl, s_base + nblk, 31)) return;
+  bool ok = grid_barrier(ctrl, s_base + nblk, 31, true);
 
   // ---------------- P1b: top-k and unit list, computed identically by every CTA
-  {
-    float *ls = reinterpret_cast<float *>(hs);  // T * E floats, before h is staged there
-    for (int i = tid; i < T * E; i += kFThreads) ls[i] = __ldcg(a.logits + i) + (a.bias ? __ldg(a.bias + i % E) : 0.f);
-    __syncthreads();
-    // top-k per token: every 32-expert chunk is sorted by one warp (top 16 kept), then the
-    // chunks' lists are merged pairwise (bitonic merge of a list and its partner reversed)
-    const int nch = (E + 31) / 32;
-    int npow = 1;
-    while (npow < nch) npow <<= 1;
-    for (int task = warp; task < T * npow; task += kFWarps) {
-      const int t = task / npow, c = task % npow, e = c * 32 + lane;
-      unsigned long long v = (c < nch && e < E) ? topk_code(ls[(size_t)t * E + e], e) : 0ull;
+  if (ok) {
+    // every 32-expert chunk of every token is sorted by one warp straight from the logits (top 16
+    // kept); then one warp per token merges the chunks' lists: lane c holds list c in registers,
+    // each round the warp takes the best head (max key, then lowest index) and that lane shifts
+    const int nch = (E + 31) / 32;  // <= 16
+    for (int task = warp; task < T * nch; task += kFWarps) {
+      const int t = task / nch, c = task % nch, e = c * 32 + lane;
+      unsigned long long v = 0ull;
+      if (e < E) v = topk_code(__ldcg(a.logits + (size_t)t * E + e) + (a.bias ? __ldg(a.bias + e) : 0.f), e);
       v = warp_sort32_desc(v);
       if (lane < 16) plist[(size_t)task * 16 + lane] = v;
     }
+    if (T > 1)
+      for (int e = tid; e < E; e += kFThreads) s_firstof[e] = 0x7fffffff;
     __syncthreads();
-    unsigned long long *cur = plist, *nxt = plist + (size_t)kDecodeMaxT * 16 * 16;  // ping-pong halves
-    for (int len = npow; len > 1; len >>= 1) {  // lists of each token: len -> len / 2
-      for (int task = warp; task < T * (len / 2); task += kFWarps) {
-        const int t = task / (len / 2), c = task % (len / 2);
-        const unsigned long long *la = cur + ((size_t)t * npow + 2 * c) * 16;
-        const unsigned long long *lb = cur + ((size_t)t * npow + 2 * c + 1) * 16;
-        unsigned long long v = (lane < 16) ? la[lane] : lb[31 - lane];
-        v = warp_merge32_desc(v);
-        if (lane < 16) nxt[((size_t)t * npow + c) * 16 + lane] = v;
+    if (warp < T) {
+      unsigned long long c[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) c[i] = (lane < nch) ? plist[((size_t)warp * nch + lane) * 16 + i] : 0ull;
+      float my_val = -INFINITY;
+      int my_idx = 0;
+      for (int j = 0; j < k; ++j) {
+        const uint32_t hk = (uint32_t)(c[0] >> 32);
+        const uint32_t m = __reduce_max_sync(0xffffffffu, hk);
+        const uint32_t lo = (hk == m) ? (uint32_t)c[0] : 0u;
+        const uint32_t win = __reduce_max_sync(0xffffffffu, lo);  // max of (~index) = lowest index
+        const bool is_win = (hk == m) && ((uint32_t)c[0] == win);
+#pragma unroll
+        for (int i = 0; i < 15; ++i) c[i] = is_win ? c[i + 1] : c[i];
+        c[15] = is_win ? 0ull : c[15];
+        if (lane == j) {
+          my_val = key_to_logit(m);
+          my_idx = (int)(0xFFFFFFFFu - win);
+        }
       }
+      topk_finish(my_val, my_idx, k, s_idx + warp * k, s_w + warp * k);
+    }
+    __syncthreads();
+    const int P = T * k;
+    if (T > 1) {  // expert -> first pair choosing it
+      for (int p = tid; p < P; p += kFThreads) atomicMin(&s_firstof[s_idx[p]], p);
       __syncthreads();
-      unsigned long long *tmp = cur;
-      cur = nxt;
-      nxt = tmp;
     }
-    if (warp < T) {  // list 0 of token `warp` holds its top 16 in descending order
-      const unsigned long long v = (lane < k) ? cur[(size_t)warp * npow * 16 + lane] : 0ull;
-      const float val = (lane < k) ? key_to_logit((uint32_t)(v >> 32)) : -INFINITY;
-      const int ix = (lane < k) ? (int)(0xFFFFFFFFu - (uint32_t)v) : 0;
-      topk_finish(val, ix, k, s_idx + warp * k, s_w + warp * k);
-    }
-    __syncthreads();
-    build_units(s_idx, s_w, T, k, E, a.has_shared, su, &misc[0], us);
-    if (blockIdx.x == 0)
-      for (int i = tid; i < T * k; i += kFThreads) {
-        a.idx[i] = s_idx[i];
-        a.w[i] = s_w[i];
+    if (warp == 0) {
+      // units: the distinct experts of the P = T*k (< 64) selections in order of first
+      // appearance (token-major), then the shared expert. Pair p leads its unit when it is the
+      // first pair to choose its expert (one token's k experts are distinct, so at T = 1 every
+      // pair leads); a leader's unit number is the count of leaders before it.
+      int fp[2];
+      bool lead[2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int p = lane + 32 * hh;
+        fp[hh] = (p < P) ? (T > 1 ? s_firstof[s_idx[p]] : p) : p;
+        lead[hh] = (p < P) && fp[hh] == p;
       }
-    if (warp == 0) {  // slot table of the down phase: present (unit, token) columns in unit order
+      const unsigned b0 = __ballot_sync(0xffffffffu, lead[0]), b1 = __ballot_sync(0xffffffffu, lead[1]);
+      const int nr = __popc(b0) + __popc(b1);
+      auto unit_of = [&](int q) {
+        return q < 32 ? __popc(b0 & ((1u << q) - 1u)) : __popc(b0) + __popc(b1 & ((1u << (q - 32)) - 1u));
+      };
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int p = lane + 32 * hh;
+        if (lead[hh]) {
+          DecUnit &d = su[unit_of(p)];
+          d.expert = s_idx[p];
+          d.set = 0;
+          d.mask = 0;
+          d.xrow0 = 0;
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) d.w[cc] = 0.0f;
+        }
+      }
+      if (a.has_shared && lane == 0) {
+        DecUnit &d = su[nr];
+        d.expert = 0;
+        d.set = 1;
+        d.mask = (1 << T) - 1;
+        d.xrow0 = 0;
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) d.w[cc] = cc < T ? 1.0f : 0.0f;
+      }
+      __syncwarp();
+      // every (unit, token) is one pair: an expert appears at most once per token
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int p = lane + 32 * hh;
+        if (p < P) {
+          DecUnit &d = su[unit_of(fp[hh])];
+          atomicOr(&d.mask, 1 << (p / k));
+          d.w[p / k] = s_w[p];
+        }
+      }
+      __syncwarp();
+      const int nu = nr + (a.has_shared ? 1 : 0);
+      if (lane == 0) misc[0] = nu;
+      // slot table of the down phase: present (unit, token) columns in unit order
       int used = 0;
-      for (int base = 0; base < misc[0]; base += 32) {
+      for (int base = 0; base < nu; base += 32) {
         const int u = base + lane;
-        const int c = (u < misc[0]) ? __popc(su[u].mask & 0xff) : 0;
-        int incl = c;
+        const int cnt = (u < nu) ? __popc(su[u].mask & 0xff) : 0;
+        int incl = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const int n = __shfl_up_sync(0xffffffffu, incl, o);
           if (lane >= o) incl += n;
         }
-        if (u < misc[0]) s_slot[u] = used + incl - c;
+        if (u < nu) {
+          int sl = used + incl - cnt;
+          s_slot[u] = sl;
+          const int m = su[u].mask & 0xff;
+          for (int cc = 0; cc < 8; ++cc)
+            if ((m >> cc) & 1) s_src[sl++] = u * 8 + cc;
+        }
         used += __shfl_sync(0xffffffffu, incl, 31);
       }
-      if (lane == 0) s_slot[misc[0]] = used;
+      if (lane == 0) s_slot[nu] = used;
     }
-    __syncthreads();
-    for (int u = tid; u < misc[0]; u += kFThreads) {
-      int sl = s_slot[u];
-      const int m = su[u].mask & 0xff;
-      for (int c = 0; c < 8; ++c)
-        if ((m >> c) & 1) s_src[sl++] = u * 8 + c;
-    }
-    __syncthreads();
-  }
-  const int nu = misc[0];
-  // down-projection rows of this CTA's P3 output block(s) into L2 (16 rows x I, for every unit)
-  for (int rb = blockIdx.x; rb < H / 16; rb += gridDim.x) {
-    const size_t rowb = (size_t)I / 4, srowb = (size_t)I / 32 * 2;
-    for (int u = warp; u < nu; u += kFWarps) {
-      const DecUnit &un = su[u];
-      const MatView mv = mat_sel(a.routed, a.shared, un.set, 2, un.expert);
-      prefetch_range(mv.codes + (size_t)rb * 16 * rowb, 16 * rowb, lane, 32);
-      prefetch_range(mv.scales + (size_t)rb * 16 * (I / 32), 16 * srowb, lane, 32);
-      if (Q3) prefetch_range(mv.hibits + (size_t)rb * 16 * (I / 8), 16 * rowb / 2, lane, 32);
-    }
-  }
-
-  // ---------------- P2: gate/up + SwiGLU, one (unit, 16-row block) group per CTA at a time
-  {
-    const int rbs = I / 16, G2 = nu * rbs;
-    const int mat = warp >> 3, slice = warp & 7;  // warps 0-7 gate, 8-15 up; slice = K step (mod 8)
-    const int nsteps = (H + kStepK - 1) / kStepK;  // <= 8 (H <= 2048)
-    const __half *xs_base = x16;
-    StepFrag f;
-    int gi = blockIdx.x;
-    if (gi < G2) {
-      const DecUnit &un = su[gi / rbs];
-      load_step<Q3>(f, mat_sel(a.routed, a.shared, un.set, mat, un.expert), (gi % rbs) * 16, slice, slice < nsteps);
-    }
-    for (; gi < G2; gi += gridDim.x) {
-      const int u = gi / rbs, r0 = (gi % rbs) * 16;
-      const DecUnit &un = su[u];
-      // next group's weights go out before this group is computed
-      StepFrag fn;
-      const int gn = gi + gridDim.x;
-      if (gn < G2) {
-        const DecUnit &un2 = su[gn / rbs];
-        load_step<Q3>(fn, mat_sel(a.routed, a.shared, un2.set, mat, un2.expert), (gn % rbs) * 16, slice,
-                      slice < nsteps);
+    if (blockIdx.x == 0)
+      for (int i = tid; i < P; i += kFThreads) {
+        a.idx[i] = s_idx[i];
+        a.w[i] = s_w[i];
       }
-      const bool colok = (un.mask >> g) & 1;
+    __syncthreads();
+  }
+  const int nu = ok ? misc[0] : 0;
+  const int rbs8 = I / 8;                     // gate/up items per unit
+  const int n_gu = nu * rbs8;
+  const int n_mine = (n_gu > (int)blockIdx.x) ? (n_gu - (int)blockIdx.x + G - 1) / G : 0;
+  const int n_rb = (H / 16 > (int)blockIdx.x) ? (H / 16 - (int)blockIdx.x + G - 1) / G : 0;  // down row blocks
+  const int npieces = (nu + a.dpu - 1) / a.dpu;  // down slots per row block
+  const int n_total = n_mine + n_rb * npieces;
+  const int nsteps_gu = (H + kStepK - 1) / kStepK;  // <= 8
+  const int nsteps_dn = (I + kStepK - 1) / kStepK;
+
+  // ---------------- fills: fill q of this CTA (gate/up items, then down pieces) goes to slot
+  // q % R; it is issued by one whole warp (cp.async, 16 bytes per lane per instruction), whose
+  // 32 lanes then arrive on the slot's barrier when their copies have landed
+  auto issue_fill = [&](int q) {
+    const int s = q % R;
+    const uint32_t dst0 = ring0 + (uint32_t)(s * S);
+    if (q < n_mine) {
+      const int i = (int)blockIdx.x + q * G;
+      const DecUnit &un = su[i / rbs8];
+      const int r0 = (i % rbs8) * 8;
+      const int nc = Q3 ? 6 : 4;
+      for (int c = 0; c < nc; ++c) {
+        const CopyDesc d = gu_copy<Q3>(a, un, r0, c);
+        const char *src = static_cast<const char *>(d.src);
+        for (uint32_t off = 16u * lane; off < d.bytes; off += 512u) cp_async16(dst0 + d.off + off, src + off);
+      }
+    } else {
+      const int j = q - n_mine, rbl = j / npieces, dp = j % npieces;
+      const int rb = (int)blockIdx.x + rbl * G;
+      const int nun = min(a.dpu, nu - dp * a.dpu);
+      const int per = Q3 ? 3 : 2;
+      for (int m = 0; m < nun; ++m) {
+        const DecUnit &un = su[dp * a.dpu + m];
+        for (int c = 0; c < per; ++c) {
+          const CopyDesc d = dn_copy<Q3>(a, un, rb, m, c);
+          const char *src = static_cast<const char *>(d.src);
+          for (uint32_t off = 16u * lane; off < d.bytes; off += 512u) cp_async16(dst0 + d.off + off, src + off);
+        }
+      }
+    }
+    cp_async_arrive(full(s));
+  };
+  if (ok)
+    for (int q = warp; q < min(n_total, R); q += kFWarps) issue_fill(q);
+
+  // ---------------- P2: gate/up + SwiGLU; group grp takes this CTA's items grp, grp + 2, ...
+  if (ok) {
+    const int grp = warp >> 3, j8 = warp & 7, gtid = tid & 255;
+    int buf = 0;
+    for (int q = grp; q < n_mine; q += 2, buf ^= 1) {
+      const int i = (int)blockIdx.x + q * G;
+      const int u = i / rbs8, r0 = (i % rbs8) * 8;
+      const DecUnit &un = su[u];
+      const int s = q % R;
+      const bool have = wait_bar(full(s), (uint32_t)(q / R) & 1u, 42);
       float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
-      if (slice < nsteps)
-        mma_step<Q3>(acc, acc2, f, xs_base + (size_t)g * xs16, slice * kStepK + 64 * t4,
-                     colok && slice * kStepK + 64 * t4 < H);
-      float *pw = part + warp * 16 * 8;
+      const int k0 = j8 * kStepK + 64 * t4;
+      if (have && j8 < nsteps_gu && k0 < H) {
+        const uint8_t *sl = ringp + (size_t)s * S;
+        const uint8_t *ca = sl + (size_t)g * (H / 4), *cb = sl + 2 * H + (size_t)g * (H / 4);
+        const uint16_t *sa = reinterpret_cast<const uint16_t *>(sl + 4 * H) + (size_t)g * (H / 32);
+        const uint16_t *sb = reinterpret_cast<const uint16_t *>(sl + 4 * H + H / 2) + (size_t)g * (H / 32);
+        const uint8_t *ha = sl + 5 * H + (size_t)g * (H / 8), *hb = sl + 6 * H + (size_t)g * (H / 8);
+        StepFrag f;
+        frag_from_smem<Q3>(f, ca, cb, sa, sb, ha, hb, k0);
+        mma_step<Q3>(acc, acc2, f, x16 + (size_t)g * xs16, k0, (un.mask >> g) & 1);
+      }
+      float *pw = part + (((size_t)(grp * 2 + buf) * 8 + j8) * 16) * 8;
       pw[g * 8 + 2 * t4] = acc[0] + acc2[0];
       pw[g * 8 + 2 * t4 + 1] = acc[1] + acc2[1];
       pw[(g + 8) * 8 + 2 * t4] = acc[2] + acc2[2];
       pw[(g + 8) * 8 + 2 * t4 + 1] = acc[3] + acc2[3];
-      __syncthreads();
-      if (tid < 128) {  // one (row, column) per thread; fixed-order sums of the 8 K slices
-        const int row = tid & 15, col = tid >> 4;
+      named_sync(kBarGroup0 + grp, 256);
+      // every warp of the group is done with the slot: its next fill goes out now
+      if (j8 == 7 && q + R < n_total) issue_fill(q + R);
+      if (gtid < 64) {  // one (feature, token) per thread; fixed-order sums of the 8 K steps
+        const int row = gtid & 7, col = gtid >> 3;
         if ((un.mask >> col) & 1) {
+          const float *pb = part + ((size_t)(grp * 2 + buf) * 8 * 16) * 8;
           float gv = 0.f, uv = 0.f;
 #pragma unroll
           for (int sl = 0; sl < 8; ++sl) {
-            gv += part[(sl * 16 + row) * 8 + col];
-            uv += part[((8 + sl) * 16 + row) * 8 + col];
+            gv += pb[(sl * 16 + row) * 8 + col];
+            uv += pb[(sl * 16 + 8 + row) * 8 + col];
           }
           const float hv = gv / (1.0f + expf(-gv)) * uv;
           a.hdec[((size_t)u * 8 + col) * I + r0 + row] = __half_as_ushort(__float2half_rn(hv));
         }
       }
-      __syncthreads();
-      f = fn;
     }
   }
   __threadfence();
-  if (!grid_barrier(ctrl, s_base + 2 * (unsigned long long)nblk, 32)) return;
+  ok = grid_barrier(ctrl, s_base + 2 * (unsigned long long)nblk, 32, ok) && ok;
 
   // ---------------- P3: down projection + weighted combine (+ residual) for 16 output features per CTA
-  {
+  if (ok) {
     const int nslots = s_slot[nu];
-    const int nsteps = (I + kStepK - 1) / kStepK;
     const int xstride = I + 4;
-    const int n_items = nu * nsteps;
-    for (int rb = blockIdx.x; rb < H / 16; rb += gridDim.x) {
-      const int r0 = rb * 16;
-      // this warp's first two items' weights are requested before h is staged
-      StepFrag f0, f1;
-      if (warp < n_items) {
-        const DecUnit &un = su[warp / nsteps];
-        load_step<Q3>(f0, mat_sel(a.routed, a.shared, un.set, 2, un.expert), r0, warp % nsteps, true);
-      }
-      if (warp + kFWarps < n_items) {
-        const DecUnit &un = su[(warp + kFWarps) / nsteps];
-        load_step<Q3>(f1, mat_sel(a.routed, a.shared, un.set, 2, un.expert), r0, (warp + kFWarps) % nsteps, true);
-      }
+    const int n_items = nu * nsteps_dn;
+    const int dn = a.dn_bytes;
+    for (int rbl = 0; rbl < n_rb; ++rbl) {
+      const int r0 = ((int)blockIdx.x + rbl * G) * 16;
+      const int qb = n_mine + rbl * npieces;
+      for (int i = tid; i < npieces; i += kFThreads) s_pcnt[i] = 0;
       {  // stage every present h column (16-byte loads, issued before the stores)
         const int I8 = I / 8, total = nslots * I8;
         for (int v0 = tid; v0 < total; v0 += 4 * kFThreads) {
@@ -416,24 +670,43 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       }
       __syncthreads();
       float tot[4] = {0.f, 0.f, 0.f, 0.f};
-      int j = 0;
-      for (int it = warp; it < n_items; it += kFWarps, ++j) {
-        const int u = it / nsteps, st = it % nsteps;
+      for (int it = warp; it < n_items; it += kFWarps) {
+        const int u = it / nsteps_dn, st = it % nsteps_dn;
+        const int d = u / a.dpu, qd = qb + d, s = qd % R;
+        const bool have = wait_bar(full(s), (uint32_t)(qd / R) & 1u, 43);
         const DecUnit &un = su[u];
-        const bool colok = (un.mask >> g) & 1;
+        const int k0 = st * kStepK + 64 * t4;
+        const bool kok = k0 < I;
+        const bool colok = ((un.mask >> g) & 1) && kok;
         const int slot = s_slot[u] + __popc(un.mask & ((1u << g) - 1u));
         const __half *xcol = hs + (size_t)(colok ? slot : 0) * xstride;
-        StepFrag f;
-        if (j == 0) f = f0;
-        else if (j == 1) f = f1;
-        else load_step<Q3>(f, mat_sel(a.routed, a.shared, un.set, 2, un.expert), r0, st, true);
         float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_step<Q3>(acc, acc2, f, xcol, st * kStepK + 64 * t4, colok && st * kStepK + 64 * t4 < I);
+        if (have && kok) {
+          const uint8_t *pc = ringp + (size_t)s * S + (size_t)(u % a.dpu) * dn;
+          const uint8_t *ca = pc + (size_t)g * (I / 4), *cb = pc + (size_t)(g + 8) * (I / 4);
+          const uint16_t *sa = reinterpret_cast<const uint16_t *>(pc + 4 * I) + (size_t)g * (I / 32);
+          const uint16_t *sb = reinterpret_cast<const uint16_t *>(pc + 4 * I) + (size_t)(g + 8) * (I / 32);
+          const uint8_t *ha = pc + 5 * I + (size_t)g * (I / 8), *hb = pc + 5 * I + (size_t)(g + 8) * (I / 8);
+          StepFrag f;
+          frag_from_smem<Q3>(f, ca, cb, sa, sb, ha, hb, k0);
+          mma_step<Q3>(acc, acc2, f, xcol, k0, colok);
+        }
         const float wa = un.w[2 * t4], wb = un.w[2 * t4 + 1];
         tot[0] = fmaf(wa, acc[0] + acc2[0], tot[0]);
         tot[1] = fmaf(wb, acc[1] + acc2[1], tot[1]);
         tot[2] = fmaf(wa, acc[2] + acc2[2], tot[2]);
         tot[3] = fmaf(wb, acc[3] + acc2[3], tot[3]);
+        // the warp that finishes a piece's last item refills its slot at once
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+          const int nun = min(a.dpu, nu - d * a.dpu);
+          __threadfence_block();
+          last = (atomicAdd(&s_pcnt[d], 1) == nun * nsteps_dn - 1) ? 1 : 0;
+          __threadfence_block();
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last && qd + R < n_total) issue_fill(qd + R);
       }
       float *rw = red + warp * 16 * 8;
       rw[g * 8 + 2 * t4] = tot[0];
@@ -451,29 +724,45 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       __syncthreads();
     }
   }
+
+  // ---------------- no copy may still be writing this CTA's shared memory when it exits
+  cp_async_wait_all();
 }
 
-cudaError_t launch_decode_fused(const uint16_t *x, int T, int H, const float *Wr, const float *bias, int E, int k,
-                                int I, const moe_expert_set &routed, const moe_expert_set *shared,
-                                const float *residual, float *y, float *logits, int32_t *idx, float *w,
-                                uint16_t *hdec, Ctrl *ctrl, cudaStream_t s) {
+cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float eps, int T, int H, const float *Wr,
+                                const float *bias, int E, int k, int I, const moe_expert_set &routed,
+                                const moe_expert_set *shared, const float *residual, float *y, float *logits,
+                                int32_t *idx, float *w, uint16_t *hdec, Ctrl *ctrl, cudaStream_t s) {
   const int hs_cols = T * k + (shared ? T : 0);
-  if (T < 1 || T > kDecodeMaxT || E > 512 || H > 2048 || I > 1024 || hs_cols > kFSlots ||
-      k > 16 ||
-      (size_t)T * E * 4 > (size_t)kFSlots * (I + 4) * 2)
+  if (T < 1 || T > kDecodeMaxT || E > kFMaxE || H > 2048 || I > 1024 || hs_cols > kFSlots || k > 16)
     return cudaErrorNotSupported;
-  const FusedLayout L = fused_layout(T, H, I);
   const bool q3 = routed.gate.qtype == MOE_Q3;
+  const int gu_bytes = (q3 ? 7 : 5) * H;  // 8 gate + 8 up rows: codes, scales (, hi bits)
+  const int dn_bytes = (q3 ? 7 : 5) * I;  // 16 down rows
+  const int slot_bytes = (int)fl_align((size_t)(gu_bytes > dn_bytes ? gu_bytes : dn_bytes), 128);
+  const int dpu = slot_bytes / dn_bytes;
+  const FusedLayout L0 = fused_layout(T, H, E, I, hs_cols, 0, slot_bytes);
+  if (L0.total >= (size_t)kFSmemMax) return cudaErrorNotSupported;
+  int ring = (int)(((size_t)kFSmemMax - L0.total) / slot_bytes);
+  if (ring > kFMaxRing) ring = kFMaxRing;
+  {  // no more slots than one CTA can fill: its gate/up items plus its down pieces at the most units
+    const int G = num_sms(), max_units = T * k + (shared ? 1 : 0);
+    const int need = (max_units * (I / 8) + G - 1) / G + ((H / 16 + G - 1) / G) * ((max_units + dpu - 1) / dpu);
+    if (ring > need) ring = need;
+  }
+  if (ring < 2) return cudaErrorNotSupported;
+  const FusedLayout L = fused_layout(T, H, E, I, hs_cols, ring, slot_bytes);
   const void *fn = q3 ? reinterpret_cast<const void *>(decode_fused_kernel<true>)
                       : reinterpret_cast<const void *>(decode_fused_kernel<false>);
-  cudaError_t e = smem_limit_once_impl(fn, L.total);
+  cudaError_t e = smem_limit_once_impl(fn, kFSmemMax);
   if (e != cudaSuccess) return e;
-  int dev = 0, per_sm = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorNotSupported;
+  int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kFThreads, L.total) != cudaSuccess || per_sm < 1)
     return cudaErrorNotSupported;
   FusedArgs a;
   a.x = x;
+  a.r_norm = r_norm;
+  a.eps = eps;
   a.T = T;
   a.H = H;
   a.E = E;
@@ -491,6 +780,11 @@ cudaError_t launch_decode_fused(const uint16_t *x, int T, int H, const float *Wr
   a.w = w;
   a.hdec = hdec;
   a.ctrl = ctrl;
+  a.ring = ring;
+  a.slot_bytes = slot_bytes;
+  a.gu_bytes = gu_bytes;
+  a.dn_bytes = dn_bytes;
+  a.dpu = dpu;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms());
   cfg.blockDim = dim3(kFThreads);
