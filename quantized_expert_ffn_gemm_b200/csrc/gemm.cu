@@ -35,9 +35,7 @@ namespace moe {
 constexpr int kBK = 64;            // K per pipeline stage (one 128-byte swizzle row of fp16)
 constexpr int kBM = 128;           // weight rows per tile (MMA M)
 constexpr int kBNMax = 192;        // token rows per tile (MMA N upper bound; TMEM: 2 x 192 + A ring)
-constexpr int kBoxRows = 32;       // rows per TMA box of the activation tile
-constexpr int kThreads = 320;      // warp 0 TMA, warp 1 MMA/TMEM, warps 2..9 dequant + epilogue
-constexpr int kDqThreads = 256;
+constexpr int kBoxRows = 64;       // rows per TMA box of the activation tile (fewer, larger requests)
 
 struct GemmArgs {
   const int32_t *offsets;
@@ -69,9 +67,11 @@ __device__ __forceinline__ void record_timeout(Ctrl *c, int where) { set_device_
 // TMEM (512 columns): accumulators at columns 0 and 256 (up to 192 columns each; acc_full:
 // tile's MMAs done, acc_empty: drained), A stages at 192, 224, 448 and 480. The deeper
 // shared-memory ring lets the TMA run far enough ahead to cover HBM latency.
-// MODE_GU: A rows 0-63 are gate rows f0..f0+63 and rows 64-127 the up rows of the same features
-// (one accumulator holds both); the epilogue pairs quadrant 0 with 2 and 1 with 3 through shared
-// memory and writes h = silu(gate) * up. MODE_DN: A rows are 128 rows of W_down.
+// MODE_GU: A row 2i is gate row f0+i and row 2i+1 the up row of the same feature (64 features,
+// one accumulator holds both), so the epilogue pairs adjacent lanes with one shuffle per value
+// and writes h = silu(gate) * up. The TMA still brings the 64 gate rows' codes (smem rows 0-63)
+// and the 64 up rows' codes (rows 64-127); the dequant warps read them interleaved.
+// MODE_DN: A rows are 128 rows of W_down.
 enum { MODE_GU = 0, MODE_DN = 1 };
 
 constexpr int kStagesB = 8;
@@ -83,10 +83,8 @@ struct SmemV2 {
   static constexpr int kB = kBNMax * kBK * 2;   // 24 KB activation tile
   static constexpr int kRaw = kBM * kBK / 4;    // 2 KB packed codes
   static constexpr int kStage = kB + kRaw;      // multiple of 1024 (128B-swizzle atoms)
-  static constexpr int kXch = 2 * 16 * 32 * 4;  // gate/up exchange: 2 pairs x 16 columns x 32 lanes
-  static constexpr int kXchOff = kStagesB * kStage;
-  static constexpr int kBar = kXchOff + kXch;
-  static constexpr int kNumBars = 2 * kStagesB + 2 * kStagesA + 4 + 4;  // + gate/up exchange: full and free per pair
+  static constexpr int kBar = kStagesB * kStage;
+  static constexpr int kNumBars = 2 * kStagesB + 2 * kStagesA + 4;
   static constexpr int kBytes = kBar + kNumBars * 8 + 16;
 };
 
@@ -153,10 +151,7 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
   constexpr int kB0 = 2 * kStagesB + 2 * kStagesA;
   auto acc_full = [&](int b) { return bar0 + 8u * (kB0 + b); };
   auto acc_empty = [&](int b) { return bar0 + 8u * (kB0 + 2 + b); };
-  auto x_full = [&](int pr) { return bar0 + 8u * (kB0 + 4 + pr); };
-  auto x_free = [&](int pr) { return bar0 + 8u * (kB0 + 6 + pr); };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + SL::kBar + SL::kNumBars * 8);
-  float *xch = reinterpret_cast<float *>(gbase + SL::kXchOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -171,8 +166,6 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
     for (int b = 0; b < 2; ++b) {
       mbar_init(acc_full(b), 1);
       mbar_init(acc_empty(b), 4);
-      mbar_init(x_full(b), 1);
-      mbar_init(x_free(b), 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -228,17 +221,35 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
         tc_fence_after();
         const uint32_t idesc = idesc_f16(cur.N);
         const uint32_t d = tmem + (uint32_t)(b * 256);
-        for (int ks = 0; ks < nk; ++ks) {
+        // the next stage's barriers are tested while this stage's MMAs queue up, so a stage whose
+        // operands are already in place costs no wait between the MMA groups
+        {
+          const int g = tl * nk;
+          if (!mbar_wait(full_b(g % kStagesB), (uint32_t)(g / kStagesB) & 1u) ||
+              !mbar_wait(full_a(g % kStagesA), (uint32_t)(g / kStagesA) & 1u)) {
+            record_timeout(ctrl, 23);
+            ok = false;
+          }
+        }
+        for (int ks = 0; ks < nk && ok; ++ks) {
           const int g = tl * nk + ks;
           const int s = g % kStagesB, sa = g % kStagesA;
-          const uint32_t ph = (uint32_t)(g / kStagesB) & 1u, pha = (uint32_t)(g / kStagesA) & 1u;
-          if (!mbar_wait(full_b(s), ph) || !mbar_wait(full_a(sa), pha)) { record_timeout(ctrl, 23); ok = false; break; }
           tc_fence_after();
+          tc_mma_ts(d, tmem + a_col(sa), sw128_desc(sB(s)), idesc, ks != 0 ? 1u : 0u);
+          const bool more = ks + 1 < nk;
+          const int s1 = (g + 1) % kStagesB, sa1 = (g + 1) % kStagesA;
+          const uint32_t ph1 = (uint32_t)((g + 1) / kStagesB) & 1u, pha1 = (uint32_t)((g + 1) / kStagesA) & 1u;
+          const bool rb = more && mbar_test(full_b(s1), ph1);
+          const bool ra = more && mbar_test(full_a(sa1), pha1);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            tc_mma_ts(d, tmem + a_col(sa) + 8u * kk, sw128_desc(sB(s) + kk * 32), idesc, (ks | kk) != 0 ? 1u : 0u);
+          for (int kk = 1; kk < kBK / 16; ++kk)
+            tc_mma_ts(d, tmem + a_col(sa) + 8u * kk, sw128_desc(sB(s) + kk * 32), idesc, 1u);
           tc_commit(empty_b(s));
           tc_commit(empty_a(sa));
+          if (more && ((!rb && !mbar_wait(full_b(s1), ph1)) || (!ra && !mbar_wait(full_a(sa1), pha1)))) {
+            record_timeout(ctrl, 23);
+            ok = false;
+          }
         }
         if (ok) tc_commit(acc_full(b));
         cur = nxt;
@@ -252,7 +263,8 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
     const int qd = warp & 3;
     const int r = 32 * qd + lane, par = (warp - 2) >> 2;
     const uint32_t a_lane = (uint32_t)(32 * qd) << 16;
-    const int mat = (MODE == MODE_GU) ? (r >> 6) : 0;
+    const int mat = (MODE == MODE_GU) ? (r & 1) : 0;
+    const int crow = (MODE == MODE_GU) ? ((r & 1) ? 64 + (r >> 1) : (r >> 1)) : r;  // code row in the stage
     const int total_g = n_my * nk;
     // per-tile pointers to this row's scales (two per stage: one u32) and Q3 hi words (two per stage)
     auto row_ptrs = [&](int tl, const uint32_t *&sp, const uint2 *&hp) {
@@ -261,7 +273,7 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
       const int grp = args.tiles[entry].x;
       const int set = (grp == args.shared_group) ? 1 : 0;
       const int expert = set ? 0 : grp;
-      const int wrow = (MODE == MODE_GU) ? mt * 64 + (r & 63) : mt * kBM + r;
+      const int wrow = (MODE == MODE_GU) ? mt * 64 + (r >> 1) : mt * kBM + r;
       const size_t grow = (size_t)expert * args.M + wrow;
       const uint16_t *sc = set ? (mat ? args.scales[1][1] : args.scales[1][0])
                                : (mat ? args.scales[0][1] : args.scales[0][0]);
@@ -302,7 +314,7 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
         // codes landed; the MMAs that read this A stage last time are complete
         if (!mbar_wait(full_b(s), ph) || !mbar_wait(empty_a(sa), pha ^ 1u)) { record_timeout(ctrl, 24); ok = false; break; }
         tc_fence_after();
-        const uint4 cw = *reinterpret_cast<const uint4 *>(gbase + (sR(s) - base) + r * 16);
+        const uint4 cw = *reinterpret_cast<const uint4 *>(gbase + (sR(s) - base) + crow * 16);
         const __half2 d0 = __half2half2(__ushort_as_half((uint16_t)(sc[j] & 0xffffu)));
         const __half2 d1 = __half2half2(__ushort_as_half((uint16_t)(sc[j] >> 16)));
         uint32_t p[32];
@@ -330,7 +342,6 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
     // ------------------------------------------------ epilogue warps 10..13 (lane quadrants 2, 3, 0, 1)
     const int q = warp & 3;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    uint32_t xphase = 0;  // gate/up exchange rounds of this warp's pair
     bool ok = true;
     TileInfo cur = get_tile(args, blockIdx.x, n_mtiles);
     for (int tl = 0; tl < n_my && ok; ++tl) {
@@ -345,55 +356,38 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
       const uint32_t taddr = tmem + lane_base + (uint32_t)(b * 256);
       if (MODE == MODE_DN) {
         const int f = cur.mt * kBM + 32 * q + lane;
+        uint16_t *op = args.out + (size_t)cur.row_base * args.ldo + f;
         for (int c0 = 0; c0 < cur.N; c0 += 16) {
           uint32_t v[16];
           tmem_ld16(taddr + c0, v);
-          tmem_ld_wait();
+          tmem_ld_wait16(v);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int n = c0 + j;
-            if (n < cur.n_valid)
-              args.out[(size_t)(cur.row_base + n) * args.ldo + f] = __half_as_ushort(__float2half_rn(__uint_as_float(v[j])));
+            if (n < cur.n_valid) op[(size_t)n * args.ldo] = __half_as_ushort(__float2half_rn(__uint_as_float(v[j])));
           }
         }
       } else {
-        // gate quadrants 0/1 hand their values to up quadrants 2/3 (pairs 0-2 and 1-3) through a
-        // 16-column shared buffer per pair, handed back and forth with two mbarriers (bounded waits)
-        const int pair = q & 1;
-        float *xb = xch + pair * 16 * 32;
-        const int f = cur.mt * 64 + 32 * pair + lane;
-        for (int c0 = 0; c0 < cur.N && ok; c0 += 16, ++xphase) {
+        // A rows alternate gate / up of the same feature, so lanes 2i and 2i+1 hold the gate and
+        // up accumulators of feature f: per 16 columns each lane sends its partner the 8 values
+        // the partner needs (one shuffle each); the gate lane finishes columns 0-7, the up lane 8-15
+        const int f = cur.mt * 64 + 16 * q + (lane >> 1);
+        const bool up_lane = lane & 1;
+        uint16_t *op = args.out + (size_t)cur.row_base * args.ldo + f;
+        for (int c0 = 0; c0 < cur.N; c0 += 16) {
           uint32_t v[16];
           tmem_ld16(taddr + c0, v);
-          tmem_ld_wait();
-          if (q < 2) {
-            ok = __all_sync(0xffffffffu, mbar_wait(x_free(pair), (xphase & 1u) ^ 1u));
-            if (!ok) break;
+          tmem_ld_wait16(v);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) xb[j * 32 + lane] = __uint_as_float(v[j]);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(x_full(pair));
-          } else {
-            ok = __all_sync(0xffffffffu, mbar_wait(x_full(pair), xphase & 1u));
-            if (!ok) break;
-            float gv[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) gv[j] = xb[j * 32 + lane];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(x_free(pair));
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int n = c0 + j;
-              const float uv = __uint_as_float(v[j]);
-              const float hv = gv[j] / (1.0f + expf(-gv[j])) * uv;
-              if (n < cur.n_valid)
-                args.out[(size_t)(cur.row_base + n) * args.ldo + f] = __half_as_ushort(__float2half_rn(hv));
-            }
+          for (int j = 0; j < 8; ++j) {
+            const float mine_lo = __uint_as_float(v[j]), mine_hi = __uint_as_float(v[j + 8]);
+            const float other = __shfl_xor_sync(0xffffffffu, up_lane ? mine_lo : mine_hi, 1);
+            const float gv = up_lane ? other : mine_lo;  // gate value of column c0 + j (+8 on the up lane)
+            const float uv = up_lane ? mine_hi : other;
+            const int n = c0 + j + (up_lane ? 8 : 0);
+            const float hv = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+            if (n < cur.n_valid) op[(size_t)n * args.ldo] = __half_as_ushort(__float2half_rn(hv));
           }
-        }
-        if (!ok) {
-          if (lane == 0) record_timeout(ctrl, 26);
-          break;
         }
       }
       tc_fence_before();
