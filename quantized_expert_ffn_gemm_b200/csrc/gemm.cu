@@ -32,7 +32,8 @@
 
 namespace moe {
 
-constexpr int kBK = 64;            // K per pipeline stage (one 128-byte swizzle row of fp16)
+constexpr int kBK = 128;           // K per pipeline stage: two 64-wide 128-byte swizzle sub-tiles
+constexpr int kSubK = 64;          // K of one swizzle sub-tile (128 bytes of fp16 per row)
 constexpr int kBM = 128;           // weight rows per tile (MMA M)
 constexpr int kBNMax = 192;        // token rows per tile (MMA N upper bound; TMEM: 2 x 192 + A ring)
 constexpr int kBoxRows = 64;       // rows per TMA box of the activation tile (fewer, larger requests)
@@ -61,12 +62,14 @@ __device__ __forceinline__ void record_timeout(Ctrl *c, int where) { set_device_
 //   warp 1      TMEM owner and single-thread MMA issuer
 //   warps 2-9   dequant: code plane + per-block scales (+ Q3 hi bits) -> fp16 A tile
 //   warps 10-13 epilogue: TMEM -> registers -> global, one lane quadrant each
-// Two rings. Shared memory: kStagesB stages of activation tile + code plane (full_b: TMA landed,
-// empty_b: the stage's MMAs are done). TMEM: kStagesA stages of the dequantized A tile, 128
-// lanes x 32 columns (full_a: written by the dequant warps, empty_a: the stage's MMAs are done).
-// TMEM (512 columns): accumulators at columns 0 and 256 (up to 192 columns each; acc_full:
-// tile's MMAs done, acc_empty: drained), A stages at 192, 224, 448 and 480. The deeper
-// shared-memory ring lets the TMA run far enough ahead to cover HBM latency.
+// A stage covers K = 128 (eight MMAs, one commit: every tcgen05.mma costs ~100 cycles of issue
+// at these shapes, so the per-stage waits and commits are spread over eight of them). Two
+// rings. Shared memory: kStagesB stages of activation tile (two 64-wide swizzled sub-tiles) +
+// code plane (full_b: TMA landed, empty_b: the stage's MMAs are done). TMEM: kStagesA stages of
+// the dequantized A tile, 128 lanes x 64 columns (full_a: written by the dequant warps; a stage
+// is reused once empty_b of the stage kStagesA back has completed). TMEM (512 columns):
+// accumulators at columns 0 and 256 (up to 192 columns each; acc_full: tile's MMAs done,
+// acc_empty: drained), A stages at 192 and 448.
 // MODE_GU: A row 2i is gate row f0+i and row 2i+1 the up row of the same feature (64 features,
 // one accumulator holds both), so the epilogue pairs adjacent lanes with one shuffle per value
 // and writes h = silu(gate) * up. The TMA still brings the 64 gate rows' codes (smem rows 0-63)
@@ -74,25 +77,26 @@ __device__ __forceinline__ void record_timeout(Ctrl *c, int where) { set_device_
 // MODE_DN: A rows are 128 rows of W_down.
 enum { MODE_GU = 0, MODE_DN = 1 };
 
-constexpr int kStagesB = 8;
-constexpr int kStagesA = 4;
+constexpr int kStagesB = 4;
+constexpr int kStagesA = 2;
 constexpr int kThreadsV2 = 448;
 constexpr int kEpiWarp0 = 10;
 
 struct SmemV2 {
-  static constexpr int kB = kBNMax * kBK * 2;   // 24 KB activation tile
-  static constexpr int kRaw = kBM * kBK / 4;    // 2 KB packed codes
-  static constexpr int kStage = kB + kRaw;      // multiple of 1024 (128B-swizzle atoms)
+  static constexpr int kSub = kBNMax * kSubK * 2;  // 24 KB: one 64-wide sub-tile of the activation rows
+  static constexpr int kB = 2 * kSub;              // 48 KB activation tile (K = 128)
+  static constexpr int kRaw = kBM * kBK / 4;       // 4 KB packed codes
+  static constexpr int kStage = kB + kRaw;         // multiple of 1024 (128B-swizzle atoms)
   static constexpr int kBar = kStagesB * kStage;
-  static constexpr int kNumBars = 2 * kStagesB + 2 * kStagesA + 4;
+  static constexpr int kNumBars = 2 * kStagesB + kStagesA + 4;
   static constexpr int kBytes = kBar + kNumBars * 8 + 16;
 };
 
-static_assert(SmemV2::kStage % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
-static_assert(kStagesA == 4, "TMEM holds four A stages");
+static_assert(SmemV2::kStage % 1024 == 0 && SmemV2::kSub % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+static_assert(kStagesA == 2, "TMEM holds two A stages");
 
-// TMEM column of A stage s
-__device__ __forceinline__ uint32_t a_col(int s) { return 192u + 32u * (uint32_t)(s & 1) + 256u * (uint32_t)(s >> 1); }
+// TMEM column of A stage s (64 columns: 128 K of fp16 pairs)
+__device__ __forceinline__ uint32_t a_col(int s) { return 192u + 256u * (uint32_t)s; }
 
 struct TileInfo {
   int expert, set, row_base, n_valid, N, mt;
@@ -147,8 +151,7 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
   auto full_b = [&](int s) { return bar0 + 8u * s; };
   auto empty_b = [&](int s) { return bar0 + 8u * (kStagesB + s); };
   auto full_a = [&](int s) { return bar0 + 8u * (2 * kStagesB + s); };
-  auto empty_a = [&](int s) { return bar0 + 8u * (2 * kStagesB + kStagesA + s); };
-  constexpr int kB0 = 2 * kStagesB + 2 * kStagesA;
+  constexpr int kB0 = 2 * kStagesB + kStagesA;
   auto acc_full = [&](int b) { return bar0 + 8u * (kB0 + b); };
   auto acc_empty = [&](int b) { return bar0 + 8u * (kB0 + 2 + b); };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + SL::kBar + SL::kNumBars * 8);
@@ -159,10 +162,7 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
       mbar_init(full_b(s), 1);
       mbar_init(empty_b(s), 1);
     }
-    for (int s = 0; s < kStagesA; ++s) {
-      mbar_init(full_a(s), 128);  // the four dequant warps of the stage's parity
-      mbar_init(empty_a(s), 1);
-    }
+    for (int s = 0; s < kStagesA; ++s) mbar_init(full_a(s), 256);  // all eight dequant warps
     for (int b = 0; b < 2; ++b) {
       mbar_init(acc_full(b), 1);
       mbar_init(acc_empty(b), 4);
@@ -187,7 +187,7 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
       for (int tl = 0; tl < n_my && ok; ++tl) {
         const TileInfo nxt = (tl + 1 < n_my) ? get_tile(args, blockIdx.x + (tl + 1) * G, n_mtiles) : cur;
         const int nbox = (cur.N + kBoxRows - 1) / kBoxRows;
-        const uint32_t tx = (uint32_t)nbox * kBoxRows * kBK * 2 + SL::kRaw;
+        const uint32_t tx = (uint32_t)nbox * kBoxRows * kBK * 2 + SL::kRaw;  // both sub-tiles + codes
         const CUtensorMap *mc0 = cur.set ? &tm_c0s : &tm_c0r;
         const CUtensorMap *mc1 = cur.set ? &tm_c1s : &tm_c1r;
         const int wrow = (MODE == MODE_GU) ? cur.expert * args.M + cur.mt * 64 : cur.expert * args.M + cur.mt * kBM;
@@ -197,8 +197,10 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
           const uint32_t ph = (uint32_t)(g / kStagesB) & 1u;
           if (!mbar_wait(empty_b(s), ph ^ 1u)) { record_timeout(ctrl, 21); ok = false; break; }
           mbar_arrive_expect_tx(full_b(s), tx);
-          for (int b = 0; b < nbox; ++b)
-            tma_load_2d(sB(s) + b * kBoxRows * kBK * 2, &tm_b, ks * kBK, cur.row_base + b * kBoxRows, full_b(s));
+          for (int h = 0; h < 2; ++h)
+            for (int b = 0; b < nbox; ++b)
+              tma_load_2d(sB(s) + h * SL::kSub + b * kBoxRows * kSubK * 2, &tm_b, ks * kBK + h * kSubK,
+                          cur.row_base + b * kBoxRows, full_b(s));
           if (MODE == MODE_GU) {  // gate rows -> A rows 0..63, up rows -> A rows 64..127
             tma_load_2d(sR(s), mc0, ks * (kBK / 4), wrow, full_b(s));
             tma_load_2d(sR(s) + 64 * (kBK / 4), mc1, ks * (kBK / 4), wrow, full_b(s));
@@ -242,10 +244,9 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
           const bool rb = more && mbar_test(full_b(s1), ph1);
           const bool ra = more && mbar_test(full_a(sa1), pha1);
 #pragma unroll
-          for (int kk = 1; kk < kBK / 16; ++kk)
-            tc_mma_ts(d, tmem + a_col(sa) + 8u * kk, sw128_desc(sB(s) + kk * 32), idesc, 1u);
-          tc_commit(empty_b(s));
-          tc_commit(empty_a(sa));
+          for (int kk = 1; kk < kBK / 16; ++kk)  // sub-tile kk / 4, 32 bytes per 16 K inside it
+            tc_mma_ts(d, tmem + a_col(sa) + 8u * kk, sw128_desc(sB(s) + (kk >> 2) * SL::kSub + (kk & 3) * 32), idesc, 1u);
+          tc_commit(empty_b(s));  // frees the smem stage, and (kStagesA stages on) the TMEM A stage
           if (more && ((!rb && !mbar_wait(full_b(s1), ph1)) || (!ra && !mbar_wait(full_a(sa1), pha1)))) {
             record_timeout(ctrl, 23);
             ok = false;
@@ -258,15 +259,16 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
   } else if (warp < kEpiWarp0) {
     // ------------------------------------------------ dequant warps
     // warp w writes TMEM lanes 32*(w%4)..+31 (the lanes a warp may access): A row r = that lane.
-    // Warps 2-5 dequantize the even stages and warps 6-9 the odd ones, a thread a whole 64-weight
-    // row slice (both 32-weight blocks) of its stage, so two stages are in flight at once.
+    // Warps 2-5 take K 0..63 of every stage and warps 6-9 K 64..127, a thread one 64-weight row
+    // slice (two 32-weight blocks) per stage.
     const int qd = warp & 3;
-    const int r = 32 * qd + lane, par = (warp - 2) >> 2;
+    const int r = 32 * qd + lane, hh = (warp - 2) >> 2;
     const uint32_t a_lane = (uint32_t)(32 * qd) << 16;
     const int mat = (MODE == MODE_GU) ? (r & 1) : 0;
     const int crow = (MODE == MODE_GU) ? ((r & 1) ? 64 + (r >> 1) : (r >> 1)) : r;  // code row in the stage
     const int total_g = n_my * nk;
-    // per-tile pointers to this row's scales (two per stage: one u32) and Q3 hi words (two per stage)
+    // per-tile pointers to this row's scales (two per 64-weight slice: one u32) and Q3 hi words
+    // (two per slice: one uint2); slice 2 ks + hh of the row is this thread's share of stage ks
     auto row_ptrs = [&](int tl, const uint32_t *&sp, const uint2 *&hp) {
       const int ti = blockIdx.x + tl * G;
       const int entry = ti / n_mtiles, mt = ti - entry * n_mtiles;
@@ -279,11 +281,10 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
                                : (mat ? args.scales[0][1] : args.scales[0][0]);
       const uint8_t *hb = set ? (mat ? args.hibits[1][1] : args.hibits[1][0])
                               : (mat ? args.hibits[0][1] : args.hibits[0][0]);
-      sp = reinterpret_cast<const uint32_t *>(sc + grow * (K / 32));
-      hp = args.q3 ? reinterpret_cast<const uint2 *>(hb + grow * (K / 8)) : nullptr;
+      sp = reinterpret_cast<const uint32_t *>(sc + grow * (K / 32)) + hh;
+      hp = args.q3 ? reinterpret_cast<const uint2 *>(hb + grow * (K / 8)) + hh : nullptr;
     };
-    // scales (and Q3 hi words) are fetched four of this warp's stages (eight stages) ahead into a
-    // 4-entry register ring
+    // scales (and Q3 hi words) are fetched four stages ahead into a 4-entry register ring
     int pf_tl = 0;
     const uint32_t *pf_sp;
     const uint2 *pf_hp;
@@ -291,8 +292,8 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
     auto fetch = [&](int g, uint32_t &scv, uint2 &hv) {
       const int tl = g / nk;
       if (tl != pf_tl) { pf_tl = tl; row_ptrs(tl, pf_sp, pf_hp); }
-      scv = __ldg(pf_sp + g % nk);
-      if (args.q3) hv = __ldg(pf_hp + g % nk);
+      scv = __ldg(pf_sp + 2 * (g % nk));
+      if (args.q3) hv = __ldg(pf_hp + 2 * (g % nk));
     };
     uint32_t sc[4];
     uint2 hw[4];
@@ -300,21 +301,26 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
     for (int j = 0; j < 4; ++j) {
       sc[j] = 0u;
       hw[j] = make_uint2(0u, 0u);
-      const int g = par + 2 * j;
-      if (g < total_g) fetch(g, sc[j], hw[j]);
+      if (j < total_g) fetch(j, sc[j], hw[j]);
     }
     bool ok = true;
-    for (int i0 = 0; par + 2 * i0 < total_g && ok; i0 += 4) {
+    for (int g0 = 0; g0 < total_g && ok; g0 += 4) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int g = par + 2 * (i0 + j);
+        const int g = g0 + j;
         if (g >= total_g) break;
         const int s = g % kStagesB, sa = g % kStagesA;
-        const uint32_t ph = (uint32_t)(g / kStagesB) & 1u, pha = (uint32_t)(g / kStagesA) & 1u;
-        // codes landed; the MMAs that read this A stage last time are complete
-        if (!mbar_wait(full_b(s), ph) || !mbar_wait(empty_a(sa), pha ^ 1u)) { record_timeout(ctrl, 24); ok = false; break; }
+        const uint32_t ph = (uint32_t)(g / kStagesB) & 1u;
+        // codes landed; and the MMAs that last read this A stage (stage g - kStagesA) are complete
+        if (!mbar_wait(full_b(s), ph)) { record_timeout(ctrl, 24); ok = false; break; }
+        if (g >= kStagesA &&
+            !mbar_wait(empty_b((g - kStagesA) % kStagesB), (uint32_t)((g - kStagesA) / kStagesB) & 1u)) {
+          record_timeout(ctrl, 24);
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint4 cw = *reinterpret_cast<const uint4 *>(gbase + (sR(s) - base) + crow * 16);
+        const uint4 cw = *reinterpret_cast<const uint4 *>(gbase + (sR(s) - base) + crow * (kBK / 4) + hh * 16);
         const __half2 d0 = __half2half2(__ushort_as_half((uint16_t)(sc[j] & 0xffffu)));
         const __half2 d1 = __half2half2(__ushort_as_half((uint16_t)(sc[j] >> 16)));
         uint32_t p[32];
@@ -329,12 +335,13 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
           dq2_word(cw.z, d1, p + 16);
           dq2_word(cw.w, d1, p + 24);
         }
-        tmem_st16(tmem + a_lane + a_col(sa), p);
-        tmem_st16(tmem + a_lane + a_col(sa) + 16u, p + 16);
+        const uint32_t ta = tmem + a_lane + a_col(sa) + 32u * hh;
+        tmem_st16(ta, p);
+        tmem_st16(ta + 16u, p + 16);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(full_a(sa));
-        const int gp = g + 8;  // refill this ring slot
+        const int gp = g + 4;  // refill this ring slot
         if (gp < total_g) fetch(gp, sc[j], hw[j]);
       }
     }
@@ -526,9 +533,9 @@ cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, i
   if (e != cudaSuccess) return e;
 
   CUtensorMap tx, th, cg, cu, cd, sg, su, sd;
-  bool ok = encode_tensor_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x_perm, H, n_rows, kBK, kBoxRows,
+  bool ok = encode_tensor_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x_perm, H, n_rows, kSubK, kBoxRows,
                                  CU_TENSOR_MAP_SWIZZLE_128B) &&
-            encode_tensor_map_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h_perm, I, n_rows, kBK, kBoxRows,
+            encode_tensor_map_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h_perm, I, n_rows, kSubK, kBoxRows,
                                  CU_TENSOR_MAP_SWIZZLE_128B) &&
             make_code_map(&cg, routed.gate, 64) && make_code_map(&cu, routed.up, 64) &&
             make_code_map(&cd, routed.down, kBM) && make_code_map(&sg, sh.gate, 64) && make_code_map(&su, sh.up, 64) &&
