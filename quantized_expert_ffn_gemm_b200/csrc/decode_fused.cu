@@ -108,7 +108,9 @@ __host__ __device__ inline FusedLayout fused_layout(int T, int H, int E, int I, 
 // all CTAs are co-resident (cooperative launch). Barrier j of a launch completes when the arrival
 // counter reaches base + j * nblocks. Every CTA arrives, even after an earlier failure, so the
 // count stays whole; it waits only when `wait` is set. Returns false when the wait gave up (or
-// was not made). Called by every thread of the CTA.
+// was not made). Called by every thread of the CTA: the CTA barrier orders the CTA's writes
+// before thread 0's fence and release-add; thread 0's acquire loads and the closing CTA barrier
+// order the CTA's later reads after every other CTA's arrival.
 __device__ bool grid_barrier(Ctrl *c, unsigned long long target, int where, bool wait) {
   __shared__ int s_ok;
   __syncthreads();
@@ -348,24 +350,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       d[1] = make_uint2(o[2], o[3]);
     }
   }
-  {  // into L2 while the router runs: the shared expert's rows and the router bias
-    const int nthr = gridDim.x * kFThreads, first = blockIdx.x * kFThreads + tid;
-    if (a.has_shared) {
-      const size_t cb = (size_t)I * H / 4, sb = (size_t)I * H / 32 * 2;
-      prefetch_range(a.shared.gate.codes, cb, first, nthr);
-      prefetch_range(a.shared.up.codes, cb, first, nthr);
-      prefetch_range(a.shared.down.codes, cb, first, nthr);
-      prefetch_range(a.shared.gate.scales, sb, first, nthr);
-      prefetch_range(a.shared.up.scales, sb, first, nthr);
-      prefetch_range(a.shared.down.scales, sb, first, nthr);
-      if (Q3) {
-        prefetch_range(a.shared.gate.hibits, cb / 2, first, nthr);
-        prefetch_range(a.shared.up.hibits, cb / 2, first, nthr);
-        prefetch_range(a.shared.down.hibits, cb / 2, first, nthr);
-      }
-    }
-    if (a.bias) prefetch_range(a.bias, (size_t)E * 4, tid, kFThreads);
-  }
+  if (a.bias) prefetch_range(a.bias, (size_t)E * 4, tid, kFThreads);
   __syncthreads();
 
   // ---------------- P1: router logits, four warps per expert (each a quarter of H), fp32
@@ -413,14 +398,15 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       __syncthreads();
     }
   }
-  __threadfence();
   bool ok = grid_barrier(ctrl, s_base + nblk, 31, true);
 
   // ---------------- P1b: top-k and unit list, computed identically by every CTA
   if (ok) {
-    // every 32-expert chunk of every token is sorted by one warp straight from the logits (top 16
-    // kept); then one warp per token merges the chunks' lists: lane c holds list c in registers,
-    // each round the warp takes the best head (max key, then lowest index) and that lane shifts
+    // every 32-expert chunk of every token is sorted by one warp straight from the logits
+    // (64-bit codes: order-preserving key, then ~index, so the lower index wins ties; top 16
+    // kept); then one warp per token merges the chunks' lists: lane c holds list c in
+    // registers, each round the warp takes the best head (max key, then lowest index) and that
+    // lane shifts its list
     const int nch = (E + 31) / 32;  // <= 16
     for (int task = warp; task < T * nch; task += kFWarps) {
       const int t = task / nch, c = task % nch, e = c * 32 + lane;
@@ -428,6 +414,23 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       if (e < E) v = topk_code(__ldcg(a.logits + (size_t)t * E + e) + (a.bias ? __ldg(a.bias + e) : 0.f), e);
       v = warp_sort32_desc(v);
       if (lane < 16) plist[(size_t)task * 16 + lane] = v;
+    }
+    {  // into L2 while the top-k runs: the shared expert's rows (always selected)
+      const int nthr = gridDim.x * kFThreads, first = blockIdx.x * kFThreads + tid;
+      if (a.has_shared) {
+        const size_t cb = (size_t)I * H / 4, sb = (size_t)I * H / 32 * 2;
+        prefetch_range(a.shared.gate.codes, cb, first, nthr);
+        prefetch_range(a.shared.up.codes, cb, first, nthr);
+        prefetch_range(a.shared.down.codes, cb, first, nthr);
+        prefetch_range(a.shared.gate.scales, sb, first, nthr);
+        prefetch_range(a.shared.up.scales, sb, first, nthr);
+        prefetch_range(a.shared.down.scales, sb, first, nthr);
+        if (Q3) {
+          prefetch_range(a.shared.gate.hibits, cb / 2, first, nthr);
+          prefetch_range(a.shared.up.hibits, cb / 2, first, nthr);
+          prefetch_range(a.shared.down.hibits, cb / 2, first, nthr);
+        }
+      }
     }
     if (T > 1)
       for (int e = tid; e < E; e += kFThreads) s_firstof[e] = 0x7fffffff;
@@ -551,7 +554,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   const int npieces = (nu + a.dpu - 1) / a.dpu;  // down slots per row block
   const int n_total = n_mine + n_rb * npieces;
   const int nsteps_gu = (H + kStepK - 1) / kStepK;  // <= 8
-  const int nsteps_dn = (I + kStepK - 1) / kStepK;
+  const int nhalf_dn = (I + kStepK / 2 - 1) / (kStepK / 2);  // down items are half steps (128 wide)
 
   // ---------------- fills: fill q of this CTA (gate/up items, then down pieces) goes to slot
   // q % R; it is issued by one whole warp (cp.async, 16 bytes per lane per instruction), whose
@@ -634,14 +637,13 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       }
     }
   }
-  __threadfence();
   ok = grid_barrier(ctrl, s_base + 2 * (unsigned long long)nblk, 32, ok) && ok;
 
   // ---------------- P3: down projection + weighted combine (+ residual) for 16 output features per CTA
   if (ok) {
     const int nslots = s_slot[nu];
     const int xstride = I + 4;
-    const int n_items = nu * nsteps_dn;
+    const int n_items = nu * nhalf_dn;
     const int dn = a.dn_bytes;
     for (int rbl = 0; rbl < n_rb; ++rbl) {
       const int r0 = ((int)blockIdx.x + rbl * G) * 16;
@@ -671,11 +673,11 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       __syncthreads();
       float tot[4] = {0.f, 0.f, 0.f, 0.f};
       for (int it = warp; it < n_items; it += kFWarps) {
-        const int u = it / nsteps_dn, st = it % nsteps_dn;
+        const int u = it / nhalf_dn, hsi = it % nhalf_dn;
         const int d = u / a.dpu, qd = qb + d, s = qd % R;
         const bool have = wait_bar(full(s), (uint32_t)(qd / R) & 1u, 43);
         const DecUnit &un = su[u];
-        const int k0 = st * kStepK + 64 * t4;
+        const int k0 = hsi * (kStepK / 2) + 32 * t4;
         const bool kok = k0 < I;
         const bool colok = ((un.mask >> g) & 1) && kok;
         const int slot = s_slot[u] + __popc(un.mask & ((1u << g) - 1u));
@@ -687,9 +689,16 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
           const uint16_t *sa = reinterpret_cast<const uint16_t *>(pc + 4 * I) + (size_t)g * (I / 32);
           const uint16_t *sb = reinterpret_cast<const uint16_t *>(pc + 4 * I) + (size_t)(g + 8) * (I / 32);
           const uint8_t *ha = pc + 5 * I + (size_t)g * (I / 8), *hb = pc + 5 * I + (size_t)(g + 8) * (I / 8);
-          StepFrag f;
-          frag_from_smem<Q3>(f, ca, cb, sa, sb, ha, hb, k0);
-          mma_step<Q3>(acc, acc2, f, xcol, k0, colok);
+          HalfFrag f;
+          f.w0 = *reinterpret_cast<const uint2 *>(ca + k0 / 4);
+          f.w1 = *reinterpret_cast<const uint2 *>(cb + k0 / 4);
+          f.d0 = sa[k0 / 32];
+          f.d1 = sb[k0 / 32];
+          if (Q3) {
+            f.h0 = *reinterpret_cast<const uint32_t *>(ha + k0 / 8);
+            f.h1 = *reinterpret_cast<const uint32_t *>(hb + k0 / 8);
+          }
+          mma_half_step<Q3>(acc, acc2, f, xcol, k0, colok);
         }
         const float wa = un.w[2 * t4], wb = un.w[2 * t4 + 1];
         tot[0] = fmaf(wa, acc[0] + acc2[0], tot[0]);
@@ -702,7 +711,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
         if (lane == 0) {
           const int nun = min(a.dpu, nu - d * a.dpu);
           __threadfence_block();
-          last = (atomicAdd(&s_pcnt[d], 1) == nun * nsteps_dn - 1) ? 1 : 0;
+          last = (atomicAdd(&s_pcnt[d], 1) == nun * nhalf_dn - 1) ? 1 : 0;
           __threadfence_block();
         }
         last = __shfl_sync(0xffffffffu, last, 0);

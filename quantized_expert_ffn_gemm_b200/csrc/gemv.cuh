@@ -125,6 +125,46 @@ __device__ __forceinline__ void mma_step(float acc[4], float acc2[4], const Step
   }
 }
 
+// Half of a step: a 16-row x 128-wide K slice, lane (g, t) holding the 32-weight block
+// kbase..kbase+31 (kbase = slice start + 32 t) of rows g and g+8: two code words per row, one
+// scale per row, and (Q3) one hi word per row. Same pair decoder and MMA-K order as mma_step.
+struct HalfFrag {
+  uint2 w0, w1;
+  uint16_t d0, d1;
+  uint32_t h0, h1;
+};
+
+template <bool Q3>
+__device__ __forceinline__ void mma_half_step(float acc[4], float acc2[4], const HalfFrag &f, const __half *xcol,
+                                              int kbase, bool bok) {
+  const uint32_t wr0[2] = {f.w0.x, f.w0.y};
+  const uint32_t wr1[2] = {f.w1.x, f.w1.y};
+  const __half2 dd0 = __half2half2(__ushort_as_half(f.d0));
+  const __half2 dd1 = __half2half2(__ushort_as_half(f.d1));
+#pragma unroll
+  for (int wq = 0; wq < 2; ++wq) {
+    uint32_t p0[8], p1[8];
+    if (Q3) {
+      dq3_word(wr0[wq], f.h0, wq, dd0, p0);
+      dq3_word(wr1[wq], f.h1, wq, dd1, p1);
+    } else {
+      dq2_word(wr0[wq], dd0, p0);
+      dq2_word(wr1[wq], dd1, p1);
+    }
+#pragma unroll
+    for (int mm = 0; mm < 4; ++mm) {
+      const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
+      uint32_t b0 = 0, b1 = 0;
+      if (bok) {
+        const uint2 bv = *reinterpret_cast<const uint2 *>(xcol + xs_pos(kbase + 16 * wq + 4 * mm));
+        b0 = bv.x;
+        b1 = bv.y;
+      }
+      mma16816((mm & 1) ? acc2 : acc, a, b0, b1);
+    }
+  }
+}
+
 // acc += W[r0..r0+15, steps s0..s0+NS-1] * X^T; all of the batch's loads are issued first
 template <bool Q3, int NS>
 __device__ __forceinline__ void rows16_batch(const MatView &m, int r0, int s0, int nsteps, const __half *xcol,
