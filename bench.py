@@ -60,6 +60,30 @@ def workload_shape(name: str) -> synth.LayerShape:
     return synth.WORKLOADS[wl["shape"]]
 
 
+# DRAM bytes (read + write) per launch of the dominant kernels, from the committed ncu captures
+# (profiles/*.md), valid only for the kernel source they were taken on: the file's sha256 is
+# checked at run time and the figure is dropped (traffic = null) once the source has changed.
+TRAFFIC = {
+    # kernel: (source files, sha256 of their concatenation at capture time, bytes per launch, profile)
+}
+
+
+def traffic_for(kernel: str):
+    import hashlib
+    ent = TRAFFIC.get(kernel)
+    if ent is None:
+        return None
+    srcs, sha, nbytes, _ = ent
+    h = hashlib.sha256()
+    try:
+        for src in srcs:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+    except OSError:
+        return None
+    return nbytes if h.hexdigest() == sha else None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -303,7 +327,7 @@ def run_ours(args, world, rank, local):
         d_ms, d_n = kt[dom]
         achieved = algo / (d_ms / d_n / 1e3) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"], "unit": "GB/s",
-                "frac": round(achieved / pk["hbm"], 4), "traffic": None, "peak_source": pk["src"],
+                "frac": round(achieved / pk["hbm"], 4), "traffic": traffic_for(dom), "peak_source": pk["src"],
                 "algorithmic_bytes_per_launch": int(algo), "avg_launch_us": round(d_ms / d_n * 1e3, 3)}
         layer_bytes = units_avg * (gu_b + dn_b) + E * H * 4 + T * H * 2 + T * H * 4
         layer_gbs = layer_bytes / (ms_max / K / lps / 1e3) / 1e9
@@ -317,7 +341,7 @@ def run_ours(args, world, rank, local):
         flops = 2.0 * 2 * rows * H * I
         achieved = flops / (d_ms / d_n / 1e3) / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": pk["tc_sus"],
-                "unit": "TFLOP/s", "frac": round(achieved / pk["tc_sus"], 4), "traffic": None,
+                "unit": "TFLOP/s", "frac": round(achieved / pk["tc_sus"], 4), "traffic": traffic_for(dom),
                 "peak_source": pk["src"] + " sustained bf16 (fp16 MMA runs at the bf16 rate)",
                 "algorithmic_flops_per_launch": flops, "avg_launch_us": round(d_ms / d_n * 1e3, 1)}
         layer_flops = 2.0 * 3 * rows * H * I + 2.0 * T * E * H

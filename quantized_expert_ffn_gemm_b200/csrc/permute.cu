@@ -41,14 +41,31 @@ perm_scan_kernel(int32_t *__restrict__ hist, int nchunks, int E, int P, int T, i
   extern __shared__ int32_t s_cnt[];  // [E] totals, then exclusive offsets
   __shared__ int32_t s_warp[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-  // pass 1: per-expert totals
-  for (int e = warp; e < E; e += nw) {
-    const int32_t *h = hist + (size_t)e * nchunks;
-    int s = 0;
-    for (int c = lane; c < nchunks; c += 32) s += h[c];
+  // pass 1: per-expert totals, four experts per warp iteration so their loads are in flight together
+  for (int e0 = warp; e0 < E; e0 += 4 * nw) {
+    int sum[4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) s_cnt[e] = s;
+    for (int u = 0; u < 4; ++u) {
+      const int e = e0 + u * nw;
+      sum[u] = 0;
+      if (e < E) {
+        const int32_t *h = hist + (size_t)e * nchunks;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int c = lane + 32 * i;
+          if (c < nchunks) sum[u] += h[c];
+        }
+        for (int c = lane + 128; c < nchunks; c += 32) sum[u] += h[c];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      int v = sum[u];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      const int e = e0 + u * nw;
+      if (lane == 0 && e < E) s_cnt[e] = v;
+    }
   }
   __syncthreads();
   // exclusive scan of the E totals (contiguous runs per thread, then a block scan of the runs)
@@ -88,21 +105,30 @@ perm_scan_kernel(int32_t *__restrict__ hist, int nchunks, int E, int P, int T, i
     }
   }
   __syncthreads();
-  // pass 2: first row of every (expert, chunk): the expert's offset + the exclusive prefix over chunks
+  // pass 2: first row of every (expert, chunk): the expert's offset + the exclusive prefix over
+  // chunks (the chunk counts of up to 128 chunks are loaded before any is scanned)
   for (int e = warp; e < E; e += nw) {
     int32_t *h = hist + (size_t)e * nchunks;
     int run = s_cnt[e];
-    for (int c0 = 0; c0 < nchunks; c0 += 32) {
-      const int c = c0 + lane;
-      const int x = (c < nchunks) ? h[c] : 0;
-      int incl = x;
+    for (int c0 = 0; c0 < nchunks; c0 += 128) {
+      int xv[4];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
+      for (int i = 0; i < 4; ++i) {
+        const int c = c0 + 32 * i + lane;
+        xv[i] = (c < nchunks) ? h[c] : 0;
       }
-      if (c < nchunks) h[c] = run + incl - x;
-      run += __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = c0 + 32 * i + lane;
+        int incl = xv[i];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int n = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += n;
+        }
+        if (c < nchunks) h[c] = run + incl - xv[i];
+        run += __shfl_sync(0xffffffffu, incl, 31);
+      }
     }
   }
   if (tid == 0) {
@@ -123,9 +149,18 @@ perm_scatter_kernel(const int32_t *__restrict__ idx, int P, int k, int E, const 
   for (int e = lane; e < E; e += 32) cursor[e] = hist[(size_t)e * nchunks + c];
   __syncwarp();
   const int p0 = c * kPermChunk, p1 = min(P, p0 + kPermChunk);
-  for (int pb = p0; pb < p1; pb += 32) {
+  int ev[kPermChunk / 32];  // the chunk's expert ids, loaded before the in-order walk
+#pragma unroll
+  for (int i = 0; i < kPermChunk / 32; ++i) {
+    const int p = p0 + 32 * i + lane;
+    ev[i] = (p < p1) ? idx[p] : -1;
+  }
+#pragma unroll
+  for (int i = 0; i < kPermChunk / 32; ++i) {
+    const int pb = p0 + 32 * i;
+    if (pb >= p1) break;
     int p = pb + lane;
-    int e = (p < p1) ? idx[p] : -1;
+    int e = ev[i];
     bool ok = (p < p1) && e >= 0 && e < E;
     int key = ok ? e : -1 - lane;  // invalid lanes form singleton groups
     unsigned grp = __match_any_sync(0xffffffffu, key);
