@@ -65,6 +65,10 @@ def workload_shape(name: str) -> synth.LayerShape:
 # checked at run time and the figure is dropped (traffic = null) once the source has changed.
 TRAFFIC = {
     # kernel: (source files, sha256 of their concatenation at capture time, bytes per launch, profile)
+    "gemm_gate_up": (["quantized_expert_ffn_gemm_b200/csrc/gemm.cu", "quantized_expert_ffn_gemm_b200/csrc/tc.cuh",
+                      "quantized_expert_ffn_gemm_b200/csrc/dequant.cuh"],
+                     "157cefd9e230dc80d25b94d71f92251909b253f4c478998441e41f8d3954b7fa", 787024128,
+                     "profiles/grouped_gemm_prefill8k.md"),
 }
 
 
