@@ -232,7 +232,9 @@ __device__ __forceinline__ void frag_from_smem(StepFrag &f, const uint8_t *ca, c
 
 }  // namespace
 
-template <bool Q3>
+// TMAX: the largest token count the instance takes (1, 2, 4 or 8); the token loops of the router
+// are unrolled to TMAX, so the common single-token instance carries no code for the others.
+template <bool Q3, int TMAX>
 __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int T = a.T, H = a.H, E = a.E, k = a.k, I = a.I;
@@ -359,16 +361,16 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
     for (int e0 = blockIdx.x, it = 0; e0 < E; e0 += 4 * G, ++it) {
       const int e = e0 + es * G;
       if (it > 0) load_router(e);
-      float acc[kDecodeMaxT];
+      float acc[TMAX];
 #pragma unroll
-      for (int t = 0; t < kDecodeMaxT; ++t) acc[t] = 0.0f;
+      for (int t = 0; t < TMAX; ++t) acc[t] = 0.0f;
       if (e < E) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int h4 = lane + 32 * u;
           if (h4 >= HQ) continue;
 #pragma unroll
-          for (int t = 0; t < kDecodeMaxT; ++t) {
+          for (int t = 0; t < TMAX; ++t) {
             if (t < T) {
               const uint2 xb = reinterpret_cast<const uint2 *>(xraw + (size_t)t * H)[qh * HQ + h4];
               acc[t] = fmaf(rv[u].x, __uint_as_float(xb.x << 16), acc[t]);
@@ -380,7 +382,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
         }
       }
 #pragma unroll
-      for (int t = 0; t < kDecodeMaxT; ++t) {
+      for (int t = 0; t < TMAX; ++t) {
         if (t < T) {
           const float sum = warp_sum(acc[t]);
           if (lane == 0) rp[(es * 4 + qh) * kDecodeMaxT + t] = sum;
@@ -761,8 +763,13 @@ cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float ep
   }
   if (ring < 2) return cudaErrorNotSupported;
   const FusedLayout L = fused_layout(T, H, E, I, hs_cols, ring, slot_bytes);
-  const void *fn = q3 ? reinterpret_cast<const void *>(decode_fused_kernel<true>)
-                      : reinterpret_cast<const void *>(decode_fused_kernel<false>);
+  const int tmax = T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8;
+#define MOE_FUSED_FN(Q, TM) reinterpret_cast<const void *>(decode_fused_kernel<Q, TM>)
+  const void *fn = q3 ? (tmax == 1 ? MOE_FUSED_FN(true, 1) : tmax == 2 ? MOE_FUSED_FN(true, 2)
+                         : tmax == 4 ? MOE_FUSED_FN(true, 4) : MOE_FUSED_FN(true, 8))
+                      : (tmax == 1 ? MOE_FUSED_FN(false, 1) : tmax == 2 ? MOE_FUSED_FN(false, 2)
+                         : tmax == 4 ? MOE_FUSED_FN(false, 4) : MOE_FUSED_FN(false, 8));
+#undef MOE_FUSED_FN
   cudaError_t e = smem_limit_once_impl(fn, kFSmemMax);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
@@ -806,7 +813,8 @@ cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float ep
   cfg.numAttrs = 1;
   {
     KTimer kt_(KID_DECODE_FUSED, s);
-    e = q3 ? cudaLaunchKernelEx(&cfg, decode_fused_kernel<true>, a) : cudaLaunchKernelEx(&cfg, decode_fused_kernel<false>, a);
+    void *args[] = {&a};
+    e = cudaLaunchKernelExC(&cfg, fn, args);
   }
   return e;
 }
