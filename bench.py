@@ -467,6 +467,44 @@ def run_reference(args, world, rank):
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_crossover(args):
+    """Layer time at small batches through each expert path (the decode-to-prefill crossover):
+    T tokens of the decode-shaped layer (H=2048, E=512, top-10, I=512, shared expert, Q2, Zipf(1.1)
+    router bias), weights rotating over 8 layers, CUDA-event device time per call, one JSON line
+    per (T, path). Not a benchmark line of the contract: it informs the AUTO path's switch point."""
+    import quantized_expert_ffn_gemm_b200 as moe
+    torch.cuda.set_device(0)
+    shape = synth.WORKLOADS["decode1"]
+    H, E, k, I = shape.H, shape.E, shape.k, shape.I
+    layers = build_layers(shape, 8)
+    Tmax = 128
+    ws = moe.Workspace.for_layer(H, E, k, I, True, Tmax)
+    handles = [moe.LayerHandle(Wr, b, rs, ss, k, ws) for (Wr, b, rs, ss) in layers]
+    xs = [synth.make_x(shape.seed, Tmax, H, stream=9000 + i).cuda() for i in range(8)]
+    y = torch.empty(Tmax, H, dtype=torch.float32, device="cuda")
+    paths = {"auto": moe.PATH_AUTO, "gemv": moe.PATH_GEMV, "gemm": moe.PATH_GEMM}
+    for T in (1, 2, 4, 5, 6, 8, 12, 16, 24, 32, 48, 64, 96, 128):
+        for name, path in paths.items():
+            try:
+                for i in range(8):
+                    handles[i % 8].forward(xs[i % 8][:T], y[:T], path=path)
+                torch.cuda.synchronize()
+            except moe.MoeError as e:
+                print(json.dumps({"T": T, "path": name, "unsupported": str(e)}), flush=True)
+                continue
+            n = 64
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for i in range(n):
+                handles[i % 8].forward(xs[i % 8][:T], y[:T], path=path)
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) / n * 1e3
+            print(json.dumps({"T": T, "path": name, "us_per_layer": round(us, 2),
+                              "tokens_per_s": round(T / (us * 1e-6), 1)}), flush=True)
+    assert moe.read_device_error(ws) == 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -478,7 +516,12 @@ def main():
     ap.add_argument("--layers", type=int, default=None,
                     help="distinct layer weight sets to rotate over (default 48 for decode, 4 for prefill)")
     ap.add_argument("--breakdown", action="store_true", help="also time T=4 and T=8192 on rank 0 (extra keys)")
+    ap.add_argument("--crossover", action="store_true",
+                    help="time the expert paths at T = 1..128 (one JSON line per T and path) and exit")
     args = ap.parse_args()
+    if args.crossover:
+        run_crossover(args)
+        return
     if args.steps is None:
         args.steps = DEFAULT_STEPS[args.workload]
     if args.warmup is None:

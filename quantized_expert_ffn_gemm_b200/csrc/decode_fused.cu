@@ -109,13 +109,14 @@ __host__ __device__ inline FusedLayout fused_layout(int T, int H, int E, int I, 
 // counter reaches base + j * nblocks. Every CTA arrives, even after an earlier failure, so the
 // count stays whole; it waits only when `wait` is set. Returns false when the wait gave up (or
 // was not made). Called by every thread of the CTA: the CTA barrier orders the CTA's writes
-// before thread 0's fence and release-add; thread 0's acquire loads and the closing CTA barrier
-// order the CTA's later reads after every other CTA's arrival.
+// before thread 0's release-add; thread 0's acquire loads and the closing CTA barrier order the
+// CTA's later reads after every other CTA's arrival.
 __device__ bool grid_barrier(Ctrl *c, unsigned long long target, int where, bool wait) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
+    // a release add: the CTA's writes ordered before it by the CTA barrier are visible to any
+    // CTA whose acquire load sees the count (no separate fence needed)
     asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(&c->bar_arrivals) : "memory");
     int ok = wait ? 1 : 0;
     const uint64_t t0 = global_ns();

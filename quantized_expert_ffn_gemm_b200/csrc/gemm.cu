@@ -225,10 +225,11 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
         const uint32_t d = tmem + (uint32_t)(b * 256);
         // the next stage's barriers are tested while this stage's MMAs queue up, so a stage whose
         // operands are already in place costs no wait between the MMA groups
+        // full_a alone gates a stage: the dequant warps arrive on it only after they have seen
+        // the stage's TMA complete (full_b), so the activation tile is in place too
         {
           const int g = tl * nk;
-          if (!mbar_wait(full_b(g % kStagesB), (uint32_t)(g / kStagesB) & 1u) ||
-              !mbar_wait(full_a(g % kStagesA), (uint32_t)(g / kStagesA) & 1u)) {
+          if (!mbar_wait(full_a(g % kStagesA), (uint32_t)(g / kStagesA) & 1u)) {
             record_timeout(ctrl, 23);
             ok = false;
           }
@@ -236,18 +237,24 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
         for (int ks = 0; ks < nk && ok; ++ks) {
           const int g = tl * nk + ks;
           const int s = g % kStagesB, sa = g % kStagesA;
+          // operand addresses of the stage's eight MMAs, computed before the first is issued (the
+          // descriptor's start-address field is addr >> 4 in 14 bits; offsets inside the stage
+          // never carry out of it: shared memory is below 256 KB)
+          const uint64_t db = sw128_desc(sB(s));
+          const uint32_t ta = tmem + a_col(sa);
           tc_fence_after();
-          tc_mma_ts(d, tmem + a_col(sa), sw128_desc(sB(s)), idesc, ks != 0 ? 1u : 0u);
+          tc_mma_ts(d, ta, db, idesc, ks != 0 ? 1u : 0u);
           const bool more = ks + 1 < nk;
-          const int s1 = (g + 1) % kStagesB, sa1 = (g + 1) % kStagesA;
-          const uint32_t ph1 = (uint32_t)((g + 1) / kStagesB) & 1u, pha1 = (uint32_t)((g + 1) / kStagesA) & 1u;
-          const bool rb = more && mbar_test(full_b(s1), ph1);
-          const bool ra = more && mbar_test(full_a(sa1), pha1);
+          const int sa1 = (g + 1) % kStagesA;
+          const uint32_t pha1 = (uint32_t)((g + 1) / kStagesA) & 1u;
+          bool ra = false;
 #pragma unroll
-          for (int kk = 1; kk < kBK / 16; ++kk)  // sub-tile kk / 4, 32 bytes per 16 K inside it
-            tc_mma_ts(d, tmem + a_col(sa) + 8u * kk, sw128_desc(sB(s) + (kk >> 2) * SL::kSub + (kk & 3) * 32), idesc, 1u);
+          for (int kk = 1; kk < kBK / 16; ++kk) {  // sub-tile kk / 4, 32 bytes per 16 K inside it
+            tc_mma_ts(d, ta + 8u * kk, db + (uint64_t)((((kk >> 2) * SL::kSub) + (kk & 3) * 32) >> 4), idesc, 1u);
+            if (more && kk == 5) ra = mbar_test(full_a(sa1), pha1);  // next stage, tested while MMAs queue
+          }
           tc_commit(empty_b(s));  // frees the smem stage, and (kStagesA stages on) the TMEM A stage
-          if (more && ((!rb && !mbar_wait(full_b(s1), ph1)) || (!ra && !mbar_wait(full_a(sa1), pha1)))) {
+          if (more && !ra && !mbar_wait(full_a(sa1), pha1)) {
             record_timeout(ctrl, 23);
             ok = false;
           }

@@ -180,22 +180,37 @@ perm_scatter_kernel(const int32_t *__restrict__ idx, int P, int k, int E, const 
 }
 
 // ---------------------------------------------------------------- gather rows (bf16 -> fp16)
+// one warp per row: the source token is read once, then the row's 16-byte chunks are loaded four
+// at a time per lane before any is converted and stored
 __global__ void __launch_bounds__(256)
 perm_gather_kernel(const uint16_t *__restrict__ x, int H, const int32_t *__restrict__ src, int P, int rows,
                    uint16_t *__restrict__ x_perm) {
-  const int H8 = H >> 3;
-  const size_t total = (size_t)rows * H8;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
-    int r = (int)(i / H8), c = (int)(i % H8);
-    int t = (r < P) ? src[r] : r - P;
-    uint4 v = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * H) + c);
-    uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+  const int lane = threadIdx.x & 31, H8 = H >> 3;
+  for (int r = blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += gridDim.x * 8) {
+    const int t = (r < P) ? src[r] : r - P;
+    const uint4 *xs = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
+    uint4 *xd = reinterpret_cast<uint4 *>(x_perm + (size_t)r * H);
+    for (int c0 = lane; c0 < H8; c0 += 128) {
+      uint4 v[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      __half2 h = __floats2half2_rn(__uint_as_float(in[j] << 16), __uint_as_float(in[j] & 0xffff0000u));
-      out[j] = *reinterpret_cast<uint32_t *>(&h);
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + 32 * u;
+        v[u] = (c < H8) ? __ldg(xs + c) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + 32 * u;
+        if (c >= H8) break;
+        const uint32_t in[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        uint32_t out[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          __half2 h = __floats2half2_rn(__uint_as_float(in[j] << 16), __uint_as_float(in[j] & 0xffff0000u));
+          out[j] = *reinterpret_cast<uint32_t *>(&h);
+        }
+        xd[c] = make_uint4(out[0], out[1], out[2], out[3]);
+      }
     }
-    reinterpret_cast<uint4 *>(x_perm + (size_t)r * H)[c] = make_uint4(out[0], out[1], out[2], out[3]);
   }
 }
 
@@ -229,7 +244,7 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const uint16
     }
   }
   const int rows = P + (with_shared ? T : 0);
-  size_t want = ((size_t)rows * (H / 8) + 255) / 256, cap = (size_t)num_sms() * 16;
+  size_t want = ((size_t)rows + 7) / 8, cap = (size_t)num_sms() * 16;
   int grid = (int)(want < cap ? want : cap);
   {
     KTimer kt_(KID_PERM_GATHER, s);
@@ -240,54 +255,67 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const uint16
 
 // ---------------------------------------------------------------- combine
 // y[t,h] = sum_j w[t,j] out[row_of[t,j], h] (fixed j order) + shared[t,h] + residual[t,h]
+// One warp per token: lanes j < k hold the token's rows and weights (broadcast by shuffle), each
+// lane then owns 8-column chunks and issues the k row loads of a chunk before accumulating them.
 __global__ void __launch_bounds__(256)
 combine_kernel(const uint16_t *__restrict__ out, const int32_t *__restrict__ row_of, const float *__restrict__ w,
                int T, int k, int H, const uint16_t *__restrict__ shared, const float *residual, float *y) {
-  const int H8 = H >> 3;
-  const size_t total = (size_t)T * H8;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
-    int t = (int)(i / H8), c = (int)(i % H8);
-    float acc[8];
+  const int lane = threadIdx.x & 31, H8 = H >> 3;
+  for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += gridDim.x * 8) {
+    const int my_row = (lane < k) ? row_of[(size_t)t * k + lane] : -1;
+    const float my_w = (lane < k) ? w[(size_t)t * k + lane] : 0.0f;
+    for (int c = lane; c < H8; c += 32) {
+      float acc[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
-    if (residual) {
-      float4 r0 = reinterpret_cast<const float4 *>(residual + (size_t)t * H)[2 * c];
-      float4 r1 = reinterpret_cast<const float4 *>(residual + (size_t)t * H)[2 * c + 1];
-      acc[0] = r0.x; acc[1] = r0.y; acc[2] = r0.z; acc[3] = r0.w;
-      acc[4] = r1.x; acc[5] = r1.y; acc[6] = r1.z; acc[7] = r1.w;
-    }
-    for (int j = 0; j < k; ++j) {
-      int row = row_of[(size_t)t * k + j];
-      if (row < 0) continue;
-      float wj = w[(size_t)t * k + j];
-      uint4 v = __ldg(reinterpret_cast<const uint4 *>(out + (size_t)row * H) + c);
-      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&vv[q]));
-        acc[2 * q] = fmaf(wj, f.x, acc[2 * q]);
-        acc[2 * q + 1] = fmaf(wj, f.y, acc[2 * q + 1]);
+      for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+      if (residual) {
+        const float4 r0 = reinterpret_cast<const float4 *>(residual + (size_t)t * H)[2 * c];
+        const float4 r1 = reinterpret_cast<const float4 *>(residual + (size_t)t * H)[2 * c + 1];
+        acc[0] = r0.x; acc[1] = r0.y; acc[2] = r0.z; acc[3] = r0.w;
+        acc[4] = r1.x; acc[5] = r1.y; acc[6] = r1.z; acc[7] = r1.w;
       }
-    }
-    if (shared) {
-      uint4 v = __ldg(reinterpret_cast<const uint4 *>(shared + (size_t)t * H) + c);
-      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+      for (int j0 = 0; j0 < k; j0 += 4) {
+        uint4 v[4];
+        float wj[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&vv[q]));
-        acc[2 * q] += f.x;
-        acc[2 * q + 1] += f.y;
+        for (int u = 0; u < 4; ++u) {
+          const int rj = __shfl_sync(0xffffffffu, my_row, (j0 + u) & 31);
+          wj[u] = __shfl_sync(0xffffffffu, my_w, (j0 + u) & 31);
+          const bool use = j0 + u < k && rj >= 0;  // rows past k or flagged (-1) add nothing
+          v[u] = use ? __ldg(reinterpret_cast<const uint4 *>(out + (size_t)rj * H) + c) : make_uint4(0, 0, 0, 0);
+          if (!use) wj[u] = 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&vv[q]));
+            acc[2 * q] = fmaf(wj[u], f.x, acc[2 * q]);
+            acc[2 * q + 1] = fmaf(wj[u], f.y, acc[2 * q + 1]);
+          }
+        }
       }
+      if (shared) {
+        const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(shared + (size_t)t * H) + c);
+        const uint32_t vv[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&vv[q]));
+          acc[2 * q] += f.x;
+          acc[2 * q + 1] += f.y;
+        }
+      }
+      float4 *yo = reinterpret_cast<float4 *>(y + (size_t)t * H);
+      yo[2 * c] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      yo[2 * c + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
-    float4 *yo = reinterpret_cast<float4 *>(y + (size_t)t * H);
-    yo[2 * c] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    yo[2 * c + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
 }
 
 cudaError_t launch_combine(const uint16_t *out_perm, const int32_t *row_of, const float *w, int T, int k, int H,
                            const uint16_t *shared_out, const float *residual, float *y, cudaStream_t s) {
-  size_t want = ((size_t)T * (H / 8) + 255) / 256, cap = (size_t)num_sms() * 16;
+  size_t want = ((size_t)T + 7) / 8, cap = (size_t)num_sms() * 16;
   int grid = (int)(want < cap ? want : cap);
   {
     KTimer kt_(KID_COMBINE, s);
