@@ -175,10 +175,11 @@ moe_status moe_combine(const uint16_t *out_perm, const int32_t *row_of, const fl
                        int32_t H, const uint16_t *shared_out_opt, const float *residual_opt, float *y,
                        void *stream);
 
-/* One full MoE layer: router + top-k, then either (T <= 4 or path == GEMV) the decode path
- * (dequant-GEMV over the distinct selected experts, down projection fused with the weighted
- * combine) or the prefill path (permute, tcgen05 grouped GEMM gate/up with fused SwiGLU,
- * grouped GEMM down, combine).
+/* One full MoE layer: router + top-k, then either the decode path (T <= 8 and path != GEMM, or
+ * path == GEMV: dequant-GEMV over the distinct selected experts, down projection fused with the
+ * weighted combine; for small enough T one cooperative kernel does the whole layer) or the
+ * prefill path (permute, tcgen05 grouped GEMM gate/up with fused SwiGLU, grouped GEMM down,
+ * combine).
  *   y = sum_j w_j FFN_{idx_j}(x) + FFN_shared(x) (+ residual)      fp32 [T,H]
  * x bf16 [T,H]; Wr fp32 [E,H]; bias fp32 [E] or NULL; routed: gate/up [E][I][H], down [E][H][I];
  * shared_opt: one expert (n_experts = 1) when desc->has_shared; residual_opt fp32 [T,H] or NULL
@@ -234,6 +235,15 @@ const char *moe_kernel_name(int32_t kernel);
 /* Synchronise `stream`, read the workspace's device error word into *code (MOE_OK,
  * MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT) and clear it. */
 moe_status moe_read_device_error(void *ws, int32_t *code, void *stream);
+
+/* Test hook for the failure path of the device-side waits. Launches two CTAs that arrive at the
+ * grid barrier the fused decode kernel uses and then wait for one arrival more than they made;
+ * the wait gives up after limit_ms (1..2000) and records MOE_ERR_TIMEOUT in the workspace error
+ * word (read and clear it with moe_read_device_error). Nothing traps and the context stays
+ * usable; each CTA takes its own arrival back after giving up, so the workspace serves the next
+ * call unchanged. ws: any initialised workspace (at least its 128-byte control area), 16-byte
+ * aligned; errors: MOE_ERR_WORKSPACE / MOE_ERR_ALIGNMENT / MOE_ERR_INVALID_ARG on the host. */
+moe_status moe_test_barrier_timeout(void *ws, size_t ws_bytes, int32_t limit_ms, void *stream);
 
 #ifdef __cplusplus
 }

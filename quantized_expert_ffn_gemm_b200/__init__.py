@@ -26,7 +26,8 @@ Q2, Q3 = 2, 3
 EXPORTED = ["moe_status_string", "moe_workspace_bytes", "moe_workspace_init", "moe_rmsnorm_bf16",
             "moe_router_topk", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
             "moe_stack_forward", "moe_dequant_rows", "moe_read_device_error", "moe_timing_enable",
-            "moe_timing_read", "moe_kernel_count", "moe_kernel_name", "moe_router_topk_static"]
+            "moe_timing_read", "moe_kernel_count", "moe_kernel_name", "moe_router_topk_static",
+            "moe_test_barrier_timeout"]
 
 
 class MoeError(RuntimeError):
@@ -265,6 +266,13 @@ def dequant_rows(m, expert: int, row0: int, nrows: int):
     _check("moe_dequant_rows", lib().moe_dequant_rows(ctypes.byref(q), expert, row0, nrows, _p(f32), _p(f16),
                                                       _stream()))
     return f32, f16
+
+
+def test_barrier_timeout(ws: Workspace, limit_ms: int = 50):
+    """moe_test_barrier_timeout: make the fused kernel's grid barrier wait for an arrival that never
+    comes; the wait gives up after limit_ms and MOE_ERR_TIMEOUT lands in the workspace error word."""
+    _check("moe_test_barrier_timeout", lib().moe_test_barrier_timeout(ws.ptr, ws.size,
+                                                                      int(limit_ms), _stream()))
 
 
 def read_device_error(ws: Workspace) -> int:

@@ -291,8 +291,10 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
   const moe_expert_set *sh = hs ? shared_opt : nullptr;
   cudaError_t e = cudaSuccess;
 
-  const bool decode = (T <= kDecodeMaxT) && path != MOE_PATH_GEMM && (path == MOE_PATH_GEMV || T <= 4) &&
-                      decode_router_fits(T, H, E);
+  // decode path (distinct experts' weights read once, tokens as MMA columns) up to 8 tokens: at
+  // T = 5..8 it takes about half the time of the grouped GEMM, whose 16-row tiles are bound by MMA
+  // issue (measured by bench.py --crossover)
+  const bool decode = (T <= kDecodeMaxT) && path != MOE_PATH_GEMM && decode_router_fits(T, H, E);
   if (decode) {
     DecUnit *units = at<DecUnit>(ws, L.units);
     uint16_t *hdec = at<uint16_t>(ws, L.hdec);
@@ -378,7 +380,7 @@ moe_status moe_stack_forward(const float *r_in, int32_t T, int32_t L, const floa
   uint16_t *u = at<uint16_t>(ws, LY.u16);
   cudaStream_t s = (cudaStream_t)stream;
   // decode-sized batches: RMSNorm runs inside the fused layer kernel (one launch per layer)
-  const bool fused = path == MOE_PATH_AUTO && T <= 4 && decode_router_fits(T, H, E);
+  const bool fused = path == MOE_PATH_AUTO && T <= kDecodeMaxT && decode_router_fits(T, H, E);
   for (int l = 0; l < L; ++l) {
     const float *r = (l == 0) ? r_in : r_out;
     const float *b = bias ? bias[l] : nullptr;
@@ -447,6 +449,15 @@ int32_t moe_kernel_count(void) { return KID_COUNT; }
 
 const char *moe_kernel_name(int32_t kernel) {
   return (kernel >= 0 && kernel < KID_COUNT) ? kKernelNames[kernel] : nullptr;
+}
+
+moe_status moe_test_barrier_timeout(void *ws, size_t ws_bytes, int32_t limit_ms, void *stream) {
+  if (!ws) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < sizeof(Ctrl)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_ALIGNMENT;
+  if (limit_ms < 1 || limit_ms > 2000) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_barrier_starve(static_cast<Ctrl *>(ws), 2, (uint64_t)limit_ms * 1000000ull,
+                                           (cudaStream_t)stream));
 }
 
 moe_status moe_read_device_error(void *ws, int32_t *code, void *stream) {

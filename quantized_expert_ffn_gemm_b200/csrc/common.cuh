@@ -141,6 +141,10 @@ cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float ep
                                 const moe_expert_set *shared, const float *residual, float *y, float *logits,
                                 int32_t *idx, float *w, uint16_t *hdec, Ctrl *ctrl, cudaStream_t s);
 
+// test hook: a grid barrier that waits for one arrival more than the `ctas` CTAs make, giving up
+// after limit_ns with MOE_ERR_TIMEOUT in the control area
+cudaError_t launch_barrier_starve(Ctrl *ctrl, int ctas, uint64_t limit_ns, cudaStream_t s);
+
 // prefill path (tcgen05 grouped GEMM)
 int gemm_shape_supported(int H, int I);
 cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, int n_rows, int E, int H, int I,

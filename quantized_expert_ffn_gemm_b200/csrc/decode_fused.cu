@@ -111,7 +111,8 @@ __host__ __device__ inline FusedLayout fused_layout(int T, int H, int E, int I, 
 // was not made). Called by every thread of the CTA: the CTA barrier orders the CTA's writes
 // before thread 0's release-add; thread 0's acquire loads and the closing CTA barrier order the
 // CTA's later reads after every other CTA's arrival.
-__device__ bool grid_barrier(Ctrl *c, unsigned long long target, int where, bool wait) {
+__device__ bool grid_barrier(Ctrl *c, unsigned long long target, int where, bool wait,
+                             uint64_t limit_ns = kWaitLimitNs) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -125,7 +126,7 @@ __device__ bool grid_barrier(Ctrl *c, unsigned long long target, int where, bool
       asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(&c->bar_arrivals) : "memory");
       if ((long long)(v - target) >= 0) break;
       __nanosleep(32);
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         ok = 0;
         set_device_error(c, MOE_ERR_TIMEOUT, where);
         break;
@@ -739,6 +740,39 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
 
   // ---------------- no copy may still be writing this CTA's shared memory when it exits
   cp_async_wait_all();
+}
+
+// Test hook of the failure path: every CTA arrives at the fused kernel's grid barrier, which is
+// then asked to wait for one arrival more than were made. The wait gives up after limit_ns and
+// records MOE_ERR_TIMEOUT; nothing traps and the context stays usable. Each CTA then takes its
+// arrival back, so the count is again a whole number of earlier launches' arrivals (which is what
+// the fused kernel's base computation assumes).
+__global__ void barrier_starve_kernel(Ctrl *ctrl, uint64_t limit_ns) {
+  __shared__ unsigned long long s_base;
+  if (threadIdx.x == 0) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(&ctrl->bar_arrivals) : "memory");
+    s_base = v;
+  }
+  __syncthreads();
+  // the base is read before any CTA of this launch arrives only if all read before the first add,
+  // which nothing guarantees; the target base + grid + 1 is out of reach either way, since at most
+  // grid arrivals follow any CTA's read
+  const bool ok = grid_barrier(ctrl, s_base + gridDim.x + 1, 39, true, limit_ns);
+  if (threadIdx.x == 0 && !ok) atomicAdd(&ctrl->bar_arrivals, ~0ull);
+}
+
+cudaError_t launch_barrier_starve(Ctrl *ctrl, int ctas, uint64_t limit_ns, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(32);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, barrier_starve_kernel, ctrl, limit_ns);
 }
 
 cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float eps, int T, int H, const float *Wr,

@@ -199,6 +199,20 @@ def test_cross_path_gemv_vs_gemm(name, T):
     assert rel_err(ya.cpu().numpy(), yb.cpu().numpy()) <= Y_TOL
 
 
+@pytest.mark.parametrize("name,T", [("mid", 5), ("mid", 8), ("decode4", 5), ("decode4", 6), ("decode4", 8)])
+def test_layer_forward_decode_batches(name, T):
+    # 5-8 tokens take the decode path under AUTO: the fused kernel where its shared-memory plan
+    # fits (top-4 layer; top-10 at T=5), the separate decode kernels beyond (top-10 at T=6, 8).
+    # Fresh tokens on the cached layer's weights, every token against the oracle.
+    L0, (_, Wr, b, routed, shared) = layer_of(name)
+    s = L0.shape
+    L = synth.LayerInputs(s, synth.make_x(s.seed, T, s.H, stream=40 + T), L0.Wr, L0.bias, L0.routed, L0.shared)
+    ws = moe.Workspace.for_layer(s.H, s.E, s.k, s.I, s.shared, T)
+    y, idx, _ = moe.layer_forward(L.x.cuda(), Wr, b, routed, shared, s.k, ws, want_routing=True)
+    assert moe.read_device_error(ws) == 0
+    check_layer(y.cpu().numpy(), idx.cpu().numpy(), L, range(T))
+
+
 def test_mtp_verify_T4_equals_four_T1():
     L, (x, Wr, b, routed, shared) = layer_of("decode4")
     ws = ws_for(L)
@@ -213,6 +227,28 @@ def test_zero_tokens_is_noop():
     ws = ws_for(L)
     y = moe.layer_forward(x[:0], Wr, b, routed, shared, 2, ws)
     assert y.shape == (0, 256)
+
+
+# ----------------------------------------------------------------------------- failure path
+def test_starved_barrier_times_out_and_context_survives():
+    # A grid barrier waiting for an arrival that never comes gives up after its limit, reports
+    # MOE_ERR_TIMEOUT through the workspace error word, and leaves the context and the workspace
+    # fit for the next call (which must still match the oracle).
+    L, (x, Wr, b, routed, shared) = layer_of("decode1")
+    s = L.shape
+    ws = ws_for(L)
+    y0 = moe.layer_forward(x, Wr, b, routed, shared, s.k, ws)
+    assert moe.read_device_error(ws) == 0
+    import time
+    t0 = time.perf_counter()
+    moe.test_barrier_timeout(ws, limit_ms=20)
+    assert moe.read_device_error(ws) == moe.MOE_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 1.5           # the limit, not a hang
+    assert moe.read_device_error(ws) == 0            # reading cleared the word
+    y1, idx, _ = moe.layer_forward(x, Wr, b, routed, shared, s.k, ws, want_routing=True)
+    assert moe.read_device_error(ws) == 0
+    assert torch.equal(y0, y1)
+    check_layer(y1.cpu().numpy(), idx.cpu().numpy(), L, range(s.T))
 
 
 # ----------------------------------------------------------------------------- RMSNorm and stacks
