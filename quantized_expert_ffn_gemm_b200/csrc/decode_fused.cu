@@ -47,6 +47,7 @@ constexpr int kFMaxUnits = kFSlots + 1;
 constexpr int kFMaxRing = 16;               // shared-memory slots for weight copies
 constexpr int kFMaxE = 512;                 // experts the fused kernel takes
 constexpr int kFSmemMax = 226 * 1024;       // dynamic shared memory (a little is left for static)
+constexpr int kDnBatch = 4;                 // down half steps (K = 128 each) whose loads go out together
 
 // named barriers (0 is __syncthreads): one per gate/up group
 constexpr int kBarGroup0 = 1;
@@ -94,7 +95,7 @@ __host__ __device__ inline FusedLayout fused_layout(int T, int H, int E, int I, 
   L.misc = take(16 * 4);
   L.slot = take((size_t)(kFMaxUnits + 1) * 4);
   L.src = take((size_t)kFSlots * 4);
-  L.plist = take((size_t)T * 16 * 16 * 8);      // top-16 code lists (tokens x 32-expert chunks)
+  L.plist = take((size_t)T * 16 * 16 * 8);      // top-16 code lists: [token][rank][32-expert chunk]
   L.firstof = take((size_t)E * 4);                // expert -> first pair choosing it
   L.pcnt = take((size_t)(kFMaxUnits + 1) * 4);
   L.bars = take((size_t)kFMaxRing * 8);
@@ -417,7 +418,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       unsigned long long v = 0ull;
       if (e < E) v = topk_code(__ldcg(a.logits + (size_t)t * E + e) + (a.bias ? __ldg(a.bias + e) : 0.f), e);
       v = warp_sort32_desc(v);
-      if (lane < 16) plist[(size_t)task * 16 + lane] = v;
+      if (lane < 16) plist[((size_t)t * 16 + lane) * 16 + c] = v;  // rank-major: the merge reads across chunks
     }
     {  // into L2 while the top-k runs: the shared expert's rows (always selected)
       const int nthr = gridDim.x * kFThreads, first = blockIdx.x * kFThreads + tid;
@@ -442,7 +443,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
     if (warp < T) {
       unsigned long long c[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) c[i] = (lane < nch) ? plist[((size_t)warp * nch + lane) * 16 + i] : 0ull;
+      for (int i = 0; i < 16; ++i) c[i] = (lane < nch) ? plist[((size_t)warp * 16 + i) * 16 + lane] : 0ull;
       float my_val = -INFINITY;
       int my_idx = 0;
       for (int j = 0; j < k; ++j) {
@@ -596,6 +597,9 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
     for (int q = warp; q < min(n_total, R); q += kFWarps) issue_fill(q);
 
   // ---------------- P2: gate/up + SwiGLU; group grp takes this CTA's items grp, grp + 2, ...
+  // The ring has an even number of slots, so the items that share a slot (q, q + R, ...) all
+  // fall to one group, which takes them in order: a parity wait then never runs two phases
+  // ahead of the slot's last completed fill (where it would mistake the older phase for its own).
   if (ok) {
     const int grp = warp >> 3, j8 = warp & 7, gtid = tid & 255;
     int buf = 0;
@@ -643,11 +647,15 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   }
   ok = grid_barrier(ctrl, s_base + 2 * (unsigned long long)nblk, 32, ok) && ok;
 
-  // ---------------- P3: down projection + weighted combine (+ residual) for 16 output features per CTA
+  // ---------------- P3: down projection + weighted combine (+ residual) for 16 output features per CTA.
+  // Piece d of a row block shares its slot with piece d - R. Before waiting on piece d's fill a
+  // warp waits until piece d - R is consumed (its last consumer then issues piece d's fill), so
+  // the parity wait is at most one phase ahead; for d < R the slot's previous phase belongs to a
+  // P2 item or to an earlier row block, consumed before this row block starts. Units are taken in
+  // increasing order, so the lowest waiting piece can always proceed.
   if (ok) {
     const int nslots = s_slot[nu];
     const int xstride = I + 4;
-    const int n_items = nu * nhalf_dn;
     const int dn = a.dn_bytes;
     for (int rbl = 0; rbl < n_rb; ++rbl) {
       const int r0 = ((int)blockIdx.x + rbl * G) * 16;
@@ -676,46 +684,68 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       }
       __syncthreads();
       float tot[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int it = warp; it < n_items; it += kFWarps) {
-        const int u = it / nhalf_dn, hsi = it % nhalf_dn;
+      // one unit per warp item: its 16 down rows over all of K (the half steps' shared-memory
+      // loads go out together, then the MMAs)
+      for (int u = warp; u < nu; u += kFWarps) {
         const int d = u / a.dpu, qd = qb + d, s = qd % R;
+        if (d >= R) {  // piece d - R, in the same slot, fully consumed first (bounded wait)
+          const int need_n = min(a.dpu, nu - (d - R) * a.dpu);
+          const uint64_t t0 = global_ns();
+          while (!s_abort && *reinterpret_cast<volatile int *>(&s_pcnt[d - R]) < need_n) {
+            if (global_ns() - t0 > kWaitLimitNs) {
+              s_abort = 1;
+              set_device_error(ctrl, MOE_ERR_TIMEOUT, 44);
+            }
+          }
+          __syncwarp();
+        }
         const bool have = wait_bar(full(s), (uint32_t)(qd / R) & 1u, 43);
         const DecUnit &un = su[u];
-        const int k0 = hsi * (kStepK / 2) + 32 * t4;
-        const bool kok = k0 < I;
-        const bool colok = ((un.mask >> g) & 1) && kok;
+        const bool colok = (un.mask >> g) & 1;
         const int slot = s_slot[u] + __popc(un.mask & ((1u << g) - 1u));
         const __half *xcol = hs + (size_t)(colok ? slot : 0) * xstride;
         float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
-        if (have && kok) {
+        if (have) {
           const uint8_t *pc = ringp + (size_t)s * S + (size_t)(u % a.dpu) * dn;
           const uint8_t *ca = pc + (size_t)g * (I / 4), *cb = pc + (size_t)(g + 8) * (I / 4);
           const uint16_t *sa = reinterpret_cast<const uint16_t *>(pc + 4 * I) + (size_t)g * (I / 32);
           const uint16_t *sb = reinterpret_cast<const uint16_t *>(pc + 4 * I) + (size_t)(g + 8) * (I / 32);
           const uint8_t *ha = pc + 5 * I + (size_t)g * (I / 8), *hb = pc + 5 * I + (size_t)(g + 8) * (I / 8);
-          HalfFrag f;
-          f.w0 = *reinterpret_cast<const uint2 *>(ca + k0 / 4);
-          f.w1 = *reinterpret_cast<const uint2 *>(cb + k0 / 4);
-          f.d0 = sa[k0 / 32];
-          f.d1 = sb[k0 / 32];
-          if (Q3) {
-            f.h0 = *reinterpret_cast<const uint32_t *>(ha + k0 / 8);
-            f.h1 = *reinterpret_cast<const uint32_t *>(hb + k0 / 8);
+          for (int h0 = 0; h0 < nhalf_dn; h0 += kDnBatch) {
+            HalfFrag f[kDnBatch];
+#pragma unroll
+            for (int b = 0; b < kDnBatch; ++b) {
+              const int k0 = (h0 + b) * (kStepK / 2) + 32 * t4;
+              if (k0 < I) {
+                f[b].w0 = *reinterpret_cast<const uint2 *>(ca + k0 / 4);
+                f[b].w1 = *reinterpret_cast<const uint2 *>(cb + k0 / 4);
+                f[b].d0 = sa[k0 / 32];
+                f[b].d1 = sb[k0 / 32];
+                if (Q3) {
+                  f[b].h0 = *reinterpret_cast<const uint32_t *>(ha + k0 / 8);
+                  f[b].h1 = *reinterpret_cast<const uint32_t *>(hb + k0 / 8);
+                }
+              }
+            }
+#pragma unroll
+            for (int b = 0; b < kDnBatch; ++b) {
+              const int k0 = (h0 + b) * (kStepK / 2) + 32 * t4;
+              if (k0 < I) mma_half_step<Q3>(acc, acc2, f[b], xcol, k0, colok);
+            }
           }
-          mma_half_step<Q3>(acc, acc2, f, xcol, k0, colok);
         }
         const float wa = un.w[2 * t4], wb = un.w[2 * t4 + 1];
         tot[0] = fmaf(wa, acc[0] + acc2[0], tot[0]);
         tot[1] = fmaf(wb, acc[1] + acc2[1], tot[1]);
         tot[2] = fmaf(wa, acc[2] + acc2[2], tot[2]);
         tot[3] = fmaf(wb, acc[3] + acc2[3], tot[3]);
-        // the warp that finishes a piece's last item refills its slot at once
+        // the warp that finishes a piece's last unit refills its slot at once
         __syncwarp();
         int last = 0;
         if (lane == 0) {
           const int nun = min(a.dpu, nu - d * a.dpu);
           __threadfence_block();
-          last = (atomicAdd(&s_pcnt[d], 1) == nun * nhalf_dn - 1) ? 1 : 0;
+          last = (atomicAdd(&s_pcnt[d], 1) == nun - 1) ? 1 : 0;
           __threadfence_block();
         }
         last = __shfl_sync(0xffffffffu, last, 0);
@@ -796,6 +826,7 @@ cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float ep
     const int need = (max_units * (I / 8) + G - 1) / G + ((H / 16 + G - 1) / G) * ((max_units + dpu - 1) / dpu);
     if (ring > need) ring = need;
   }
+  ring &= ~1;  // even: the slots' items fall to one gate/up group each (see the kernel's P2)
   if (ring < 2) return cudaErrorNotSupported;
   const FusedLayout L = fused_layout(T, H, E, I, hs_cols, ring, slot_bytes);
   const int tmax = T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8;

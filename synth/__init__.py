@@ -252,6 +252,10 @@ WORKLOADS = {
     # decode step / MTP verify: T=1 or 4, Zipf(1.1) router bias, shared expert
     "decode1": LayerShape("decode1", 1, 2048, 512, 10, 512, Q2, True, 1.1),
     "decode4": LayerShape("decode4", 4, 2048, 512, 10, 512, Q2, True, 1.1),
+    # verify pass over one token and five prompt-lookup drafts (T=6), same layer shape
+    "verify6": LayerShape("verify6", 6, 2048, 512, 10, 512, Q2, True, 1.1),
+    # pruned variant: 256 of the 512 experts kept per layer, otherwise the decode layer
+    "decode1_pruned256": LayerShape("decode1_pruned256", 1, 2048, 256, 10, 512, Q2, True, 1.1),
     # prefill chunk: 8192 tokens, uniform router, shared expert
     "prefill8k": LayerShape("prefill8k", 8192, 2048, 512, 10, 512, Q2, True, None),
     # prefill with 3-bit weights and Zipf(1.2) skew, no shared expert

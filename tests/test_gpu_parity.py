@@ -164,7 +164,8 @@ def test_expert_ffn_rows(name, path):
 
 
 # ----------------------------------------------------------------------------- layer forward
-@pytest.mark.parametrize("name,ntok", [("tiny", 64), ("decode1", 1), ("decode4", 4), ("mid", 300),
+@pytest.mark.parametrize("name,ntok", [("tiny", 64), ("decode1", 1), ("decode4", 4), ("verify6", 6),
+                                       ("decode1_pruned256", 1), ("mid", 300),
                                        ("mid_q3", 200), ("prefill8k", 24), ("prefill2k_q3", 24)])
 def test_layer_forward(name, ntok):
     L, (x, Wr, b, routed, shared) = layer_of(name)
@@ -199,10 +200,13 @@ def test_cross_path_gemv_vs_gemm(name, T):
     assert rel_err(ya.cpu().numpy(), yb.cpu().numpy()) <= Y_TOL
 
 
-@pytest.mark.parametrize("name,T", [("mid", 5), ("mid", 8), ("decode4", 5), ("decode4", 6), ("decode4", 8)])
+@pytest.mark.parametrize("name,T", [("mid", 5), ("mid", 8), ("decode4", 5), ("decode4", 6), ("decode4", 8),
+                                    ("prefill8k", 4), ("prefill8k", 5)])
 def test_layer_forward_decode_batches(name, T):
     # 5-8 tokens take the decode path under AUTO: the fused kernel where its shared-memory plan
     # fits (top-4 layer; top-10 at T=5), the separate decode kernels beyond (top-10 at T=6, 8).
+    # With the uniform router of the prefill layer, 5 tokens choose ~50 distinct experts: more
+    # down pieces than shared-memory slots, so two pieces of one row block share a slot.
     # Fresh tokens on the cached layer's weights, every token against the oracle.
     L0, (_, Wr, b, routed, shared) = layer_of(name)
     s = L0.shape
