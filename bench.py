@@ -63,20 +63,28 @@ def workload_shape(name: str) -> synth.LayerShape:
 
 
 # DRAM bytes (read + write) per launch of the dominant kernels, from the committed ncu captures
-# (profiles/*.md), valid only for the kernel source they were taken on: the file's sha256 is
-# checked at run time and the figure is dropped (traffic = null) once the source has changed.
+# (profiles/*.md), valid only for the kernel source and the launch shape they were taken on: the
+# sources' sha256 is checked at run time and the figure is dropped (traffic = null) once the
+# source has changed, or for a workload whose launches differ from the captured one.
+_DEC_SRC = ["quantized_expert_ffn_gemm_b200/csrc/decode_fused.cu", "quantized_expert_ffn_gemm_b200/csrc/common.cuh",
+            "quantized_expert_ffn_gemm_b200/csrc/dequant.cuh", "quantized_expert_ffn_gemm_b200/csrc/gemv.cuh",
+            "quantized_expert_ffn_gemm_b200/csrc/tc.cuh", "quantized_expert_ffn_gemm_b200/csrc/topk.cuh"]
+_GEMM_SRC = ["quantized_expert_ffn_gemm_b200/csrc/gemm.cu", "quantized_expert_ffn_gemm_b200/csrc/tc.cuh",
+             "quantized_expert_ffn_gemm_b200/csrc/dequant.cuh"]
 TRAFFIC = {
-    # kernel: (source files, sha256 of their concatenation at capture time, bytes per launch, profile)
-    "gemm_gate_up": (["quantized_expert_ffn_gemm_b200/csrc/gemm.cu", "quantized_expert_ffn_gemm_b200/csrc/tc.cuh",
-                      "quantized_expert_ffn_gemm_b200/csrc/dequant.cuh"],
-                     "f5ad8aca8c32a2576bfdf9f5a1d66e6cbeb86fb1fb932b6adae357c9fbff935a", 786358272,
-                     "profiles/grouped_gemm_prefill8k.md"),
+    # (kernel, workloads with the captured launch shape): (sources, sha256, bytes per launch, profile)
+    ("gemm_gate_up", ("prefill8k", "stack_prefill")):
+        (_GEMM_SRC, "f5ad8aca8c32a2576bfdf9f5a1d66e6cbeb86fb1fb932b6adae357c9fbff935a", 786358272,
+         "profiles/grouped_gemm_prefill8k.md"),
+    ("decode_fused", ("decode1",)):
+        (_DEC_SRC, "a5d3e5e3c41bbea67c9e7daa51d8d90d767f00d17c80b3c00876d3b84accd6f3", 15117824,
+         "profiles/decode_fused_kernel_decode1.md"),
 }
 
 
-def traffic_for(kernel: str):
+def traffic_for(kernel: str, workload: str):
     import hashlib
-    ent = TRAFFIC.get(kernel)
+    ent = next((v for (kn, wls), v in TRAFFIC.items() if kn == kernel and workload in wls), None)
     if ent is None:
         return None
     srcs, sha, nbytes, _ = ent
@@ -341,7 +349,7 @@ def run_ours(args, world, rank, local):
                 d_ms / d_n * 1e3)
         achieved = algo / (launch_us / 1e6) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"], "unit": "GB/s",
-                "frac": round(achieved / pk["hbm"], 4), "traffic": traffic_for(dom), "peak_source": pk["src"],
+                "frac": round(achieved / pk["hbm"], 4), "traffic": traffic_for(dom, args.workload), "peak_source": pk["src"],
                 "algorithmic_bytes_per_launch": int(algo), "avg_launch_us": round(launch_us, 3),
                 "launch_timing": timing}
         layer_bytes = units_avg * (gu_b + dn_b) + E * H * 4 + T * H * 2 + T * H * 4
@@ -360,7 +368,7 @@ def run_ours(args, world, rank, local):
         capped = bool(sm and smax and sm < 0.95 * smax)
         peak_tc = pk["tc_sus"] if capped else pk["tc"]
         roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak_tc,
-                "unit": "TFLOP/s", "frac": round(achieved / peak_tc, 4), "traffic": traffic_for(dom),
+                "unit": "TFLOP/s", "frac": round(achieved / peak_tc, 4), "traffic": traffic_for(dom, args.workload),
                 "peak_source": pk["src"] + (" sustained" if capped else " burst") +
                 " bf16 (fp16 MMA runs at the bf16 rate; SM clock %s of %s MHz under load)" % (sm, smax),
                 "frac_of_other_peak": round(achieved / (pk["tc"] if capped else pk["tc_sus"]), 4),
