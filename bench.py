@@ -527,8 +527,17 @@ def run_crossover(args):
             e1.record()
             torch.cuda.synchronize()
             us = e0.elapsed_time(e1) / n * 1e3
+            # per-kernel device time: the same calls queued behind a sleep kernel, events per launch
+            nk = 16
+            moe.timing_enable(True)
+            torch.cuda._sleep(int(4e6))
+            for i in range(nk):
+                handles[i % 8].forward(xs[i % 8][:T], y[:T], path=path)
+            torch.cuda.synchronize()
+            moe.timing_enable(False)
+            kt = {kn: round(ms_ / nk * 1e3, 2) for kn, (ms_, _) in sorted(moe.timing_read().items())}
             print(json.dumps({"T": T, "path": name, "us_per_layer": round(us, 2),
-                              "tokens_per_s": round(T / (us * 1e-6), 1)}), flush=True)
+                              "tokens_per_s": round(T / (us * 1e-6), 1), "kernels_us": kt}), flush=True)
     assert moe.read_device_error(ws) == 0
 
 

@@ -236,7 +236,8 @@ moe_status moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, int32_
     return cuda_status(launch_grouped_ffn(x_perm, offsets, n_rows, E, H, I, *routed, shared_opt,
                                           at<uint16_t>(ws, L.hperm), out_perm, at<int2>(ws, L.tiles), ctrl, s));
   DecUnit *units = at<DecUnit>(ws, L.units);
-  const int max_units = (n_rows + 7) / 8 + n_groups;
+  // a group of n rows makes ceil(n / 8) units: at most rows / 8 + (non-empty groups) in all
+  const int max_units = (n_rows + 7) / 8 + (n_groups < n_rows ? n_groups : n_rows);
   cudaError_t e = launch_decode_units_from_offsets(offsets, n_groups, shared_opt ? 1 : 0, n_rows, units, ctrl, s);
   if (e == cudaSuccess)
     e = launch_decode_gate_up(x_perm, 0, H, I, *routed, shared_opt, units, max_units, ctrl, at<uint16_t>(ws, L.hdec), s);
@@ -335,7 +336,7 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
                                at<int2>(ws, L.tiles), ctrl, s);
       } else {
         DecUnit *units = at<DecUnit>(ws, L.units);
-        const int n_groups = E + hs, max_units = (rows + 7) / 8 + n_groups;
+        const int n_groups = E + hs, max_units = (rows + 7) / 8 + (n_groups < rows ? n_groups : rows);
         e = launch_decode_units_from_offsets(offsets, n_groups, hs, rows, units, ctrl, s);
         if (e == cudaSuccess)
           e = launch_decode_gate_up(xperm, 0, H, I, *routed, sh, units, max_units, ctrl, at<uint16_t>(ws, L.hdec), s);

@@ -229,12 +229,17 @@ dec_down_kernel(int H, int I, moe_expert_set routed, moe_expert_set shared, cons
           mma_step<Q3>(acc, acc2, fl, xcol, st * kStepK + 64 * t, colok && st * kStepK + 64 * t < I);
 #pragma unroll
           for (int e = 0; e < 4; ++e) acc[e] += acc2[e];
-        } else {  // rows mode with several K steps: one step at a time (keeps register use low)
+        } else {  // rows mode with several K steps: two steps' loads in flight, then their MMAs
           const MatView mv = mat_sel(routed, shared, un.set, 2, un.expert);
-          for (int st = 0; st < nsteps; ++st) {
-            StepFrag fl;
-            load_step<Q3>(fl, mv, r0, st, true);
-            mma_step<Q3>(acc, acc2, fl, xcol, st * kStepK + 64 * t, colok && st * kStepK + 64 * t < I);
+          for (int st = 0; st < nsteps; st += 2) {
+            StepFrag fl[2];
+            load_step<Q3>(fl[0], mv, r0, st, true);
+            load_step<Q3>(fl[1], mv, r0, st + 1, st + 1 < nsteps);
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+              const int kb = (st + b) * kStepK + 64 * t;
+              if (st + b < nsteps) mma_step<Q3>(acc, acc2, fl[b], xcol, kb, colok && kb < I);
+            }
           }
 #pragma unroll
           for (int e = 0; e < 4; ++e) acc[e] += acc2[e];
@@ -295,39 +300,86 @@ cudaError_t launch_decode_down(int H, int I, const moe_expert_set &routed, const
 }
 
 // ---------------------------------------------------------------- units for grouped rows
-// rows mode for moe_expert_ffn: group g's rows [off[g], off[g+1]) in chunks of 8 columns
-__global__ void units_from_offsets_kernel(const int32_t *__restrict__ off, int n_groups, int shared_group,
-                                          int n_rows, DecUnit *__restrict__ units, Ctrl *__restrict__ ctrl) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  int nu = 0;
-  for (int gi = 0; gi < n_groups; ++gi) {
+// rows mode for moe_expert_ffn: group g's rows [off[g], off[g+1]) in chunks of 8 columns. One
+// CTA: each thread takes a group, a block-wide exclusive scan of the groups' chunk counts gives
+// each group's first unit, and the groups are walked in blocks of kUnitsThreads. Units come out
+// in group order, then row order, as a serial walk would produce them.
+constexpr int kUnitsThreads = 1024;
+
+__global__ void __launch_bounds__(kUnitsThreads)
+units_from_offsets_kernel(const int32_t *__restrict__ off, int n_groups, int shared_group, int n_rows,
+                          DecUnit *__restrict__ units, Ctrl *__restrict__ ctrl) {
+  __shared__ int s_warp[kUnitsThreads / 32];
+  __shared__ int s_base, s_bad;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    s_base = 0;
+    s_bad = 0x7fffffff;
+  }
+  __syncthreads();
+  for (int gi = tid; gi < n_groups; gi += kUnitsThreads) {  // malformed offsets: flag, run nothing
     const int a = off[gi], b = off[gi + 1];
-    if (a < 0 || b < a || b > n_rows) {  // malformed offsets: flag and run nothing
-      set_device_error(ctrl, MOE_ERR_DEVICE_CHECK, gi);
-      nu = 0;
-      break;
+    if (a < 0 || b < a || b > n_rows) atomicMin(&s_bad, gi);
+  }
+  __syncthreads();
+  if (s_bad != 0x7fffffff) {
+    if (tid == 0) {
+      set_device_error(ctrl, MOE_ERR_DEVICE_CHECK, s_bad);
+      ctrl->n_units = 0;
     }
-    for (int r = a; r < b; r += 8) {
+    return;
+  }
+  for (int c0 = 0; c0 < n_groups; c0 += kUnitsThreads) {
+    const int gi = c0 + tid;
+    int a = 0, cnt = 0, nrow = 0;
+    if (gi < n_groups) {
+      a = off[gi];
+      nrow = off[gi + 1] - a;
+      cnt = (nrow + 7) / 8;
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int v = s_warp[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+      }
+      s_warp[lane] = v;  // inclusive sums of the warps' totals
+    }
+    __syncthreads();
+    const int first = s_base + (warp ? s_warp[warp - 1] : 0) + incl - cnt;
+    for (int j = 0; j < cnt; ++j) {
       DecUnit un;
       un.expert = (gi == shared_group) ? 0 : gi;
       un.set = (gi == shared_group) ? 1 : 0;
-      const int n = min(8, b - r);
+      const int n = min(8, nrow - 8 * j);
       un.mask = (1 << n) - 1;
-      un.xrow0 = r;
+      un.xrow0 = a + 8 * j;
 #pragma unroll
       for (int c = 0; c < 8; ++c) un.w[c] = 1.0f;
-      units[nu++] = un;
+      units[first + j] = un;
     }
+    __syncthreads();  // every thread has read s_base and s_warp
+    if (tid == kUnitsThreads - 1) s_base = first + cnt;
+    __syncthreads();
   }
-  ctrl->n_units = nu;
+  if (tid == 0) ctrl->n_units = s_base;
 }
 
 cudaError_t launch_decode_units_from_offsets(const int32_t *offsets, int n_groups, int has_shared_group, int n_rows,
                                              DecUnit *units, Ctrl *ctrl, cudaStream_t s) {
   {
     KTimer kt_(KID_DEC_UNITS, s);
-    units_from_offsets_kernel<<<1, 32, 0, s>>>(offsets, n_groups, has_shared_group ? n_groups - 1 : -1, n_rows, units,
-                                               ctrl);
+    units_from_offsets_kernel<<<1, kUnitsThreads, 0, s>>>(offsets, n_groups, has_shared_group ? n_groups - 1 : -1,
+                                                          n_rows, units, ctrl);
   }
   return cudaGetLastError();
 }

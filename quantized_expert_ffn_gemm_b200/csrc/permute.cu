@@ -106,28 +106,40 @@ perm_scan_kernel(int32_t *__restrict__ hist, int nchunks, int E, int P, int T, i
   }
   __syncthreads();
   // pass 2: first row of every (expert, chunk): the expert's offset + the exclusive prefix over
-  // chunks (the chunk counts of up to 128 chunks are loaded before any is scanned)
-  for (int e = warp; e < E; e += nw) {
-    int32_t *h = hist + (size_t)e * nchunks;
-    int run = s_cnt[e];
-    for (int c0 = 0; c0 < nchunks; c0 += 128) {
-      int xv[4];
+  // chunks. Four experts per warp iteration, and each expert's chunk counts (up to 128 at a
+  // time) are loaded before any is scanned, so a warp has up to 16 loads in flight.
+  for (int e0 = warp; e0 < E; e0 += 4 * nw) {
+    int run[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int c = c0 + 32 * i + lane;
-        xv[i] = (c < nchunks) ? h[c] : 0;
+    for (int u = 0; u < 4; ++u) run[u] = (e0 + u * nw < E) ? s_cnt[e0 + u * nw] : 0;
+    for (int c0 = 0; c0 < nchunks; c0 += 128) {
+      int xv[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * nw;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int c = c0 + 32 * i + lane;
+          xv[u][i] = (e < E && c < nchunks) ? hist[(size_t)e * nchunks + c] : 0;
+        }
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int c = c0 + 32 * i + lane;
-        int incl = xv[i];
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * nw;
+        if (e >= E) break;  // warp-uniform
+        int32_t *h = hist + (size_t)e * nchunks;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int n = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += n;
+        for (int i = 0; i < 4; ++i) {
+          const int c = c0 + 32 * i + lane;
+          int incl = xv[u][i];
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+          }
+          if (c < nchunks) h[c] = run[u] + incl - xv[u][i];
+          run[u] += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (c < nchunks) h[c] = run + incl - xv[i];
-        run += __shfl_sync(0xffffffffu, incl, 31);
       }
     }
   }
@@ -255,20 +267,24 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const uint16
 
 // ---------------------------------------------------------------- combine
 // y[t,h] = sum_j w[t,j] out[row_of[t,j], h] (fixed j order) + shared[t,h] + residual[t,h]
-// One warp per token: lanes j < k hold the token's rows and weights (broadcast by shuffle), each
-// lane then owns 8-column chunks and issues the k row loads of a chunk before accumulating them.
+// One warp per (token, 256-column segment) item, so a small batch still spreads over many warps:
+// lanes j < k hold the token's rows and weights (broadcast by shuffle), each lane owns one
+// 8-column chunk and issues the k row loads of it before accumulating them.
 __global__ void __launch_bounds__(256)
 combine_kernel(const uint16_t *__restrict__ out, const int32_t *__restrict__ row_of, const float *__restrict__ w,
                int T, int k, int H, const uint16_t *__restrict__ shared, const float *residual, float *y) {
-  const int lane = threadIdx.x & 31, H8 = H >> 3;
-  for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += gridDim.x * 8) {
+  const int lane = threadIdx.x & 31, H8 = H >> 3, nseg = (H8 + 31) >> 5;
+  const long long n_items = (long long)T * nseg;
+  for (long long it = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); it < n_items; it += (long long)gridDim.x * 8) {
+    const int t = (int)(it / nseg), c = (int)(it % nseg) * 32 + lane;
     const int my_row = (lane < k) ? row_of[(size_t)t * k + lane] : -1;
     const float my_w = (lane < k) ? w[(size_t)t * k + lane] : 0.0f;
-    for (int c = lane; c < H8; c += 32) {
+    const bool cok = c < H8;  // every lane stays for the shuffles
+    {
       float acc[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
-      if (residual) {
+      if (residual && cok) {
         const float4 r0 = reinterpret_cast<const float4 *>(residual + (size_t)t * H)[2 * c];
         const float4 r1 = reinterpret_cast<const float4 *>(residual + (size_t)t * H)[2 * c + 1];
         acc[0] = r0.x; acc[1] = r0.y; acc[2] = r0.z; acc[3] = r0.w;
@@ -281,7 +297,7 @@ combine_kernel(const uint16_t *__restrict__ out, const int32_t *__restrict__ row
         for (int u = 0; u < 4; ++u) {
           const int rj = __shfl_sync(0xffffffffu, my_row, (j0 + u) & 31);
           wj[u] = __shfl_sync(0xffffffffu, my_w, (j0 + u) & 31);
-          const bool use = j0 + u < k && rj >= 0;  // rows past k or flagged (-1) add nothing
+          const bool use = cok && j0 + u < k && rj >= 0;  // rows past k or flagged (-1) add nothing
           v[u] = use ? __ldg(reinterpret_cast<const uint4 *>(out + (size_t)rj * H) + c) : make_uint4(0, 0, 0, 0);
           if (!use) wj[u] = 0.0f;
         }
@@ -296,7 +312,7 @@ combine_kernel(const uint16_t *__restrict__ out, const int32_t *__restrict__ row
           }
         }
       }
-      if (shared) {
+      if (shared && cok) {
         const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(shared + (size_t)t * H) + c);
         const uint32_t vv[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
@@ -306,16 +322,20 @@ combine_kernel(const uint16_t *__restrict__ out, const int32_t *__restrict__ row
           acc[2 * q + 1] += f.y;
         }
       }
-      float4 *yo = reinterpret_cast<float4 *>(y + (size_t)t * H);
-      yo[2 * c] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      yo[2 * c + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      if (cok) {
+        float4 *yo = reinterpret_cast<float4 *>(y + (size_t)t * H);
+        yo[2 * c] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        yo[2 * c + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      }
     }
   }
 }
 
 cudaError_t launch_combine(const uint16_t *out_perm, const int32_t *row_of, const float *w, int T, int k, int H,
                            const uint16_t *shared_out, const float *residual, float *y, cudaStream_t s) {
-  size_t want = ((size_t)T + 7) / 8, cap = (size_t)num_sms() * 16;
+  // items of (token, 256-column segment), eight warps per block
+  const size_t nseg = ((size_t)(H / 8) + 31) / 32;
+  size_t want = ((size_t)T * nseg + 7) / 8, cap = (size_t)num_sms() * 16;
   int grid = (int)(want < cap ? want : cap);
   {
     KTimer kt_(KID_COMBINE, s);
