@@ -9,7 +9,9 @@
 // Decode (T <= 8): one kernel. Every warp produces whole logits (one expert, all T tokens,
 // Wr read once with 128-bit loads); the last CTA to finish (atomic ticket) runs the top-k and,
 // for the decode expert path, groups the selected (token, slot) pairs by distinct expert.
-// Prefill: a tiled fp32 GEMM for the logits, then one warp per token for the top-k.
+// 9..128 tokens: fp32 dot products with each expert's row held in registers, then one warp per
+// token for the top-k. Prefill: tensor-core logits with an exact refine of the candidates near
+// the k-th (or a tiled fp32 GEMM where that path does not apply), then the top-k.
 #include "common.cuh"
 #include "topk.cuh"
 
@@ -347,9 +349,72 @@ topk_refine_kernel(float *__restrict__ logits, const uint16_t *__restrict__ x, c
 
 bool router_refine_supported(int H, int E) { return H <= 2048 && E <= 512; }
 
+// ---------------------------------------------------------------- small batches (9..128 tokens)
+// Plain fp32 dot products on the CUDA cores: at these sizes the tensor-core router's fixed costs
+// (splitting Wr into planes, a K loop over 3H, the exact refine) dominate. A CTA takes 4 experts;
+// warp (e, half) keeps its expert's fp32 row in registers (Wr read once) and walks the tokens of
+// its half two at a time, both tokens' x loads in flight together. The logits are exact fp32
+// dot products (no refine needed); the bias is added by the top-k kernel.
+constexpr int kRouterMidMaxT = 128;
+constexpr int kRouterMidWarps = 8;
+
+__global__ void __launch_bounds__(kRouterMidWarps * 32)
+router_mid_kernel(const uint16_t *__restrict__ x, int T, int H, const float *__restrict__ Wr, int E,
+                  float *__restrict__ logits) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 4 + (warp & 3), half = warp >> 2;
+  if (e >= E) return;
+  const int H4 = H >> 2;  // H <= 2048: at most 16 float4 per lane
+  const float4 *wr = reinterpret_cast<const float4 *>(Wr + (size_t)e * H);
+  float4 wv[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int h4 = lane + 32 * j;
+    wv[j] = (h4 < H4) ? __ldg(wr + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int t0 = 2 * half; t0 < T; t0 += 4) {  // half 0: tokens 0,1,4,5,...; half 1: 2,3,6,7,...
+    uint2 xv[2][16];
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      const int t = t0 + b;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int h4 = lane + 32 * j;
+        xv[b][j] = (t < T && h4 < H4) ? __ldg(reinterpret_cast<const uint2 *>(x + (size_t)t * H) + h4)
+                                      : make_uint2(0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      float acc = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        acc = fmaf(wv[j].x, __uint_as_float(xv[b][j].x << 16), acc);
+        acc = fmaf(wv[j].y, __uint_as_float(xv[b][j].x & 0xffff0000u), acc);
+        acc = fmaf(wv[j].z, __uint_as_float(xv[b][j].y << 16), acc);
+        acc = fmaf(wv[j].w, __uint_as_float(xv[b][j].y & 0xffff0000u), acc);
+      }
+      acc = warp_sum(acc);
+      if (lane == 0 && t0 + b < T) logits[(size_t)(t0 + b) * E + e] = acc;
+    }
+  }
+}
+
 cudaError_t launch_router_prefill(const uint16_t *x, int T, int H, const float *Wr, const float *bias, int E, int k,
                                   int32_t *idx, float *w, float *logits, uint16_t *wsplit, Ctrl *ctrl, cudaStream_t s) {
   cudaError_t e;
+  if (T <= kRouterMidMaxT && H <= 2048) {
+    {
+      KTimer kt_(KID_ROUTER_GEMM, s);
+      router_mid_kernel<<<(E + 3) / 4, kRouterMidWarps * 32, 0, s>>>(x, T, H, Wr, E, logits);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    {
+      KTimer kt_(KID_TOPK, s);
+      topk_kernel<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(logits, bias, T, E, k, idx, w);
+    }
+    return cudaGetLastError();
+  }
   if (router_tc_supported(H, E) && router_refine_supported(H, E)) {
     e = launch_router_tc(x, T, H, Wr, bias, E, wsplit, logits, ctrl, s);  // logits include the bias
     if (e != cudaSuccess) return e;

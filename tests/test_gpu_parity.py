@@ -76,6 +76,21 @@ def test_router_topk(name):
     assert moe.read_device_error(ws) == 0
 
 
+@pytest.mark.parametrize("T", [12, 100])
+def test_router_topk_mid_batch(T):
+    # 9..128 tokens take the CUDA-core fp32 router (exact fp32 logits, no refine step)
+    L0, (_, Wr, b, _, _) = layer_of("decode4")
+    s = L0.shape
+    x = synth.make_x(s.seed, T, s.H, stream=60 + T)
+    ws = moe.Workspace.for_layer(s.H, s.E, s.k, s.I, s.shared, T)
+    idx, w, logits = moe.router_topk(x.cuda(), Wr, b, s.k, ws, want_logits=True)
+    idx_ref, w_ref, lg_ref, gap = oracle.router_topk(x, L0.Wr, L0.bias, s.k)
+    lg = logits.cpu().double().numpy()
+    assert np.abs(lg - lg_ref).max() < 1e-5 * max(1.0, np.abs(lg_ref).max())
+    compare_routing(idx.cpu().numpy(), w.cpu().numpy(), idx_ref, w_ref, gap, lg_ref)
+    assert moe.read_device_error(ws) == 0
+
+
 def test_router_prefill_8k_all_tokens():
     L, (x, Wr, b, _, _) = layer_of("prefill8k")
     ws = ws_for(L)
@@ -201,12 +216,13 @@ def test_cross_path_gemv_vs_gemm(name, T):
 
 
 @pytest.mark.parametrize("name,T", [("mid", 5), ("mid", 8), ("decode4", 5), ("decode4", 6), ("decode4", 8),
-                                    ("prefill8k", 4), ("prefill8k", 5)])
+                                    ("prefill8k", 4), ("prefill8k", 5), ("decode4", 12), ("prefill2k_q3", 100)])
 def test_layer_forward_decode_batches(name, T):
     # 5-8 tokens take the decode path under AUTO: the fused kernel where its shared-memory plan
     # fits (top-4 layer; top-10 at T=5), the separate decode kernels beyond (top-10 at T=6, 8).
     # With the uniform router of the prefill layer, 5 tokens choose ~50 distinct experts: more
     # down pieces than shared-memory slots, so two pieces of one row block share a slot.
+    # 12 and 100 tokens: the small-batch router, then the grouped GEMM.
     # Fresh tokens on the cached layer's weights, every token against the oracle.
     L0, (_, Wr, b, routed, shared) = layer_of(name)
     s = L0.shape
