@@ -35,14 +35,61 @@ perm_hist_kernel(const int32_t *__restrict__ idx, int P, int E, int32_t *__restr
 // counts[e] = sum_c hist[e][c]; offsets = exclusive scan over e; hist[e][c] <- first row of
 // chunk c in expert e. One warp per expert at a time: its lanes read the expert's chunk counts
 // (contiguous) and scan them with shuffles, so the loads of all warps are in flight together.
+constexpr size_t kScanSmemMax = 200 * 1024;
+
 __global__ void __launch_bounds__(1024)
-perm_scan_kernel(int32_t *__restrict__ hist, int nchunks, int E, int P, int T, int with_shared,
+perm_scan_kernel(int32_t *__restrict__ hist, int nchunks, int E, int P, int T, int with_shared, int staged,
                  int32_t *__restrict__ counts, int32_t *__restrict__ offsets) {
-  extern __shared__ int32_t s_cnt[];  // [E] totals, then exclusive offsets
+  extern __shared__ int32_t s_cnt[];  // [E] totals, then exclusive offsets; then [E][nchunks] if staged
   __shared__ int32_t s_warp[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;  // experts per thread in the scan
+  // one chunk (up to kPermChunk pairs): the chunk counts are the totals, read by the scanning
+  // threads themselves in one round of loads; the two warp passes below are skipped
+  const bool one = nchunks == 1;
+  // several chunks, when the whole histogram fits in shared memory (staged): it is copied in with
+  // one round of 16-byte loads into rows of an odd stride (32 consecutive experts then fall on 32
+  // banks); each thread sums and later prefixes its own experts' rows there, and the prefixes go
+  // back with coalesced stores. The warp passes below serve only histograms too large to stage.
+  const bool stg = staged && !one;
+  const int Pp = nchunks | 1;
+  int32_t *s_h = s_cnt + ((E + 3) & ~3);
+  auto sidx = [&](int q) { return (q / nchunks) * Pp + q % nchunks; };  // global [e][c] -> shared
+  if (stg) {
+    const int n = E * nchunks, n4 = n >> 2;
+    const int4 *g4 = reinterpret_cast<const int4 *>(hist);
+    for (int i0 = tid; i0 < n4; i0 += 8 * (int)blockDim.x) {  // 8 loads in flight per thread
+      int4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = i0 + j * (int)blockDim.x;
+        v[j] = (i < n4) ? g4[i] : make_int4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = i0 + j * (int)blockDim.x;
+        if (i < n4) {
+          s_h[sidx(4 * i)] = v[j].x;
+          s_h[sidx(4 * i + 1)] = v[j].y;
+          s_h[sidx(4 * i + 2)] = v[j].z;
+          s_h[sidx(4 * i + 3)] = v[j].w;
+        }
+      }
+    }
+    for (int q = 4 * n4 + tid; q < n; q += blockDim.x) s_h[sidx(q)] = hist[q];
+    __syncthreads();
+    for (int i = 0; i < per; ++i) {  // this thread's experts: row totals
+      const int e = tid * per + i;
+      if (e < E) {
+        const int32_t *row = s_h + (size_t)e * Pp;
+        int tot = 0;
+        for (int c = 0; c < nchunks; ++c) tot += row[c];
+        s_cnt[e] = tot;
+      }
+    }
+  }
   // pass 1: per-expert totals, four experts per warp iteration so their loads are in flight together
-  for (int e0 = warp; e0 < E; e0 += 4 * nw) {
+  for (int e0 = warp; !one && !stg && e0 < E; e0 += 4 * nw) {
     int sum[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -69,11 +116,10 @@ perm_scan_kernel(int32_t *__restrict__ hist, int nchunks, int E, int P, int T, i
   }
   __syncthreads();
   // exclusive scan of the E totals (contiguous runs per thread, then a block scan of the runs)
-  const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;
   int mysum = 0;
   for (int i = 0; i < per; ++i) {
     const int e = tid * per + i;
-    if (e < E) mysum += s_cnt[e];
+    if (e < E) mysum += one ? hist[e] : s_cnt[e];
   }
   int v = mysum;
 #pragma unroll
@@ -97,18 +143,37 @@ perm_scan_kernel(int32_t *__restrict__ hist, int nchunks, int E, int P, int T, i
   for (int i = 0; i < per; ++i) {
     const int e = tid * per + i;
     if (e < E) {
-      const int c = s_cnt[e];
+      const int c = one ? hist[e] : s_cnt[e];
       counts[e] = c;
       offsets[e] = base;
-      s_cnt[e] = base;  // this thread alone reads and rewrites entry e
+      if (one) {
+        hist[e] = base;  // the chunk's first row in expert e
+      } else if (stg) {  // first row of every chunk of expert e, in place in its shared row
+        int32_t *row = s_h + (size_t)e * Pp;
+        int run = base;
+        for (int cc = 0; cc < nchunks; ++cc) {
+          const int v = row[cc];
+          row[cc] = run;
+          run += v;
+        }
+      } else {
+        s_cnt[e] = base;  // this thread alone reads and rewrites entry e
+      }
       base += c;
     }
   }
   __syncthreads();
+  if (stg) {  // the prefixes back to global memory, 16-byte stores
+    const int n = E * nchunks, n4 = n >> 2;
+    int4 *g4 = reinterpret_cast<int4 *>(hist);
+    for (int i = tid; i < n4; i += blockDim.x)
+      g4[i] = make_int4(s_h[sidx(4 * i)], s_h[sidx(4 * i + 1)], s_h[sidx(4 * i + 2)], s_h[sidx(4 * i + 3)]);
+    for (int q = 4 * n4 + tid; q < n; q += blockDim.x) hist[q] = s_h[sidx(q)];
+  }
   // pass 2: first row of every (expert, chunk): the expert's offset + the exclusive prefix over
   // chunks. Four experts per warp iteration, and each expert's chunk counts (up to 128 at a
   // time) are loaded before any is scanned, so a warp has up to 16 loads in flight.
-  for (int e0 = warp; e0 < E; e0 += 4 * nw) {
+  for (int e0 = warp; !one && !stg && e0 < E; e0 += 4 * nw) {
     int run[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) run[u] = (e0 + u * nw < E) ? s_cnt[e0 + u * nw] : 0;
@@ -243,7 +308,15 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const uint16
   }
   {
     KTimer kt_(KID_PERM_SCAN, s);
-    perm_scan_kernel<<<1, 1024, esm, s>>>(hist, nchunks, E, P, T, with_shared, counts, offsets);
+    // the histogram staged in shared memory when it fits (8192 tokens x top-10: 160 KB)
+    const size_t hsm = (size_t)E * (nchunks | 1) * 4, esm4 = (size_t)((E + 3) & ~3) * 4;  // odd row stride
+    const int staged = (nchunks > 1 && esm4 + hsm <= kScanSmemMax) ? 1 : 0;
+    const size_t sm = staged ? esm4 + hsm : esm;
+    if (staged) {
+      const cudaError_t e = smem_limit_once(perm_scan_kernel, kScanSmemMax);
+      if (e != cudaSuccess) return e;
+    }
+    perm_scan_kernel<<<1, 1024, sm, s>>>(hist, nchunks, E, P, T, with_shared, staged, counts, offsets);
   }
   {
     KTimer kt_(KID_PERM_SCATTER, s);
