@@ -317,6 +317,10 @@ topk_refine_kernel(float *__restrict__ logits, const uint16_t *__restrict__ x, c
   float *ex = s_ex[warp];
   for (int e = lane; e < E; e += 32) ex[e] = -INFINITY;
   __syncwarp();
+  // candidate c's exact value is also kept by lane c (the first 32), so the final top-k is one
+  // 32-wide sort of the candidates instead of k rounds over all E entries
+  int nc = 0, ce = 0;
+  float cv = -INFINITY;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     unsigned bal = __ballot_sync(0xffffffffu, (lane + 32 * i < E) && val[i] >= thr);
@@ -337,10 +341,25 @@ topk_refine_kernel(float *__restrict__ logits, const uint16_t *__restrict__ x, c
         }
       }
       acc = warp_sum(acc);
-      if (lane == 0) ex[e] = acc + (bias ? bias[e] : 0.0f);
+      const float v = acc + (bias ? bias[e] : 0.0f);
+      if (lane == 0) ex[e] = v;
+      if (lane == nc) {  // nc is warp-uniform
+        ce = e;
+        cv = v;
+      }
+      ++nc;
     }
   }
-  __syncwarp();
+  if (nc <= 32) {  // the top-k is among the candidates (every approximate top-k value is >= thr)
+    unsigned long long code = (lane < nc) ? topk_code(cv, ce) : 0ull;
+    code = warp_sort32_desc(code);
+    const float my_val = key_to_logit((uint32_t)(code >> 32));
+    const int my_idx = (int)(0xFFFFFFFFu - (uint32_t)code);
+    topk_finish(my_val, my_idx, k, idx + (size_t)t * k, w + (size_t)t * k);
+    if (lane < nc) l[ce] = cv;  // exact values where computed
+    return;
+  }
+  __syncwarp();  // more than 32 candidates (a crowd of near-equal logits): over all E entries
   warp_topk<16>(ex, nullptr, E, k, idx + (size_t)t * k, w + (size_t)t * k);
   __syncwarp();
   for (int e = lane; e < E; e += 32)  // exact values where computed
