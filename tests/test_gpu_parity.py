@@ -105,8 +105,12 @@ def test_router_prefill_8k_all_tokens():
 
 # ----------------------------------------------------------------------------- permute / combine
 @pytest.mark.parametrize("T,k,E,shared", [(8192, 10, 512, True), (37, 3, 16, False), (1, 10, 512, True),
-                                          (5, 1, 4, False)])
+                                          (5, 1, 4, False), (3000, 7, 301, True), (12000, 10, 512, False)])
 def test_permute_bit_exact(T, k, E, shared):
+    # the scan runs one of three ways: a single 1024-pair chunk (read in one round of loads), a
+    # histogram staged in shared memory (8192 x 10 over 512 experts; 3000 x 7 over 301 experts,
+    # an odd size), or, when the histogram is too large to stage (12000 x 10: 118 chunks), warp
+    # passes over global memory
     rng = np.random.default_rng(T + k)
     idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
     x = synth.make_x(1, T, 256)
