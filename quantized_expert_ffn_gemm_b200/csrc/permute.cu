@@ -257,25 +257,29 @@ perm_scatter_kernel(const int32_t *__restrict__ idx, int P, int k, int E, const 
 }
 
 // ---------------------------------------------------------------- gather rows (bf16 -> fp16)
-// one warp per row: the source token is read once, then the row's 16-byte chunks are loaded four
-// at a time per lane before any is converted and stored
+// one warp per row: the row's 16-byte chunks are all loaded (eight per lane at H = 2048) before
+// any is converted and stored, and the warp's next source token is read meanwhile
 __global__ void __launch_bounds__(256)
 perm_gather_kernel(const uint16_t *__restrict__ x, int H, const int32_t *__restrict__ src, int P, int rows,
                    uint16_t *__restrict__ x_perm) {
-  const int lane = threadIdx.x & 31, H8 = H >> 3;
-  for (int r = blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += gridDim.x * 8) {
-    const int t = (r < P) ? src[r] : r - P;
+  const int lane = threadIdx.x & 31, H8 = H >> 3, stride = gridDim.x * 8;
+  int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  int t = (r < rows) ? ((r < P) ? src[r] : r - P) : 0;
+  for (; r < rows; r += stride) {
+    // the next row's source token is requested along with this row's data
+    const int rn = r + stride;
+    const int tn = (rn < rows) ? ((rn < P) ? src[rn] : rn - P) : 0;
     const uint4 *xs = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
     uint4 *xd = reinterpret_cast<uint4 *>(x_perm + (size_t)r * H);
-    for (int c0 = lane; c0 < H8; c0 += 128) {
-      uint4 v[4];
+    for (int c0 = lane; c0 < H8; c0 += 256) {  // H = 2048: the whole row in one round of loads
+      uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const int c = c0 + 32 * u;
         v[u] = (c < H8) ? __ldg(xs + c) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const int c = c0 + 32 * u;
         if (c >= H8) break;
         const uint32_t in[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
@@ -288,6 +292,7 @@ perm_gather_kernel(const uint16_t *__restrict__ x, int H, const int32_t *__restr
         xd[c] = make_uint4(out[0], out[1], out[2], out[3]);
       }
     }
+    t = tn;
   }
 }
 
