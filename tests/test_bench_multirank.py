@@ -88,3 +88,23 @@ def test_replicas_draw_distinct_tokens():
     a = synth.make_x(0, 1, 256, stream=bench.replica_x_stream(0, 0))
     b = synth.make_x(0, 1, 256, stream=bench.replica_x_stream(1, 0))
     assert not torch.equal(a, b)
+
+
+def test_traffic_figure_follows_source_hash_and_launch_shape(tmp_path, monkeypatch):
+    # a committed DRAM-traffic figure is reported only for the launch shape it was captured on
+    # and only while the captured kernel source is unchanged
+    sys.path.insert(0, ROOT)
+    import hashlib
+    import bench
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "TRAFFIC", {("k", ("shape_a",)): (["k.cu"], sha, 1234, "profiles/k.md")})
+    assert bench.traffic_for("k", "shape_a") == 1234
+    assert bench.traffic_for("k", "shape_b") is None      # another launch shape
+    assert bench.traffic_for("other", "shape_a") is None  # no capture of that kernel
+    src.write_text("kernel v2\n")
+    assert bench.traffic_for("k", "shape_a") is None      # the source changed since the capture
+    (tmp_path / "k.cu").unlink()
+    assert bench.traffic_for("k", "shape_a") is None      # source missing
