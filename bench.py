@@ -77,7 +77,7 @@ TRAFFIC = {
         (_GEMM_SRC, "f5ad8aca8c32a2576bfdf9f5a1d66e6cbeb86fb1fb932b6adae357c9fbff935a", 786358272,
          "profiles/grouped_gemm_prefill8k.md"),
     ("decode_fused", ("decode1",)):
-        (_DEC_SRC, "a5d3e5e3c41bbea67c9e7daa51d8d90d767f00d17c80b3c00876d3b84accd6f3", 15117824,
+        (_DEC_SRC, "079b8a42801687ba382781d35128bd3914e45a1093ae366b7f07f8b8b245e47d", 15117824,
          "profiles/decode_fused_kernel_decode1.md"),
 }
 

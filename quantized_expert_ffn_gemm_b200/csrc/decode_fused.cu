@@ -25,7 +25,12 @@
 //       summed in fixed order and h goes to the workspace.
 //   --  grid barrier
 //   P3  down projection fused with the weighted combine: each CTA owns 16 output features, its
-//       warps split the (unit, K step) items, partials are reduced in fixed order (no atomics).
+//       warps take whole units (16 down rows over all of I, the half steps' loads issued
+//       together), partials are reduced in fixed order (no atomics).
+// Each slot's fills are consumed in phase order: the ring has an even number of slots so the
+// gate/up items sharing a slot fall to one group, and a down piece first waits until the piece
+// one ring behind it is consumed. A parity wait can then never run two phases ahead of its
+// slot's last completed fill, where it would take the older phase for its own.
 // The grid barrier is one 64-bit arrival counter in the workspace (every launch adds 2 x grid;
 // a CTA waits for the launch's base + j x grid). It and every mbarrier wait are bounded in time
 // and report MOE_ERR_TIMEOUT instead of hanging; before the CTA exits every thread waits for its
