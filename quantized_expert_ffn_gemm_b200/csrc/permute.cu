@@ -33,8 +33,11 @@ perm_hist_kernel(const int32_t *__restrict__ idx, int P, int E, int32_t *__restr
 
 // ---------------------------------------------------------------- scan (one CTA)
 // counts[e] = sum_c hist[e][c]; offsets = exclusive scan over e; hist[e][c] <- first row of
-// chunk c in expert e. One warp per expert at a time: its lanes read the expert's chunk counts
-// (contiguous) and scan them with shuffles, so the loads of all warps are in flight together.
+// chunk c in expert e. The kernel is bound by dependent round trips to memory, so it makes as
+// few as it can: a single chunk is read by the scanning threads in one round of loads; a
+// histogram that fits in shared memory is staged there in one round and scanned row by row; a
+// larger one is walked by warps (one expert per warp at a time, its lanes reading the expert's
+// chunk counts and scanning them with shuffles, four experts' loads in flight together).
 constexpr size_t kScanSmemMax = 200 * 1024;
 
 __global__ void __launch_bounds__(1024)
