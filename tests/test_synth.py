@@ -52,3 +52,18 @@ def test_workload_shapes():
     assert L.routed.gate.codes.shape == (16, 128, 64)
     assert L.routed.down.codes.shape == (16, 256, 32)
     assert L.shared is None and L.bias is None
+
+
+def test_workload_table_matches_the_stated_configs():
+    # the shapes the tests and the benchmark use, as the design notes state them
+    W = synth.WORKLOADS
+    for name in ("decode1", "decode4", "verify6", "decode1_pruned256"):
+        s = W[name]
+        assert (s.H, s.k, s.I, s.qtype, s.shared, s.zipf_s) == (2048, 10, 512, synth.Q2, True, 1.1)
+    assert [W[n].T for n in ("decode1", "decode4", "verify6", "decode1_pruned256")] == [1, 4, 6, 1]
+    assert W["decode1"].E == W["decode4"].E == W["verify6"].E == 512 and W["decode1_pruned256"].E == 256
+    p = W["prefill8k"]
+    assert (p.T, p.H, p.E, p.k, p.I, p.qtype, p.shared, p.zipf_s) == (8192, 2048, 512, 10, 512, synth.Q2, True, None)
+    q = W["prefill2k_q3"]
+    assert (q.T, q.E, q.k, q.qtype, q.shared, q.zipf_s) == (2048, 512, 10, synth.Q3, False, 1.2)
+    assert synth.STACK["L"] == 48 and synth.STACK["eps"] == 1e-6
