@@ -175,11 +175,14 @@ moe_status moe_combine(const uint16_t *out_perm, const int32_t *row_of, const fl
                        int32_t H, const uint16_t *shared_out_opt, const float *residual_opt, float *y,
                        void *stream);
 
-/* One full MoE layer: router + top-k, then either the decode path (T <= 8 and path != GEMM, or
- * path == GEMV: dequant-GEMV over the distinct selected experts, down projection fused with the
- * weighted combine; for small enough T one cooperative kernel does the whole layer) or the
- * prefill path (permute, tcgen05 grouped GEMM gate/up with fused SwiGLU, grouped GEMM down,
- * combine).
+/* One full MoE layer. T <= 8 with path AUTO or GEMV: the decode path (router + top-k, then a
+ * dequant-GEMV over the distinct selected experts with the tokens as MMA columns, down
+ * projection fused with the weighted combine; under AUTO one cooperative kernel does the whole
+ * layer where its shared-memory plan fits). Otherwise: router + top-k (fp32 dot products on the
+ * CUDA cores up to 128 tokens, tensor-core logits with an exact refine of the candidates above),
+ * permute, the expert FFN (AUTO / GEMM: tcgen05 grouped GEMM gate/up with fused SwiGLU, then
+ * down; GEMV: the decode GEMV kernels over 8-row chunks of each expert's rows), combine. Every
+ * path computes the same function within the parity tolerance.
  *   y = sum_j w_j FFN_{idx_j}(x) + FFN_shared(x) (+ residual)      fp32 [T,H]
  * x bf16 [T,H]; Wr fp32 [E,H]; bias fp32 [E] or NULL; routed: gate/up [E][I][H], down [E][H][I];
  * shared_opt: one expert (n_experts = 1) when desc->has_shared; residual_opt fp32 [T,H] or NULL
