@@ -136,3 +136,31 @@ def test_stack_validation(lib):
                                  FAKE, ctypes.c_size_t(1 << 40), None) == 1
     assert lib.moe_stack_forward(FAKE, 4, -1, None, None, ctypes.byref(d), None, None, ctypes.c_float(1e-6), FAKE, 0,
                                  FAKE, ctypes.c_size_t(1 << 40), None) == 1
+
+
+def test_static_router_validation(lib):
+    # host-side checks of the workspace-free router; none of these calls reaches the device
+    def call(x=FAKE, T=1, H=2048, Wr=FAKE, E=512, k=10, idx=FAKE, w=FAKE):
+        return lib.moe_router_topk_static(x, T, H, Wr, None, E, k, idx, w, None, None)
+    assert call(H=100) == moe.MOE_ERR_INVALID_ARG        # H not a multiple of 64
+    assert call(k=0) == moe.MOE_ERR_INVALID_ARG
+    assert call(k=11, E=10) == moe.MOE_ERR_INVALID_ARG   # k > E
+    assert call(T=-1) == moe.MOE_ERR_INVALID_ARG
+    assert call(T=9) == moe.MOE_ERR_UNSUPPORTED           # beyond the fixed scratch
+    assert call(T=0) == moe.MOE_OK                        # nothing to do
+    assert call(x=None) == moe.MOE_ERR_INVALID_ARG
+    assert call(x=FAKE_MIS) == moe.MOE_ERR_ALIGNMENT
+
+
+def test_kernel_names_and_timing_queries(lib):
+    n = lib.moe_kernel_count()
+    names = [lib.moe_kernel_name(i) for i in range(n)]
+    assert n > 0 and all(names) and len(set(names)) == n  # every kernel id has its own name
+    assert lib.moe_kernel_name(n) is None and lib.moe_kernel_name(-1) is None
+    ms, cnt = ctypes.c_double(0.0), ctypes.c_int32(0)
+    assert lib.moe_timing_read(-1, ctypes.byref(ms), ctypes.byref(cnt)) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_timing_read(n, ctypes.byref(ms), ctypes.byref(cnt)) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_timing_read(0, None, ctypes.byref(cnt)) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_timing_enable(0) == moe.MOE_OK
+    assert lib.moe_timing_read(0, ctypes.byref(ms), ctypes.byref(cnt)) == moe.MOE_OK
+    assert cnt.value == 0 and ms.value == 0.0             # nothing was timed
