@@ -12,7 +12,8 @@ module only marshals numpy arrays through ctypes. Each function names the passag
     Strata Engine Benchmarked", section "Where Strata Is Fast: Not Magic, but Logistics";
   - MTP verify passes give the same output as one-token passes: Strata DETAILS.md,
     "How it works" (speculation bullet);
-  - Q2/Q3 block formats: the stated stand-in (32 weights, fp16 scale d, w = d(c-2) / d(c-4)).
+  - Q2/Q3 block formats: the stated stand-in (32 weights, fp16 scale d, w = d(c-2) / d(c-4));
+    Q4 (4-bit codes, w = d(c-8)) is a further stand-in of the same family.
 
 Parity status: every function here is pinned by `tests/test_oracle_pins.py` against closed
 forms, brute force and textbook/library routines (the pages print no worked example).

@@ -16,7 +16,8 @@
  *     "Two-Day Port, 8x Faster Prefill: Strata Engine Benchmarked", section
  *     "Where Strata Is Fast: Not Magic, but Logistics" (MMQ paragraph).
  *   - block formats (stand-in): Q2 = 32 weights of 2-bit codes c and one fp16 scale d,
- *     w = d*(c-2); Q3 = 3-bit codes, w = d*(c-4).
+ *     w = d*(c-2); Q3 = 3-bit codes, w = d*(c-4); Q4 (a further stand-in of the same family)
+ *     = 4-bit codes, w = d*(c-8).
  *
  * Arithmetic is fp64 throughout (exact products of exactly-decoded inputs, fp64 sums), except
  * where a rounding is part of the definition (the bf16 output of RMSNorm) or where the
@@ -29,6 +30,8 @@
  *   word q (weights 16q..16q+15) holds weight 16q+2i+h (i=0..7, h=0..1) at bits 16h+2i..16h+2i+1.
  *   Q3 adds a 1-bit plane, one 32-bit little-endian word per block, holding bit 2 of the code of
  *   weight 16q+2i+h at bit 16h+8q+i.  code = low2 | hibit<<2.
+ *   Q4 has one 4-bit plane [n][rows][K/2]: per block four 32-bit little-endian words; word q
+ *   (weights 8q..8q+7) holds weight 8q+2i+h (i=0..3, h=0..1) at bits 16h+4i..16h+4i+3.
  */
 #include <math.h>
 #include <stdint.h>
@@ -39,9 +42,9 @@
 #endif
 
 typedef struct {
-  int32_t qtype;          /* 2 (Q2) or 3 (Q3) */
+  int32_t qtype;          /* 2 (Q2), 3 (Q3) or 4 (Q4) */
   int32_t n_experts, rows, K;
-  const uint8_t *codes;   /* [n][rows][K/4] */
+  const uint8_t *codes;   /* [n][rows][K/4]; Q4: [n][rows][K/2] */
   const uint8_t *hibits;  /* [n][rows][K/8], Q3 only */
   const uint16_t *scales; /* [n][rows][K/32], fp16 bit patterns */
 } oq_mat;
@@ -109,6 +112,11 @@ static double round_f16(double v) { return oracle_half_to_double(oracle_double_t
 int oracle_code(const oq_mat *m, int e, int r, int k) {
   size_t row = (size_t)e * m->rows + r;
   int b = k >> 5, j = k & 31;
+  if (m->qtype == 4) {  /* word j/8 of the block, pair (i, h) = ((j%8)/2, j%2) at bit 16h+4i */
+    const uint8_t *w4 = m->codes + row * (size_t)(m->K / 2) + (size_t)b * 16 + (size_t)(j >> 3) * 4;
+    int bit = 16 * (j & 1) + 4 * ((j & 7) >> 1);
+    return (w4[bit >> 3] >> (bit & 7)) & 15;
+  }
   int q = j >> 4, jj = j & 15, h = jj & 1, i = jj >> 1;
   const uint8_t *w = m->codes + row * (size_t)(m->K / 4) + (size_t)b * 8 + (size_t)q * 4;
   int bit = 16 * h + 2 * i;
@@ -120,11 +128,11 @@ int oracle_code(const oq_mat *m, int e, int r, int k) {
   return lo | (hi << 2);
 }
 
-/* w = d * (c - q0), q0 = 2 (Q2) or 4 (Q3), d the block's fp16 scale */
+/* w = d * (c - q0), q0 = 2 (Q2), 4 (Q3) or 8 (Q4), d the block's fp16 scale */
 double oracle_weight(const oq_mat *m, int e, int r, int k) {
   size_t row = (size_t)e * m->rows + r;
   double d = oracle_half_to_double(m->scales[row * (size_t)(m->K / 32) + (k >> 5)]);
-  int q0 = (m->qtype == 2) ? 2 : 4;
+  int q0 = (m->qtype == 2) ? 2 : (m->qtype == 3) ? 4 : 8;
   return d * (double)(oracle_code(m, e, r, k) - q0);
 }
 

@@ -1,7 +1,7 @@
 """Seeded synthetic inputs for the quantized MoE layer (shared by the oracle and the CUDA path).
 
 This module holds no arithmetic of the method. It only draws inputs: activations, router
-weights, per-expert router biases and packed Q2/Q3 expert weights, each from one
+weights, per-expert router biases and packed Q2/Q3/Q4 expert weights, each from one
 counter-based generator, so any slice (one expert, one token) can be regenerated alone and
 the bits do not depend on the device or on the number of threads.
 
@@ -49,7 +49,7 @@ K_RESID = 7
 MAT_GATE, MAT_UP, MAT_DOWN = 0, 1, 2
 SET_ROUTED, SET_SHARED = 0, 1
 
-Q2, Q3 = 2, 3
+Q2, Q3, Q4 = 2, 3, 4
 
 
 def tid(kind: int, layer: int = 0, mat: int = 0, index: int = 0) -> int:
@@ -134,7 +134,8 @@ def scales_f16(seed: int, tids, n: int, device="cpu", lo: float = 0.005, hi: flo
 class QMat:
     """One matrix kind (gate, up or down) for n experts: rows output features, K reduction dim.
 
-    codes  uint8 [n, rows, K/4]   2-bit plane (Q2 codes, or the low 2 bits of Q3 codes)
+    codes  uint8 [n, rows, K/4]   2-bit plane (Q2 codes, or the low 2 bits of Q3 codes);
+                                  Q4: [n, rows, K/2], the 4-bit codes
     hibits uint8 [n, rows, K/8]   Q3 only: bit 2 of each code; None for Q2
     scales fp16  [n, rows, K/32]  one scale per block of 32 weights along K
     """
@@ -180,11 +181,12 @@ class ExpertSet:
 def make_qmat(seed: int, layer: int, set_id: int, mat: int, qtype: int, n: int, rows: int, K: int,
               device="cpu", experts=None) -> QMat:
     """Packed weights of experts `experts` (default 0..n-1); codes uniform, d ~ U(0.005, 0.02)."""
-    assert K % 32 == 0 and qtype in (Q2, Q3)
+    assert K % 32 == 0 and qtype in (Q2, Q3, Q4)
     ex = list(range(n)) if experts is None else list(experts)
     m = set_id * 3 + mat
-    codes = random_bytes(seed, [tid(K_CODES, layer, m, e) for e in ex], rows * K // 4, device)
-    codes = codes.reshape(len(ex), rows, K // 4)
+    cb = K // 2 if qtype == Q4 else K // 4  # bytes of the code plane per row (4-bit or 2-bit codes)
+    codes = random_bytes(seed, [tid(K_CODES, layer, m, e) for e in ex], rows * cb, device)
+    codes = codes.reshape(len(ex), rows, cb)
     hib = None
     if qtype == Q3:
         hib = random_bytes(seed, [tid(K_HIBITS, layer, m, e) for e in ex], rows * K // 8, device)

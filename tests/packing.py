@@ -1,5 +1,7 @@
 """Test-side packer for the Q2/Q3 block planes, written from the layout definition in
-include/moe_ffn.h (independently of the oracle's and the CUDA library's decoders).
+include/moe_ffn.h, and for the Q4 plane from its stated layout (4-bit codes; per 32-weight block
+four 32-bit words, word q holding weight 8q+2i+h at bits 16h+4i), independently of the oracle's
+and the CUDA library's decoders.
 
 Used to build weights whose integer codes the test knows, so a decoder can be checked against
 values that never went through it.
@@ -33,6 +35,18 @@ def pack_hi_plane(codes: np.ndarray) -> np.ndarray:
     return words.view(np.uint8).reshape(*lead, K // 8)
 
 
+def pack_q4_plane(codes: np.ndarray) -> np.ndarray:
+    """codes int [..., K] (values 0..15) -> uint8 [..., K/2] 4-bit plane; per block four words,
+    word q holds weight 8q+2i+h at bits 16h+4i."""
+    c = np.asarray(codes, np.int64) & 15
+    *lead, K = c.shape
+    assert K % 32 == 0
+    c = c.reshape(*lead, K // 8, 4, 2)           # [..., word, i, h]
+    shifts = (16 * np.arange(2)[None, :] + 4 * np.arange(4)[:, None])  # [i, h]
+    words = (c << shifts).sum(axis=(-2, -1)).astype(np.uint32)  # [..., K/8]
+    return words.view(np.uint8).reshape(*lead, K // 2)
+
+
 class KnownQMat:
     """A QMat-like object built from known integer codes and fp16 scales."""
 
@@ -41,14 +55,14 @@ class KnownQMat:
         self.qtype = qtype
         self.n, self.rows, self.K = codes.shape
         self.int_codes = codes
-        self.codes = pack_lo_plane(codes)
+        self.codes = pack_q4_plane(codes) if qtype == 4 else pack_lo_plane(codes)
         self.hibits = pack_hi_plane(codes) if qtype == 3 else None
         self.scales = np.asarray(scales_f16, np.float16).view(np.uint16)
         assert self.scales.shape == (self.n, self.rows, self.K // 32)
 
     def dense(self) -> np.ndarray:
         """fp64 weights [n, rows, K] = d * (c - q0), from the known codes (no decoding)."""
-        q0 = 2 if self.qtype == 2 else 4
+        q0 = {2: 2, 3: 4, 4: 8}[self.qtype]
         d = self.scales.view(np.float16).astype(np.float64)
         return np.repeat(d, 32, axis=-1) * (self.int_codes - q0)
 
@@ -59,7 +73,7 @@ class KnownSet:
 
 
 def random_known_set(rng, qtype, n, H, I, scale_range=(0.005, 0.02)):
-    cmax = 4 if qtype == 2 else 8
+    cmax = {2: 4, 3: 8, 4: 16}[qtype]
 
     def mat(rows, K):
         codes = rng.integers(0, cmax, size=(n, rows, K))

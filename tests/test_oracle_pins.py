@@ -81,21 +81,22 @@ class _Raw:
 def test_dequant_hand_built_blocks(case):
     name, qt, lo, hi, codes = case
     d16 = np.float16(0.0137)
-    m = _Raw(qt, lo.reshape(1, 1, 8), None if hi is None else hi.reshape(1, 1, 4),
+    m = _Raw(qt, lo.reshape(1, 1, lo.size), None if hi is None else hi.reshape(1, 1, 4),
              np.array([[[d16.view(np.uint16)]]], np.uint16), 1, 32)
+    assert lo.size == (16 if qt == 4 else 8)
     for k in range(32):
         assert oracle.code(m, 0, 0, k) == codes[k], (name, k)
     vals, v16 = oracle.dequant_rows(m, 0, 0, 1)
-    q0 = 2 if qt == 2 else 4
+    q0 = {2: 2, 3: 4, 4: 8}[qt]
     expect = float(d16) * (np.array(codes) - q0)
     assert np.array_equal(vals[0], expect)                      # exact closed form d*(c-q0)
     assert np.array_equal(v16[0], expect.astype(np.float16).view(np.uint16))  # RNE to fp16
 
 
-@pytest.mark.parametrize("qtype", [2, 3])
+@pytest.mark.parametrize("qtype", [2, 3, 4])
 def test_pack_decode_roundtrip_every_code_every_position(qtype):
     # every code value at every one of the 32 positions, several scale magnitudes and signs
-    cmax = 4 if qtype == 2 else 8
+    cmax = {2: 4, 3: 8, 4: 16}[qtype]
     rows = cmax * 32
     codes = np.zeros((1, rows, 64), np.int64)
     for c in range(cmax):
@@ -112,15 +113,16 @@ def test_pack_decode_roundtrip_every_code_every_position(qtype):
     assert np.array_equal(vals, km.dense()[0])
 
 
-def test_synth_planes_have_uniform_codes():
-    qm = synth.make_qmat(0, 0, 0, 0, 3, 2, 64, 256)
-    cnt = np.zeros(8)
+@pytest.mark.parametrize("qtype,ncodes,bound", [(3, 8, 30.0), (4, 16, 45.0)])
+def test_synth_planes_have_uniform_codes(qtype, ncodes, bound):
+    qm = synth.make_qmat(0, 0, 0, 0, qtype, 2, 64, 256)
+    cnt = np.zeros(ncodes)
     for r in range(64):
         for k in range(256):
             cnt[oracle.code(qm, 1, r, k)] += 1
-    expect = cnt.sum() / 8
+    expect = cnt.sum() / ncodes
     chi2 = ((cnt - expect) ** 2 / expect).sum()
-    assert chi2 < 30.0  # 7 dof; p ~ 1e-4
+    assert chi2 < bound  # 7 / 15 dof; p ~ 1e-4
 
 
 # ----------------------------------------------------------------------------- router / top-k
@@ -255,7 +257,7 @@ def _bf16_rows(rng, T, H):
     return x, x.double().numpy()
 
 
-@pytest.mark.parametrize("qtype", [2, 3])
+@pytest.mark.parametrize("qtype", [2, 3, 4])
 def test_one_hot_router_reduces_to_dense_swiglu(qtype):
     rng = np.random.default_rng(10 + qtype)
     T, H, E, I = 5, 64, 4, 32
@@ -278,7 +280,7 @@ def test_expert_rows_hook_matches_dense():
     assert np.allclose(out, dense_ffn(ks, 1, xd), rtol=1e-12, atol=1e-14)
 
 
-@pytest.mark.parametrize("qtype", [2, 3])
+@pytest.mark.parametrize("qtype", [2, 3, 4])
 def test_sparse_layer_equals_dense_mask_definition(qtype):
     # y_t = sum_{e<E} [e in S(t)] w_{t,e} FFN_e(x_t) + FFN_shared(x_t), all E experts evaluated densely
     rng = np.random.default_rng(20 + qtype)
@@ -310,7 +312,7 @@ def test_zero_scales_leave_shared_only_and_zero_codes_give_zero():
     y, _, _, _ = oracle.layer_forward(x, Wr, None, 2, ks, sh)
     assert np.allclose(y, dense_ffn(sh, 0, xd), rtol=1e-12, atol=1e-14)
     # every code equal to the offset q0 -> all weights are exactly zero -> y = residual
-    for qtype, q0 in ((2, 2), (3, 4)):
+    for qtype, q0 in ((2, 2), (3, 4), (4, 8)):
         def m(rows, K):
             return KnownQMat(qtype, np.full((E, rows, K), q0), np.full((E, rows, K // 32), 0.01, np.float16))
         zs = KnownSet(m(I, H), m(I, H), m(H, I))
