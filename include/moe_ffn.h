@@ -76,7 +76,7 @@ enum {
   MOE_ERR_INVALID_ARG = 1,   /* null pointer, bad size, k out of range, H or I not a multiple of 32 */
   MOE_ERR_ALIGNMENT = 2,     /* a device pointer is not 16-byte aligned */
   MOE_ERR_WORKSPACE = 3,     /* workspace missing or smaller than moe_workspace_bytes() */
-  MOE_ERR_UNSUPPORTED = 4,   /* valid request this build cannot run (e.g. forced GEMM path, H % 128 != 0) */
+  MOE_ERR_UNSUPPORTED = 4,   /* valid request the library cannot run (e.g. forced GEMM path, H % 128 != 0) */
   MOE_ERR_CUDA = 5,          /* a CUDA runtime/driver call failed (launch error, no device) */
   MOE_ERR_DEVICE_CHECK = 6,  /* reported by moe_read_device_error: a device-side index check failed */
   MOE_ERR_TIMEOUT = 7        /* reported by moe_read_device_error: a bounded device wait gave up */

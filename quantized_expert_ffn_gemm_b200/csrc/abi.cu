@@ -92,7 +92,7 @@ bool shape_ok(int H, int E, int k, int I) {
          I % 64 == 0 && I <= 16384;
 }
 
-// H or I a multiple of 32 but not of 64 is a valid layer this build does not run
+// H or I a multiple of 32 but not of 64 is a valid layer the library does not run
 moe_status shape_status(int H, int E, int k, int I) {
   if (shape_ok(H, E, k, I)) return MOE_OK;
   if (H > 0 && H % 32 == 0 && I > 0 && I % 32 == 0 && E >= 1 && E <= kMaxE && k >= 1 && k <= kMaxK && k <= E)
