@@ -15,6 +15,8 @@ come from HBM as in a real 48-layer decode; prefill steps rotate over 4 layers (
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 Under torchrun each rank runs an independent replica (the layer shards by tokens with no
 exchange); rank 0 prints one JSON line with the whole-job throughput (max time over ranks).
+On one GPU the default run (decode1) also times decode4 (480 steps) and prefill8k (8 steps) and
+reports them under "breakdown", so one line carries the metric at T = 1, 4 and 8192.
 """
 from __future__ import annotations
 
@@ -54,6 +56,12 @@ DEFAULT_WARMUP = {"decode1": 480, "decode4": 480, "verify6": 480, "decode1_prune
                   "stack_prefill": 3}
 
 
+# extra workloads timed after the T=1 headline (steps, warm-up steps), and the keys kept for each
+BREAKDOWN = {"decode4": (480, 48), "prefill8k": (8, 3)}
+BREAKDOWN_KEYS = ("value", "unit", "steps", "warmup", "ms_per_step", "config", "roofline", "roofline_layer",
+                  "kernels_us_per_step", "e2e", "gpu_launches", "clocks")
+
+
 def workload_shape(name: str) -> synth.LayerShape:
     wl = WORKLOADS[name]
     if wl.get("stack"):
@@ -62,23 +70,21 @@ def workload_shape(name: str) -> synth.LayerShape:
     return synth.WORKLOADS[wl["shape"]]
 
 
-# DRAM bytes (read + write) per launch of the dominant kernels, from the committed ncu captures
-# (profiles/*.md), valid only for the kernel source and the launch shape they were taken on: the
-# sources' sha256 is checked at run time and the figure is dropped (traffic = null) once the
-# source has changed, or for a workload whose launches differ from the captured one.
+# DRAM bytes (read + write) per launch of the dominant kernels, from ncu captures of these kernel
+# sources, valid only for the source and the launch shape they were taken on: the sources' sha256
+# is checked at run time and the figure is dropped (traffic = null) once the source has changed,
+# or for a workload whose launches differ from the captured one.
 _DEC_SRC = ["quantized_expert_ffn_gemm_b200/csrc/decode_fused.cu", "quantized_expert_ffn_gemm_b200/csrc/common.cuh",
             "quantized_expert_ffn_gemm_b200/csrc/dequant.cuh", "quantized_expert_ffn_gemm_b200/csrc/gemv.cuh",
             "quantized_expert_ffn_gemm_b200/csrc/tc.cuh", "quantized_expert_ffn_gemm_b200/csrc/topk.cuh"]
 _GEMM_SRC = ["quantized_expert_ffn_gemm_b200/csrc/gemm.cu", "quantized_expert_ffn_gemm_b200/csrc/tc.cuh",
              "quantized_expert_ffn_gemm_b200/csrc/dequant.cuh"]
 TRAFFIC = {
-    # (kernel, workloads with the captured launch shape): (sources, sha256, bytes per launch, profile)
+    # (kernel, workloads with the captured launch shape): (sources, sha256, DRAM bytes per launch)
     ("gemm_gate_up", ("prefill8k", "stack_prefill")):
-        (_GEMM_SRC, "f5ad8aca8c32a2576bfdf9f5a1d66e6cbeb86fb1fb932b6adae357c9fbff935a", 786358272,
-         "profiles/grouped_gemm_prefill8k.md"),
+        (_GEMM_SRC, "f5ad8aca8c32a2576bfdf9f5a1d66e6cbeb86fb1fb932b6adae357c9fbff935a", 786358272),
     ("decode_fused", ("decode1",)):
-        (_DEC_SRC, "079b8a42801687ba382781d35128bd3914e45a1093ae366b7f07f8b8b245e47d", 15117824,
-         "profiles/decode_fused_kernel_decode1.md"),
+        (_DEC_SRC, "079b8a42801687ba382781d35128bd3914e45a1093ae366b7f07f8b8b245e47d", 15117824),
 }
 
 
@@ -87,7 +93,7 @@ def traffic_for(kernel: str, workload: str):
     ent = next((v for (kn, wls), v in TRAFFIC.items() if kn == kernel and workload in wls), None)
     if ent is None:
         return None
-    srcs, sha, nbytes, _ = ent
+    srcs, sha, nbytes = ent
     h = hashlib.sha256()
     try:
         for src in srcs:
@@ -222,20 +228,33 @@ def expert_bytes(shape: synth.LayerShape):
     return gu, dn
 
 
-def run_ours(args, world, rank, local):
+def same_weights(a: synth.LayerShape, b: synth.LayerShape) -> bool:
+    """Two workloads draw the same layer weights (they differ at most in T)."""
+    return (a.H, a.E, a.k, a.I, a.qtype, a.shared, a.zipf_s, a.seed) == (b.H, b.E, b.k, b.I, b.qtype, b.shared,
+                                                                         b.zipf_s, b.seed)
+
+
+def run_ours(args, world, rank, local, workload=None, steps=None, warmup=None, layers=None):
+    """Time `workload` (default: args.workload) for `steps` steps after `warmup` warm-up steps
+    (default: args.steps / args.warmup); `layers` reuses another workload's device weights."""
     import quantized_expert_ffn_gemm_b200 as moe
-    wl = WORKLOADS[args.workload]
-    shape = workload_shape(args.workload)
+    workload = workload or args.workload
+    wl = WORKLOADS[workload]
+    shape = workload_shape(workload)
     is_stack = bool(wl.get("stack"))
     T, H, E, k, I = shape.T, shape.H, shape.E, shape.k, shape.I
-    n_layers = args.layers or wl["layers"]
+    n_layers = (args.layers if workload == args.workload else None) or wl["layers"]
     dev = torch.device("cuda", torch.cuda.current_device())
-    layers = build_layers(shape, n_layers)
+    if layers is None or len(layers) < n_layers:
+        layers = build_layers(shape, n_layers)
+    layers = layers[:n_layers]
+    K = args.steps if steps is None else steps
+    W = args.warmup if warmup is None else warmup
     ws = moe.Workspace.for_layer(H, E, k, I, shape.shared, T)
     y = torch.empty(T, H, dtype=torch.float32, device=dev)
     if is_stack:
         # independent seeded residual-stream inputs, one per step (tokens do not feed each other)
-        n_x = min(args.steps, 256) if T <= 8 else 2
+        n_x = min(K, 256) if T <= 8 else 2
         xs = [synth.make_residual(shape.seed, T, H, stream=replica_x_stream(rank, i)).to(dev) for i in range(n_x)]
         stack = moe.Stack([l[0] for l in layers], None, [l[2] for l in layers],
                           [l[3] for l in layers] if shape.shared else None, k)
@@ -250,7 +269,6 @@ def run_ours(args, world, rank, local):
         def step(i, x=None, idx_out=None):
             handles[i % n_layers].forward(xs[i % n_x] if x is None else x, y, idx_out=idx_out)
 
-    K, W = args.steps, args.warmup
     for i in range(W):
         step(i)
     torch.cuda.synchronize()
@@ -330,14 +348,18 @@ def run_ours(args, world, rank, local):
         # decode: HBM bound. With the fused kernel the whole layer is one launch and its algorithmic
         # bytes are the distinct active experts + the fp32 router + x + y; with the separate kernels
         # the dominant one is the gate/up dequant-GEMV.
+        # `achieved` counts the distinct active experts' packed bytes only (the benchmark spec's metric:
+        # "% of HBM on active-expert bytes"); the all-bytes figure adds the fp32 router, x and y.
         gu_b, dn_b = expert_bytes(shape)
         units_avg = units_total / Kt
         if "decode_fused" in kt:
             dom = "decode_fused"
-            algo = units_avg * (gu_b + dn_b) + E * H * 4 + T * H * 2 + T * H * 4
+            algo = units_avg * (gu_b + dn_b)
+            algo_all = algo + E * H * 4 + T * H * 2 + T * H * 4
         else:
             dom = "dec_gate_up"
-            algo = units_avg * gu_b + T * H * 2 + units_avg * T * I * 2
+            algo = units_avg * gu_b
+            algo_all = algo + T * H * 2 + units_avg * T * I * 2
         d_ms, d_n = kt[dom]
         launch_us = d_ms / d_n * 1e3
         timing = "events around each launch (blocks queued behind a sleep kernel)"
@@ -348,10 +370,14 @@ def run_ours(args, world, rank, local):
             timing = "timed region (graph replay) / launches of the kernel in it; per-launch events gave %.2f us" % (
                 d_ms / d_n * 1e3)
         achieved = algo / (launch_us / 1e6) / 1e9
+        ach_all = algo_all / (launch_us / 1e6) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"], "unit": "GB/s",
-                "frac": round(achieved / pk["hbm"], 4), "traffic": traffic_for(dom, args.workload), "peak_source": pk["src"],
+                "frac": round(achieved / pk["hbm"], 4), "traffic": traffic_for(dom, workload), "peak_source": pk["src"],
+                "metric_bytes": "distinct active experts' packed bytes (north-star metric)",
                 "algorithmic_bytes_per_launch": int(algo), "avg_launch_us": round(launch_us, 3),
-                "launch_timing": timing}
+                "all_bytes_per_launch": int(algo_all), "all_bytes_achieved": round(ach_all, 1),
+                "all_bytes_frac": round(ach_all / pk["hbm"], 4),
+                "distinct_experts_avg": round(units_avg, 2), "launch_timing": timing}
         layer_bytes = units_avg * (gu_b + dn_b) + E * H * 4 + T * H * 2 + T * H * 4
         layer_gbs = layer_bytes / (ms_max / K / lps / 1e3) / 1e9
         roof_layer = {"bound": "hbm", "bytes_per_step": int(layer_bytes), "achieved": round(layer_gbs, 1),
@@ -368,7 +394,7 @@ def run_ours(args, world, rank, local):
         capped = bool(sm and smax and sm < 0.95 * smax)
         peak_tc = pk["tc_sus"] if capped else pk["tc"]
         roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak_tc,
-                "unit": "TFLOP/s", "frac": round(achieved / peak_tc, 4), "traffic": traffic_for(dom, args.workload),
+                "unit": "TFLOP/s", "frac": round(achieved / peak_tc, 4), "traffic": traffic_for(dom, workload),
                 "peak_source": pk["src"] + (" sustained" if capped else " burst") +
                 " bf16 (fp16 MMA runs at the bf16 rate; SM clock %s of %s MHz under load)" % (sm, smax),
                 "frac_of_other_peak": round(achieved / (pk["tc"] if capped else pk["tc_sus"]), 4),
@@ -409,7 +435,7 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(ms_max / K, 6), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16 (MMA operands; fp32 accumulate, router, y; weights Q2/Q3)", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {'48-layer stack of MoE layers' if is_stack else 'MoE layer'} "
+        "config": {"workload": f"{workload}: {'48-layer stack of MoE layers' if is_stack else 'MoE layer'} "
                                f"T={T}, H={H}, E={E}, top-{k}, I={I}, "
                                f"{'Q3' if shape.qtype == 3 else 'Q2'}, shared={int(shape.shared)}, "
                                f"router bias={'Zipf(%s)' % shape.zipf_s if shape.zipf_s else 'none'}",
@@ -551,7 +577,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="distinct layer weight sets to rotate over (default 48 for decode, 4 for prefill)")
-    ap.add_argument("--breakdown", action="store_true", help="also time T=4 and T=8192 on rank 0 (extra keys)")
+    ap.add_argument("--no-breakdown", action="store_true",
+                    help="time only --workload (by default a single-GPU run of the T=1 decode layer also times "
+                         "the T=4 verify layer and the T=8192 prefill layer, reported under 'breakdown')")
     ap.add_argument("--crossover", action="store_true",
                     help="time the expert paths at T = 1..128 (one JSON line per T and path) and exit")
     args = ap.parse_args()
@@ -574,7 +602,16 @@ def main():
 
     world, rank, local = dist_setup()
     try:
-        out, shape, _ = run_ours(args, world, rank, local)
+        out, shape, layers = run_ours(args, world, rank, local)
+        if world == 1 and args.workload == "decode1" and not args.no_breakdown:
+            # the metric is quoted at T = 1, 4 and 8192: the other two in the same run, each its own
+            # timed region with fixed step counts (decode4 reuses the decode layers' weights)
+            out["breakdown"] = {}
+            for name, (K, W) in BREAKDOWN.items():
+                o, _, _ = run_ours(args, world, rank, local, workload=name, steps=K, warmup=W,
+                                   layers=layers if same_weights(shape, workload_shape(name)) else None)
+                out["breakdown"][name] = {key: o[key] for key in BREAKDOWN_KEYS if key in o}
+                torch.cuda.empty_cache()
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             wl = WORKLOADS[args.workload]
             out["cpu_baseline"] = cpu_baseline(shape, wl["layers"] if wl.get("stack") else 1)

@@ -123,7 +123,9 @@ size_t moe_workspace_bytes(const moe_layer_desc *desc, int32_t T);
  * zero on exit). Call once on a freshly allocated workspace before its first use. */
 moe_status moe_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
-/* RMSNorm with no learned gain (the stack's pre-router normalisation):
+/* RMSNorm with no learned gain, the stack's pre-router normalisation (the 48-layer stack of
+ * "Strata vs Llama.cpp vs vLLM", "How Strata is designed to work"; the pages give no norm
+ * details, so this is the plain reading: eps inside the square root, no gain, bf16 output):
  *   u[t,h] = bf16_rne( r[t,h] / sqrt(mean_h r[t,h]^2 + eps) ), fp32 arithmetic.
  * r fp32 [T,H] -> u bf16 [T,H]. */
 moe_status moe_rmsnorm_bf16(const float *r, int32_t T, int32_t H, float eps, uint16_t *u, void *stream);
@@ -141,7 +143,10 @@ moe_status moe_router_topk(const uint16_t *x, int32_t T, int32_t H, const float 
                            int32_t E, int32_t k, int32_t *idx, float *w, float *logits_opt,
                            void *ws, size_t ws_bytes, void *stream);
 
-/* Token permutation into expert-contiguous rows (stable counting sort by expert).
+/* Token permutation into expert-contiguous rows (stable counting sort by expert), so each active
+ * expert's tokens form one block its weights are applied to at once ("Two-Day Port, 8x Faster
+ * Prefill: Strata Engine Benchmarked", "Where Strata Is Fast: Not Magic, but Logistics": the
+ * larger the batch, the more tokens share each expert's weights).
  *   counts[e]        number of (t,j) with idx[t,j] == e
  *   offsets[0..E]    exclusive scan of counts; with_shared: offsets[E+1] = T*k + T
  *   row_of[t*k+j]    row of pair (t,j); rows of one expert are in token order
@@ -154,7 +159,9 @@ moe_status moe_permute(const int32_t *idx, int32_t T, int32_t k, int32_t E, cons
                        int32_t with_shared, int32_t *counts, int32_t *offsets, int32_t *row_of, int32_t *src,
                        uint16_t *x_perm, void *ws, size_t ws_bytes, void *stream);
 
-/* Grouped expert FFN over expert-contiguous rows: for every row r < n_rows of group g
+/* Grouped expert FFN over expert-contiguous rows, dequantizing the block weights inside the
+ * multiply ("Two-Day Port, 8x Faster Prefill: Strata Engine Benchmarked", "Where Strata Is Fast:
+ * Not Magic, but Logistics", MMQ paragraph): for every row r < n_rows of group g
  * (offsets[g] <= r < offsets[g+1]):
  *   out_perm[r,:] = fp16( W_down[g] ( silu(W_gate[g] x_perm[r]) * (W_up[g] x_perm[r]) ) )
  * Groups 0..E-1 use `routed`; with shared_opt != NULL, group E (rows offsets[E]..offsets[E+1])
@@ -167,7 +174,9 @@ moe_status moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, int32_
                           int32_t I, const moe_expert_set *routed, const moe_expert_set *shared_opt,
                           uint16_t *out_perm, int32_t path, void *ws, size_t ws_bytes, void *stream);
 
-/* Un-permute and weighted combine:
+/* Un-permute and weighted combine (each token's output is its k experts' outputs weighted by
+ * the routing weights, plus the always-on shared expert: "Strata vs Llama.cpp vs vLLM", "How
+ * Strata is designed to work"; Strata DETAILS.md, "How it works"):
  *   y[t,:] = sum_{j<k} w[t,j] out_perm[row_of[t,j],:] + shared_out[t,:] + residual[t,:]
  * summed in fixed j order in fp32. out_perm fp16; shared_out_opt fp16 [T,H] or NULL;
  * residual_opt fp32 [T,H] or NULL (may alias y); y fp32 [T,H]. */
@@ -175,7 +184,10 @@ moe_status moe_combine(const uint16_t *out_perm, const int32_t *row_of, const fl
                        int32_t H, const uint16_t *shared_out_opt, const float *residual_opt, float *y,
                        void *stream);
 
-/* One full MoE layer. T <= 8 with path AUTO or GEMV: the decode path (router + top-k, then a
+/* One full MoE layer (512 routed experts, 10 active per token, a shared expert; 8,192-token
+ * prefill chunks and 1-4-token decode / MTP-verify passes: "Strata vs Llama.cpp vs vLLM", "How
+ * Strata is designed to work"; Strata DETAILS.md, "How it works"). T <= 8 with path AUTO or
+ * GEMV: the decode path (router + top-k, then a
  * dequant-GEMV over the distinct selected experts with the tokens as MMA columns, down
  * projection fused with the weighted combine; under AUTO one cooperative kernel does the whole
  * layer where its shared-memory plan fits). Otherwise: router + top-k (fp32 dot products on the
@@ -194,7 +206,8 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
                              int32_t *idx_out_opt, float *w_out_opt, int32_t path,
                              void *ws, size_t ws_bytes, void *stream);
 
-/* A stack of L layers with pre-router RMSNorm and a residual stream (attention omitted):
+/* A stack of L layers with pre-router RMSNorm and a residual stream, attention omitted (the
+ * 48 MoE layers of "Strata vs Llama.cpp vs vLLM", "How Strata is designed to work"):
  *   r_0 = r_in;  r_{l+1} = r_l + layer_l( bf16(RMSNorm_eps(r_l)) );  r_out = r_L
  * r_in, r_out fp32 [T,H] (r_out may equal r_in). Wr[l], bias[l] (bias may be NULL, or
  * bias[l] NULL), routed[l], shared[l] (NULL when desc->has_shared == 0): per-layer arrays
@@ -204,22 +217,26 @@ moe_status moe_stack_forward(const float *r_in, int32_t T, int32_t L, const floa
                              const moe_expert_set *routed, const moe_expert_set *shared, float eps,
                              float *r_out, int32_t path, void *ws, size_t ws_bytes, void *stream);
 
-/* Test hook: dequantize rows row0..row0+nrows-1 of one expert.
+/* Test hook: dequantize rows row0..row0+nrows-1 of one expert with the decoder the expert
+ * kernels use (the block formats are the stand-in stated at the top of this file).
  *   out_f32[r,k] = d*(c-q0) in fp32 (exact); out_f16[r,k] = fp16_rne(d*(c-q0)), the value the
  *   expert kernels feed to the tensor cores. Either output may be NULL. [nrows, K] each. */
 moe_status moe_dequant_rows(const moe_qmat *m, int32_t expert, int32_t row0, int32_t nrows, float *out_f32,
                             uint16_t *out_f16, void *stream);
 
-/* Router and top-k without a workspace, for callers that cannot allocate device memory (code
- * running under CUDA-graph capture, plugins whose host application owns all device memory,
- * runtimes with no device allocator). The pages have no counterpart: this is a variant of
- * moe_router_topk (same arguments, same results) whose scratch -- a control word and the [T][E]
- * fp32 logits -- is a fixed array inside the library (about 128 KB, held on every GPU that loads
- * the library until the process exits). Limits: T <= 8, E <= 4096 (and T * max(H, E) * 4 <=
- * 200 KB); larger requests return MOE_ERR_UNSUPPORTED. The first call on each device looks up
- * the array's device address and should come before any stream capture. All calls share the
- * array: calls that overlap on the GPU race and must be serialised by the caller. It allocates
- * no memory. */
+/* Router and top-k without a workspace, for callers that cannot allocate device memory: plugins
+ * hosted by an application that owns and budgets all device memory and gives its plugins no
+ * allocator, or runtimes that lay out all device memory ahead of time and have no allocator at
+ * run time. The pages have no counterpart: this is a variant of moe_router_topk (same
+ * arguments, same results, the same shape rules and status codes) whose scratch -- a control
+ * word and the [T][E] fp32 logits -- is a fixed array inside the library (about 128 KB, held on
+ * every GPU that loads the library until the process exits). Limits: T <= 8, E <= 4096 (and
+ * T * max(H, E) * 4 <= 200 KB); larger requests return MOE_ERR_UNSUPPORTED. The first call on
+ * each device looks up the array's device address and should come before any stream capture.
+ * All calls share the array, which keeps the last call's contents (each call clears what must
+ * start at zero): calls that overlap on the GPU race and must be serialised by the caller. The
+ * router kernel records no device-side error, so the array's error word needs no reader. It
+ * allocates no memory. */
 moe_status moe_router_topk_static(const uint16_t *x, int32_t T, int32_t H, const float *Wr, const float *bias,
                                   int32_t E, int32_t k, int32_t *idx, float *w, float *logits_opt, void *stream);
 

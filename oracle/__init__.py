@@ -100,9 +100,19 @@ class QMatView:
     """Keeps the numpy arrays alive and exposes the C struct."""
 
     def __init__(self, qm):
+        assert qm.qtype in (2, 3, 4), f"unknown block format {qm.qtype}"
         self.codes = _np(qm.codes, np.uint8)
         self.hibits = None if qm.hibits is None else _np(qm.hibits, np.uint8)
         self.scales = _np(qm.scales, np.uint16)
+        # plane shapes: codes K/4 bytes per row (K/2 for the 4-bit plane), hi bits K/8 for Q3 only,
+        # one scale per 32-weight block; a wrong shape would make the C decoder read past the array
+        n, rows, K = int(qm.n), int(qm.rows), int(qm.K)
+        assert K % 32 == 0 and self.codes.shape[-1] == (K // 2 if qm.qtype == 4 else K // 4)
+        assert self.codes.size == n * rows * self.codes.shape[-1]
+        assert (self.hibits is not None) == (qm.qtype == 3)
+        if self.hibits is not None:
+            assert self.hibits.shape[-1] == K // 8 and self.hibits.size == n * rows * K // 8
+        assert self.scales.size == n * rows * K // 32
         self.s = _QMat(qm.qtype, qm.n, qm.rows, qm.K, _ptr(self.codes), _ptr(self.hibits), _ptr(self.scales))
 
     @property

@@ -108,8 +108,10 @@ static double round_f16(double v) { return oracle_half_to_double(oracle_double_t
 
 /* ---------------------------------------------------------------- dequantization */
 
-/* integer code of weight (e, r, k) from the packed planes (layout in the file header) */
+/* integer code of weight (e, r, k) from the packed planes (layout in the file header); -1 for a
+ * block format other than Q2, Q3 or Q4 (nothing is read then) */
 int oracle_code(const oq_mat *m, int e, int r, int k) {
+  if (m->qtype != 2 && m->qtype != 3 && m->qtype != 4) return -1;
   size_t row = (size_t)e * m->rows + r;
   int b = k >> 5, j = k & 31;
   if (m->qtype == 4) {  /* word j/8 of the block, pair (i, h) = ((j%8)/2, j%2) at bit 16h+4i */

@@ -65,16 +65,39 @@ int num_sms() {
 }
 
 cudaError_t smem_limit_once_impl(const void *func, size_t bytes) {
-  // per-kernel record of the limit already set (keyed by the kernel's host stub address)
+  // record of the limits already set, keyed by (device, kernel host stub): the attribute belongs
+  // to the current device's context, so every device a process uses gets its own raise
+  struct Done {
+    int dev;
+    const void *func;
+    size_t bytes;
+  };
   static std::mutex mu;
-  static std::vector<std::pair<const void *, size_t>> done;
+  static std::vector<Done> done;
   if (bytes == 0) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lk(mu);
   for (auto &d : done)
-    if (d.first == func && d.second >= bytes) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess) done.push_back({func, bytes});
+    if (d.dev == dev && d.func == func && d.bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done.push_back({dev, func, bytes});
   return e;
+}
+
+bool layer_shape_ok(int H, int E, int k, int I) {
+  return H > 0 && H % 64 == 0 && H <= 16384 && E >= 1 && E <= kMaxE && k >= 1 && k <= kMaxK && k <= E && I > 0 &&
+         I % 64 == 0 && I <= 16384;
+}
+
+// H or I a multiple of 32 but not of 64 (or beyond the sizes above) is a valid layer the library
+// does not run
+moe_status layer_shape_status(int H, int E, int k, int I) {
+  if (layer_shape_ok(H, E, k, I)) return MOE_OK;
+  if (H > 0 && H % 32 == 0 && I > 0 && I % 32 == 0 && E >= 1 && E <= kMaxE && k >= 1 && k <= kMaxK && k <= E)
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_ERR_INVALID_ARG;
 }
 
 }  // namespace moe
@@ -87,18 +110,8 @@ inline bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-bool shape_ok(int H, int E, int k, int I) {
-  return H > 0 && H % 64 == 0 && H <= 16384 && E >= 1 && E <= kMaxE && k >= 1 && k <= kMaxK && k <= E && I > 0 &&
-         I % 64 == 0 && I <= 16384;
-}
-
-// H or I a multiple of 32 but not of 64 is a valid layer the library does not run
-moe_status shape_status(int H, int E, int k, int I) {
-  if (shape_ok(H, E, k, I)) return MOE_OK;
-  if (H > 0 && H % 32 == 0 && I > 0 && I % 32 == 0 && E >= 1 && E <= kMaxE && k >= 1 && k <= kMaxK && k <= E)
-    return MOE_ERR_UNSUPPORTED;
-  return MOE_ERR_INVALID_ARG;
-}
+inline bool shape_ok(int H, int E, int k, int I) { return layer_shape_ok(H, E, k, I); }
+inline moe_status shape_status(int H, int E, int k, int I) { return layer_shape_status(H, E, k, I); }
 
 moe_status check_qmat(const moe_qmat &m, int n_experts, int rows, int K) {
   if (m.qtype != MOE_Q2 && m.qtype != MOE_Q3) return MOE_ERR_INVALID_ARG;

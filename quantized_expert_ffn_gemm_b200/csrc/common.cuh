@@ -153,6 +153,12 @@ cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, i
 
 int num_sms();
 
+// shape rules every entry point applies: H and I multiples of 64 up to 16384, 1 <= E <= kMaxE,
+// 1 <= k <= min(E, kMaxK); a layer outside them that is still well formed (H, I multiples of 32)
+// gives MOE_ERR_UNSUPPORTED, anything else MOE_ERR_INVALID_ARG
+bool layer_shape_ok(int H, int E, int k, int I);
+moe_status layer_shape_status(int H, int E, int k, int I);
+
 // Raise a kernel's dynamic shared memory limit once per process (kept out of later launches so
 // that launches can be captured into CUDA graphs).
 cudaError_t smem_limit_once_impl(const void *func, size_t bytes);

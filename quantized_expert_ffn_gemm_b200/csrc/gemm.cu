@@ -419,7 +419,7 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
 }
 
 // ---------------------------------------------------------------- tile list
-// entries (group, first row within the group) for every 256-row slice of every non-empty group
+// entries (group, first row within the group) for every kBNMax-row (192-row) slice of every non-empty group
 // (offsets that are not monotone or run past n_rows flag the error word and yield no tiles)
 __global__ void __launch_bounds__(1024) tile_list_kernel(const int32_t *__restrict__ off, int G, int n_rows,
                                                          int2 *__restrict__ tiles, Ctrl *__restrict__ ctrl) {

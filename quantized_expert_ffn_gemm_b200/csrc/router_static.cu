@@ -1,10 +1,10 @@
 // Router + top-k for callers that cannot allocate device memory.
 //
 // moe_router_topk needs a caller-provided workspace for its scratch (the last-CTA ticket and the
-// [T][E] logits the top-k reads back). Some callers have no way to obtain one: code that runs
-// while a CUDA graph is being captured (where new allocations are not allowed), plugins hosted by
-// an application that owns every device allocation, or runtimes without a device allocator at
-// all. This variant keeps its scratch in a fixed-size array inside the library instead, so the
+// [T][E] logits the top-k reads back). Some callers have no way to obtain one: plugins hosted by
+// an application that owns and budgets every device allocation and hands its plugins none, or
+// runtimes that lay out all device memory ahead of time and have no allocator to call at run
+// time. This variant keeps its scratch in a fixed-size array inside the library instead, so the
 // caller passes only inputs and outputs.
 //
 // The array lives in every GPU that loads the library until the process exits. In host code the
@@ -13,6 +13,10 @@
 // therefore come before any stream capture. All calls share the one array: calls that overlap on
 // the GPU (different streams, or different host threads) race on it and must be serialised by
 // the caller.
+//
+// The array also holds a control area with an error word. The router kernel records no
+// device-side error (it has no bounded waits and no index inputs), so this word is only cleared
+// by each call, never set, and nothing is lost by having no reader for it.
 #include <mutex>
 
 #include "common.cuh"
@@ -56,7 +60,11 @@ using namespace moe;
 extern "C" moe_status moe_router_topk_static(const uint16_t *x, int32_t T, int32_t H, const float *Wr,
                                              const float *bias, int32_t E, int32_t k, int32_t *idx, float *w,
                                              float *logits_opt, void *stream) {
-  if (H <= 0 || H % 64 != 0 || E < 1 || k < 1 || k > kMaxK || k > E || T < 0) return MOE_ERR_INVALID_ARG;
+  // the shape rules of moe_router_topk first (the same arguments get the same status) ...
+  const moe_status st = layer_shape_status(H, E, k, 64);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  // ... then the limits of the fixed scratch
   if (T > kStaticMaxT || E > kStaticMaxE || (size_t)T * (H > E ? H : E) * 4 > 200 * 1024)
     return MOE_ERR_UNSUPPORTED;  // beyond the fixed scratch (or the single-kernel router's shared memory)
   if (T == 0) return MOE_OK;

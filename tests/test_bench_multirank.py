@@ -100,7 +100,7 @@ def test_traffic_figure_follows_source_hash_and_launch_shape(tmp_path, monkeypat
     src.write_text("kernel v1\n")
     sha = hashlib.sha256(src.read_bytes()).hexdigest()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "TRAFFIC", {("k", ("shape_a",)): (["k.cu"], sha, 1234, "profiles/k.md")})
+    monkeypatch.setattr(bench, "TRAFFIC", {("k", ("shape_a",)): (["k.cu"], sha, 1234)})
     assert bench.traffic_for("k", "shape_a") == 1234
     assert bench.traffic_for("k", "shape_b") is None      # another launch shape
     assert bench.traffic_for("other", "shape_a") is None  # no capture of that kernel

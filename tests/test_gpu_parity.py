@@ -193,7 +193,7 @@ def test_layer_forward(name, ntok):
     y, idx, w = moe.layer_forward(x, Wr, b, routed, shared, s.k, ws, want_routing=True)
     assert moe.read_device_error(ws) == 0
     tokens = np.arange(s.T) if ntok >= s.T else np.sort(np.random.default_rng(5).choice(s.T, ntok, replace=False))
-    err, flips = check_layer(y.cpu().numpy(), idx.cpu().numpy(), L, tokens)
+    err, flips = check_layer(y.cpu().numpy(), idx.cpu().numpy(), L, tokens, w_gpu=w.cpu().numpy())
     print(f"{name}: max|dy|/rms = {err:.3e}, near-tie flips {len(flips)}")
 
 
@@ -202,11 +202,12 @@ def test_layer_forward_with_residual_in_place():
     s = L.shape
     r = synth.make_residual(9, s.T, s.H).cuda()
     ws = ws_for(L)
-    y, idx, _ = moe.layer_forward(x, Wr, b, routed, shared, s.k, ws, residual=r.clone(), want_routing=True)
+    y, idx, w = moe.layer_forward(x, Wr, b, routed, shared, s.k, ws, residual=r.clone(), want_routing=True)
     y2 = r.clone()
     moe.layer_forward(x, Wr, b, routed, shared, s.k, ws, residual=y2, y=y2)  # aliasing residual and y
     assert torch.equal(y, y2)
-    check_layer(y.cpu().numpy(), idx.cpu().numpy(), L, range(0, s.T, 7), residual=r.cpu().numpy())
+    check_layer(y.cpu().numpy(), idx.cpu().numpy(), L, range(0, s.T, 7), residual=r.cpu().numpy(),
+                w_gpu=w.cpu().numpy())
 
 
 @pytest.mark.parametrize("name,T", [("mid", 64), ("mid", 4), ("mid_q3", 4), ("tiny", 4)])
@@ -232,9 +233,9 @@ def test_layer_forward_decode_batches(name, T):
     s = L0.shape
     L = synth.LayerInputs(s, synth.make_x(s.seed, T, s.H, stream=40 + T), L0.Wr, L0.bias, L0.routed, L0.shared)
     ws = moe.Workspace.for_layer(s.H, s.E, s.k, s.I, s.shared, T)
-    y, idx, _ = moe.layer_forward(L.x.cuda(), Wr, b, routed, shared, s.k, ws, want_routing=True)
+    y, idx, w = moe.layer_forward(L.x.cuda(), Wr, b, routed, shared, s.k, ws, want_routing=True)
     assert moe.read_device_error(ws) == 0
-    check_layer(y.cpu().numpy(), idx.cpu().numpy(), L, range(T))
+    check_layer(y.cpu().numpy(), idx.cpu().numpy(), L, range(T), w_gpu=w.cpu().numpy())
 
 
 def test_mtp_verify_T4_equals_four_T1():
@@ -269,10 +270,10 @@ def test_starved_barrier_times_out_and_context_survives():
     assert moe.read_device_error(ws) == moe.MOE_ERR_TIMEOUT
     assert time.perf_counter() - t0 < 1.5           # the limit, not a hang
     assert moe.read_device_error(ws) == 0            # reading cleared the word
-    y1, idx, _ = moe.layer_forward(x, Wr, b, routed, shared, s.k, ws, want_routing=True)
+    y1, idx, w = moe.layer_forward(x, Wr, b, routed, shared, s.k, ws, want_routing=True)
     assert moe.read_device_error(ws) == 0
     assert torch.equal(y0, y1)
-    check_layer(y1.cpu().numpy(), idx.cpu().numpy(), L, range(s.T))
+    check_layer(y1.cpu().numpy(), idx.cpu().numpy(), L, range(s.T), w_gpu=w.cpu().numpy())
 
 
 # ----------------------------------------------------------------------------- RMSNorm and stacks

@@ -380,3 +380,63 @@ def test_stack_is_token_independent():
     for t in (0, 3, 5):
         r1, _ = oracle.stack_forward(r0[t:t + 1], layers, 2)
         assert np.array_equal(r1[0], rT[t])
+
+
+def _bf16_rne(v: np.ndarray) -> np.ndarray:
+    """Round fp64 values (normal range) to the nearest bfloat16, ties to even, exactly: an 8-bit
+    significand m in [128, 256) scaled by a power of two (np.rint rounds half to even)."""
+    m, e = np.frexp(v)                      # v = m 2^e, |m| in [0.5, 1)
+    return np.ldexp(np.rint(m * 256.0), e - 8)
+
+
+def test_bf16_rne_helper_against_torch():
+    # the test-side rounding used below agrees with torch on fp32 inputs (no double rounding there)
+    rng = np.random.default_rng(41)
+    v = rng.normal(0, 3, 5000).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(_bf16_rne(v.astype(np.float64)), ref)
+
+
+def test_stack_of_zero_weight_layers_is_the_identity():
+    # every code equal to q0 makes every weight exactly 0: each layer adds 0 to the residual
+    # stream, so the stack returns its input bit for bit (a dropped residual would return 0)
+    rng = np.random.default_rng(42)
+    T, H, E, I = 5, 64, 4, 32
+
+    def zero_set(n, qtype):
+        q0 = {2: 2, 3: 4}[qtype]
+        m = lambda rows, K: KnownQMat(qtype, np.full((n, rows, K), q0), np.full((n, rows, K // 32), 0.01, np.float16))
+        return KnownSet(m(I, H), m(I, H), m(H, I))
+
+    layers = [(rng.normal(0, 0.02, (E, H)).astype(np.float32), None, zero_set(E, q), zero_set(1, q))
+              for q in (2, 3, 2)]
+    r0 = (rng.normal(0, 2, (T, H))).astype(np.float32)
+    rL, _ = oracle.stack_forward(r0, layers, 2)
+    assert np.array_equal(rL, r0)
+
+
+def test_stack_of_one_hot_layers_matches_hand_composition():
+    # r_{l+1} = r_l + FFN_{e_l}(u_l) + FFN_shared_l(u_l), u_l = bf16(r_l / sqrt(mean(r_l^2) + eps)),
+    # the residual stream kept in fp32 between layers. A one-hot router (k = 1, a +100 bias on
+    # expert e_l) makes the routed part the dense SwiGLU FFN of e_l with weight exactly 1.
+    # Composed here from the known dense weights, numpy and an exact bf16 rounding; a large eps
+    # (0.5) tells eps inside the square root from eps added to it, distinct experts per layer
+    # make the layer order matter.
+    rng = np.random.default_rng(43)
+    T, H, E, I, eps = 4, 64, 4, 32, 0.5
+    chosen = [2, 0, 3]
+    layers = []
+    for l, e in enumerate(chosen):
+        Wr = rng.normal(0, 0.02, (E, H)).astype(np.float32)
+        bias = np.zeros(E, np.float32)
+        bias[e] = 100.0
+        layers.append((Wr, bias, random_known_set(rng, 2 + (l % 2), E, H, I), random_known_set(rng, 2 + (l % 2), 1, H, I)))
+    r0 = (rng.normal(0, 1.5, (T, H))).astype(np.float32)
+    got, idxs = oracle.stack_forward(r0, layers, 1, eps=eps)
+    r = r0.astype(np.float64)
+    for (Wr, bias, ks, sh), e, idx in zip(layers, chosen, idxs):
+        assert (idx == e).all()
+        u = _bf16_rne(r / np.sqrt((r ** 2).mean(axis=1, keepdims=True) + eps))
+        r = (r + dense_ffn(ks, e, u) + dense_ffn(sh, 0, u)).astype(np.float32).astype(np.float64)
+    assert np.allclose(got, r, rtol=1e-9, atol=1e-12)
+    assert not np.allclose(got, r0, rtol=1e-3)     # the layers did change the stream

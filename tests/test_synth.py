@@ -55,7 +55,8 @@ def test_workload_shapes():
 
 
 def test_workload_table_matches_the_stated_configs():
-    # the shapes the tests and the benchmark use, as the design notes state them
+    # the shapes the tests and the benchmark use: the decode, verify, pruned, prefill, skewed Q3 and
+    # stack workloads (H=2048, E=512, top-10, I=512 unless stated otherwise)
     W = synth.WORKLOADS
     for name in ("decode1", "decode4", "verify6", "decode1_pruned256"):
         s = W[name]

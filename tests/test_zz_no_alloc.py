@@ -1,9 +1,9 @@
 """The workspace-free router entry point, moe_router_topk_static.
 
-Some callers cannot allocate device memory: code that runs during CUDA-graph capture (where new
-allocations are not allowed), plugins whose host application owns every device allocation, or
-runtimes with no device allocator at all. For them the library offers a router/top-k whose
-scratch is a fixed array inside the library, so nothing has to be allocated or passed in.
+Some callers cannot allocate device memory: plugins whose host application owns and budgets
+every device allocation and gives them no allocator, or runtimes that lay out all device memory
+ahead of time and have no allocator at run time. For them the library offers a router/top-k
+whose scratch is a fixed array inside the library, so nothing has to be allocated or passed in.
 
 This file runs last (pytest collects files by name) so that, if it fails, a run stopping at the
 first failure has already run everything else. Each test compares the workspace-free call with
@@ -61,3 +61,18 @@ def test_static_router_rejects_sizes_beyond_its_scratch():
     with pytest.raises(moe.MoeError) as ei:
         moe.router_topk_static(x, Wr, b, s.k)
     assert ei.value.code == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_static_router_applies_the_same_shape_rules():
+    # the same arguments give the same status as moe_router_topk: H beyond 16384 is a valid but
+    # unsupported shape, H not a multiple of 32 an invalid one, k > E invalid
+    x = torch.zeros(1, 16448, dtype=torch.bfloat16, device="cuda")
+    Wr = torch.zeros(16, 16448, dtype=torch.float32, device="cuda")
+    ws = moe.Workspace.for_layer(256, 16, 2, 64, False, 1)
+    for xx, WW, k, code in ((x, Wr, 2, moe.MOE_ERR_UNSUPPORTED), (x[:, :80], Wr[:, :80], 2, moe.MOE_ERR_INVALID_ARG),
+                            (x[:, :256], Wr[:4, :256], 5, moe.MOE_ERR_INVALID_ARG)):
+        with pytest.raises(moe.MoeError) as e_static:
+            moe.router_topk_static(xx.contiguous(), WW.contiguous(), None, k)
+        with pytest.raises(moe.MoeError) as e_ws:
+            moe.router_topk(xx.contiguous(), WW.contiguous(), None, k, ws)
+        assert e_static.value.code == e_ws.value.code == code
