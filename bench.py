@@ -42,6 +42,7 @@ WORKLOADS = {
     "decode4": dict(shape="decode4", layers=48),
     "verify6": dict(shape="verify6", layers=48),
     "decode1_pruned256": dict(shape="decode1_pruned256", layers=48),
+    "decode1_q4": dict(shape="decode1_q4", layers=48),
     "prefill8k": dict(shape="prefill8k", layers=4),
     "prefill2k_q3": dict(shape="prefill2k_q3", layers=4),
     # the 48-layer stack (RMSNorm before each router, residual stream, prefill-shaped layers with
@@ -50,9 +51,11 @@ WORKLOADS = {
     "stack_prefill": dict(shape="stack", T=8192, layers=48, stack=True),
 }
 METRIC = "MoE-layer tokens/s at T=1/4/8192; % of HBM or bf16 tensor-core roofline"
-DEFAULT_STEPS = {"decode1": 4800, "decode4": 4800, "verify6": 4800, "decode1_pruned256": 4800, "prefill8k": 40, "prefill2k_q3": 60, "stack_decode": 256,
+DEFAULT_STEPS = {"decode1": 4800, "decode4": 4800, "verify6": 4800, "decode1_pruned256": 4800, "decode1_q4": 4800,
+                 "prefill8k": 40, "prefill2k_q3": 60, "stack_decode": 256,
                  "stack_prefill": 4}
-DEFAULT_WARMUP = {"decode1": 480, "decode4": 480, "verify6": 480, "decode1_pruned256": 480, "prefill8k": 5, "prefill2k_q3": 5, "stack_decode": 16,
+DEFAULT_WARMUP = {"decode1": 480, "decode4": 480, "verify6": 480, "decode1_pruned256": 480, "decode1_q4": 480,
+                  "prefill8k": 5, "prefill2k_q3": 5, "stack_decode": 16,
                   "stack_prefill": 3}
 
 
@@ -222,7 +225,7 @@ def build_layers(shape: synth.LayerShape, n_layers: int, device="cuda"):
 
 def expert_bytes(shape: synth.LayerShape):
     """Packed bytes of one expert: (gate+up, down)."""
-    per_w = 0.25 + (0.125 if shape.qtype == synth.Q3 else 0.0) + 2.0 / 32
+    per_w = {synth.Q2: 0.25, synth.Q3: 0.375, synth.Q4: 0.5}[shape.qtype] + 2.0 / 32  # codes + fp16 scale
     gu = 2 * shape.I * shape.H * per_w
     dn = shape.H * shape.I * per_w
     return gu, dn
@@ -437,7 +440,7 @@ def run_ours(args, world, rank, local, workload=None, steps=None, warmup=None, l
         "dtype": "f16 (MMA operands; fp32 accumulate, router, y; weights Q2/Q3)", "data": "synthetic",
         "config": {"workload": f"{workload}: {'48-layer stack of MoE layers' if is_stack else 'MoE layer'} "
                                f"T={T}, H={H}, E={E}, top-{k}, I={I}, "
-                               f"{'Q3' if shape.qtype == 3 else 'Q2'}, shared={int(shape.shared)}, "
+                               f"Q{shape.qtype}, shared={int(shape.shared)}, "
                                f"router bias={'Zipf(%s)' % shape.zipf_s if shape.zipf_s else 'none'}",
                    "T": T, "layers_rotated": n_layers, "graph_steps": G,
                    "l2": "inputs larger than L2: steps rotate over %d layer weight sets (%.1f GB)" % (

@@ -22,6 +22,8 @@
  *   The pages do not fix the quantization formats; this library implements the stand-in:
  *     Q2: blocks of 32 weights, 2-bit codes c, one fp16 scale d, w = d*(c-2)
  *     Q3: blocks of 32 weights, 3-bit codes c, one fp16 scale d, w = d*(c-4)
+ *     Q4: blocks of 32 weights, 4-bit codes c, one fp16 scale d, w = d*(c-8) (a further format of
+ *         the same family, for layers that keep more bits)
  *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library allocates no
@@ -46,7 +48,10 @@
  *     codes  uint8 [n_experts][rows][K/4]  2-bit plane: Q2 codes, or the low 2 bits of Q3 codes.
  *            Per block, two 32-bit little-endian words; word q (weights 16q..16q+15) holds
  *            weight 16q+2i+h (i = 0..7, h = 0..1) at bits 16h+2i .. 16h+2i+1.
- *     hibits uint8 [n_experts][rows][K/8]  Q3 only (NULL for Q2): per block one 32-bit
+ *            Q4: uint8 [n_experts][rows][K/2], the 4-bit plane: per block four 32-bit
+ *            little-endian words; word q (weights 8q..8q+7) holds weight 8q+2i+h (i = 0..3,
+ *            h = 0..1) at bits 16h+4i .. 16h+4i+3.
+ *     hibits uint8 [n_experts][rows][K/8]  Q3 only (NULL for Q2 and Q4): per block one 32-bit
  *            little-endian word holding bit 2 of the code of weight 16q+2i+h at bit 16h+8q+i.
  *     scales fp16  [n_experts][rows][K/32] one scale per block.
  *   gate and up: rows = I, K = H.  down: rows = H, K = I.
@@ -82,18 +87,18 @@ enum {
   MOE_ERR_TIMEOUT = 7        /* reported by moe_read_device_error: a bounded device wait gave up */
 };
 
-enum { MOE_Q2 = 2, MOE_Q3 = 3 };
+enum { MOE_Q2 = 2, MOE_Q3 = 3, MOE_Q4 = 4 };
 
 /* expert-FFN path selection */
 enum { MOE_PATH_AUTO = 0, MOE_PATH_GEMV = 1, MOE_PATH_GEMM = 2 };
 
 typedef struct moe_qmat {
-  int32_t qtype;            /* MOE_Q2 or MOE_Q3 */
+  int32_t qtype;            /* MOE_Q2, MOE_Q3 or MOE_Q4 (all matrices of a layer share one) */
   int32_t n_experts;
   int32_t rows;
   int32_t K;
-  const uint8_t *codes;     /* [n_experts][rows][K/4] */
-  const uint8_t *hibits;    /* [n_experts][rows][K/8] for Q3, NULL for Q2 */
+  const uint8_t *codes;     /* [n_experts][rows][K/4]; Q4: [n_experts][rows][K/2] */
+  const uint8_t *hibits;    /* [n_experts][rows][K/8] for Q3, NULL for Q2 and Q4 */
   const uint16_t *scales;   /* [n_experts][rows][K/32] fp16 bits */
 } moe_qmat;
 
@@ -166,9 +171,10 @@ moe_status moe_permute(const int32_t *idx, int32_t T, int32_t k, int32_t E, cons
  *   out_perm[r,:] = fp16( W_down[g] ( silu(W_gate[g] x_perm[r]) * (W_up[g] x_perm[r]) ) )
  * Groups 0..E-1 use `routed`; with shared_opt != NULL, group E (rows offsets[E]..offsets[E+1])
  * uses the shared expert. offsets (device) has E+1 (+1) monotone entries with
- * offsets[last] <= n_rows. path: MOE_PATH_GEMM = tcgen05 grouped GEMM (needs H % 128 == 0
- * and I % 128 == 0), MOE_PATH_GEMV = dequant-GEMV, MOE_PATH_AUTO picks the GEMM when
- * n_rows > 64 and the GEMM shape rule holds, the GEMV otherwise.
+ * offsets[last] <= n_rows. path: MOE_PATH_GEMM = tcgen05 grouped GEMM for every group (needs
+ * H % 128 == 0 and I % 128 == 0), MOE_PATH_GEMV = dequant-GEMV for every group, MOE_PATH_AUTO:
+ * where the GEMM shape rule holds, groups of at most 32 rows on the dequant-GEMV (weights
+ * streamed once per 8 rows) and the larger groups on the grouped GEMM; the GEMV otherwise.
  * x_perm fp16 [n_rows,H]; out_perm fp16 [n_rows,H]. */
 moe_status moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, int32_t n_rows, int32_t E, int32_t H,
                           int32_t I, const moe_expert_set *routed, const moe_expert_set *shared_opt,
@@ -192,8 +198,9 @@ moe_status moe_combine(const uint16_t *out_perm, const int32_t *row_of, const fl
  * projection fused with the weighted combine; under AUTO one cooperative kernel does the whole
  * layer where its shared-memory plan fits). Otherwise: router + top-k (fp32 dot products on the
  * CUDA cores up to 128 tokens, tensor-core logits with an exact refine of the candidates above),
- * permute, the expert FFN (AUTO / GEMM: tcgen05 grouped GEMM gate/up with fused SwiGLU, then
- * down; GEMV: the decode GEMV kernels over 8-row chunks of each expert's rows), combine. Every
+ * permute, the expert FFN (GEMM: tcgen05 grouped GEMM gate/up with fused SwiGLU, then down;
+ * GEMV: the decode GEMV kernels over 8-row chunks of each expert's rows; AUTO: experts with at
+ * most 32 rows on the GEMV kernels, the others on the grouped GEMM), combine. Every
  * path computes the same function within the parity tolerance.
  *   y = sum_j w_j FFN_{idx_j}(x) + FFN_shared(x) (+ residual)      fp32 [T,H]
  * x bf16 [T,H]; Wr fp32 [E,H]; bias fp32 [E] or NULL; routed: gate/up [E][I][H], down [E][H][I];

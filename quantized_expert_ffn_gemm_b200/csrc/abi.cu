@@ -114,10 +114,10 @@ inline bool shape_ok(int H, int E, int k, int I) { return layer_shape_ok(H, E, k
 inline moe_status shape_status(int H, int E, int k, int I) { return layer_shape_status(H, E, k, I); }
 
 moe_status check_qmat(const moe_qmat &m, int n_experts, int rows, int K) {
-  if (m.qtype != MOE_Q2 && m.qtype != MOE_Q3) return MOE_ERR_INVALID_ARG;
+  if (m.qtype != MOE_Q2 && m.qtype != MOE_Q3 && m.qtype != MOE_Q4) return MOE_ERR_INVALID_ARG;
   if (m.n_experts != n_experts || m.rows != rows || m.K != K) return MOE_ERR_INVALID_ARG;
   if (!m.codes || !m.scales) return MOE_ERR_INVALID_ARG;
-  if (m.qtype == MOE_Q3 && !m.hibits) return MOE_ERR_INVALID_ARG;
+  if ((m.qtype == MOE_Q3) != (m.hibits != nullptr)) return MOE_ERR_INVALID_ARG;  // hi bits exactly for Q3
   if (!aligned16(m.codes) || !aligned16(m.scales) || (m.hibits && !aligned16(m.hibits))) return MOE_ERR_ALIGNMENT;
   return MOE_OK;
 }
@@ -135,6 +135,36 @@ moe_status check_set(const moe_expert_set *s, int n, int H, int I) {
 template <class T>
 T *at(void *ws, size_t off) {
   return reinterpret_cast<T *>(static_cast<unsigned char *>(ws) + off);
+}
+
+// Groups of at most this many rows take the dequant-GEMV kernels under AUTO (weights streamed
+// once per 8 rows, rows as MMA columns); larger groups take the tcgen05 grouped GEMM, whose tiles
+// cost about the same whatever their row count up to ~96 rows (measured), so a small group there
+// wastes most of a tile.
+constexpr int kSmallGroupRows = 32;
+
+// Expert FFN over expert-contiguous rows by path: GEMM (every group on the grouped GEMM), GEMV
+// (every group on the GEMV kernels), AUTO with the GEMM available: small groups on the GEMV
+// kernels and the rest on the grouped GEMM (disjoint rows of out_perm).
+cudaError_t expert_rows(const uint16_t *xperm, const int32_t *offsets, int rows, int E, int H, int I,
+                        const moe_expert_set &routed, const moe_expert_set *sh, uint16_t *hperm, uint16_t *operm,
+                        int2 *tiles, DecUnit *units, uint16_t *hdec, Ctrl *ctrl, cudaStream_t s, int path, bool gemm_ok) {
+  const int n_groups = E + (sh ? 1 : 0);
+  const bool hybrid = path == MOE_PATH_AUTO && gemm_ok;
+  cudaError_t e = cudaSuccess;
+  if (path == MOE_PATH_GEMM || hybrid) {
+    e = launch_grouped_ffn(xperm, offsets, rows, E, H, I, routed, sh, hperm, operm, tiles, ctrl, s,
+                           hybrid ? kSmallGroupRows : 0);
+    if (e != cudaSuccess || !hybrid) return e;
+  }
+  // a group of n rows makes ceil(n / 8) units: at most rows / 8 + (non-empty groups) in all
+  const int max_units = (rows + 7) / 8 + (n_groups < rows ? n_groups : rows);
+  e = launch_decode_units_from_offsets(offsets, n_groups, sh ? 1 : 0, rows, units, ctrl, s,
+                                       hybrid ? kSmallGroupRows : 0);
+  if (e == cudaSuccess) e = launch_decode_gate_up(xperm, 0, H, I, routed, sh, units, max_units, ctrl, hdec, s);
+  if (e == cudaSuccess)
+    e = launch_decode_down(H, I, routed, sh, units, max_units, ctrl, hdec, nullptr, nullptr, 0, operm, s);
+  return e;
 }
 
 bool decode_router_fits(int T, int H, int E) {
@@ -241,23 +271,10 @@ moe_status moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, int32_
   if (!aligned16(ws)) return MOE_ERR_ALIGNMENT;
   const bool gemm_ok = gemm_shape_supported(H, I) != 0;
   if (path == MOE_PATH_GEMM && !gemm_ok) return MOE_ERR_UNSUPPORTED;
-  const bool use_gemm = (path == MOE_PATH_GEMM) || (path == MOE_PATH_AUTO && gemm_ok && n_rows > 64);
   Ctrl *ctrl = at<Ctrl>(ws, L.ctrl);
-  cudaStream_t s = (cudaStream_t)stream;
-  const int n_groups = E + (shared_opt ? 1 : 0);
-  if (use_gemm)
-    return cuda_status(launch_grouped_ffn(x_perm, offsets, n_rows, E, H, I, *routed, shared_opt,
-                                          at<uint16_t>(ws, L.hperm), out_perm, at<int2>(ws, L.tiles), ctrl, s));
-  DecUnit *units = at<DecUnit>(ws, L.units);
-  // a group of n rows makes ceil(n / 8) units: at most rows / 8 + (non-empty groups) in all
-  const int max_units = (n_rows + 7) / 8 + (n_groups < n_rows ? n_groups : n_rows);
-  cudaError_t e = launch_decode_units_from_offsets(offsets, n_groups, shared_opt ? 1 : 0, n_rows, units, ctrl, s);
-  if (e == cudaSuccess)
-    e = launch_decode_gate_up(x_perm, 0, H, I, *routed, shared_opt, units, max_units, ctrl, at<uint16_t>(ws, L.hdec), s);
-  if (e == cudaSuccess)
-    e = launch_decode_down(H, I, *routed, shared_opt, units, max_units, ctrl, at<uint16_t>(ws, L.hdec), nullptr,
-                           nullptr, 0, out_perm, s);
-  return cuda_status(e);
+  return cuda_status(expert_rows(x_perm, offsets, n_rows, E, H, I, *routed, shared_opt, at<uint16_t>(ws, L.hperm),
+                                 out_perm, at<int2>(ws, L.tiles), at<DecUnit>(ws, L.units),
+                                 at<uint16_t>(ws, L.hdec), ctrl, (cudaStream_t)stream, path, gemm_ok));
 }
 
 moe_status moe_combine(const uint16_t *out_perm, const int32_t *row_of, const float *w, int32_t T, int32_t k,
@@ -318,7 +335,7 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
     e = cudaErrorNotSupported;
     if (path == MOE_PATH_AUTO) {
       e = launch_decode_fused(x, nullptr, 0.0f, T, H, Wr, bias, E, k, I, *routed, sh, residual_opt, y, logits, idx, w,
-                              hdec, ctrl, s);
+                              hdec, reinterpret_cast<unsigned *>(units), ctrl, s);
       if (e == cudaErrorCooperativeLaunchTooLarge) {
         (void)cudaGetLastError();
         e = cudaErrorNotSupported;
@@ -342,22 +359,10 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
     if (e == cudaSuccess)
       e = launch_permute(idx, T, k, E, x, H, hs, counts, offsets, row_of, src, xperm, at<int32_t>(ws, L.hist), ctrl,
                          s);
-    const bool use_gemm = (path == MOE_PATH_GEMM) || (path == MOE_PATH_AUTO && gemm_ok);
-    if (e == cudaSuccess) {
-      if (use_gemm) {
-        e = launch_grouped_ffn(xperm, offsets, rows, E, H, I, *routed, sh, at<uint16_t>(ws, L.hperm), operm,
-                               at<int2>(ws, L.tiles), ctrl, s);
-      } else {
-        DecUnit *units = at<DecUnit>(ws, L.units);
-        const int n_groups = E + hs, max_units = (rows + 7) / 8 + (n_groups < rows ? n_groups : rows);
-        e = launch_decode_units_from_offsets(offsets, n_groups, hs, rows, units, ctrl, s);
-        if (e == cudaSuccess)
-          e = launch_decode_gate_up(xperm, 0, H, I, *routed, sh, units, max_units, ctrl, at<uint16_t>(ws, L.hdec), s);
-        if (e == cudaSuccess)
-          e = launch_decode_down(H, I, *routed, sh, units, max_units, ctrl, at<uint16_t>(ws, L.hdec), nullptr,
-                                 nullptr, 0, operm, s);
-      }
-    }
+    if (e == cudaSuccess)
+      e = expert_rows(xperm, offsets, rows, E, H, I, *routed, sh, at<uint16_t>(ws, L.hperm), operm,
+                      at<int2>(ws, L.tiles), at<DecUnit>(ws, L.units), at<uint16_t>(ws, L.hdec), ctrl, s, path,
+                      gemm_ok);
     if (e == cudaSuccess)
       e = launch_combine(operm, row_of, w, T, k, H, hs ? operm + (size_t)P * H : nullptr, residual_opt, y, s);
   }
@@ -391,22 +396,24 @@ moe_status moe_stack_forward(const float *r_in, int32_t T, int32_t L, const floa
     if (hs && (st = check_set(&shared[l], 1, H, I)) != MOE_OK) return st;
     if (!Wr[l]) return MOE_ERR_INVALID_ARG;
   }
+  for (int l = 0; l < L; ++l)
+    if (!aligned16(Wr[l]) || (bias && bias[l] && !aligned16(bias[l]))) return MOE_ERR_ALIGNMENT;
   uint16_t *u = at<uint16_t>(ws, LY.u16);
   cudaStream_t s = (cudaStream_t)stream;
-  // decode-sized batches: RMSNorm runs inside the fused layer kernel (one launch per layer)
-  const bool fused = path == MOE_PATH_AUTO && T <= kDecodeMaxT && decode_router_fits(T, H, E);
+  // decode-sized batches: the fused decode kernel walks all the layers in one launch (RMSNorm
+  // inside, a grid barrier between layers, the next layer's router rows and shared expert
+  // requested into L2 while the current layer finishes)
+  if (path == MOE_PATH_AUTO && T <= kDecodeMaxT && decode_router_fits(T, H, E)) {
+    cudaError_t e = launch_decode_stack(r_in, eps, T, L, H, Wr, bias, E, k, I, routed, hs ? shared : nullptr, r_out,
+                                        at<float>(ws, LY.logits), at<int32_t>(ws, LY.idx), at<float>(ws, LY.w),
+                                        at<uint16_t>(ws, LY.hdec), at<unsigned>(ws, LY.units), at<Ctrl>(ws, LY.ctrl),
+                                        s);
+    if (e == cudaSuccess) return MOE_OK;
+    if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge) return cuda_status(e);
+    (void)cudaGetLastError();
+  }
   for (int l = 0; l < L; ++l) {
     const float *r = (l == 0) ? r_in : r_out;
-    const float *b = bias ? bias[l] : nullptr;
-    if (!aligned16(Wr[l]) || (b && !aligned16(b))) return MOE_ERR_ALIGNMENT;
-    if (fused) {
-      cudaError_t e = launch_decode_fused(nullptr, r, eps, T, H, Wr[l], b, E, k, I, routed[l], hs ? &shared[l] : nullptr,
-                                          r, r_out, at<float>(ws, LY.logits), at<int32_t>(ws, LY.idx),
-                                          at<float>(ws, LY.w), at<uint16_t>(ws, LY.hdec), at<Ctrl>(ws, LY.ctrl), s);
-      if (e == cudaSuccess) continue;
-      if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge) return cuda_status(e);
-      (void)cudaGetLastError();
-    }
     if ((st = moe_rmsnorm_bf16(r, T, H, eps, u, stream)) != MOE_OK) return st;
     st = moe_layer_forward(u, T, Wr[l], bias ? bias[l] : nullptr, desc, &routed[l], hs ? &shared[l] : nullptr, r, r_out,
                            nullptr, nullptr, path, ws, ws_bytes, s);

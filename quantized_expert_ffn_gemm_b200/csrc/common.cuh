@@ -122,8 +122,9 @@ cudaError_t launch_dequant_rows(const moe_qmat &m, int expert, int row0, int nro
                                 cudaStream_t s);
 
 // decode path: units are read from `units` (count in ctrl->n_units, at most max_units)
+// (groups of more than max_rows rows are skipped when max_rows > 0)
 cudaError_t launch_decode_units_from_offsets(const int32_t *offsets, int n_groups, int has_shared_group, int n_rows,
-                                             DecUnit *units, Ctrl *ctrl, cudaStream_t s);
+                                             DecUnit *units, Ctrl *ctrl, cudaStream_t s, int max_rows = 0);
 cudaError_t launch_decode_gate_up(const void *x, int x_is_bf16, int H, int I, const moe_expert_set &routed,
                                   const moe_expert_set *shared, const DecUnit *units, int max_units, Ctrl *ctrl,
                                   uint16_t *hdec, cudaStream_t s);
@@ -135,11 +136,21 @@ cudaError_t launch_decode_down(int H, int I, const moe_expert_set &routed, const
 // fused decode layer (one cooperative kernel: router, top-k, gate/up, down + combine);
 // returns cudaErrorNotSupported when the shape or the device cannot take it (callers fall back).
 // With r_norm != NULL the tokens are x = bf16(RMSNorm_eps(r_norm)) (x unused), bit-identical to
-// launch_rmsnorm followed by the layer.
+// launch_rmsnorm followed by the layer. unit_ready: T*k + 1 counters of workspace scratch (the
+// kernel zeroes them itself before use).
 cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float eps, int T, int H, const float *Wr,
                                 const float *bias, int E, int k, int I, const moe_expert_set &routed,
                                 const moe_expert_set *shared, const float *residual, float *y, float *logits,
-                                int32_t *idx, float *w, uint16_t *hdec, Ctrl *ctrl, cudaStream_t s);
+                                int32_t *idx, float *w, uint16_t *hdec, unsigned *unit_ready, Ctrl *ctrl,
+                                cudaStream_t s);
+
+// the fused decode kernel over the L layers of a stack in one launch per 48 layers (RMSNorm of the
+// stream before each router, residual added in place): r_out = stack(r_in). Per-layer arrays are
+// host arrays (as moe_stack_forward takes them); cudaErrorNotSupported when the shape cannot take it.
+cudaError_t launch_decode_stack(const float *r_in, float eps, int T, int L, int H, const float *const *Wr,
+                                const float *const *bias, int E, int k, int I, const moe_expert_set *routed,
+                                const moe_expert_set *shared, float *r_out, float *logits, int32_t *idx, float *w,
+                                uint16_t *hdec, unsigned *unit_ready, Ctrl *ctrl, cudaStream_t s);
 
 // test hook: a grid barrier that waits for one arrival more than the `ctas` CTAs make, giving up
 // after limit_ns with MOE_ERR_TIMEOUT in the control area
@@ -147,9 +158,10 @@ cudaError_t launch_barrier_starve(Ctrl *ctrl, int ctas, uint64_t limit_ns, cudaS
 
 // prefill path (tcgen05 grouped GEMM)
 int gemm_shape_supported(int H, int I);
+// groups of at most min_rows rows are skipped (min_rows > 0: the caller runs them on the GEMV path)
 cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, int n_rows, int E, int H, int I,
                                const moe_expert_set &routed, const moe_expert_set *shared, uint16_t *h_perm,
-                               uint16_t *out_perm, int2 *tiles, Ctrl *ctrl, cudaStream_t s);
+                               uint16_t *out_perm, int2 *tiles, Ctrl *ctrl, cudaStream_t s, int min_rows = 0);
 
 int num_sms();
 

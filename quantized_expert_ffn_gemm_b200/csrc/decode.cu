@@ -25,21 +25,24 @@ namespace moe {
 // warps in flight. Partials are summed in shared memory in fixed order.
 constexpr int kGuWarps = 8;
 
-template <bool SRC_BF16, bool Q3>
+template <bool SRC_BF16, int QT>
 __global__ void __launch_bounds__(kGuWarps * 32)
 dec_gate_up_kernel(const void *__restrict__ x, int H, int I, moe_expert_set routed, moe_expert_set shared,
                    const DecUnit *__restrict__ units, Ctrl *__restrict__ ctrl, uint16_t *__restrict__ hdec) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int u = blockIdx.x;
-  if (u >= ctrl->n_units) return;
+  const int n_units = ctrl->n_units;
+  // units are taken grid-stride (the grid is sized by the device, not by the largest possible
+  // unit count, so an empty or short unit list costs no flood of idle CTAs)
+  for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
   const DecUnit un = units[u];
   if (un.expert < 0 || un.expert >= (un.set ? shared.gate.n_experts : routed.gate.n_experts)) {
     if (threadIdx.x == 0 && blockIdx.y == 0) set_device_error(ctrl, MOE_ERR_DEVICE_CHECK, un.expert);
-    return;
+    continue;
   }
   const int xstride = H + 4;
   __half *xs = reinterpret_cast<__half *>(smem_raw);
   __shared__ float part[kGuWarps][16][8];
+  __syncthreads();  // the previous unit's reads of xs and part are done
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int mat = warp >> 2, slice = warp & 3;
   const MatView mv = mat_sel(routed, shared, un.set, mat, un.expert);
@@ -51,21 +54,21 @@ dec_gate_up_kernel(const void *__restrict__ x, int H, int I, moe_expert_set rout
   if (nsteps <= 8) {
     // at most two steps per slice: request them before staging the activations
     StepFrag f[2];
-    load_step<Q3>(f[0], mv, r0, slice, slice < nsteps);
-    load_step<Q3>(f[1], mv, r0, slice + 4, slice + 4 < nsteps);
+    load_step<QT>(f[0], mv, r0, slice, slice < nsteps);
+    load_step<QT>(f[1], mv, r0, slice + 4, slice + 4 < nsteps);
     stage_x<SRC_BF16>(x, un.xrow0, un.mask, H, xs, xstride);
     __syncthreads();
-    if (slice < nsteps) mma_step<Q3>(acc, acc2, f[0], xcol, slice * kStepK + 64 * t,
+    if (slice < nsteps) mma_step<QT>(acc, acc2, f[0], xcol, slice * kStepK + 64 * t,
                                      colok && slice * kStepK + 64 * t < H);
-    if (slice + 4 < nsteps) mma_step<Q3>(acc, acc2, f[1], xcol, (slice + 4) * kStepK + 64 * t,
+    if (slice + 4 < nsteps) mma_step<QT>(acc, acc2, f[1], xcol, (slice + 4) * kStepK + 64 * t,
                                          colok && (slice + 4) * kStepK + 64 * t < H);
   } else {
     stage_x<SRC_BF16>(x, un.xrow0, un.mask, H, xs, xstride);
     __syncthreads();
     for (int st = slice; st < nsteps; st += 4) {
       StepFrag f;
-      load_step<Q3>(f, mv, r0, st, true);
-      mma_step<Q3>(acc, acc2, f, xcol, st * kStepK + 64 * t, colok && st * kStepK + 64 * t < H);
+      load_step<QT>(f, mv, r0, st, true);
+      mma_step<QT>(acc, acc2, f, xcol, st * kStepK + 64 * t, colok && st * kStepK + 64 * t < H);
     }
   }
   part[warp][g][2 * t] = acc[0] + acc2[0];
@@ -82,9 +85,10 @@ dec_gate_up_kernel(const void *__restrict__ x, int H, int I, moe_expert_set rout
       hdec[((size_t)u * 8 + col) * I + r0 + row] = __half_as_ushort(__float2half_rn(hv));
     }
   }
+  }  // units
 }
 
-template <bool B, bool Q>
+template <bool B, int Q>
 static cudaError_t launch_gu(dim3 grid, size_t smem, cudaStream_t s, const void *x, int H, int I,
                              const moe_expert_set &routed, const moe_expert_set &sh, const DecUnit *units, Ctrl *ctrl,
                              uint16_t *hdec) {
@@ -101,14 +105,16 @@ cudaError_t launch_decode_gate_up(const void *x, int x_is_bf16, int H, int I, co
                                   const moe_expert_set *shared, const DecUnit *units, int max_units, Ctrl *ctrl,
                                   uint16_t *hdec, cudaStream_t s) {
   const moe_expert_set sh = shared ? *shared : routed;
-  const dim3 grid(max_units, I / 16);
+  // about eight CTAs per SM in all; each walks units grid-stride
+  const int cap = (8 * num_sms() + I / 16 - 1) / (I / 16);
+  const dim3 grid(max_units < cap ? (max_units > 0 ? max_units : 1) : cap, I / 16);
   const size_t smem = (size_t)8 * (H + 4) * 2;
-  const bool q3 = routed.gate.qtype == MOE_Q3;
+  const int qt = routed.gate.qtype;
+#define MOE_GU(B, Q) launch_gu<B, Q>(grid, smem, s, x, H, I, routed, sh, units, ctrl, hdec)
   if (x_is_bf16)
-    return q3 ? launch_gu<true, true>(grid, smem, s, x, H, I, routed, sh, units, ctrl, hdec)
-              : launch_gu<true, false>(grid, smem, s, x, H, I, routed, sh, units, ctrl, hdec);
-  return q3 ? launch_gu<false, true>(grid, smem, s, x, H, I, routed, sh, units, ctrl, hdec)
-            : launch_gu<false, false>(grid, smem, s, x, H, I, routed, sh, units, ctrl, hdec);
+    return qt == MOE_Q3 ? MOE_GU(true, 3) : qt == MOE_Q4 ? MOE_GU(true, 4) : MOE_GU(true, 2);
+  return qt == MOE_Q3 ? MOE_GU(false, 3) : qt == MOE_Q4 ? MOE_GU(false, 4) : MOE_GU(false, 2);
+#undef MOE_GU
 }
 
 // ---------------------------------------------------------------- down (+ weighted combine)
@@ -122,7 +128,7 @@ constexpr int kDownWarps = 16;
 constexpr int kDownSlots = 64;     // h columns staged at once
 constexpr int kDownMaxUnits = 128; // unit records cached in shared memory at a time
 
-template <bool Q3>
+template <int QT>
 __global__ void __launch_bounds__(kDownWarps * 32)
 dec_down_kernel(int H, int I, moe_expert_set routed, moe_expert_set shared, const DecUnit *__restrict__ units,
                 Ctrl *__restrict__ ctrl, const uint16_t *__restrict__ hdec, float *__restrict__ y,
@@ -180,7 +186,7 @@ dec_down_kernel(int H, int I, moe_expert_set routed, moe_expert_set shared, cons
         if (it < n_items && (per_unit > 1 || nsteps == 1)) {
           const DecUnit &un = s_units[u0 + it / per_unit - ub];
           if (un.expert >= 0 && un.expert < (un.set ? shared.down.n_experts : routed.down.n_experts)) {
-            load_step<Q3>(f[j], mat_sel(routed, shared, un.set, 2, un.expert), r0, per_unit > 1 ? it % per_unit : 0,
+            load_step<QT>(f[j], mat_sel(routed, shared, un.set, 2, un.expert), r0, per_unit > 1 ? it % per_unit : 0,
                           true);
             okv[j] = true;
           }
@@ -225,20 +231,20 @@ dec_down_kernel(int H, int I, moe_expert_set routed, moe_expert_set shared, cons
           StepFrag fl;
           if (j == 0 && okv[0]) fl = f[0];
           else if (j == 1 && okv[1]) fl = f[1];
-          else load_step<Q3>(fl, mat_sel(routed, shared, un.set, 2, un.expert), r0, st, true);
-          mma_step<Q3>(acc, acc2, fl, xcol, st * kStepK + 64 * t, colok && st * kStepK + 64 * t < I);
+          else load_step<QT>(fl, mat_sel(routed, shared, un.set, 2, un.expert), r0, st, true);
+          mma_step<QT>(acc, acc2, fl, xcol, st * kStepK + 64 * t, colok && st * kStepK + 64 * t < I);
 #pragma unroll
           for (int e = 0; e < 4; ++e) acc[e] += acc2[e];
         } else {  // rows mode with several K steps: two steps' loads in flight, then their MMAs
           const MatView mv = mat_sel(routed, shared, un.set, 2, un.expert);
           for (int st = 0; st < nsteps; st += 2) {
             StepFrag fl[2];
-            load_step<Q3>(fl[0], mv, r0, st, true);
-            load_step<Q3>(fl[1], mv, r0, st + 1, st + 1 < nsteps);
+            load_step<QT>(fl[0], mv, r0, st, true);
+            load_step<QT>(fl[1], mv, r0, st + 1, st + 1 < nsteps);
 #pragma unroll
             for (int b = 0; b < 2; ++b) {
               const int kb = (st + b) * kStepK + 64 * t;
-              if (st + b < nsteps) mma_step<Q3>(acc, acc2, fl[b], xcol, kb, colok && kb < I);
+              if (st + b < nsteps) mma_step<QT>(acc, acc2, fl[b], xcol, kb, colok && kb < I);
             }
           }
 #pragma unroll
@@ -284,23 +290,20 @@ cudaError_t launch_decode_down(int H, int I, const moe_expert_set &routed, const
   (void)max_units;
   const moe_expert_set sh = shared ? *shared : routed;
   const size_t smem = (size_t)kDownSlots * (I + 4) * 2;
-  const bool q3 = routed.gate.qtype == MOE_Q3;
-  cudaError_t e = q3 ? smem_limit_once(dec_down_kernel<true>, smem) : smem_limit_once(dec_down_kernel<false>, smem);
+  const int qt = routed.gate.qtype;
+  auto fn = qt == MOE_Q3 ? dec_down_kernel<3> : qt == MOE_Q4 ? dec_down_kernel<4> : dec_down_kernel<2>;
+  cudaError_t e = smem_limit_once(fn, smem);
   if (e != cudaSuccess) return e;
   {
     KTimer kt_(KID_DEC_DOWN, s);
-    if (q3)
-      dec_down_kernel<true><<<H / 16, kDownWarps * 32, smem, s>>>(H, I, routed, sh, units, ctrl, hdec, y, residual, T,
-                                                                  out_rows);
-    else
-      dec_down_kernel<false><<<H / 16, kDownWarps * 32, smem, s>>>(H, I, routed, sh, units, ctrl, hdec, y, residual,
-                                                                   T, out_rows);
+    fn<<<H / 16, kDownWarps * 32, smem, s>>>(H, I, routed, sh, units, ctrl, hdec, y, residual, T, out_rows);
   }
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- units for grouped rows
-// rows mode for moe_expert_ffn: group g's rows [off[g], off[g+1]) in chunks of 8 columns. One
+// rows mode for moe_expert_ffn: group g's rows [off[g], off[g+1]) in chunks of 8 columns (only
+// groups of at most max_rows rows when max_rows > 0: the larger ones go to the grouped GEMM). One
 // CTA: each thread takes a group, a block-wide exclusive scan of the groups' chunk counts gives
 // each group's first unit, and the groups are walked in blocks of kUnitsThreads. Units come out
 // in group order, then row order, as a serial walk would produce them.
@@ -308,7 +311,7 @@ constexpr int kUnitsThreads = 1024;
 
 __global__ void __launch_bounds__(kUnitsThreads)
 units_from_offsets_kernel(const int32_t *__restrict__ off, int n_groups, int shared_group, int n_rows,
-                          DecUnit *__restrict__ units, Ctrl *__restrict__ ctrl) {
+                          int max_rows, DecUnit *__restrict__ units, Ctrl *__restrict__ ctrl) {
   __shared__ int s_warp[kUnitsThreads / 32];
   __shared__ int s_base, s_bad;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -335,7 +338,7 @@ units_from_offsets_kernel(const int32_t *__restrict__ off, int n_groups, int sha
     if (gi < n_groups) {
       a = off[gi];
       nrow = off[gi + 1] - a;
-      cnt = (nrow + 7) / 8;
+      cnt = (max_rows > 0 && nrow > max_rows) ? 0 : (nrow + 7) / 8;  // larger groups: the grouped GEMM
     }
     int incl = cnt;
 #pragma unroll
@@ -375,11 +378,11 @@ units_from_offsets_kernel(const int32_t *__restrict__ off, int n_groups, int sha
 }
 
 cudaError_t launch_decode_units_from_offsets(const int32_t *offsets, int n_groups, int has_shared_group, int n_rows,
-                                             DecUnit *units, Ctrl *ctrl, cudaStream_t s) {
+                                             DecUnit *units, Ctrl *ctrl, cudaStream_t s, int max_rows) {
   {
     KTimer kt_(KID_DEC_UNITS, s);
     units_from_offsets_kernel<<<1, kUnitsThreads, 0, s>>>(offsets, n_groups, has_shared_group ? n_groups - 1 : -1,
-                                                          n_rows, units, ctrl);
+                                                          n_rows, max_rows, units, ctrl);
   }
   return cudaGetLastError();
 }

@@ -10,31 +10,35 @@
 // then sees the layer's expert bytes requested within a few hundred nanoseconds instead of as a
 // chain of dependent round trips.
 //
-// One grid of one CTA per SM (16 warps) runs three phases with two grid barriers:
+// One grid of one CTA per SM (16 warps) runs three phases with one grid barrier:
 //   P1  router logits: four warps per expert split H (the fp32 router rows are requested before
 //       the tokens are staged); the shared expert's rows are prefetched into L2 meanwhile.
 //   --  grid barrier
-//   P1b every CTA computes the same top-k (each warp sorts a 32-expert slice, one warp per token
-//       merges the slices' heads) and the distinct-expert unit list (deterministic), so no second
-//       exchange is needed. The warps then issue this CTA's copies: gate/up items (unit, 8
-//       features: 8 gate rows + 8 up rows over all of H) dealt round-robin over CTAs, then the
-//       down rows of the CTA's 16 output features for every unit.
+//   P1b every CTA computes the same top-k (a threshold from each 32-expert chunk's largest logits,
+//       then one warp sorts the few logits above it) and the distinct-expert unit list
+//       (deterministic), so no second exchange is needed. The warps then issue this CTA's
+//       copies: gate/up items (unit, 8 features: 8 gate + 8 up rows over all of H) dealt
+//       round-robin over CTAs, then the down rows of the CTA's 16 output features for every unit.
 //   P2  gate/up + SwiGLU: two groups of 8 warps take alternate items; in a group warp j runs
 //       K step j (256 wide) on the tensor cores (mma.sync m16n8k16 with A rows 0-7 = gate and
 //       8-15 = up rows of the same features, fp16 operands, fp32 accumulate); the partials are
-//       summed in fixed order and h goes to the workspace.
-//   --  grid barrier
+//       summed in fixed order, h goes to the workspace and the item is counted on its unit's
+//       readiness counter (a release add).
 //   P3  down projection fused with the weighted combine: each CTA owns 16 output features, its
 //       warps take whole units (16 down rows over all of I, the half steps' loads issued
-//       together), partials are reduced in fixed order (no atomics).
+//       together). A unit's warp waits only for that unit's counter to reach its item count (no
+//       second grid barrier: early units' down work overlaps later units' gate/up), stages the
+//       unit's h columns, and runs; partials are reduced in fixed order (no atomics).
 // Each slot's fills are consumed in phase order: the ring has an even number of slots so the
-// gate/up items sharing a slot fall to one group, and a down piece first waits until the piece
-// one ring behind it is consumed. A parity wait can then never run two phases ahead of its
-// slot's last completed fill, where it would take the older phase for its own.
-// The grid barrier is one 64-bit arrival counter in the workspace (every launch adds 2 x grid;
-// a CTA waits for the launch's base + j x grid). It and every mbarrier wait are bounded in time
-// and report MOE_ERR_TIMEOUT instead of hanging; before the CTA exits every thread waits for its
-// own outstanding copies (cp.async.wait_all), so no copy is still writing its shared memory.
+// gate/up items sharing a slot fall to one group, a CTA barrier separates a CTA's P2 from its
+// P3, and a down piece first waits until the piece one ring behind it is consumed. A parity wait
+// can then never run two phases ahead of its slot's last completed fill, where it would take the
+// older phase for its own.
+// The grid barrier is one 64-bit arrival counter in the workspace (every launch adds the grid
+// size; a CTA waits for the launch's base + grid). It, the readiness waits and every mbarrier
+// wait are bounded in time and report MOE_ERR_TIMEOUT instead of hanging; before the CTA exits
+// every thread waits for its own outstanding copies (cp.async.wait_all), so no copy is still
+// writing its shared memory.
 #include "common.cuh"
 #include "dequant.cuh"
 #include "gemv.cuh"
@@ -71,6 +75,7 @@ struct FusedArgs {
   int32_t *idx;
   float *w;
   uint16_t *hdec;
+  unsigned *ready;  // per unit: gate/up items whose h is written (zeroed before the first barrier)
   Ctrl *ctrl;
   int ring;        // slots in the ring
   int slot_bytes;  // bytes per slot
@@ -79,8 +84,28 @@ struct FusedArgs {
   int dpu;         // units per down slot
 };
 
+// matrix pointers of one decode unit (gate, up, down), looked up once per unit
+struct UnitMats {
+  const uint8_t *codes[3];
+  const uint16_t *scales[3];
+  const uint8_t *hibits[3];
+};
+
+// Per-layer pointers of a stack run in one launch (moe_stack_forward at decode sizes): the kernel
+// walks the layers with a grid barrier between them. Passed as a kernel parameter (~12 KB for
+// kStackMaxL layers; longer stacks are launched in pieces).
+constexpr int kStackMaxL = 48;
+struct StackLayers {
+  int n;                                 // layers in this launch
+  const float *Wr[kStackMaxL];
+  const float *bias[kStackMaxL];         // entries may be NULL
+  moe_expert_set routed[kStackMaxL];
+  moe_expert_set shared[kStackMaxL];     // used when has_shared
+};
+
 struct FusedLayout {
-  size_t xraw, x16, hs, part, red, units, sidx, sw, misc, slot, src, plist, firstof, pcnt, bars, ring, total;
+  size_t xraw, x16, hs, part, red, units, umats, sidx, sw, misc, slot, src, keys, ctop, cand, firstof, pcnt, bars, ring,
+      total;
 };
 
 __host__ __device__ inline size_t fl_align(size_t v, size_t a = 16) { return (v + a - 1) & ~(a - 1); }
@@ -95,12 +120,15 @@ __host__ __device__ inline FusedLayout fused_layout(int T, int H, int E, int I, 
   L.part = take((size_t)2 * 2 * 8 * 16 * 8 * 4);  // [group][buffer][K step][16 rows][8 columns]
   L.red = take((size_t)kFWarps * 16 * 8 * 4);
   L.units = take((size_t)kFMaxUnits * sizeof(DecUnit));
+  L.umats = take((size_t)kFMaxUnits * sizeof(UnitMats));
   L.sidx = take((size_t)kDecodeMaxT * kMaxK * 4);
   L.sw = take((size_t)kDecodeMaxT * kMaxK * 4);
   L.misc = take(16 * 4);
   L.slot = take((size_t)(kFMaxUnits + 1) * 4);
   L.src = take((size_t)kFSlots * 4);
-  L.plist = take((size_t)T * 16 * 16 * 8);      // top-16 code lists: [token][rank][32-expert chunk]
+  L.keys = take((size_t)T * E * 4);              // [token][expert] order-preserving logit keys
+  L.ctop = take((size_t)T * 32 * 8);             // [token][32] chunk-top codes (threshold candidates)
+  L.cand = take((size_t)T * 32 * 8 + 128);       // [token][32] codes above the threshold, [8] counts, [8] tau
   L.firstof = take((size_t)E * 4);                // expert -> first pair choosing it
   L.pcnt = take((size_t)(kFMaxUnits + 1) * 4);
   L.bars = take((size_t)kFMaxRing * 8);
@@ -154,6 +182,23 @@ __device__ __forceinline__ void prefetch_range(const void *p, size_t bytes, int 
   for (size_t off = (size_t)first * 128; off < bytes; off += (size_t)nthr * 128) prefetch_l2(c + off);
 }
 
+// an expert set's single (shared) expert into L2, lines spread over the grid's threads
+template <int QT>
+__device__ __forceinline__ void prefetch_shared(const moe_expert_set &sh, int I, int H, int first, int nthr) {
+  const size_t cb = (size_t)I * code_row_bytes(QT, H), sb = (size_t)I * H / 32 * 2;
+  prefetch_range(sh.gate.codes, cb, first, nthr);
+  prefetch_range(sh.up.codes, cb, first, nthr);
+  prefetch_range(sh.down.codes, cb, first, nthr);
+  prefetch_range(sh.gate.scales, sb, first, nthr);
+  prefetch_range(sh.up.scales, sb, first, nthr);
+  prefetch_range(sh.down.scales, sb, first, nthr);
+  if (QT == 3) {
+    prefetch_range(sh.gate.hibits, cb / 2, first, nthr);
+    prefetch_range(sh.up.hibits, cb / 2, first, nthr);
+    prefetch_range(sh.down.hibits, cb / 2, first, nthr);
+  }
+}
+
 // 16-byte global -> shared async copy (L2 only); both addresses 16-byte aligned
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -169,70 +214,74 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// One contiguous piece of a slot fill, as (source, offset in the slot, bytes).
-//   gate/up slot: [gate codes 8 x H/4][up codes 8 x H/4][gate scales 8 x H/32][up scales]
-//                 [gate hi 8 x H/8][up hi]                     (5H bytes; Q3 7H)
-//   down slot:    dpu pieces of [codes 16 x I/4][scales 16 x I/32][hi 16 x I/8]   (5I; Q3 7I)
+// One contiguous piece of a slot fill, as (source, offset in the slot, bytes). With CR the code
+// bytes of one gate/up row (H/4; H/2 for the 4-bit plane) and CD those of one down row:
+//   gate/up slot: [gate codes 8 x CR][up codes 8 x CR][gate scales 8 x H/32][up scales]
+//                 [gate hi 8 x H/8][up hi]                     (Q2 5H bytes, Q3 7H, Q4 9H)
+//   down slot:    dpu pieces of [codes 16 x CD][scales 16 x I/32][hi 16 x I/8]   (Q2 5I, Q3 7I, Q4 9I)
 struct CopyDesc {
   const void *src;
   uint32_t off, bytes;
 };
 
-template <bool Q3>
-__device__ __forceinline__ CopyDesc gu_copy(const FusedArgs &a, const DecUnit &un, int r0, int c) {
-  const int H = a.H;
+template <int QT>
+__device__ __forceinline__ CopyDesc gu_copy(const FusedArgs &a, const UnitMats &um, int r0, int c) {
+  const int H = a.H, CR = code_row_bytes(QT, H);
   const int which = c & 1;  // 0 gate, 1 up
-  const MatView m = mat_sel(a.routed, a.shared, un.set, which, un.expert);
   CopyDesc d;
   if (c < 2) {
-    d.src = m.codes + (size_t)r0 * (H / 4);
-    d.bytes = 2 * H;
-    d.off = which * 2 * H;
+    d.src = um.codes[which] + (size_t)r0 * CR;
+    d.bytes = 8 * CR;
+    d.off = which * 8 * CR;
   } else if (c < 4) {
-    d.src = m.scales + (size_t)r0 * (H / 32);
+    d.src = um.scales[which] + (size_t)r0 * (H / 32);
     d.bytes = H / 2;
-    d.off = 4 * H + which * (H / 2);
+    d.off = 16 * CR + which * (H / 2);
   } else {
-    d.src = m.hibits + (size_t)r0 * (H / 8);
+    d.src = um.hibits[which] + (size_t)r0 * (H / 8);
     d.bytes = H;
-    d.off = 5 * H + which * H;
+    d.off = 16 * CR + H + which * H;
   }
   return d;
 }
 
-template <bool Q3>
-__device__ __forceinline__ CopyDesc dn_copy(const FusedArgs &a, const DecUnit &un, int rb, int slot_unit, int c) {
-  const int I = a.I;
-  const MatView m = mat_sel(a.routed, a.shared, un.set, 2, un.expert);
+template <int QT>
+__device__ __forceinline__ CopyDesc dn_copy(const FusedArgs &a, const UnitMats &um, int rb, int slot_unit, int c) {
+  const int I = a.I, CD = code_row_bytes(QT, I);
   const size_t row = (size_t)rb * 16;
   const uint32_t base = (uint32_t)(slot_unit * a.dn_bytes);
   CopyDesc d;
   if (c == 0) {
-    d.src = m.codes + row * (I / 4);
-    d.bytes = 4 * I;
+    d.src = um.codes[2] + row * CD;
+    d.bytes = 16 * CD;
     d.off = base;
   } else if (c == 1) {
-    d.src = m.scales + row * (I / 32);
+    d.src = um.scales[2] + row * (I / 32);
     d.bytes = I;
-    d.off = base + 4 * I;
+    d.off = base + 16 * CD;
   } else {
-    d.src = m.hibits + row * (I / 8);
+    d.src = um.hibits[2] + row * (I / 8);
     d.bytes = 2 * I;
-    d.off = base + 5 * I;
+    d.off = base + 16 * CD + I;
   }
   return d;
 }
 
 // one lane's share of a 16-row x 256-wide K step read from a staged slot: the code rows of MMA
 // rows g and g+8 start at ca / cb, their scales at sa / sb (halves), their hi bits at ha / hb
-template <bool Q3>
+template <int QT>
 __device__ __forceinline__ void frag_from_smem(StepFrag &f, const uint8_t *ca, const uint8_t *cb, const uint16_t *sa,
                                                const uint16_t *sb, const uint8_t *ha, const uint8_t *hb, int k0) {
-  f.w0 = *reinterpret_cast<const uint4 *>(ca + k0 / 4);
-  f.w1 = *reinterpret_cast<const uint4 *>(cb + k0 / 4);
+  const int co = code_row_bytes(QT, k0);
+  f.w0 = *reinterpret_cast<const uint4 *>(ca + co);
+  f.w1 = *reinterpret_cast<const uint4 *>(cb + co);
+  if (QT == 4) {
+    f.w0b = *reinterpret_cast<const uint4 *>(ca + co + 16);
+    f.w1b = *reinterpret_cast<const uint4 *>(cb + co + 16);
+  }
   f.d0 = *reinterpret_cast<const uint32_t *>(sa + k0 / 32);
   f.d1 = *reinterpret_cast<const uint32_t *>(sb + k0 / 32);
-  if (Q3) {
+  if (QT == 3) {
     f.h0 = *reinterpret_cast<const uint2 *>(ha + k0 / 8);
     f.h1 = *reinterpret_cast<const uint2 *>(hb + k0 / 8);
   }
@@ -242,8 +291,8 @@ __device__ __forceinline__ void frag_from_smem(StepFrag &f, const uint8_t *ca, c
 
 // TMAX: the largest token count the instance takes (1, 2, 4 or 8); the token loops of the router
 // are unrolled to TMAX, so the common single-token instance carries no code for the others.
-template <bool Q3, int TMAX>
-__global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedArgs a) {
+template <int QT, int TMAX, bool STACK>
+__device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers *SL) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int T = a.T, H = a.H, E = a.E, k = a.k, I = a.I;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
@@ -255,12 +304,17 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   float *part = reinterpret_cast<float *>(smem + L.part);
   float *red = reinterpret_cast<float *>(smem + L.red);
   DecUnit *su = reinterpret_cast<DecUnit *>(smem + L.units);
+  UnitMats *s_um = reinterpret_cast<UnitMats *>(smem + L.umats);
   int32_t *s_idx = reinterpret_cast<int32_t *>(smem + L.sidx);
   float *s_w = reinterpret_cast<float *>(smem + L.sw);
   int *misc = reinterpret_cast<int *>(smem + L.misc);
   int *s_slot = reinterpret_cast<int *>(smem + L.slot);
   int *s_src = reinterpret_cast<int *>(smem + L.src);
-  unsigned long long *plist = reinterpret_cast<unsigned long long *>(smem + L.plist);
+  uint32_t *s_key = reinterpret_cast<uint32_t *>(smem + L.keys);
+  unsigned long long *s_ctop = reinterpret_cast<unsigned long long *>(smem + L.ctop);
+  unsigned long long *s_cand = reinterpret_cast<unsigned long long *>(smem + L.cand);
+  int *s_ccnt = reinterpret_cast<int *>(smem + L.cand + (size_t)T * 32 * 8);  // [token] candidates found
+  unsigned long long *s_tau = reinterpret_cast<unsigned long long *>(s_ccnt + kDecodeMaxT);  // [token] threshold
   int *s_firstof = reinterpret_cast<int *>(smem + L.firstof);
   int *s_pcnt = reinterpret_cast<int *>(smem + L.pcnt);
   const uint32_t bar_full0 = smem_u32(smem + L.bars);
@@ -274,7 +328,8 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   const unsigned nblk = gridDim.x;
   __shared__ unsigned long long s_base;
   __shared__ volatile int s_abort;
-  if (tid == 0) {  // arrivals of earlier launches: a whole number of 2 x grid (before this CTA arrives)
+  __shared__ int s_pbase[kFMaxRing];  // phases each slot completed in earlier layers of this launch
+  if (tid == 0) {  // arrivals of earlier launches: a whole number of grids (before this CTA arrives)
     unsigned long long v;
     asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(&ctrl->bar_arrivals) : "memory");
     s_base = v - v % nblk;
@@ -282,6 +337,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
     for (int s = 0; s < R; ++s) mbar_init(full(s), 32);  // one arrival per lane of the filling warp
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if (tid < kFMaxRing) s_pbase[tid] = 0;
   // a bounded wait that gives up at once after an earlier wait of this CTA gave up
   auto wait_bar = [&](uint32_t bar, uint32_t parity, int where) -> bool {
     if (s_abort) return false;
@@ -290,6 +346,20 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
     set_device_error(ctrl, MOE_ERR_TIMEOUT, where);
     return false;
   };
+  // parity of fill q's phase: the slot's phases of earlier layers, then one per fill q, q + R, ...
+  auto fill_parity = [&](int q) { return (uint32_t)(s_pbase[q % R] + q / R) & 1u; };
+  const int nl = STACK ? SL->n : 1;
+  bool ok = true;
+
+  for (int l = 0; l < nl; ++l) {
+  // this layer's pointers: the launch's arguments, or stack layer l (its input and residual are
+  // the stream r: r_in for the first layer, then r_out, which every layer updates in place)
+  const float *const lWr = STACK ? SL->Wr[l] : a.Wr;
+  const float *const lbias = STACK ? SL->bias[l] : a.bias;
+  const moe_expert_set &lRS = STACK ? SL->routed[l] : a.routed;
+  const moe_expert_set &lSS = STACK ? SL->shared[l] : a.shared;
+  const float *const lrn = (STACK && l > 0) ? a.y : a.r_norm;
+  const float *const lres = (STACK && l > 0) ? a.y : a.residual;
 
   // ---------------- P0: this warp's router rows are requested first, then the tokens are staged
   const int H4 = H / 4, HQ = H4 / 4;  // float4 per quarter of a router row (<= 128: H <= 2048)
@@ -299,22 +369,26 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int h4 = lane + 32 * u;
-      rv[u] = (e < E && h4 < HQ) ? __ldcs(reinterpret_cast<const float4 *>(a.Wr + (size_t)e * H) + qh * HQ + h4)
+      rv[u] = (e < E && h4 < HQ) ? __ldcs(reinterpret_cast<const float4 *>(lWr + (size_t)e * H) + qh * HQ + h4)
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   };
   load_router((int)blockIdx.x + es * G);
   __shared__ float s_inv[kDecodeMaxT];
-  if (a.r_norm) {
+  if (lrn) {
     // RMSNorm of the residual stream (no gain): the same summation order and rounding as the
     // stand-alone RMSNorm kernel (256 threads: strided fmaf chains, warp butterflies, 8 warp
-    // partials in order), so u is bit-identical to it
+    // partials in order), so u is bit-identical to it. Coherent (L2) loads: in a stack launch
+    // the stream was written by other CTAs in the previous layer.
     __shared__ float s_part[kDecodeMaxT][8];
     if (tid < 256) {
       for (int t = 0; t < T; ++t) {
-        const float *row = a.r_norm + (size_t)t * H;
+        const float *row = lrn + (size_t)t * H;
         float ss = 0.0f;
-        for (int h = tid; h < H; h += 256) ss = fmaf(__ldg(row + h), __ldg(row + h), ss);
+        for (int h = tid; h < H; h += 256) {
+          const float rv1 = __ldcg(row + h);
+          ss = fmaf(rv1, rv1, ss);
+        }
         ss = warp_sum(ss);
         if (lane == 0) s_part[t][warp] = ss;
       }
@@ -332,10 +406,10 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
     const int H8 = H / 8, n = T * H8;
     for (int i = tid; i < n; i += kFThreads) {
       uint4 v;
-      if (a.r_norm) {
+      if (lrn) {
         const int t = i / H8;
-        const float4 f0 = __ldg(reinterpret_cast<const float4 *>(a.r_norm) + 2 * i);
-        const float4 f1 = __ldg(reinterpret_cast<const float4 *>(a.r_norm) + 2 * i + 1);
+        const float4 f0 = __ldcg(reinterpret_cast<const float4 *>(lrn) + 2 * i);
+        const float4 f1 = __ldcg(reinterpret_cast<const float4 *>(lrn) + 2 * i + 1);
         const float iv = s_inv[t];
         auto pk = [&](float lo, float hi) {
           const __nv_bfloat16 bl = __float2bfloat16_rn(lo * iv), bh = __float2bfloat16_rn(hi * iv);
@@ -360,7 +434,10 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       d[1] = make_uint2(o[2], o[3]);
     }
   }
-  if (a.bias) prefetch_range(a.bias, (size_t)E * 4, tid, kFThreads);
+  if (lbias) prefetch_range(lbias, (size_t)E * 4, tid, kFThreads);
+  // per-unit readiness counters start at zero; every increment comes after the first grid barrier
+  if (blockIdx.x == 0)
+    for (int u = tid; u <= T * k; u += kFThreads) a.ready[u] = 0u;
   __syncthreads();
 
   // ---------------- P1: router logits, four warps per expert (each a quarter of H), fp32
@@ -408,64 +485,98 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       __syncthreads();
     }
   }
-  bool ok = grid_barrier(ctrl, s_base + nblk, 31, true);
+  ok = grid_barrier(ctrl, s_base + (unsigned long long)(2 * l + 1) * nblk, 31, true) && ok;
 
   // ---------------- P1b: top-k and unit list, computed identically by every CTA
   if (ok) {
-    // every 32-expert chunk of every token is sorted by one warp straight from the logits
-    // (64-bit codes: order-preserving key, then ~index, so the lower index wins ties; top 16
-    // kept); then one warp per token merges the chunks' lists: lane c holds list c in
-    // registers, each round the warp takes the best head (max key, then lowest index) and that
-    // lane shifts its list
-    const int nch = (E + 31) / 32;  // <= 16
+    // Top-k by threshold. Codes are (order-preserving 32-bit key of logit + bias) << 32 | ~index,
+    // so code order is the routing order (larger logit first, equal logits: lower index first)
+    // and codes are unique. (1) For every token each 32-expert chunk gives its m = ceil(k / nch)
+    // largest codes (warp max reductions); the k-th largest of these nch * m <= 31 chunk tops is a
+    // threshold tau no larger than the token's k-th largest code, since k distinct codes reach it.
+    // (2) The codes >= tau (at least k; with the router's logits ~15, never more than 32 in the
+    // workloads' statistics) are gathered and one warp sorts them: its first k lanes are the
+    // top-k. (3) If more than 32 codes reach tau (mass ties), the warp instead takes k rounds of
+    // arg-max over all E codes of the token.
+    const int nch = (E + 31) / 32;       // <= 16
+    const int m = (k + nch - 1) / nch;   // chunk tops per chunk: nch * m <= nch + k - 1 <= 31
+#pragma unroll 1
     for (int task = warp; task < T * nch; task += kFWarps) {
       const int t = task / nch, c = task % nch, e = c * 32 + lane;
-      unsigned long long v = 0ull;
-      if (e < E) v = topk_code(__ldcg(a.logits + (size_t)t * E + e) + (a.bias ? __ldg(a.bias + e) : 0.f), e);
-      v = warp_sort32_desc(v);
-      if (lane < 16) plist[((size_t)t * 16 + lane) * 16 + c] = v;  // rank-major: the merge reads across chunks
+      uint32_t key = 0u;
+      if (e < E) {
+        key = logit_key(__ldcg(a.logits + (size_t)t * E + e) + (lbias ? __ldg(lbias + e) : 0.f));
+        s_key[t * E + e] = key;
+      }
+      const uint32_t nidx = (e < E) ? 0xFFFFFFFFu - (uint32_t)e : 0u;
+      uint32_t live = key;
+#pragma unroll 1
+      for (int r = 0; r < m; ++r) {  // the chunk's r-th largest code
+        const uint32_t mk = __reduce_max_sync(0xffffffffu, live);
+        const uint32_t lo = __reduce_max_sync(0xffffffffu, (live == mk) ? nidx : 0u);
+        if (lane == 0) s_ctop[t * 32 + c * m + r] = ((unsigned long long)mk << 32) | lo;
+        if (live == mk && nidx == lo) live = 0u;
+      }
     }
     {  // into L2 while the top-k runs: the shared expert's rows (always selected)
       const int nthr = gridDim.x * kFThreads, first = blockIdx.x * kFThreads + tid;
-      if (a.has_shared) {
-        const size_t cb = (size_t)I * H / 4, sb = (size_t)I * H / 32 * 2;
-        prefetch_range(a.shared.gate.codes, cb, first, nthr);
-        prefetch_range(a.shared.up.codes, cb, first, nthr);
-        prefetch_range(a.shared.down.codes, cb, first, nthr);
-        prefetch_range(a.shared.gate.scales, sb, first, nthr);
-        prefetch_range(a.shared.up.scales, sb, first, nthr);
-        prefetch_range(a.shared.down.scales, sb, first, nthr);
-        if (Q3) {
-          prefetch_range(a.shared.gate.hibits, cb / 2, first, nthr);
-          prefetch_range(a.shared.up.hibits, cb / 2, first, nthr);
-          prefetch_range(a.shared.down.hibits, cb / 2, first, nthr);
-        }
-      }
+      if (a.has_shared && !(STACK && l > 0)) prefetch_shared<QT>(lSS, I, H, first, nthr);  // later layers: earlier
     }
     if (T > 1)
       for (int e = tid; e < E; e += kFThreads) s_firstof[e] = 0x7fffffff;
     __syncthreads();
+    if (warp < T) {  // the threshold: the k-th largest chunk top
+      const unsigned long long v = warp_sort32_desc(lane < nch * m ? s_ctop[warp * 32 + lane] : 0ull);
+      if (lane == k - 1) s_tau[warp] = v;
+      if (lane == 0) s_ccnt[warp] = 0;
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int task = warp; task < T * nch; task += kFWarps) {  // gather the codes >= tau
+      const int t = task / nch, e = (task % nch) * 32 + lane;
+      const unsigned long long code =
+          (e < E) ? ((unsigned long long)s_key[t * E + e] << 32) | (0xFFFFFFFFu - (uint32_t)e) : 0ull;
+      const bool in = (e < E) && code >= s_tau[t];
+      const unsigned bal = __ballot_sync(0xffffffffu, in);
+      int base = 0;
+      if (lane == 0 && bal) base = atomicAdd(&s_ccnt[t], __popc(bal));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      const int pos = base + __popc(bal & ((1u << lane) - 1u));
+      if (in && pos < 32) s_cand[t * 32 + pos] = code;
+    }
+    __syncthreads();
     if (warp < T) {
-      unsigned long long c[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) c[i] = (lane < nch) ? plist[((size_t)warp * 16 + i) * 16 + lane] : 0ull;
-      float my_val = -INFINITY;
-      int my_idx = 0;
-      for (int j = 0; j < k; ++j) {
-        const uint32_t hk = (uint32_t)(c[0] >> 32);
-        const uint32_t m = __reduce_max_sync(0xffffffffu, hk);
-        const uint32_t lo = (hk == m) ? (uint32_t)c[0] : 0u;
-        const uint32_t win = __reduce_max_sync(0xffffffffu, lo);  // max of (~index) = lowest index
-        const bool is_win = (hk == m) && ((uint32_t)c[0] == win);
-#pragma unroll
-        for (int i = 0; i < 15; ++i) c[i] = is_win ? c[i + 1] : c[i];
-        c[15] = is_win ? 0ull : c[15];
-        if (lane == j) {
-          my_val = key_to_logit(m);
-          my_idx = (int)(0xFFFFFFFFu - win);
+      const int t = warp, n = s_ccnt[t];
+      unsigned long long *sel = s_ctop + t * 32;  // reused: the selected codes in slot order
+      if (n <= 32) {  // sort the candidates: lane r holds the r-th largest
+        const unsigned long long v = warp_sort32_desc(lane < n ? s_cand[t * 32 + lane] : 0ull);
+        if (lane < k) sel[lane] = v;
+      } else {  // mass ties: k rounds of arg-max over the token's E codes
+        uint32_t taken = 0u;  // bit i: expert lane + 32 i already selected
+#pragma unroll 1
+        for (int j = 0; j < k; ++j) {
+          unsigned long long best = 0ull;
+          int bi = -1;
+#pragma unroll 1
+          for (int i = 0; i < nch; ++i) {
+            const int e = lane + 32 * i;
+            if (e >= E || ((taken >> i) & 1u)) continue;
+            const unsigned long long code = ((unsigned long long)s_key[t * E + e] << 32) | (0xFFFFFFFFu - (uint32_t)e);
+            if (code > best) {
+              best = code;
+              bi = i;
+            }
+          }
+          const uint32_t mk = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32));
+          const uint32_t lo = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32) == mk ? (uint32_t)best : 0u);
+          if (bi >= 0 && (uint32_t)(best >> 32) == mk && (uint32_t)best == lo) taken |= 1u << bi;
+          if (lane == 0) sel[j] = ((unsigned long long)mk << 32) | lo;
         }
       }
-      topk_finish(my_val, my_idx, k, s_idx + warp * k, s_w + warp * k);
+      __syncwarp();
+      const unsigned long long v = lane < k ? sel[lane] : 0ull;
+      topk_finish(key_to_logit((uint32_t)(v >> 32)), (int)(0xFFFFFFFFu - (uint32_t)v), k, s_idx + t * k,
+                  s_w + t * k);
     }
     __syncthreads();
     const int P = T * k;
@@ -555,6 +666,15 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
         a.w[i] = s_w[i];
       }
     __syncthreads();
+    // each unit's gate / up / down plane pointers, looked up once (the fills read them from here)
+    for (int i = tid; i < 3 * misc[0]; i += kFThreads) {
+      const int u = i / 3, which = i % 3;
+      const MatView mv = mat_sel(lRS, lSS, su[u].set, which, su[u].expert);
+      s_um[u].codes[which] = mv.codes;
+      s_um[u].scales[which] = mv.scales;
+      s_um[u].hibits[which] = mv.hibits;
+    }
+    __syncthreads();
   }
   const int nu = ok ? misc[0] : 0;
   const int rbs8 = I / 8;                     // gate/up items per unit
@@ -574,11 +694,12 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
     const uint32_t dst0 = ring0 + (uint32_t)(s * S);
     if (q < n_mine) {
       const int i = (int)blockIdx.x + q * G;
-      const DecUnit &un = su[i / rbs8];
+      const UnitMats &um = s_um[i / rbs8];
       const int r0 = (i % rbs8) * 8;
-      const int nc = Q3 ? 6 : 4;
+      const int nc = QT == 3 ? 6 : 4;
+#pragma unroll 1
       for (int c = 0; c < nc; ++c) {
-        const CopyDesc d = gu_copy<Q3>(a, un, r0, c);
+        const CopyDesc d = gu_copy<QT>(a, um, r0, c);
         const char *src = static_cast<const char *>(d.src);
         for (uint32_t off = 16u * lane; off < d.bytes; off += 512u) cp_async16(dst0 + d.off + off, src + off);
       }
@@ -586,11 +707,12 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       const int j = q - n_mine, rbl = j / npieces, dp = j % npieces;
       const int rb = (int)blockIdx.x + rbl * G;
       const int nun = min(a.dpu, nu - dp * a.dpu);
-      const int per = Q3 ? 3 : 2;
+      const int per = QT == 3 ? 3 : 2;
       for (int m = 0; m < nun; ++m) {
-        const DecUnit &un = su[dp * a.dpu + m];
+        const UnitMats &um = s_um[dp * a.dpu + m];
+#pragma unroll 1
         for (int c = 0; c < per; ++c) {
-          const CopyDesc d = dn_copy<Q3>(a, un, rb, m, c);
+          const CopyDesc d = dn_copy<QT>(a, um, rb, m, c);
           const char *src = static_cast<const char *>(d.src);
           for (uint32_t off = 16u * lane; off < d.bytes; off += 512u) cp_async16(dst0 + d.off + off, src + off);
         }
@@ -613,18 +735,19 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       const int u = i / rbs8, r0 = (i % rbs8) * 8;
       const DecUnit &un = su[u];
       const int s = q % R;
-      const bool have = wait_bar(full(s), (uint32_t)(q / R) & 1u, 42);
+      const bool have = wait_bar(full(s), fill_parity(q), 42);
       float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
       const int k0 = j8 * kStepK + 64 * t4;
       if (have && j8 < nsteps_gu && k0 < H) {
         const uint8_t *sl = ringp + (size_t)s * S;
-        const uint8_t *ca = sl + (size_t)g * (H / 4), *cb = sl + 2 * H + (size_t)g * (H / 4);
-        const uint16_t *sa = reinterpret_cast<const uint16_t *>(sl + 4 * H) + (size_t)g * (H / 32);
-        const uint16_t *sb = reinterpret_cast<const uint16_t *>(sl + 4 * H + H / 2) + (size_t)g * (H / 32);
-        const uint8_t *ha = sl + 5 * H + (size_t)g * (H / 8), *hb = sl + 6 * H + (size_t)g * (H / 8);
+        const int CR = code_row_bytes(QT, H);
+        const uint8_t *ca = sl + (size_t)g * CR, *cb = sl + 8 * CR + (size_t)g * CR;
+        const uint16_t *sa = reinterpret_cast<const uint16_t *>(sl + 16 * CR) + (size_t)g * (H / 32);
+        const uint16_t *sb = reinterpret_cast<const uint16_t *>(sl + 16 * CR + H / 2) + (size_t)g * (H / 32);
+        const uint8_t *ha = sl + 16 * CR + H + (size_t)g * (H / 8), *hb = sl + 16 * CR + 2 * H + (size_t)g * (H / 8);
         StepFrag f;
-        frag_from_smem<Q3>(f, ca, cb, sa, sb, ha, hb, k0);
-        mma_step<Q3>(acc, acc2, f, x16 + (size_t)g * xs16, k0, (un.mask >> g) & 1);
+        frag_from_smem<QT>(f, ca, cb, sa, sb, ha, hb, k0);
+        mma_step<QT>(acc, acc2, f, x16 + (size_t)g * xs16, k0, (un.mask >> g) & 1);
       }
       float *pw = part + (((size_t)(grp * 2 + buf) * 8 + j8) * 16) * 8;
       pw[g * 8 + 2 * t4] = acc[0] + acc2[0];
@@ -648,9 +771,27 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
           a.hdec[((size_t)u * 8 + col) * I + r0 + row] = __half_as_ushort(__float2half_rn(hv));
         }
       }
+      // the item's h is written: count it for its unit (the group barrier orders the 64 stores
+      // before the release add, as in the grid barrier)
+      named_sync(kBarGroup0 + grp, 256);
+      if (gtid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(a.ready + u) : "memory");
     }
   }
-  ok = grid_barrier(ctrl, s_base + 2 * (unsigned long long)nblk, 32, ok) && ok;
+  // This CTA's gate/up items are all consumed (the ring rule of P3 below needs it); no grid
+  // barrier: each down unit waits for its own unit's h instead.
+  __syncthreads();
+  if (STACK && l + 1 < nl) {
+    // into L2 for the next layer while this one finishes: this CTA's router rows (the experts its
+    // warps load first), the router bias, and a share of the next shared expert
+    const int nthr = gridDim.x * kFThreads, first = blockIdx.x * kFThreads + tid;
+    const float *nWr = SL->Wr[l + 1];
+    for (int es2 = 0; es2 < 4; ++es2) {
+      const int e = (int)blockIdx.x + es2 * G;
+      if (e < E) prefetch_range(nWr + (size_t)e * H, (size_t)H * 4, tid, kFThreads);
+    }
+    if (SL->bias[l + 1] && blockIdx.x == 1) prefetch_range(SL->bias[l + 1], (size_t)E * 4, tid, kFThreads);
+    if (a.has_shared) prefetch_shared<QT>(SL->shared[l + 1], I, H, first, nthr);
+  }
 
   // ---------------- P3: down projection + weighted combine (+ residual) for 16 output features per CTA.
   // Piece d of a row block shares its slot with piece d - R. Before waiting on piece d's fill a
@@ -659,34 +800,12 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   // P2 item or to an earlier row block, consumed before this row block starts. Units are taken in
   // increasing order, so the lowest waiting piece can always proceed.
   if (ok) {
-    const int nslots = s_slot[nu];
     const int xstride = I + 4;
     const int dn = a.dn_bytes;
     for (int rbl = 0; rbl < n_rb; ++rbl) {
       const int r0 = ((int)blockIdx.x + rbl * G) * 16;
       const int qb = n_mine + rbl * npieces;
       for (int i = tid; i < npieces; i += kFThreads) s_pcnt[i] = 0;
-      {  // stage every present h column (16-byte loads, issued before the stores)
-        const int I8 = I / 8, total = nslots * I8;
-        for (int v0 = tid; v0 < total; v0 += 4 * kFThreads) {
-          uint4 v[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int vi = v0 + j * kFThreads;
-            v[j] = (vi < total) ? __ldcg(reinterpret_cast<const uint4 *>(a.hdec + (size_t)s_src[vi / I8] * I) + vi % I8)
-                                : make_uint4(0, 0, 0, 0);
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int vi = v0 + j * kFThreads;
-            if (vi < total) {
-              uint2 *d = reinterpret_cast<uint2 *>(hs + (size_t)(vi / I8) * xstride + xs_pos(8 * (vi % I8)));
-              d[0] = make_uint2(v[j].x, v[j].y);
-              d[1] = make_uint2(v[j].z, v[j].w);
-            }
-          }
-        }
-      }
       __syncthreads();
       float tot[4] = {0.f, 0.f, 0.f, 0.f};
       // one unit per warp item: its 16 down rows over all of K (the half steps' shared-memory
@@ -704,29 +823,69 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
           }
           __syncwarp();
         }
-        const bool have = wait_bar(full(s), (uint32_t)(qd / R) & 1u, 43);
         const DecUnit &un = su[u];
+        if (rbl == 0) {
+          // the unit's h: wait until all its gate/up items are counted (bounded), then stage its
+          // present columns (16-byte loads from L2); they stay for later row blocks
+          if (lane == 0) {
+            const uint64_t t0 = global_ns();
+            for (;;) {
+              unsigned v;
+              asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a.ready + u) : "memory");
+              if (v >= (unsigned)rbs8 || s_abort) break;
+              __nanosleep(32);
+              if (global_ns() - t0 > kWaitLimitNs) {
+                s_abort = 1;
+                set_device_error(ctrl, MOE_ERR_TIMEOUT, 45);
+                break;
+              }
+            }
+          }
+          __syncwarp();
+          unsigned v;
+          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a.ready + u) : "memory");
+          (void)v;
+          const int I8 = I / 8, c0 = s_slot[u], nc = s_slot[u + 1] - c0;
+          for (int vi = lane; vi < nc * I8; vi += 32) {
+            const uint4 hv = __ldcg(reinterpret_cast<const uint4 *>(a.hdec + (size_t)s_src[c0 + vi / I8] * I) + vi % I8);
+            uint2 *dd = reinterpret_cast<uint2 *>(hs + (size_t)(c0 + vi / I8) * xstride + xs_pos(8 * (vi % I8)));
+            dd[0] = make_uint2(hv.x, hv.y);
+            dd[1] = make_uint2(hv.z, hv.w);
+          }
+          __syncwarp();
+        }
+        const bool have = wait_bar(full(s), fill_parity(qd), 43);
         const bool colok = (un.mask >> g) & 1;
         const int slot = s_slot[u] + __popc(un.mask & ((1u << g) - 1u));
         const __half *xcol = hs + (size_t)(colok ? slot : 0) * xstride;
         float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
         if (have) {
           const uint8_t *pc = ringp + (size_t)s * S + (size_t)(u % a.dpu) * dn;
-          const uint8_t *ca = pc + (size_t)g * (I / 4), *cb = pc + (size_t)(g + 8) * (I / 4);
-          const uint16_t *sa = reinterpret_cast<const uint16_t *>(pc + 4 * I) + (size_t)g * (I / 32);
-          const uint16_t *sb = reinterpret_cast<const uint16_t *>(pc + 4 * I) + (size_t)(g + 8) * (I / 32);
-          const uint8_t *ha = pc + 5 * I + (size_t)g * (I / 8), *hb = pc + 5 * I + (size_t)(g + 8) * (I / 8);
+          const int CD = code_row_bytes(QT, I);
+          const uint8_t *ca = pc + (size_t)g * CD, *cb = pc + (size_t)(g + 8) * CD;
+          const uint16_t *sa = reinterpret_cast<const uint16_t *>(pc + 16 * CD) + (size_t)g * (I / 32);
+          const uint16_t *sb = reinterpret_cast<const uint16_t *>(pc + 16 * CD) + (size_t)(g + 8) * (I / 32);
+          const uint8_t *ha = pc + 16 * CD + I + (size_t)g * (I / 8), *hb = pc + 16 * CD + I + (size_t)(g + 8) * (I / 8);
           for (int h0 = 0; h0 < nhalf_dn; h0 += kDnBatch) {
             HalfFrag f[kDnBatch];
 #pragma unroll
             for (int b = 0; b < kDnBatch; ++b) {
               const int k0 = (h0 + b) * (kStepK / 2) + 32 * t4;
               if (k0 < I) {
-                f[b].w0 = *reinterpret_cast<const uint2 *>(ca + k0 / 4);
-                f[b].w1 = *reinterpret_cast<const uint2 *>(cb + k0 / 4);
+                if (QT == 4) {  // one 16-byte block per row
+                  const uint4 c0 = *reinterpret_cast<const uint4 *>(ca + k0 / 2);
+                  const uint4 c1 = *reinterpret_cast<const uint4 *>(cb + k0 / 2);
+                  f[b].w0 = make_uint2(c0.x, c0.y);
+                  f[b].w0b = make_uint2(c0.z, c0.w);
+                  f[b].w1 = make_uint2(c1.x, c1.y);
+                  f[b].w1b = make_uint2(c1.z, c1.w);
+                } else {
+                  f[b].w0 = *reinterpret_cast<const uint2 *>(ca + k0 / 4);
+                  f[b].w1 = *reinterpret_cast<const uint2 *>(cb + k0 / 4);
+                }
                 f[b].d0 = sa[k0 / 32];
                 f[b].d1 = sb[k0 / 32];
-                if (Q3) {
+                if (QT == 3) {
                   f[b].h0 = *reinterpret_cast<const uint32_t *>(ha + k0 / 8);
                   f[b].h1 = *reinterpret_cast<const uint32_t *>(hb + k0 / 8);
                 }
@@ -735,7 +894,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
 #pragma unroll
             for (int b = 0; b < kDnBatch; ++b) {
               const int k0 = (h0 + b) * (kStepK / 2) + 32 * t4;
-              if (k0 < I) mma_half_step<Q3>(acc, acc2, f[b], xcol, k0, colok);
+              if (k0 < I) mma_half_step<QT>(acc, acc2, f[b], xcol, k0, colok);
             }
           }
         }
@@ -764,7 +923,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       __syncthreads();
       for (int i = tid; i < 16 * T; i += kFThreads) {
         const int row = i % 16, col = i / 16;
-        float sum = a.residual ? a.residual[(size_t)col * H + r0 + row] : 0.0f;
+        float sum = lres ? lres[(size_t)col * H + r0 + row] : 0.0f;
 #pragma unroll
         for (int wi = 0; wi < kFWarps; ++wi) sum += red[(wi * 16 + row) * 8 + col];
         a.y[(size_t)col * H + r0 + row] = sum;
@@ -773,8 +932,28 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
     }
   }
 
+  if (STACK && l + 1 < nl) {
+    // the next layer normalises the whole stream: every CTA's rows of this layer first
+    ok = grid_barrier(ctrl, s_base + (unsigned long long)(2 * l + 2) * nblk, 33, ok) && ok;
+    if (tid < R) s_pbase[tid] += n_total / R + (tid < n_total % R ? 1 : 0);  // every fill was consumed
+    __syncthreads();
+  }
+  }  // layers
+
   // ---------------- no copy may still be writing this CTA's shared memory when it exits
   cp_async_wait_all();
+}
+
+template <int QT, int TMAX>
+__global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedArgs a) {
+  fused_body<QT, TMAX, false>(a, nullptr);
+}
+
+// the same, over the layers of a stack in one launch
+template <int QT, int TMAX>
+__global__ void __launch_bounds__(kFThreads, 1) decode_stack_kernel(const FusedArgs a,
+                                                                   const __grid_constant__ StackLayers SL) {
+  fused_body<QT, TMAX, true>(a, &SL);
 }
 
 // Test hook of the failure path: every CTA arrives at the fused kernel's grid barrier, which is
@@ -810,52 +989,92 @@ cudaError_t launch_barrier_starve(Ctrl *ctrl, int ctas, uint64_t limit_ns, cudaS
   return cudaLaunchKernelEx(&cfg, barrier_starve_kernel, ctrl, limit_ns);
 }
 
-cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float eps, int T, int H, const float *Wr,
-                                const float *bias, int E, int k, int I, const moe_expert_set &routed,
-                                const moe_expert_set *shared, const float *residual, float *y, float *logits,
-                                int32_t *idx, float *w, uint16_t *hdec, Ctrl *ctrl, cudaStream_t s) {
-  const int hs_cols = T * k + (shared ? T : 0);
-  if (T < 1 || T > kDecodeMaxT || E > kFMaxE || H > 2048 || I > 1024 || hs_cols > kFSlots || k > 16)
-    return cudaErrorNotSupported;
-  const bool q3 = routed.gate.qtype == MOE_Q3;
-  const int gu_bytes = (q3 ? 7 : 5) * H;  // 8 gate + 8 up rows: codes, scales (, hi bits)
-  const int dn_bytes = (q3 ? 7 : 5) * I;  // 16 down rows
+// Shapes, ring and shared-memory plan of a fused launch; false when the shape or the device cannot
+// take the kernel.
+static bool fused_plan(int T, int H, int E, int k, int I, const moe_expert_set &routed, bool has_shared, bool stack,
+                       FusedArgs &a, const void *&fn, size_t &smem) {
+  const int hs_cols = T * k + (has_shared ? T : 0);
+  if (T < 1 || T > kDecodeMaxT || E > kFMaxE || H > 2048 || I > 1024 || hs_cols > kFSlots || k > 16) return false;
+  const int qt = routed.gate.qtype;
+  const int per = qt == MOE_Q3 ? 7 : qt == MOE_Q4 ? 9 : 5;  // bytes per 16 weights: codes, scales (, hi bits)
+  const int gu_bytes = per * H;  // 8 gate + 8 up rows
+  const int dn_bytes = per * I;  // 16 down rows
   const int slot_bytes = (int)fl_align((size_t)(gu_bytes > dn_bytes ? gu_bytes : dn_bytes), 128);
   const int dpu = slot_bytes / dn_bytes;
   const FusedLayout L0 = fused_layout(T, H, E, I, hs_cols, 0, slot_bytes);
-  if (L0.total >= (size_t)kFSmemMax) return cudaErrorNotSupported;
+  if (L0.total >= (size_t)kFSmemMax) return false;
   int ring = (int)(((size_t)kFSmemMax - L0.total) / slot_bytes);
   if (ring > kFMaxRing) ring = kFMaxRing;
   {  // no more slots than one CTA can fill: its gate/up items plus its down pieces at the most units
-    const int G = num_sms(), max_units = T * k + (shared ? 1 : 0);
+    const int G = num_sms(), max_units = T * k + (has_shared ? 1 : 0);
     const int need = (max_units * (I / 8) + G - 1) / G + ((H / 16 + G - 1) / G) * ((max_units + dpu - 1) / dpu);
     if (ring > need) ring = need;
   }
   ring &= ~1;  // even: the slots' items fall to one gate/up group each (see the kernel's P2)
-  if (ring < 2) return cudaErrorNotSupported;
+  if (ring < 2) return false;
   const FusedLayout L = fused_layout(T, H, E, I, hs_cols, ring, slot_bytes);
   const int tmax = T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8;
-#define MOE_FUSED_FN(Q, TM) reinterpret_cast<const void *>(decode_fused_kernel<Q, TM>)
-  const void *fn = q3 ? (tmax == 1 ? MOE_FUSED_FN(true, 1) : tmax == 2 ? MOE_FUSED_FN(true, 2)
-                         : tmax == 4 ? MOE_FUSED_FN(true, 4) : MOE_FUSED_FN(true, 8))
-                      : (tmax == 1 ? MOE_FUSED_FN(false, 1) : tmax == 2 ? MOE_FUSED_FN(false, 2)
-                         : tmax == 4 ? MOE_FUSED_FN(false, 4) : MOE_FUSED_FN(false, 8));
+#define MOE_FUSED_FN(K, Q, TM) reinterpret_cast<const void *>(K<Q, TM>)
+#define MOE_FUSED_T(K, Q) (tmax == 1 ? MOE_FUSED_FN(K, Q, 1) : tmax == 2 ? MOE_FUSED_FN(K, Q, 2) \
+                           : tmax == 4 ? MOE_FUSED_FN(K, Q, 4) : MOE_FUSED_FN(K, Q, 8))
+  if (stack)
+    fn = qt == MOE_Q3 ? MOE_FUSED_T(decode_stack_kernel, 3)
+         : qt == MOE_Q4 ? MOE_FUSED_T(decode_stack_kernel, 4) : MOE_FUSED_T(decode_stack_kernel, 2);
+  else
+    fn = qt == MOE_Q3 ? MOE_FUSED_T(decode_fused_kernel, 3)
+         : qt == MOE_Q4 ? MOE_FUSED_T(decode_fused_kernel, 4) : MOE_FUSED_T(decode_fused_kernel, 2);
+#undef MOE_FUSED_T
 #undef MOE_FUSED_FN
-  cudaError_t e = smem_limit_once_impl(fn, kFSmemMax);
-  if (e != cudaSuccess) return e;
+  if (smem_limit_once_impl(fn, kFSmemMax) != cudaSuccess) return false;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kFThreads, L.total) != cudaSuccess || per_sm < 1)
-    return cudaErrorNotSupported;
-  FusedArgs a;
-  a.x = x;
-  a.r_norm = r_norm;
-  a.eps = eps;
+    return false;
+  a = FusedArgs{};
   a.T = T;
   a.H = H;
   a.E = E;
   a.k = k;
   a.I = I;
-  a.has_shared = shared ? 1 : 0;
+  a.has_shared = has_shared ? 1 : 0;
+  a.ring = ring;
+  a.slot_bytes = slot_bytes;
+  a.gu_bytes = gu_bytes;
+  a.dn_bytes = dn_bytes;
+  a.dpu = dpu;
+  smem = L.total;
+  return true;
+}
+
+static cudaError_t fused_launch(const void *fn, size_t smem, void **args, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms());
+  cfg.blockDim = dim3(kFThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  KTimer kt_(KID_DECODE_FUSED, s);
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float eps, int T, int H, const float *Wr,
+                                const float *bias, int E, int k, int I, const moe_expert_set &routed,
+                                const moe_expert_set *shared, const float *residual, float *y, float *logits,
+                                int32_t *idx, float *w, uint16_t *hdec, unsigned *unit_ready, Ctrl *ctrl,
+                                cudaStream_t s) {
+  FusedArgs a;
+  const void *fn = nullptr;
+  size_t smem = 0;
+  if (!fused_plan(T, H, E, k, I, routed, shared != nullptr, false, a, fn, smem)) {
+    (void)cudaGetLastError();
+    return cudaErrorNotSupported;
+  }
+  a.x = x;
+  a.r_norm = r_norm;
+  a.eps = eps;
   a.Wr = Wr;
   a.bias = bias;
   a.routed = routed;
@@ -866,28 +1085,53 @@ cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float ep
   a.idx = idx;
   a.w = w;
   a.hdec = hdec;
+  a.ready = unit_ready;
   a.ctrl = ctrl;
-  a.ring = ring;
-  a.slot_bytes = slot_bytes;
-  a.gu_bytes = gu_bytes;
-  a.dn_bytes = dn_bytes;
-  a.dpu = dpu;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(num_sms());
-  cfg.blockDim = dim3(kFThreads);
-  cfg.dynamicSmemBytes = L.total;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  {
-    KTimer kt_(KID_DECODE_FUSED, s);
-    void *args[] = {&a};
-    e = cudaLaunchKernelExC(&cfg, fn, args);
+  void *args[] = {&a};
+  return fused_launch(fn, smem, args, s);
+}
+
+cudaError_t launch_decode_stack(const float *r_in, float eps, int T, int L, int H, const float *const *Wr,
+                                const float *const *bias, int E, int k, int I, const moe_expert_set *routed,
+                                const moe_expert_set *shared, float *r_out, float *logits, int32_t *idx, float *w,
+                                uint16_t *hdec, unsigned *unit_ready, Ctrl *ctrl, cudaStream_t s) {
+  FusedArgs a;
+  const void *fn = nullptr;
+  size_t smem = 0;
+  if (L < 1 || !fused_plan(T, H, E, k, I, routed[0], shared != nullptr, true, a, fn, smem)) {
+    (void)cudaGetLastError();
+    return cudaErrorNotSupported;
   }
-  return e;
+  for (int l = 1; l < L; ++l)  // one block format for the whole launch
+    if (routed[l].gate.qtype != routed[0].gate.qtype) return cudaErrorNotSupported;
+  a.eps = eps;
+  a.y = r_out;
+  a.logits = logits;
+  a.idx = idx;
+  a.w = w;
+  a.hdec = hdec;
+  a.ready = unit_ready;
+  a.ctrl = ctrl;
+  a.routed = routed[0];
+  a.shared = shared ? shared[0] : routed[0];
+  static thread_local StackLayers sl;  // ~12 KB: kept off the host stack
+  for (int l0 = 0; l0 < L; l0 += kStackMaxL) {
+    const int n = L - l0 < kStackMaxL ? L - l0 : kStackMaxL;
+    sl.n = n;
+    for (int j = 0; j < n; ++j) {
+      sl.Wr[j] = Wr[l0 + j];
+      sl.bias[j] = bias ? bias[l0 + j] : nullptr;
+      sl.routed[j] = routed[l0 + j];
+      sl.shared[j] = shared ? shared[l0 + j] : routed[l0 + j];
+    }
+    // the first layer of a piece reads the stream from r_in (first piece) or r_out (later pieces)
+    a.r_norm = l0 == 0 ? r_in : r_out;
+    a.residual = l0 == 0 ? r_in : r_out;
+    void *args[] = {&a, &sl};
+    cudaError_t e = fused_launch(fn, smem, args, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace moe

@@ -11,6 +11,12 @@
 // gives pairs 4..7 the same way. Subtracting M_p + q0 is exact (small integers), and one fp16
 // multiply by d rounds d(c - q0) once (exact for Q2; Q3 codes 1 and 7 round d*(+-3) to nearest).
 //
+// Q4 (4-bit codes, w = d(c-8)): per block four words, word q (weights 8q..8q+7) holding weight
+// 8q+2i+h (i = 0..3, h = 0..1) at bits 16h+4i. Pairs 0 and 1 sit at bits 0-3 and 4-7 of both
+// halves: masked and OR-ed with M = 1024 (ulp 1) and M = 64 (ulp 2^-4) they give M + c exactly;
+// the word shifted right by 8 gives pairs 2 and 3 the same way. (M + c) - (M + 8) = c - 8 is exact
+// and one fp16 multiply by d rounds d(c - 8) once.
+//
 // Q3: the 1-bit plane holds, per block, one word with bit 2 of weight 16q+2i+h at bit 16h+8q+i.
 // The word pre-shifted so that pair i of half-block q lands on bits i+2 / 18+i, masked and OR-ed
 // with M_h = 2^(10-i) (ulp 2^-i), is (M_h + 4 hi) exactly; (x_lo - (M_p + 4 + M_h)) + x_hi =
@@ -101,6 +107,19 @@ __device__ __forceinline__ void dq3_word(uint32_t w, uint32_t hw, int q, __half2
     const uint32_t tl = (src & (0x00030003u << (2 * p))) | dq_magic(p);
     const uint32_t th = (hs & (0x00010001u << (j + 2))) | dq3_hmag(j);
     const __half2 v = __hadd2_rn(__hsub2_rn(h2bits(tl), h2bits(dq3_sub(j))), h2bits(th));
+    out[j] = bits_h2(__hmul2_rn(v, d2));
+  }
+}
+
+// One Q4 word (8 weights) -> 4 half2 in natural K order (out[j] = weights 2j, 2j+1), times d.
+__device__ __forceinline__ void dq4_word(uint32_t w, __half2 d2, uint32_t out[4]) {
+  const uint32_t w8 = w >> 8;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t src = (j < 2) ? w : w8;
+    const bool hi = j & 1;  // bits 4-7 (magic 64) or 0-3 (magic 1024)
+    const uint32_t t = (src & (hi ? 0x00F000F0u : 0x000F000Fu)) | (hi ? 0x54005400u : 0x64006400u);
+    const __half2 v = __hsub2_rn(h2bits(t), h2bits(hi ? 0x54805480u : 0x64086408u));  // M + 8
     out[j] = bits_h2(__hmul2_rn(v, d2));
   }
 }

@@ -47,7 +47,6 @@ struct GemmArgs {
   int K;                           // reduction dim (H for gate/up, I for down)
   int M;                           // weight rows per expert (I for gate/up, H for down)
   int shared_group;                // group index served by the shared expert, -1 if none
-  int q3;
   const uint16_t *scales[2][2];    // [set][mat]
   const uint8_t *hibits[2][2];     // [set][mat]
 };
@@ -82,17 +81,24 @@ constexpr int kStagesA = 2;
 constexpr int kThreadsV2 = 448;
 constexpr int kEpiWarp0 = 10;
 
+// bytes of the code plane per weight row for K weights: 2-bit plane K/4, 4-bit plane (Q4) K/2
+__host__ __device__ constexpr int gemm_code_bytes(int qt, int K) { return qt == 4 ? K / 2 : K / 4; }
+
+template <int QT>
 struct SmemV2 {
   static constexpr int kSub = kBNMax * kSubK * 2;  // 24 KB: one 64-wide sub-tile of the activation rows
   static constexpr int kB = 2 * kSub;              // 48 KB activation tile (K = 128)
-  static constexpr int kRaw = kBM * kBK / 4;       // 4 KB packed codes
+  static constexpr int kRowCodes = gemm_code_bytes(QT, kBK);  // code bytes of one weight row per stage
+  static constexpr int kRaw = kBM * kRowCodes;     // 4 KB packed codes (8 KB for the 4-bit plane)
   static constexpr int kStage = kB + kRaw;         // multiple of 1024 (128B-swizzle atoms)
   static constexpr int kBar = kStagesB * kStage;
   static constexpr int kNumBars = 2 * kStagesB + kStagesA + 4;
   static constexpr int kBytes = kBar + kNumBars * 8 + 16;
 };
 
-static_assert(SmemV2::kStage % 1024 == 0 && SmemV2::kSub % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+static_assert(SmemV2<2>::kStage % 1024 == 0 && SmemV2<4>::kStage % 1024 == 0 && SmemV2<2>::kSub % 1024 == 0,
+              "stages keep the 1024-byte swizzle alignment");
+static_assert(SmemV2<4>::kBytes + 1024 <= 232448, "the 4-bit plane's stages fit the shared-memory limit");
 static_assert(kStagesA == 2, "TMEM holds two A stages");
 
 // TMEM column of A stage s (64 columns: 128 K of fp16 pairs)
@@ -128,12 +134,12 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t r[16]) {
       : "memory");
 }
 
-template <int MODE>
+template <int MODE, int QT>
 __global__ void __launch_bounds__(kThreadsV2, 1)
 grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c0r,
                   const __grid_constant__ CUtensorMap tm_c1r, const __grid_constant__ CUtensorMap tm_c0s,
                   const __grid_constant__ CUtensorMap tm_c1s, const GemmArgs args) {
-  using SL = SmemV2;
+  using SL = SmemV2<QT>;
   extern __shared__ uint8_t smem_raw[];
   Ctrl *ctrl = args.ctrl;
   const int n_mtiles = (MODE == MODE_GU) ? args.M / 64 : args.M / kBM;
@@ -202,10 +208,10 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
               tma_load_2d(sB(s) + h * SL::kSub + b * kBoxRows * kSubK * 2, &tm_b, ks * kBK + h * kSubK,
                           cur.row_base + b * kBoxRows, full_b(s));
           if (MODE == MODE_GU) {  // gate rows -> A rows 0..63, up rows -> A rows 64..127
-            tma_load_2d(sR(s), mc0, ks * (kBK / 4), wrow, full_b(s));
-            tma_load_2d(sR(s) + 64 * (kBK / 4), mc1, ks * (kBK / 4), wrow, full_b(s));
+            tma_load_2d(sR(s), mc0, ks * SL::kRowCodes, wrow, full_b(s));
+            tma_load_2d(sR(s) + 64 * SL::kRowCodes, mc1, ks * SL::kRowCodes, wrow, full_b(s));
           } else {
-            tma_load_2d(sR(s), mc0, ks * (kBK / 4), wrow, full_b(s));
+            tma_load_2d(sR(s), mc0, ks * SL::kRowCodes, wrow, full_b(s));
           }
         }
         cur = nxt;
@@ -289,7 +295,7 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
       const uint8_t *hb = set ? (mat ? args.hibits[1][1] : args.hibits[1][0])
                               : (mat ? args.hibits[0][1] : args.hibits[0][0]);
       sp = reinterpret_cast<const uint32_t *>(sc + grow * (K / 32)) + hh;
-      hp = args.q3 ? reinterpret_cast<const uint2 *>(hb + grow * (K / 8)) + hh : nullptr;
+      hp = QT == 3 ? reinterpret_cast<const uint2 *>(hb + grow * (K / 8)) + hh : nullptr;
     };
     // scales (and Q3 hi words) are fetched four stages ahead into a 4-entry register ring
     int pf_tl = 0;
@@ -300,7 +306,7 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
       const int tl = g / nk;
       if (tl != pf_tl) { pf_tl = tl; row_ptrs(tl, pf_sp, pf_hp); }
       scv = __ldg(pf_sp + 2 * (g % nk));
-      if (args.q3) hv = __ldg(pf_hp + 2 * (g % nk));
+      if (QT == 3) hv = __ldg(pf_hp + 2 * (g % nk));
     };
     uint32_t sc[4];
     uint2 hw[4];
@@ -318,20 +324,26 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
         if (g >= total_g) break;
         const int s = g % kStagesB, sa = g % kStagesA;
         const uint32_t ph = (uint32_t)(g / kStagesB) & 1u;
-        // codes landed; and the MMAs that last read this A stage (stage g - kStagesA) are complete
+        // codes landed: dequantize into registers first, so that the arithmetic is off the chain
+        // MMA(g - kStagesA) done -> A stage written -> MMA(g)
         if (!mbar_wait(full_b(s), ph)) { record_timeout(ctrl, 24); ok = false; break; }
-        if (g >= kStagesA &&
-            !mbar_wait(empty_b((g - kStagesA) % kStagesB), (uint32_t)((g - kStagesA) / kStagesB) & 1u)) {
-          record_timeout(ctrl, 24);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint4 cw = *reinterpret_cast<const uint4 *>(gbase + (sR(s) - base) + crow * (kBK / 4) + hh * 16);
+        // this thread's 64 weights of the stage: 16 code bytes (32 for the 4-bit plane)
+        const uint8_t *cp = gbase + (sR(s) - base) + crow * SL::kRowCodes + hh * (SL::kRowCodes / 2);
+        const uint4 cw = *reinterpret_cast<const uint4 *>(cp);
         const __half2 d0 = __half2half2(__ushort_as_half((uint16_t)(sc[j] & 0xffffu)));
         const __half2 d1 = __half2half2(__ushort_as_half((uint16_t)(sc[j] >> 16)));
         uint32_t p[32];
-        if (args.q3) {
+        if (QT == 4) {  // eight 8-weight words, words 0-3 in block 0 and 4-7 in block 1
+          const uint4 cw2 = *reinterpret_cast<const uint4 *>(cp + 16);
+          dq4_word(cw.x, d0, p);
+          dq4_word(cw.y, d0, p + 4);
+          dq4_word(cw.z, d0, p + 8);
+          dq4_word(cw.w, d0, p + 12);
+          dq4_word(cw2.x, d1, p + 16);
+          dq4_word(cw2.y, d1, p + 20);
+          dq4_word(cw2.z, d1, p + 24);
+          dq4_word(cw2.w, d1, p + 28);
+        } else if (QT == 3) {
           dq3_word(cw.x, hw[j].x, 0, d0, p);
           dq3_word(cw.y, hw[j].x, 1, d0, p + 8);
           dq3_word(cw.z, hw[j].y, 0, d1, p + 16);
@@ -342,6 +354,14 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
           dq2_word(cw.z, d1, p + 16);
           dq2_word(cw.w, d1, p + 24);
         }
+        // the MMAs that last read this A stage (stage g - kStagesA) are complete
+        if (g >= kStagesA &&
+            !mbar_wait(empty_b((g - kStagesA) % kStagesB), (uint32_t)((g - kStagesA) / kStagesB) & 1u)) {
+          record_timeout(ctrl, 24);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         const uint32_t ta = tmem + a_lane + a_col(sa) + 32u * hh;
         tmem_st16(ta, p);
         tmem_st16(ta + 16u, p + 16);
@@ -419,14 +439,25 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
 }
 
 // ---------------------------------------------------------------- tile list
-// entries (group, first row within the group) for every kBNMax-row (192-row) slice of every non-empty group
-// (offsets that are not monotone or run past n_rows flag the error word and yield no tiles)
+// Entries (group, first row within the group) for every kBNMax-row (192-row) slice of every
+// non-empty group, ordered longest first: by the slice's row count rounded up to the MMA's N
+// granule of 16, descending (full 192-row slices first, the smallest remainders last). The
+// persistent GEMM deals entries round-robin, so every CTA starts on the heavy tiles and the light
+// ones fill the end of the schedule: with a skewed router a few experts take >1000 rows and many
+// take a handful, and the long tiles no longer land at the tail. Within a size class the order
+// is whatever the shared-memory cursors give; it does not change any result (every tile writes
+// its own output rows). Offsets that are not monotone or run past n_rows flag the error word and
+// yield no tiles. Groups of at most min_rows rows get no tiles (the caller runs them elsewhere).
+constexpr int kTileClasses = kBNMax / 16;  // N granules 1..12
+
 __global__ void __launch_bounds__(1024) tile_list_kernel(const int32_t *__restrict__ off, int G, int n_rows,
-                                                         int2 *__restrict__ tiles, Ctrl *__restrict__ ctrl) {
-  __shared__ int s_warp[32];
+                                                         int min_rows, int2 *__restrict__ tiles,
+                                                         Ctrl *__restrict__ ctrl) {
+  __shared__ int s_cnt[kTileClasses + 1], s_cur[kTileClasses + 1];
   __shared__ int s_bad;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   if (tid == 0) s_bad = 0;
+  if (tid <= kTileClasses) s_cnt[tid] = 0;
   __syncthreads();
   for (int g = tid; g < G; g += blockDim.x)
     if (off[g] < 0 || off[g + 1] < off[g] || off[g + 1] > n_rows) s_bad = 1;
@@ -438,40 +469,33 @@ __global__ void __launch_bounds__(1024) tile_list_kernel(const int32_t *__restri
     }
     return;
   }
-  const int per = (G + 1023) / 1024;  // <= 5
-  int cnt[5];
-  int mine = 0;
-  for (int i = 0; i < per; ++i) {
-    const int g = tid * per + i;
-    int c = 0;
-    if (g < G) c = (off[g + 1] - off[g] + kBNMax - 1) / kBNMax;
-    cnt[i] = c;
-    mine += c;
+  // size class of a slice with n rows (1..192): ceil(n / 16), 1..kTileClasses
+  for (int g = tid; g < G; g += blockDim.x) {
+    const int n = off[g + 1] - off[g];
+    if (n <= min_rows) continue;  // left to the small-group path
+    if (n >= kBNMax) atomicAdd(&s_cnt[kTileClasses], n / kBNMax);
+    if (n % kBNMax) atomicAdd(&s_cnt[(n % kBNMax + 15) / 16], 1);
   }
-  int v = mine;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int n = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += n;
-  }
-  if (lane == 31) s_warp[warp] = v;
   __syncthreads();
-  if (warp == 0) {
-    int wv = s_warp[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int n = __shfl_up_sync(0xffffffffu, wv, o);
-      if (lane >= o) wv += n;
+  if (tid == 0) {  // classes in descending order: each class's first position
+    int pos = 0;
+    for (int c = kTileClasses; c >= 1; --c) {
+      s_cur[c] = pos;
+      pos += s_cnt[c];
     }
-    s_warp[lane] = wv;
+    ctrl->n_tiles = pos;
   }
   __syncthreads();
-  int pos = v - mine + (warp > 0 ? s_warp[warp - 1] : 0);
-  for (int i = 0; i < per; ++i) {
-    const int g = tid * per + i;
-    for (int j = 0; j < cnt[i]; ++j) tiles[pos++] = make_int2(g, j * kBNMax);
+  for (int g = tid; g < G; g += blockDim.x) {
+    const int n = off[g + 1] - off[g];
+    if (n <= min_rows) continue;
+    const int full = n / kBNMax;
+    if (full) {
+      const int p = atomicAdd(&s_cur[kTileClasses], full);
+      for (int j = 0; j < full; ++j) tiles[p + j] = make_int2(g, j * kBNMax);
+    }
+    if (n % kBNMax) tiles[atomicAdd(&s_cur[(n % kBNMax + 15) / 16], 1)] = make_int2(g, full * kBNMax);
   }
-  if (tid == 1023) ctrl->n_tiles = pos;
 }
 
 // ---------------------------------------------------------------- host side
@@ -481,21 +505,30 @@ namespace {
 namespace {
 
 bool make_code_map(CUtensorMap *map, const moe_qmat &m, int box_rows) {
-  return encode_tensor_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, m.codes, (uint64_t)m.K / 4,
-                              (uint64_t)m.n_experts * m.rows, kBK / 4, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
+  return encode_tensor_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, m.codes, (uint64_t)gemm_code_bytes(m.qtype, m.K),
+                              (uint64_t)m.n_experts * m.rows, gemm_code_bytes(m.qtype, kBK), box_rows,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+template <int MODE, int QT>
+cudaError_t launch_v2q(const CUtensorMap &tb, const CUtensorMap &c0r, const CUtensorMap &c1r, const CUtensorMap &c0s,
+                       const CUtensorMap &c1s, const GemmArgs &a, cudaStream_t s) {
+  const int smem = SmemV2<QT>::kBytes + 1024;
+  cudaError_t e = smem_limit_once(grouped_v2_kernel<MODE, QT>, smem);
+  if (e != cudaSuccess) return e;
+  {
+    KTimer kt_(MODE == MODE_GU ? KID_GEMM_GATE_UP : KID_GEMM_DOWN, s);
+    grouped_v2_kernel<MODE, QT><<<num_sms(), kThreadsV2, smem, s>>>(tb, c0r, c1r, c0s, c1s, a);
+  }
+  return cudaGetLastError();
 }
 
 template <int MODE>
 cudaError_t launch_v2(const CUtensorMap &tb, const CUtensorMap &c0r, const CUtensorMap &c1r, const CUtensorMap &c0s,
-                      const CUtensorMap &c1s, const GemmArgs &a, cudaStream_t s) {
-  const int smem = SmemV2::kBytes + 1024;
-  cudaError_t e = smem_limit_once(grouped_v2_kernel<MODE>, smem);
-  if (e != cudaSuccess) return e;
-  {
-    KTimer kt_(MODE == MODE_GU ? KID_GEMM_GATE_UP : KID_GEMM_DOWN, s);
-    grouped_v2_kernel<MODE><<<num_sms(), kThreadsV2, smem, s>>>(tb, c0r, c1r, c0s, c1s, a);
-  }
-  return cudaGetLastError();
+                      const CUtensorMap &c1s, const GemmArgs &a, int qt, cudaStream_t s) {
+  if (qt == MOE_Q3) return launch_v2q<MODE, 3>(tb, c0r, c1r, c0s, c1s, a, s);
+  if (qt == MOE_Q4) return launch_v2q<MODE, 4>(tb, c0r, c1r, c0s, c1s, a, s);
+  return launch_v2q<MODE, 2>(tb, c0r, c1r, c0s, c1s, a, s);
 }
 
 }  // namespace
@@ -529,12 +562,12 @@ int gemm_shape_supported(int H, int I) { return (H % 128 == 0 && I % 128 == 0 &&
 
 cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, int n_rows, int E, int H, int I,
                                const moe_expert_set &routed, const moe_expert_set *shared, uint16_t *h_perm,
-                               uint16_t *out_perm, int2 *tiles, Ctrl *ctrl, cudaStream_t s) {
+                               uint16_t *out_perm, int2 *tiles, Ctrl *ctrl, cudaStream_t s, int min_rows) {
   const int G = E + (shared ? 1 : 0);
   const moe_expert_set &sh = shared ? *shared : routed;
   {
     KTimer kt_(KID_TILE_LIST, s);
-    tile_list_kernel<<<1, 1024, 0, s>>>(offsets, G, n_rows, tiles, ctrl);
+    tile_list_kernel<<<1, 1024, 0, s>>>(offsets, G, n_rows, min_rows, tiles, ctrl);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -554,7 +587,6 @@ cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, i
   a.tiles = tiles;
   a.ctrl = ctrl;
   a.shared_group = shared ? E : -1;
-  a.q3 = routed.gate.qtype == MOE_Q3 ? 1 : 0;
   // kernel 1: gate/up + SwiGLU -> h_perm
   a.out = h_perm;
   a.ldo = I;
@@ -568,7 +600,7 @@ cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, i
   a.hibits[0][1] = routed.up.hibits;
   a.hibits[1][0] = sh.gate.hibits;
   a.hibits[1][1] = sh.up.hibits;
-  e = launch_v2<MODE_GU>(tx, cg, cu, sg, su, a, s);
+  e = launch_v2<MODE_GU>(tx, cg, cu, sg, su, a, routed.gate.qtype, s);
   if (e != cudaSuccess) return e;
   // kernel 2: down -> out_perm
   a.out = out_perm;
@@ -583,7 +615,7 @@ cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, i
   a.hibits[0][1] = nullptr;
   a.hibits[1][0] = sh.down.hibits;
   a.hibits[1][1] = nullptr;
-  return launch_v2<MODE_DN>(th, cd, cd, sd, sd, a, s);
+  return launch_v2<MODE_DN>(th, cd, cd, sd, sd, a, routed.gate.qtype, s);
 }
 
 }  // namespace moe

@@ -1,7 +1,8 @@
 // Dequant-GEMV building blocks for 1-8 activation columns (decode / MTP verify): a warp owns 16
 // weight rows; lane (g, t) holds rows g and g+8 and a 64-weight slice of each 256-wide K step
-// (one 16-byte code load per row per step); each 16-weight word is dequantized to fp16 pairs and
-// fed to mma.sync m16n8k16 with the activation columns as the 8 MMA columns (fp32 accumulate).
+// (one 16-byte code load per row per step for the 2-bit plane, two for the 4-bit plane); each
+// code word is dequantized to fp16 pairs and fed to mma.sync m16n8k16 with the activation
+// columns as the 8 MMA columns (fp32 accumulate). QT is the block format: 2 (Q2), 3 (Q3), 4 (Q4).
 // Activations are staged in shared memory as fp16 with a per-64-chunk rotation so the fragment
 // loads of the four K slices hit distinct banks.
 #pragma once
@@ -12,6 +13,9 @@
 namespace moe {
 
 constexpr int kStepK = 256;       // K covered by one warp step (4 lanes x 64 weights)
+
+// bytes of the code plane per weight row of K weights: 2-bit plane K/4, 4-bit plane K/2
+__host__ __device__ constexpr int code_row_bytes(int qt, int K) { return qt == 4 ? K / 2 : K / 4; }
 
 __device__ __forceinline__ void mma16816(float c[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -26,6 +30,11 @@ __device__ __forceinline__ void mma16816(float c[4], const uint32_t a[4], uint32
 __device__ __forceinline__ int xs_pos(int k) {
   const int ch = k >> 6, q = k & 63;
   return (ch << 6) + ((q + 16 * (ch & 3)) & 63);
+}
+
+// word i (0..3) of a 16-byte fragment, by selects (no local-memory indexing)
+__device__ __forceinline__ uint32_t sel4(const uint4 &v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
 struct MatView {
@@ -45,11 +54,11 @@ __device__ __forceinline__ MatView mat_sel(const moe_expert_set &r, const moe_ex
   const uint8_t *codes = MOE_SEL(codes);
   const uint8_t *hib = MOE_SEL(hibits);
   const uint16_t *sc = MOE_SEL(scales);
-  const int rows = MOE_SEL(rows), K = MOE_SEL(K);
+  const int rows = MOE_SEL(rows), K = MOE_SEL(K), qt = MOE_SEL(qtype);
 #undef MOE_SEL
   MatView v;
   const size_t row0 = (size_t)expert * rows;
-  v.codes = codes + row0 * (K / 4);
+  v.codes = codes + row0 * code_row_bytes(qt, K);
   v.hibits = hib ? hib + row0 * (K / 8) : nullptr;
   v.scales = sc + row0 * (K / 32);
   v.K = K;
@@ -59,33 +68,41 @@ __device__ __forceinline__ MatView mat_sel(const moe_expert_set &r, const moe_ex
 __device__ __forceinline__ MatView mat_of(const moe_qmat &m, int expert) {
   MatView v;
   const size_t row0 = (size_t)expert * m.rows;
-  v.codes = m.codes + row0 * (m.K / 4);
+  v.codes = m.codes + row0 * code_row_bytes(m.qtype, m.K);
   v.hibits = m.hibits ? m.hibits + row0 * (m.K / 8) : nullptr;
   v.scales = m.scales + row0 * (m.K / 32);
   v.K = m.K;
   return v;
 }
 
-// one lane's share of a 16-row x 256-wide K step: 16 code bytes of rows g and g+8, their two
-// block scales, and (Q3) the two blocks' hi-bit words
+// one lane's share of a 16-row x 256-wide K step: the code bytes of rows g and g+8 (16 each for the
+// 2-bit plane; 32 for the 4-bit plane, the second 16 in w0b / w1b), their two block scales, and
+// (Q3) the two blocks' hi-bit words
 struct StepFrag {
   uint4 w0, w1;
+  uint4 w0b, w1b;
   uint32_t d0, d1;
   uint2 h0, h1;
 };
 
-template <bool Q3>
+template <int QT>
 __device__ __forceinline__ void load_step(StepFrag &f, const MatView &m, int r0, int step, bool valid) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int k0 = step * kStepK + 64 * t;
   const bool ok = valid && k0 < m.K;
-  const size_t rs = (size_t)m.K / 4, ss = (size_t)m.K / 32, hs = (size_t)m.K / 8;
+  const size_t rs = (size_t)code_row_bytes(QT, m.K), ss = (size_t)m.K / 32, hs = (size_t)m.K / 8;
+  const size_t co = (size_t)code_row_bytes(QT, k0);
   const size_t ra = (size_t)(r0 + g), rb = (size_t)(r0 + g + 8);
-  f.w0 = ok ? __ldcs(reinterpret_cast<const uint4 *>(m.codes + ra * rs + k0 / 4)) : make_uint4(0, 0, 0, 0);
-  f.w1 = ok ? __ldcs(reinterpret_cast<const uint4 *>(m.codes + rb * rs + k0 / 4)) : make_uint4(0, 0, 0, 0);
+  const uint4 z4 = make_uint4(0, 0, 0, 0);
+  f.w0 = ok ? __ldcs(reinterpret_cast<const uint4 *>(m.codes + ra * rs + co)) : z4;
+  f.w1 = ok ? __ldcs(reinterpret_cast<const uint4 *>(m.codes + rb * rs + co)) : z4;
+  if (QT == 4) {
+    f.w0b = ok ? __ldcs(reinterpret_cast<const uint4 *>(m.codes + ra * rs + co) + 1) : z4;
+    f.w1b = ok ? __ldcs(reinterpret_cast<const uint4 *>(m.codes + rb * rs + co) + 1) : z4;
+  }
   f.d0 = ok ? __ldcs(reinterpret_cast<const uint32_t *>(m.scales + ra * ss + k0 / 32)) : 0u;
   f.d1 = ok ? __ldcs(reinterpret_cast<const uint32_t *>(m.scales + rb * ss + k0 / 32)) : 0u;
-  if (Q3) {
+  if (QT == 3) {
     f.h0 = ok ? __ldcs(reinterpret_cast<const uint2 *>(m.hibits + ra * hs + k0 / 8)) : make_uint2(0, 0);
     f.h1 = ok ? __ldcs(reinterpret_cast<const uint2 *>(m.hibits + rb * hs + k0 / 8)) : make_uint2(0, 0);
   }
@@ -93,107 +110,155 @@ __device__ __forceinline__ void load_step(StepFrag &f, const MatView &m, int r0,
 
 // dequantize the fragment (zero codes with zero scales give zero weights) and run the step's 16
 // MMAs; B fragments come from the lane's column in shared memory when `bok`, else zero
-template <bool Q3>
+template <int QT>
 __device__ __forceinline__ void mma_step(float acc[4], float acc2[4], const StepFrag &f, const __half *xcol, int kbase,
                                          bool bok) {
-  const uint32_t wr0[4] = {f.w0.x, f.w0.y, f.w0.z, f.w0.w};
-  const uint32_t wr1[4] = {f.w1.x, f.w1.y, f.w1.z, f.w1.w};
+  if constexpr (QT == 4) {  // eight 8-weight words per row: word wq in block wq/4, two MMAs per word
 #pragma unroll
-  for (int wq = 0; wq < 4; ++wq) {  // word wq: block wq/2, half q = wq%2
-    const int blk = wq >> 1, q = wq & 1;
-    const __half2 dd0 = __half2half2(__ushort_as_half((uint16_t)(f.d0 >> (16 * blk))));
-    const __half2 dd1 = __half2half2(__ushort_as_half((uint16_t)(f.d1 >> (16 * blk))));
-    uint32_t p0[8], p1[8];
-    if (Q3) {
-      dq3_word(wr0[wq], blk ? f.h0.y : f.h0.x, q, dd0, p0);
-      dq3_word(wr1[wq], blk ? f.h1.y : f.h1.x, q, dd1, p1);
-    } else {
-      dq2_word(wr0[wq], dd0, p0);
-      dq2_word(wr1[wq], dd1, p1);
-    }
+    for (int wq = 0; wq < 8; ++wq) {
+      const int blk = wq >> 2;
+      const uint32_t w0 = blk ? sel4(f.w0b, wq & 3) : sel4(f.w0, wq & 3);
+      const uint32_t w1 = blk ? sel4(f.w1b, wq & 3) : sel4(f.w1, wq & 3);
+      const __half2 dd0 = __half2half2(__ushort_as_half((uint16_t)(f.d0 >> (16 * blk))));
+      const __half2 dd1 = __half2half2(__ushort_as_half((uint16_t)(f.d1 >> (16 * blk))));
+      uint32_t p0[4], p1[4];
+      dq4_word(w0, dd0, p0);
+      dq4_word(w1, dd1, p1);
 #pragma unroll
-    for (int mm = 0; mm < 4; ++mm) {  // MMA 4*wq + mm uses pairs 2mm, 2mm+1 of this word
-      const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
-      uint32_t b0 = 0, b1 = 0;
-      if (bok) {
-        const uint2 bv = *reinterpret_cast<const uint2 *>(xcol + xs_pos(kbase + 16 * wq + 4 * mm));
-        b0 = bv.x;
-        b1 = bv.y;
+      for (int mm = 0; mm < 2; ++mm) {
+        const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
+        uint32_t b0 = 0, b1 = 0;
+        if (bok) {
+          const uint2 bv = *reinterpret_cast<const uint2 *>(xcol + xs_pos(kbase + 8 * wq + 4 * mm));
+          b0 = bv.x;
+          b1 = bv.y;
+        }
+        mma16816(mm ? acc2 : acc, a, b0, b1);
       }
-      mma16816((mm & 1) ? acc2 : acc, a, b0, b1);
+    }
+  } else {
+#pragma unroll
+    for (int wq = 0; wq < 4; ++wq) {  // word wq: block wq/2, half q = wq%2
+      const int blk = wq >> 1, q = wq & 1;
+      const uint32_t w0 = sel4(f.w0, wq), w1 = sel4(f.w1, wq);
+      const __half2 dd0 = __half2half2(__ushort_as_half((uint16_t)(f.d0 >> (16 * blk))));
+      const __half2 dd1 = __half2half2(__ushort_as_half((uint16_t)(f.d1 >> (16 * blk))));
+      uint32_t p0[8], p1[8];
+      if (QT == 3) {
+        dq3_word(w0, blk ? f.h0.y : f.h0.x, q, dd0, p0);
+        dq3_word(w1, blk ? f.h1.y : f.h1.x, q, dd1, p1);
+      } else {
+        dq2_word(w0, dd0, p0);
+        dq2_word(w1, dd1, p1);
+      }
+#pragma unroll
+      for (int mm = 0; mm < 4; ++mm) {  // MMA 4*wq + mm uses pairs 2mm, 2mm+1 of this word
+        const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
+        uint32_t b0 = 0, b1 = 0;
+        if (bok) {
+          const uint2 bv = *reinterpret_cast<const uint2 *>(xcol + xs_pos(kbase + 16 * wq + 4 * mm));
+          b0 = bv.x;
+          b1 = bv.y;
+        }
+        mma16816((mm & 1) ? acc2 : acc, a, b0, b1);
+      }
     }
   }
 }
 
 // Half of a step: a 16-row x 128-wide K slice, lane (g, t) holding the 32-weight block
-// kbase..kbase+31 (kbase = slice start + 32 t) of rows g and g+8: two code words per row, one
-// scale per row, and (Q3) one hi word per row. Same pair decoder and MMA-K order as mma_step.
+// kbase..kbase+31 (kbase = slice start + 32 t) of rows g and g+8: two code words per row (four
+// for the 4-bit plane, the last two in w0b / w1b), one scale per row, and (Q3) one hi word per
+// row. Same pair decoder and MMA-K order as mma_step.
 struct HalfFrag {
   uint2 w0, w1;
+  uint2 w0b, w1b;
   uint16_t d0, d1;
   uint32_t h0, h1;
 };
 
-template <bool Q3>
+template <int QT>
 __device__ __forceinline__ void mma_half_step(float acc[4], float acc2[4], const HalfFrag &f, const __half *xcol,
                                               int kbase, bool bok) {
-  const uint32_t wr0[2] = {f.w0.x, f.w0.y};
-  const uint32_t wr1[2] = {f.w1.x, f.w1.y};
-  const __half2 dd0 = __half2half2(__ushort_as_half(f.d0));
-  const __half2 dd1 = __half2half2(__ushort_as_half(f.d1));
+  if constexpr (QT == 4) {
+    const __half2 dd0 = __half2half2(__ushort_as_half(f.d0));
+    const __half2 dd1 = __half2half2(__ushort_as_half(f.d1));
 #pragma unroll
-  for (int wq = 0; wq < 2; ++wq) {
-    uint32_t p0[8], p1[8];
-    if (Q3) {
-      dq3_word(wr0[wq], f.h0, wq, dd0, p0);
-      dq3_word(wr1[wq], f.h1, wq, dd1, p1);
-    } else {
-      dq2_word(wr0[wq], dd0, p0);
-      dq2_word(wr1[wq], dd1, p1);
-    }
+    for (int wq = 0; wq < 4; ++wq) {
+      const uint2 a0 = (wq >> 1) ? f.w0b : f.w0, a1 = (wq >> 1) ? f.w1b : f.w1;
+      uint32_t p0[4], p1[4];
+      dq4_word((wq & 1) ? a0.y : a0.x, dd0, p0);
+      dq4_word((wq & 1) ? a1.y : a1.x, dd1, p1);
 #pragma unroll
-    for (int mm = 0; mm < 4; ++mm) {
-      const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
-      uint32_t b0 = 0, b1 = 0;
-      if (bok) {
-        const uint2 bv = *reinterpret_cast<const uint2 *>(xcol + xs_pos(kbase + 16 * wq + 4 * mm));
-        b0 = bv.x;
-        b1 = bv.y;
+      for (int mm = 0; mm < 2; ++mm) {
+        const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
+        uint32_t b0 = 0, b1 = 0;
+        if (bok) {
+          const uint2 bv = *reinterpret_cast<const uint2 *>(xcol + xs_pos(kbase + 8 * wq + 4 * mm));
+          b0 = bv.x;
+          b1 = bv.y;
+        }
+        mma16816(mm ? acc2 : acc, a, b0, b1);
       }
-      mma16816((mm & 1) ? acc2 : acc, a, b0, b1);
+    }
+  } else {
+    const __half2 dd0 = __half2half2(__ushort_as_half(f.d0));
+    const __half2 dd1 = __half2half2(__ushort_as_half(f.d1));
+#pragma unroll
+    for (int wq = 0; wq < 2; ++wq) {
+      const uint32_t w0 = wq ? f.w0.y : f.w0.x, w1 = wq ? f.w1.y : f.w1.x;
+      uint32_t p0[8], p1[8];
+      if (QT == 3) {
+        dq3_word(w0, f.h0, wq, dd0, p0);
+        dq3_word(w1, f.h1, wq, dd1, p1);
+      } else {
+        dq2_word(w0, dd0, p0);
+        dq2_word(w1, dd1, p1);
+      }
+#pragma unroll
+      for (int mm = 0; mm < 4; ++mm) {
+        const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
+        uint32_t b0 = 0, b1 = 0;
+        if (bok) {
+          const uint2 bv = *reinterpret_cast<const uint2 *>(xcol + xs_pos(kbase + 16 * wq + 4 * mm));
+          b0 = bv.x;
+          b1 = bv.y;
+        }
+        mma16816((mm & 1) ? acc2 : acc, a, b0, b1);
+      }
     }
   }
 }
 
 // acc += W[r0..r0+15, steps s0..s0+NS-1] * X^T; all of the batch's loads are issued first
-template <bool Q3, int NS>
+template <int QT, int NS>
 __device__ __forceinline__ void rows16_batch(const MatView &m, int r0, int s0, int nsteps, const __half *xcol,
                                              bool colok, float acc[4]) {
   const int t = threadIdx.x & 3;
   StepFrag f[NS];
 #pragma unroll
-  for (int s = 0; s < NS; ++s) load_step<Q3>(f[s], m, r0, s0 + s, s0 + s < nsteps);
+  for (int s = 0; s < NS; ++s) load_step<QT>(f[s], m, r0, s0 + s, s0 + s < nsteps);
   float acc2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int s = 0; s < NS; ++s) {
     const int kbase = (s0 + s) * kStepK + 64 * t;
-    mma_step<Q3>(acc, acc2, f[s], xcol, kbase, colok && (s0 + s < nsteps) && kbase < m.K);
+    mma_step<QT>(acc, acc2, f[s], xcol, kbase, colok && (s0 + s < nsteps) && kbase < m.K);
   }
 #pragma unroll
   for (int e = 0; e < 4; ++e) acc[e] += acc2[e];
 }
 
 // full K of 16 rows: batches of 8 steps, then a tail batch of 4, 2 or 1
-template <bool Q3>
+template <int QT>
 __device__ __forceinline__ void rows16(const MatView &m, int r0, const __half *xcol, bool colok, float acc[4]) {
   const int nsteps = (m.K + kStepK - 1) / kStepK;
   int s = 0;
-  for (; s + 8 <= nsteps; s += 8) rows16_batch<Q3, 8>(m, r0, s, nsteps, xcol, colok, acc);
+  for (; s + 8 <= nsteps; s += 8) rows16_batch<QT, 8>(m, r0, s, nsteps, xcol, colok, acc);
   const int rem = nsteps - s;
-  if (rem > 4) rows16_batch<Q3, 8>(m, r0, s, nsteps, xcol, colok, acc);
-  else if (rem > 2) rows16_batch<Q3, 4>(m, r0, s, nsteps, xcol, colok, acc);
-  else if (rem == 2) rows16_batch<Q3, 2>(m, r0, s, nsteps, xcol, colok, acc);
-  else if (rem == 1) rows16_batch<Q3, 1>(m, r0, s, nsteps, xcol, colok, acc);
+  if (rem > 4) rows16_batch<QT, 8>(m, r0, s, nsteps, xcol, colok, acc);
+  else if (rem > 2) rows16_batch<QT, 4>(m, r0, s, nsteps, xcol, colok, acc);
+  else if (rem == 2) rows16_batch<QT, 2>(m, r0, s, nsteps, xcol, colok, acc);
+  else if (rem == 1) rows16_batch<QT, 1>(m, r0, s, nsteps, xcol, colok, acc);
 }
 
 // stage columns of the activation source into shared memory (fp16, rotated layout). 16-byte

@@ -457,35 +457,45 @@ cudaError_t launch_rmsnorm(const float *r, int T, int H, float eps, uint16_t *u,
 // ---------------------------------------------------------------- dequant test hook
 // thread per (row, 16-weight word); fp16 output through the same pair decoder the GEMM uses
 __global__ void dequant_rows_kernel(moe_qmat m, int expert, int row0, int nrows, float *out_f32, uint16_t *out_f16) {
-  const int words = m.K / 16;
+  // one code word per thread: 16 weights of the 2-bit plane, 8 of the 4-bit plane
+  const bool q4 = m.qtype == MOE_Q4;
+  const int per = q4 ? 8 : 16;
+  const int words = m.K / per;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= nrows * words) return;
   const int r = i / words, wq = i % words;
   const size_t row = (size_t)expert * m.rows + row0 + r;
-  const int blk = wq >> 1, q = wq & 1;
-  const uint32_t w = reinterpret_cast<const uint32_t *>(m.codes + row * (m.K / 4))[wq];
+  const int blk = wq / (32 / per), q = wq % (32 / per);
+  const uint32_t w = reinterpret_cast<const uint32_t *>(m.codes + row * (q4 ? m.K / 2 : m.K / 4))[wq];
   const uint16_t dbits = m.scales[row * (m.K / 32) + blk];
   const __half d = __ushort_as_half(dbits);
   uint32_t pairs[8];
   if (m.qtype == MOE_Q2) {
     dq2_word(w, __half2half2(d), pairs);
+  } else if (q4) {
+    dq4_word(w, __half2half2(d), pairs);
   } else {
     const uint32_t hw = reinterpret_cast<const uint32_t *>(m.hibits + row * (m.K / 8))[blk];
     dq3_word(w, hw, q, __half2half2(d), pairs);
   }
   const float df = __half2float(d);
-  const int q0 = (m.qtype == MOE_Q2) ? 2 : 4;
-  for (int j = 0; j < 16; ++j) {
-    const int kk = wq * 16 + j;
+  const int q0 = (m.qtype == MOE_Q2) ? 2 : q4 ? 8 : 4;
+  for (int j = 0; j < per; ++j) {
+    const int kk = wq * per + j;
     const uint16_t hb = (uint16_t)((pairs[j >> 1] >> (16 * (j & 1))) & 0xffffu);
     if (out_f16) out_f16[(size_t)r * m.K + kk] = hb;
     if (out_f32) {
       // integer code recovered from the packed planes (independent of the fp16 path)
-      const int jj = j, ii = jj >> 1, h = jj & 1;
-      int c = (int)((w >> (16 * h + 2 * ii)) & 3u);
-      if (m.qtype == MOE_Q3) {
-        const uint32_t hw = reinterpret_cast<const uint32_t *>(m.hibits + row * (m.K / 8))[blk];
-        c |= (int)((hw >> (16 * h + 8 * q + ii)) & 1u) << 2;
+      const int ii = j >> 1, h = j & 1;
+      int c;
+      if (q4) {
+        c = (int)((w >> (16 * h + 4 * ii)) & 15u);
+      } else {
+        c = (int)((w >> (16 * h + 2 * ii)) & 3u);
+        if (m.qtype == MOE_Q3) {
+          const uint32_t hw = reinterpret_cast<const uint32_t *>(m.hibits + row * (m.K / 8))[blk];
+          c |= (int)((hw >> (16 * h + 8 * q + ii)) & 1u) << 2;
+        }
       }
       out_f32[(size_t)r * m.K + kk] = df * (float)(c - q0);
     }
@@ -494,7 +504,7 @@ __global__ void dequant_rows_kernel(moe_qmat m, int expert, int row0, int nrows,
 
 cudaError_t launch_dequant_rows(const moe_qmat &m, int expert, int row0, int nrows, float *out_f32, uint16_t *out_f16,
                                 cudaStream_t s) {
-  const int n = nrows * (m.K / 16);
+  const int n = nrows * (m.K / (m.qtype == MOE_Q4 ? 8 : 16));
   {
     KTimer kt_(KID_DEQUANT_ROWS, s);
     dequant_rows_kernel<<<(n + 255) / 256, 256, 0, s>>>(m, expert, row0, nrows, out_f32, out_f16);

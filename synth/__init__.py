@@ -262,6 +262,8 @@ WORKLOADS = {
     "prefill8k": LayerShape("prefill8k", 8192, 2048, 512, 10, 512, Q2, True, None),
     # prefill with 3-bit weights and Zipf(1.2) skew, no shared expert
     "prefill2k_q3": LayerShape("prefill2k_q3", 2048, 2048, 512, 10, 512, Q3, False, 1.2),
+    # the decode layer with 4-bit weights (the Q4 stand-in), otherwise decode1
+    "decode1_q4": LayerShape("decode1_q4", 1, 2048, 512, 10, 512, Q4, True, 1.1),
 }
 
 # 48-layer stack: RMSNorm (eps 1e-6) before each router, residual add, config-3 shaped layers

@@ -88,6 +88,8 @@ def test_layer_forward_validation(lib):
     assert _lf(lib, routed=_set(codes=FAKE_MIS.value)) == moe.MOE_ERR_ALIGNMENT
     assert _lf(lib, routed=_set(qtype=3)) == moe.MOE_ERR_INVALID_ARG       # Q3 without the hi-bit plane
     assert _lf(lib, routed=_set(qtype=5)) == moe.MOE_ERR_INVALID_ARG
+    assert _lf(lib, routed=_set(qtype=2, hib=FAKE.value)) == moe.MOE_ERR_INVALID_ARG  # hi bits belong to Q3 only
+    assert _lf(lib, routed=_set(qtype=4, hib=FAKE.value)) == moe.MOE_ERR_INVALID_ARG
     assert _lf(lib, routed=_set(E=511)) == moe.MOE_ERR_INVALID_ARG         # set shape disagrees with desc
     assert _lf(lib, ws=None) == moe.MOE_ERR_WORKSPACE
     assert _lf(lib, wsb=1024) == moe.MOE_ERR_WORKSPACE

@@ -19,6 +19,7 @@ pytestmark = pytest.mark.gpu
 
 MID = synth.LayerShape("mid", 300, 512, 32, 4, 256, synth.Q2, True, 1.1, seed=3)
 MID_Q3 = synth.LayerShape("mid_q3", 200, 512, 32, 4, 256, synth.Q3, False, 1.2, seed=4)
+MID_Q4 = synth.LayerShape("mid_q4", 300, 512, 32, 4, 256, synth.Q4, True, 1.1, seed=5)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -32,7 +33,7 @@ _cache = {}
 
 def layer_of(name):
     if name not in _cache:
-        shape = {"mid": MID, "mid_q3": MID_Q3}.get(name) or synth.WORKLOADS[name]
+        shape = {"mid": MID, "mid_q3": MID_Q3, "mid_q4": MID_Q4}.get(name) or synth.WORKLOADS[name]
         L = synth.make_layer(shape)
         _cache[name] = (L, to_dev(L))
     return _cache[name]
@@ -52,7 +53,7 @@ def test_generator_device_bits_match_cpu():
 
 
 # ----------------------------------------------------------------------------- dequant
-@pytest.mark.parametrize("qtype", [synth.Q2, synth.Q3])
+@pytest.mark.parametrize("qtype", [synth.Q2, synth.Q3, synth.Q4])
 def test_dequant_rows_bit_exact(qtype):
     qm = synth.make_qmat(7, 0, 0, 0, qtype, 4, 96, 512)
     dm = qm.to("cuda")
@@ -156,9 +157,10 @@ def test_combine_matches_definition():
 
 
 # ----------------------------------------------------------------------------- expert FFN (both paths)
-@pytest.mark.parametrize("name", ["tiny", "mid", "mid_q3"])
-@pytest.mark.parametrize("path", [moe.PATH_GEMV, moe.PATH_GEMM])
+@pytest.mark.parametrize("name", ["tiny", "mid", "mid_q3", "mid_q4"])
+@pytest.mark.parametrize("path", [moe.PATH_GEMV, moe.PATH_GEMM, moe.PATH_AUTO])
 def test_expert_ffn_rows(name, path):
+    # AUTO splits the groups: those of at most 32 rows on the GEMV kernels, the rest on the GEMM
     L, (x, Wr, b, routed, shared) = layer_of(name)
     s = L.shape
     idx_ref, _, _, _ = oracle.router_topk(L.x, L.Wr, L.bias, s.k)
@@ -184,8 +186,8 @@ def test_expert_ffn_rows(name, path):
 
 # ----------------------------------------------------------------------------- layer forward
 @pytest.mark.parametrize("name,ntok", [("tiny", 64), ("decode1", 1), ("decode4", 4), ("verify6", 6),
-                                       ("decode1_pruned256", 1), ("mid", 300),
-                                       ("mid_q3", 200), ("prefill8k", 24), ("prefill2k_q3", 24)])
+                                       ("decode1_pruned256", 1), ("decode1_q4", 1), ("mid", 300),
+                                       ("mid_q3", 200), ("mid_q4", 300), ("prefill8k", 24), ("prefill2k_q3", 64)])
 def test_layer_forward(name, ntok):
     L, (x, Wr, b, routed, shared) = layer_of(name)
     s = L.shape
@@ -193,6 +195,11 @@ def test_layer_forward(name, ntok):
     y, idx, w = moe.layer_forward(x, Wr, b, routed, shared, s.k, ws, want_routing=True)
     assert moe.read_device_error(ws) == 0
     tokens = np.arange(s.T) if ntok >= s.T else np.sort(np.random.default_rng(5).choice(s.T, ntok, replace=False))
+    if ntok < s.T:  # and tokens routed to the most popular expert (its rows fill several full tiles)
+        flat = idx.cpu().numpy()
+        top = np.bincount(flat.reshape(-1), minlength=s.E).argmax()
+        heavy = np.nonzero((flat == top).any(axis=1))[0]
+        tokens = np.union1d(tokens, heavy[np.linspace(0, len(heavy) - 1, 8).astype(int)])
     err, flips = check_layer(y.cpu().numpy(), idx.cpu().numpy(), L, tokens, w_gpu=w.cpu().numpy())
     print(f"{name}: max|dy|/rms = {err:.3e}, near-tie flips {len(flips)}")
 
@@ -210,7 +217,7 @@ def test_layer_forward_with_residual_in_place():
                 w_gpu=w.cpu().numpy())
 
 
-@pytest.mark.parametrize("name,T", [("mid", 64), ("mid", 4), ("mid_q3", 4), ("tiny", 4)])
+@pytest.mark.parametrize("name,T", [("mid", 64), ("mid", 4), ("mid_q3", 4), ("tiny", 4), ("mid_q4", 64)])
 def test_cross_path_gemv_vs_gemm(name, T):
     L, (x, Wr, b, routed, shared) = layer_of(name)
     s = L.shape
@@ -221,7 +228,8 @@ def test_cross_path_gemv_vs_gemm(name, T):
 
 
 @pytest.mark.parametrize("name,T", [("mid", 5), ("mid", 8), ("decode4", 5), ("decode4", 6), ("decode4", 8),
-                                    ("prefill8k", 4), ("prefill8k", 5), ("decode4", 12), ("prefill2k_q3", 100)])
+                                    ("prefill8k", 4), ("prefill8k", 5), ("decode4", 12), ("prefill2k_q3", 100),
+                                    ("decode1_q4", 4), ("decode1_q4", 8), ("mid_q4", 5)])
 def test_layer_forward_decode_batches(name, T):
     # 5-8 tokens take the decode path under AUTO: the fused kernel where its shared-memory plan
     # fits (top-4 layer; top-10 at T=5), the separate decode kernels beyond (top-10 at T=6, 8).

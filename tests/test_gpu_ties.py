@@ -111,3 +111,21 @@ def test_layer_routing_exact_ties_lower_index_wins(T, path, masked):
     _, idx, w = moe.layer_forward(x.cuda(), Wr_d, b_d, routed, shared, K, ws, path=path, want_routing=True)
     assert moe.read_device_error(ws) == 0
     _check(idx, w, idx_ref, w_ref)
+
+
+@pytest.mark.parametrize("T", [1, 4, 12, 300])
+def test_all_logits_equal_take_the_lowest_indices(T):
+    # a zero router makes every logit 0: each token must take experts 0..k-1 in that order with
+    # equal weights 1/k (more tied candidates than one warp holds: the paths' fallbacks run)
+    _, _, _, _, _, routed, shared = _setup(False)
+    Wr0 = torch.zeros(E, H, dtype=torch.float32, device="cuda")
+    x = _tokens(T, np.zeros(0, np.int64), stream=200 + T)
+    idx_ref, w_ref, _, gap = oracle.router_topk(x, Wr0.cpu(), None, K)
+    assert (gap == 0).all() and (idx_ref == np.arange(K)).all()
+    ws = moe.Workspace.for_layer(H, E, K, I, True, T)
+    idx, w = moe.router_topk(x.cuda(), Wr0, None, K, ws)
+    _check(idx, w, idx_ref, w_ref)
+    if T <= 4:  # the fused decode kernel's own top-k
+        _, idx, w = moe.layer_forward(x.cuda(), Wr0, None, routed, shared, K, ws, want_routing=True)
+        _check(idx, w, idx_ref, w_ref)
+    assert moe.read_device_error(ws) == 0

@@ -8,9 +8,9 @@ one fewer and the wait mistakes the older phase for its own; two more and it nev
 
 The schedule modelled here is the kernel's: fills 0..R-1 are issued at the start, fill q + R
 when fill q has been consumed; gate/up items alternate between two warp groups, each taking its
-items in order, with an even R; after the grid barrier the down phase's warps take whole units
-(warp w: units w, w + 16, ...), a unit of piece d first waiting until piece d - R is fully
-consumed. The test drives that schedule with fills landing and consumers advancing in random
+items in order, with an even R; after the CTA barrier that closes the gate/up phase the down
+phase's warps take whole units (warp w: units w, w + 16, ...), a unit of piece d first waiting
+until piece d - R is fully consumed. The test drives that schedule with fills landing and consumers advancing in random
 order and checks the wait rule at every wait, and that the schedule never deadlocks. Variants
 with the rules the kernel relies on removed (an odd R, no wait for the piece one ring behind,
 items dealt to every warp) must break the rule, so the check is known to see the failure it

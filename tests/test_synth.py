@@ -67,4 +67,6 @@ def test_workload_table_matches_the_stated_configs():
     assert (p.T, p.H, p.E, p.k, p.I, p.qtype, p.shared, p.zipf_s) == (8192, 2048, 512, 10, 512, synth.Q2, True, None)
     q = W["prefill2k_q3"]
     assert (q.T, q.E, q.k, q.qtype, q.shared, q.zipf_s) == (2048, 512, 10, synth.Q3, False, 1.2)
+    q4 = W["decode1_q4"]
+    assert (q4.T, q4.H, q4.E, q4.k, q4.I, q4.qtype, q4.shared, q4.zipf_s) == (1, 2048, 512, 10, 512, synth.Q4, True, 1.1)
     assert synth.STACK["L"] == 48 and synth.STACK["eps"] == 1e-6
