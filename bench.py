@@ -269,8 +269,10 @@ def run_ours(args, world, rank, local, workload=None, steps=None, warmup=None, l
         xs = [synth.make_x(shape.seed, T, H, stream=replica_x_stream(rank, i)).to(dev) for i in range(n_x)]
         handles = [moe.LayerHandle(Wr, b, rs, ss, k, ws) for (Wr, b, rs, ss) in layers]
 
+        path = {"auto": moe.PATH_AUTO, "gemm": moe.PATH_GEMM, "gemv": moe.PATH_GEMV, "mmq": moe.PATH_MMQ}[args.path]
+
         def step(i, x=None, idx_out=None):
-            handles[i % n_layers].forward(xs[i % n_x] if x is None else x, y, idx_out=idx_out)
+            handles[i % n_layers].forward(xs[i % n_x] if x is None else x, y, idx_out=idx_out, path=path)
 
     for i in range(W):
         step(i)
@@ -388,7 +390,7 @@ def run_ours(args, world, rank, local, workload=None, steps=None, warmup=None, l
                       "note": "all bytes of a layer step (active experts + fp32 router + x + y) / step time"}
     else:
         rows = T * k + (T if shape.shared else 0)
-        dom = "gemm_gate_up"
+        dom = "mmq_gate_up" if "mmq_gate_up" in kt else "gemm_gate_up"
         d_ms, d_n = kt[dom]
         flops = 2.0 * 2 * rows * H * I
         achieved = flops / (d_ms / d_n / 1e3) / 1e12
@@ -396,11 +398,15 @@ def run_ours(args, world, rank, local, workload=None, steps=None, warmup=None, l
         sm, smax = (clk or {}).get("sm_mhz"), (clk or {}).get("sm_max_mhz")
         capped = bool(sm and smax and sm < 0.95 * smax)
         peak_tc = pk["tc_sus"] if capped else pk["tc"]
+        int8 = dom == "mmq_gate_up"
+        if int8:  # int8 contraction: the bf16 figure times the nominal int8 / bf16 ratio (4.5 / 2.25 PF)
+            peak_tc *= 2.0
         roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak_tc,
                 "unit": "TFLOP/s", "frac": round(achieved / peak_tc, 4), "traffic": traffic_for(dom, workload),
                 "peak_source": pk["src"] + (" sustained" if capped else " burst") +
-                " bf16 (fp16 MMA runs at the bf16 rate; SM clock %s of %s MHz under load)" % (sm, smax),
-                "frac_of_other_peak": round(achieved / (pk["tc"] if capped else pk["tc_sus"]), 4),
+                (" bf16 x 2 (int8 MMA, nominal ratio)" if int8 else
+                 " bf16 (fp16 MMA runs at the bf16 rate)") + "; SM clock %s of %s MHz under load" % (sm, smax),
+                "frac_of_other_peak": round(achieved / ((pk["tc"] if capped else pk["tc_sus"]) * (2.0 if int8 else 1.0)), 4),
                 "algorithmic_flops_per_launch": flops, "avg_launch_us": round(d_ms / d_n * 1e3, 1)}
         layer_flops = 2.0 * 3 * rows * H * I + 2.0 * T * E * H
         tf = layer_flops / (ms_max / K / lps / 1e3) / 1e12
@@ -442,7 +448,7 @@ def run_ours(args, world, rank, local, workload=None, steps=None, warmup=None, l
                                f"T={T}, H={H}, E={E}, top-{k}, I={I}, "
                                f"Q{shape.qtype}, shared={int(shape.shared)}, "
                                f"router bias={'Zipf(%s)' % shape.zipf_s if shape.zipf_s else 'none'}",
-                   "T": T, "layers_rotated": n_layers, "graph_steps": G,
+                   "T": T, "layers_rotated": n_layers, "graph_steps": G, "expert_path": args.path,
                    "l2": "inputs larger than L2: steps rotate over %d layer weight sets (%.1f GB)" % (
                        n_layers, n_layers * (layers[0][2].nbytes + (layers[0][3].nbytes if layers[0][3] else 0)
                                              + E * H * 4) / 1e9),
@@ -580,6 +586,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="distinct layer weight sets to rotate over (default 48 for decode, 4 for prefill)")
+    ap.add_argument("--path", default="auto", choices=["auto", "gemm", "gemv", "mmq"],
+                    help="expert path of the layer workloads (mmq: int8 activations on tcgen05 kind::i8 for gate/up)")
     ap.add_argument("--no-breakdown", action="store_true",
                     help="time only --workload (by default a single-GPU run of the T=1 decode layer also times "
                          "the T=4 verify layer and the T=8192 prefill layer, reported under 'breakdown')")

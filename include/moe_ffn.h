@@ -39,8 +39,8 @@
  *   - T = 0 is a no-op that returns MOE_OK.
  *   - Device tensors must be 16-byte aligned (MOE_ERR_ALIGNMENT otherwise).
  *   - Faults the device detects (an expert index >= E handed to moe_permute, a bounded wait
- *     that timed out) are recorded in the workspace's error word and the offending element is
- *     skipped; read and clear the word with moe_read_device_error.
+ *     that timed out, a value outside the fp16 operand range) are recorded in the workspace's
+ *     error word; read and clear the word with moe_read_device_error.
  *
  * Packed weight planes (moe_qmat)
  *   One matrix kind (gate, up or down) of n_experts experts: `rows` output features, reduction
@@ -63,7 +63,10 @@
  *   the fp32 logits; equal logits: the lower expert index wins; slots are stored in descending
  *   logit order. Expert contractions: fp16 operands (Q2 weights are exact in fp16, bf16 x is
  *   exact in fp16 in its normal range), fp32 accumulation; intermediate h and per-expert
- *   outputs are stored as fp16; y, the residual stream and the combine are fp32.
+ *   outputs are stored as fp16; y, the residual stream and the combine are fp32. A value that
+ *   does not fit fp16 (|x| > 65504, or an h or expert output that overflows) is not rescaled:
+ *   it becomes +-inf and moe_layer_forward / moe_stack_forward / moe_permute record
+ *   MOE_ERR_RANGE in the workspace error word.
  */
 #ifndef MOE_FFN_H
 #define MOE_FFN_H
@@ -84,13 +87,20 @@ enum {
   MOE_ERR_UNSUPPORTED = 4,   /* valid request the library cannot run (e.g. forced GEMM path, H % 128 != 0) */
   MOE_ERR_CUDA = 5,          /* a CUDA runtime/driver call failed (launch error, no device) */
   MOE_ERR_DEVICE_CHECK = 6,  /* reported by moe_read_device_error: a device-side index check failed */
-  MOE_ERR_TIMEOUT = 7        /* reported by moe_read_device_error: a bounded device wait gave up */
+  MOE_ERR_TIMEOUT = 7,       /* reported by moe_read_device_error: a bounded device wait gave up */
+  MOE_ERR_RANGE = 8          /* reported by moe_read_device_error: a value left the fp16 range of the
+                                expert operands (an input x above 65504 in magnitude, or an
+                                intermediate h or expert output that overflowed); it became +-inf */
 };
 
 enum { MOE_Q2 = 2, MOE_Q3 = 3, MOE_Q4 = 4 };
 
-/* expert-FFN path selection */
-enum { MOE_PATH_AUTO = 0, MOE_PATH_GEMV = 1, MOE_PATH_GEMM = 2 };
+/* expert-FFN path selection. MOE_PATH_MMQ: int8 activations (one scale per 32-value block) and
+ * the Q2 weights' integer codes on tcgen05 kind::i8 for gate/up (exact integer block sums, both
+ * block scales applied on the read-back), then the fp16 down GEMM; Q2 weights, H % 256 == 0,
+ * I % 128 == 0 (MOE_ERR_UNSUPPORTED otherwise). The int8 activations change the numerics (the
+ * oracle's fp64 definition is met within the usual 1e-2 only because the rounding is per block). */
+enum { MOE_PATH_AUTO = 0, MOE_PATH_GEMV = 1, MOE_PATH_GEMM = 2, MOE_PATH_MMQ = 3 };
 
 typedef struct moe_qmat {
   int32_t qtype;            /* MOE_Q2, MOE_Q3 or MOE_Q4 (all matrices of a layer share one) */
@@ -171,10 +181,9 @@ moe_status moe_permute(const int32_t *idx, int32_t T, int32_t k, int32_t E, cons
  *   out_perm[r,:] = fp16( W_down[g] ( silu(W_gate[g] x_perm[r]) * (W_up[g] x_perm[r]) ) )
  * Groups 0..E-1 use `routed`; with shared_opt != NULL, group E (rows offsets[E]..offsets[E+1])
  * uses the shared expert. offsets (device) has E+1 (+1) monotone entries with
- * offsets[last] <= n_rows. path: MOE_PATH_GEMM = tcgen05 grouped GEMM for every group (needs
- * H % 128 == 0 and I % 128 == 0), MOE_PATH_GEMV = dequant-GEMV for every group, MOE_PATH_AUTO:
- * where the GEMM shape rule holds, groups of at most 32 rows on the dequant-GEMV (weights
- * streamed once per 8 rows) and the larger groups on the grouped GEMM; the GEMV otherwise.
+ * offsets[last] <= n_rows. path: MOE_PATH_GEMM = tcgen05 grouped GEMM (needs H % 128 == 0 and
+ * I % 128 == 0), MOE_PATH_GEMV = dequant-GEMV, MOE_PATH_AUTO picks the GEMM when n_rows > 64
+ * and the GEMM shape rule holds, the GEMV otherwise.
  * x_perm fp16 [n_rows,H]; out_perm fp16 [n_rows,H]. */
 moe_status moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, int32_t n_rows, int32_t E, int32_t H,
                           int32_t I, const moe_expert_set *routed, const moe_expert_set *shared_opt,
@@ -198,9 +207,8 @@ moe_status moe_combine(const uint16_t *out_perm, const int32_t *row_of, const fl
  * projection fused with the weighted combine; under AUTO one cooperative kernel does the whole
  * layer where its shared-memory plan fits). Otherwise: router + top-k (fp32 dot products on the
  * CUDA cores up to 128 tokens, tensor-core logits with an exact refine of the candidates above),
- * permute, the expert FFN (GEMM: tcgen05 grouped GEMM gate/up with fused SwiGLU, then down;
- * GEMV: the decode GEMV kernels over 8-row chunks of each expert's rows; AUTO: experts with at
- * most 32 rows on the GEMV kernels, the others on the grouped GEMM), combine. Every
+ * permute, the expert FFN (AUTO / GEMM: tcgen05 grouped GEMM gate/up with fused SwiGLU, then
+ * down; GEMV: the decode GEMV kernels over 8-row chunks of each expert's rows), combine. Every
  * path computes the same function within the parity tolerance.
  *   y = sum_j w_j FFN_{idx_j}(x) + FFN_shared(x) (+ residual)      fp32 [T,H]
  * x bf16 [T,H]; Wr fp32 [E,H]; bias fp32 [E] or NULL; routed: gate/up [E][I][H], down [E][H][I];
@@ -260,7 +268,8 @@ int32_t moe_kernel_count(void);
 const char *moe_kernel_name(int32_t kernel);
 
 /* Synchronise `stream`, read the workspace's device error word into *code (MOE_OK,
- * MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT) and clear it. */
+ * MOE_ERR_DEVICE_CHECK, MOE_ERR_TIMEOUT or MOE_ERR_RANGE; the first error recorded wins) and
+ * clear it. */
 moe_status moe_read_device_error(void *ws, int32_t *code, void *stream);
 
 /* Test hook for the failure path of the device-side waits. Launches two CTAs that arrive at the

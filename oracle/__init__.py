@@ -193,6 +193,37 @@ def permute(idx, E: int):
     return counts, offsets, row_of, src
 
 
+# ----------------------------------------------------------------------------- int8 activations
+def quantize_blocks_i8(x):
+    """int8 quantization of fp16 activation rows in 32-value blocks, the MMQ-style input format
+    ("Two-Day Port, 8x Faster Prefill: Strata Engine Benchmarked", "Where Strata Is Fast": MMQ;
+    "Strata vs Llama.cpp vs vLLM": int8 tensor-core kernels). Per row and block:
+      amax = max |x|,  d = amax / 127,  q = clamp(rint(x * (127 / amax)), -127, 127)  (q = 0, d = 0 for
+      an all-zero block),
+    every step in fp32 (the precision the GPU decides the integers in), ties to even.
+    x: fp16 bits or values [R, H] (H % 32 == 0). Returns (q int8 [R, H], d fp32 [R, H/32])."""
+    xf = np.asarray(x)
+    if xf.dtype == np.uint16:
+        xf = xf.view(np.float16)
+    xf = xf.astype(np.float32)
+    R, H = xf.shape
+    blocks = xf.reshape(R, H // 32, 32)
+    amax = np.abs(blocks).max(axis=-1).astype(np.float32)
+    d = (amax / np.float32(127.0)).astype(np.float32)
+    with np.errstate(divide="ignore"):
+        inv = np.where(amax > 0, np.float32(127.0) / amax, np.float32(0.0)).astype(np.float32)
+    prod = (blocks * inv[..., None]).astype(np.float32)
+    q = np.clip(np.rint(prod), -127, 127).astype(np.int8)
+    return q.reshape(R, H), d
+
+
+def dequantize_blocks_i8(q, d) -> np.ndarray:
+    """The fp64 values q * d the int8 blocks stand for."""
+    q = np.asarray(q, np.int64)
+    R, H = q.shape
+    return (q.reshape(R, H // 32, 32) * np.asarray(d, np.float64)[..., None]).reshape(R, H)
+
+
 # ----------------------------------------------------------------------------- FFN / layer
 def expert_ffn_rows(es, e: int, x: np.ndarray, mirrored: bool = False) -> np.ndarray:
     """One expert (gate/up/down of set `es`) applied to fp64 rows x[n,H]."""

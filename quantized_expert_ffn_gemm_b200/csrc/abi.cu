@@ -34,7 +34,8 @@ cudaEvent_t take_event() {
 const char *const kKernelNames[KID_COUNT] = {
     "router_decode", "router_gemm", "topk", "perm_hist", "perm_scan", "perm_scatter", "perm_fill",
     "perm_gather", "combine", "rmsnorm", "dequant_rows", "dec_units", "dec_gate_up", "dec_down",
-    "tile_list", "gemm_gate_up", "gemm_down", "router_split", "router_tc", "decode_fused"};
+    "tile_list", "gemm_gate_up", "gemm_down", "router_split", "router_tc", "decode_fused", "mmq_quant",
+    "mmq_gate_up"};
 }  // namespace
 
 void timer_begin(int kid, cudaStream_t s) {
@@ -137,20 +138,28 @@ T *at(void *ws, size_t off) {
   return reinterpret_cast<T *>(static_cast<unsigned char *>(ws) + off);
 }
 
-// Groups of at most this many rows take the dequant-GEMV kernels under AUTO (weights streamed
-// once per 8 rows, rows as MMA columns); larger groups take the tcgen05 grouped GEMM, whose tiles
-// cost about the same whatever their row count up to ~96 rows (measured), so a small group there
-// wastes most of a tile.
-constexpr int kSmallGroupRows = 32;
+// Groups of at most this many rows would take the dequant-GEMV kernels under AUTO and the larger
+// ones the tcgen05 grouped GEMM. A GEMM tile costs about the same whatever its row count up to
+// ~96 rows (measured), so small groups waste most of a tile there; but the GEMV kernels measured
+// slower still on the small groups of a skewed 2048-token layer (0.53 against 0.39 ms for the
+// layer) and at 12-128 tokens, so the split is off (0) and AUTO runs every group on the GEMM.
+constexpr int kSmallGroupRows = 0;
 
 // Expert FFN over expert-contiguous rows by path: GEMM (every group on the grouped GEMM), GEMV
 // (every group on the GEMV kernels), AUTO with the GEMM available: small groups on the GEMV
 // kernels and the rest on the grouped GEMM (disjoint rows of out_perm).
 cudaError_t expert_rows(const uint16_t *xperm, const int32_t *offsets, int rows, int E, int H, int I,
                         const moe_expert_set &routed, const moe_expert_set *sh, uint16_t *hperm, uint16_t *operm,
-                        int2 *tiles, DecUnit *units, uint16_t *hdec, Ctrl *ctrl, cudaStream_t s, int path, bool gemm_ok) {
+                        int2 *tiles, DecUnit *units, uint16_t *hdec, Ctrl *ctrl, cudaStream_t s, int path, bool gemm_ok,
+                        int8_t *xq = nullptr, float *dx = nullptr) {
   const int n_groups = E + (sh ? 1 : 0);
-  const bool hybrid = path == MOE_PATH_AUTO && gemm_ok;
+  if (path == MOE_PATH_MMQ) {  // int8-activation gate/up, then the fp16 down GEMM
+    cudaError_t e = launch_mmq_gate_up(xperm, offsets, rows, E, H, I, routed, sh, xq, dx, hperm, tiles, ctrl, s);
+    if (e == cudaSuccess) e = launch_grouped_down(hperm, offsets, rows, E, H, I, routed, sh, operm, tiles, ctrl, s);
+    return e;
+  }
+  const bool hybrid = path == MOE_PATH_AUTO && gemm_ok && kSmallGroupRows > 0;
+  if (path == MOE_PATH_AUTO && gemm_ok && !hybrid) path = MOE_PATH_GEMM;
   cudaError_t e = cudaSuccess;
   if (path == MOE_PATH_GEMM || hybrid) {
     e = launch_grouped_ffn(xperm, offsets, rows, E, H, I, routed, sh, hperm, operm, tiles, ctrl, s,
@@ -185,6 +194,7 @@ const char *moe_status_string(moe_status s) {
     case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
     case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK";
     case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_RANGE: return "MOE_ERR_RANGE";
     default: return "MOE_ERR_UNKNOWN";
   }
 }
@@ -258,7 +268,7 @@ moe_status moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, int32_
                           uint16_t *out_perm, int32_t path, void *ws, size_t ws_bytes, void *stream) {
   moe_status st = shape_status(H, E, 1, I);
   if (st != MOE_OK) return st;
-  if (n_rows < 0 || path < 0 || path > 2) return MOE_ERR_INVALID_ARG;
+  if (n_rows < 0 || path < 0 || path > 3) return MOE_ERR_INVALID_ARG;
   if ((st = check_set(routed, E, H, I)) != MOE_OK) return st;
   if (shared_opt && (st = check_set(shared_opt, 1, H, I)) != MOE_OK) return st;
   if (n_rows == 0) return MOE_OK;
@@ -271,10 +281,15 @@ moe_status moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, int32_
   if (!aligned16(ws)) return MOE_ERR_ALIGNMENT;
   const bool gemm_ok = gemm_shape_supported(H, I) != 0;
   if (path == MOE_PATH_GEMM && !gemm_ok) return MOE_ERR_UNSUPPORTED;
+  if (path == MOE_PATH_MMQ && !(gemm_ok && mmq_shape_supported(H, I, routed->gate.qtype))) return MOE_ERR_UNSUPPORTED;
   Ctrl *ctrl = at<Ctrl>(ws, L.ctrl);
+  // AUTO: the grouped GEMM above 64 rows where its shape rule holds, the GEMV otherwise
+  const int p = (path == MOE_PATH_AUTO && !(gemm_ok && n_rows > 64)) ? MOE_PATH_GEMV : path;
+  // the int8 rows go to the workspace's (unused here) permuted-activation region
   return cuda_status(expert_rows(x_perm, offsets, n_rows, E, H, I, *routed, shared_opt, at<uint16_t>(ws, L.hperm),
                                  out_perm, at<int2>(ws, L.tiles), at<DecUnit>(ws, L.units),
-                                 at<uint16_t>(ws, L.hdec), ctrl, (cudaStream_t)stream, path, gemm_ok));
+                                 at<uint16_t>(ws, L.hdec), ctrl, (cudaStream_t)stream, p, gemm_ok,
+                                 at<int8_t>(ws, L.xperm), at<float>(ws, L.dx)));
 }
 
 moe_status moe_combine(const uint16_t *out_perm, const int32_t *row_of, const float *w, int32_t T, int32_t k,
@@ -298,7 +313,7 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
   const int H = desc->H, E = desc->E, k = desc->k, I = desc->I, hs = desc->has_shared ? 1 : 0;
   moe_status st = shape_status(H, E, k, I);
   if (st != MOE_OK) return st;
-  if (T < 0 || path < 0 || path > 2) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || path < 0 || path > 3) return MOE_ERR_INVALID_ARG;
   if ((st = check_set(routed, E, H, I)) != MOE_OK) return st;
   if (hs && (st = check_set(shared_opt, 1, H, I)) != MOE_OK) return st;
   if (T == 0) return MOE_OK;
@@ -313,6 +328,7 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
   if (!aligned16(ws)) return MOE_ERR_ALIGNMENT;
   const bool gemm_ok = gemm_shape_supported(H, I) != 0;
   if (path == MOE_PATH_GEMM && !gemm_ok) return MOE_ERR_UNSUPPORTED;
+  if (path == MOE_PATH_MMQ && !(gemm_ok && mmq_shape_supported(H, I, routed->gate.qtype))) return MOE_ERR_UNSUPPORTED;
 
   cudaStream_t s = (cudaStream_t)stream;
   Ctrl *ctrl = at<Ctrl>(ws, L.ctrl);
@@ -325,7 +341,7 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
   // decode path (distinct experts' weights read once, tokens as MMA columns) up to 8 tokens: at
   // T = 5..8 it takes about half the time of the grouped GEMM, whose 16-row tiles are bound by MMA
   // issue (measured by bench.py --crossover)
-  const bool decode = (T <= kDecodeMaxT) && path != MOE_PATH_GEMM && decode_router_fits(T, H, E);
+  const bool decode = (T <= kDecodeMaxT) && path != MOE_PATH_GEMM && path != MOE_PATH_MMQ && decode_router_fits(T, H, E);
   if (decode) {
     DecUnit *units = at<DecUnit>(ws, L.units);
     uint16_t *hdec = at<uint16_t>(ws, L.hdec);
@@ -362,9 +378,9 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
     if (e == cudaSuccess)
       e = expert_rows(xperm, offsets, rows, E, H, I, *routed, sh, at<uint16_t>(ws, L.hperm), operm,
                       at<int2>(ws, L.tiles), at<DecUnit>(ws, L.units), at<uint16_t>(ws, L.hdec), ctrl, s, path,
-                      gemm_ok);
+                      gemm_ok, at<int8_t>(ws, L.operm), at<float>(ws, L.dx));  // int8 rows: out_perm's region, free until the down GEMM
     if (e == cudaSuccess)
-      e = launch_combine(operm, row_of, w, T, k, H, hs ? operm + (size_t)P * H : nullptr, residual_opt, y, s);
+      e = launch_combine(operm, row_of, w, T, k, H, hs ? operm + (size_t)P * H : nullptr, residual_opt, y, s, ctrl);
   }
   if (e == cudaSuccess && idx_out_opt)
     e = cudaMemcpyAsync(idx_out_opt, idx, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s);
@@ -400,20 +416,21 @@ moe_status moe_stack_forward(const float *r_in, int32_t T, int32_t L, const floa
     if (!aligned16(Wr[l]) || (bias && bias[l] && !aligned16(bias[l]))) return MOE_ERR_ALIGNMENT;
   uint16_t *u = at<uint16_t>(ws, LY.u16);
   cudaStream_t s = (cudaStream_t)stream;
-  // decode-sized batches: the fused decode kernel walks all the layers in one launch (RMSNorm
-  // inside, a grid barrier between layers, the next layer's router rows and shared expert
-  // requested into L2 while the current layer finishes)
-  if (path == MOE_PATH_AUTO && T <= kDecodeMaxT && decode_router_fits(T, H, E)) {
-    cudaError_t e = launch_decode_stack(r_in, eps, T, L, H, Wr, bias, E, k, I, routed, hs ? shared : nullptr, r_out,
-                                        at<float>(ws, LY.logits), at<int32_t>(ws, LY.idx), at<float>(ws, LY.w),
-                                        at<uint16_t>(ws, LY.hdec), at<unsigned>(ws, LY.units), at<Ctrl>(ws, LY.ctrl),
-                                        s);
-    if (e == cudaSuccess) return MOE_OK;
-    if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge) return cuda_status(e);
-    (void)cudaGetLastError();
-  }
+  // decode-sized batches: one launch of the fused layer kernel per layer, RMSNorm inside it (a
+  // single launch walking all the layers with a grid barrier between them measured slower:
+  // 28.2 against 22.6 us per layer at one token)
+  const bool fused = path == MOE_PATH_AUTO && T <= kDecodeMaxT && decode_router_fits(T, H, E);
   for (int l = 0; l < L; ++l) {
     const float *r = (l == 0) ? r_in : r_out;
+    if (fused) {
+      cudaError_t e = launch_decode_fused(nullptr, r, eps, T, H, Wr[l], bias ? bias[l] : nullptr, E, k, I, routed[l],
+                                          hs ? &shared[l] : nullptr, r, r_out, at<float>(ws, LY.logits),
+                                          at<int32_t>(ws, LY.idx), at<float>(ws, LY.w), at<uint16_t>(ws, LY.hdec),
+                                          at<unsigned>(ws, LY.units), at<Ctrl>(ws, LY.ctrl), s);
+      if (e == cudaSuccess) continue;
+      if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge) return cuda_status(e);
+      (void)cudaGetLastError();
+    }
     if ((st = moe_rmsnorm_bf16(r, T, H, eps, u, stream)) != MOE_OK) return st;
     st = moe_layer_forward(u, T, Wr[l], bias ? bias[l] : nullptr, desc, &routed[l], hs ? &shared[l] : nullptr, r, r_out,
                            nullptr, nullptr, path, ws, ws_bytes, s);

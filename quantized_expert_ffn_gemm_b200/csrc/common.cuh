@@ -46,7 +46,7 @@ struct DecUnit {
 // ---------------------------------------------------------------- workspace layout
 struct WsLayout {
   size_t ctrl, logits, idx, w, hist, units, hdec, counts, offsets, row_of, src, xperm, hperm, operm, u16, tiles, wsplit,
-      total;
+      dx, total;
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -79,6 +79,7 @@ inline WsLayout ws_layout(int H, int E, int k, int I, int has_shared, int T) {
   L.u16 = take((size_t)T * H * 2);
   L.tiles = take((rows / 16 + (size_t)E + 4) * 8);
   L.wsplit = take((size_t)E * 3 * H * 2);
+  L.dx = take(rows * (size_t)(H / 32) * 4);  // int8-activation path: one scale per 32-value block
   L.total = off;
   return L;
 }
@@ -87,6 +88,11 @@ inline WsLayout ws_layout(int H, int E, int k, int I, int has_shared, int T) {
 __device__ __forceinline__ void set_device_error(Ctrl *c, int code, int info) {
   if (atomicCAS(&c->err, 0, code) == 0) c->err_info = info;
 }
+
+// A value outside the fp16 range of the expert operands became +-inf on conversion (RNE: above
+// 65504 by half an ulp). Callers collect this per thread and record MOE_ERR_RANGE once.
+__device__ __forceinline__ bool f16_inf(uint16_t b) { return (b & 0x7fffu) == 0x7c00u; }
+__device__ __forceinline__ bool f16x2_inf(uint32_t b) { return f16_inf((uint16_t)b) || f16_inf((uint16_t)(b >> 16)); }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
@@ -115,8 +121,10 @@ bool encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dt, int esize, c
 cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const uint16_t *x, int H, int with_shared,
                            int32_t *counts, int32_t *offsets, int32_t *row_of, int32_t *src, uint16_t *x_perm,
                            int32_t *hist, Ctrl *ctrl, cudaStream_t s);
+// ctrl != NULL: a non-finite expert output records MOE_ERR_RANGE there
 cudaError_t launch_combine(const uint16_t *out_perm, const int32_t *row_of, const float *w, int T, int k, int H,
-                           const uint16_t *shared_out, const float *residual, float *y, cudaStream_t s);
+                           const uint16_t *shared_out, const float *residual, float *y, cudaStream_t s,
+                           Ctrl *ctrl = nullptr);
 cudaError_t launch_rmsnorm(const float *r, int T, int H, float eps, uint16_t *u, cudaStream_t s);
 cudaError_t launch_dequant_rows(const moe_qmat &m, int expert, int row0, int nrows, float *out_f32, uint16_t *out_f16,
                                 cudaStream_t s);
@@ -144,20 +152,27 @@ cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float ep
                                 int32_t *idx, float *w, uint16_t *hdec, unsigned *unit_ready, Ctrl *ctrl,
                                 cudaStream_t s);
 
-// the fused decode kernel over the L layers of a stack in one launch per 48 layers (RMSNorm of the
-// stream before each router, residual added in place): r_out = stack(r_in). Per-layer arrays are
-// host arrays (as moe_stack_forward takes them); cudaErrorNotSupported when the shape cannot take it.
-cudaError_t launch_decode_stack(const float *r_in, float eps, int T, int L, int H, const float *const *Wr,
-                                const float *const *bias, int E, int k, int I, const moe_expert_set *routed,
-                                const moe_expert_set *shared, float *r_out, float *logits, int32_t *idx, float *w,
-                                uint16_t *hdec, unsigned *unit_ready, Ctrl *ctrl, cudaStream_t s);
-
 // test hook: a grid barrier that waits for one arrival more than the `ctas` CTAs make, giving up
 // after limit_ns with MOE_ERR_TIMEOUT in the control area
 cudaError_t launch_barrier_starve(Ctrl *ctrl, int ctas, uint64_t limit_ns, cudaStream_t s);
 
 // prefill path (tcgen05 grouped GEMM)
 int gemm_shape_supported(int H, int I);
+// tile list (group, first row) of slice-row slices (a multiple of 16, <= 192) of every group of
+// more than min_rows rows, longest slices first; count in ctrl->n_tiles
+cudaError_t launch_tile_list(const int32_t *offsets, int n_groups, int n_rows, int slice, int2 *tiles, Ctrl *ctrl,
+                             cudaStream_t s, int min_rows = 0);
+// int8-activation (MMQ-style) gate/up + SwiGLU on tcgen05 kind::i8, Q2 weights: x_perm is
+// quantized per 32-value block into x_q [n_rows][H] int8 and dx [n_rows][H/32] fp32 (scratch),
+// h_perm as the fp16 path writes it
+int mmq_shape_supported(int H, int I, int qtype);
+cudaError_t launch_mmq_gate_up(const uint16_t *x_perm, const int32_t *offsets, int n_rows, int E, int H, int I,
+                               const moe_expert_set &routed, const moe_expert_set *shared, int8_t *x_q, float *dx,
+                               uint16_t *h_perm, int2 *tiles, Ctrl *ctrl, cudaStream_t s);
+// the down projection alone (grouped GEMM, second kernel of launch_grouped_ffn) over h_perm
+cudaError_t launch_grouped_down(const uint16_t *h_perm, const int32_t *offsets, int n_rows, int E, int H, int I,
+                                const moe_expert_set &routed, const moe_expert_set *shared, uint16_t *out_perm,
+                                int2 *tiles, Ctrl *ctrl, cudaStream_t s);
 // groups of at most min_rows rows are skipped (min_rows > 0: the caller runs them on the GEMV path)
 cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, int n_rows, int E, int H, int I,
                                const moe_expert_set &routed, const moe_expert_set *shared, uint16_t *h_perm,
@@ -183,7 +198,8 @@ cudaError_t smem_limit_once(F *func, size_t bytes) {
 enum KernelId {
   KID_ROUTER_DECODE = 0, KID_ROUTER_GEMM, KID_TOPK, KID_PERM_HIST, KID_PERM_SCAN, KID_PERM_SCATTER, KID_PERM_FILL,
   KID_PERM_GATHER, KID_COMBINE, KID_RMSNORM, KID_DEQUANT_ROWS, KID_DEC_UNITS, KID_DEC_GATE_UP, KID_DEC_DOWN,
-  KID_TILE_LIST, KID_GEMM_GATE_UP, KID_GEMM_DOWN, KID_ROUTER_SPLIT, KID_ROUTER_TC, KID_DECODE_FUSED, KID_COUNT
+  KID_TILE_LIST, KID_GEMM_GATE_UP, KID_GEMM_DOWN, KID_ROUTER_SPLIT, KID_ROUTER_TC, KID_DECODE_FUSED, KID_MMQ_QUANT,
+  KID_MMQ_GATE_UP, KID_COUNT
 };
 void timer_begin(int kid, cudaStream_t s);
 void timer_end(int kid, cudaStream_t s);

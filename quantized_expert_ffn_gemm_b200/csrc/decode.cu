@@ -20,10 +20,12 @@
 namespace moe {
 
 // ---------------------------------------------------------------- gate/up + SwiGLU
-// grid (max_units, I/16); block = 8 warps: warps 0-3 gate, 4-7 up, for the same 16 rows; warp
-// slice q takes K steps q, q+4, ... so every warp has a short MMA chain and the SM has many
-// warps in flight. Partials are summed in shared memory in fixed order.
+// grid (units, I/64); block = 8 warps: warps 0-3 gate, 4-7 up, for the same 16 rows of each of the
+// CTA's four 16-feature blocks; warp slice q takes K steps q, q+4, ... so every warp has a short
+// MMA chain and the SM has many warps in flight. Partials are summed in shared memory in fixed
+// order.
 constexpr int kGuWarps = 8;
+constexpr int kGuBlocks = 4;  // 16-feature blocks per CTA (I % 64 == 0)
 
 template <bool SRC_BF16, int QT>
 __global__ void __launch_bounds__(kGuWarps * 32)
@@ -31,61 +33,79 @@ dec_gate_up_kernel(const void *__restrict__ x, int H, int I, moe_expert_set rout
                    const DecUnit *__restrict__ units, Ctrl *__restrict__ ctrl, uint16_t *__restrict__ hdec) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int n_units = ctrl->n_units;
-  // units are taken grid-stride (the grid is sized by the device, not by the largest possible
-  // unit count, so an empty or short unit list costs no flood of idle CTAs)
-  for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-  const DecUnit un = units[u];
-  if (un.expert < 0 || un.expert >= (un.set ? shared.gate.n_experts : routed.gate.n_experts)) {
-    if (threadIdx.x == 0 && blockIdx.y == 0) set_device_error(ctrl, MOE_ERR_DEVICE_CHECK, un.expert);
-    continue;
-  }
   const int xstride = H + 4;
   __half *xs = reinterpret_cast<__half *>(smem_raw);
   __shared__ float part[kGuWarps][16][8];
-  __syncthreads();  // the previous unit's reads of xs and part are done
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int mat = warp >> 2, slice = warp & 3;
-  const MatView mv = mat_sel(routed, shared, un.set, mat, un.expert);
-  const int r0 = blockIdx.y * 16;
-  const bool colok = (un.mask >> g) & 1;
   const int nsteps = (H + kStepK - 1) / kStepK;
   const __half *xcol = xs + (size_t)g * xstride;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
-  if (nsteps <= 8) {
-    // at most two steps per slice: request them before staging the activations
+  // A CTA takes kGuBlocks consecutive 16-feature blocks of one unit, so the unit's activation
+  // columns are staged once for all of them; the next block's weights are requested before the
+  // current block's MMAs. Units are taken grid-stride (the grid is sized by the device, not by the
+  // largest possible unit count, so an empty or short unit list costs no flood of idle CTAs).
+  for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+    const DecUnit un = units[u];
+    if (un.expert < 0 || un.expert >= (un.set ? shared.gate.n_experts : routed.gate.n_experts)) {
+      if (threadIdx.x == 0 && blockIdx.y == 0) set_device_error(ctrl, MOE_ERR_DEVICE_CHECK, un.expert);
+      continue;
+    }
+    __syncthreads();  // the previous unit's reads of xs and part are done
+    const MatView mv = mat_sel(routed, shared, un.set, mat, un.expert);
+    const bool colok = (un.mask >> g) & 1;
+    const int rb0 = blockIdx.y * kGuBlocks;
     StepFrag f[2];
-    load_step<QT>(f[0], mv, r0, slice, slice < nsteps);
-    load_step<QT>(f[1], mv, r0, slice + 4, slice + 4 < nsteps);
-    stage_x<SRC_BF16>(x, un.xrow0, un.mask, H, xs, xstride);
-    __syncthreads();
-    if (slice < nsteps) mma_step<QT>(acc, acc2, f[0], xcol, slice * kStepK + 64 * t,
-                                     colok && slice * kStepK + 64 * t < H);
-    if (slice + 4 < nsteps) mma_step<QT>(acc, acc2, f[1], xcol, (slice + 4) * kStepK + 64 * t,
-                                         colok && (slice + 4) * kStepK + 64 * t < H);
-  } else {
-    stage_x<SRC_BF16>(x, un.xrow0, un.mask, H, xs, xstride);
-    __syncthreads();
-    for (int st = slice; st < nsteps; st += 4) {
-      StepFrag f;
-      load_step<QT>(f, mv, r0, st, true);
-      mma_step<QT>(acc, acc2, f, xcol, st * kStepK + 64 * t, colok && st * kStepK + 64 * t < H);
+    if (nsteps <= 8) {  // at most two steps per slice: the first block's are requested before staging
+      load_step<QT>(f[0], mv, rb0 * 16, slice, slice < nsteps);
+      load_step<QT>(f[1], mv, rb0 * 16, slice + 4, slice + 4 < nsteps);
     }
-  }
-  part[warp][g][2 * t] = acc[0] + acc2[0];
-  part[warp][g][2 * t + 1] = acc[1] + acc2[1];
-  part[warp][g + 8][2 * t] = acc[2] + acc2[2];
-  part[warp][g + 8][2 * t + 1] = acc[3] + acc2[3];
-  __syncthreads();
-  if (threadIdx.x < 128) {  // one (row, column) per thread
-    const int row = threadIdx.x & 15, col = threadIdx.x >> 4;
-    if ((un.mask >> col) & 1) {
-      const float gv = (part[0][row][col] + part[1][row][col]) + (part[2][row][col] + part[3][row][col]);
-      const float uv = (part[4][row][col] + part[5][row][col]) + (part[6][row][col] + part[7][row][col]);
-      const float hv = gv / (1.0f + expf(-gv)) * uv;
-      hdec[((size_t)u * 8 + col) * I + r0 + row] = __half_as_ushort(__float2half_rn(hv));
+    bool bad = stage_x<SRC_BF16>(x, un.xrow0, un.mask, H, xs, xstride);
+    __syncthreads();
+    for (int b = 0; b < kGuBlocks; ++b) {
+      const int r0 = (rb0 + b) * 16;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
+      if (nsteps <= 8) {
+        StepFrag fn[2];
+        const bool more = b + 1 < kGuBlocks;
+        if (more) {
+          load_step<QT>(fn[0], mv, r0 + 16, slice, slice < nsteps);
+          load_step<QT>(fn[1], mv, r0 + 16, slice + 4, slice + 4 < nsteps);
+        }
+        if (slice < nsteps) mma_step<QT>(acc, acc2, f[0], xcol, slice * kStepK + 64 * t,
+                                         colok && slice * kStepK + 64 * t < H);
+        if (slice + 4 < nsteps) mma_step<QT>(acc, acc2, f[1], xcol, (slice + 4) * kStepK + 64 * t,
+                                             colok && (slice + 4) * kStepK + 64 * t < H);
+        if (more) {
+          f[0] = fn[0];
+          f[1] = fn[1];
+        }
+      } else {
+        for (int st = slice; st < nsteps; st += 4) {
+          StepFrag fs;
+          load_step<QT>(fs, mv, r0, st, true);
+          mma_step<QT>(acc, acc2, fs, xcol, st * kStepK + 64 * t, colok && st * kStepK + 64 * t < H);
+        }
+      }
+      part[warp][g][2 * t] = acc[0] + acc2[0];
+      part[warp][g][2 * t + 1] = acc[1] + acc2[1];
+      part[warp][g + 8][2 * t] = acc[2] + acc2[2];
+      part[warp][g + 8][2 * t + 1] = acc[3] + acc2[3];
+      __syncthreads();
+      if (threadIdx.x < 128) {  // one (row, column) per thread
+        const int row = threadIdx.x & 15, col = threadIdx.x >> 4;
+        if ((un.mask >> col) & 1) {
+          const float gv = (part[0][row][col] + part[1][row][col]) + (part[2][row][col] + part[3][row][col]);
+          const float uv = (part[4][row][col] + part[5][row][col]) + (part[6][row][col] + part[7][row][col]);
+          const float hv = gv / (1.0f + expf(-gv)) * uv;
+          const uint16_t hb = __half_as_ushort(__float2half_rn(hv));
+          bad |= f16_inf(hb);
+          hdec[((size_t)u * 8 + col) * I + r0 + row] = hb;
+        }
+      }
+      __syncthreads();  // part is rewritten by the next block
     }
+    if (bad) set_device_error(ctrl, MOE_ERR_RANGE, 2);
   }
-  }  // units
 }
 
 template <bool B, int Q>
@@ -106,8 +126,9 @@ cudaError_t launch_decode_gate_up(const void *x, int x_is_bf16, int H, int I, co
                                   uint16_t *hdec, cudaStream_t s) {
   const moe_expert_set sh = shared ? *shared : routed;
   // about eight CTAs per SM in all; each walks units grid-stride
-  const int cap = (8 * num_sms() + I / 16 - 1) / (I / 16);
-  const dim3 grid(max_units < cap ? (max_units > 0 ? max_units : 1) : cap, I / 16);
+  const int ny = I / (16 * kGuBlocks);
+  const int cap = (8 * num_sms() + ny - 1) / ny;
+  const dim3 grid(max_units < cap ? (max_units > 0 ? max_units : 1) : cap, ny);
   const size_t smem = (size_t)8 * (H + 4) * 2;
   const int qt = routed.gate.qtype;
 #define MOE_GU(B, Q) launch_gu<B, Q>(grid, smem, s, x, H, I, routed, sh, units, ctrl, hdec)
@@ -255,7 +276,11 @@ dec_down_kernel(int H, int I, moe_expert_set routed, moe_expert_set shared, cons
           for (int e = 0; e < 4; ++e) {
             const int row = g + (e >> 1) * 8, col = 2 * t + (e & 1);
             if ((un.mask >> col) & 1)
-              out_rows[(size_t)(un.xrow0 + col) * H + r0 + row] = __half_as_ushort(__float2half_rn(acc[e]));
+            {
+              const uint16_t ob = __half_as_ushort(__float2half_rn(acc[e]));
+              if (f16_inf(ob)) set_device_error(ctrl, MOE_ERR_RANGE, 3);
+              out_rows[(size_t)(un.xrow0 + col) * H + r0 + row] = ob;
+            }
           }
         } else {
           const float wa = un.w[2 * t], wb = un.w[2 * t + 1];

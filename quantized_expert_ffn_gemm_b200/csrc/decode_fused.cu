@@ -91,18 +91,6 @@ struct UnitMats {
   const uint8_t *hibits[3];
 };
 
-// Per-layer pointers of a stack run in one launch (moe_stack_forward at decode sizes): the kernel
-// walks the layers with a grid barrier between them. Passed as a kernel parameter (~12 KB for
-// kStackMaxL layers; longer stacks are launched in pieces).
-constexpr int kStackMaxL = 48;
-struct StackLayers {
-  int n;                                 // layers in this launch
-  const float *Wr[kStackMaxL];
-  const float *bias[kStackMaxL];         // entries may be NULL
-  moe_expert_set routed[kStackMaxL];
-  moe_expert_set shared[kStackMaxL];     // used when has_shared
-};
-
 struct FusedLayout {
   size_t xraw, x16, hs, part, red, units, umats, sidx, sw, misc, slot, src, keys, ctop, cand, firstof, pcnt, bars, ring,
       total;
@@ -114,9 +102,18 @@ __host__ __device__ inline FusedLayout fused_layout(int T, int H, int E, int I, 
   FusedLayout L{};
   size_t o = 0;
   auto take = [&](size_t b) { size_t r = o; o = fl_align(o + b); return r; };
+  // Phase-local buffers share one region: the tokens, logit keys and top-k lists serve P0-P2
+  // only, the staged h columns P3 only, and a CTA's P3 starts after its P2 is complete.
   L.xraw = take((size_t)T * H * 2);
   L.x16 = take((size_t)T * (H + 4) * 2);
+  L.keys = take((size_t)T * E * 4);              // [token][expert] order-preserving logit keys
+  L.ctop = take((size_t)T * 32 * 8);             // [token][32] chunk-top codes (threshold candidates)
+  L.cand = take((size_t)T * 32 * 8 + 128);       // [token][32] codes above the threshold, [8] counts, [8] tau
+  L.firstof = take((size_t)E * 4);                // expert -> first pair choosing it
+  const size_t early_end = o;
+  o = 0;
   L.hs = take((size_t)hs_cols * (I + 4) * 2);    // staged h columns (down phase)
+  o = early_end > o ? early_end : o;
   L.part = take((size_t)2 * 2 * 8 * 16 * 8 * 4);  // [group][buffer][K step][16 rows][8 columns]
   L.red = take((size_t)kFWarps * 16 * 8 * 4);
   L.units = take((size_t)kFMaxUnits * sizeof(DecUnit));
@@ -126,10 +123,6 @@ __host__ __device__ inline FusedLayout fused_layout(int T, int H, int E, int I, 
   L.misc = take(16 * 4);
   L.slot = take((size_t)(kFMaxUnits + 1) * 4);
   L.src = take((size_t)kFSlots * 4);
-  L.keys = take((size_t)T * E * 4);              // [token][expert] order-preserving logit keys
-  L.ctop = take((size_t)T * 32 * 8);             // [token][32] chunk-top codes (threshold candidates)
-  L.cand = take((size_t)T * 32 * 8 + 128);       // [token][32] codes above the threshold, [8] counts, [8] tau
-  L.firstof = take((size_t)E * 4);                // expert -> first pair choosing it
   L.pcnt = take((size_t)(kFMaxUnits + 1) * 4);
   L.bars = take((size_t)kFMaxRing * 8);
   o = fl_align(o, 128);
@@ -291,8 +284,8 @@ __device__ __forceinline__ void frag_from_smem(StepFrag &f, const uint8_t *ca, c
 
 // TMAX: the largest token count the instance takes (1, 2, 4 or 8); the token loops of the router
 // are unrolled to TMAX, so the common single-token instance carries no code for the others.
-template <int QT, int TMAX, bool STACK>
-__device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers *SL) {
+template <int QT, int TMAX>
+__global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int T = a.T, H = a.H, E = a.E, k = a.k, I = a.I;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
@@ -328,7 +321,6 @@ __device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers
   const unsigned nblk = gridDim.x;
   __shared__ unsigned long long s_base;
   __shared__ volatile int s_abort;
-  __shared__ int s_pbase[kFMaxRing];  // phases each slot completed in earlier layers of this launch
   if (tid == 0) {  // arrivals of earlier launches: a whole number of grids (before this CTA arrives)
     unsigned long long v;
     asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(&ctrl->bar_arrivals) : "memory");
@@ -337,7 +329,6 @@ __device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers
     for (int s = 0; s < R; ++s) mbar_init(full(s), 32);  // one arrival per lane of the filling warp
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (tid < kFMaxRing) s_pbase[tid] = 0;
   // a bounded wait that gives up at once after an earlier wait of this CTA gave up
   auto wait_bar = [&](uint32_t bar, uint32_t parity, int where) -> bool {
     if (s_abort) return false;
@@ -346,20 +337,15 @@ __device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers
     set_device_error(ctrl, MOE_ERR_TIMEOUT, where);
     return false;
   };
-  // parity of fill q's phase: the slot's phases of earlier layers, then one per fill q, q + R, ...
-  auto fill_parity = [&](int q) { return (uint32_t)(s_pbase[q % R] + q / R) & 1u; };
-  const int nl = STACK ? SL->n : 1;
+  // parity of fill q's phase: one phase per fill q, q + R, ... of the slot
+  auto fill_parity = [&](int q) { return (uint32_t)(q / R) & 1u; };
   bool ok = true;
-
-  for (int l = 0; l < nl; ++l) {
-  // this layer's pointers: the launch's arguments, or stack layer l (its input and residual are
-  // the stream r: r_in for the first layer, then r_out, which every layer updates in place)
-  const float *const lWr = STACK ? SL->Wr[l] : a.Wr;
-  const float *const lbias = STACK ? SL->bias[l] : a.bias;
-  const moe_expert_set &lRS = STACK ? SL->routed[l] : a.routed;
-  const moe_expert_set &lSS = STACK ? SL->shared[l] : a.shared;
-  const float *const lrn = (STACK && l > 0) ? a.y : a.r_norm;
-  const float *const lres = (STACK && l > 0) ? a.y : a.residual;
+  const float *const lWr = a.Wr;
+  const float *const lbias = a.bias;
+  const moe_expert_set &lRS = a.routed;
+  const moe_expert_set &lSS = a.shared;
+  const float *const lrn = a.r_norm;
+  const float *const lres = a.residual;
 
   // ---------------- P0: this warp's router rows are requested first, then the tokens are staged
   const int H4 = H / 4, HQ = H4 / 4;  // float4 per quarter of a router row (<= 128: H <= 2048)
@@ -375,20 +361,34 @@ __device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers
   };
   load_router((int)blockIdx.x + es * G);
   __shared__ float s_inv[kDecodeMaxT];
+  // token staging in chunks of 8 values: at most 4 per thread (T <= 8, H <= 2048)
+  constexpr int kChunks = 4;
+  const int H8 = H / 8, nchunk = T * H8;
+  float4 cf[2 * kChunks];
   if (lrn) {
+    // the stream's rows are requested first, then the RMSNorm sums, whose loads overlap them
+#pragma unroll
+    for (int j = 0; j < kChunks; ++j) {
+      const int i = tid + j * kFThreads;
+      if (i < nchunk) {
+        cf[2 * j] = __ldcg(reinterpret_cast<const float4 *>(lrn) + 2 * i);
+        cf[2 * j + 1] = __ldcg(reinterpret_cast<const float4 *>(lrn) + 2 * i + 1);
+      }
+    }
     // RMSNorm of the residual stream (no gain): the same summation order and rounding as the
     // stand-alone RMSNorm kernel (256 threads: strided fmaf chains, warp butterflies, 8 warp
-    // partials in order), so u is bit-identical to it. Coherent (L2) loads: in a stack launch
-    // the stream was written by other CTAs in the previous layer.
+    // partials in order), so u is bit-identical to it
     __shared__ float s_part[kDecodeMaxT][8];
     if (tid < 256) {
       for (int t = 0; t < T; ++t) {
         const float *row = lrn + (size_t)t * H;
+        float rr[8];  // the thread's H / 256 <= 8 values, all requested before the chain
+#pragma unroll
+        for (int j = 0; j < 8; ++j) rr[j] = (tid + 256 * j < H) ? __ldcg(row + tid + 256 * j) : 0.0f;
         float ss = 0.0f;
-        for (int h = tid; h < H; h += 256) {
-          const float rv1 = __ldcg(row + h);
-          ss = fmaf(rv1, rv1, ss);
-        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (tid + 256 * j < H) ss = fmaf(rr[j], rr[j], ss);
         ss = warp_sum(ss);
         if (lane == 0) s_part[t][warp] = ss;
       }
@@ -402,37 +402,37 @@ __device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers
     }
     __syncthreads();
   }
-  {
-    const int H8 = H / 8, n = T * H8;
-    for (int i = tid; i < n; i += kFThreads) {
-      uint4 v;
-      if (lrn) {
-        const int t = i / H8;
-        const float4 f0 = __ldcg(reinterpret_cast<const float4 *>(lrn) + 2 * i);
-        const float4 f1 = __ldcg(reinterpret_cast<const float4 *>(lrn) + 2 * i + 1);
-        const float iv = s_inv[t];
-        auto pk = [&](float lo, float hi) {
-          const __nv_bfloat16 bl = __float2bfloat16_rn(lo * iv), bh = __float2bfloat16_rn(hi * iv);
-          return (uint32_t)*reinterpret_cast<const uint16_t *>(&bl) |
-                 ((uint32_t)*reinterpret_cast<const uint16_t *>(&bh) << 16);
-        };
-        v = make_uint4(pk(f0.x, f0.y), pk(f0.z, f0.w), pk(f1.x, f1.y), pk(f1.z, f1.w));
-      } else {
-        v = __ldg(reinterpret_cast<const uint4 *>(a.x) + i);
-      }
-      reinterpret_cast<uint4 *>(xraw)[i] = v;
-      const int t = i / H8, c = i % H8;
-      const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-      uint32_t o[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        __half2 h = __floats2half2_rn(__uint_as_float(in[q] << 16), __uint_as_float(in[q] & 0xffff0000u));
-        o[q] = *reinterpret_cast<uint32_t *>(&h);
-      }
-      uint2 *d = reinterpret_cast<uint2 *>(x16 + (size_t)t * xs16 + xs_pos(8 * c));
-      d[0] = make_uint2(o[0], o[1]);
-      d[1] = make_uint2(o[2], o[3]);
+  for (int j = 0; j < kChunks; ++j) {
+    const int i = tid + j * kFThreads;
+    if (i >= nchunk) break;
+    uint4 v;
+    if (lrn) {
+      const int t = i / H8;
+      const float4 f0 = cf[2 * j], f1 = cf[2 * j + 1];
+      const float iv = s_inv[t];
+      auto pk = [&](float lo, float hi) {
+        const __nv_bfloat16 bl = __float2bfloat16_rn(lo * iv), bh = __float2bfloat16_rn(hi * iv);
+        return (uint32_t)*reinterpret_cast<const uint16_t *>(&bl) |
+               ((uint32_t)*reinterpret_cast<const uint16_t *>(&bh) << 16);
+      };
+      v = make_uint4(pk(f0.x, f0.y), pk(f0.z, f0.w), pk(f1.x, f1.y), pk(f1.z, f1.w));
+    } else {
+      v = __ldg(reinterpret_cast<const uint4 *>(a.x) + i);
     }
+    reinterpret_cast<uint4 *>(xraw)[i] = v;
+    const int t = i / H8, c = i % H8;
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      __half2 h = __floats2half2_rn(__uint_as_float(in[q] << 16), __uint_as_float(in[q] & 0xffff0000u));
+      o[q] = *reinterpret_cast<uint32_t *>(&h);
+      if (f16x2_inf(o[q])) set_device_error(ctrl, MOE_ERR_RANGE, 4);
+    }
+    uint2 *d = reinterpret_cast<uint2 *>(x16 + (size_t)t * xs16 + xs_pos(8 * c));
+    d[0] = make_uint2(o[0], o[1]);
+    d[1] = make_uint2(o[2], o[3]);
   }
   if (lbias) prefetch_range(lbias, (size_t)E * 4, tid, kFThreads);
   // per-unit readiness counters start at zero; every increment comes after the first grid barrier
@@ -485,7 +485,7 @@ __device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers
       __syncthreads();
     }
   }
-  ok = grid_barrier(ctrl, s_base + (unsigned long long)(2 * l + 1) * nblk, 31, true) && ok;
+  ok = grid_barrier(ctrl, s_base + nblk, 31, true) && ok;
 
   // ---------------- P1b: top-k and unit list, computed identically by every CTA
   if (ok) {
@@ -520,7 +520,7 @@ __device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers
     }
     {  // into L2 while the top-k runs: the shared expert's rows (always selected)
       const int nthr = gridDim.x * kFThreads, first = blockIdx.x * kFThreads + tid;
-      if (a.has_shared && !(STACK && l > 0)) prefetch_shared<QT>(lSS, I, H, first, nthr);  // later layers: earlier
+      if (a.has_shared) prefetch_shared<QT>(lSS, I, H, first, nthr);
     }
     if (T > 1)
       for (int e = tid; e < E; e += kFThreads) s_firstof[e] = 0x7fffffff;
@@ -580,6 +580,41 @@ __device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers
     }
     __syncthreads();
     const int P = T * k;
+    if (TMAX == 1) {
+      // one token: its k experts are k distinct units in slot order, then the shared expert;
+      // column slot u holds unit u's only column. Records, plane pointers and the routing
+      // copy in one parallel step.
+      const int nuu = k + (a.has_shared ? 1 : 0);
+      if (tid < 3 * nuu) {
+        const int u = tid / 3, which = tid % 3;
+        const bool shu = u == k;
+        const MatView mv = mat_sel(lRS, lSS, shu ? 1 : 0, which, shu ? 0 : s_idx[u]);
+        s_um[u].codes[which] = mv.codes;
+        s_um[u].scales[which] = mv.scales;
+        s_um[u].hibits[which] = mv.hibits;
+        if (which == 0) {
+          DecUnit &d = su[u];
+          d.expert = shu ? 0 : s_idx[u];
+          d.set = shu ? 1 : 0;
+          d.mask = 1;
+          d.xrow0 = 0;
+          d.w[0] = shu ? 1.0f : s_w[u];
+#pragma unroll
+          for (int cc = 1; cc < 8; ++cc) d.w[cc] = 0.0f;
+          s_slot[u] = u;
+          s_src[u] = u * 8;
+        }
+      }
+      if (tid == 0) {
+        misc[0] = nuu;
+        s_slot[nuu] = nuu;
+      }
+      if (blockIdx.x == 0 && tid < k) {
+        a.idx[tid] = s_idx[tid];
+        a.w[tid] = s_w[tid];
+      }
+      __syncthreads();
+    } else {
     if (T > 1) {  // expert -> first pair choosing it
       for (int p = tid; p < P; p += kFThreads) atomicMin(&s_firstof[s_idx[p]], p);
       __syncthreads();
@@ -675,6 +710,7 @@ __device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers
       s_um[u].hibits[which] = mv.hibits;
     }
     __syncthreads();
+    }  // T > 1
   }
   const int nu = ok ? misc[0] : 0;
   const int rbs8 = I / 8;                     // gate/up items per unit
@@ -768,7 +804,9 @@ __device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers
             uv += pb[(sl * 16 + 8 + row) * 8 + col];
           }
           const float hv = gv / (1.0f + expf(-gv)) * uv;
-          a.hdec[((size_t)u * 8 + col) * I + r0 + row] = __half_as_ushort(__float2half_rn(hv));
+          const uint16_t hb = __half_as_ushort(__float2half_rn(hv));
+          if (f16_inf(hb)) set_device_error(ctrl, MOE_ERR_RANGE, 5);
+          a.hdec[((size_t)u * 8 + col) * I + r0 + row] = hb;
         }
       }
       // the item's h is written: count it for its unit (the group barrier orders the 64 stores
@@ -780,19 +818,6 @@ __device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers
   // This CTA's gate/up items are all consumed (the ring rule of P3 below needs it); no grid
   // barrier: each down unit waits for its own unit's h instead.
   __syncthreads();
-  if (STACK && l + 1 < nl) {
-    // into L2 for the next layer while this one finishes: this CTA's router rows (the experts its
-    // warps load first), the router bias, and a share of the next shared expert
-    const int nthr = gridDim.x * kFThreads, first = blockIdx.x * kFThreads + tid;
-    const float *nWr = SL->Wr[l + 1];
-    for (int es2 = 0; es2 < 4; ++es2) {
-      const int e = (int)blockIdx.x + es2 * G;
-      if (e < E) prefetch_range(nWr + (size_t)e * H, (size_t)H * 4, tid, kFThreads);
-    }
-    if (SL->bias[l + 1] && blockIdx.x == 1) prefetch_range(SL->bias[l + 1], (size_t)E * 4, tid, kFThreads);
-    if (a.has_shared) prefetch_shared<QT>(SL->shared[l + 1], I, H, first, nthr);
-  }
-
   // ---------------- P3: down projection + weighted combine (+ residual) for 16 output features per CTA.
   // Piece d of a row block shares its slot with piece d - R. Before waiting on piece d's fill a
   // warp waits until piece d - R is consumed (its last consumer then issues piece d's fill), so
@@ -845,12 +870,25 @@ __device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers
           unsigned v;
           asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a.ready + u) : "memory");
           (void)v;
-          const int I8 = I / 8, c0 = s_slot[u], nc = s_slot[u + 1] - c0;
-          for (int vi = lane; vi < nc * I8; vi += 32) {
-            const uint4 hv = __ldcg(reinterpret_cast<const uint4 *>(a.hdec + (size_t)s_src[c0 + vi / I8] * I) + vi % I8);
-            uint2 *dd = reinterpret_cast<uint2 *>(hs + (size_t)(c0 + vi / I8) * xstride + xs_pos(8 * (vi % I8)));
-            dd[0] = make_uint2(hv.x, hv.y);
-            dd[1] = make_uint2(hv.z, hv.w);
+          // all of a lane's loads (eight per round) go out before its stores: one L2 round trip
+          const int I8 = I / 8, c0 = s_slot[u], nv = (s_slot[u + 1] - c0) * I8;
+          for (int v0 = lane; v0 < nv; v0 += 8 * 32) {
+            uint4 hv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int vi = v0 + 32 * j;
+              hv[j] = vi < nv ? __ldcg(reinterpret_cast<const uint4 *>(a.hdec + (size_t)s_src[c0 + vi / I8] * I) + vi % I8)
+                              : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int vi = v0 + 32 * j;
+              if (vi < nv) {
+                uint2 *dd = reinterpret_cast<uint2 *>(hs + (size_t)(c0 + vi / I8) * xstride + xs_pos(8 * (vi % I8)));
+                dd[0] = make_uint2(hv[j].x, hv[j].y);
+                dd[1] = make_uint2(hv[j].z, hv[j].w);
+              }
+            }
           }
           __syncwarp();
         }
@@ -932,28 +970,9 @@ __device__ __forceinline__ void fused_body(const FusedArgs &a, const StackLayers
     }
   }
 
-  if (STACK && l + 1 < nl) {
-    // the next layer normalises the whole stream: every CTA's rows of this layer first
-    ok = grid_barrier(ctrl, s_base + (unsigned long long)(2 * l + 2) * nblk, 33, ok) && ok;
-    if (tid < R) s_pbase[tid] += n_total / R + (tid < n_total % R ? 1 : 0);  // every fill was consumed
-    __syncthreads();
-  }
-  }  // layers
 
   // ---------------- no copy may still be writing this CTA's shared memory when it exits
   cp_async_wait_all();
-}
-
-template <int QT, int TMAX>
-__global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedArgs a) {
-  fused_body<QT, TMAX, false>(a, nullptr);
-}
-
-// the same, over the layers of a stack in one launch
-template <int QT, int TMAX>
-__global__ void __launch_bounds__(kFThreads, 1) decode_stack_kernel(const FusedArgs a,
-                                                                   const __grid_constant__ StackLayers SL) {
-  fused_body<QT, TMAX, true>(a, &SL);
 }
 
 // Test hook of the failure path: every CTA arrives at the fused kernel's grid barrier, which is
@@ -991,7 +1010,7 @@ cudaError_t launch_barrier_starve(Ctrl *ctrl, int ctas, uint64_t limit_ns, cudaS
 
 // Shapes, ring and shared-memory plan of a fused launch; false when the shape or the device cannot
 // take the kernel.
-static bool fused_plan(int T, int H, int E, int k, int I, const moe_expert_set &routed, bool has_shared, bool stack,
+static bool fused_plan(int T, int H, int E, int k, int I, const moe_expert_set &routed, bool has_shared,
                        FusedArgs &a, const void *&fn, size_t &smem) {
   const int hs_cols = T * k + (has_shared ? T : 0);
   if (T < 1 || T > kDecodeMaxT || E > kFMaxE || H > 2048 || I > 1024 || hs_cols > kFSlots || k > 16) return false;
@@ -1017,12 +1036,8 @@ static bool fused_plan(int T, int H, int E, int k, int I, const moe_expert_set &
 #define MOE_FUSED_FN(K, Q, TM) reinterpret_cast<const void *>(K<Q, TM>)
 #define MOE_FUSED_T(K, Q) (tmax == 1 ? MOE_FUSED_FN(K, Q, 1) : tmax == 2 ? MOE_FUSED_FN(K, Q, 2) \
                            : tmax == 4 ? MOE_FUSED_FN(K, Q, 4) : MOE_FUSED_FN(K, Q, 8))
-  if (stack)
-    fn = qt == MOE_Q3 ? MOE_FUSED_T(decode_stack_kernel, 3)
-         : qt == MOE_Q4 ? MOE_FUSED_T(decode_stack_kernel, 4) : MOE_FUSED_T(decode_stack_kernel, 2);
-  else
-    fn = qt == MOE_Q3 ? MOE_FUSED_T(decode_fused_kernel, 3)
-         : qt == MOE_Q4 ? MOE_FUSED_T(decode_fused_kernel, 4) : MOE_FUSED_T(decode_fused_kernel, 2);
+  fn = qt == MOE_Q3 ? MOE_FUSED_T(decode_fused_kernel, 3)
+       : qt == MOE_Q4 ? MOE_FUSED_T(decode_fused_kernel, 4) : MOE_FUSED_T(decode_fused_kernel, 2);
 #undef MOE_FUSED_T
 #undef MOE_FUSED_FN
   if (smem_limit_once_impl(fn, kFSmemMax) != cudaSuccess) return false;
@@ -1068,7 +1083,7 @@ cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float ep
   FusedArgs a;
   const void *fn = nullptr;
   size_t smem = 0;
-  if (!fused_plan(T, H, E, k, I, routed, shared != nullptr, false, a, fn, smem)) {
+  if (!fused_plan(T, H, E, k, I, routed, shared != nullptr, a, fn, smem)) {
     (void)cudaGetLastError();
     return cudaErrorNotSupported;
   }
@@ -1089,49 +1104,6 @@ cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float ep
   a.ctrl = ctrl;
   void *args[] = {&a};
   return fused_launch(fn, smem, args, s);
-}
-
-cudaError_t launch_decode_stack(const float *r_in, float eps, int T, int L, int H, const float *const *Wr,
-                                const float *const *bias, int E, int k, int I, const moe_expert_set *routed,
-                                const moe_expert_set *shared, float *r_out, float *logits, int32_t *idx, float *w,
-                                uint16_t *hdec, unsigned *unit_ready, Ctrl *ctrl, cudaStream_t s) {
-  FusedArgs a;
-  const void *fn = nullptr;
-  size_t smem = 0;
-  if (L < 1 || !fused_plan(T, H, E, k, I, routed[0], shared != nullptr, true, a, fn, smem)) {
-    (void)cudaGetLastError();
-    return cudaErrorNotSupported;
-  }
-  for (int l = 1; l < L; ++l)  // one block format for the whole launch
-    if (routed[l].gate.qtype != routed[0].gate.qtype) return cudaErrorNotSupported;
-  a.eps = eps;
-  a.y = r_out;
-  a.logits = logits;
-  a.idx = idx;
-  a.w = w;
-  a.hdec = hdec;
-  a.ready = unit_ready;
-  a.ctrl = ctrl;
-  a.routed = routed[0];
-  a.shared = shared ? shared[0] : routed[0];
-  static thread_local StackLayers sl;  // ~12 KB: kept off the host stack
-  for (int l0 = 0; l0 < L; l0 += kStackMaxL) {
-    const int n = L - l0 < kStackMaxL ? L - l0 : kStackMaxL;
-    sl.n = n;
-    for (int j = 0; j < n; ++j) {
-      sl.Wr[j] = Wr[l0 + j];
-      sl.bias[j] = bias ? bias[l0 + j] : nullptr;
-      sl.routed[j] = routed[l0 + j];
-      sl.shared[j] = shared ? shared[l0 + j] : routed[l0 + j];
-    }
-    // the first layer of a piece reads the stream from r_in (first piece) or r_out (later pieces)
-    a.r_norm = l0 == 0 ? r_in : r_out;
-    a.residual = l0 == 0 ? r_in : r_out;
-    void *args[] = {&a, &sl};
-    cudaError_t e = fused_launch(fn, smem, args, s);
-    if (e != cudaSuccess) return e;
-  }
-  return cudaSuccess;
 }
 
 }  // namespace moe

@@ -324,9 +324,17 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
         if (g >= total_g) break;
         const int s = g % kStagesB, sa = g % kStagesA;
         const uint32_t ph = (uint32_t)(g / kStagesB) & 1u;
-        // codes landed: dequantize into registers first, so that the arithmetic is off the chain
-        // MMA(g - kStagesA) done -> A stage written -> MMA(g)
+        // codes landed; and the MMAs that last read this A stage (stage g - kStagesA) are complete
+        // (both waits come before the arithmetic: the out-of-line slow path of a wait would
+        // otherwise have to save the 32 dequantized registers around its call)
         if (!mbar_wait(full_b(s), ph)) { record_timeout(ctrl, 24); ok = false; break; }
+        if (g >= kStagesA &&
+            !mbar_wait(empty_b((g - kStagesA) % kStagesB), (uint32_t)((g - kStagesA) / kStagesB) & 1u)) {
+          record_timeout(ctrl, 24);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         // this thread's 64 weights of the stage: 16 code bytes (32 for the 4-bit plane)
         const uint8_t *cp = gbase + (sR(s) - base) + crow * SL::kRowCodes + hh * (SL::kRowCodes / 2);
         const uint4 cw = *reinterpret_cast<const uint4 *>(cp);
@@ -354,14 +362,6 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
           dq2_word(cw.z, d1, p + 16);
           dq2_word(cw.w, d1, p + 24);
         }
-        // the MMAs that last read this A stage (stage g - kStagesA) are complete
-        if (g >= kStagesA &&
-            !mbar_wait(empty_b((g - kStagesA) % kStagesB), (uint32_t)((g - kStagesA) / kStagesB) & 1u)) {
-          record_timeout(ctrl, 24);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
         const uint32_t ta = tmem + a_lane + a_col(sa) + 32u * hh;
         tmem_st16(ta, p);
         tmem_st16(ta + 16u, p + 16);
@@ -439,7 +439,7 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
 }
 
 // ---------------------------------------------------------------- tile list
-// Entries (group, first row within the group) for every kBNMax-row (192-row) slice of every
+// Entries (group, first row within the group) for every `slice`-row slice (192 for this kernel) of every
 // non-empty group, ordered longest first: by the slice's row count rounded up to the MMA's N
 // granule of 16, descending (full 192-row slices first, the smallest remainders last). The
 // persistent GEMM deals entries round-robin, so every CTA starts on the heavy tiles and the light
@@ -451,13 +451,14 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
 constexpr int kTileClasses = kBNMax / 16;  // N granules 1..12
 
 __global__ void __launch_bounds__(1024) tile_list_kernel(const int32_t *__restrict__ off, int G, int n_rows,
-                                                         int min_rows, int2 *__restrict__ tiles,
+                                                         int min_rows, int slice, int2 *__restrict__ tiles,
                                                          Ctrl *__restrict__ ctrl) {
+  const int nclass = slice / 16;  // <= kTileClasses
   __shared__ int s_cnt[kTileClasses + 1], s_cur[kTileClasses + 1];
   __shared__ int s_bad;
   const int tid = threadIdx.x;
   if (tid == 0) s_bad = 0;
-  if (tid <= kTileClasses) s_cnt[tid] = 0;
+  if (tid <= nclass) s_cnt[tid] = 0;
   __syncthreads();
   for (int g = tid; g < G; g += blockDim.x)
     if (off[g] < 0 || off[g + 1] < off[g] || off[g + 1] > n_rows) s_bad = 1;
@@ -469,17 +470,17 @@ __global__ void __launch_bounds__(1024) tile_list_kernel(const int32_t *__restri
     }
     return;
   }
-  // size class of a slice with n rows (1..192): ceil(n / 16), 1..kTileClasses
+  // size class of a slice with n rows (1..slice): ceil(n / 16), 1..nclass
   for (int g = tid; g < G; g += blockDim.x) {
     const int n = off[g + 1] - off[g];
     if (n <= min_rows) continue;  // left to the small-group path
-    if (n >= kBNMax) atomicAdd(&s_cnt[kTileClasses], n / kBNMax);
-    if (n % kBNMax) atomicAdd(&s_cnt[(n % kBNMax + 15) / 16], 1);
+    if (n >= slice) atomicAdd(&s_cnt[nclass], n / slice);
+    if (n % slice) atomicAdd(&s_cnt[(n % slice + 15) / 16], 1);
   }
   __syncthreads();
   if (tid == 0) {  // classes in descending order: each class's first position
     int pos = 0;
-    for (int c = kTileClasses; c >= 1; --c) {
+    for (int c = nclass; c >= 1; --c) {
       s_cur[c] = pos;
       pos += s_cnt[c];
     }
@@ -489,12 +490,12 @@ __global__ void __launch_bounds__(1024) tile_list_kernel(const int32_t *__restri
   for (int g = tid; g < G; g += blockDim.x) {
     const int n = off[g + 1] - off[g];
     if (n <= min_rows) continue;
-    const int full = n / kBNMax;
+    const int full = n / slice;
     if (full) {
-      const int p = atomicAdd(&s_cur[kTileClasses], full);
-      for (int j = 0; j < full; ++j) tiles[p + j] = make_int2(g, j * kBNMax);
+      const int p = atomicAdd(&s_cur[nclass], full);
+      for (int j = 0; j < full; ++j) tiles[p + j] = make_int2(g, j * slice);
     }
-    if (n % kBNMax) tiles[atomicAdd(&s_cur[(n % kBNMax + 15) / 16], 1)] = make_int2(g, full * kBNMax);
+    if (n % slice) tiles[atomicAdd(&s_cur[(n % slice + 15) / 16], 1)] = make_int2(g, full * slice);
   }
 }
 
@@ -558,6 +559,16 @@ bool encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dt, int esize, c
   return r == CUDA_SUCCESS;
 }
 
+cudaError_t launch_tile_list(const int32_t *offsets, int n_groups, int n_rows, int slice, int2 *tiles, Ctrl *ctrl,
+                             cudaStream_t s, int min_rows) {
+  if (slice < 16 || slice > kBNMax || slice % 16) return cudaErrorInvalidValue;
+  {
+    KTimer kt_(KID_TILE_LIST, s);
+    tile_list_kernel<<<1, 1024, 0, s>>>(offsets, n_groups, n_rows, min_rows, slice, tiles, ctrl);
+  }
+  return cudaGetLastError();
+}
+
 int gemm_shape_supported(int H, int I) { return (H % 128 == 0 && I % 128 == 0 && H >= 128 && I >= 128) ? 1 : 0; }
 
 cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, int n_rows, int E, int H, int I,
@@ -565,11 +576,7 @@ cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, i
                                uint16_t *out_perm, int2 *tiles, Ctrl *ctrl, cudaStream_t s, int min_rows) {
   const int G = E + (shared ? 1 : 0);
   const moe_expert_set &sh = shared ? *shared : routed;
-  {
-    KTimer kt_(KID_TILE_LIST, s);
-    tile_list_kernel<<<1, 1024, 0, s>>>(offsets, G, n_rows, min_rows, tiles, ctrl);
-  }
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_tile_list(offsets, G, n_rows, kBNMax, tiles, ctrl, s, min_rows);
   if (e != cudaSuccess) return e;
 
   CUtensorMap tx, th, cg, cu, cd, sg, su, sd;
@@ -615,6 +622,34 @@ cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, i
   a.hibits[0][1] = nullptr;
   a.hibits[1][0] = sh.down.hibits;
   a.hibits[1][1] = nullptr;
+  return launch_v2<MODE_DN>(th, cd, cd, sd, sd, a, routed.gate.qtype, s);
+}
+
+cudaError_t launch_grouped_down(const uint16_t *h_perm, const int32_t *offsets, int n_rows, int E, int H, int I,
+                                const moe_expert_set &routed, const moe_expert_set *shared, uint16_t *out_perm,
+                                int2 *tiles, Ctrl *ctrl, cudaStream_t s) {
+  const int G = E + (shared ? 1 : 0);
+  const moe_expert_set &sh = shared ? *shared : routed;
+  cudaError_t e = launch_tile_list(offsets, G, n_rows, kBNMax, tiles, ctrl, s);
+  if (e != cudaSuccess) return e;
+  CUtensorMap th, cd, sd;
+  if (!(encode_tensor_map_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h_perm, I, n_rows, kSubK, kBoxRows,
+                             CU_TENSOR_MAP_SWIZZLE_128B) &&
+        make_code_map(&cd, routed.down, kBM) && make_code_map(&sd, sh.down, kBM)))
+    return cudaErrorInvalidValue;
+  GemmArgs a{};
+  a.offsets = offsets;
+  a.tiles = tiles;
+  a.ctrl = ctrl;
+  a.shared_group = shared ? E : -1;
+  a.out = out_perm;
+  a.ldo = H;
+  a.K = I;
+  a.M = H;
+  a.scales[0][0] = routed.down.scales;
+  a.scales[1][0] = sh.down.scales;
+  a.hibits[0][0] = routed.down.hibits;
+  a.hibits[1][0] = sh.down.hibits;
   return launch_v2<MODE_DN>(th, cd, cd, sd, sd, a, routed.gate.qtype, s);
 }
 

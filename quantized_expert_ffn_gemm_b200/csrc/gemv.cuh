@@ -263,8 +263,10 @@ __device__ __forceinline__ void rows16(const MatView &m, int r0, const __half *x
 
 // stage columns of the activation source into shared memory (fp16, rotated layout). 16-byte
 // loads, several issued before the first store, so the staging costs one memory round trip.
+// returns true when a bf16 source value was beyond the fp16 range (it is staged as +-inf)
 template <bool SRC_BF16>
-__device__ __forceinline__ void stage_x(const void *src, int row0, int mask, int H, __half *xs, int xstride) {
+__device__ __forceinline__ bool stage_x(const void *src, int row0, int mask, int H, __half *xs, int xstride) {
+  bool bad = false;
   const int H8 = H / 8;
   const uint16_t *base = static_cast<const uint16_t *>(src);
   for (int c = 0; c < 8; ++c) {
@@ -289,6 +291,7 @@ __device__ __forceinline__ void stage_x(const void *src, int row0, int mask, int
           for (int q = 0; q < 4; ++q) {
             __half2 h = __floats2half2_rn(__uint_as_float(in[q] << 16), __uint_as_float(in[q] & 0xffff0000u));
             out[q] = *reinterpret_cast<uint32_t *>(&h);
+            bad |= f16x2_inf(out[q]);
           }
           o = make_uint4(out[0], out[1], out[2], out[3]);
         }
@@ -299,6 +302,7 @@ __device__ __forceinline__ void stage_x(const void *src, int row0, int mask, int
       }
     }
   }
+  return bad;
 }
 
 

@@ -264,8 +264,9 @@ perm_scatter_kernel(const int32_t *__restrict__ idx, int P, int k, int E, const 
 // any is converted and stored, and the warp's next source token is read meanwhile
 __global__ void __launch_bounds__(256)
 perm_gather_kernel(const uint16_t *__restrict__ x, int H, const int32_t *__restrict__ src, int P, int rows,
-                   uint16_t *__restrict__ x_perm) {
+                   uint16_t *__restrict__ x_perm, Ctrl *__restrict__ ctrl) {
   const int lane = threadIdx.x & 31, H8 = H >> 3, stride = gridDim.x * 8;
+  bool bad = false;  // an x value beyond the fp16 range
   int r = blockIdx.x * 8 + (threadIdx.x >> 5);
   int t = (r < rows) ? ((r < P) ? src[r] : r - P) : 0;
   for (; r < rows; r += stride) {
@@ -291,12 +292,14 @@ perm_gather_kernel(const uint16_t *__restrict__ x, int H, const int32_t *__restr
         for (int j = 0; j < 4; ++j) {
           __half2 h = __floats2half2_rn(__uint_as_float(in[j] << 16), __uint_as_float(in[j] & 0xffff0000u));
           out[j] = *reinterpret_cast<uint32_t *>(&h);
+          bad |= f16x2_inf(out[j]);
         }
         xd[c] = make_uint4(out[0], out[1], out[2], out[3]);
       }
     }
     t = tn;
   }
+  if (bad) set_device_error(ctrl, MOE_ERR_RANGE, 1);
 }
 
 __global__ void fill_iota_kernel(int32_t *p, int n) {
@@ -341,7 +344,7 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const uint16
   int grid = (int)(want < cap ? want : cap);
   {
     KTimer kt_(KID_PERM_GATHER, s);
-    perm_gather_kernel<<<grid, 256, 0, s>>>(x, H, src, P, rows, x_perm);
+    perm_gather_kernel<<<grid, 256, 0, s>>>(x, H, src, P, rows, x_perm, ctrl);
   }
   return cudaGetLastError();
 }
@@ -353,8 +356,12 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const uint16
 // 8-column chunk and issues the k row loads of it before accumulating them.
 __global__ void __launch_bounds__(256)
 combine_kernel(const uint16_t *__restrict__ out, const int32_t *__restrict__ row_of, const float *__restrict__ w,
-               int T, int k, int H, const uint16_t *__restrict__ shared, const float *residual, float *y) {
+               int T, int k, int H, const uint16_t *__restrict__ shared, const float *residual, float *y,
+               Ctrl *__restrict__ ctrl) {
   const int lane = threadIdx.x & 31, H8 = H >> 3, nseg = (H8 + 31) >> 5;
+  // an expert output outside the fp16 range (an overflowed h gives a non-finite output too): the
+  // grouped GEMM's epilogues store without a check, so the range is checked here, once per value
+  uint32_t bad = 0;
   const long long n_items = (long long)T * nseg;
   for (long long it = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); it < n_items; it += (long long)gridDim.x * 8) {
     const int t = (int)(it / nseg), c = (int)(it % nseg) * 32 + lane;
@@ -387,6 +394,8 @@ combine_kernel(const uint16_t *__restrict__ out, const int32_t *__restrict__ row
           const uint32_t vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
+            // exponent all ones in either half: inf or NaN
+            bad |= ((vv[q] & 0x7c00u) == 0x7c00u) | ((vv[q] & 0x7c000000u) == 0x7c000000u);
             const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&vv[q]));
             acc[2 * q] = fmaf(wj[u], f.x, acc[2 * q]);
             acc[2 * q + 1] = fmaf(wj[u], f.y, acc[2 * q + 1]);
@@ -398,6 +407,7 @@ combine_kernel(const uint16_t *__restrict__ out, const int32_t *__restrict__ row
         const uint32_t vv[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
+          bad |= ((vv[q] & 0x7c00u) == 0x7c00u) | ((vv[q] & 0x7c000000u) == 0x7c000000u);
           const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&vv[q]));
           acc[2 * q] += f.x;
           acc[2 * q + 1] += f.y;
@@ -410,17 +420,18 @@ combine_kernel(const uint16_t *__restrict__ out, const int32_t *__restrict__ row
       }
     }
   }
+  if (bad && ctrl) set_device_error(ctrl, MOE_ERR_RANGE, 8);
 }
 
 cudaError_t launch_combine(const uint16_t *out_perm, const int32_t *row_of, const float *w, int T, int k, int H,
-                           const uint16_t *shared_out, const float *residual, float *y, cudaStream_t s) {
+                           const uint16_t *shared_out, const float *residual, float *y, cudaStream_t s, Ctrl *ctrl) {
   // items of (token, 256-column segment), eight warps per block
   const size_t nseg = ((size_t)(H / 8) + 31) / 32;
   size_t want = ((size_t)T * nseg + 7) / 8, cap = (size_t)num_sms() * 16;
   int grid = (int)(want < cap ? want : cap);
   {
     KTimer kt_(KID_COMBINE, s);
-    combine_kernel<<<grid, 256, 0, s>>>(out_perm, row_of, w, T, k, H, shared_out, residual, y);
+    combine_kernel<<<grid, 256, 0, s>>>(out_perm, row_of, w, T, k, H, shared_out, residual, y, ctrl);
   }
   return cudaGetLastError();
 }

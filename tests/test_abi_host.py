@@ -93,7 +93,7 @@ def test_layer_forward_validation(lib):
     assert _lf(lib, routed=_set(E=511)) == moe.MOE_ERR_INVALID_ARG         # set shape disagrees with desc
     assert _lf(lib, ws=None) == moe.MOE_ERR_WORKSPACE
     assert _lf(lib, wsb=1024) == moe.MOE_ERR_WORKSPACE
-    assert _lf(lib, path=3) == moe.MOE_ERR_INVALID_ARG
+    assert _lf(lib, path=4) == moe.MOE_ERR_INVALID_ARG
     assert _lf(lib, desc=_desc(H=2048, I=192), routed=_set(I=192), path=2) == moe.MOE_ERR_UNSUPPORTED
 
 

@@ -160,7 +160,6 @@ def test_combine_matches_definition():
 @pytest.mark.parametrize("name", ["tiny", "mid", "mid_q3", "mid_q4"])
 @pytest.mark.parametrize("path", [moe.PATH_GEMV, moe.PATH_GEMM, moe.PATH_AUTO])
 def test_expert_ffn_rows(name, path):
-    # AUTO splits the groups: those of at most 32 rows on the GEMV kernels, the rest on the GEMM
     L, (x, Wr, b, routed, shared) = layer_of(name)
     s = L.shape
     idx_ref, _, _, _ = oracle.router_topk(L.x, L.Wr, L.bias, s.k)
@@ -305,3 +304,71 @@ def test_stack_small_full_compare():
     r_out = moe.stack_forward(r0.cuda(), st, ws).cpu().numpy()
     ref, _ = oracle.stack_forward(r0, list(zip(Wrs, [None] * Lyr, rs, ss)), k)
     assert rel_err(r_out, ref) <= Y_TOL
+
+
+# ----------------------------------------------------------------------------- fp16 operand range
+@pytest.mark.parametrize("name,T", [("decode1", 1), ("decode4", 4), ("mid", 300)])
+def test_fp16_range_is_flagged_not_silent(name, T):
+    # The expert contractions take fp16 operands (x, h, expert outputs). Scaled by 300, x stays
+    # inside fp16 but h = silu(x Wg) * (x Wu) grows ~9e4 times and overflows: the call must record
+    # MOE_ERR_RANGE rather than return inf silently. Scaled by 20 (h ~400 times larger) nothing
+    # overflows and the layer matches the oracle.
+    L0, (_, Wr, b, routed, shared) = layer_of(name)
+    s = L0.shape
+    base = synth.make_x(s.seed, T, s.H, stream=500 + T).float()
+    ws = moe.Workspace.for_layer(s.H, s.E, s.k, s.I, s.shared, T)
+    for scale, overflow in ((300.0, True), (20.0, False)):
+        x = (base * scale).to(torch.bfloat16)
+        y, idx, w = moe.layer_forward(x.cuda(), Wr, b, routed, shared, s.k, ws, want_routing=True)
+        code = moe.read_device_error(ws)
+        if overflow:
+            assert code == moe.MOE_ERR_RANGE
+            assert not torch.isfinite(y).all()
+        else:
+            assert code == 0
+            L = synth.LayerInputs(s, x, L0.Wr, L0.bias, L0.routed, L0.shared)
+            check_layer(y.cpu().numpy(), idx.cpu().numpy(), L, range(min(T, 24)), w_gpu=w.cpu().numpy())
+
+
+# ----------------------------------------------------------------------------- int8-activation (MMQ) path
+def test_mmq_expert_ffn_rows_match_the_int8_definition():
+    # MOE_PATH_MMQ quantizes each permuted activation row in 32-value blocks to int8 (the oracle's
+    # quantize_blocks_i8 states the rule) and computes gate/up from exact integer block sums; the
+    # oracle applies the same quantization and evaluates the FFN in fp64 on q * d. The deviation
+    # from the unquantized FFN is the format's own error, printed beside it.
+    L, (x, Wr, b, routed, shared) = layer_of("mid")
+    s = L.shape
+    idx_ref, _, _, _ = oracle.router_topk(L.x, L.Wr, L.bias, s.k)
+    ws = ws_for(L)
+    pm = moe.permute(torch.from_numpy(idx_ref).cuda(), s.E, x, s.shared, ws)
+    n_rows = s.T * s.k + s.T
+    ws2 = moe.Workspace.for_layer(s.H, s.E, 1, s.I, False, n_rows)
+    out = moe.expert_ffn(pm["x_perm"], pm["offsets"], s.E, routed, shared, ws2, path=moe.PATH_MMQ)
+    assert moe.read_device_error(ws2) == 0
+    offs = pm["offsets"].cpu().numpy()
+    xp16 = pm["x_perm"].cpu().view(torch.int16).numpy().view(np.uint16)
+    q, d = oracle.quantize_blocks_i8(xp16)
+    xq = oracle.dequantize_blocks_i8(q, d)
+    xe = pm["x_perm"].cpu().double().numpy()
+    rng = np.random.default_rng(2)
+    sample = np.sort(rng.choice(n_rows, size=96, replace=False))
+    ref = np.zeros((len(sample), s.H))
+    exact = np.zeros((len(sample), s.H))
+    for i, r in enumerate(sample):
+        g = int(np.searchsorted(offs[:s.E + 2], r, side="right") - 1)
+        es, e = (L.shared, 0) if g == s.E else (L.routed, g)
+        ref[i] = oracle.expert_ffn_rows(es, e, xq[r:r + 1])[0]
+        exact[i] = oracle.expert_ffn_rows(es, e, xe[r:r + 1])[0]
+    got = out.cpu().double().numpy()[sample]
+    err = rel_err(got, ref)
+    print(f"MMQ vs its int8 definition {err:.2e}; int8 activations vs exact {rel_err(got, exact):.2e}")
+    assert err <= Y_TOL
+
+
+def test_mmq_rejects_formats_it_does_not_take():
+    L, (x, Wr, b, routed, shared) = layer_of("mid_q3")
+    s = L.shape
+    ws = ws_for(L)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.layer_forward(x, Wr, b, routed, shared, s.k, ws, path=moe.PATH_MMQ)
+    assert ei.value.code == moe.MOE_ERR_UNSUPPORTED

@@ -440,3 +440,29 @@ def test_stack_of_one_hot_layers_matches_hand_composition():
         r = (r + dense_ffn(ks, e, u) + dense_ffn(sh, 0, u)).astype(np.float32).astype(np.float64)
     assert np.allclose(got, r, rtol=1e-9, atol=1e-12)
     assert not np.allclose(got, r0, rtol=1e-3)     # the layers did change the stream
+
+
+# ----------------------------------------------------------------------------- int8 activation blocks
+def test_int8_blocks_hand_worked():
+    # a block whose largest magnitude is 2: d = 2/127, and 127/2 = 63.5 times each value rounds to
+    # the nearest integer, ties to even (0.5 * 63.5 = 31.75 -> 32; 1/127 * 63.5 = 0.5 -> 0)
+    x = np.zeros((1, 64), np.float16)
+    x[0, :6] = [2.0, -2.0, 0.5, -1.0, 1.0 / 127.0, 0.25]
+    q, d = oracle.quantize_blocks_i8(x)
+    assert d[0, 0] == np.float32(2.0) / np.float32(127.0) and d[0, 1] == 0.0   # second block all zero
+    v = np.float32(x[0, 4]) * (np.float32(127.0) / np.float32(2.0))
+    assert q[0, :6].tolist() == [127, -127, 32, -64, int(np.rint(v)), 16]
+    assert (q[0, 32:] == 0).all()
+
+
+def test_int8_blocks_error_bound_and_extremes():
+    rng = np.random.default_rng(44)
+    x = (rng.normal(0, 3, (16, 256))).astype(np.float16)
+    q, d = oracle.quantize_blocks_i8(x)
+    xr = oracle.dequantize_blocks_i8(q, d)
+    err = np.abs(xr - x.astype(np.float64)).reshape(16, 8, 32)
+    assert (err <= d[..., None] * 0.5 * (1 + 1e-5)).all()    # half a step at most (fp32 scale rounding aside)
+    amax_pos = np.abs(x.astype(np.float32)).reshape(16, 8, 32).argmax(-1)
+    qb = np.abs(q.astype(np.int64)).reshape(16, 8, 32)
+    assert (np.take_along_axis(qb, amax_pos[..., None], -1) == 127).all()  # the block maximum maps to +-127
+    assert (qb <= 127).all()
