@@ -1,6 +1,7 @@
 // C-ABI entry points of libmoe_ffn.so (declared in include/moe_ffn.h): argument validation on
 // the host, workspace carving, path selection and kernel launches. No entry point allocates
 // device memory, synchronises (except moe_read_device_error) or aborts.
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -63,6 +64,14 @@ int num_sms() {
     cached[dev] = n;
   }
   return cached[dev];
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char *v = getenv("MOE_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
 }
 
 cudaError_t smem_limit_once_impl(const void *func, size_t bytes) {
@@ -426,7 +435,8 @@ moe_status moe_stack_forward(const float *r_in, int32_t T, int32_t L, const floa
       cudaError_t e = launch_decode_fused(nullptr, r, eps, T, H, Wr[l], bias ? bias[l] : nullptr, E, k, I, routed[l],
                                           hs ? &shared[l] : nullptr, r, r_out, at<float>(ws, LY.logits),
                                           at<int32_t>(ws, LY.idx), at<float>(ws, LY.w), at<uint16_t>(ws, LY.hdec),
-                                          at<unsigned>(ws, LY.units), at<Ctrl>(ws, LY.ctrl), s);
+                                          at<unsigned>(ws, LY.units), at<Ctrl>(ws, LY.ctrl), s,
+                                          l + 1 < L ? Wr[l + 1] : nullptr);
       if (e == cudaSuccess) continue;
       if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge) return cuda_status(e);
       (void)cudaGetLastError();

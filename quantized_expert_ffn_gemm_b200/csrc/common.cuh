@@ -94,6 +94,15 @@ __device__ __forceinline__ void set_device_error(Ctrl *c, int code, int info) {
 __device__ __forceinline__ bool f16_inf(uint16_t b) { return (b & 0x7fffu) == 0x7c00u; }
 __device__ __forceinline__ bool f16x2_inf(uint32_t b) { return f16_inf((uint16_t)b) || f16_inf((uint16_t)(b >> 16)); }
 
+// Programmatic dependent launch. A kernel launched with the programmatic stream-serialization
+// attribute may be scheduled before the previous kernel on its stream has finished, once that
+// kernel's CTAs have all executed pdl_launch_dependents (or exited). pdl_wait returns when the
+// previous kernel has completed and its memory operations are visible, at once when the launch
+// had no such predecessor; a kernel launched that way reads or writes nothing a predecessor may
+// touch before it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
 }
@@ -145,12 +154,13 @@ cudaError_t launch_decode_down(int H, int I, const moe_expert_set &routed, const
 // returns cudaErrorNotSupported when the shape or the device cannot take it (callers fall back).
 // With r_norm != NULL the tokens are x = bf16(RMSNorm_eps(r_norm)) (x unused), bit-identical to
 // launch_rmsnorm followed by the layer. unit_ready: T*k + 1 counters of workspace scratch (the
-// kernel zeroes them itself before use).
+// kernel zeroes them itself before use). next_Wr (optional): the router rows of the layer that
+// follows in a stack, prefetched into L2 during the down phase.
 cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float eps, int T, int H, const float *Wr,
                                 const float *bias, int E, int k, int I, const moe_expert_set &routed,
                                 const moe_expert_set *shared, const float *residual, float *y, float *logits,
                                 int32_t *idx, float *w, uint16_t *hdec, unsigned *unit_ready, Ctrl *ctrl,
-                                cudaStream_t s);
+                                cudaStream_t s, const float *next_Wr = nullptr);
 
 // test hook: a grid barrier that waits for one arrival more than the `ctas` CTAs make, giving up
 // after limit_ns with MOE_ERR_TIMEOUT in the control area
@@ -179,6 +189,8 @@ cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, i
                                uint16_t *out_perm, int2 *tiles, Ctrl *ctrl, cudaStream_t s, int min_rows = 0);
 
 int num_sms();
+// programmatic dependent launches on (default) unless the environment sets MOE_PDL=0
+bool pdl_enabled();
 
 // shape rules every entry point applies: H and I multiples of 64 up to 16384, 1 <= E <= kMaxE,
 // 1 <= k <= min(E, kMaxK); a layer outside them that is still well formed (H, I multiples of 32)

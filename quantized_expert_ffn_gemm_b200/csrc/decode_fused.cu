@@ -68,6 +68,7 @@ struct FusedArgs {
   int T, H, E, k, I, has_shared;
   const float *Wr;
   const float *bias;
+  const float *next_Wr;  // the next layer's router rows (stack), prefetched into L2 during P3, or NULL
   moe_expert_set routed, shared;
   const float *residual;
   float *y;
@@ -321,6 +322,11 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   const unsigned nblk = gridDim.x;
   __shared__ unsigned long long s_base;
   __shared__ volatile int s_abort;
+  // The next launch on the stream (the next layer) may be scheduled now; its CTAs take SMs as this
+  // grid's CTAs leave them. Nothing the previous launch writes (the control words, the workspace,
+  // the tokens) is touched before it has completed.
+  pdl_launch_dependents();
+  pdl_wait();
   if (tid == 0) {  // arrivals of earlier launches: a whole number of grids (before this CTA arrives)
     unsigned long long v;
     asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(&ctrl->bar_arrivals) : "memory");
@@ -818,6 +824,8 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   // This CTA's gate/up items are all consumed (the ring rule of P3 below needs it); no grid
   // barrier: each down unit waits for its own unit's h instead.
   __syncthreads();
+  // in a stack, the next layer's router rows go to L2 now: HBM is otherwise idle in the down phase
+  if (a.next_Wr) prefetch_range(a.next_Wr, (size_t)E * H * 4, (int)blockIdx.x * kFThreads + tid, G * kFThreads);
   // ---------------- P3: down projection + weighted combine (+ residual) for 16 output features per CTA.
   // Piece d of a row block shares its slot with piece d - R. Before waiting on piece d's fill a
   // warp waits until piece d - R is consumed (its last consumer then issues piece d's fill), so
@@ -1066,12 +1074,19 @@ static cudaError_t fused_launch(const void *fn, size_t smem, void **args, cudaSt
   cfg.blockDim = dim3(kFThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
   KTimer kt_(KID_DECODE_FUSED, s);
+  if (pdl_enabled()) {  // may start while the previous kernel on the stream finishes
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelExC(&cfg, fn, args) == cudaSuccess) return cudaSuccess;
+    (void)cudaGetLastError();  // the attribute pair was refused: launch without the overlap
+  }
+  cfg.numAttrs = 1;
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
@@ -1079,7 +1094,7 @@ cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float ep
                                 const float *bias, int E, int k, int I, const moe_expert_set &routed,
                                 const moe_expert_set *shared, const float *residual, float *y, float *logits,
                                 int32_t *idx, float *w, uint16_t *hdec, unsigned *unit_ready, Ctrl *ctrl,
-                                cudaStream_t s) {
+                                cudaStream_t s, const float *next_Wr) {
   FusedArgs a;
   const void *fn = nullptr;
   size_t smem = 0;
@@ -1092,6 +1107,7 @@ cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float ep
   a.eps = eps;
   a.Wr = Wr;
   a.bias = bias;
+  a.next_Wr = next_Wr;
   a.routed = routed;
   a.shared = shared ? *shared : routed;
   a.residual = residual;
