@@ -43,6 +43,7 @@ WORKLOADS = {
     "verify6": dict(shape="verify6", layers=48),
     "decode1_pruned256": dict(shape="decode1_pruned256", layers=48),
     "decode1_q4": dict(shape="decode1_q4", layers=48),
+    "batch32": dict(shape="batch32", layers=48),
     "prefill8k": dict(shape="prefill8k", layers=4),
     "prefill2k_q3": dict(shape="prefill2k_q3", layers=4),
     # the 48-layer stack (RMSNorm before each router, residual stream, prefill-shaped layers with
@@ -52,9 +53,11 @@ WORKLOADS = {
 }
 METRIC = "MoE-layer tokens/s at T=1/4/8192; % of HBM or bf16 tensor-core roofline"
 DEFAULT_STEPS = {"decode1": 4800, "decode4": 4800, "verify6": 4800, "decode1_pruned256": 4800, "decode1_q4": 4800,
+                 "batch32": 960,
                  "prefill8k": 40, "prefill2k_q3": 60, "stack_decode": 256,
                  "stack_prefill": 4}
 DEFAULT_WARMUP = {"decode1": 480, "decode4": 480, "verify6": 480, "decode1_pruned256": 480, "decode1_q4": 480,
+                  "batch32": 96,
                   "prefill8k": 5, "prefill2k_q3": 5, "stack_decode": 16,
                   "stack_prefill": 3}
 
@@ -269,7 +272,8 @@ def run_ours(args, world, rank, local, workload=None, steps=None, warmup=None, l
         xs = [synth.make_x(shape.seed, T, H, stream=replica_x_stream(rank, i)).to(dev) for i in range(n_x)]
         handles = [moe.LayerHandle(Wr, b, rs, ss, k, ws) for (Wr, b, rs, ss) in layers]
 
-        path = {"auto": moe.PATH_AUTO, "gemm": moe.PATH_GEMM, "gemv": moe.PATH_GEMV, "mmq": moe.PATH_MMQ}[args.path]
+        path = {"auto": moe.PATH_AUTO, "gemm": moe.PATH_GEMM, "gemv": moe.PATH_GEMV, "mmq": moe.PATH_MMQ,
+                "mid": moe.PATH_MID}[args.path]
 
         def step(i, x=None, idx_out=None):
             handles[i % n_layers].forward(xs[i % n_x] if x is None else x, y, idx_out=idx_out, path=path)
@@ -329,7 +333,7 @@ def run_ours(args, world, rank, local, workload=None, steps=None, warmup=None, l
     nblk = max(1, min(10 if T <= 8 else 3, K // G))
     if is_stack:
         nblk = 1
-    idx_bufs = [torch.empty(T, k, dtype=torch.int32, device=dev) for _ in range(G)] if (T <= 8 and not is_stack) else None
+    idx_bufs = [torch.empty(T, k, dtype=torch.int32, device=dev) for _ in range(G)] if (T <= 128 and not is_stack) else None
     units_total = 0
     moe.timing_enable(True)
     for bi in range(nblk):
@@ -349,10 +353,11 @@ def run_ours(args, world, rank, local, workload=None, steps=None, warmup=None, l
     Ktl = Kt * lps
     pk = peaks()
 
-    if T <= 8:
+    if T <= 8 or "mid_expert" in kt:
         # decode: HBM bound. With the fused kernel the whole layer is one launch and its algorithmic
         # bytes are the distinct active experts + the fp32 router + x + y; with the separate kernels
-        # the dominant one is the gate/up dequant-GEMV.
+        # the dominant one is the gate/up dequant-GEMV; on the mid-batch path the expert kernel
+        # (every distinct expert's gate/up/down bytes, its partial rows written).
         # `achieved` counts the distinct active experts' packed bytes only (the benchmark spec's metric:
         # "% of HBM on active-expert bytes"); the all-bytes figure adds the fp32 router, x and y.
         gu_b, dn_b = expert_bytes(shape)
@@ -361,6 +366,10 @@ def run_ours(args, world, rank, local, workload=None, steps=None, warmup=None, l
             dom = "decode_fused"
             algo = units_avg * (gu_b + dn_b)
             algo_all = algo + E * H * 4 + T * H * 2 + T * H * 4
+        elif "mid_expert" in kt:
+            dom = "mid_expert"
+            algo = units_avg * (gu_b + dn_b)
+            algo_all = algo + T * H * 2 + (I // 128) * (T * k + (T if shape.shared else 0)) * H * 4
         else:
             dom = "dec_gate_up"
             algo = units_avg * gu_b
@@ -532,8 +541,9 @@ def run_reference(args, world, rank):
 def run_crossover(args):
     """Layer time at small batches through each expert path (the decode-to-prefill crossover):
     T tokens of the decode-shaped layer (H=2048, E=512, top-10, I=512, shared expert, Q2, Zipf(1.1)
-    router bias), weights rotating over 8 layers, CUDA-event device time per call, one JSON line
-    per (T, path). Not a benchmark line of the contract: it informs the AUTO path's switch point."""
+    router bias), weights rotating over 8 layers, CUDA-event device time per call (calls issued one
+    by one, and the same calls replayed from a CUDA graph), one JSON line per (T, path). Not a
+    benchmark line of the contract: it informs the AUTO path's switch points."""
     import quantized_expert_ffn_gemm_b200 as moe
     torch.cuda.set_device(0)
     shape = synth.WORKLOADS["decode1"]
@@ -544,7 +554,7 @@ def run_crossover(args):
     handles = [moe.LayerHandle(Wr, b, rs, ss, k, ws) for (Wr, b, rs, ss) in layers]
     xs = [synth.make_x(shape.seed, Tmax, H, stream=9000 + i).cuda() for i in range(8)]
     y = torch.empty(Tmax, H, dtype=torch.float32, device="cuda")
-    paths = {"auto": moe.PATH_AUTO, "gemv": moe.PATH_GEMV, "gemm": moe.PATH_GEMM}
+    paths = {"auto": moe.PATH_AUTO, "gemv": moe.PATH_GEMV, "gemm": moe.PATH_GEMM, "mid": moe.PATH_MID}
     for T in (1, 2, 4, 5, 6, 8, 12, 16, 24, 32, 48, 64, 96, 128):
         for name, path in paths.items():
             try:
@@ -562,6 +572,21 @@ def run_crossover(args):
             e1.record()
             torch.cuda.synchronize()
             us = e0.elapsed_time(e1) / n * 1e3
+            # the same calls replayed from a CUDA graph (eight layers per graph, eight replays)
+            xg = [xs[i][:T].contiguous() for i in range(8)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(8):
+                    handles[i].forward(xg[i], y[:T], path=path)
+            g.replay()
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(8):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            us_graph = e0.elapsed_time(e1) / 64 * 1e3
+            del g
             # per-kernel device time: the same calls queued behind a sleep kernel, events per launch
             nk = 16
             moe.timing_enable(True)
@@ -571,7 +596,7 @@ def run_crossover(args):
             torch.cuda.synchronize()
             moe.timing_enable(False)
             kt = {kn: round(ms_ / nk * 1e3, 2) for kn, (ms_, _) in sorted(moe.timing_read().items())}
-            print(json.dumps({"T": T, "path": name, "us_per_layer": round(us, 2),
+            print(json.dumps({"T": T, "path": name, "us_per_layer": round(us, 2), "us_per_layer_graph": round(us_graph, 2),
                               "tokens_per_s": round(T / (us * 1e-6), 1), "kernels_us": kt}), flush=True)
     assert moe.read_device_error(ws) == 0
 
@@ -586,7 +611,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="distinct layer weight sets to rotate over (default 48 for decode, 4 for prefill)")
-    ap.add_argument("--path", default="auto", choices=["auto", "gemm", "gemv", "mmq"],
+    ap.add_argument("--path", default="auto", choices=["auto", "gemm", "gemv", "mmq", "mid"],
                     help="expert path of the layer workloads (mmq: int8 activations on tcgen05 kind::i8 for gate/up)")
     ap.add_argument("--no-breakdown", action="store_true",
                     help="time only --workload (by default a single-GPU run of the T=1 decode layer also times "

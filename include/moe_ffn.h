@@ -100,7 +100,13 @@ enum { MOE_Q2 = 2, MOE_Q3 = 3, MOE_Q4 = 4 };
  * block scales applied on the read-back), then the fp16 down GEMM; Q2 weights, H % 256 == 0,
  * I % 128 == 0 (MOE_ERR_UNSUPPORTED otherwise). The int8 activations change the numerics (the
  * oracle's fp64 definition is met within the usual 1e-2 only because the rounding is per block). */
-enum { MOE_PATH_AUTO = 0, MOE_PATH_GEMV = 1, MOE_PATH_GEMM = 2, MOE_PATH_MMQ = 3 };
+/* MOE_PATH_MID (moe_layer_forward and moe_stack_forward only): the mid-batch path for 1..128 tokens
+ * (small verify passes and batches; Strata DETAILS.md, "How it works"). Each selected expert's
+ * tokens are grouped into units of up to 8 straight from the routing (no permuted copy); every
+ * (unit, 128-feature slice) item runs gate/up + SwiGLU and that slice of the down projection into
+ * fp32 partial rows, summed per token in a fixed order. Needs I % 128 == 0 and H <= 4096
+ * (MOE_ERR_UNSUPPORTED otherwise; moe_expert_ffn returns it for this path). */
+enum { MOE_PATH_AUTO = 0, MOE_PATH_GEMV = 1, MOE_PATH_GEMM = 2, MOE_PATH_MMQ = 3, MOE_PATH_MID = 4 };
 
 typedef struct moe_qmat {
   int32_t qtype;            /* MOE_Q2, MOE_Q3 or MOE_Q4 (all matrices of a layer share one) */

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe_ffn.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_ALIGNMENT, MOE_ERR_WORKSPACE = 0, 1, 2, 3
 MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK, MOE_ERR_TIMEOUT, MOE_ERR_RANGE = 4, 5, 6, 7, 8
-PATH_AUTO, PATH_GEMV, PATH_GEMM, PATH_MMQ = 0, 1, 2, 3
+PATH_AUTO, PATH_GEMV, PATH_GEMM, PATH_MMQ, PATH_MID = 0, 1, 2, 3, 4
 Q2, Q3, Q4 = 2, 3, 4
 
 EXPORTED = ["moe_status_string", "moe_workspace_bytes", "moe_workspace_init", "moe_rmsnorm_bf16",

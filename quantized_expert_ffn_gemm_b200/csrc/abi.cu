@@ -36,7 +36,7 @@ const char *const kKernelNames[KID_COUNT] = {
     "router_decode", "router_gemm", "topk", "perm_hist", "perm_scan", "perm_scatter", "perm_fill",
     "perm_gather", "combine", "rmsnorm", "dequant_rows", "dec_units", "dec_gate_up", "dec_down",
     "tile_list", "gemm_gate_up", "gemm_down", "router_split", "router_tc", "decode_fused", "mmq_quant",
-    "mmq_gate_up"};
+    "mmq_gate_up", "mid_plan", "mid_expert", "mid_combine"};
 }  // namespace
 
 void timer_begin(int kid, cudaStream_t s) {
@@ -185,6 +185,13 @@ cudaError_t expert_rows(const uint16_t *xperm, const int32_t *offsets, int rows,
   return e;
 }
 
+// token counts for which AUTO takes the mid-batch path when the fused decode kernel does not take
+// the shape (bench.py --crossover on the decode-shaped layer, calls replayed from a CUDA graph:
+// equal to the separate decode kernels at 8 tokens and slower at 6, 0.80x the grouped GEMM at 12,
+// 0.91x at 16, equal at 24..32, 0.94x at 64; the grouped GEMM is faster from 96 tokens)
+constexpr int kAutoMidLo = 8;
+constexpr int kAutoMidHi = 64;
+
 bool decode_router_fits(int T, int H, int E) {
   return T <= kDecodeMaxT && (size_t)T * (H > E ? H : E) * 4 <= 200 * 1024;
 }
@@ -277,7 +284,8 @@ moe_status moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, int32_
                           uint16_t *out_perm, int32_t path, void *ws, size_t ws_bytes, void *stream) {
   moe_status st = shape_status(H, E, 1, I);
   if (st != MOE_OK) return st;
-  if (n_rows < 0 || path < 0 || path > 3) return MOE_ERR_INVALID_ARG;
+  if (n_rows < 0 || path < 0 || path > 4) return MOE_ERR_INVALID_ARG;
+  if (path == MOE_PATH_MID) return MOE_ERR_UNSUPPORTED;  // the mid-batch path works from the routing
   if ((st = check_set(routed, E, H, I)) != MOE_OK) return st;
   if (shared_opt && (st = check_set(shared_opt, 1, H, I)) != MOE_OK) return st;
   if (n_rows == 0) return MOE_OK;
@@ -322,7 +330,7 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
   const int H = desc->H, E = desc->E, k = desc->k, I = desc->I, hs = desc->has_shared ? 1 : 0;
   moe_status st = shape_status(H, E, k, I);
   if (st != MOE_OK) return st;
-  if (T < 0 || path < 0 || path > 3) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || path < 0 || path > 4) return MOE_ERR_INVALID_ARG;
   if ((st = check_set(routed, E, H, I)) != MOE_OK) return st;
   if (hs && (st = check_set(shared_opt, 1, H, I)) != MOE_OK) return st;
   if (T == 0) return MOE_OK;
@@ -338,6 +346,12 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
   const bool gemm_ok = gemm_shape_supported(H, I) != 0;
   if (path == MOE_PATH_GEMM && !gemm_ok) return MOE_ERR_UNSUPPORTED;
   if (path == MOE_PATH_MMQ && !(gemm_ok && mmq_shape_supported(H, I, routed->gate.qtype))) return MOE_ERR_UNSUPPORTED;
+  const bool mid_ok = mid_shape_supported(T, H, E, I);
+  if (path == MOE_PATH_MID && !mid_ok) return MOE_ERR_UNSUPPORTED;
+  const bool fused_fits = path == MOE_PATH_AUTO && T <= kDecodeMaxT && decode_router_fits(T, H, E) &&
+                          decode_fused_fits(T, H, E, k, I, *routed, hs != 0);
+  const bool mid = path == MOE_PATH_MID ||
+                   (path == MOE_PATH_AUTO && !fused_fits && mid_ok && T >= kAutoMidLo && T <= kAutoMidHi);
 
   cudaStream_t s = (cudaStream_t)stream;
   Ctrl *ctrl = at<Ctrl>(ws, L.ctrl);
@@ -350,7 +364,8 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
   // decode path (distinct experts' weights read once, tokens as MMA columns) up to 8 tokens: at
   // T = 5..8 it takes about half the time of the grouped GEMM, whose 16-row tiles are bound by MMA
   // issue (measured by bench.py --crossover)
-  const bool decode = (T <= kDecodeMaxT) && path != MOE_PATH_GEMM && path != MOE_PATH_MMQ && decode_router_fits(T, H, E);
+  const bool decode = (T <= kDecodeMaxT) && !mid && path != MOE_PATH_GEMM && path != MOE_PATH_MMQ &&
+                      decode_router_fits(T, H, E);
   if (decode) {
     DecUnit *units = at<DecUnit>(ws, L.units);
     uint16_t *hdec = at<uint16_t>(ws, L.hdec);
@@ -381,6 +396,11 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
       e = launch_router_decode(x, T, H, Wr, bias, E, k, idx, w, logits, 0, 0, at<DecUnit>(ws, L.units), ctrl, s);
     else
       e = launch_router_prefill(x, T, H, Wr, bias, E, k, idx, w, logits, at<uint16_t>(ws, L.wsplit), ctrl, s);
+    if (mid) {
+      if (e == cudaSuccess)
+        e = launch_mid_ffn(x, T, H, E, k, I, idx, w, *routed, sh, residual_opt, y, at<MidUnit>(ws, L.units), row_of,
+                           src, at<float>(ws, L.mid), ctrl, s);  // src: the partial rows' tokens
+    } else {
     if (e == cudaSuccess)
       e = launch_permute(idx, T, k, E, x, H, hs, counts, offsets, row_of, src, xperm, at<int32_t>(ws, L.hist), ctrl,
                          s);
@@ -390,6 +410,7 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
                       gemm_ok, at<int8_t>(ws, L.operm), at<float>(ws, L.dx));  // int8 rows: out_perm's region, free until the down GEMM
     if (e == cudaSuccess)
       e = launch_combine(operm, row_of, w, T, k, H, hs ? operm + (size_t)P * H : nullptr, residual_opt, y, s, ctrl);
+    }
   }
   if (e == cudaSuccess && idx_out_opt)
     e = cudaMemcpyAsync(idx_out_opt, idx, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s);

@@ -28,7 +28,8 @@ struct Ctrl {
   int n_units;              // decode: number of (expert, token-set) units built by the router
   int n_tiles;              // prefill: number of (group, row-tile) entries in the tile list
   unsigned long long bar_arrivals;  // fused decode: grid barrier arrivals (every launch adds 2 x grid)
-  int pad1[20];
+  int mid_pairs;            // mid-batch path: routed (token, slot) pairs with a valid expert
+  int pad1[19];
 };
 static_assert(sizeof(Ctrl) == 128, "control area is 128 bytes");
 
@@ -43,10 +44,28 @@ struct DecUnit {
   float w[8];
 };
 
+// A mid-batch unit: one expert applied to up to kMidNT tokens (MMA column tiles of 8), partial rows
+// row0 .. row0 + ncol - 1, whose tokens are listed in row_tok (so no permuted copy of the
+// activations is needed).
+struct MidUnit {
+  int expert;
+  int set;   // 0 routed, 1 shared
+  int ncol;  // 1..kMidNT
+  int row0;
+  int pad[8];
+};
+static_assert(sizeof(MidUnit) == sizeof(DecUnit), "mid units share the decode units' workspace region");
+
+constexpr int kMidFS = 128;   // features per mid-batch work item (one 128-wide half step of a down row)
+constexpr int kMidMaxT = 128; // tokens the mid-batch path takes
+constexpr int kMidMaxH = 4096;
+// tokens per mid-batch unit: four MMA column tiles while they fit in shared memory
+__host__ __device__ constexpr int mid_unit_tokens(int H) { return H <= 2048 ? 32 : 16; }
+
 // ---------------------------------------------------------------- workspace layout
 struct WsLayout {
   size_t ctrl, logits, idx, w, hist, units, hdec, counts, offsets, row_of, src, xperm, hperm, operm, u16, tiles, wsplit,
-      dx, total;
+      dx, mid, total;
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -80,6 +99,10 @@ inline WsLayout ws_layout(int H, int E, int k, int I, int has_shared, int T) {
   L.tiles = take((rows / 16 + (size_t)E + 4) * 8);
   L.wsplit = take((size_t)E * 3 * H * 2);
   L.dx = take(rows * (size_t)(H / 32) * 4);  // int8-activation path: one scale per 32-value block
+  {  // mid-batch path: fp32 partial outputs [I / kMidFS slices][rows][H], for up to kMidMaxT tokens
+    const size_t tm = (size_t)(T < kMidMaxT ? T : kMidMaxT);
+    L.mid = take(I % kMidFS == 0 ? (size_t)(I / kMidFS) * tm * (size_t)(k + has_shared) * H * 4 : 0);
+  }
   L.total = off;
   return L;
 }
@@ -102,6 +125,25 @@ __device__ __forceinline__ bool f16x2_inf(uint32_t b) { return f16_inf((uint16_t
 // touch before it.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+bool pdl_enabled();
+
+// launch a kernel that calls pdl_wait() before touching anything an earlier kernel on the stream
+// writes, with programmatic stream serialization when enabled
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
@@ -162,6 +204,17 @@ cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float ep
                                 int32_t *idx, float *w, uint16_t *hdec, unsigned *unit_ready, Ctrl *ctrl,
                                 cudaStream_t s, const float *next_Wr = nullptr);
 
+// mid-batch path (about 6..128 tokens; I % kMidFS == 0): units of <= 8 tokens per selected expert
+// built from the routing (no permutation), items (unit, kMidFS-feature slice) that run gate/up,
+// SwiGLU and their slice of the down projection into fp32 partial rows, then a fixed-order combine
+bool mid_shape_supported(int T, int H, int E, int I);
+cudaError_t launch_mid_ffn(const uint16_t *x, int T, int H, int E, int k, int I, const int32_t *idx, const float *w,
+                           const moe_expert_set &routed, const moe_expert_set *shared, const float *residual, float *y,
+                           MidUnit *units, int32_t *row_of, int32_t *row_tok, float *part, Ctrl *ctrl, cudaStream_t s);
+
+// whether launch_decode_fused takes this shape on the current device
+bool decode_fused_fits(int T, int H, int E, int k, int I, const moe_expert_set &routed, bool has_shared);
+
 // test hook: a grid barrier that waits for one arrival more than the `ctas` CTAs make, giving up
 // after limit_ns with MOE_ERR_TIMEOUT in the control area
 cudaError_t launch_barrier_starve(Ctrl *ctrl, int ctas, uint64_t limit_ns, cudaStream_t s);
@@ -189,8 +242,7 @@ cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, i
                                uint16_t *out_perm, int2 *tiles, Ctrl *ctrl, cudaStream_t s, int min_rows = 0);
 
 int num_sms();
-// programmatic dependent launches on (default) unless the environment sets MOE_PDL=0
-bool pdl_enabled();
+// (pdl_enabled: programmatic dependent launches are on unless the environment sets MOE_PDL=0)
 
 // shape rules every entry point applies: H and I multiples of 64 up to 16384, 1 <= E <= kMaxE,
 // 1 <= k <= min(E, kMaxK); a layer outside them that is still well formed (H, I multiples of 32)
@@ -211,7 +263,7 @@ enum KernelId {
   KID_ROUTER_DECODE = 0, KID_ROUTER_GEMM, KID_TOPK, KID_PERM_HIST, KID_PERM_SCAN, KID_PERM_SCATTER, KID_PERM_FILL,
   KID_PERM_GATHER, KID_COMBINE, KID_RMSNORM, KID_DEQUANT_ROWS, KID_DEC_UNITS, KID_DEC_GATE_UP, KID_DEC_DOWN,
   KID_TILE_LIST, KID_GEMM_GATE_UP, KID_GEMM_DOWN, KID_ROUTER_SPLIT, KID_ROUTER_TC, KID_DECODE_FUSED, KID_MMQ_QUANT,
-  KID_MMQ_GATE_UP, KID_COUNT
+  KID_MMQ_GATE_UP, KID_MID_PLAN, KID_MID_EXPERT, KID_MID_COMBINE, KID_COUNT
 };
 void timer_begin(int kid, cudaStream_t s);
 void timer_end(int kid, cudaStream_t s);

@@ -45,6 +45,9 @@
 #include "tc.cuh"
 #include "topk.cuh"
 
+#include <mutex>
+#include <vector>
+
 namespace moe {
 
 namespace {
@@ -1066,6 +1069,33 @@ static bool fused_plan(int T, int H, int E, int k, int I, const moe_expert_set &
   a.dpu = dpu;
   smem = L.total;
   return true;
+}
+
+bool decode_fused_fits(int T, int H, int E, int k, int I, const moe_expert_set &routed, bool has_shared) {
+  // answers are kept per (device, shape): the plan queries the occupancy calculator
+  struct Seen {
+    int dev, T, H, E, k, I, qt, sh;
+    bool ok;
+  };
+  static std::mutex mu;
+  static std::vector<Seen> seen;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const int qt = routed.gate.qtype, sh = has_shared ? 1 : 0;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (const Seen &q : seen)
+      if (q.dev == dev && q.T == T && q.H == H && q.E == E && q.k == k && q.I == I && q.qt == qt && q.sh == sh)
+        return q.ok;
+  }
+  FusedArgs a;
+  const void *fn = nullptr;
+  size_t smem = 0;
+  const bool ok = fused_plan(T, H, E, k, I, routed, has_shared, a, fn, smem);
+  if (!ok) (void)cudaGetLastError();
+  std::lock_guard<std::mutex> lk(mu);
+  if (seen.size() < 4096) seen.push_back({dev, T, H, E, k, I, qt, sh, ok});
+  return ok;
 }
 
 static cudaError_t fused_launch(const void *fn, size_t smem, void **args, cudaStream_t s) {

@@ -108,6 +108,31 @@ __device__ __forceinline__ void load_step(StepFrag &f, const MatView &m, int r0,
   }
 }
 
+// load_step with the two MMA row halves from different matrices: MMA row g is row ra of ma and
+// MMA row g+8 is row rb of mb (gate row and up row of one feature), both for lane group g
+template <int QT>
+__device__ __forceinline__ void load_step_pair(StepFrag &f, const MatView &ma, int ra, const MatView &mb, int rb,
+                                               int step, bool valid) {
+  const int lane = threadIdx.x & 31, t = lane & 3;
+  const int k0 = step * kStepK + 64 * t;
+  const bool ok = valid && k0 < ma.K;
+  const size_t rs = (size_t)code_row_bytes(QT, ma.K), ss = (size_t)ma.K / 32, hs = (size_t)ma.K / 8;
+  const size_t co = (size_t)code_row_bytes(QT, k0);
+  const uint4 z4 = make_uint4(0, 0, 0, 0);
+  f.w0 = ok ? __ldcs(reinterpret_cast<const uint4 *>(ma.codes + (size_t)ra * rs + co)) : z4;
+  f.w1 = ok ? __ldcs(reinterpret_cast<const uint4 *>(mb.codes + (size_t)rb * rs + co)) : z4;
+  if (QT == 4) {
+    f.w0b = ok ? __ldcs(reinterpret_cast<const uint4 *>(ma.codes + (size_t)ra * rs + co) + 1) : z4;
+    f.w1b = ok ? __ldcs(reinterpret_cast<const uint4 *>(mb.codes + (size_t)rb * rs + co) + 1) : z4;
+  }
+  f.d0 = ok ? __ldcs(reinterpret_cast<const uint32_t *>(ma.scales + (size_t)ra * ss + k0 / 32)) : 0u;
+  f.d1 = ok ? __ldcs(reinterpret_cast<const uint32_t *>(mb.scales + (size_t)rb * ss + k0 / 32)) : 0u;
+  if (QT == 3) {
+    f.h0 = ok ? __ldcs(reinterpret_cast<const uint2 *>(ma.hibits + (size_t)ra * hs + k0 / 8)) : make_uint2(0, 0);
+    f.h1 = ok ? __ldcs(reinterpret_cast<const uint2 *>(mb.hibits + (size_t)rb * hs + k0 / 8)) : make_uint2(0, 0);
+  }
+}
+
 // dequantize the fragment (zero codes with zero scales give zero weights) and run the step's 16
 // MMAs; B fragments come from the lane's column in shared memory when `bok`, else zero
 template <int QT>
@@ -230,6 +255,32 @@ __device__ __forceinline__ void mma_half_step(float acc[4], float acc2[4], const
   }
 }
 
+// a lane's HalfFrag straight from global memory: rows r0+g and r0+g+8 of m, the 32-weight block
+// starting at K offset kk (a multiple of 32)
+template <int QT>
+__device__ __forceinline__ void load_half(HalfFrag &f, const MatView &m, int r0, int kk) {
+  const int g = (threadIdx.x & 31) >> 2;
+  const size_t rs = (size_t)code_row_bytes(QT, m.K), ss = (size_t)m.K / 32, hs = (size_t)m.K / 8;
+  const size_t ra = (size_t)(r0 + g), rb = ra + 8;
+  if (QT == 4) {
+    const uint4 c0 = __ldcs(reinterpret_cast<const uint4 *>(m.codes + ra * rs + kk / 2));
+    const uint4 c1 = __ldcs(reinterpret_cast<const uint4 *>(m.codes + rb * rs + kk / 2));
+    f.w0 = make_uint2(c0.x, c0.y);
+    f.w0b = make_uint2(c0.z, c0.w);
+    f.w1 = make_uint2(c1.x, c1.y);
+    f.w1b = make_uint2(c1.z, c1.w);
+  } else {
+    f.w0 = __ldcs(reinterpret_cast<const uint2 *>(m.codes + ra * rs + kk / 4));
+    f.w1 = __ldcs(reinterpret_cast<const uint2 *>(m.codes + rb * rs + kk / 4));
+  }
+  f.d0 = __ldcs(m.scales + ra * ss + kk / 32);
+  f.d1 = __ldcs(m.scales + rb * ss + kk / 32);
+  if (QT == 3) {
+    f.h0 = __ldcs(reinterpret_cast<const uint32_t *>(m.hibits + ra * hs + kk / 8));
+    f.h1 = __ldcs(reinterpret_cast<const uint32_t *>(m.hibits + rb * hs + kk / 8));
+  }
+}
+
 // acc += W[r0..r0+15, steps s0..s0+NS-1] * X^T; all of the batch's loads are issued first
 template <int QT, int NS>
 __device__ __forceinline__ void rows16_batch(const MatView &m, int r0, int s0, int nsteps, const __half *xcol,
@@ -305,5 +356,37 @@ __device__ __forceinline__ bool stage_x(const void *src, int row0, int mask, int
   return bad;
 }
 
+// stage_x for an arbitrary token per column: column c < ncol is row tok[c] of the bf16 source
+__device__ __forceinline__ bool stage_x_tokens(const uint16_t *src, const int *tok, int ncol, int H, __half *xs,
+                                               int xstride) {
+  bool bad = false;
+  const int H8 = H / 8, n = ncol * H8;
+  for (int i0 = threadIdx.x; i0 < n; i0 += 4 * blockDim.x) {
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = i0 + j * blockDim.x;
+      v[j] = (i < n) ? __ldg(reinterpret_cast<const uint4 *>(src + (size_t)tok[i / H8] * H) + i % H8)
+                     : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = i0 + j * blockDim.x;
+      if (i >= n) break;
+      const uint32_t in[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+      uint32_t out[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        __half2 h = __floats2half2_rn(__uint_as_float(in[q] << 16), __uint_as_float(in[q] & 0xffff0000u));
+        out[q] = *reinterpret_cast<uint32_t *>(&h);
+        bad |= f16x2_inf(out[q]);
+      }
+      uint2 *d = reinterpret_cast<uint2 *>(xs + (size_t)(i / H8) * xstride + xs_pos(8 * (i % H8)));
+      d[0] = make_uint2(out[0], out[1]);
+      d[1] = make_uint2(out[2], out[3]);
+    }
+  }
+  return bad;
+}
 
 }  // namespace moe

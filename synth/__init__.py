@@ -264,6 +264,8 @@ WORKLOADS = {
     "prefill2k_q3": LayerShape("prefill2k_q3", 2048, 2048, 512, 10, 512, Q3, False, 1.2),
     # the decode layer with 4-bit weights (the Q4 stand-in), otherwise decode1
     "decode1_q4": LayerShape("decode1_q4", 1, 2048, 512, 10, 512, Q4, True, 1.1),
+    # a small batch of 32 tokens through the decode layer (between decode and prefill)
+    "batch32": LayerShape("batch32", 32, 2048, 512, 10, 512, Q2, True, 1.1),
 }
 
 # 48-layer stack: RMSNorm (eps 1e-6) before each router, residual add, config-3 shaped layers

@@ -93,7 +93,9 @@ def test_layer_forward_validation(lib):
     assert _lf(lib, routed=_set(E=511)) == moe.MOE_ERR_INVALID_ARG         # set shape disagrees with desc
     assert _lf(lib, ws=None) == moe.MOE_ERR_WORKSPACE
     assert _lf(lib, wsb=1024) == moe.MOE_ERR_WORKSPACE
-    assert _lf(lib, path=4) == moe.MOE_ERR_INVALID_ARG
+    assert _lf(lib, path=5) == moe.MOE_ERR_INVALID_ARG
+    assert _lf(lib, desc=_desc(H=2048, I=192), routed=_set(I=192), path=4) == moe.MOE_ERR_UNSUPPORTED  # mid: I % 128
+    assert _lf(lib, T=129, path=4) == moe.MOE_ERR_UNSUPPORTED               # mid: at most 128 tokens
     assert _lf(lib, desc=_desc(H=2048, I=192), routed=_set(I=192), path=2) == moe.MOE_ERR_UNSUPPORTED
 
 
