@@ -54,8 +54,9 @@ namespace {
 
 constexpr int kFWarps = 16;
 constexpr int kFThreads = kFWarps * 32;
-constexpr int kFSlots = 64;                 // h columns (token, expert) of a step staged for the down phase
+constexpr int kFSlots = 96;                 // h columns (token, expert) of a step staged for the down phase
 constexpr int kFMaxUnits = kFSlots + 1;
+constexpr int kPairsPerLane = kFSlots / 32; // (token, slot) pairs per lane of the unit-list warp
 constexpr int kFMaxRing = 16;               // shared-memory slots for weight copies
 constexpr int kFMaxE = 512;                 // experts the fused kernel takes
 constexpr int kFSmemMax = 226 * 1024;       // dynamic shared memory (a little is left for static)
@@ -629,25 +630,35 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       __syncthreads();
     }
     if (warp == 0) {
-      // units: the distinct experts of the P = T*k (< 64) selections in order of first
+      // units: the distinct experts of the P = T*k (<= kFSlots) selections in order of first
       // appearance (token-major), then the shared expert. Pair p leads its unit when it is the
       // first pair to choose its expert (one token's k experts are distinct, so at T = 1 every
       // pair leads); a leader's unit number is the count of leaders before it.
-      int fp[2];
-      bool lead[2];
+      int fp[kPairsPerLane];
+      bool lead[kPairsPerLane];
+      unsigned bl[kPairsPerLane];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
+      for (int hh = 0; hh < kPairsPerLane; ++hh) {
         const int p = lane + 32 * hh;
         fp[hh] = (p < P) ? (T > 1 ? s_firstof[s_idx[p]] : p) : p;
         lead[hh] = (p < P) && fp[hh] == p;
+        bl[hh] = __ballot_sync(0xffffffffu, lead[hh]);
       }
-      const unsigned b0 = __ballot_sync(0xffffffffu, lead[0]), b1 = __ballot_sync(0xffffffffu, lead[1]);
-      const int nr = __popc(b0) + __popc(b1);
+      int nr = 0;
+#pragma unroll
+      for (int hh = 0; hh < kPairsPerLane; ++hh) nr += __popc(bl[hh]);
       auto unit_of = [&](int q) {
-        return q < 32 ? __popc(b0 & ((1u << q) - 1u)) : __popc(b0) + __popc(b1 & ((1u << (q - 32)) - 1u));
+        int n = 0;
+#pragma unroll
+        for (int hh = 0; hh < kPairsPerLane; ++hh) {
+          const int lo = 32 * hh;
+          if (q >= lo + 32) n += __popc(bl[hh]);
+          else if (q > lo) n += __popc(bl[hh] & ((1u << (q - lo)) - 1u));
+        }
+        return n;
       };
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
+      for (int hh = 0; hh < kPairsPerLane; ++hh) {
         const int p = lane + 32 * hh;
         if (lead[hh]) {
           DecUnit &d = su[unit_of(p)];
@@ -671,7 +682,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       __syncwarp();
       // every (unit, token) is one pair: an expert appears at most once per token
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
+      for (int hh = 0; hh < kPairsPerLane; ++hh) {
         const int p = lane + 32 * hh;
         if (p < P) {
           DecUnit &d = su[unit_of(fp[hh])];
