@@ -278,14 +278,15 @@ const char *moe_kernel_name(int32_t kernel);
  * clear it. */
 moe_status moe_read_device_error(void *ws, int32_t *code, void *stream);
 
-/* Test hook for the failure path of the device-side waits. Launches two CTAs that arrive at the
- * grid barrier the fused decode kernel uses and then wait for one arrival more than they made;
- * the wait gives up after limit_ms (1..2000) and records MOE_ERR_TIMEOUT in the workspace error
- * word (read and clear it with moe_read_device_error). Nothing traps and the context stays
- * usable; each CTA takes its own arrival back after giving up, so the workspace serves the next
- * call unchanged. ws: any initialised workspace (at least its 128-byte control area), 16-byte
- * aligned; errors: MOE_ERR_WORKSPACE / MOE_ERR_ALIGNMENT / MOE_ERR_INVALID_ARG on the host. */
-moe_status moe_test_barrier_timeout(void *ws, size_t ws_bytes, int32_t limit_ms, void *stream);
+/* Test hook for the failure path of the device-side waits. Launches one warp that waits, with the
+ * bounded wait the fused decode kernel uses for its exchanged router logits, for a logit word
+ * whose launch tag no launch writes; every lane gives up after limit_ms (1..2000) and
+ * MOE_ERR_TIMEOUT is recorded in the workspace error word (read and clear it with
+ * moe_read_device_error). Nothing traps, the context stays usable and nothing but the error word
+ * is written, so the workspace serves the next call unchanged. ws: an initialised workspace of at
+ * least moe_workspace_bytes(desc, 1) bytes for some layer (its control area), 16-byte aligned;
+ * errors: MOE_ERR_WORKSPACE / MOE_ERR_ALIGNMENT / MOE_ERR_INVALID_ARG on the host. */
+moe_status moe_test_wait_timeout(void *ws, size_t ws_bytes, int32_t limit_ms, void *stream);
 
 #ifdef __cplusplus
 }

@@ -27,7 +27,7 @@ EXPORTED = ["moe_status_string", "moe_workspace_bytes", "moe_workspace_init", "m
             "moe_router_topk", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
             "moe_stack_forward", "moe_dequant_rows", "moe_read_device_error", "moe_timing_enable",
             "moe_timing_read", "moe_kernel_count", "moe_kernel_name", "moe_router_topk_static",
-            "moe_test_barrier_timeout"]
+            "moe_test_wait_timeout"]
 
 
 class MoeError(RuntimeError):
@@ -268,11 +268,11 @@ def dequant_rows(m, expert: int, row0: int, nrows: int):
     return f32, f16
 
 
-def test_barrier_timeout(ws: Workspace, limit_ms: int = 50):
-    """moe_test_barrier_timeout: make the fused kernel's grid barrier wait for an arrival that never
-    comes; the wait gives up after limit_ms and MOE_ERR_TIMEOUT lands in the workspace error word."""
-    _check("moe_test_barrier_timeout", lib().moe_test_barrier_timeout(ws.ptr, ws.size,
-                                                                      int(limit_ms), _stream()))
+def test_wait_timeout(ws: Workspace, limit_ms: int = 50):
+    """moe_test_wait_timeout: make the fused kernel's logit-exchange wait poll for a tag that no
+    launch writes; the wait gives up after limit_ms and MOE_ERR_TIMEOUT lands in the workspace error
+    word."""
+    _check("moe_test_wait_timeout", lib().moe_test_wait_timeout(ws.ptr, ws.size, int(limit_ms), _stream()))
 
 
 def read_device_error(ws: Workspace) -> int:

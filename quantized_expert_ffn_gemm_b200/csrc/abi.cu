@@ -224,7 +224,10 @@ moe_status moe_workspace_init(void *ws, size_t ws_bytes, void *stream) {
   if (!ws) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < sizeof(Ctrl)) return MOE_ERR_WORKSPACE;
   if (!aligned16(ws)) return MOE_ERR_ALIGNMENT;
-  return cuda_status(cudaMemsetAsync(ws, 0, sizeof(Ctrl), (cudaStream_t)stream));
+  // the control block and the fused decode kernel's exchange area behind it (a smaller buffer
+  // serves no layer call; its control block is still cleared)
+  return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes < kControlBytes ? ws_bytes : kControlBytes,
+                                     (cudaStream_t)stream));
 }
 
 moe_status moe_rmsnorm_bf16(const float *r, int32_t T, int32_t H, float eps, uint16_t *u, void *stream) {
@@ -374,8 +377,8 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
     // does not take): separate router / gate-up / down kernels
     e = cudaErrorNotSupported;
     if (path == MOE_PATH_AUTO) {
-      e = launch_decode_fused(x, nullptr, 0.0f, T, H, Wr, bias, E, k, I, *routed, sh, residual_opt, y, logits, idx, w,
-                              hdec, reinterpret_cast<unsigned *>(units), ctrl, s);
+      e = launch_decode_fused(x, nullptr, 0.0f, T, H, Wr, bias, E, k, I, *routed, sh, residual_opt, y, idx, w, hdec,
+                              ctrl, s);
       if (e == cudaErrorCooperativeLaunchTooLarge) {
         (void)cudaGetLastError();
         e = cudaErrorNotSupported;
@@ -454,9 +457,8 @@ moe_status moe_stack_forward(const float *r_in, int32_t T, int32_t L, const floa
     const float *r = (l == 0) ? r_in : r_out;
     if (fused) {
       cudaError_t e = launch_decode_fused(nullptr, r, eps, T, H, Wr[l], bias ? bias[l] : nullptr, E, k, I, routed[l],
-                                          hs ? &shared[l] : nullptr, r, r_out, at<float>(ws, LY.logits),
-                                          at<int32_t>(ws, LY.idx), at<float>(ws, LY.w), at<uint16_t>(ws, LY.hdec),
-                                          at<unsigned>(ws, LY.units), at<Ctrl>(ws, LY.ctrl), s,
+                                          hs ? &shared[l] : nullptr, r, r_out, at<int32_t>(ws, LY.idx),
+                                          at<float>(ws, LY.w), at<uint16_t>(ws, LY.hdec), at<Ctrl>(ws, LY.ctrl), s,
                                           l + 1 < L ? Wr[l + 1] : nullptr);
       if (e == cudaSuccess) continue;
       if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge) return cuda_status(e);
@@ -520,13 +522,12 @@ const char *moe_kernel_name(int32_t kernel) {
   return (kernel >= 0 && kernel < KID_COUNT) ? kKernelNames[kernel] : nullptr;
 }
 
-moe_status moe_test_barrier_timeout(void *ws, size_t ws_bytes, int32_t limit_ms, void *stream) {
+moe_status moe_test_wait_timeout(void *ws, size_t ws_bytes, int32_t limit_ms, void *stream) {
   if (!ws) return MOE_ERR_WORKSPACE;
-  if (ws_bytes < sizeof(Ctrl)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < kControlBytes) return MOE_ERR_WORKSPACE;
   if (!aligned16(ws)) return MOE_ERR_ALIGNMENT;
   if (limit_ms < 1 || limit_ms > 2000) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_barrier_starve(static_cast<Ctrl *>(ws), 2, (uint64_t)limit_ms * 1000000ull,
-                                           (cudaStream_t)stream));
+  return cuda_status(launch_wait_starve(static_cast<Ctrl *>(ws), (uint64_t)limit_ms * 1000000ull, (cudaStream_t)stream));
 }
 
 moe_status moe_read_device_error(void *ws, int32_t *code, void *stream) {

@@ -27,11 +27,26 @@ struct Ctrl {
   unsigned gemm_ticket[4];  // tile counters of the persistent grouped GEMM
   int n_units;              // decode: number of (expert, token-set) units built by the router
   int n_tiles;              // prefill: number of (group, row-tile) entries in the tile list
-  unsigned long long bar_arrivals;  // fused decode: grid barrier arrivals (every launch adds 2 x grid)
+  unsigned long long pad_u64;
   int mid_pairs;            // mid-batch path: routed (token, slot) pairs with a valid expert
-  int pad1[19];
+  int pad2;
+  unsigned long long fused_launches;  // fused decode: CTAs started (every launch adds its grid size)
+  int pad1[16];
 };
-static_assert(sizeof(Ctrl) == 128, "control area is 128 bytes");
+static_assert(sizeof(Ctrl) == 128, "control block is 128 bytes");
+
+// The fused decode kernel's exchange area, the rest of the control area (zeroed once by
+// moe_workspace_init and used by that kernel only): router logits as (launch tag << 32 | fp32 bits)
+// words that readers poll for their own launch's tag, and per-unit readiness counters in two sets
+// used by alternate launches (a launch zeroes the other set for the next one).
+constexpr int kFusedMaxE = 512;   // experts the fused decode kernel takes
+constexpr int kFusedMaxUnits = 128;
+struct FusedSync {
+  unsigned long long logit[kDecodeMaxT * kFusedMaxE];
+  unsigned ready[2][kFusedMaxUnits];
+};
+constexpr size_t kCtrlStride = 256;  // the control block, then the exchange area
+constexpr size_t kControlBytes = kCtrlStride + sizeof(FusedSync);
 
 // A decode "unit": one expert applied to up to 8 activation rows (MMA columns).
 //   rows xrow0 .. xrow0+7 of the activation source, column c present iff bit c of mask;
@@ -81,7 +96,7 @@ inline WsLayout ws_layout(int H, int E, int k, int I, int has_shared, int T) {
   size_t units = (size_t)kDecodeMaxT * k + 1;
   size_t row_units = (rows + 7) / 8 + (size_t)E + 2;
   if (row_units > units) units = row_units;
-  L.ctrl = take(sizeof(Ctrl));
+  L.ctrl = take(kControlBytes);  // control block + the fused decode kernel's exchange area
   L.logits = take((size_t)T * E * 4);
   L.idx = take(Tk * 4);
   L.w = take(Tk * 4);
@@ -195,14 +210,14 @@ cudaError_t launch_decode_down(int H, int I, const moe_expert_set &routed, const
 // fused decode layer (one cooperative kernel: router, top-k, gate/up, down + combine);
 // returns cudaErrorNotSupported when the shape or the device cannot take it (callers fall back).
 // With r_norm != NULL the tokens are x = bf16(RMSNorm_eps(r_norm)) (x unused), bit-identical to
-// launch_rmsnorm followed by the layer. unit_ready: T*k + 1 counters of workspace scratch (the
-// kernel zeroes them itself before use). next_Wr (optional): the router rows of the layer that
-// follows in a stack, prefetched into L2 during the down phase.
+// launch_rmsnorm followed by the layer. ctrl: the workspace's control area (control block and the
+// exchange area behind it). next_Wr (optional): the router rows of the layer that follows in a
+// stack, prefetched into L2 during the down phase.
 cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float eps, int T, int H, const float *Wr,
                                 const float *bias, int E, int k, int I, const moe_expert_set &routed,
-                                const moe_expert_set *shared, const float *residual, float *y, float *logits,
-                                int32_t *idx, float *w, uint16_t *hdec, unsigned *unit_ready, Ctrl *ctrl,
-                                cudaStream_t s, const float *next_Wr = nullptr);
+                                const moe_expert_set *shared, const float *residual, float *y, int32_t *idx,
+                                float *w, uint16_t *hdec, Ctrl *ctrl, cudaStream_t s,
+                                const float *next_Wr = nullptr);
 
 // mid-batch path (about 6..128 tokens; I % kMidFS == 0): units of <= 8 tokens per selected expert
 // built from the routing (no permutation), items (unit, kMidFS-feature slice) that run gate/up,
@@ -215,9 +230,9 @@ cudaError_t launch_mid_ffn(const uint16_t *x, int T, int H, int E, int k, int I,
 // whether launch_decode_fused takes this shape on the current device
 bool decode_fused_fits(int T, int H, int E, int k, int I, const moe_expert_set &routed, bool has_shared);
 
-// test hook: a grid barrier that waits for one arrival more than the `ctas` CTAs make, giving up
-// after limit_ns with MOE_ERR_TIMEOUT in the control area
-cudaError_t launch_barrier_starve(Ctrl *ctrl, int ctas, uint64_t limit_ns, cudaStream_t s);
+// test hook: the fused kernel's logit exchange wait, for a tag no launch writes; it gives up after
+// limit_ns with MOE_ERR_TIMEOUT in the control block
+cudaError_t launch_wait_starve(Ctrl *ctrl, uint64_t limit_ns, cudaStream_t s);
 
 // prefill path (tcgen05 grouped GEMM)
 int gemm_shape_supported(int H, int I);

@@ -10,11 +10,13 @@
 // then sees the layer's expert bytes requested within a few hundred nanoseconds instead of as a
 // chain of dependent round trips.
 //
-// One grid of one CTA per SM (16 warps) runs three phases with one grid barrier:
+// One grid of one CTA per SM (16 warps) runs three phases with no grid barrier:
 //   P1  router logits: four warps per expert split H (the fp32 router rows are requested before
-//       the tokens are staged); the shared expert's rows are prefetched into L2 meanwhile.
-//   --  grid barrier
-//   P1b every CTA computes the same top-k (a threshold from each 32-expert chunk's largest logits,
+//       the tokens are staged); each logit is published as one 64-bit word, this launch's tag in
+//       the high half and the fp32 value in the low half.
+//   P1b every CTA polls the E logit words of its tokens until each carries this launch's tag (tag
+//       and value arrive in one store, so a word that shows the tag holds its value; the shared
+//       expert's rows are prefetched into L2 meanwhile), then computes the same top-k (a threshold from each 32-expert chunk's largest logits,
 //       then one warp sorts the few logits above it) and the distinct-expert unit list
 //       (deterministic), so no second exchange is needed. The warps then issue this CTA's
 //       copies: gate/up items (unit, 8 features: 8 gate + 8 up rows over all of H) dealt
@@ -34,11 +36,13 @@
 // P3, and a down piece first waits until the piece one ring behind it is consumed. A parity wait
 // can then never run two phases ahead of its slot's last completed fill, where it would take the
 // older phase for its own.
-// The grid barrier is one 64-bit arrival counter in the workspace (every launch adds the grid
-// size; a CTA waits for the launch's base + grid). It, the readiness waits and every mbarrier
-// wait are bounded in time and report MOE_ERR_TIMEOUT instead of hanging; before the CTA exits
-// every thread waits for its own outstanding copies (cp.async.wait_all), so no copy is still
-// writing its shared memory.
+// A launch's tag is its number + 1: every CTA adds one to a 64-bit counter in the control block at
+// its start, so the count before the add, divided by the grid, is the launch number (launches do
+// not overlap past griddepcontrol.wait). The readiness counters come in two sets used by alternate
+// launches; a launch zeroes the set the next one will use. The logit polls, the readiness waits
+// and every mbarrier wait are bounded in time and report MOE_ERR_TIMEOUT instead of hanging;
+// before the CTA exits every thread waits for its own outstanding copies (cp.async.wait_all), so
+// no copy is still writing its shared memory.
 #include "common.cuh"
 #include "dequant.cuh"
 #include "gemv.cuh"
@@ -57,8 +61,9 @@ constexpr int kFThreads = kFWarps * 32;
 constexpr int kFSlots = 96;                 // h columns (token, expert) of a step staged for the down phase
 constexpr int kFMaxUnits = kFSlots + 1;
 constexpr int kPairsPerLane = kFSlots / 32; // (token, slot) pairs per lane of the unit-list warp
+static_assert(kFMaxUnits <= kFusedMaxUnits, "readiness counters per unit");
 constexpr int kFMaxRing = 16;               // shared-memory slots for weight copies
-constexpr int kFMaxE = 512;                 // experts the fused kernel takes
+constexpr int kFMaxE = kFusedMaxE;          // experts the fused kernel takes
 constexpr int kFSmemMax = 226 * 1024;       // dynamic shared memory (a little is left for static)
 constexpr int kDnBatch = 4;                 // down half steps (K = 128 each) whose loads go out together
 
@@ -76,12 +81,10 @@ struct FusedArgs {
   moe_expert_set routed, shared;
   const float *residual;
   float *y;
-  float *logits;
   int32_t *idx;
   float *w;
   uint16_t *hdec;
-  unsigned *ready;  // per unit: gate/up items whose h is written (zeroed before the first barrier)
-  Ctrl *ctrl;
+  Ctrl *ctrl;       // control block; the exchange area (tagged logits, readiness counters) follows it
   int ring;        // slots in the ring
   int slot_bytes;  // bytes per slot
   int gu_bytes;    // bytes of one gate/up item
@@ -137,37 +140,24 @@ __host__ __device__ inline FusedLayout fused_layout(int T, int H, int E, int I, 
   return L;
 }
 
-// all CTAs are co-resident (cooperative launch). Barrier j of a launch completes when the arrival
-// counter reaches base + j * nblocks. Every CTA arrives, even after an earlier failure, so the
-// count stays whole; it waits only when `wait` is set. Returns false when the wait gave up (or
-// was not made). Called by every thread of the CTA: the CTA barrier orders the CTA's writes
-// before thread 0's release-add; thread 0's acquire loads and the closing CTA barrier order the
-// CTA's later reads after every other CTA's arrival.
-__device__ bool grid_barrier(Ctrl *c, unsigned long long target, int where, bool wait,
-                             uint64_t limit_ns = kWaitLimitNs) {
-  __shared__ int s_ok;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    // a release add: the CTA's writes ordered before it by the CTA barrier are visible to any
-    // CTA whose acquire load sees the count (no separate fence needed)
-    asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(&c->bar_arrivals) : "memory");
-    int ok = wait ? 1 : 0;
-    const uint64_t t0 = global_ns();
-    while (wait) {
-      unsigned long long v;
-      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(&c->bar_arrivals) : "memory");
-      if ((long long)(v - target) >= 0) break;
-      __nanosleep(32);
-      if (global_ns() - t0 > limit_ns) {
-        ok = 0;
-        set_device_error(c, MOE_ERR_TIMEOUT, where);
-        break;
-      }
-    }
-    s_ok = ok;
+// Poll a logit word until it carries `tag` (the writer's single 64-bit store makes tag and value
+// arrive together, so no fence is needed), giving up after limit_ns or when *abort is set. The
+// first load goes out at once; only a miss starts the clock.
+__device__ __forceinline__ bool poll_tagged(const unsigned long long *p, uint32_t tag, uint64_t limit_ns,
+                                            const volatile int *abort, unsigned long long &v) {
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  if ((uint32_t)(v >> 32) == tag) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    __nanosleep(32);
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    if ((uint32_t)(v >> 32) == tag) return true;
+    if ((abort && *abort) || global_ns() - t0 > limit_ns) return false;
   }
-  __syncthreads();
-  return s_ok != 0;
+}
+
+__device__ __forceinline__ FusedSync *fused_sync(Ctrl *c) {
+  return reinterpret_cast<FusedSync *>(reinterpret_cast<char *>(c) + kCtrlStride);
 }
 
 __device__ __forceinline__ void prefetch_l2(const void *p) {
@@ -324,17 +314,21 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   const int xs16 = H + 4;
   const int G = gridDim.x;
   const unsigned nblk = gridDim.x;
-  __shared__ unsigned long long s_base;
+  FusedSync *const fs = fused_sync(ctrl);
+  __shared__ uint32_t s_tag;
   __shared__ volatile int s_abort;
   // The next launch on the stream (the next layer) may be scheduled now; its CTAs take SMs as this
   // grid's CTAs leave them. Nothing the previous launch writes (the control words, the workspace,
   // the tokens) is touched before it has completed.
   pdl_launch_dependents();
   pdl_wait();
-  if (tid == 0) {  // arrivals of earlier launches: a whole number of grids (before this CTA arrives)
-    unsigned long long v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(&ctrl->bar_arrivals) : "memory");
-    s_base = v - v % nblk;
+  // This launch's number: every CTA of every launch adds one at its start and launches do not
+  // overlap past the wait above, so the count before this CTA's add, divided by the grid, is the
+  // same for all of this launch's CTAs. Its tag marks this launch's logit words; its parity picks
+  // the set of readiness counters. The add's result is first needed after the tokens are staged.
+  unsigned long long launch_no = 0;
+  if (tid == 0) {
+    launch_no = atomicAdd(&ctrl->fused_launches, 1ull);
     s_abort = 0;
     for (int s = 0; s < R; ++s) mbar_init(full(s), 32);  // one arrival per lane of the filling warp
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -445,10 +439,13 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
     d[1] = make_uint2(o[2], o[3]);
   }
   if (lbias) prefetch_range(lbias, (size_t)E * 4, tid, kFThreads);
-  // per-unit readiness counters start at zero; every increment comes after the first grid barrier
-  if (blockIdx.x == 0)
-    for (int u = tid; u <= T * k; u += kFThreads) a.ready[u] = 0u;
+  if (tid == 0) s_tag = (uint32_t)(launch_no / nblk) + 1u;
   __syncthreads();
+  const uint32_t tag = s_tag;
+  unsigned *const ready = fs->ready[tag & 1u];
+  // the other set serves the next launch: the previous launch, its last user, has completed
+  if (blockIdx.x == 0)
+    for (int u = tid; u < kFusedMaxUnits; u += kFThreads) fs->ready[(tag & 1u) ^ 1u][u] = 0u;
 
   // ---------------- P1: router logits, four warps per expert (each a quarter of H), fp32
   {
@@ -488,14 +485,15 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
         const int ee = tid / T, t = tid % T, eg = e0 + ee * G;
         if (eg < E) {
           const float *q4 = rp + ee * 4 * kDecodeMaxT;
-          a.logits[(size_t)t * E + eg] =
-              (q4[t] + q4[kDecodeMaxT + t]) + (q4[2 * kDecodeMaxT + t] + q4[3 * kDecodeMaxT + t]);
+          const float lg = (q4[t] + q4[kDecodeMaxT + t]) + (q4[2 * kDecodeMaxT + t] + q4[3 * kDecodeMaxT + t]);
+          const unsigned long long word = ((unsigned long long)tag << 32) | __float_as_uint(lg);
+          asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(fs->logit + (size_t)t * E + eg), "l"(word)
+                       : "memory");
         }
       }
       __syncthreads();
     }
   }
-  ok = grid_barrier(ctrl, s_base + nblk, 31, true) && ok;
 
   // ---------------- P1b: top-k and unit list, computed identically by every CTA
   if (ok) {
@@ -514,8 +512,13 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
     for (int task = warp; task < T * nch; task += kFWarps) {
       const int t = task / nch, c = task % nch, e = c * 32 + lane;
       uint32_t key = 0u;
-      if (e < E) {
-        key = logit_key(__ldcg(a.logits + (size_t)t * E + e) + (lbias ? __ldg(lbias + e) : 0.f));
+      if (e < E) {  // the logit word of this launch (bounded wait for its writer)
+        unsigned long long v;
+        if (!poll_tagged(fs->logit + (size_t)t * E + e, tag, kWaitLimitNs, &s_abort, v) && !s_abort) {
+          s_abort = 1;
+          set_device_error(ctrl, MOE_ERR_TIMEOUT, 31);
+        }
+        key = logit_key(__uint_as_float((uint32_t)v) + (lbias ? __ldg(lbias + e) : 0.f));
         s_key[t * E + e] = key;
       }
       const uint32_t nidx = (e < E) ? 0xFFFFFFFFu - (uint32_t)e : 0u;
@@ -535,6 +538,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
     if (T > 1)
       for (int e = tid; e < E; e += kFThreads) s_firstof[e] = 0x7fffffff;
     __syncthreads();
+    ok = ok && !s_abort;  // a logit that never arrived: no routing, no expert work
     if (warp < T) {  // the threshold: the k-th largest chunk top
       const unsigned long long v = warp_sort32_desc(lane < nch * m ? s_ctop[warp * 32 + lane] : 0ull);
       if (lane == k - 1) s_tau[warp] = v;
@@ -832,7 +836,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       // the item's h is written: count it for its unit (the group barrier orders the 64 stores
       // before the release add, as in the grid barrier)
       named_sync(kBarGroup0 + grp, 256);
-      if (gtid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(a.ready + u) : "memory");
+      if (gtid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ready + u) : "memory");
     }
   }
   // This CTA's gate/up items are all consumed (the ring rule of P3 below needs it); no grid
@@ -878,7 +882,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
             const uint64_t t0 = global_ns();
             for (;;) {
               unsigned v;
-              asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a.ready + u) : "memory");
+              asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ready + u) : "memory");
               if (v >= (unsigned)rbs8 || s_abort) break;
               __nanosleep(32);
               if (global_ns() - t0 > kWaitLimitNs) {
@@ -890,7 +894,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
           }
           __syncwarp();
           unsigned v;
-          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a.ready + u) : "memory");
+          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ready + u) : "memory");
           (void)v;
           // all of a lane's loads (eight per round) go out before its stores: one L2 round trip
           const int I8 = I / 8, c0 = s_slot[u], nv = (s_slot[u + 1] - c0) * I8;
@@ -997,37 +1001,19 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   cp_async_wait_all();
 }
 
-// Test hook of the failure path: every CTA arrives at the fused kernel's grid barrier, which is
-// then asked to wait for one arrival more than were made. The wait gives up after limit_ns and
-// records MOE_ERR_TIMEOUT; nothing traps and the context stays usable. Each CTA then takes its
-// arrival back, so the count is again a whole number of earlier launches' arrivals (which is what
-// the fused kernel's base computation assumes).
-__global__ void barrier_starve_kernel(Ctrl *ctrl, uint64_t limit_ns) {
-  __shared__ unsigned long long s_base;
-  if (threadIdx.x == 0) {
-    unsigned long long v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(&ctrl->bar_arrivals) : "memory");
-    s_base = v;
-  }
-  __syncthreads();
-  // the base is read before any CTA of this launch arrives only if all read before the first add,
-  // which nothing guarantees; the target base + grid + 1 is out of reach either way, since at most
-  // grid arrivals follow any CTA's read
-  const bool ok = grid_barrier(ctrl, s_base + gridDim.x + 1, 39, true, limit_ns);
-  if (threadIdx.x == 0 && !ok) atomicAdd(&ctrl->bar_arrivals, ~0ull);
+// Test hook of the failure path: one warp waits, with the fused kernel's logit-exchange wait, for
+// a tag that no launch writes (launch tags count up from 1 and would reach this one only after
+// 2^32 - 1 launches). Each lane's wait gives up after limit_ns and MOE_ERR_TIMEOUT is recorded;
+// nothing is written but the error word, nothing traps and the context stays usable.
+__global__ void wait_starve_kernel(Ctrl *ctrl, uint64_t limit_ns) {
+  unsigned long long v;
+  if (!poll_tagged(fused_sync(ctrl)->logit + threadIdx.x, 0xFFFFFFFFu, limit_ns, nullptr, v))
+    set_device_error(ctrl, MOE_ERR_TIMEOUT, 39);
 }
 
-cudaError_t launch_barrier_starve(Ctrl *ctrl, int ctas, uint64_t limit_ns, cudaStream_t s) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ctas);
-  cfg.blockDim = dim3(32);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, barrier_starve_kernel, ctrl, limit_ns);
+cudaError_t launch_wait_starve(Ctrl *ctrl, uint64_t limit_ns, cudaStream_t s) {
+  wait_starve_kernel<<<1, 32, 0, s>>>(ctrl, limit_ns);
+  return cudaGetLastError();
 }
 
 // Shapes, ring and shared-memory plan of a fused launch; false when the shape or the device cannot
@@ -1133,9 +1119,8 @@ static cudaError_t fused_launch(const void *fn, size_t smem, void **args, cudaSt
 
 cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float eps, int T, int H, const float *Wr,
                                 const float *bias, int E, int k, int I, const moe_expert_set &routed,
-                                const moe_expert_set *shared, const float *residual, float *y, float *logits,
-                                int32_t *idx, float *w, uint16_t *hdec, unsigned *unit_ready, Ctrl *ctrl,
-                                cudaStream_t s, const float *next_Wr) {
+                                const moe_expert_set *shared, const float *residual, float *y, int32_t *idx,
+                                float *w, uint16_t *hdec, Ctrl *ctrl, cudaStream_t s, const float *next_Wr) {
   FusedArgs a;
   const void *fn = nullptr;
   size_t smem = 0;
@@ -1153,11 +1138,9 @@ cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float ep
   a.shared = shared ? *shared : routed;
   a.residual = residual;
   a.y = y;
-  a.logits = logits;
   a.idx = idx;
   a.w = w;
   a.hdec = hdec;
-  a.ready = unit_ready;
   a.ctrl = ctrl;
   void *args[] = {&a};
   return fused_launch(fn, smem, args, s);

@@ -126,12 +126,12 @@ def test_router_permute_combine_validation(lib):
     assert lib.moe_workspace_init(FAKE, ctypes.c_size_t(16), None) == 3
 
 
-def test_barrier_timeout_hook_validation(lib):
+def test_wait_timeout_hook_validation(lib):
     # host-side argument checks only; the timeout itself is exercised on the GPU
-    assert lib.moe_test_barrier_timeout(None, ctypes.c_size_t(1 << 20), 20, None) == moe.MOE_ERR_WORKSPACE
-    assert lib.moe_test_barrier_timeout(FAKE, ctypes.c_size_t(64), 20, None) == moe.MOE_ERR_WORKSPACE
-    assert lib.moe_test_barrier_timeout(FAKE, ctypes.c_size_t(1 << 20), 0, None) == moe.MOE_ERR_INVALID_ARG
-    assert lib.moe_test_barrier_timeout(FAKE, ctypes.c_size_t(1 << 20), 5000, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_test_wait_timeout(None, ctypes.c_size_t(1 << 20), 20, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_test_wait_timeout(FAKE, ctypes.c_size_t(1024), 20, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_test_wait_timeout(FAKE, ctypes.c_size_t(1 << 20), 0, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_test_wait_timeout(FAKE, ctypes.c_size_t(1 << 20), 5000, None) == moe.MOE_ERR_INVALID_ARG
 
 
 def test_stack_validation(lib):

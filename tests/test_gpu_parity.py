@@ -262,10 +262,10 @@ def test_zero_tokens_is_noop():
 
 
 # ----------------------------------------------------------------------------- failure path
-def test_starved_barrier_times_out_and_context_survives():
-    # A grid barrier waiting for an arrival that never comes gives up after its limit, reports
-    # MOE_ERR_TIMEOUT through the workspace error word, and leaves the context and the workspace
-    # fit for the next call (which must still match the oracle).
+def test_starved_wait_times_out_and_context_survives():
+    # The fused kernel's logit-exchange wait, polling for a tag that never arrives, gives up after
+    # its limit, reports MOE_ERR_TIMEOUT through the workspace error word, and leaves the context
+    # and the workspace fit for the next call (which must still match the oracle).
     L, (x, Wr, b, routed, shared) = layer_of("decode1")
     s = L.shape
     ws = ws_for(L)
@@ -273,7 +273,7 @@ def test_starved_barrier_times_out_and_context_survives():
     assert moe.read_device_error(ws) == 0
     import time
     t0 = time.perf_counter()
-    moe.test_barrier_timeout(ws, limit_ms=20)
+    moe.test_wait_timeout(ws, limit_ms=20)
     assert moe.read_device_error(ws) == moe.MOE_ERR_TIMEOUT
     assert time.perf_counter() - t0 < 1.5           # the limit, not a hang
     assert moe.read_device_error(ws) == 0            # reading cleared the word
