@@ -85,12 +85,16 @@ _DEC_SRC = ["quantized_expert_ffn_gemm_b200/csrc/decode_fused.cu", "quantized_ex
             "quantized_expert_ffn_gemm_b200/csrc/tc.cuh", "quantized_expert_ffn_gemm_b200/csrc/topk.cuh"]
 _GEMM_SRC = ["quantized_expert_ffn_gemm_b200/csrc/gemm.cu", "quantized_expert_ffn_gemm_b200/csrc/tc.cuh",
              "quantized_expert_ffn_gemm_b200/csrc/dequant.cuh"]
+_MID_SRC = ["quantized_expert_ffn_gemm_b200/csrc/mid.cu", "quantized_expert_ffn_gemm_b200/csrc/common.cuh",
+            "quantized_expert_ffn_gemm_b200/csrc/dequant.cuh", "quantized_expert_ffn_gemm_b200/csrc/gemv.cuh"]
 TRAFFIC = {
     # (kernel, workloads with the captured launch shape): (sources, sha256, DRAM bytes per launch)
     ("gemm_gate_up", ("prefill8k", "stack_prefill")):
-        (_GEMM_SRC, "f5ad8aca8c32a2576bfdf9f5a1d66e6cbeb86fb1fb932b6adae357c9fbff935a", 786358272),
+        (_GEMM_SRC, "4973eaa737f0c89dba7e023c10b843e0bcbed182f4dbe40b7fc3e74b446fe30c", 863316224),
     ("decode_fused", ("decode1",)):
         (_DEC_SRC, "079b8a42801687ba382781d35128bd3914e45a1093ae366b7f07f8b8b245e47d", 15117824),
+    ("mid_expert", ("batch32",)):
+        (_MID_SRC, "17c6b89e453fea4a857d913221474e60272445c7aabe453d804734421b2fd54f", 47095808),
 }
 
 

@@ -539,10 +539,17 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       for (int e = tid; e < E; e += kFThreads) s_firstof[e] = 0x7fffffff;
     __syncthreads();
     ok = ok && !s_abort;  // a logit that never arrived: no routing, no expert work
-    if (warp < T) {  // the threshold: the k-th largest chunk top
-      const unsigned long long v = warp_sort32_desc(lane < nch * m ? s_ctop[warp * 32 + lane] : 0ull);
-      if (lane == k - 1) s_tau[warp] = v;
-      if (lane == 0) s_ccnt[warp] = 0;
+    if (warp < T) {  // the threshold: the k-th largest chunk top (0 when fewer than k are nonzero)
+      if (lane == 0) {
+        s_tau[warp] = 0ull;
+        s_ccnt[warp] = 0;
+      }
+      __syncwarp();
+      const int cnt = nch * m;
+      if (lane < cnt) {
+        const unsigned long long v = s_ctop[warp * 32 + lane];
+        if (v != 0ull && rank_desc32(s_ctop + warp * 32, cnt, v) == k - 1) s_tau[warp] = v;
+      }
     }
     __syncthreads();
 #pragma unroll 1
@@ -562,9 +569,13 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
     if (warp < T) {
       const int t = warp, n = s_ccnt[t];
       unsigned long long *sel = s_ctop + t * 32;  // reused: the selected codes in slot order
-      if (n <= 32) {  // sort the candidates: lane r holds the r-th largest
-        const unsigned long long v = warp_sort32_desc(lane < n ? s_cand[t * 32 + lane] : 0ull);
-        if (lane < k) sel[lane] = v;
+      if (n <= 32) {  // rank the candidates: slot r of sel gets the r-th largest
+        // lane r's code goes to slot rank(code): the candidates are distinct, nonzero codes
+        if (lane < n) {
+          const unsigned long long v = s_cand[t * 32 + lane];
+          const int r = rank_desc32(s_cand + t * 32, n, v);
+          if (r < k) sel[r] = v;
+        }
       } else {  // mass ties: k rounds of arg-max over the token's E codes
         uint32_t taken = 0u;  // bit i: expert lane + 32 i already selected
 #pragma unroll 1

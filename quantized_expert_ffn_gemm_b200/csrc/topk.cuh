@@ -66,6 +66,20 @@ __device__ __forceinline__ void sort16_desc(unsigned long long c[16]) {
 __device__ __forceinline__ unsigned long long cmax64(unsigned long long a, unsigned long long b) { return a > b ? a : b; }
 __device__ __forceinline__ unsigned long long cmin64(unsigned long long a, unsigned long long b) { return a < b ? a : b; }
 
+// How many of the first n (<= 32) codes of s exceed v: with distinct codes, v's position in
+// descending order. Every lane reads all n from shared memory (broadcast reads, independent of one
+// another), so ranking a warp's worth of codes costs about one pass over them instead of the
+// dependent stages of a sorting network.
+__device__ __forceinline__ int rank_desc32(const unsigned long long *s, int n, unsigned long long v) {
+  int r0 = 0, r1 = 0;
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    r0 += (j < n && s[j] > v) ? 1 : 0;
+    r1 += (j + 1 < n && s[j + 1] > v) ? 1 : 0;
+  }
+  return r0 + r1;
+}
+
 // sort the warp's 32 codes into descending lane order
 __device__ __forceinline__ unsigned long long warp_sort32_desc(unsigned long long v) {
   const int lane = threadIdx.x & 31;
