@@ -30,20 +30,22 @@ struct Ctrl {
   unsigned long long pad_u64;
   int mid_pairs;            // mid-batch path: routed (token, slot) pairs with a valid expert
   int pad2;
-  unsigned long long fused_launches;  // fused decode: CTAs started (every launch adds its grid size)
-  int pad1[16];
+  int pad1[18];
 };
 static_assert(sizeof(Ctrl) == 128, "control block is 128 bytes");
 
 // The fused decode kernel's exchange area, the rest of the control area (zeroed once by
 // moe_workspace_init and used by that kernel only): router logits as (launch tag << 32 | fp32 bits)
-// words that readers poll for their own launch's tag, and per-unit readiness counters in two sets
-// used by alternate launches (a launch zeroes the other set for the next one).
+// words that readers poll for their own launch's tag, per-unit readiness counters in two sets
+// used by alternate launches (a launch zeroes the other set for the next one), and each CTA's
+// count of the launches it has started (every launch runs one CTA per SM, so the counts agree).
 constexpr int kFusedMaxE = 512;   // experts the fused decode kernel takes
 constexpr int kFusedMaxUnits = 128;
+constexpr int kFusedMaxGrid = 256;  // CTAs of a fused launch (one per SM)
 struct FusedSync {
   unsigned long long logit[kDecodeMaxT * kFusedMaxE];
   unsigned ready[2][kFusedMaxUnits];
+  unsigned seq[kFusedMaxGrid];  // per CTA: launches it has started (all equal between launches)
 };
 constexpr size_t kCtrlStride = 256;  // the control block, then the exchange area
 constexpr size_t kControlBytes = kCtrlStride + sizeof(FusedSync);

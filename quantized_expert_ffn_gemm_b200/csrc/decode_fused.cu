@@ -12,10 +12,10 @@
 //
 // One grid of one CTA per SM (16 warps) runs three phases with no grid barrier:
 //   P1  router logits: four warps per expert split H (the fp32 router rows are requested before
-//       the tokens are staged); each logit is published as one 64-bit word, this launch's tag in
-//       the high half and the fp32 value in the low half.
+//       the tokens are staged); each logit is published as one 64-bit word (an atomic exchange),
+//       this launch's tag in the high half and the fp32 value in the low half.
 //   P1b every CTA polls the E logit words of its tokens until each carries this launch's tag (tag
-//       and value arrive in one store, so a word that shows the tag holds its value; the shared
+//       and value arrive in one write, so a word that shows the tag holds its value; the shared
 //       expert's rows are prefetched into L2 meanwhile), then computes the same top-k (a threshold from each 32-expert chunk's largest logits,
 //       then one warp sorts the few logits above it) and the distinct-expert unit list
 //       (deterministic), so no second exchange is needed. The warps then issue this CTA's
@@ -36,9 +36,9 @@
 // P3, and a down piece first waits until the piece one ring behind it is consumed. A parity wait
 // can then never run two phases ahead of its slot's last completed fill, where it would take the
 // older phase for its own.
-// A launch's tag is its number + 1: every CTA adds one to a 64-bit counter in the control block at
-// its start, so the count before the add, divided by the grid, is the launch number (launches do
-// not overlap past griddepcontrol.wait). The readiness counters come in two sets used by alternate
+// A launch's tag is its number + 1: every CTA keeps its own count of started launches in the
+// exchange area and advances it once per launch, so all CTAs of a launch agree on it (launches
+// do not overlap past griddepcontrol.wait). The readiness counters come in two sets used by alternate
 // launches; a launch zeroes the set the next one will use. The logit polls, the readiness waits
 // and every mbarrier wait are bounded in time and report MOE_ERR_TIMEOUT instead of hanging;
 // before the CTA exits every thread waits for its own outstanding copies (cp.async.wait_all), so
@@ -140,7 +140,7 @@ __host__ __device__ inline FusedLayout fused_layout(int T, int H, int E, int I, 
   return L;
 }
 
-// Poll a logit word until it carries `tag` (the writer's single 64-bit store makes tag and value
+// Poll a logit word until it carries `tag` (the writer's single 64-bit exchange makes tag and value
 // arrive together, so no fence is needed), giving up after limit_ns or when *abort is set. The
 // first load goes out at once; only a miss starts the clock.
 __device__ __forceinline__ bool poll_tagged(const unsigned long long *p, uint32_t tag, uint64_t limit_ns,
@@ -313,7 +313,6 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   Ctrl *ctrl = a.ctrl;
   const int xs16 = H + 4;
   const int G = gridDim.x;
-  const unsigned nblk = gridDim.x;
   FusedSync *const fs = fused_sync(ctrl);
   __shared__ uint32_t s_tag;
   __shared__ volatile int s_abort;
@@ -322,13 +321,14 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   // the tokens) is touched before it has completed.
   pdl_launch_dependents();
   pdl_wait();
-  // This launch's number: every CTA of every launch adds one at its start and launches do not
-  // overlap past the wait above, so the count before this CTA's add, divided by the grid, is the
-  // same for all of this launch's CTAs. Its tag marks this launch's logit words; its parity picks
-  // the set of readiness counters. The add's result is first needed after the tokens are staged.
-  unsigned long long launch_no = 0;
+  // This launch's tag: one more than the launches this CTA's slot has counted (each CTA reads and
+  // advances only its own slot, and every launch advances every slot once, so all of a launch's
+  // CTAs read the same count; launches do not overlap past the wait above). The tag marks this
+  // launch's logit words; its parity picks the set of readiness counters. The load's result is
+  // first needed after the tokens are staged.
+  uint32_t launch_no = 0;
   if (tid == 0) {
-    launch_no = atomicAdd(&ctrl->fused_launches, 1ull);
+    launch_no = *reinterpret_cast<volatile const uint32_t *>(&fs->seq[blockIdx.x]);
     s_abort = 0;
     for (int s = 0; s < R; ++s) mbar_init(full(s), 32);  // one arrival per lane of the filling warp
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -439,7 +439,10 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
     d[1] = make_uint2(o[2], o[3]);
   }
   if (lbias) prefetch_range(lbias, (size_t)E * 4, tid, kFThreads);
-  if (tid == 0) s_tag = (uint32_t)(launch_no / nblk) + 1u;
+  if (tid == 0) {
+    s_tag = launch_no + 1u;
+    fs->seq[blockIdx.x] = launch_no + 1u;  // read by this CTA's slot in the next launch only
+  }
   __syncthreads();
   const uint32_t tag = s_tag;
   unsigned *const ready = fs->ready[tag & 1u];
@@ -486,9 +489,10 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
         if (eg < E) {
           const float *q4 = rp + ee * 4 * kDecodeMaxT;
           const float lg = (q4[t] + q4[kDecodeMaxT + t]) + (q4[2 * kDecodeMaxT + t] + q4[3 * kDecodeMaxT + t]);
+          // an atomic exchange rather than a relaxed store: it is performed at L2 at once, so the
+          // word reaches the polling CTAs sooner (measured: all logits in ~0.9 us earlier)
           const unsigned long long word = ((unsigned long long)tag << 32) | __float_as_uint(lg);
-          asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(fs->logit + (size_t)t * E + eg), "l"(word)
-                       : "memory");
+          atomicExch(fs->logit + (size_t)t * E + eg, word);
         }
       }
       __syncthreads();
@@ -1032,7 +1036,9 @@ cudaError_t launch_wait_starve(Ctrl *ctrl, uint64_t limit_ns, cudaStream_t s) {
 static bool fused_plan(int T, int H, int E, int k, int I, const moe_expert_set &routed, bool has_shared,
                        FusedArgs &a, const void *&fn, size_t &smem) {
   const int hs_cols = T * k + (has_shared ? T : 0);
-  if (T < 1 || T > kDecodeMaxT || E > kFMaxE || H > 2048 || I > 1024 || hs_cols > kFSlots || k > 16) return false;
+  if (T < 1 || T > kDecodeMaxT || E > kFMaxE || H > 2048 || I > 1024 || hs_cols > kFSlots || k > 16 ||
+      num_sms() > kFusedMaxGrid)
+    return false;
   const int qt = routed.gate.qtype;
   const int per = qt == MOE_Q3 ? 7 : qt == MOE_Q4 ? 9 : 5;  // bytes per 16 weights: codes, scales (, hi bits)
   const int gu_bytes = per * H;  // 8 gate + 8 up rows
