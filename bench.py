@@ -92,7 +92,7 @@ TRAFFIC = {
     ("gemm_gate_up", ("prefill8k", "stack_prefill")):
         (_GEMM_SRC, "4973eaa737f0c89dba7e023c10b843e0bcbed182f4dbe40b7fc3e74b446fe30c", 863316224),
     ("decode_fused", ("decode1",)):
-        (_DEC_SRC, "079b8a42801687ba382781d35128bd3914e45a1093ae366b7f07f8b8b245e47d", 15117824),
+        (_DEC_SRC, "ab9722e6aca444c671e3ee9a4f3713519adcb5909c38506670f9f3632a713fbd", 15127808),
     ("mid_expert", ("batch32",)):
         (_MID_SRC, "17c6b89e453fea4a857d913221474e60272445c7aabe453d804734421b2fd54f", 47095808),
 }
