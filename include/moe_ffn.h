@@ -32,6 +32,13 @@
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Every call
  *     only enqueues work on it and returns; nothing synchronises except
  *     moe_read_device_error.
+ *   - The library's kernels are launched with programmatic stream serialization: a launch may
+ *     begin while the previous kernel on the stream finishes, but only when that kernel allows
+ *     it (this library's kernels do, at their entry; set MOE_PDL=0 in the environment to turn
+ *     it off). Everything a predecessor may write is read only after it has completed, except
+ *     the layers' router weights Wr, which the fused decode kernel starts reading early: a
+ *     kernel that writes Wr and allows its dependents to start before it ends (CUDA's
+ *     programmatic launch completion) must not directly precede a layer call.
  *   - bf16 / fp16 tensors are passed as uint16_t bit patterns. Layouts are row-major and
  *     contiguous: x, y, r: [T,H]; idx, w: [T,k]; Wr: [E,H].
  *   - Arguments are validated on the host before anything is enqueued; on error nothing runs

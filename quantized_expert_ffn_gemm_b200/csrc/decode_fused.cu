@@ -316,6 +316,23 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   FusedSync *const fs = fused_sync(ctrl);
   __shared__ uint32_t s_tag;
   __shared__ volatile int s_abort;
+  // ---------------- P0: this warp's router rows are requested first, then the tokens are staged
+  const int H4 = H / 4, HQ = H4 / 4;  // float4 per quarter of a router row (<= 128: H <= 2048)
+  const int es = warp >> 2, qh = warp & 3;
+  float4 rv[4];
+  auto load_router = [&](int e) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int h4 = lane + 32 * u;
+      rv[u] = (e < E && h4 < HQ) ? __ldcs(reinterpret_cast<const float4 *>(a.Wr + (size_t)e * H) + qh * HQ + h4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  // The router rows are weights, which no kernel of this library writes; and a launch can start
+  // before its predecessor has finished only behind a kernel that allowed it (this library's
+  // kernels do, at their entry). So they are requested before the wait below, and their fetch
+  // overlaps the previous layer's last CTAs.
+  load_router((int)blockIdx.x + es * G);
   // The next launch on the stream (the next layer) may be scheduled now; its CTAs take SMs as this
   // grid's CTAs leave them. Nothing the previous launch writes (the control words, the workspace,
   // the tokens) is touched before it has completed.
@@ -351,19 +368,6 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   const float *const lrn = a.r_norm;
   const float *const lres = a.residual;
 
-  // ---------------- P0: this warp's router rows are requested first, then the tokens are staged
-  const int H4 = H / 4, HQ = H4 / 4;  // float4 per quarter of a router row (<= 128: H <= 2048)
-  const int es = warp >> 2, qh = warp & 3;
-  float4 rv[4];
-  auto load_router = [&](int e) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int h4 = lane + 32 * u;
-      rv[u] = (e < E && h4 < HQ) ? __ldcs(reinterpret_cast<const float4 *>(lWr + (size_t)e * H) + qh * HQ + h4)
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  };
-  load_router((int)blockIdx.x + es * G);
   __shared__ float s_inv[kDecodeMaxT];
   // token staging in chunks of 8 values: at most 4 per thread (T <= 8, H <= 2048)
   constexpr int kChunks = 4;
