@@ -26,7 +26,7 @@ import torch
 import oracle
 import quantized_expert_ffn_gemm_b200 as moe
 import synth
-from tests.gpu_util import W_TOL
+from tests.gpu_util import W_TOL, check_layer, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -129,3 +129,19 @@ def test_all_logits_equal_take_the_lowest_indices(T):
         _, idx, w = moe.layer_forward(x.cuda(), Wr0, None, routed, shared, K, ws, want_routing=True)
         _check(idx, w, idx_ref, w_ref)
     assert moe.read_device_error(ws) == 0
+
+
+@pytest.mark.parametrize("E", [33, 40, 97])
+@pytest.mark.parametrize("T", [1, 3, 8])
+def test_fused_topk_with_a_partial_last_chunk(E, T):
+    # E not a multiple of 32: the last 32-expert chunk is partial, so some chunks hold fewer valid
+    # experts than the chunk tops they contribute (at E = 33, k = 10: five tops from a 1-expert
+    # chunk) and the threshold must fall to 0 with more candidates than one warp holds; the fused
+    # decode kernel's routing and y still match the oracle
+    s = synth.LayerShape(f"partial{E}", T, 256, E, 10, 128, synth.Q2, True, 1.1, seed=21)
+    L = synth.make_layer(s)
+    x, Wr, b, routed, shared = to_dev(L)
+    ws = moe.Workspace.for_layer(s.H, s.E, s.k, s.I, True, T)
+    y, idx, w = moe.layer_forward(x, Wr, b, routed, shared, s.k, ws, want_routing=True)
+    assert moe.read_device_error(ws) == 0
+    check_layer(y.cpu().numpy(), idx.cpu().numpy(), L, range(T), w_gpu=w.cpu().numpy())
