@@ -218,11 +218,13 @@ moe_status moe_combine(const uint16_t *out_perm, const int32_t *row_of, const fl
  * GEMV: the decode path (router + top-k, then a
  * dequant-GEMV over the distinct selected experts with the tokens as MMA columns, down
  * projection fused with the weighted combine; under AUTO one cooperative kernel does the whole
- * layer where its shared-memory plan fits). Otherwise: router + top-k (fp32 dot products on the
- * CUDA cores up to 128 tokens, tensor-core logits with an exact refine of the candidates above),
- * permute, the expert FFN (AUTO / GEMM: tcgen05 grouped GEMM gate/up with fused SwiGLU, then
- * down; GEMV: the decode GEMV kernels over 8-row chunks of each expert's rows), combine. Every
- * path computes the same function within the parity tolerance.
+ * layer where its shared-memory plan fits, T*k + T <= 96). AUTO with 8..64 tokens where that
+ * kernel does not fit, or path MID: the mid-batch path (MOE_PATH_MID above). Otherwise: router +
+ * top-k (fp32 dot products on the CUDA cores up to 128 tokens, tensor-core logits with an exact
+ * refine of the candidates above), permute, the expert FFN (AUTO / GEMM: tcgen05 grouped GEMM
+ * gate/up with fused SwiGLU, then down; GEMV: the decode GEMV kernels over 8-row chunks of each
+ * expert's rows; MMQ: int8 activations for gate/up), combine. Every path computes the same
+ * function within the parity tolerance.
  *   y = sum_j w_j FFN_{idx_j}(x) + FFN_shared(x) (+ residual)      fp32 [T,H]
  * x bf16 [T,H]; Wr fp32 [E,H]; bias fp32 [E] or NULL; routed: gate/up [E][I][H], down [E][H][I];
  * shared_opt: one expert (n_experts = 1) when desc->has_shared; residual_opt fp32 [T,H] or NULL
@@ -234,6 +236,18 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
                              int32_t *idx_out_opt, float *w_out_opt, int32_t path,
                              void *ws, size_t ws_bytes, void *stream);
 
+/* moe_layer_forward with the tokens and the output in HOST memory: x_host bf16 [T,H] is copied to
+ * the workspace, the layer runs on it (no residual), and y lands in y_host fp32 [T,H]; one call
+ * enqueues the host-to-device copy, the layer and the device-to-host copy on `stream` and returns
+ * (the copies are asynchronous for page-locked host buffers; y_host is complete once the stream
+ * has reached this point). The weights, the workspace and the optional routing outputs stay in
+ * device memory; other arguments and errors as moe_layer_forward (MOE_ERR_INVALID_ARG for a
+ * NULL x_host or y_host). */
+moe_status moe_layer_forward_host(const uint16_t *x_host, int32_t T, const float *Wr, const float *bias,
+                                  const moe_layer_desc *desc, const moe_expert_set *routed,
+                                  const moe_expert_set *shared_opt, float *y_host, int32_t *idx_out_opt,
+                                  float *w_out_opt, int32_t path, void *ws, size_t ws_bytes, void *stream);
+
 /* A stack of L layers with pre-router RMSNorm and a residual stream, attention omitted (the
  * 48 MoE layers of "Strata vs Llama.cpp vs vLLM", "How Strata is designed to work"):
  *   r_0 = r_in;  r_{l+1} = r_l + layer_l( bf16(RMSNorm_eps(r_l)) );  r_out = r_L
@@ -244,6 +258,15 @@ moe_status moe_stack_forward(const float *r_in, int32_t T, int32_t L, const floa
                              const float *const *bias, const moe_layer_desc *desc,
                              const moe_expert_set *routed, const moe_expert_set *shared, float eps,
                              float *r_out, int32_t path, void *ws, size_t ws_bytes, void *stream);
+
+/* moe_stack_forward with the residual stream in HOST memory: r_in_host fp32 [T,H] is copied to the
+ * workspace, the stack runs there in place, and the result lands in r_out_host fp32 [T,H] (may be
+ * the same buffer); one call enqueues the two copies and the stack on `stream` and returns.
+ * Weights and workspace in device memory; other arguments and errors as moe_stack_forward. */
+moe_status moe_stack_forward_host(const float *r_in_host, int32_t T, int32_t L, const float *const *Wr,
+                                  const float *const *bias, const moe_layer_desc *desc, const moe_expert_set *routed,
+                                  const moe_expert_set *shared, float eps, float *r_out_host, int32_t path, void *ws,
+                                  size_t ws_bytes, void *stream);
 
 /* Test hook: dequantize rows row0..row0+nrows-1 of one expert with the decoder the expert
  * kernels use (the block formats are the stand-in stated at the top of this file).

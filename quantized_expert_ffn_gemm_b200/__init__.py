@@ -27,7 +27,7 @@ EXPORTED = ["moe_status_string", "moe_workspace_bytes", "moe_workspace_init", "m
             "moe_router_topk", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
             "moe_stack_forward", "moe_dequant_rows", "moe_read_device_error", "moe_timing_enable",
             "moe_timing_read", "moe_kernel_count", "moe_kernel_name", "moe_router_topk_static",
-            "moe_test_wait_timeout"]
+            "moe_test_wait_timeout", "moe_layer_forward_host", "moe_stack_forward_host"]
 
 
 class MoeError(RuntimeError):
@@ -257,6 +257,19 @@ def stack_forward(r_in: torch.Tensor, stack: Stack, ws: Workspace, eps: float = 
     return r_out
 
 
+def stack_forward_host(r_in_host: torch.Tensor, stack: Stack, ws: Workspace, eps: float = 1e-6,
+                       path: int = PATH_AUTO, r_out_host: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """moe_stack_forward_host: the residual stream in host memory (page-locked for asynchronous
+    copies); r_out_host may be r_in_host."""
+    T, H = r_in_host.shape
+    if r_out_host is None:
+        r_out_host = torch.empty_like(r_in_host)
+    _check("moe_stack_forward_host", lib().moe_stack_forward_host(
+        _p(r_in_host), T, stack.L, stack.wr_arr, stack.b_arr, ctypes.byref(stack.desc), stack.r_arr, stack.s_arr,
+        ctypes.c_float(eps), _p(r_out_host), path, ws.ptr, ws.size, _stream()))
+    return r_out_host
+
+
 def dequant_rows(m, expert: int, row0: int, nrows: int):
     """(fp32 [nrows,K], fp16 [nrows,K]) dequantized rows of one expert, computed on the GPU."""
     q = qmat(m)
@@ -309,6 +322,7 @@ class LayerHandle:
     and for tight decode loops)."""
 
     _fast = None
+    _fast_host = None
 
     def __init__(self, Wr: torch.Tensor, bias: Optional[torch.Tensor], routed, shared, k: int, ws: Workspace):
         L = lib()
@@ -316,6 +330,8 @@ class LayerHandle:
             vp, i32 = ctypes.c_void_p, ctypes.c_int32
             proto = ctypes.CFUNCTYPE(i32, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, ctypes.c_size_t, vp)
             LayerHandle._fast = proto(("moe_layer_forward", L))
+            proto_h = ctypes.CFUNCTYPE(i32, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, ctypes.c_size_t, vp)
+            LayerHandle._fast_host = proto_h(("moe_layer_forward_host", L))
         self.refs = (Wr, bias, routed, shared, ws)  # keep the tensors alive
         self.H, self.E, self.k, self.I = Wr.shape[1], Wr.shape[0], k, routed.gate.rows
         self.desc = layer_desc(self.H, self.E, k, self.I, shared is not None)
@@ -336,3 +352,16 @@ class LayerHandle:
         if code != MOE_OK:
             raise MoeError("moe_layer_forward", code)
         return y
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, idx_out: Optional[torch.Tensor] = None,
+                     w_out: Optional[torch.Tensor] = None, path: int = PATH_AUTO):
+        """moe_layer_forward_host: x and y in host memory (page-locked for asynchronous copies); the
+        copies and the layer are enqueued on the current stream by one C call."""
+        wr, b, d, rs, ss = self._a
+        code = LayerHandle._fast_host(x_host.data_ptr(), x_host.shape[0], wr, b, d, rs, ss, y_host.data_ptr(),
+                                      None if idx_out is None else idx_out.data_ptr(),
+                                      None if w_out is None else w_out.data_ptr(), path, self._ws[0], self._ws[1],
+                                      torch.cuda.current_stream().cuda_stream)
+        if code != MOE_OK:
+            raise MoeError("moe_layer_forward_host", code)
+        return y_host

@@ -324,11 +324,13 @@ moe_status moe_combine(const uint16_t *out_perm, const int32_t *row_of, const fl
       launch_combine(out_perm, row_of, w, T, k, H, shared_out_opt, residual_opt, y, (cudaStream_t)stream));
 }
 
-moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, const float *bias,
-                             const moe_layer_desc *desc, const moe_expert_set *routed,
-                             const moe_expert_set *shared_opt, const float *residual_opt, float *y,
-                             int32_t *idx_out_opt, float *w_out_opt, int32_t path, void *ws, size_t ws_bytes,
-                             void *stream) {
+// the layer's argument checks and, with run set, its launches (the host-buffer entry point checks
+// first and enqueues its copies only for a call that will run)
+static moe_status layer_forward_impl(const uint16_t *x, int32_t T, const float *Wr, const float *bias,
+                                     const moe_layer_desc *desc, const moe_expert_set *routed,
+                                     const moe_expert_set *shared_opt, const float *residual_opt, float *y,
+                                     int32_t *idx_out_opt, float *w_out_opt, int32_t path, void *ws, size_t ws_bytes,
+                                     void *stream, bool run) {
   if (!desc) return MOE_ERR_INVALID_ARG;
   const int H = desc->H, E = desc->E, k = desc->k, I = desc->I, hs = desc->has_shared ? 1 : 0;
   moe_status st = shape_status(H, E, k, I);
@@ -355,6 +357,7 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
                           decode_fused_fits(T, H, E, k, I, *routed, hs != 0);
   const bool mid = path == MOE_PATH_MID ||
                    (path == MOE_PATH_AUTO && !fused_fits && mid_ok && T >= kAutoMidLo && T <= kAutoMidHi);
+  if (!run) return MOE_OK;
 
   cudaStream_t s = (cudaStream_t)stream;
   Ctrl *ctrl = at<Ctrl>(ws, L.ctrl);
@@ -422,16 +425,48 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
   return cuda_status(e);
 }
 
-moe_status moe_stack_forward(const float *r_in, int32_t T, int32_t L, const float *const *Wr,
-                             const float *const *bias, const moe_layer_desc *desc, const moe_expert_set *routed,
-                             const moe_expert_set *shared, float eps, float *r_out, int32_t path, void *ws,
-                             size_t ws_bytes, void *stream) {
+moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, const float *bias,
+                             const moe_layer_desc *desc, const moe_expert_set *routed,
+                             const moe_expert_set *shared_opt, const float *residual_opt, float *y,
+                             int32_t *idx_out_opt, float *w_out_opt, int32_t path, void *ws, size_t ws_bytes,
+                             void *stream) {
+  return layer_forward_impl(x, T, Wr, bias, desc, routed, shared_opt, residual_opt, y, idx_out_opt, w_out_opt, path,
+                            ws, ws_bytes, stream, true);
+}
+
+moe_status moe_layer_forward_host(const uint16_t *x_host, int32_t T, const float *Wr, const float *bias,
+                                  const moe_layer_desc *desc, const moe_expert_set *routed,
+                                  const moe_expert_set *shared_opt, float *y_host, int32_t *idx_out_opt,
+                                  float *w_out_opt, int32_t path, void *ws, size_t ws_bytes, void *stream) {
+  if (!desc || T < 0) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!x_host || !y_host)) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && !ws) return MOE_ERR_WORKSPACE;
+  const int H = desc->H;
+  const WsLayout L = ws_layout(H, desc->E, desc->k, desc->I, desc->has_shared ? 1 : 0, T);
+  uint16_t *xd = T > 0 ? at<uint16_t>(ws, L.xio) : nullptr;
+  float *yd = T > 0 ? at<float>(ws, L.yio) : nullptr;
+  moe_status st = layer_forward_impl(xd, T, Wr, bias, desc, routed, shared_opt, nullptr, yd, idx_out_opt, w_out_opt,
+                                     path, ws, ws_bytes, stream, false);
+  if (st != MOE_OK || T == 0) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(xd, x_host, (size_t)T * H * 2, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
+  st = layer_forward_impl(xd, T, Wr, bias, desc, routed, shared_opt, nullptr, yd, idx_out_opt, w_out_opt, path, ws,
+                          ws_bytes, stream, true);
+  if (st != MOE_OK) return st;
+  return cuda_status(cudaMemcpyAsync(y_host, yd, (size_t)T * H * 4, cudaMemcpyDeviceToHost, s));
+}
+
+// the stack's argument checks and, with run set, its work (as layer_forward_impl)
+static moe_status stack_forward_impl(const float *r_in, int32_t T, int32_t L, const float *const *Wr,
+                                     const float *const *bias, const moe_layer_desc *desc,
+                                     const moe_expert_set *routed, const moe_expert_set *shared, float eps,
+                                     float *r_out, int32_t path, void *ws, size_t ws_bytes, void *stream, bool run) {
   if (!desc || L < 0 || T < 0 || !(eps >= 0.0f)) return MOE_ERR_INVALID_ARG;
   const int H = desc->H, E = desc->E, k = desc->k, I = desc->I, hs = desc->has_shared ? 1 : 0;
   moe_status st = shape_status(H, E, k, I);
   if (st != MOE_OK) return st;
   if (T == 0 || L == 0) {
-    if (T > 0 && r_out != r_in && r_in && r_out)
+    if (run && T > 0 && r_out != r_in && r_in && r_out)
       return cuda_status(cudaMemcpyAsync(r_out, r_in, (size_t)T * H * 4, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
     return MOE_OK;
   }
@@ -448,6 +483,10 @@ moe_status moe_stack_forward(const float *r_in, int32_t T, int32_t L, const floa
   for (int l = 0; l < L; ++l)
     if (!aligned16(Wr[l]) || (bias && bias[l] && !aligned16(bias[l]))) return MOE_ERR_ALIGNMENT;
   uint16_t *u = at<uint16_t>(ws, LY.u16);
+  // what the layer entry point checks besides (the path and whether it takes this shape)
+  st = layer_forward_impl(u, T, Wr[0], bias ? bias[0] : nullptr, desc, &routed[0], hs ? &shared[0] : nullptr, r_out,
+                          r_out, nullptr, nullptr, path, ws, ws_bytes, stream, false);
+  if (st != MOE_OK || !run) return st;
   cudaStream_t s = (cudaStream_t)stream;
   // decode-sized batches: one launch of the fused layer kernel per layer, RMSNorm inside it (a
   // single launch walking all the layers with a grid barrier between them measured slower:
@@ -470,6 +509,35 @@ moe_status moe_stack_forward(const float *r_in, int32_t T, int32_t L, const floa
     if (st != MOE_OK) return st;
   }
   return MOE_OK;
+}
+
+moe_status moe_stack_forward(const float *r_in, int32_t T, int32_t L, const float *const *Wr,
+                             const float *const *bias, const moe_layer_desc *desc, const moe_expert_set *routed,
+                             const moe_expert_set *shared, float eps, float *r_out, int32_t path, void *ws,
+                             size_t ws_bytes, void *stream) {
+  return stack_forward_impl(r_in, T, L, Wr, bias, desc, routed, shared, eps, r_out, path, ws, ws_bytes, stream, true);
+}
+
+moe_status moe_stack_forward_host(const float *r_in_host, int32_t T, int32_t L, const float *const *Wr,
+                                  const float *const *bias, const moe_layer_desc *desc, const moe_expert_set *routed,
+                                  const moe_expert_set *shared, float eps, float *r_out_host, int32_t path, void *ws,
+                                  size_t ws_bytes, void *stream) {
+  if (!desc || T < 0 || L < 0) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!r_in_host || !r_out_host)) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && !ws) return MOE_ERR_WORKSPACE;
+  const int H = desc->H;
+  float *rd = T > 0 ? at<float>(ws, ws_layout(H, desc->E, desc->k, desc->I, desc->has_shared ? 1 : 0, T).yio)
+                    : nullptr;
+  // the stack runs in place on the staged stream (each layer reads its input rows before
+  // writing them)
+  moe_status st = stack_forward_impl(rd, T, L, Wr, bias, desc, routed, shared, eps, rd, path, ws, ws_bytes, stream,
+                                     false);
+  if (st != MOE_OK || T == 0) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(rd, r_in_host, (size_t)T * H * 4, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
+  st = stack_forward_impl(rd, T, L, Wr, bias, desc, routed, shared, eps, rd, path, ws, ws_bytes, stream, true);
+  if (st != MOE_OK) return st;
+  return cuda_status(cudaMemcpyAsync(r_out_host, rd, (size_t)T * H * 4, cudaMemcpyDeviceToHost, s));
 }
 
 moe_status moe_dequant_rows(const moe_qmat *m, int32_t expert, int32_t row0, int32_t nrows, float *out_f32,

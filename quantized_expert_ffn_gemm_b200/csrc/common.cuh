@@ -82,7 +82,7 @@ __host__ __device__ constexpr int mid_unit_tokens(int H) { return H <= 2048 ? 32
 // ---------------------------------------------------------------- workspace layout
 struct WsLayout {
   size_t ctrl, logits, idx, w, hist, units, hdec, counts, offsets, row_of, src, xperm, hperm, operm, u16, tiles, wsplit,
-      dx, mid, total;
+      dx, mid, xio, yio, total;
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -120,6 +120,8 @@ inline WsLayout ws_layout(int H, int E, int k, int I, int has_shared, int T) {
     const size_t tm = (size_t)(T < kMidMaxT ? T : kMidMaxT);
     L.mid = take(I % kMidFS == 0 ? (size_t)(I / kMidFS) * tm * (size_t)(k + has_shared) * H * 4 : 0);
   }
+  L.xio = take((size_t)T * H * 2);  // host-buffer entry points: the tokens, and y or the residual stream
+  L.yio = take((size_t)T * H * 4);
   L.total = off;
   return L;
 }

@@ -142,6 +142,37 @@ def test_stack_validation(lib):
                                  FAKE, ctypes.c_size_t(1 << 40), None) == 1
 
 
+def _lfh(lib, T=1, desc=None, routed=None, x_host=FAKE, y_host=FAKE, ws=FAKE, wsb=1 << 40, path=0):
+    desc = desc or _desc()
+    routed = routed or _set()
+    return lib.moe_layer_forward_host(x_host, T, FAKE, None, ctypes.byref(desc), ctypes.byref(routed), None, y_host,
+                                      None, None, path, ws, ctypes.c_size_t(wsb), None)
+
+
+def test_host_buffer_entry_points_validate_before_enqueueing(lib):
+    # every rejection comes from the host checks that run before the first copy is enqueued
+    assert _lfh(lib, T=0) == moe.MOE_OK
+    assert _lfh(lib, T=-1) == moe.MOE_ERR_INVALID_ARG
+    assert _lfh(lib, x_host=None) == moe.MOE_ERR_INVALID_ARG
+    assert _lfh(lib, y_host=None) == moe.MOE_ERR_INVALID_ARG
+    assert _lfh(lib, ws=None) == moe.MOE_ERR_WORKSPACE
+    assert _lfh(lib, wsb=1024) == moe.MOE_ERR_WORKSPACE
+    assert _lfh(lib, path=5) == moe.MOE_ERR_INVALID_ARG
+    assert _lfh(lib, desc=_desc(H=2016)) == moe.MOE_ERR_UNSUPPORTED
+    assert _lfh(lib, T=129, path=4) == moe.MOE_ERR_UNSUPPORTED
+    assert _lfh(lib, routed=_set(qtype=3)) == moe.MOE_ERR_INVALID_ARG
+    d = _desc()
+    eps = ctypes.c_float(1e-6)
+    assert lib.moe_stack_forward_host(None, 4, 2, None, None, ctypes.byref(d), None, None, eps, FAKE, 0, FAKE,
+                                      ctypes.c_size_t(1 << 40), None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_stack_forward_host(FAKE, 4, 2, None, None, ctypes.byref(d), None, None, eps, FAKE, 0, FAKE,
+                                      ctypes.c_size_t(1 << 40), None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_stack_forward_host(FAKE, 4, 2, None, None, ctypes.byref(d), None, None, eps, FAKE, 0, None,
+                                      ctypes.c_size_t(1 << 40), None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_stack_forward_host(FAKE, 0, 2, None, None, ctypes.byref(d), None, None, eps, FAKE, 0, FAKE,
+                                      ctypes.c_size_t(1 << 40), None) == moe.MOE_OK
+
+
 def test_static_router_validation(lib):
     # host-side checks of the workspace-free router; none of these calls reaches the device
     def call(x=FAKE, T=1, H=2048, Wr=FAKE, E=512, k=10, idx=FAKE, w=FAKE):

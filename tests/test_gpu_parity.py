@@ -372,3 +372,40 @@ def test_mmq_rejects_formats_it_does_not_take():
     with pytest.raises(moe.MoeError) as ei:
         moe.layer_forward(x, Wr, b, routed, shared, s.k, ws, path=moe.PATH_MMQ)
     assert ei.value.code == moe.MOE_ERR_UNSUPPORTED
+
+
+# ----------------------------------------------------------------------------- host-buffer entry points
+@pytest.mark.parametrize("name,T,path", [("decode1", 1, moe.PATH_AUTO), ("decode4", 4, moe.PATH_AUTO),
+                                         ("mid", 32, moe.PATH_MID), ("mid", 300, moe.PATH_AUTO)])
+def test_layer_forward_host_buffers_match_the_device_call(name, T, path):
+    # the tokens and y in page-locked host memory, one C call enqueuing copy, layer, copy: the
+    # same y, bit for bit, as the device-pointer call
+    L, (x, Wr, b, routed, shared) = layer_of(name)
+    s = L.shape
+    x = x[:T].contiguous()
+    ws = moe.Workspace.for_layer(s.H, s.E, s.k, s.I, s.shared, T)
+    h = moe.LayerHandle(Wr, b, routed, shared, s.k, ws)
+    y_dev = torch.empty(T, s.H, dtype=torch.float32, device="cuda")
+    h.forward(x, y_dev, path=path)
+    x_host = x.cpu().pin_memory()
+    y_host = torch.full((T, s.H), float("nan"), dtype=torch.float32).pin_memory()
+    h.forward_host(x_host, y_host, path=path)
+    torch.cuda.synchronize()
+    assert moe.read_device_error(ws) == 0
+    assert torch.equal(y_host, y_dev.cpu())
+
+
+def test_stack_forward_host_buffers_match_the_device_call():
+    H, E, k, I, Lyr, T = 256, 16, 2, 128, 3, 5
+    Wrs = [synth.make_router(0, l, E, H).cuda() for l in range(Lyr)]
+    rs = [synth.make_expert_set(0, l, 0, 2, E, H, I, "cuda") for l in range(Lyr)]
+    ss = [synth.make_expert_set(0, l, 1, 2, 1, H, I, "cuda") for l in range(Lyr)]
+    st = moe.Stack(Wrs, None, rs, ss, k)
+    ws = moe.Workspace.for_layer(H, E, k, I, True, T)
+    r0 = synth.make_residual(4, T, H)
+    dev = moe.stack_forward(r0.cuda(), st, ws).cpu()
+    r_host = r0.clone().pin_memory()
+    moe.stack_forward_host(r_host, st, ws, r_out_host=r_host)  # in place on the host buffer
+    torch.cuda.synchronize()
+    assert moe.read_device_error(ws) == 0
+    assert torch.equal(r_host, dev)
