@@ -434,6 +434,33 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
                             ws, ws_bytes, stream, true);
 }
 
+// Host <-> workspace copies of the host-buffer entry points: up to kSmallIo bytes between a
+// device-mapped page-locked host buffer and the workspace run as a copy kernel (a few
+// microseconds less latency per transfer than a copy-engine transfer); anything else, pageable
+// memory included, through cudaMemcpyAsync.
+constexpr size_t kSmallIo = 256 * 1024;
+
+static const void *mapped_host(const void *p, size_t bytes) {
+  if (bytes > kSmallIo || bytes % 16 != 0 || !aligned16(p)) return nullptr;
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return (at.type == cudaMemoryTypeHost && at.devicePointer && aligned16(at.devicePointer)) ? at.devicePointer
+                                                                                            : nullptr;
+}
+
+static cudaError_t copy_in(void *dst_dev, const void *src_host, size_t bytes, cudaStream_t s) {
+  if (const void *d = mapped_host(src_host, bytes)) return launch_io_copy(d, dst_dev, bytes, true, s);
+  return cudaMemcpyAsync(dst_dev, src_host, bytes, cudaMemcpyHostToDevice, s);
+}
+
+static cudaError_t copy_out(void *dst_host, const void *src_dev, size_t bytes, cudaStream_t s) {
+  if (const void *d = mapped_host(dst_host, bytes)) return launch_io_copy(src_dev, const_cast<void *>(d), bytes, false, s);
+  return cudaMemcpyAsync(dst_host, src_dev, bytes, cudaMemcpyDeviceToHost, s);
+}
+
 moe_status moe_layer_forward_host(const uint16_t *x_host, int32_t T, const float *Wr, const float *bias,
                                   const moe_layer_desc *desc, const moe_expert_set *routed,
                                   const moe_expert_set *shared_opt, float *y_host, int32_t *idx_out_opt,
@@ -449,11 +476,11 @@ moe_status moe_layer_forward_host(const uint16_t *x_host, int32_t T, const float
                                      path, ws, ws_bytes, stream, false);
   if (st != MOE_OK || T == 0) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  if (cudaMemcpyAsync(xd, x_host, (size_t)T * H * 2, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (copy_in(xd, x_host, (size_t)T * H * 2, s) != cudaSuccess) return MOE_ERR_CUDA;
   st = layer_forward_impl(xd, T, Wr, bias, desc, routed, shared_opt, nullptr, yd, idx_out_opt, w_out_opt, path, ws,
                           ws_bytes, stream, true);
   if (st != MOE_OK) return st;
-  return cuda_status(cudaMemcpyAsync(y_host, yd, (size_t)T * H * 4, cudaMemcpyDeviceToHost, s));
+  return cuda_status(copy_out(y_host, yd, (size_t)T * H * 4, s));
 }
 
 // the stack's argument checks and, with run set, its work (as layer_forward_impl)
@@ -534,10 +561,10 @@ moe_status moe_stack_forward_host(const float *r_in_host, int32_t T, int32_t L, 
                                      false);
   if (st != MOE_OK || T == 0) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  if (cudaMemcpyAsync(rd, r_in_host, (size_t)T * H * 4, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (copy_in(rd, r_in_host, (size_t)T * H * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
   st = stack_forward_impl(rd, T, L, Wr, bias, desc, routed, shared, eps, rd, path, ws, ws_bytes, stream, true);
   if (st != MOE_OK) return st;
-  return cuda_status(cudaMemcpyAsync(r_out_host, rd, (size_t)T * H * 4, cudaMemcpyDeviceToHost, s));
+  return cuda_status(copy_out(r_out_host, rd, (size_t)T * H * 4, s));
 }
 
 moe_status moe_dequant_rows(const moe_qmat *m, int32_t expert, int32_t row0, int32_t nrows, float *out_f32,

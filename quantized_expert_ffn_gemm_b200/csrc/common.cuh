@@ -231,6 +231,10 @@ cudaError_t launch_mid_ffn(const uint16_t *x, int T, int H, int E, int k, int I,
                            const moe_expert_set &routed, const moe_expert_set *shared, const float *residual, float *y,
                            MidUnit *units, int32_t *row_of, int32_t *row_tok, float *part, Ctrl *ctrl, cudaStream_t s);
 
+// copy `bytes` (a multiple of 16, both ends 16-byte aligned and device-addressable) with a kernel;
+// early: the source is read before the wait for the previous kernel on the stream
+cudaError_t launch_io_copy(const void *src, void *dst, size_t bytes, bool early, cudaStream_t s);
+
 // whether launch_decode_fused takes this shape on the current device
 bool decode_fused_fits(int T, int H, int E, int k, int I, const moe_expert_set &routed, bool has_shared);
 

@@ -361,7 +361,6 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   // parity of fill q's phase: one phase per fill q, q + R, ... of the slot
   auto fill_parity = [&](int q) { return (uint32_t)(q / R) & 1u; };
   bool ok = true;
-  const float *const lWr = a.Wr;
   const float *const lbias = a.bias;
   const moe_expert_set &lRS = a.routed;
   const moe_expert_set &lSS = a.shared;
@@ -1089,31 +1088,44 @@ static bool fused_plan(int T, int H, int E, int k, int I, const moe_expert_set &
   return true;
 }
 
-bool decode_fused_fits(int T, int H, int E, int k, int I, const moe_expert_set &routed, bool has_shared) {
-  // answers are kept per (device, shape): the plan queries the occupancy calculator
-  struct Seen {
+// fused_plan, kept per (device, shape): the plan queries the occupancy calculator and raises the
+// kernel's shared-memory limit, host work a decode step should not repeat
+static bool fused_plan_cached(int T, int H, int E, int k, int I, const moe_expert_set &routed, bool has_shared,
+                              FusedArgs &a, const void *&fn, size_t &smem) {
+  struct Plan {
     int dev, T, H, E, k, I, qt, sh;
     bool ok;
+    FusedArgs a;
+    const void *fn;
+    size_t smem;
   };
   static std::mutex mu;
-  static std::vector<Seen> seen;
+  static std::vector<Plan> plans;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   const int qt = routed.gate.qtype, sh = has_shared ? 1 : 0;
   {
     std::lock_guard<std::mutex> lk(mu);
-    for (const Seen &q : seen)
-      if (q.dev == dev && q.T == T && q.H == H && q.E == E && q.k == k && q.I == I && q.qt == qt && q.sh == sh)
+    for (const Plan &q : plans)
+      if (q.dev == dev && q.T == T && q.H == H && q.E == E && q.k == k && q.I == I && q.qt == qt && q.sh == sh) {
+        a = q.a;
+        fn = q.fn;
+        smem = q.smem;
         return q.ok;
+      }
   }
-  FusedArgs a;
-  const void *fn = nullptr;
-  size_t smem = 0;
   const bool ok = fused_plan(T, H, E, k, I, routed, has_shared, a, fn, smem);
   if (!ok) (void)cudaGetLastError();
   std::lock_guard<std::mutex> lk(mu);
-  if (seen.size() < 4096) seen.push_back({dev, T, H, E, k, I, qt, sh, ok});
+  if (plans.size() < 4096) plans.push_back({dev, T, H, E, k, I, qt, sh, ok, a, fn, smem});
   return ok;
+}
+
+bool decode_fused_fits(int T, int H, int E, int k, int I, const moe_expert_set &routed, bool has_shared) {
+  FusedArgs a;
+  const void *fn = nullptr;
+  size_t smem = 0;
+  return fused_plan_cached(T, H, E, k, I, routed, has_shared, a, fn, smem);
 }
 
 static cudaError_t fused_launch(const void *fn, size_t smem, void **args, cudaStream_t s) {
@@ -1145,10 +1157,7 @@ cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float ep
   FusedArgs a;
   const void *fn = nullptr;
   size_t smem = 0;
-  if (!fused_plan(T, H, E, k, I, routed, shared != nullptr, a, fn, smem)) {
-    (void)cudaGetLastError();
-    return cudaErrorNotSupported;
-  }
+  if (!fused_plan_cached(T, H, E, k, I, routed, shared != nullptr, a, fn, smem)) return cudaErrorNotSupported;
   a.x = x;
   a.r_norm = r_norm;
   a.eps = eps;

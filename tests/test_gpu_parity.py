@@ -375,11 +375,13 @@ def test_mmq_rejects_formats_it_does_not_take():
 
 
 # ----------------------------------------------------------------------------- host-buffer entry points
+@pytest.mark.parametrize("pinned", [True, False])
 @pytest.mark.parametrize("name,T,path", [("decode1", 1, moe.PATH_AUTO), ("decode4", 4, moe.PATH_AUTO),
                                          ("mid", 32, moe.PATH_MID), ("mid", 300, moe.PATH_AUTO)])
-def test_layer_forward_host_buffers_match_the_device_call(name, T, path):
-    # the tokens and y in page-locked host memory, one C call enqueuing copy, layer, copy: the
-    # same y, bit for bit, as the device-pointer call
+def test_layer_forward_host_buffers_match_the_device_call(name, T, path, pinned):
+    # the tokens and y in host memory, one C call enqueuing copy, layer, copy: the same y, bit for
+    # bit, as the device-pointer call (page-locked buffers move by a copy kernel when small,
+    # pageable ones by cudaMemcpyAsync)
     L, (x, Wr, b, routed, shared) = layer_of(name)
     s = L.shape
     x = x[:T].contiguous()
@@ -387,8 +389,10 @@ def test_layer_forward_host_buffers_match_the_device_call(name, T, path):
     h = moe.LayerHandle(Wr, b, routed, shared, s.k, ws)
     y_dev = torch.empty(T, s.H, dtype=torch.float32, device="cuda")
     h.forward(x, y_dev, path=path)
-    x_host = x.cpu().pin_memory()
-    y_host = torch.full((T, s.H), float("nan"), dtype=torch.float32).pin_memory()
+    x_host = x.cpu()
+    y_host = torch.full((T, s.H), float("nan"), dtype=torch.float32)
+    if pinned:
+        x_host, y_host = x_host.pin_memory(), y_host.pin_memory()
     h.forward_host(x_host, y_host, path=path)
     torch.cuda.synchronize()
     assert moe.read_device_error(ws) == 0
