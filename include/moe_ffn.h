@@ -239,8 +239,9 @@ moe_status moe_layer_forward(const uint16_t *x, int32_t T, const float *Wr, cons
 /* moe_layer_forward with the tokens and the output in HOST memory: x_host bf16 [T,H] is copied to
  * the workspace, the layer runs on it (no residual), and y lands in y_host fp32 [T,H]; one call
  * enqueues the host-to-device copy, the layer and the device-to-host copy on `stream` and returns
- * (the copies are asynchronous for page-locked host buffers; y_host is complete once the stream
- * has reached this point). The weights, the workspace and the optional routing outputs stay in
+ * (the copies are asynchronous for page-locked host buffers, and those of up to 256 KB run as a
+ * copy kernel reading or writing the mapped host buffer; y_host is complete once the stream has
+ * reached this point). The weights, the workspace and the optional routing outputs stay in
  * device memory; other arguments and errors as moe_layer_forward (MOE_ERR_INVALID_ARG for a
  * NULL x_host or y_host). */
 moe_status moe_layer_forward_host(const uint16_t *x_host, int32_t T, const float *Wr, const float *bias,
