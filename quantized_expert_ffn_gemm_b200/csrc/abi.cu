@@ -147,16 +147,12 @@ T *at(void *ws, size_t off) {
   return reinterpret_cast<T *>(static_cast<unsigned char *>(ws) + off);
 }
 
-// Groups of at most this many rows would take the dequant-GEMV kernels under AUTO and the larger
-// ones the tcgen05 grouped GEMM. A GEMM tile costs about the same whatever its row count up to
-// ~96 rows (measured), so small groups waste most of a tile there; but the GEMV kernels measured
-// slower still on the small groups of a skewed 2048-token layer (0.53 against 0.39 ms for the
-// layer) and at 12-128 tokens, so the split is off (0) and AUTO runs every group on the GEMM.
-constexpr int kSmallGroupRows = 0;
-
 // Expert FFN over expert-contiguous rows by path: GEMM (every group on the grouped GEMM), GEMV
-// (every group on the GEMV kernels), AUTO with the GEMM available: small groups on the GEMV
-// kernels and the rest on the grouped GEMM (disjoint rows of out_perm).
+// (every group on the GEMV kernels), MMQ (int8 gate/up, fp16 down), AUTO: the grouped GEMM where
+// it takes the shape. (Splitting AUTO by group size, small groups on the GEMV kernels, was
+// measured: a GEMM tile costs about the same whatever its row count up to ~96 rows, but the GEMV
+// kernels were slower still on the small groups of a skewed 2048-token layer, 0.53 against
+// 0.39 ms, and at 12-128 tokens.)
 cudaError_t expert_rows(const uint16_t *xperm, const int32_t *offsets, int rows, int E, int H, int I,
                         const moe_expert_set &routed, const moe_expert_set *sh, uint16_t *hperm, uint16_t *operm,
                         int2 *tiles, DecUnit *units, uint16_t *hdec, Ctrl *ctrl, cudaStream_t s, int path, bool gemm_ok,
@@ -167,18 +163,12 @@ cudaError_t expert_rows(const uint16_t *xperm, const int32_t *offsets, int rows,
     if (e == cudaSuccess) e = launch_grouped_down(hperm, offsets, rows, E, H, I, routed, sh, operm, tiles, ctrl, s);
     return e;
   }
-  const bool hybrid = path == MOE_PATH_AUTO && gemm_ok && kSmallGroupRows > 0;
-  if (path == MOE_PATH_AUTO && gemm_ok && !hybrid) path = MOE_PATH_GEMM;
-  cudaError_t e = cudaSuccess;
-  if (path == MOE_PATH_GEMM || hybrid) {
-    e = launch_grouped_ffn(xperm, offsets, rows, E, H, I, routed, sh, hperm, operm, tiles, ctrl, s,
-                           hybrid ? kSmallGroupRows : 0);
-    if (e != cudaSuccess || !hybrid) return e;
-  }
+  if (path == MOE_PATH_AUTO && gemm_ok) path = MOE_PATH_GEMM;
+  if (path == MOE_PATH_GEMM)
+    return launch_grouped_ffn(xperm, offsets, rows, E, H, I, routed, sh, hperm, operm, tiles, ctrl, s);
   // a group of n rows makes ceil(n / 8) units: at most rows / 8 + (non-empty groups) in all
   const int max_units = (rows + 7) / 8 + (n_groups < rows ? n_groups : rows);
-  e = launch_decode_units_from_offsets(offsets, n_groups, sh ? 1 : 0, rows, units, ctrl, s,
-                                       hybrid ? kSmallGroupRows : 0);
+  cudaError_t e = launch_decode_units_from_offsets(offsets, n_groups, sh ? 1 : 0, rows, units, ctrl, s);
   if (e == cudaSuccess) e = launch_decode_gate_up(xperm, 0, H, I, routed, sh, units, max_units, ctrl, hdec, s);
   if (e == cudaSuccess)
     e = launch_decode_down(H, I, routed, sh, units, max_units, ctrl, hdec, nullptr, nullptr, 0, operm, s);

@@ -200,9 +200,8 @@ cudaError_t launch_dequant_rows(const moe_qmat &m, int expert, int row0, int nro
                                 cudaStream_t s);
 
 // decode path: units are read from `units` (count in ctrl->n_units, at most max_units)
-// (groups of more than max_rows rows are skipped when max_rows > 0)
 cudaError_t launch_decode_units_from_offsets(const int32_t *offsets, int n_groups, int has_shared_group, int n_rows,
-                                             DecUnit *units, Ctrl *ctrl, cudaStream_t s, int max_rows = 0);
+                                             DecUnit *units, Ctrl *ctrl, cudaStream_t s);
 cudaError_t launch_decode_gate_up(const void *x, int x_is_bf16, int H, int I, const moe_expert_set &routed,
                                   const moe_expert_set *shared, const DecUnit *units, int max_units, Ctrl *ctrl,
                                   uint16_t *hdec, cudaStream_t s);
@@ -244,10 +243,10 @@ cudaError_t launch_wait_starve(Ctrl *ctrl, uint64_t limit_ns, cudaStream_t s);
 
 // prefill path (tcgen05 grouped GEMM)
 int gemm_shape_supported(int H, int I);
-// tile list (group, first row) of slice-row slices (a multiple of 16, <= 192) of every group of
-// more than min_rows rows, longest slices first; count in ctrl->n_tiles
+// tile list (group, first row) of slice-row slices (a multiple of 16, <= 192) of every group,
+// longest slices first; count in ctrl->n_tiles
 cudaError_t launch_tile_list(const int32_t *offsets, int n_groups, int n_rows, int slice, int2 *tiles, Ctrl *ctrl,
-                             cudaStream_t s, int min_rows = 0);
+                             cudaStream_t s);
 // int8-activation (MMQ-style) gate/up + SwiGLU on tcgen05 kind::i8, Q2 weights: x_perm is
 // quantized per 32-value block into x_q [n_rows][H] int8 and dx [n_rows][H/32] fp32 (scratch),
 // h_perm as the fp16 path writes it
@@ -259,10 +258,9 @@ cudaError_t launch_mmq_gate_up(const uint16_t *x_perm, const int32_t *offsets, i
 cudaError_t launch_grouped_down(const uint16_t *h_perm, const int32_t *offsets, int n_rows, int E, int H, int I,
                                 const moe_expert_set &routed, const moe_expert_set *shared, uint16_t *out_perm,
                                 int2 *tiles, Ctrl *ctrl, cudaStream_t s);
-// groups of at most min_rows rows are skipped (min_rows > 0: the caller runs them on the GEMV path)
 cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, int n_rows, int E, int H, int I,
                                const moe_expert_set &routed, const moe_expert_set *shared, uint16_t *h_perm,
-                               uint16_t *out_perm, int2 *tiles, Ctrl *ctrl, cudaStream_t s, int min_rows = 0);
+                               uint16_t *out_perm, int2 *tiles, Ctrl *ctrl, cudaStream_t s);
 
 int num_sms();
 // (pdl_enabled: programmatic dependent launches are on unless the environment sets MOE_PDL=0)

@@ -327,8 +327,7 @@ cudaError_t launch_decode_down(int H, int I, const moe_expert_set &routed, const
 }
 
 // ---------------------------------------------------------------- units for grouped rows
-// rows mode for moe_expert_ffn: group g's rows [off[g], off[g+1]) in chunks of 8 columns (only
-// groups of at most max_rows rows when max_rows > 0: the larger ones go to the grouped GEMM). One
+// rows mode for moe_expert_ffn: group g's rows [off[g], off[g+1]) in chunks of 8 columns. One
 // CTA: each thread takes a group, a block-wide exclusive scan of the groups' chunk counts gives
 // each group's first unit, and the groups are walked in blocks of kUnitsThreads. Units come out
 // in group order, then row order, as a serial walk would produce them.
@@ -336,7 +335,7 @@ constexpr int kUnitsThreads = 1024;
 
 __global__ void __launch_bounds__(kUnitsThreads)
 units_from_offsets_kernel(const int32_t *__restrict__ off, int n_groups, int shared_group, int n_rows,
-                          int max_rows, DecUnit *__restrict__ units, Ctrl *__restrict__ ctrl) {
+                          DecUnit *__restrict__ units, Ctrl *__restrict__ ctrl) {
   __shared__ int s_warp[kUnitsThreads / 32];
   __shared__ int s_base, s_bad;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -363,7 +362,7 @@ units_from_offsets_kernel(const int32_t *__restrict__ off, int n_groups, int sha
     if (gi < n_groups) {
       a = off[gi];
       nrow = off[gi + 1] - a;
-      cnt = (max_rows > 0 && nrow > max_rows) ? 0 : (nrow + 7) / 8;  // larger groups: the grouped GEMM
+      cnt = (nrow + 7) / 8;
     }
     int incl = cnt;
 #pragma unroll
@@ -403,11 +402,11 @@ units_from_offsets_kernel(const int32_t *__restrict__ off, int n_groups, int sha
 }
 
 cudaError_t launch_decode_units_from_offsets(const int32_t *offsets, int n_groups, int has_shared_group, int n_rows,
-                                             DecUnit *units, Ctrl *ctrl, cudaStream_t s, int max_rows) {
+                                             DecUnit *units, Ctrl *ctrl, cudaStream_t s) {
   {
     KTimer kt_(KID_DEC_UNITS, s);
     units_from_offsets_kernel<<<1, kUnitsThreads, 0, s>>>(offsets, n_groups, has_shared_group ? n_groups - 1 : -1,
-                                                          n_rows, max_rows, units, ctrl);
+                                                          n_rows, units, ctrl);
   }
   return cudaGetLastError();
 }

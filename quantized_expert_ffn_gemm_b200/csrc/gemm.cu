@@ -475,11 +475,11 @@ grouped_v2_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
 // take a handful, and the long tiles no longer land at the tail. Within a size class the order
 // is whatever the shared-memory cursors give; it does not change any result (every tile writes
 // its own output rows). Offsets that are not monotone or run past n_rows flag the error word and
-// yield no tiles. Groups of at most min_rows rows get no tiles (the caller runs them elsewhere).
+// yield no tiles.
 constexpr int kTileClasses = kBNMax / 16;  // N granules 1..12
 
 __global__ void __launch_bounds__(1024) tile_list_kernel(const int32_t *__restrict__ off, int G, int n_rows,
-                                                         int min_rows, int slice, int2 *__restrict__ tiles,
+                                                         int slice, int2 *__restrict__ tiles,
                                                          Ctrl *__restrict__ ctrl) {
   const int nclass = slice / 16;  // <= kTileClasses
   __shared__ int s_cnt[kTileClasses + 1], s_cur[kTileClasses + 1];
@@ -501,7 +501,6 @@ __global__ void __launch_bounds__(1024) tile_list_kernel(const int32_t *__restri
   // size class of a slice with n rows (1..slice): ceil(n / 16), 1..nclass
   for (int g = tid; g < G; g += blockDim.x) {
     const int n = off[g + 1] - off[g];
-    if (n <= min_rows) continue;  // left to the small-group path
     if (n >= slice) atomicAdd(&s_cnt[nclass], n / slice);
     if (n % slice) atomicAdd(&s_cnt[(n % slice + 15) / 16], 1);
   }
@@ -517,7 +516,6 @@ __global__ void __launch_bounds__(1024) tile_list_kernel(const int32_t *__restri
   __syncthreads();
   for (int g = tid; g < G; g += blockDim.x) {
     const int n = off[g + 1] - off[g];
-    if (n <= min_rows) continue;
     const int full = n / slice;
     if (full) {
       const int p = atomicAdd(&s_cur[nclass], full);
@@ -588,11 +586,11 @@ bool encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dt, int esize, c
 }
 
 cudaError_t launch_tile_list(const int32_t *offsets, int n_groups, int n_rows, int slice, int2 *tiles, Ctrl *ctrl,
-                             cudaStream_t s, int min_rows) {
+                             cudaStream_t s) {
   if (slice < 16 || slice > kBNMax || slice % 16) return cudaErrorInvalidValue;
   {
     KTimer kt_(KID_TILE_LIST, s);
-    tile_list_kernel<<<1, 1024, 0, s>>>(offsets, n_groups, n_rows, min_rows, slice, tiles, ctrl);
+    tile_list_kernel<<<1, 1024, 0, s>>>(offsets, n_groups, n_rows, slice, tiles, ctrl);
   }
   return cudaGetLastError();
 }
@@ -601,10 +599,10 @@ int gemm_shape_supported(int H, int I) { return (H % 128 == 0 && I % 128 == 0 &&
 
 cudaError_t launch_grouped_ffn(const uint16_t *x_perm, const int32_t *offsets, int n_rows, int E, int H, int I,
                                const moe_expert_set &routed, const moe_expert_set *shared, uint16_t *h_perm,
-                               uint16_t *out_perm, int2 *tiles, Ctrl *ctrl, cudaStream_t s, int min_rows) {
+                               uint16_t *out_perm, int2 *tiles, Ctrl *ctrl, cudaStream_t s) {
   const int G = E + (shared ? 1 : 0);
   const moe_expert_set &sh = shared ? *shared : routed;
-  cudaError_t e = launch_tile_list(offsets, G, n_rows, kBNMax, tiles, ctrl, s, min_rows);
+  cudaError_t e = launch_tile_list(offsets, G, n_rows, kBNMax, tiles, ctrl, s);
   if (e != cudaSuccess) return e;
 
   CUtensorMap tx, th, cg, cu, cd, sg, su, sd;
