@@ -284,7 +284,7 @@ moe_status moe_dequant_rows(const moe_qmat *m, int32_t expert, int32_t row0, int
  * word and the [T][E] fp32 logits -- is a fixed array inside the library (about 128 KB, held on
  * every GPU that loads the library until the process exits). Limits: T <= 8, E <= 4096 (and
  * T * max(H, E) * 4 <= 200 KB); larger requests return MOE_ERR_UNSUPPORTED. The first call on
- * each device looks up the array's device address and should come before any stream capture.
+ * each device looks up the array's device address (a host-side runtime query, kept per device).
  * All calls share the array, which keeps the last call's contents (each call clears what must
  * start at zero): calls that overlap on the GPU race and must be serialised by the caller. The
  * router kernel records no device-side error, so the array's error word needs no reader. It

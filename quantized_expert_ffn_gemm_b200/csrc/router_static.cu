@@ -9,8 +9,8 @@
 //
 // The array lives in every GPU that loads the library until the process exits. In host code the
 // array's name is only a host-side stand-in, so its device address is looked up once per device
-// (cudaGetSymbolAddress, with that device current) on the first call; that first call should
-// therefore come before any stream capture. All calls share the one array: calls that overlap on
+// (cudaGetSymbolAddress, with that device current) on the first call and kept in a per-device
+// table. All calls share the one array: calls that overlap on
 // the GPU (different streams, or different host threads) race on it and must be serialised by
 // the caller.
 //
