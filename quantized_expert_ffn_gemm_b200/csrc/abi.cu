@@ -370,8 +370,8 @@ static moe_status layer_forward_impl(const uint16_t *x, int32_t T, const float *
     // does not take): separate router / gate-up / down kernels
     e = cudaErrorNotSupported;
     if (path == MOE_PATH_AUTO) {
-      e = launch_decode_fused(x, nullptr, 0.0f, T, H, Wr, bias, E, k, I, *routed, sh, residual_opt, y, idx, w, hdec,
-                              ctrl, s);
+      e = launch_decode_fused(x, nullptr, 0.0f, T, H, Wr, bias, E, k, I, *routed, sh, residual_opt, y, idx, w, ctrl,
+                              s);
       if (e == cudaErrorCooperativeLaunchTooLarge) {
         (void)cudaGetLastError();
         e = cudaErrorNotSupported;
@@ -514,7 +514,7 @@ static moe_status stack_forward_impl(const float *r_in, int32_t T, int32_t L, co
     if (fused) {
       cudaError_t e = launch_decode_fused(nullptr, r, eps, T, H, Wr[l], bias ? bias[l] : nullptr, E, k, I, routed[l],
                                           hs ? &shared[l] : nullptr, r, r_out, at<int32_t>(ws, LY.idx),
-                                          at<float>(ws, LY.w), at<uint16_t>(ws, LY.hdec), at<Ctrl>(ws, LY.ctrl), s,
+                                          at<float>(ws, LY.w), at<Ctrl>(ws, LY.ctrl), s,
                                           l + 1 < L ? Wr[l + 1] : nullptr);
       if (e == cudaSuccess) continue;
       if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge) return cuda_status(e);

@@ -35,15 +35,24 @@ struct Ctrl {
 static_assert(sizeof(Ctrl) == 128, "control block is 128 bytes");
 
 // The fused decode kernel's exchange area, the rest of the control area (zeroed once by
-// moe_workspace_init and used by that kernel only): router logits as (launch tag << 32 | fp32 bits)
-// words that readers poll for their own launch's tag, per-unit readiness counters in two sets
-// used by alternate launches (a launch zeroes the other set for the next one), and each CTA's
-// count of the launches it has started (every launch runs one CTA per SM, so the counts agree).
-constexpr int kFusedMaxE = 512;   // experts the fused decode kernel takes
+// moe_workspace_init and used by that kernel only). Router logits cross CTAs as 64-bit words
+// (launch tag << 32 | fp32 bits) that readers poll until they carry their own launch's tag, so no
+// fence or counter is needed. The gate/up output h of one- and two-token launches goes the same
+// way (two fp16 values and the tag per word, one row of I / 2 words per (unit, token) column of
+// the down phase); larger launches, whose down phase reads several times more h, store plain fp16
+// rows and count each unit's items on a readiness counter (two sets used by alternate launches; a
+// launch zeroes the set the next one uses). Each CTA also keeps its count of the launches it has
+// started (every launch runs one CTA per SM, so the counts agree). Tags start at 1 on zeroed
+// memory, so no word left from earlier use carries a live tag.
+constexpr int kFusedMaxE = 512;     // experts the fused decode kernel takes
+constexpr int kFusedMaxCols = 96;   // (unit, token) h columns of one launch
 constexpr int kFusedMaxUnits = 128;
+constexpr int kFusedMaxI = 1024;    // intermediate size the fused decode kernel takes
 constexpr int kFusedMaxGrid = 256;  // CTAs of a fused launch (one per SM)
 struct FusedSync {
   unsigned long long logit[kDecodeMaxT * kFusedMaxE];
+  unsigned long long hword[kFusedMaxCols * (kFusedMaxI / 2)];  // tagged h (1-2 tokens)
+  uint16_t hval[kFusedMaxCols * kFusedMaxI];                   // plain h (3-8 tokens)
   unsigned ready[2][kFusedMaxUnits];
   unsigned seq[kFusedMaxGrid];  // per CTA: launches it has started (all equal between launches)
 };
@@ -219,8 +228,7 @@ cudaError_t launch_decode_down(int H, int I, const moe_expert_set &routed, const
 cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float eps, int T, int H, const float *Wr,
                                 const float *bias, int E, int k, int I, const moe_expert_set &routed,
                                 const moe_expert_set *shared, const float *residual, float *y, int32_t *idx,
-                                float *w, uint16_t *hdec, Ctrl *ctrl, cudaStream_t s,
-                                const float *next_Wr = nullptr);
+                                float *w, Ctrl *ctrl, cudaStream_t s, const float *next_Wr = nullptr);
 
 // mid-batch path (about 6..128 tokens; I % kMidFS == 0): units of <= 8 tokens per selected expert
 // built from the routing (no permutation), items (unit, kMidFS-feature slice) that run gate/up,

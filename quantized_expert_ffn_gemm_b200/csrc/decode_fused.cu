@@ -24,13 +24,15 @@
 //   P2  gate/up + SwiGLU: two groups of 8 warps take alternate items; in a group warp j runs
 //       K step j (256 wide) on the tensor cores (mma.sync m16n8k16 with A rows 0-7 = gate and
 //       8-15 = up rows of the same features, fp16 operands, fp32 accumulate); the partials are
-//       summed in fixed order, h goes to the workspace and the item is counted on its unit's
-//       readiness counter (a release add).
+//       summed in fixed order and h is published: at one or two tokens as tagged words (two fp16
+//       values and this launch's tag per 64-bit word, by atomic exchange: no fence, no counter);
+//       at more tokens, whose down phase reads several times more h, as plain fp16 followed by a
+//       release add on the unit's readiness counter.
 //   P3  down projection fused with the weighted combine: each CTA owns 16 output features, its
 //       warps take whole units (16 down rows over all of I, the half steps' loads issued
-//       together). A unit's warp waits only for that unit's counter to reach its item count (no
-//       second grid barrier: early units' down work overlaps later units' gate/up), stages the
-//       unit's h columns, and runs; partials are reduced in fixed order (no atomics).
+//       together). A unit's warp waits only for that unit's h (its tagged words, or its counter;
+//       no second grid barrier: early units' down work overlaps later units' gate/up), stages
+//       it, and runs; partials are reduced in fixed order (no atomics).
 // Each slot's fills are consumed in phase order: the ring has an even number of slots so the
 // gate/up items sharing a slot fall to one group, a CTA barrier separates a CTA's P2 from its
 // P3, and a down piece first waits until the piece one ring behind it is consumed. A parity wait
@@ -38,9 +40,10 @@
 // older phase for its own.
 // A launch's tag is its number + 1: every CTA keeps its own count of started launches in the
 // exchange area and advances it once per launch, so all CTAs of a launch agree on it (launches
-// do not overlap past griddepcontrol.wait). The readiness counters come in two sets used by alternate
-// launches; a launch zeroes the set the next one will use. The logit polls, the readiness waits
-// and every mbarrier wait are bounded in time and report MOE_ERR_TIMEOUT instead of hanging;
+// do not overlap past griddepcontrol.wait), and a word written by an earlier launch never carries
+// it. The readiness counters come in two sets used by alternate launches; a launch zeroes the set
+// the next one will use. The logit and h polls, the readiness waits and every mbarrier wait are
+// bounded in time and report MOE_ERR_TIMEOUT instead of hanging;
 // before the CTA exits every thread waits for its own outstanding copies (cp.async.wait_all), so
 // no copy is still writing its shared memory.
 #include "common.cuh"
@@ -58,7 +61,7 @@ namespace {
 
 constexpr int kFWarps = 16;
 constexpr int kFThreads = kFWarps * 32;
-constexpr int kFSlots = 96;                 // h columns (token, expert) of a step staged for the down phase
+constexpr int kFSlots = kFusedMaxCols;      // h columns (token, expert) of a step staged for the down phase
 constexpr int kFMaxUnits = kFSlots + 1;
 constexpr int kPairsPerLane = kFSlots / 32; // (token, slot) pairs per lane of the unit-list warp
 static_assert(kFMaxUnits <= kFusedMaxUnits, "readiness counters per unit");
@@ -83,8 +86,7 @@ struct FusedArgs {
   float *y;
   int32_t *idx;
   float *w;
-  uint16_t *hdec;
-  Ctrl *ctrl;       // control block; the exchange area (tagged logits, readiness counters) follows it
+  Ctrl *ctrl;       // control block; the exchange area (tagged logit and h words) follows it
   int ring;        // slots in the ring
   int slot_bytes;  // bytes per slot
   int gu_bytes;    // bytes of one gate/up item
@@ -341,8 +343,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   // This launch's tag: one more than the launches this CTA's slot has counted (each CTA reads and
   // advances only its own slot, and every launch advances every slot once, so all of a launch's
   // CTAs read the same count; launches do not overlap past the wait above). The tag marks this
-  // launch's logit words; its parity picks the set of readiness counters. The load's result is
-  // first needed after the tokens are staged.
+  // launch's logit and h words. The load's result is first needed after the tokens are staged.
   uint32_t launch_no = 0;
   if (tid == 0) {
     launch_no = *reinterpret_cast<volatile const uint32_t *>(&fs->seq[blockIdx.x]);
@@ -448,9 +449,11 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   }
   __syncthreads();
   const uint32_t tag = s_tag;
+  // h exchange: tagged words at one or two tokens, plain rows + per-unit readiness counters above
+  constexpr bool kTaggedH = TMAX <= 2;
   unsigned *const ready = fs->ready[tag & 1u];
   // the other set serves the next launch: the previous launch, its last user, has completed
-  if (blockIdx.x == 0)
+  if (!kTaggedH && blockIdx.x == 0)
     for (int u = tid; u < kFusedMaxUnits; u += kFThreads) fs->ready[(tag & 1u) ^ 1u][u] = 0u;
 
   // ---------------- P1: router logits, four warps per expert (each a quarter of H), fp32
@@ -835,9 +838,11 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
       named_sync(kBarGroup0 + grp, 256);
       // every warp of the group is done with the slot: its next fill goes out now
       if (j8 == 7 && q + R < n_total) issue_fill(q + R);
-      if (gtid < 64) {  // one (feature, token) per thread; fixed-order sums of the 8 K steps
+      if (gtid < 64) {  // one (feature, token) per thread (two whole warps); fixed-order sums of the 8 K steps
         const int row = gtid & 7, col = gtid >> 3;
-        if ((un.mask >> col) & 1) {
+        const bool present = (un.mask >> col) & 1;
+        uint32_t hb = 0u;
+        if (present) {
           const float *pb = part + ((size_t)(grp * 2 + buf) * 8 * 16) * 8;
           float gv = 0.f, uv = 0.f;
 #pragma unroll
@@ -846,15 +851,29 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
             uv += pb[(sl * 16 + 8 + row) * 8 + col];
           }
           const float hv = gv / (1.0f + expf(-gv)) * uv;
-          const uint16_t hb = __half_as_ushort(__float2half_rn(hv));
-          if (f16_inf(hb)) set_device_error(ctrl, MOE_ERR_RANGE, 5);
-          a.hdec[((size_t)u * 8 + col) * I + r0 + row] = hb;
+          hb = __half_as_ushort(__float2half_rn(hv));
+          if (f16_inf((uint16_t)hb)) set_device_error(ctrl, MOE_ERR_RANGE, 5);
+        }
+        const int slot = s_slot[u] + __popc(un.mask & ((1u << col) - 1u));
+        if constexpr (kTaggedH) {
+          // features row and row + 1 of a column go out as one tagged word: the word carries its
+          // own readiness, so neither a fence nor a counter is needed (an atomic exchange is
+          // performed at L2 at once)
+          const uint32_t hb1 = __shfl_down_sync(0xffffffffu, hb, 1);
+          if (present && (row & 1) == 0) {
+            const unsigned long long word = ((unsigned long long)tag << 32) | (hb1 << 16) | hb;
+            atomicExch(fs->hword + (size_t)slot * (I / 2) + (r0 + row) / 2, word);
+          }
+        } else if (present) {
+          fs->hval[(size_t)slot * I + r0 + row] = (uint16_t)hb;
         }
       }
-      // the item's h is written: count it for its unit (the group barrier orders the 64 stores
-      // before the release add, as in the grid barrier)
-      named_sync(kBarGroup0 + grp, 256);
-      if (gtid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ready + u) : "memory");
+      if constexpr (!kTaggedH) {
+        // the item's h is written: count it for its unit (the group barrier orders the 64 stores
+        // before the release add)
+        named_sync(kBarGroup0 + grp, 256);
+        if (gtid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ready + u) : "memory");
+      }
     }
   }
   // This CTA's gate/up items are all consumed (the ring rule of P3 below needs it); no grid
@@ -894,47 +913,100 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
         }
         const DecUnit &un = su[u];
         if (rbl == 0) {
-          // the unit's h: wait until all its gate/up items are counted (bounded), then stage its
-          // present columns (16-byte loads from L2); they stay for later row blocks
-          if (lane == 0) {
-            const uint64_t t0 = global_ns();
-            for (;;) {
-              unsigned v;
-              asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ready + u) : "memory");
-              if (v >= (unsigned)rbs8 || s_abort) break;
-              __nanosleep(32);
-              if (global_ns() - t0 > kWaitLimitNs) {
-                s_abort = 1;
-                set_device_error(ctrl, MOE_ERR_TIMEOUT, 45);
-                break;
+          if constexpr (kTaggedH) {
+            // the unit's h columns (contiguous column slots c0..): a lane's sixteen words are
+            // requested together and re-requested together (bounded) until every one carries this
+            // launch's tag, then their values go to the staged columns; they stay for later row blocks
+            const int I4 = I / 4, c0 = s_slot[u], nv = (s_slot[u + 1] - c0) * I4;
+            const unsigned long long *hw = fs->hword + (size_t)c0 * (I / 2);
+            for (int v0 = lane; v0 < nv; v0 += 8 * 32) {
+              unsigned long long hv[8][2];
+              auto load_missing = [&](bool first) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const int vi = v0 + 32 * j;
+                  if (vi < nv && (first || (uint32_t)(hv[j][0] >> 32) != tag || (uint32_t)(hv[j][1] >> 32) != tag))
+                    asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];"
+                                 : "=l"(hv[j][0]), "=l"(hv[j][1])
+                                 : "l"(hw + 2 * (size_t)vi)
+                                 : "memory");
+                }
+              };
+              auto all_tagged = [&]() {
+                bool ok_all = true;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                  if (v0 + 32 * j < nv)
+                    ok_all = ok_all && (uint32_t)(hv[j][0] >> 32) == tag && (uint32_t)(hv[j][1] >> 32) == tag;
+                return ok_all;
+              };
+              load_missing(true);
+              if (!all_tagged()) {
+                const uint64_t t0 = global_ns();
+                for (;;) {
+                  __nanosleep(32);
+                  load_missing(false);
+                  if (all_tagged() || s_abort) break;
+                  if (global_ns() - t0 > kWaitLimitNs) {
+                    s_abort = 1;
+                    set_device_error(ctrl, MOE_ERR_TIMEOUT, 45);
+                    break;
+                  }
+                }
+              }
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int vi = v0 + 32 * j;
+                if (vi < nv) {
+                  uint2 *dd = reinterpret_cast<uint2 *>(hs + (size_t)(c0 + vi / I4) * xstride + xs_pos(4 * (vi % I4)));
+                  *dd = make_uint2((uint32_t)hv[j][0], (uint32_t)hv[j][1]);
+                }
               }
             }
-          }
-          __syncwarp();
-          unsigned v;
-          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ready + u) : "memory");
-          (void)v;
-          // all of a lane's loads (eight per round) go out before its stores: one L2 round trip
-          const int I8 = I / 8, c0 = s_slot[u], nv = (s_slot[u + 1] - c0) * I8;
-          for (int v0 = lane; v0 < nv; v0 += 8 * 32) {
-            uint4 hv[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int vi = v0 + 32 * j;
-              hv[j] = vi < nv ? __ldcg(reinterpret_cast<const uint4 *>(a.hdec + (size_t)s_src[c0 + vi / I8] * I) + vi % I8)
-                              : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int vi = v0 + 32 * j;
-              if (vi < nv) {
-                uint2 *dd = reinterpret_cast<uint2 *>(hs + (size_t)(c0 + vi / I8) * xstride + xs_pos(8 * (vi % I8)));
-                dd[0] = make_uint2(hv[j].x, hv[j].y);
-                dd[1] = make_uint2(hv[j].z, hv[j].w);
+            __syncwarp();
+          } else {
+            // the unit's h: wait until all its gate/up items are counted (bounded), then stage its
+            // present columns (contiguous column slots c0.., 16-byte loads from L2)
+            if (lane == 0) {
+              const uint64_t t0 = global_ns();
+              for (;;) {
+                unsigned v;
+                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ready + u) : "memory");
+                if (v >= (unsigned)rbs8 || s_abort) break;
+                __nanosleep(32);
+                if (global_ns() - t0 > kWaitLimitNs) {
+                  s_abort = 1;
+                  set_device_error(ctrl, MOE_ERR_TIMEOUT, 45);
+                  break;
+                }
               }
             }
+            __syncwarp();
+            unsigned v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ready + u) : "memory");
+            (void)v;
+            // all of a lane's loads (eight per round) go out before its stores: one L2 round trip
+            const int I8 = I / 8, c0 = s_slot[u], nv = (s_slot[u + 1] - c0) * I8;
+            const uint4 *hsrc = reinterpret_cast<const uint4 *>(fs->hval + (size_t)c0 * I);
+            for (int v0 = lane; v0 < nv; v0 += 8 * 32) {
+              uint4 hv[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int vi = v0 + 32 * j;
+                hv[j] = vi < nv ? __ldcg(hsrc + vi) : make_uint4(0, 0, 0, 0);
+              }
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int vi = v0 + 32 * j;
+                if (vi < nv) {
+                  uint2 *dd = reinterpret_cast<uint2 *>(hs + (size_t)(c0 + vi / I8) * xstride + xs_pos(8 * (vi % I8)));
+                  dd[0] = make_uint2(hv[j].x, hv[j].y);
+                  dd[1] = make_uint2(hv[j].z, hv[j].w);
+                }
+              }
+            }
+            __syncwarp();
           }
-          __syncwarp();
         }
         const bool have = wait_bar(full(s), fill_parity(qd), 43);
         const bool colok = (un.mask >> g) & 1;
@@ -1153,7 +1225,7 @@ static cudaError_t fused_launch(const void *fn, size_t smem, void **args, cudaSt
 cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float eps, int T, int H, const float *Wr,
                                 const float *bias, int E, int k, int I, const moe_expert_set &routed,
                                 const moe_expert_set *shared, const float *residual, float *y, int32_t *idx,
-                                float *w, uint16_t *hdec, Ctrl *ctrl, cudaStream_t s, const float *next_Wr) {
+                                float *w, Ctrl *ctrl, cudaStream_t s, const float *next_Wr) {
   FusedArgs a;
   const void *fn = nullptr;
   size_t smem = 0;
@@ -1170,7 +1242,6 @@ cudaError_t launch_decode_fused(const uint16_t *x, const float *r_norm, float ep
   a.y = y;
   a.idx = idx;
   a.w = w;
-  a.hdec = hdec;
   a.ctrl = ctrl;
   void *args[] = {&a};
   return fused_launch(fn, smem, args, s);
