@@ -33,7 +33,7 @@ dec_gate_up_kernel(const void *__restrict__ x, int H, int I, moe_expert_set rout
                    const DecUnit *__restrict__ units, Ctrl *__restrict__ ctrl, uint16_t *__restrict__ hdec) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int n_units = ctrl->n_units;
-  const int xstride = H + 4;
+  const int xstride = xs_stride(H);
   __half *xs = reinterpret_cast<__half *>(smem_raw);
   __shared__ float part[kGuWarps][16][8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -129,7 +129,7 @@ cudaError_t launch_decode_gate_up(const void *x, int x_is_bf16, int H, int I, co
   const int ny = I / (16 * kGuBlocks);
   const int cap = (8 * num_sms() + ny - 1) / ny;
   const dim3 grid(max_units < cap ? (max_units > 0 ? max_units : 1) : cap, ny);
-  const size_t smem = (size_t)8 * (H + 4) * 2;
+  const size_t smem = (size_t)8 * xs_stride(H) * 2;
   const int qt = routed.gate.qtype;
 #define MOE_GU(B, Q) launch_gu<B, Q>(grid, smem, s, x, H, I, routed, sh, units, ctrl, hdec)
   if (x_is_bf16)
@@ -158,8 +158,8 @@ dec_down_kernel(int H, int I, moe_expert_set routed, moe_expert_set shared, cons
   const int nu = ctrl->n_units;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int r0 = blockIdx.x * 16;
-  const int xstride = I + 4;
-  __half *hs = reinterpret_cast<__half *>(smem_raw);  // kDownSlots columns x (I + 4)
+  const int xstride = xs_stride(I);
+  __half *hs = reinterpret_cast<__half *>(smem_raw);  // kDownSlots columns x xs_stride(I)
   __shared__ float red[kDownWarps][16][8];
   __shared__ __align__(16) DecUnit s_units[kDownMaxUnits];
   __shared__ int s_slot[kDownMaxUnits + 1];           // first staged slot of each unit of the chunk
@@ -314,7 +314,7 @@ cudaError_t launch_decode_down(int H, int I, const moe_expert_set &routed, const
                                const float *residual, int T, uint16_t *out_rows, cudaStream_t s) {
   (void)max_units;
   const moe_expert_set sh = shared ? *shared : routed;
-  const size_t smem = (size_t)kDownSlots * (I + 4) * 2;
+  const size_t smem = (size_t)kDownSlots * xs_stride(I) * 2;
   const int qt = routed.gate.qtype;
   auto fn = qt == MOE_Q3 ? dec_down_kernel<3> : qt == MOE_Q4 ? dec_down_kernel<4> : dec_down_kernel<2>;
   cudaError_t e = smem_limit_once(fn, smem);

@@ -115,14 +115,14 @@ __host__ __device__ inline FusedLayout fused_layout(int T, int H, int E, int I, 
   // Phase-local buffers share one region: the tokens, logit keys and top-k lists serve P0-P2
   // only, the staged h columns P3 only, and a CTA's P3 starts after its P2 is complete.
   L.xraw = take((size_t)T * H * 2);
-  L.x16 = take((size_t)T * (H + 4) * 2);
+  L.x16 = take((size_t)T * xs_stride(H) * 2);
   L.keys = take((size_t)T * E * 4);              // [token][expert] order-preserving logit keys
   L.ctop = take((size_t)T * 32 * 8);             // [token][32] chunk-top codes (threshold candidates)
   L.cand = take((size_t)T * 32 * 8 + 128);       // [token][32] codes above the threshold, [8] counts, [8] tau
   L.firstof = take((size_t)E * 4);                // expert -> first pair choosing it
   const size_t early_end = o;
   o = 0;
-  L.hs = take((size_t)hs_cols * (I + 4) * 2);    // staged h columns (down phase)
+  L.hs = take((size_t)hs_cols * xs_stride(I) * 2);    // staged h columns (down phase)
   o = early_end > o ? early_end : o;
   L.part = take((size_t)2 * 2 * 8 * 16 * 8 * 4);  // [group][buffer][K step][16 rows][8 columns]
   L.red = take((size_t)kFWarps * 16 * 8 * 4);
@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   const int R = a.ring, S = a.slot_bytes;
   auto full = [&](int s) { return bar_full0 + 8u * (uint32_t)s; };
   Ctrl *ctrl = a.ctrl;
-  const int xs16 = H + 4;
+  const int xs16 = xs_stride(H);
   const int G = gridDim.x;
   FusedSync *const fs = fused_sync(ctrl);
   __shared__ uint32_t s_tag;
@@ -888,7 +888,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   // P2 item or to an earlier row block, consumed before this row block starts. Units are taken in
   // increasing order, so the lowest waiting piece can always proceed.
   if (ok) {
-    const int xstride = I + 4;
+    const int xstride = xs_stride(I);
     const int dn = a.dn_bytes;
     for (int rbl = 0; rbl < n_rb; ++rbl) {
       const int r0 = ((int)blockIdx.x + rbl * G) * 16;

@@ -70,17 +70,20 @@ __device__ __forceinline__ uint32_t dq3_sub(int i) {
   }
 }
 
+// Pair j (weights 2j, 2j+1; j = 0..7, a compile-time constant in callers) of a Q2 word w, times d;
+// w8 = w >> 8.
+__device__ __forceinline__ uint32_t dq2_pair(uint32_t w, uint32_t w8, int j, __half2 d2) {
+  const int p = j & 3;
+  const uint32_t src = (j < 4) ? w : w8;
+  const uint32_t t = (src & (0x00030003u << (2 * p))) | dq_magic(p);
+  return bits_h2(__hmul2_rn(__hsub2_rn(h2bits(t), h2bits(dq2_sub(p))), d2));
+}
+
 // One Q2 word (16 weights) -> 8 half2 in natural K order (out[j] = weights 2j, 2j+1), times d.
 __device__ __forceinline__ void dq2_word(uint32_t w, __half2 d2, uint32_t out[8]) {
   const uint32_t w8 = w >> 8;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int p = j & 3;
-    const uint32_t src = (j < 4) ? w : w8;
-    const uint32_t t = (src & (0x00030003u << (2 * p))) | dq_magic(p);
-    const __half2 v = __hsub2_rn(h2bits(t), h2bits(dq2_sub(p)));
-    out[j] = bits_h2(__hmul2_rn(v, d2));
-  }
+  for (int j = 0; j < 8; ++j) out[j] = dq2_pair(w, w8, j, d2);
 }
 
 // Same pairs without the scale: (c - 2) exactly, for callers that apply d afterwards.
@@ -95,33 +98,39 @@ __device__ __forceinline__ void dq2_word_noscale(uint32_t w, uint32_t out[8]) {
   }
 }
 
+// Pair j of a Q3 half-block (see dq3_word): w8 = w >> 8, hs = the hi word shifted for the half
+// (q ? hw >> 6 : hw << 2).
+__device__ __forceinline__ uint32_t dq3_pair(uint32_t w, uint32_t w8, uint32_t hs, int j, __half2 d2) {
+  const int p = j & 3;
+  const uint32_t src = (j < 4) ? w : w8;
+  const uint32_t tl = (src & (0x00030003u << (2 * p))) | dq_magic(p);
+  const uint32_t th = (hs & (0x00010001u << (j + 2))) | dq3_hmag(j);
+  const __half2 v = __hadd2_rn(__hsub2_rn(h2bits(tl), h2bits(dq3_sub(j))), h2bits(th));
+  return bits_h2(__hmul2_rn(v, d2));
+}
+
 // One Q3 half-block: low-plane word w (16 weights) and the block's hi word `hw`, q = which half
 // (0: weights 0..15 of the block, 1: weights 16..31). out[j] = weights 2j, 2j+1, times d.
 __device__ __forceinline__ void dq3_word(uint32_t w, uint32_t hw, int q, __half2 d2, uint32_t out[8]) {
   const uint32_t w8 = w >> 8;
   const uint32_t hs = q ? (hw >> 6) : (hw << 2);
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int p = j & 3;
-    const uint32_t src = (j < 4) ? w : w8;
-    const uint32_t tl = (src & (0x00030003u << (2 * p))) | dq_magic(p);
-    const uint32_t th = (hs & (0x00010001u << (j + 2))) | dq3_hmag(j);
-    const __half2 v = __hadd2_rn(__hsub2_rn(h2bits(tl), h2bits(dq3_sub(j))), h2bits(th));
-    out[j] = bits_h2(__hmul2_rn(v, d2));
-  }
+  for (int j = 0; j < 8; ++j) out[j] = dq3_pair(w, w8, hs, j, d2);
+}
+
+// Pair j (0..3) of a Q4 word w (8 weights), times d; w8 = w >> 8.
+__device__ __forceinline__ uint32_t dq4_pair(uint32_t w, uint32_t w8, int j, __half2 d2) {
+  const uint32_t src = (j < 2) ? w : w8;
+  const bool hi = j & 1;  // bits 4-7 (magic 64) or 0-3 (magic 1024)
+  const uint32_t t = (src & (hi ? 0x00F000F0u : 0x000F000Fu)) | (hi ? 0x54005400u : 0x64006400u);
+  return bits_h2(__hmul2_rn(__hsub2_rn(h2bits(t), h2bits(hi ? 0x54805480u : 0x64086408u)), d2));  // - (M + 8)
 }
 
 // One Q4 word (8 weights) -> 4 half2 in natural K order (out[j] = weights 2j, 2j+1), times d.
 __device__ __forceinline__ void dq4_word(uint32_t w, __half2 d2, uint32_t out[4]) {
   const uint32_t w8 = w >> 8;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t src = (j < 2) ? w : w8;
-    const bool hi = j & 1;  // bits 4-7 (magic 64) or 0-3 (magic 1024)
-    const uint32_t t = (src & (hi ? 0x00F000F0u : 0x000F000Fu)) | (hi ? 0x54005400u : 0x64006400u);
-    const __half2 v = __hsub2_rn(h2bits(t), h2bits(hi ? 0x54805480u : 0x64086408u));  // M + 8
-    out[j] = bits_h2(__hmul2_rn(v, d2));
-  }
+  for (int j = 0; j < 4; ++j) out[j] = dq4_pair(w, w8, j, d2);
 }
 
 }  // namespace moe

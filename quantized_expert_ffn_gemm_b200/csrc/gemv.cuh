@@ -3,8 +3,10 @@
 // (one 16-byte code load per row per step for the 2-bit plane, two for the 4-bit plane); each
 // code word is dequantized to fp16 pairs and fed to mma.sync m16n8k16 with the activation
 // columns as the 8 MMA columns (fp32 accumulate). QT is the block format: 2 (Q2), 3 (Q3), 4 (Q4).
-// Activations are staged in shared memory as fp16 with a per-64-chunk rotation so the fragment
-// loads of the four K slices hit distinct banks.
+// Activations are staged in shared memory as fp16, each 64-element chunk followed by 16 halves of
+// padding and columns a multiple of 64 plus 4 halves apart, so the fragment loads of the four K
+// slices and eight columns hit distinct banks and a lane's loads within a chunk are one base
+// address plus compile-time offsets. Each MMA's four A registers are dequantized right before it.
 #pragma once
 
 #include "common.cuh"
@@ -25,12 +27,12 @@ __device__ __forceinline__ void mma16816(float c[4], const uint32_t a[4], uint32
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// shared-memory position of activation element k of a column (row stride added by the caller):
-// 64-element chunk ch keeps its elements rotated by 16*(ch%4)
-__device__ __forceinline__ int xs_pos(int k) {
-  const int ch = k >> 6, q = k & 63;
-  return (ch << 6) + ((q + 16 * (ch & 3)) & 63);
-}
+// shared-memory position of activation element k of a column (column stride added by the caller):
+// 64-element chunk ch starts at 80 ch
+__device__ __forceinline__ int xs_pos(int k) { return k + 16 * (k >> 6); }
+// column stride (halves) of a staged column of K elements: the padded length rounded up to 64,
+// plus 4
+__host__ __device__ constexpr int xs_stride(int K) { return ((K + K / 4 + 63) & ~63) + 4; }
 
 // word i (0..3) of a 16-byte fragment, by selects (no local-memory indexing)
 __device__ __forceinline__ uint32_t sel4(const uint4 &v, int i) {
@@ -134,30 +136,36 @@ __device__ __forceinline__ void load_step_pair(StepFrag &f, const MatView &ma, i
 }
 
 // dequantize the fragment (zero codes with zero scales give zero weights) and run the step's 16
-// MMAs; B fragments come from the lane's column in shared memory when `bok`, else zero
+// MMAs; B fragments come from the lane's column in shared memory when `bok`, else zero. kbase (a
+// multiple of 64) starts the lane's 64 weights, which lie in one staged chunk.
 template <int QT>
 __device__ __forceinline__ void mma_step(float acc[4], float acc2[4], const StepFrag &f, const __half *xcol, int kbase,
                                          bool bok) {
+  const __half *xb = xcol + xs_pos(kbase);
+  auto bfrag = [&](int off, uint32_t &b0, uint32_t &b1) {
+    b0 = 0u;
+    b1 = 0u;
+    if (bok) {
+      const uint2 bv = *reinterpret_cast<const uint2 *>(xb + off);
+      b0 = bv.x;
+      b1 = bv.y;
+    }
+  };
   if constexpr (QT == 4) {  // eight 8-weight words per row: word wq in block wq/4, two MMAs per word
 #pragma unroll
     for (int wq = 0; wq < 8; ++wq) {
       const int blk = wq >> 2;
       const uint32_t w0 = blk ? sel4(f.w0b, wq & 3) : sel4(f.w0, wq & 3);
       const uint32_t w1 = blk ? sel4(f.w1b, wq & 3) : sel4(f.w1, wq & 3);
+      const uint32_t w08 = w0 >> 8, w18 = w1 >> 8;
       const __half2 dd0 = __half2half2(__ushort_as_half((uint16_t)(f.d0 >> (16 * blk))));
       const __half2 dd1 = __half2half2(__ushort_as_half((uint16_t)(f.d1 >> (16 * blk))));
-      uint32_t p0[4], p1[4];
-      dq4_word(w0, dd0, p0);
-      dq4_word(w1, dd1, p1);
 #pragma unroll
       for (int mm = 0; mm < 2; ++mm) {
-        const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
-        uint32_t b0 = 0, b1 = 0;
-        if (bok) {
-          const uint2 bv = *reinterpret_cast<const uint2 *>(xcol + xs_pos(kbase + 8 * wq + 4 * mm));
-          b0 = bv.x;
-          b1 = bv.y;
-        }
+        const uint32_t a[4] = {dq4_pair(w0, w08, 2 * mm, dd0), dq4_pair(w1, w18, 2 * mm, dd1),
+                               dq4_pair(w0, w08, 2 * mm + 1, dd0), dq4_pair(w1, w18, 2 * mm + 1, dd1)};
+        uint32_t b0, b1;
+        bfrag(8 * wq + 4 * mm, b0, b1);
         mma16816(mm ? acc2 : acc, a, b0, b1);
       }
     }
@@ -166,25 +174,31 @@ __device__ __forceinline__ void mma_step(float acc[4], float acc2[4], const Step
     for (int wq = 0; wq < 4; ++wq) {  // word wq: block wq/2, half q = wq%2
       const int blk = wq >> 1, q = wq & 1;
       const uint32_t w0 = sel4(f.w0, wq), w1 = sel4(f.w1, wq);
+      const uint32_t w08 = w0 >> 8, w18 = w1 >> 8;
       const __half2 dd0 = __half2half2(__ushort_as_half((uint16_t)(f.d0 >> (16 * blk))));
       const __half2 dd1 = __half2half2(__ushort_as_half((uint16_t)(f.d1 >> (16 * blk))));
-      uint32_t p0[8], p1[8];
+      uint32_t hs0 = 0u, hs1 = 0u;
       if (QT == 3) {
-        dq3_word(w0, blk ? f.h0.y : f.h0.x, q, dd0, p0);
-        dq3_word(w1, blk ? f.h1.y : f.h1.x, q, dd1, p1);
-      } else {
-        dq2_word(w0, dd0, p0);
-        dq2_word(w1, dd1, p1);
+        const uint32_t h0 = blk ? f.h0.y : f.h0.x, h1 = blk ? f.h1.y : f.h1.x;
+        hs0 = q ? (h0 >> 6) : (h0 << 2);
+        hs1 = q ? (h1 >> 6) : (h1 << 2);
       }
 #pragma unroll
-      for (int mm = 0; mm < 4; ++mm) {  // MMA 4*wq + mm uses pairs 2mm, 2mm+1 of this word
-        const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
-        uint32_t b0 = 0, b1 = 0;
-        if (bok) {
-          const uint2 bv = *reinterpret_cast<const uint2 *>(xcol + xs_pos(kbase + 16 * wq + 4 * mm));
-          b0 = bv.x;
-          b1 = bv.y;
+      for (int mm = 0; mm < 4; ++mm) {  // MMA 4*wq + mm: pairs 2mm, 2mm+1 of this word
+        uint32_t a[4];
+        if (QT == 3) {
+          a[0] = dq3_pair(w0, w08, hs0, 2 * mm, dd0);
+          a[1] = dq3_pair(w1, w18, hs1, 2 * mm, dd1);
+          a[2] = dq3_pair(w0, w08, hs0, 2 * mm + 1, dd0);
+          a[3] = dq3_pair(w1, w18, hs1, 2 * mm + 1, dd1);
+        } else {
+          a[0] = dq2_pair(w0, w08, 2 * mm, dd0);
+          a[1] = dq2_pair(w1, w18, 2 * mm, dd1);
+          a[2] = dq2_pair(w0, w08, 2 * mm + 1, dd0);
+          a[3] = dq2_pair(w1, w18, 2 * mm + 1, dd1);
         }
+        uint32_t b0, b1;
+        bfrag(16 * wq + 4 * mm, b0, b1);
         mma16816((mm & 1) ? acc2 : acc, a, b0, b1);
       }
     }
@@ -205,50 +219,59 @@ struct HalfFrag {
 template <int QT>
 __device__ __forceinline__ void mma_half_step(float acc[4], float acc2[4], const HalfFrag &f, const __half *xcol,
                                               int kbase, bool bok) {
+  const __half *xb = xcol + xs_pos(kbase);  // kbase: a multiple of 32; its 32 weights lie in one chunk
+  auto bfrag = [&](int off, uint32_t &b0, uint32_t &b1) {
+    b0 = 0u;
+    b1 = 0u;
+    if (bok) {
+      const uint2 bv = *reinterpret_cast<const uint2 *>(xb + off);
+      b0 = bv.x;
+      b1 = bv.y;
+    }
+  };
+  const __half2 dd0 = __half2half2(__ushort_as_half(f.d0));
+  const __half2 dd1 = __half2half2(__ushort_as_half(f.d1));
   if constexpr (QT == 4) {
-    const __half2 dd0 = __half2half2(__ushort_as_half(f.d0));
-    const __half2 dd1 = __half2half2(__ushort_as_half(f.d1));
 #pragma unroll
     for (int wq = 0; wq < 4; ++wq) {
       const uint2 a0 = (wq >> 1) ? f.w0b : f.w0, a1 = (wq >> 1) ? f.w1b : f.w1;
-      uint32_t p0[4], p1[4];
-      dq4_word((wq & 1) ? a0.y : a0.x, dd0, p0);
-      dq4_word((wq & 1) ? a1.y : a1.x, dd1, p1);
+      const uint32_t w0 = (wq & 1) ? a0.y : a0.x, w1 = (wq & 1) ? a1.y : a1.x;
+      const uint32_t w08 = w0 >> 8, w18 = w1 >> 8;
 #pragma unroll
       for (int mm = 0; mm < 2; ++mm) {
-        const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
-        uint32_t b0 = 0, b1 = 0;
-        if (bok) {
-          const uint2 bv = *reinterpret_cast<const uint2 *>(xcol + xs_pos(kbase + 8 * wq + 4 * mm));
-          b0 = bv.x;
-          b1 = bv.y;
-        }
+        const uint32_t a[4] = {dq4_pair(w0, w08, 2 * mm, dd0), dq4_pair(w1, w18, 2 * mm, dd1),
+                               dq4_pair(w0, w08, 2 * mm + 1, dd0), dq4_pair(w1, w18, 2 * mm + 1, dd1)};
+        uint32_t b0, b1;
+        bfrag(8 * wq + 4 * mm, b0, b1);
         mma16816(mm ? acc2 : acc, a, b0, b1);
       }
     }
   } else {
-    const __half2 dd0 = __half2half2(__ushort_as_half(f.d0));
-    const __half2 dd1 = __half2half2(__ushort_as_half(f.d1));
 #pragma unroll
     for (int wq = 0; wq < 2; ++wq) {
       const uint32_t w0 = wq ? f.w0.y : f.w0.x, w1 = wq ? f.w1.y : f.w1.x;
-      uint32_t p0[8], p1[8];
+      const uint32_t w08 = w0 >> 8, w18 = w1 >> 8;
+      uint32_t hs0 = 0u, hs1 = 0u;
       if (QT == 3) {
-        dq3_word(w0, f.h0, wq, dd0, p0);
-        dq3_word(w1, f.h1, wq, dd1, p1);
-      } else {
-        dq2_word(w0, dd0, p0);
-        dq2_word(w1, dd1, p1);
+        hs0 = wq ? (f.h0 >> 6) : (f.h0 << 2);
+        hs1 = wq ? (f.h1 >> 6) : (f.h1 << 2);
       }
 #pragma unroll
       for (int mm = 0; mm < 4; ++mm) {
-        const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
-        uint32_t b0 = 0, b1 = 0;
-        if (bok) {
-          const uint2 bv = *reinterpret_cast<const uint2 *>(xcol + xs_pos(kbase + 16 * wq + 4 * mm));
-          b0 = bv.x;
-          b1 = bv.y;
+        uint32_t a[4];
+        if (QT == 3) {
+          a[0] = dq3_pair(w0, w08, hs0, 2 * mm, dd0);
+          a[1] = dq3_pair(w1, w18, hs1, 2 * mm, dd1);
+          a[2] = dq3_pair(w0, w08, hs0, 2 * mm + 1, dd0);
+          a[3] = dq3_pair(w1, w18, hs1, 2 * mm + 1, dd1);
+        } else {
+          a[0] = dq2_pair(w0, w08, 2 * mm, dd0);
+          a[1] = dq2_pair(w1, w18, 2 * mm, dd1);
+          a[2] = dq2_pair(w0, w08, 2 * mm + 1, dd0);
+          a[3] = dq2_pair(w1, w18, 2 * mm + 1, dd1);
         }
+        uint32_t b0, b1;
+        bfrag(16 * wq + 4 * mm, b0, b1);
         mma16816((mm & 1) ? acc2 : acc, a, b0, b1);
       }
     }
