@@ -203,26 +203,29 @@ __global__ void __launch_bounds__(kPlanThreads) mid_plan_kernel(const int32_t *_
 template <int QT>
 __device__ __forceinline__ void gu_step_tiles(float acc[kMaxTiles][4], const StepFrag &f, const __half *xb,
                                               int tstride, int nt) {
+  // each MMA's four A registers are dequantized right before it
+  auto tiles = [&](const uint32_t a[4], int off) {
+#pragma unroll
+    for (int j = 0; j < kMaxTiles; ++j)
+      if (j < nt) {
+        const uint2 bv = *reinterpret_cast<const uint2 *>(xb + j * tstride + off);
+        mma16816(acc[j], a, bv.x, bv.y);
+      }
+  };
   if constexpr (QT == 4) {
 #pragma unroll
     for (int wq = 0; wq < 8; ++wq) {
       const int blk = wq >> 2;
       const uint32_t w0 = blk ? sel4(f.w0b, wq & 3) : sel4(f.w0, wq & 3);
       const uint32_t w1 = blk ? sel4(f.w1b, wq & 3) : sel4(f.w1, wq & 3);
+      const uint32_t w08 = w0 >> 8, w18 = w1 >> 8;
       const __half2 dd0 = __half2half2(__ushort_as_half((uint16_t)(f.d0 >> (16 * blk))));
       const __half2 dd1 = __half2half2(__ushort_as_half((uint16_t)(f.d1 >> (16 * blk))));
-      uint32_t p0[4], p1[4];
-      dq4_word(w0, dd0, p0);
-      dq4_word(w1, dd1, p1);
 #pragma unroll
       for (int mm = 0; mm < 2; ++mm) {
-        const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
-#pragma unroll
-        for (int j = 0; j < kMaxTiles; ++j)
-          if (j < nt) {
-            const uint2 bv = *reinterpret_cast<const uint2 *>(xb + j * tstride + 8 * wq + 4 * mm);
-            mma16816(acc[j], a, bv.x, bv.y);
-          }
+        const uint32_t a[4] = {dq4_pair(w0, w08, 2 * mm, dd0), dq4_pair(w1, w18, 2 * mm, dd1),
+                               dq4_pair(w0, w08, 2 * mm + 1, dd0), dq4_pair(w1, w18, 2 * mm + 1, dd1)};
+        tiles(a, 8 * wq + 4 * mm);
       }
     }
   } else {
@@ -230,25 +233,30 @@ __device__ __forceinline__ void gu_step_tiles(float acc[kMaxTiles][4], const Ste
     for (int wq = 0; wq < 4; ++wq) {
       const int blk = wq >> 1, q = wq & 1;
       const uint32_t w0 = sel4(f.w0, wq), w1 = sel4(f.w1, wq);
+      const uint32_t w08 = w0 >> 8, w18 = w1 >> 8;
       const __half2 dd0 = __half2half2(__ushort_as_half((uint16_t)(f.d0 >> (16 * blk))));
       const __half2 dd1 = __half2half2(__ushort_as_half((uint16_t)(f.d1 >> (16 * blk))));
-      uint32_t p0[8], p1[8];
+      uint32_t hs0 = 0u, hs1 = 0u;
       if (QT == 3) {
-        dq3_word(w0, blk ? f.h0.y : f.h0.x, q, dd0, p0);
-        dq3_word(w1, blk ? f.h1.y : f.h1.x, q, dd1, p1);
-      } else {
-        dq2_word(w0, dd0, p0);
-        dq2_word(w1, dd1, p1);
+        const uint32_t h0 = blk ? f.h0.y : f.h0.x, h1 = blk ? f.h1.y : f.h1.x;
+        hs0 = q ? (h0 >> 6) : (h0 << 2);
+        hs1 = q ? (h1 >> 6) : (h1 << 2);
       }
 #pragma unroll
       for (int mm = 0; mm < 4; ++mm) {
-        const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
-#pragma unroll
-        for (int j = 0; j < kMaxTiles; ++j)
-          if (j < nt) {
-            const uint2 bv = *reinterpret_cast<const uint2 *>(xb + j * tstride + 16 * wq + 4 * mm);
-            mma16816(acc[j], a, bv.x, bv.y);
-          }
+        uint32_t a[4];
+        if (QT == 3) {
+          a[0] = dq3_pair(w0, w08, hs0, 2 * mm, dd0);
+          a[1] = dq3_pair(w1, w18, hs1, 2 * mm, dd1);
+          a[2] = dq3_pair(w0, w08, hs0, 2 * mm + 1, dd0);
+          a[3] = dq3_pair(w1, w18, hs1, 2 * mm + 1, dd1);
+        } else {
+          a[0] = dq2_pair(w0, w08, 2 * mm, dd0);
+          a[1] = dq2_pair(w1, w18, 2 * mm, dd1);
+          a[2] = dq2_pair(w0, w08, 2 * mm + 1, dd0);
+          a[3] = dq2_pair(w1, w18, 2 * mm + 1, dd1);
+        }
+        tiles(a, 16 * wq + 4 * mm);
       }
     }
   }
@@ -261,45 +269,52 @@ __device__ __forceinline__ void dn_half_tiles(float acc[kMaxTiles][4], const Hal
                                               int tstride, int nt) {
   const __half2 dd0 = __half2half2(__ushort_as_half(f.d0));
   const __half2 dd1 = __half2half2(__ushort_as_half(f.d1));
+  auto tiles = [&](const uint32_t a[4], int off) {
+#pragma unroll
+    for (int j = 0; j < kMaxTiles; ++j)
+      if (j < nt) {
+        const uint2 bv = *reinterpret_cast<const uint2 *>(hb + j * tstride + off);
+        mma16816(acc[j], a, bv.x, bv.y);
+      }
+  };
   if constexpr (QT == 4) {
 #pragma unroll
     for (int wq = 0; wq < 4; ++wq) {
       const uint2 a0 = (wq >> 1) ? f.w0b : f.w0, a1 = (wq >> 1) ? f.w1b : f.w1;
-      uint32_t p0[4], p1[4];
-      dq4_word((wq & 1) ? a0.y : a0.x, dd0, p0);
-      dq4_word((wq & 1) ? a1.y : a1.x, dd1, p1);
+      const uint32_t w0 = (wq & 1) ? a0.y : a0.x, w1 = (wq & 1) ? a1.y : a1.x;
+      const uint32_t w08 = w0 >> 8, w18 = w1 >> 8;
 #pragma unroll
       for (int mm = 0; mm < 2; ++mm) {
-        const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
-#pragma unroll
-        for (int j = 0; j < kMaxTiles; ++j)
-          if (j < nt) {
-            const uint2 bv = *reinterpret_cast<const uint2 *>(hb + j * tstride + 8 * wq + 4 * mm);
-            mma16816(acc[j], a, bv.x, bv.y);
-          }
+        const uint32_t a[4] = {dq4_pair(w0, w08, 2 * mm, dd0), dq4_pair(w1, w18, 2 * mm, dd1),
+                               dq4_pair(w0, w08, 2 * mm + 1, dd0), dq4_pair(w1, w18, 2 * mm + 1, dd1)};
+        tiles(a, 8 * wq + 4 * mm);
       }
     }
   } else {
 #pragma unroll
     for (int wq = 0; wq < 2; ++wq) {
       const uint32_t w0 = wq ? f.w0.y : f.w0.x, w1 = wq ? f.w1.y : f.w1.x;
-      uint32_t p0[8], p1[8];
+      const uint32_t w08 = w0 >> 8, w18 = w1 >> 8;
+      uint32_t hs0 = 0u, hs1 = 0u;
       if (QT == 3) {
-        dq3_word(w0, f.h0, wq, dd0, p0);
-        dq3_word(w1, f.h1, wq, dd1, p1);
-      } else {
-        dq2_word(w0, dd0, p0);
-        dq2_word(w1, dd1, p1);
+        hs0 = wq ? (f.h0 >> 6) : (f.h0 << 2);
+        hs1 = wq ? (f.h1 >> 6) : (f.h1 << 2);
       }
 #pragma unroll
       for (int mm = 0; mm < 4; ++mm) {
-        const uint32_t a[4] = {p0[2 * mm], p1[2 * mm], p0[2 * mm + 1], p1[2 * mm + 1]};
-#pragma unroll
-        for (int j = 0; j < kMaxTiles; ++j)
-          if (j < nt) {
-            const uint2 bv = *reinterpret_cast<const uint2 *>(hb + j * tstride + 16 * wq + 4 * mm);
-            mma16816(acc[j], a, bv.x, bv.y);
-          }
+        uint32_t a[4];
+        if (QT == 3) {
+          a[0] = dq3_pair(w0, w08, hs0, 2 * mm, dd0);
+          a[1] = dq3_pair(w1, w18, hs1, 2 * mm, dd1);
+          a[2] = dq3_pair(w0, w08, hs0, 2 * mm + 1, dd0);
+          a[3] = dq3_pair(w1, w18, hs1, 2 * mm + 1, dd1);
+        } else {
+          a[0] = dq2_pair(w0, w08, 2 * mm, dd0);
+          a[1] = dq2_pair(w1, w18, 2 * mm, dd1);
+          a[2] = dq2_pair(w0, w08, 2 * mm + 1, dd0);
+          a[3] = dq2_pair(w1, w18, 2 * mm + 1, dd1);
+        }
+        tiles(a, 16 * wq + 4 * mm);
       }
     }
   }
