@@ -90,6 +90,17 @@ def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
+# the raw handle of a device's current stream, without building a Stream object (~3 us per call
+# in the decode loop otherwise); torch's own accessor when the fast one is absent
+_raw_stream_fn = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _raw_stream(dev: int) -> int:
+    if _raw_stream_fn is not None:
+        return _raw_stream_fn(dev)
+    return torch.cuda.current_stream(dev).cuda_stream
+
+
 def qmat(m) -> QMat:
     """QMat struct from an object with qtype, n, rows, K and codes / hibits / scales device tensors."""
     return QMat(int(m.qtype), int(m.n), int(m.rows), int(m.K), m.codes.data_ptr(),
@@ -340,6 +351,7 @@ class LayerHandle:
         self._a = (Wr.data_ptr(), None if bias is None else bias.data_ptr(), ctypes.addressof(self.desc),
                    ctypes.addressof(self.rs), None if self.ss is None else ctypes.addressof(self.ss))
         self._ws = (ws.buf.data_ptr(), ws.nbytes)
+        self._dev = Wr.device.index if Wr.device.index is not None else torch.cuda.current_device()
         self._fn = LayerHandle._fast
 
     def forward(self, x: torch.Tensor, y: torch.Tensor, residual: Optional[torch.Tensor] = None,
@@ -348,7 +360,7 @@ class LayerHandle:
         code = self._fn(x.data_ptr(), x.shape[0], wr, b, d, rs, ss,
                         None if residual is None else residual.data_ptr(), y.data_ptr(),
                         None if idx_out is None else idx_out.data_ptr(), None if w_out is None else w_out.data_ptr(),
-                        path, self._ws[0], self._ws[1], torch.cuda.current_stream().cuda_stream)
+                        path, self._ws[0], self._ws[1], _raw_stream(self._dev))
         if code != MOE_OK:
             raise MoeError("moe_layer_forward", code)
         return y
@@ -361,7 +373,7 @@ class LayerHandle:
         code = LayerHandle._fast_host(x_host.data_ptr(), x_host.shape[0], wr, b, d, rs, ss, y_host.data_ptr(),
                                       None if idx_out is None else idx_out.data_ptr(),
                                       None if w_out is None else w_out.data_ptr(), path, self._ws[0], self._ws[1],
-                                      torch.cuda.current_stream().cuda_stream)
+                                      _raw_stream(self._dev))
         if code != MOE_OK:
             raise MoeError("moe_layer_forward_host", code)
         return y_host

@@ -399,6 +399,29 @@ def test_layer_forward_host_buffers_match_the_device_call(name, T, path, pinned)
     assert torch.equal(y_host, y_dev.cpu())
 
 
+@pytest.mark.parametrize("name,T", [("decode1", 1), ("decode4", 4)])
+def test_layer_forward_host_buffers_reused_with_new_contents(name, T):
+    # the same page-locked buffers for several calls, the host rewriting x between them (the copy
+    # kernels read and write the mapped buffers): every call sees this call's x
+    L, (x, Wr, b, routed, shared) = layer_of(name)
+    s = L.shape
+    ws = moe.Workspace.for_layer(s.H, s.E, s.k, s.I, s.shared, T)
+    h = moe.LayerHandle(Wr, b, routed, shared, s.k, ws)
+    x_host = torch.empty(T, s.H, dtype=torch.bfloat16).pin_memory()
+    y_host = torch.empty(T, s.H, dtype=torch.float32).pin_memory()
+    y_dev = torch.empty(T, s.H, dtype=torch.float32, device="cuda")
+    for stream in range(3):
+        xs = synth.make_x(s.seed, T, s.H, stream=stream + 1)
+        x_host.copy_(xs)
+        y_host.fill_(float("nan"))
+        h.forward_host(x_host, y_host)
+        torch.cuda.synchronize()
+        h.forward(xs.cuda(), y_dev)
+        torch.cuda.synchronize()
+        assert moe.read_device_error(ws) == 0
+        assert torch.equal(y_host, y_dev.cpu()), stream
+
+
 def test_stack_forward_host_buffers_match_the_device_call():
     H, E, k, I, Lyr, T = 256, 16, 2, 128, 3, 5
     Wrs = [synth.make_router(0, l, E, H).cuda() for l in range(Lyr)]
