@@ -90,11 +90,11 @@ _MID_SRC = ["quantized_expert_ffn_gemm_b200/csrc/mid.cu", "quantized_expert_ffn_
 TRAFFIC = {
     # (kernel, workloads with the captured launch shape): (sources, sha256, DRAM bytes per launch)
     ("gemm_gate_up", ("prefill8k", "stack_prefill")):
-        (_GEMM_SRC, "4973eaa737f0c89dba7e023c10b843e0bcbed182f4dbe40b7fc3e74b446fe30c", 863316224),
+        (_GEMM_SRC, "f08dad977b547aa9656127544c86817a1159fbae806114ced9b63f365c76169e", 862530560),
     ("decode_fused", ("decode1",)):
-        (_DEC_SRC, "ab9722e6aca444c671e3ee9a4f3713519adcb5909c38506670f9f3632a713fbd", 15127808),
+        (_DEC_SRC, "b4a6263a1bd80cf23ee14407bf0772dc785af48b7d956623805dfa00b7a861b3", 15141120),
     ("mid_expert", ("batch32",)):
-        (_MID_SRC, "17c6b89e453fea4a857d913221474e60272445c7aabe453d804734421b2fd54f", 47095808),
+        (_MID_SRC, "acc2d02342a8cb74d6fdb36322523b5cb6b5575bcf04ed7c4353561d0d314949", 47110400),
 }
 
 

@@ -371,51 +371,72 @@ bool router_refine_supported(int H, int E) { return H <= 2048 && E <= 512; }
 // ---------------------------------------------------------------- small batches (9..128 tokens)
 // Plain fp32 dot products on the CUDA cores: at these sizes the tensor-core router's fixed costs
 // (splitting Wr into planes, a K loop over 3H, the exact refine) dominate. A CTA takes 4 experts;
-// warp (e, half) keeps its expert's fp32 row in registers (Wr read once) and walks the tokens of
-// its half two at a time, both tokens' x loads in flight together. The logits are exact fp32
-// dot products (no refine needed); the bias is added by the top-k kernel.
+// warp (e, half) keeps its expert's fp32 row in registers (Wr read once). The tokens pass
+// through shared memory in chunks of 8, the next chunk's async copies in flight while the current
+// one is used, so each CTA reads x from L2 once (not once per expert) and every chunk costs one
+// round trip at most; warp half h takes tokens 4h..4h+3 of a chunk. The logits are exact fp32 dot
+// products (no refine needed); the bias is added by the top-k kernel.
 constexpr int kRouterMidMaxT = 128;
 constexpr int kRouterMidWarps = 8;
+constexpr int kRmChunk = 8;  // tokens per staged chunk
+
+__device__ __forceinline__ void rm_cp_async16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
 
 __global__ void __launch_bounds__(kRouterMidWarps * 32)
 router_mid_kernel(const uint16_t *__restrict__ x, int T, int H, const float *__restrict__ Wr, int E,
                   float *__restrict__ logits) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  extern __shared__ __align__(16) uint16_t s_xc[];  // [2][kRmChunk][H] bf16
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int e = blockIdx.x * 4 + (warp & 3), half = warp >> 2;
-  if (e >= E) return;
-  const int H4 = H >> 2;  // H <= 2048: at most 16 float4 per lane
-  const float4 *wr = reinterpret_cast<const float4 *>(Wr + (size_t)e * H);
+  const bool has_e = e < E;  // every thread takes part in the staging and the barriers
+  const int H4 = H >> 2;     // H <= 2048: at most 16 float4 per lane
+  const float4 *wr = reinterpret_cast<const float4 *>(Wr + (size_t)(has_e ? e : 0) * H);
   float4 wv[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const int h4 = lane + 32 * j;
-    wv[j] = (h4 < H4) ? __ldg(wr + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    wv[j] = (has_e && h4 < H4) ? __ldg(wr + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  for (int t0 = 2 * half; t0 < T; t0 += 4) {  // half 0: tokens 0,1,4,5,...; half 1: 2,3,6,7,...
-    uint2 xv[2][16];
+  const int nchunk = (T + kRmChunk - 1) / kRmChunk;
+  auto stage = [&](int c) {  // chunk c's rows into buffer c % 2, 16-byte async copies
+    const int t0 = c * kRmChunk, n16 = min(kRmChunk, T - t0) * H / 8;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t0 * H);
+    const uint32_t dst = (uint32_t)__cvta_generic_to_shared(s_xc + (size_t)(c & 1) * kRmChunk * H);
+    for (int i = tid; i < n16; i += kRouterMidWarps * 32) rm_cp_async16(dst + 16u * i, src + i);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  stage(0);
+  for (int c = 0; c < nchunk; ++c) {
+    if (c + 1 < nchunk) {
+      stage(c + 1);  // into the buffer chunk c - 1 used, freed by the barrier ending its iteration
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();
+    const uint16_t *xb = s_xc + (size_t)(c & 1) * kRmChunk * H;
+    const int t0 = c * kRmChunk, nt = min(kRmChunk, T - t0);
+    if (has_e) {
+#pragma unroll 1
+      for (int tt = 4 * half; tt < 4 * half + 4 && tt < nt; ++tt) {
+        const uint2 *xr = reinterpret_cast<const uint2 *>(xb + (size_t)tt * H);
+        float acc = 0.0f;
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      const int t = t0 + b;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int h4 = lane + 32 * j;
-        xv[b][j] = (t < T && h4 < H4) ? __ldg(reinterpret_cast<const uint2 *>(x + (size_t)t * H) + h4)
-                                      : make_uint2(0u, 0u);
+        for (int j = 0; j < 16; ++j) {
+          const int h4 = lane + 32 * j;
+          const uint2 xv = (h4 < H4) ? xr[h4] : make_uint2(0u, 0u);
+          acc = fmaf(wv[j].x, __uint_as_float(xv.x << 16), acc);
+          acc = fmaf(wv[j].y, __uint_as_float(xv.x & 0xffff0000u), acc);
+          acc = fmaf(wv[j].z, __uint_as_float(xv.y << 16), acc);
+          acc = fmaf(wv[j].w, __uint_as_float(xv.y & 0xffff0000u), acc);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) logits[(size_t)(t0 + tt) * E + e] = acc;
       }
     }
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      float acc = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        acc = fmaf(wv[j].x, __uint_as_float(xv[b][j].x << 16), acc);
-        acc = fmaf(wv[j].y, __uint_as_float(xv[b][j].x & 0xffff0000u), acc);
-        acc = fmaf(wv[j].z, __uint_as_float(xv[b][j].y << 16), acc);
-        acc = fmaf(wv[j].w, __uint_as_float(xv[b][j].y & 0xffff0000u), acc);
-      }
-      acc = warp_sum(acc);
-      if (lane == 0 && t0 + b < T) logits[(size_t)(t0 + b) * E + e] = acc;
-    }
+    __syncthreads();  // this buffer is refilled two chunks on
   }
 }
 
@@ -425,7 +446,9 @@ cudaError_t launch_router_prefill(const uint16_t *x, int T, int H, const float *
   if (T <= kRouterMidMaxT && H <= 2048) {
     {
       KTimer kt_(KID_ROUTER_GEMM, s);
-      router_mid_kernel<<<(E + 3) / 4, kRouterMidWarps * 32, 0, s>>>(x, T, H, Wr, E, logits);
+      const size_t smem = (size_t)2 * kRmChunk * H * 2;
+      if ((e = smem_limit_once(router_mid_kernel, smem)) != cudaSuccess) return e;
+      router_mid_kernel<<<(E + 3) / 4, kRouterMidWarps * 32, smem, s>>>(x, T, H, Wr, E, logits);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {
