@@ -237,6 +237,9 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
 topk_kernel(float *__restrict__ logits, const float *__restrict__ bias, int T, int E, int k, int32_t *__restrict__ idx,
             float *__restrict__ w) {
   __shared__ uint32_t s_taken[kTopkWarps][kMaxE / 32];
+  // launched behind the router (programmatic stream serialization): its logits are read after the wait
+  pdl_launch_dependents();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kTopkWarps + warp;
   if (t >= T) return;
@@ -399,6 +402,10 @@ router_mid_kernel(const uint16_t *__restrict__ x, int T, int H, const float *__r
     const int h4 = lane + 32 * j;
     wv[j] = (has_e && h4 < H4) ? __ldg(wr + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  // the router rows are weights, which no kernel of this library writes: they are requested before
+  // the wait for the previous kernel, whose output (the tokens) is read after it
+  pdl_launch_dependents();
+  pdl_wait();
   const int nchunk = (T + kRmChunk - 1) / kRmChunk;
   auto stage = [&](int c) {  // chunk c's rows into buffer c % 2, 16-byte async copies
     const int t0 = c * kRmChunk, n16 = min(kRmChunk, T - t0) * H / 8;
@@ -448,14 +455,17 @@ cudaError_t launch_router_prefill(const uint16_t *x, int T, int H, const float *
       KTimer kt_(KID_ROUTER_GEMM, s);
       const size_t smem = (size_t)2 * kRmChunk * H * 2;
       if ((e = smem_limit_once(router_mid_kernel, smem)) != cudaSuccess) return e;
-      router_mid_kernel<<<(E + 3) / 4, kRouterMidWarps * 32, smem, s>>>(x, T, H, Wr, E, logits);
+      e = launch_pdl(router_mid_kernel, dim3((E + 3) / 4), dim3(kRouterMidWarps * 32), smem, s, x, T, H, Wr, E,
+                     logits);
+      if (e != cudaSuccess) return e;
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {
       KTimer kt_(KID_TOPK, s);
-      topk_kernel<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(logits, bias, T, E, k, idx, w);
+      e = launch_pdl(topk_kernel, dim3((T + kTopkWarps - 1) / kTopkWarps), dim3(kTopkWarps * 32), 0, s, logits, bias,
+                     T, E, k, idx, w);
     }
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
   }
   if (router_tc_supported(H, E) && router_refine_supported(H, E)) {
     e = launch_router_tc(x, T, H, Wr, bias, E, wsplit, logits, ctrl, s);  // logits include the bias
