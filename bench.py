@@ -92,9 +92,9 @@ TRAFFIC = {
     ("gemm_gate_up", ("prefill8k", "stack_prefill")):
         (_GEMM_SRC, "f08dad977b547aa9656127544c86817a1159fbae806114ced9b63f365c76169e", 862530560),
     ("decode_fused", ("decode1",)):
-        (_DEC_SRC, "b4a6263a1bd80cf23ee14407bf0772dc785af48b7d956623805dfa00b7a861b3", 15141120),
+        (_DEC_SRC, "24d54efc7c230ccc35a74f209ddc58e849048abe294fd8a5049ee571a5d6febe", 15141120),
     ("mid_expert", ("batch32",)):
-        (_MID_SRC, "acc2d02342a8cb74d6fdb36322523b5cb6b5575bcf04ed7c4353561d0d314949", 47110400),
+        (_MID_SRC, "d7a2e191135ec3abd03d345a59391ae6e8cb5d05ce4d32b7464af980f07d577c", 47110400),
 }
 
 

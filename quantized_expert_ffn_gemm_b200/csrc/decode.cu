@@ -12,7 +12,8 @@
 // to fp16 pairs (exact for Q2) and fed to mma.sync m16n8k16 with the activations as the 8 MMA
 // columns, accumulating in fp32. The MMA sums over K inside the warp, so the split-K reduction is
 // done by the tensor core instead of a shuffle tree. Activations are staged in shared memory as
-// fp16 with a per-64-chunk rotation so the fragment loads of the four K slices hit distinct banks.
+// fp16 in the padded layout of gemv.cuh (16 halves after every 64), so the fragment loads of the
+// four K slices hit distinct banks.
 #include "common.cuh"
 #include "dequant.cuh"
 #include "gemv.cuh"

@@ -335,7 +335,7 @@ __device__ __forceinline__ void rows16(const MatView &m, int r0, const __half *x
   else if (rem == 1) rows16_batch<QT, 1>(m, r0, s, nsteps, xcol, colok, acc);
 }
 
-// stage columns of the activation source into shared memory (fp16, rotated layout). 16-byte
+// stage columns of the activation source into shared memory (fp16, padded layout). 16-byte
 // loads, several issued before the first store, so the staging costs one memory round trip.
 // returns true when a bf16 source value was beyond the fp16 range (it is staged as +-inf)
 template <bool SRC_BF16>
