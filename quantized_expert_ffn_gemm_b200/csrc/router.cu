@@ -244,16 +244,16 @@ topk_kernel(float *__restrict__ logits, const float *__restrict__ bias, int T, i
   const int t = blockIdx.x * kTopkWarps + warp;
   if (t >= T) return;
   float *l = logits + (size_t)t * E;
-  if (E <= 512) {
-    warp_topk<16>(l, bias, E, k, idx + (size_t)t * k, w + (size_t)t * k);
+  if (E <= 512) {  // the biased logits go back as they are formed (each lane rewrites only its own)
+    warp_topk<16>(l, bias, E, k, idx + (size_t)t * k, w + (size_t)t * k, bias ? l : nullptr);
   } else {
     for (int i = lane; i < kMaxE / 32; i += 32) s_taken[warp][i] = 0;
     __syncwarp();
     warp_topk_generic(l, bias, E, k, idx + (size_t)t * k, w + (size_t)t * k, s_taken[warp]);
+    __syncwarp();
+    if (bias)
+      for (int e = lane; e < E; e += 32) l[e] += bias[e];
   }
-  __syncwarp();
-  if (bias)
-    for (int e = lane; e < E; e += 32) l[e] += bias[e];
 }
 
 // ---------------------------------------------------------------- screen + exact refine

@@ -109,15 +109,24 @@ __device__ __forceinline__ unsigned long long warp_merge32_desc(unsigned long lo
 
 // E <= 512: lane L holds experts L, L+32, ... sorted; each round the warp takes the best head
 // (max key, then min index) and the winning lane shifts its list by one.
+// l_out (optional): receives logit + bias for every expert, stored as soon as it is formed.
 template <int PER_LANE>
-static __device__ void warp_topk(const float *l, const float *bias, int E, int k, int32_t *idx, float *w) {
+static __device__ void warp_topk(const float *l, const float *bias, int E, int k, int32_t *idx, float *w,
+                                 float *l_out = nullptr) {
   static_assert(PER_LANE == 16, "16 candidates per lane");
   const int lane = threadIdx.x & 31;
   unsigned long long c[16];
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {  // all loads first, then the codes (and the stores)
+    const int e = lane + 32 * i;
+    v[i] = (e < E) ? l[e] + (bias ? bias[e] : 0.0f) : 0.0f;
+  }
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int e = lane + 32 * i;
-    c[i] = (e < E) ? topk_code(l[e] + (bias ? bias[e] : 0.0f), e) : 0ull;
+    c[i] = (e < E) ? topk_code(v[i], e) : 0ull;
+    if (l_out && e < E) l_out[e] = v[i];
   }
   sort16_desc(c);
   float my_val = -INFINITY;
