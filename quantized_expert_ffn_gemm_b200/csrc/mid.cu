@@ -478,7 +478,17 @@ mid_combine_kernel(const float *__restrict__ part, int S, int n_rows, const int3
                    const float *__restrict__ residual, float *__restrict__ y, Ctrl *__restrict__ ctrl) {
   pdl_wait();
   pdl_launch_dependents();
+  // the token's partial-row indices and weights, staged once per CTA (one round trip), so each
+  // slot below costs only its partial rows' loads
+  __shared__ int s_r[kMaxK + 1];
+  __shared__ float s_w[kMaxK];
   const int t = blockIdx.x, h4 = blockIdx.y * blockDim.x + threadIdx.x;
+  if (threadIdx.x < k && t < T) {
+    s_r[threadIdx.x] = row_of[t * k + threadIdx.x];
+    s_w[threadIdx.x] = w[t * k + threadIdx.x];
+  }
+  if (threadIdx.x == 0 && t < T) s_r[k] = has_shared ? ctrl->mid_pairs + t : -1;
+  __syncthreads();
   if (t >= T || 4 * h4 >= H) return;
   const size_t slice = (size_t)n_rows * H;
   auto row_sum = [&](int r) {
@@ -495,10 +505,11 @@ mid_combine_kernel(const float *__restrict__ part, int S, int n_rows, const int3
   };
   float4 acc = residual ? __ldg(reinterpret_cast<const float4 *>(residual + (size_t)t * H) + h4)
                         : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
   for (int j = 0; j < k; ++j) {
-    const int r = row_of[t * k + j];
+    const int r = s_r[j];
     if (r < 0) continue;
-    const float wj = w[t * k + j];
+    const float wj = s_w[j];
     const float4 v = row_sum(r);
     acc.x = fmaf(wj, v.x, acc.x);
     acc.y = fmaf(wj, v.y, acc.y);
@@ -506,7 +517,7 @@ mid_combine_kernel(const float *__restrict__ part, int S, int n_rows, const int3
     acc.w = fmaf(wj, v.w, acc.w);
   }
   if (has_shared) {
-    const float4 v = row_sum(ctrl->mid_pairs + t);
+    const float4 v = row_sum(s_r[k]);
     acc.x += v.x;
     acc.y += v.y;
     acc.z += v.z;
