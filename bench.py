@@ -94,7 +94,7 @@ TRAFFIC = {
     ("decode_fused", ("decode1",)):
         (_DEC_SRC, "24d54efc7c230ccc35a74f209ddc58e849048abe294fd8a5049ee571a5d6febe", 15141120),
     ("mid_expert", ("batch32",)):
-        (_MID_SRC, "d7a2e191135ec3abd03d345a59391ae6e8cb5d05ce4d32b7464af980f07d577c", 47110400),
+        (_MID_SRC, "760d6d109b34b29b898ea700c9c08ecef00051612b946adb9eba5d181599c717", 47110400),
 }
 
 

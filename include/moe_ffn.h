@@ -218,7 +218,7 @@ moe_status moe_combine(const uint16_t *out_perm, const int32_t *row_of, const fl
  * GEMV: the decode path (router + top-k, then a
  * dequant-GEMV over the distinct selected experts with the tokens as MMA columns, down
  * projection fused with the weighted combine; under AUTO one cooperative kernel does the whole
- * layer where its shared-memory plan fits, T*k + T <= 96). AUTO with 8..64 tokens where that
+ * layer where its shared-memory plan fits, T*k + T <= 96). AUTO with 8..20 tokens where that
  * kernel does not fit, or path MID: the mid-batch path (MOE_PATH_MID above). Otherwise: router +
  * top-k (fp32 dot products on the CUDA cores up to 128 tokens, tensor-core logits with an exact
  * refine of the candidates above), permute, the expert FFN (AUTO / GEMM: tcgen05 grouped GEMM

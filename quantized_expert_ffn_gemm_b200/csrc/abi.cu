@@ -177,10 +177,9 @@ cudaError_t expert_rows(const uint16_t *xperm, const int32_t *offsets, int rows,
 
 // token counts for which AUTO takes the mid-batch path when the fused decode kernel does not take
 // the shape (bench.py --crossover on the decode-shaped layer, calls replayed from a CUDA graph:
-// equal to the separate decode kernels at 8 tokens and slower at 6, 0.80x the grouped GEMM at 12,
-// 0.91x at 16, equal at 24..32, 0.94x at 64; the grouped GEMM is faster from 96 tokens)
+// 0.82x the grouped GEMM at 12 tokens, 0.93x at 16; the grouped GEMM is 4% faster from 24 tokens)
 constexpr int kAutoMidLo = 8;
-constexpr int kAutoMidHi = 64;
+constexpr int kAutoMidHi = 20;
 
 bool decode_router_fits(int T, int H, int E) {
   return T <= kDecodeMaxT && (size_t)T * (H > E ? H : E) * 4 <= 200 * 1024;
