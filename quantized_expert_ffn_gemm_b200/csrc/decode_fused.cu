@@ -26,8 +26,8 @@
 //       8-15 = up rows of the same features, fp16 operands, fp32 accumulate); the partials are
 //       summed in fixed order and h is published: at one or two tokens as tagged words (two fp16
 //       values and this launch's tag per 64-bit word, by atomic exchange: no fence, no counter);
-//       at more tokens, whose down phase reads several times more h, as plain fp16 followed by a
-//       release add on the unit's readiness counter.
+//       at more tokens, whose down phase reads several times more h, as plain fp16 followed by an
+//       add on the unit's readiness counter (released two items at a time, behind one fence).
 //   P3  down projection fused with the weighted combine: each CTA owns 16 output features, its
 //       warps take whole units (16 down rows over all of I, the half steps' loads issued
 //       together). A unit's warp waits only for that unit's h (its tagged words, or its counter;
@@ -811,6 +811,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   if (ok) {
     const int grp = warp >> 3, j8 = warp & 7, gtid = tid & 255;
     int buf = 0;
+    int held = -1;  // counter path: a unit whose item's count waits for the group's next release
     for (int q = grp; q < n_mine; q += 2, buf ^= 1) {
       const int i = (int)blockIdx.x + q * G;
       const int u = i / rbs8, r0 = (i % rbs8) * 8;
@@ -869,10 +870,20 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
         }
       }
       if constexpr (!kTaggedH) {
-        // the item's h is written: count it for its unit (the group barrier orders the 64 stores
-        // before the release add)
-        named_sync(kBarGroup0 + grp, 256);
-        if (gtid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ready + u) : "memory");
+        // the item's h is written: count it for its unit. Releases go out for two items at a time
+        // (one group barrier and one release fence, which orders both items' stores, then two
+        // relaxed adds); an item's count is held back at most one item of its group.
+        if (held < 0 && q + 2 < n_mine) {
+          held = u;
+        } else {
+          named_sync(kBarGroup0 + grp, 256);
+          if (gtid == 0) {
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");
+            if (held >= 0) asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(ready + held) : "memory");
+            asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(ready + u) : "memory");
+          }
+          held = -1;
+        }
       }
     }
   }
