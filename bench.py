@@ -92,7 +92,7 @@ TRAFFIC = {
     ("gemm_gate_up", ("prefill8k", "stack_prefill")):
         (_GEMM_SRC, "f08dad977b547aa9656127544c86817a1159fbae806114ced9b63f365c76169e", 862530560),
     ("decode_fused", ("decode1",)):
-        (_DEC_SRC, "24d54efc7c230ccc35a74f209ddc58e849048abe294fd8a5049ee571a5d6febe", 15141120),
+        (_DEC_SRC, "df70967e1d8e4b634f2fe64869aab80ddba2a0539c8cf8a82dadcbd4794deab8", 15139328),
     ("mid_expert", ("batch32",)):
         (_MID_SRC, "760d6d109b34b29b898ea700c9c08ecef00051612b946adb9eba5d181599c717", 47110400),
 }
