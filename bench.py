@@ -94,7 +94,7 @@ TRAFFIC = {
     ("decode_fused", ("decode1",)):
         (_DEC_SRC, "df70967e1d8e4b634f2fe64869aab80ddba2a0539c8cf8a82dadcbd4794deab8", 15139328),
     ("mid_expert", ("batch32",)):
-        (_MID_SRC, "760d6d109b34b29b898ea700c9c08ecef00051612b946adb9eba5d181599c717", 47110400),
+        (_MID_SRC, "760d6d109b34b29b898ea700c9c08ecef00051612b946adb9eba5d181599c717", 46964736),
 }
 
 
