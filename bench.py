@@ -92,9 +92,9 @@ TRAFFIC = {
     ("gemm_gate_up", ("prefill8k", "stack_prefill")):
         (_GEMM_SRC, "f08dad977b547aa9656127544c86817a1159fbae806114ced9b63f365c76169e", 862530560),
     ("decode_fused", ("decode1",)):
-        (_DEC_SRC, "df70967e1d8e4b634f2fe64869aab80ddba2a0539c8cf8a82dadcbd4794deab8", 15139328),
+        (_DEC_SRC, "4fb5ea670044469b874c5e6f49109517780e50828033804764b5a3c38e8aa358", 15139328),
     ("mid_expert", ("batch32",)):
-        (_MID_SRC, "760d6d109b34b29b898ea700c9c08ecef00051612b946adb9eba5d181599c717", 46964736),
+        (_MID_SRC, "542734f9d4c124de70b242a349a1d31e01fefbd186012371cec854041c2998e2", 46964736),
 }
 
 

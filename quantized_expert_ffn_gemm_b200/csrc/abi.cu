@@ -33,8 +33,7 @@ cudaEvent_t take_event() {
   return e;
 }
 const char *const kKernelNames[KID_COUNT] = {
-    "router_decode", "router_gemm", "topk", "perm_hist", "perm_scan", "perm_scatter", "perm_fill",
-    "perm_gather", "combine", "rmsnorm", "dequant_rows", "dec_units", "dec_gate_up", "dec_down",
+    "router_decode", "router_gemm", "topk", "perm_hist", "perm_scan", "perm_scatter", "perm_gather", "combine", "rmsnorm", "dequant_rows", "dec_units", "dec_gate_up", "dec_down",
     "tile_list", "gemm_gate_up", "gemm_down", "router_split", "router_tc", "decode_fused", "mmq_quant",
     "mmq_gate_up", "mid_plan", "mid_expert", "mid_combine"};
 }  // namespace

@@ -289,9 +289,8 @@ cudaError_t smem_limit_once(F *func, size_t bytes) {
 
 // ---------------------------------------------------------------- per-kernel timing (optional)
 enum KernelId {
-  KID_ROUTER_DECODE = 0, KID_ROUTER_GEMM, KID_TOPK, KID_PERM_HIST, KID_PERM_SCAN, KID_PERM_SCATTER, KID_PERM_FILL,
-  KID_PERM_GATHER, KID_COMBINE, KID_RMSNORM, KID_DEQUANT_ROWS, KID_DEC_UNITS, KID_DEC_GATE_UP, KID_DEC_DOWN,
-  KID_TILE_LIST, KID_GEMM_GATE_UP, KID_GEMM_DOWN, KID_ROUTER_SPLIT, KID_ROUTER_TC, KID_DECODE_FUSED, KID_MMQ_QUANT,
+  KID_ROUTER_DECODE = 0, KID_ROUTER_GEMM, KID_TOPK, KID_PERM_HIST, KID_PERM_SCAN, KID_PERM_SCATTER, KID_PERM_GATHER,
+  KID_COMBINE, KID_RMSNORM, KID_DEQUANT_ROWS, KID_DEC_UNITS, KID_DEC_GATE_UP, KID_DEC_DOWN, KID_TILE_LIST, KID_GEMM_GATE_UP, KID_GEMM_DOWN, KID_ROUTER_SPLIT, KID_ROUTER_TC, KID_DECODE_FUSED, KID_MMQ_QUANT,
   KID_MMQ_GATE_UP, KID_MID_PLAN, KID_MID_EXPERT, KID_MID_COMBINE, KID_COUNT
 };
 void timer_begin(int kid, cudaStream_t s);

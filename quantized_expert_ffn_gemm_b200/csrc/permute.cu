@@ -221,11 +221,13 @@ perm_scan_kernel(int32_t *__restrict__ hist, int nchunks, int E, int P, int T, i
 }
 
 // ---------------------------------------------------------------- stable scatter (one warp per chunk)
+// n_iota > 0: the shared expert's rows, src[P + t] = t for t < n_iota, are written here too
 __global__ void __launch_bounds__(32)
 perm_scatter_kernel(const int32_t *__restrict__ idx, int P, int k, int E, const int32_t *__restrict__ hist,
-                    int32_t *__restrict__ row_of, int32_t *__restrict__ src) {
+                    int32_t *__restrict__ row_of, int32_t *__restrict__ src, int n_iota) {
   extern __shared__ int32_t cursor[];
   const int c = blockIdx.x, lane = threadIdx.x, nchunks = gridDim.x;
+  for (int t = c * 32 + lane; t < n_iota; t += nchunks * 32) src[P + t] = t;
   for (int e = lane; e < E; e += 32) cursor[e] = hist[(size_t)e * nchunks + c];
   __syncwarp();
   const int p0 = c * kPermChunk, p1 = min(P, p0 + kPermChunk);
@@ -302,11 +304,6 @@ perm_gather_kernel(const uint16_t *__restrict__ x, int H, const int32_t *__restr
   if (bad) set_device_error(ctrl, MOE_ERR_RANGE, 1);
 }
 
-__global__ void fill_iota_kernel(int32_t *p, int n) {
-  int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) p[i] = i;
-}
-
 cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const uint16_t *x, int H, int with_shared,
                            int32_t *counts, int32_t *offsets, int32_t *row_of, int32_t *src, uint16_t *x_perm,
                            int32_t *hist, Ctrl *ctrl, cudaStream_t s) {
@@ -331,13 +328,7 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const uint16
   }
   {
     KTimer kt_(KID_PERM_SCATTER, s);
-    perm_scatter_kernel<<<nchunks, 32, esm, s>>>(idx, P, k, E, hist, row_of, src);
-  }
-  if (with_shared) {  // src[P + t] = t
-    {
-      KTimer kt_(KID_PERM_FILL, s);
-      fill_iota_kernel<<<(T + 255) / 256, 256, 0, s>>>(src + P, T);
-    }
+    perm_scatter_kernel<<<nchunks, 32, esm, s>>>(idx, P, k, E, hist, row_of, src, with_shared ? T : 0);
   }
   const int rows = P + (with_shared ? T : 0);
   size_t want = ((size_t)rows + 7) / 8, cap = (size_t)num_sms() * 16;
