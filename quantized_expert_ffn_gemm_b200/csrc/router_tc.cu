@@ -9,8 +9,9 @@
 // x is bf16 already, so x.w = x.hi + x.mid + x.lo with every product exact, accumulated in fp32
 // by tcgen05.mma kind::f16 (bf16 x bf16 -> fp32) over K' = 3H: the A operand is the planes laid
 // side by side along K, the B operand is x re-read once per plane (TMA coordinate k' mod H).
-// Tile: 128 experts (M) x up to 256 tokens (N). The epilogue adds the router bias and writes
-// fp32 logits[t][e]; the top-k kernel then selects.
+// Tile: 128 experts (M) x up to 256 tokens (N, chosen per launch so the tiles fill the SMs in one
+// wave: 224 at 8,192 tokens and 512 experts, 148 CTAs). The epilogue adds the router bias and
+// writes fp32 logits[t][e]; the top-k kernel then selects.
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -47,10 +48,10 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float *__restri
 
 __global__ void __launch_bounds__(kRtThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, int T, int H,
-                 int E, const float *__restrict__ bias, float *__restrict__ logits, Ctrl *ctrl) {
+                 int E, const float *__restrict__ bias, float *__restrict__ logits, int ntile, Ctrl *ctrl) {
   extern __shared__ uint8_t smem_raw[];
-  const int m0 = blockIdx.x * 128, n0 = blockIdx.y * 256;
-  const int n_valid = min(256, T - n0);
+  const int m0 = blockIdx.x * 128, n0 = blockIdx.y * ntile;
+  const int n_valid = min(ntile, T - n0);
   if (n_valid <= 0) return;
   const int N = (n_valid + 15) & ~15;
   const int nbox = (N + 31) / 32;
@@ -166,7 +167,13 @@ cudaError_t launch_router_tc(const uint16_t *x, int T, int H, const float *Wr, c
   if (e != cudaSuccess) return e;
   {
     KTimer kt_(KID_ROUTER_TC, s);
-    router_tc_kernel<<<dim3(E / 128, (T + 255) / 256), kRtThreads, kRtSmem, s>>>(tw, tx, T, H, E, bias, logits, ctrl);
+    // token tile: a multiple of 32 (the activation boxes), at most 256, and as small as one wave
+    // of 128-expert x ntile tiles over the SMs allows
+    const int rows_tiles = E / 128;
+    int ntile = (int)(((size_t)T * rows_tiles + num_sms() - 1) / num_sms());
+    ntile = ntile < 32 ? 32 : ntile > 256 ? 256 : (ntile + 31) & ~31;
+    router_tc_kernel<<<dim3(rows_tiles, (T + ntile - 1) / ntile), kRtThreads, kRtSmem, s>>>(tw, tx, T, H, E, bias,
+                                                                                        logits, ntile, ctrl);
   }
   return cudaGetLastError();
 }
