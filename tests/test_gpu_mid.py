@@ -128,3 +128,26 @@ def test_mid_refuses_what_it_does_not_take():
     with pytest.raises(moe.MoeError) as ei:
         moe.expert_ffn(rows, offs, SMALL.E, routed, shared, ws, path=moe.PATH_MID)
     assert ei.value.code == moe.MOE_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("T,expect", [(8, "decode_fused"), (9, "mid_expert"), (20, "mid_expert"), (21, "gemm_gate_up"),
+                                      (64, "gemm_gate_up")])
+def test_auto_path_by_token_count(T, expect):
+    # AUTO: the fused decode kernel while its plan fits (8 tokens at top-10 with a shared expert),
+    # the mid-batch path up to 20 tokens, the grouped GEMM above (bench.py --crossover); the
+    # per-kernel timing hook shows which kernels a call launched
+    L, (x, Wr, b, routed, shared) = layer_of(DEC)
+    ws = moe.Workspace.for_layer(DEC.H, DEC.E, DEC.k, DEC.I, DEC.shared, T)
+    moe.layer_forward(x[:T].contiguous(), Wr, b, routed, shared, DEC.k, ws)  # plans and limits set up
+    torch.cuda.synchronize()
+    moe.timing_enable(True)
+    try:
+        moe.layer_forward(x[:T].contiguous(), Wr, b, routed, shared, DEC.k, ws)
+        torch.cuda.synchronize()
+        ran = {n for n, (ms, cnt) in moe.timing_read().items() if cnt > 0}
+    finally:
+        moe.timing_enable(False)
+    assert moe.read_device_error(ws) == 0
+    assert expect in ran, (T, sorted(ran))
+    others = {"decode_fused", "mid_expert", "gemm_gate_up"} - {expect}
+    assert not (others & ran), (T, sorted(ran))
