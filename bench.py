@@ -92,7 +92,7 @@ TRAFFIC = {
     ("gemm_gate_up", ("prefill8k", "stack_prefill")):
         (_GEMM_SRC, "f08dad977b547aa9656127544c86817a1159fbae806114ced9b63f365c76169e", 862530560),
     ("decode_fused", ("decode1",)):
-        (_DEC_SRC, "4fb5ea670044469b874c5e6f49109517780e50828033804764b5a3c38e8aa358", 15139328),
+        (_DEC_SRC, "493d5f0ca9c45b0e25764ae7b0e4fb985de1c87211ce742466b031b77ba67e27", 15141120),
     ("mid_expert", ("batch32",)):
         (_MID_SRC, "542734f9d4c124de70b242a349a1d31e01fefbd186012371cec854041c2998e2", 46964736),
 }

@@ -3,10 +3,11 @@
 // A decode step is bound by reading weights ("Strata vs Llama.cpp vs vLLM", chapter "Why LLM
 // inference is a systems problem"), and at 1-4 tokens a layer moves only ~15 MB: spread over 148
 // SMs that is ~100 KB per SM, less than one SM's shared memory. So the kernel asks for all of it
-// at once: as soon as the routing is known, the warps of every CTA issue 16-byte async copies
-// (cp.async, each warp's completion counted on one mbarrier per slot) of the CTA's whole share of
-// gate/up rows and down rows into a ring of shared-memory slots, and then work from shared memory
-// as the slots fill; a slot that is read out is refilled at once by the warp that freed it. HBM
+// at once: as soon as the routing is known, the warps of every CTA issue bulk async copies
+// (cp.async.bulk, a few contiguous runs of rows per fill, the bytes counted on one mbarrier per
+// slot) of the CTA's whole share of gate/up rows and down rows into a ring of shared-memory slots,
+// and then work from shared memory as the slots fill; a slot that is read out is refilled at once
+// by the warp that freed it. HBM
 // then sees the layer's expert bytes requested within a few hundred nanoseconds instead of as a
 // chain of dependent round trips.
 //
@@ -44,8 +45,8 @@
 // it. The readiness counters come in two sets used by alternate launches; a launch zeroes the set
 // the next one will use. The logit and h polls, the readiness waits and every mbarrier wait are
 // bounded in time and report MOE_ERR_TIMEOUT instead of hanging;
-// before the CTA exits every thread waits for its own outstanding copies (cp.async.wait_all), so
-// no copy is still writing its shared memory.
+// before the CTA exits it waits for the last fill of every slot (bounded too), so no copy is still
+// writing its shared memory.
 #include "common.cuh"
 #include "dequant.cuh"
 #include "gemv.cuh"
@@ -189,16 +190,13 @@ __device__ __forceinline__ void prefetch_shared(const moe_expert_set &sh, int I,
   }
 }
 
-// 16-byte global -> shared async copy (L2 only); both addresses 16-byte aligned
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// bulk copy global -> this CTA's shared memory, counted in bytes on `bar` (16-byte aligned
+// addresses, a multiple of 16 bytes)
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
 }
-// arrive on `bar` once every cp.async this thread issued so far has landed (counts against the
-// barrier's expected arrivals)
-__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -318,6 +316,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   FusedSync *const fs = fused_sync(ctrl);
   __shared__ uint32_t s_tag;
   __shared__ volatile int s_abort;
+  __shared__ int s_lastq[kFMaxRing];  // the last fill issued into each slot (-1: none)
   // ---------------- P0: this warp's router rows are requested first, then the tokens are staged
   const int H4 = H / 4, HQ = H4 / 4;  // float4 per quarter of a router row (<= 128: H <= 2048)
   const int es = warp >> 2, qh = warp & 3;
@@ -348,7 +347,10 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   if (tid == 0) {
     launch_no = *reinterpret_cast<volatile const uint32_t *>(&fs->seq[blockIdx.x]);
     s_abort = 0;
-    for (int s = 0; s < R; ++s) mbar_init(full(s), 32);  // one arrival per lane of the filling warp
+    for (int s = 0; s < R; ++s) {
+      mbar_init(full(s), 1);  // the filling lane's arrival, and the fill's bytes
+      s_lastq[s] = -1;
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // a bounded wait that gives up at once after an earlier wait of this CTA gave up
@@ -768,38 +770,47 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   const int nhalf_dn = (I + kStepK / 2 - 1) / (kStepK / 2);  // down items are half steps (128 wide)
 
   // ---------------- fills: fill q of this CTA (gate/up items, then down pieces) goes to slot
-  // q % R; it is issued by one whole warp (cp.async, 16 bytes per lane per instruction), whose
-  // 32 lanes then arrive on the slot's barrier when their copies have landed
+  // q % R; lane 0 of the calling warp posts the fill's byte count on the slot's barrier and issues
+  // it as a few bulk copies (each a contiguous run of rows: codes, scales, hi bits), after a proxy
+  // fence that orders the slot's earlier reads by the warps before the copies' writes. After a wait
+  // of this CTA gave up, no fill goes out (its slot's previous fill may not have been waited on).
   auto issue_fill = [&](int q) {
+    if (lane != 0 || s_abort) return;
     const int s = q % R;
     const uint32_t dst0 = ring0 + (uint32_t)(s * S);
+    fence_async_smem();
+    s_lastq[s] = q;
     if (q < n_mine) {
       const int i = (int)blockIdx.x + q * G;
       const UnitMats &um = s_um[i / rbs8];
       const int r0 = (i % rbs8) * 8;
       const int nc = QT == 3 ? 6 : 4;
+      uint32_t tot = 0;
+      for (int c = 0; c < nc; ++c) tot += gu_copy<QT>(a, um, r0, c).bytes;
+      mbar_arrive_expect_tx(full(s), tot);
 #pragma unroll 1
       for (int c = 0; c < nc; ++c) {
         const CopyDesc d = gu_copy<QT>(a, um, r0, c);
-        const char *src = static_cast<const char *>(d.src);
-        for (uint32_t off = 16u * lane; off < d.bytes; off += 512u) cp_async16(dst0 + d.off + off, src + off);
+        bulk_g2s(dst0 + d.off, d.src, d.bytes, full(s));
       }
     } else {
       const int j = q - n_mine, rbl = j / npieces, dp = j % npieces;
       const int rb = (int)blockIdx.x + rbl * G;
       const int nun = min(a.dpu, nu - dp * a.dpu);
       const int per = QT == 3 ? 3 : 2;
+      uint32_t tot = 0;
+      for (int m = 0; m < nun; ++m)
+        for (int c = 0; c < per; ++c) tot += dn_copy<QT>(a, s_um[dp * a.dpu + m], rb, m, c).bytes;
+      mbar_arrive_expect_tx(full(s), tot);
       for (int m = 0; m < nun; ++m) {
         const UnitMats &um = s_um[dp * a.dpu + m];
 #pragma unroll 1
         for (int c = 0; c < per; ++c) {
           const CopyDesc d = dn_copy<QT>(a, um, rb, m, c);
-          const char *src = static_cast<const char *>(d.src);
-          for (uint32_t off = 16u * lane; off < d.bytes; off += 512u) cp_async16(dst0 + d.off + off, src + off);
+          bulk_g2s(dst0 + d.off, d.src, d.bytes, full(s));
         }
       }
     }
-    cp_async_arrive(full(s));
   };
   if (ok)
     for (int q = warp; q < min(n_total, R); q += kFWarps) issue_fill(q);
@@ -1098,8 +1109,11 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const FusedA
   }
 
 
-  // ---------------- no copy may still be writing this CTA's shared memory when it exits
-  cp_async_wait_all();
+  // ---------------- no copy may still be writing this CTA's shared memory when it exits: the
+  // last fill of each slot has landed (an earlier one was waited on before its slot was refilled)
+  __syncthreads();
+  if (tid < R && s_lastq[tid] >= 0 && !mbar_wait(full(tid), fill_parity(s_lastq[tid])))
+    set_device_error(ctrl, MOE_ERR_TIMEOUT, 47);
 }
 
 // Test hook of the failure path: one warp waits, with the fused kernel's logit-exchange wait, for
