@@ -116,7 +116,7 @@ enum { MOE_Q2 = 2, MOE_Q3 = 3, MOE_Q4 = 4 };
 enum { MOE_PATH_AUTO = 0, MOE_PATH_GEMV = 1, MOE_PATH_GEMM = 2, MOE_PATH_MMQ = 3, MOE_PATH_MID = 4 };
 
 typedef struct moe_qmat {
-  int32_t qtype;            /* MOE_Q2, MOE_Q3 or MOE_Q4 (all matrices of a layer share one) */
+  int32_t qtype;            /* MOE_Q2, MOE_Q3 or MOE_Q4 (all matrices of a layer, shared expert included, share one; MOE_ERR_INVALID_ARG otherwise) */
   int32_t n_experts;
   int32_t rows;
   int32_t K;

@@ -279,6 +279,7 @@ moe_status moe_expert_ffn(const uint16_t *x_perm, const int32_t *offsets, int32_
   if (path == MOE_PATH_MID) return MOE_ERR_UNSUPPORTED;  // the mid-batch path works from the routing
   if ((st = check_set(routed, E, H, I)) != MOE_OK) return st;
   if (shared_opt && (st = check_set(shared_opt, 1, H, I)) != MOE_OK) return st;
+  if (shared_opt && shared_opt->gate.qtype != routed->gate.qtype) return MOE_ERR_INVALID_ARG;  // one format a layer
   if (n_rows == 0) return MOE_OK;
   if (!x_perm || !offsets || !out_perm) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x_perm) || !aligned16(out_perm) || !aligned16(offsets)) return MOE_ERR_ALIGNMENT;
@@ -326,6 +327,7 @@ static moe_status layer_forward_impl(const uint16_t *x, int32_t T, const float *
   if (T < 0 || path < 0 || path > 4) return MOE_ERR_INVALID_ARG;
   if ((st = check_set(routed, E, H, I)) != MOE_OK) return st;
   if (hs && (st = check_set(shared_opt, 1, H, I)) != MOE_OK) return st;
+  if (hs && shared_opt->gate.qtype != routed->gate.qtype) return MOE_ERR_INVALID_ARG;  // one format a layer
   if (T == 0) return MOE_OK;
   if (!x || !Wr || !y) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(Wr) || !aligned16(y) || (bias && !aligned16(bias)) ||
@@ -493,6 +495,7 @@ static moe_status stack_forward_impl(const float *r_in, int32_t T, int32_t L, co
   for (int l = 0; l < L; ++l) {
     if ((st = check_set(&routed[l], E, H, I)) != MOE_OK) return st;
     if (hs && (st = check_set(&shared[l], 1, H, I)) != MOE_OK) return st;
+    if (hs && shared[l].gate.qtype != routed[l].gate.qtype) return MOE_ERR_INVALID_ARG;  // one format a layer
     if (!Wr[l]) return MOE_ERR_INVALID_ARG;
   }
   for (int l = 0; l < L; ++l)

@@ -91,6 +91,8 @@ def test_layer_forward_validation(lib):
     assert _lf(lib, routed=_set(qtype=2, hib=FAKE.value)) == moe.MOE_ERR_INVALID_ARG  # hi bits belong to Q3 only
     assert _lf(lib, routed=_set(qtype=4, hib=FAKE.value)) == moe.MOE_ERR_INVALID_ARG
     assert _lf(lib, routed=_set(E=511)) == moe.MOE_ERR_INVALID_ARG         # set shape disagrees with desc
+    # the shared expert in another block format than the routed experts (one format per layer)
+    assert _lf(lib, desc=_desc(sh=1), shared=_set(E=1, qtype=4)) == moe.MOE_ERR_INVALID_ARG
     assert _lf(lib, ws=None) == moe.MOE_ERR_WORKSPACE
     assert _lf(lib, wsb=1024) == moe.MOE_ERR_WORKSPACE
     assert _lf(lib, path=5) == moe.MOE_ERR_INVALID_ARG
